@@ -1,0 +1,260 @@
+"""CPU oracle for the MISA / DSA token-selection indexer (test infrastructure).
+
+This module is test infrastructure: only the tests, the smoke check and the
+benchmark's CPU-baseline leg import it.  The product path never calls it, and
+it shares no code with the CUDA library: it reads the same input arrays and
+recomputes everything from the definitions, plainly and slowly, in float64.
+
+Sources (page titles; sections in quotes):
+
+* [ABS]  "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM
+  Inference", Hugging Face paper-page abstract.
+* [SUM]  same title, gist.science technical summary (Arabic and Hindi
+  renderings carry the same text), sections "Problem statement",
+  "Methodology: MISA" (step 1 block-pooled router, step 2 sparse token
+  scoring, the complexity sentence), "Hierarchical variant (MISA-dagger)".
+
+The pages do not print the indexer formula.  The reading used here is the DSA
+lightning-indexer form I_t = sum_j w_j * ReLU(q_j . k_t), with one index key
+per token shared by all heads ([ABS]: the heads share one selected token set),
+and with no extra global scale (a positive global factor changes no
+selection).  For fp8 keys the dequantised key is s_t * e4m3(code_t).
+
+Readings where the pages are silent (each also listed in the design notes):
+
+* router aggregation: r_j = |w_j| * sum_m ReLU(q_j . kbar_m)  ("aggregates
+  these scores to estimate each head's importance", [SUM] step 1);
+  parity unpinned as to the choice of aggregation (no printed number separates
+  it from signed-w, unweighted or max variants);
+* pooled key kbar_m = arithmetic mean of the keys present in block m; a
+  trailing partial block is averaged over the tokens it holds (the ceiling in
+  M = ceil(L / B)); a query's prefix is tokens 0..p_i inclusive;
+* top-k and top-h ties go to the lower token / head index; when the prefix
+  holds fewer than k tokens every token is returned, padded with -1;
+* MISA-dagger: the candidate set is the routed pass's top-k'; the fine stage
+  is the dense indexer on the candidates only, then top-k by (score, index).
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Sequence
+
+import numpy as np
+
+# --------------------------------------------------------------------------
+# Number formats
+# --------------------------------------------------------------------------
+
+
+def _e4m3_table() -> np.ndarray:
+    """All 256 e4m3 code values from the OCP 8-bit floating point definition.
+
+    Layout s.eeee.mmm, exponent bias 7, no infinities; codes 0x7F and 0xFF are
+    NaN; exponent field 0 encodes subnormals m * 2^-9.
+    """
+    t = np.empty(256, dtype=np.float64)
+    for c in range(256):
+        s = -1.0 if c & 0x80 else 1.0
+        e = (c >> 3) & 0xF
+        m = c & 0x7
+        if e == 0xF and m == 0x7:
+            t[c] = math.nan
+        elif e == 0:
+            t[c] = s * m * 2.0 ** -9
+        else:
+            t[c] = s * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return t
+
+
+E4M3 = _e4m3_table()
+
+
+def decode_e4m3(codes: np.ndarray) -> np.ndarray:
+    return E4M3[np.asarray(codes, dtype=np.uint8)]
+
+
+def decode_bf16(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> float64 (bf16 is the top half of an IEEE binary32)."""
+    with np.errstate(invalid="ignore"):
+        return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def dequantize_keys(keys: np.ndarray, dtype: str, scale: Optional[np.ndarray] = None) -> np.ndarray:
+    """Index keys of one sequence as float64 [L][d]: k_t = s_t * e4m3(code) or bf16."""
+    if dtype == "bf16":
+        return decode_bf16(keys)
+    assert scale is not None
+    return decode_e4m3(keys) * np.asarray(scale, dtype=np.float64)[:, None]
+
+
+# --------------------------------------------------------------------------
+# Dot-product counter (the cost model is checked against exact counts)
+# --------------------------------------------------------------------------
+
+
+class Counter:
+    """Counts query-head x key dot products the oracle actually evaluates."""
+
+    def __init__(self):
+        self.n = 0
+
+    def add(self, rows: int, cols: int):
+        self.n += int(rows) * int(cols)
+
+
+# --------------------------------------------------------------------------
+# Steps of the method
+# --------------------------------------------------------------------------
+
+
+def pool_keys(K: np.ndarray, L: int, B: int) -> np.ndarray:
+    """Block mean-pool of the first L keys: M = ceil(L/B) means [M][d].
+
+    [SUM] "Methodology: MISA", step 1: the prefix is cut into M = ceil(L/B)
+    blocks and each block is summarised by the mean of its index keys.
+    """
+    M = -(-L // B)
+    out = np.zeros((M, K.shape[1]), dtype=np.float64)
+    for m in range(M):
+        blk = K[m * B:min((m + 1) * B, L)]
+        out[m] = blk.sum(axis=0) / blk.shape[0]
+    return out
+
+
+def head_token_scores(q: np.ndarray, K: np.ndarray, heads: Sequence[int],
+                      counter: Optional[Counter] = None) -> np.ndarray:
+    """Per-head dot products q_j . k_t for j in ``heads``: [len(heads)][L]."""
+    Q = q[list(heads)]
+    if counter is not None:
+        counter.add(Q.shape[0], K.shape[0])
+    return Q @ K.T
+
+
+def index_scores(q: np.ndarray, w: np.ndarray, K: np.ndarray, heads: Sequence[int],
+                 counter: Optional[Counter] = None) -> np.ndarray:
+    """I_t = sum_{j in heads, ascending j} w_j * ReLU(q_j . k_t) for every row of K.
+
+    With heads = all H_I heads this is the dense DSA indexer ([SUM] "Problem
+    statement"); with the routed heads it is MISA's sparse token scoring
+    ([SUM] "Methodology: MISA", step 2).
+    """
+    heads = sorted(int(j) for j in heads)
+    A = head_token_scores(q, K, heads, counter)
+    I = np.zeros(K.shape[0], dtype=np.float64)
+    for r, j in enumerate(heads):
+        I += w[j] * np.maximum(A[r], 0.0)
+    return I
+
+
+def router_scores(q: np.ndarray, w: np.ndarray, pooled: np.ndarray,
+                  counter: Optional[Counter] = None) -> np.ndarray:
+    """Head importance r_j = |w_j| * sum_m ReLU(q_j . kbar_m) over the pooled keys.
+
+    [SUM] "Methodology: MISA", step 1: per-head affinities against the
+    block-level statistics, aggregated into a per-head importance.
+    """
+    A = head_token_scores(q, pooled, range(q.shape[0]), counter)
+    return np.abs(w.astype(np.float64)) * np.maximum(A, 0.0).sum(axis=1)
+
+
+def top_h(r: np.ndarray, h: int) -> np.ndarray:
+    """The h heads of largest r (ties to the lower head index), ascending."""
+    order = np.lexsort((np.arange(r.shape[0]), -r))
+    return np.sort(order[:h])
+
+
+def top_k(I: np.ndarray, k: int, index: Optional[np.ndarray] = None) -> np.ndarray:
+    """The k largest scores, ties to the lower token index; [k] int32 ascending, -1 padded.
+
+    ``index`` maps positions of I to token indices (candidate lists); by
+    default position t is token t.
+    """
+    n = I.shape[0]
+    idx = np.arange(n) if index is None else np.asarray(index, dtype=np.int64)
+    order = np.lexsort((idx, -I))
+    sel = np.sort(idx[order[:min(k, n)]])
+    out = np.full(k, -1, dtype=np.int32)
+    out[:sel.shape[0]] = sel
+    return out
+
+
+# --------------------------------------------------------------------------
+# Per-query pipelines
+# --------------------------------------------------------------------------
+
+
+def route_query(q, w, K, L_i, B, h, counter=None):
+    """Router for one query with prefix length L_i: returns (r [H], heads [h])."""
+    pooled = pool_keys(K, L_i, B)
+    r = router_scores(q, w, pooled, counter)
+    return r, top_h(r, h)
+
+
+def misa_query(q, w, K, L_i, B, h, k, counter=None):
+    """MISA: route, score the prefix with the routed heads, keep top-k.
+
+    Returns dict(r, heads, scores, topk).
+    """
+    r, heads = route_query(q, w, K, L_i, B, h, counter)
+    I = index_scores(q, w, K[:L_i], heads, counter)
+    return dict(r=r, heads=heads, scores=I, topk=top_k(I, k))
+
+
+def dense_query(q, w, K, L_i, k, counter=None):
+    """Dense DSA indexer: all H_I heads on the whole prefix, keep top-k."""
+    I = index_scores(q, w, K[:L_i], range(q.shape[0]), counter)
+    return dict(scores=I, topk=top_k(I, k))
+
+
+def rerank_query(q, w, K, cand, k, counter=None):
+    """Fine stage of MISA-dagger: dense scores of the candidates, keep top-k of them.
+
+    [SUM] "Hierarchical variant": the original DSA indexer (all H_I heads)
+    re-scores only the candidate set to recover the final top-k.
+    Returns dict(scores [len(cand)], topk).  Candidates equal to -1 are ignored.
+    """
+    cand = np.asarray(cand, dtype=np.int64)
+    c = cand[cand >= 0]
+    I = index_scores(q, w, K[c], range(q.shape[0]), counter)
+    return dict(scores=I, cand=c, topk=top_k(I, k, index=c))
+
+
+def misa_dagger_query(q, w, K, L_i, B, h, k_prime, k, counter=None):
+    """MISA-dagger: routed pass keeps k' candidates, dense re-rank keeps k."""
+    coarse = misa_query(q, w, K, L_i, B, h, k_prime, counter)
+    fine = rerank_query(q, w, K, coarse["topk"], k, counter)
+    return dict(coarse=coarse, fine=fine, topk=fine["topk"])
+
+
+def dot_product_count(kind: str, L_i: int, B: int, H: int, h: int, k_prime: int = 0) -> int:
+    """Cost model of [SUM] "Methodology: MISA": O(hL + H_I M) against O(H_I L)."""
+    M = -(-L_i // B)
+    if kind == "dense":
+        return H * L_i
+    if kind == "misa":
+        return h * L_i + H * M
+    if kind == "misa_dagger":
+        return h * L_i + H * M + H * min(k_prime, L_i)
+    raise ValueError(kind)
+
+
+# --------------------------------------------------------------------------
+# Whole-workload helpers (arrays laid out as the library consumes them)
+# --------------------------------------------------------------------------
+
+
+def seq_keys(keys: np.ndarray, scale: Optional[np.ndarray], dtype: str, s: int, L: Optional[int] = None):
+    """Dequantised keys of sequence s (first L tokens) as float64."""
+    kk = keys[s] if L is None else keys[s, :L]
+    sc = None if scale is None else (scale[s] if L is None else scale[s, :L])
+    return dequantize_keys(kk, dtype, sc)
+
+
+def query_arrays(q_bits: np.ndarray, w: np.ndarray, i: int):
+    return decode_bf16(q_bits[i]), np.asarray(w[i], dtype=np.float64)
+
+
+def pool_cache(keys, scale, dtype, seq_len, B):
+    """Pooled keys of every sequence over its seq_len tokens: list of [M_s][d]."""
+    return [pool_keys(seq_keys(keys, scale, dtype, s, int(seq_len[s])), int(seq_len[s]), B)
+            for s in range(keys.shape[0])]
