@@ -1,0 +1,350 @@
+"""Benchmark of the MISA-dagger decode step on B200 (one JSON line on rank 0).
+
+Workload (default): 8 decode sequences at L = 131072 with fp8 e4m3 index keys
+(one fp32 scale per token), H_I = 64 index heads, block B = 128, h = 8 routed
+heads, k' = 8192 candidates re-ranked by all heads to k = 2048.  One step:
+
+  1. misa_pool_keys  -- append the new token's key and refresh its block mean
+  2. misa_route_heads -- block-pooled router, top-8 heads per query
+  3. misa_score_topk -- routed scoring of all 131072 prefix tokens, top-k'
+  4. misa_rerank_topk -- dense re-score of the k' candidates, top-k
+
+Metric: scored head.tokens/s = sum over queries of (h L_i + H_I M_i + H_I k')
+per step / step time (also queries/s).  Inputs are synthetic (seeded
+generator), resident in HBM; L2 is flushed (256 MiB write) between timed
+steps.  --impl reference times the CPU oracle on a bounded sample instead.
+
+Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under
+torch.distributed.run (one rank per GPU, NCCL), each rank runs its own batch
+(weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_misa_b200 import inputs as G  # noqa: E402
+
+HBM_FALLBACK_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 1590.0)), "measured"
+    return HBM_FALLBACK_GBS, 1590.0, "fallback"
+
+
+def work_per_query(wl, L_i):
+    """Algorithmic head.tokens of one MISA-dagger query (cost model of the method)."""
+    M = -(-L_i // wl.B)
+    return wl.h * L_i + wl.H * M + wl.H * min(wl.k_prime, L_i)
+
+
+def score_kernel_bytes(wl):
+    """Algorithmic bytes of the routed scoring kernel per launch: keys (+scales) once,
+    the routed query heads and their weights."""
+    row = wl.d * (1 if wl.key_dtype == "fp8" else 2) + (4 if wl.key_dtype == "fp8" else 0)
+    return wl.n_seq * wl.L * row + wl.n_q * wl.h * (wl.d * 2 + 4)
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.proc, self.path = index, None, None
+
+    def start(self):
+        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{self.index}.csv")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def cpu_oracle_rate(wl, inp, n_queries, min_seconds=0.0):
+    """Time the CPU oracle's MISA-dagger pass over a sample of queries (cycling
+    through the batch until both n_queries and min_seconds are reached)."""
+    from oracle import misa_oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([t.get("num_threads", 1) for t in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    work = 0
+    done = 0
+    while done < n_queries or time.perf_counter() - t0 < min_seconds:
+        i = done % inp.wl.n_q
+        done += 1
+        s = int(inp.q_seq[i])
+        Li = int(inp.q_pos[i]) + 1
+        K = O.seq_keys(inp.keys, inp.scale, wl.key_dtype, s, Li)
+        q, w = O.query_arrays(inp.q, inp.w, i)
+        O.misa_dagger_query(q, w, K, Li, wl.B, wl.h, wl.k_prime, wl.k)
+        work += work_per_query(wl, Li)
+    dt = time.perf_counter() - t0
+    return work / dt, done / dt, dt, cores, done
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = G.make_inputs(wl.scaled(n_seq=1), seed=0)
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm-up state; steps below are all timed
+    vals, qps, secs = [], [], []
+    for _ in range(args.steps):
+        v, q, dt, cores, _ = cpu_oracle_rate(wl, inp, 1)
+        vals.append(v)
+        qps.append(q)
+        secs.append(dt)
+    value = float(np.mean(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * float(np.mean(secs)),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded generator)",
+        "config": config_block(wl, l2="n/a (CPU)"),
+        "queries_per_s": float(np.mean(qps)),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"1 query per step (sequence 0 of {wl.name}), full MISA-dagger pass in numpy fp64"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+METRIC = "indexer scored head*tokens/s (MISA-dagger decode, L=128K)"
+UNIT = "head*tokens/s"
+
+
+def config_block(wl, l2):
+    return {"workload": wl.name, "n_seq": wl.n_seq, "L": wl.L, "H_I": wl.H, "h": wl.h, "B": wl.B,
+            "k_prime": wl.k_prime, "k": wl.k, "d": wl.d, "key_dtype": "fp8_e4m3+fp32 scale", "q_dtype": "bf16",
+            "l2": l2}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="misa", choices=["misa", "reference"])
+    ap.add_argument("--workload", default="misa_dagger_decode_128k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = G.WORKLOADS[args.workload]
+    assert wl.k_prime is not None and wl.mode == "decode", "the bench step is the MISA-dagger decode step"
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from long_context_misa_b200 import misa as M
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    assert world == args.gpus, f"--gpus {args.gpus} but WORLD_SIZE={world}"
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    # ---- inputs (rank-seeded, resident in HBM) ----
+    inp = G.make_inputs(wl, seed=rank)
+    cache, qs = M.device_inputs(inp, dev)
+    # the step appends each query's own token: the cache starts one token short
+    cache.seq_len.copy_(torch.from_numpy(inp.seq_len - 1))
+    M.pool_keys(cache)
+    pos = torch.from_numpy(inp.q_pos.copy()).to(dev)
+    last = np.stack([inp.keys[s, inp.q_pos[s]:inp.q_pos[s] + 1] for s in range(wl.n_seq)])
+    new_keys = torch.from_numpy(last).to(dev).contiguous()
+    new_scale = torch.from_numpy(np.stack([inp.scale[s, inp.q_pos[s]:inp.q_pos[s] + 1]
+                                           for s in range(wl.n_seq)])).to(dev).contiguous()
+    ws = M.Workspace(dev)
+    heads = torch.empty(wl.n_q, wl.h, dtype=torch.int32, device=dev)
+    cand = torch.empty(wl.n_q, wl.k_prime, dtype=torch.int32, device=dev)
+    top = torch.empty(wl.n_q, wl.k, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    LAUNCHES_PER_STEP = 7  # append 1, route 2, score+top-k' 2, rerank+top-k 2
+
+    def step():
+        M.pool_keys(cache, new_keys, new_scale, pos, stream=stream)
+        M.route_heads(cache, qs, wl.h, heads=heads, ws=ws, stream=stream)
+        M.score_topk(cache, qs, heads, wl.k_prime, topk=cand, ws=ws, stream=stream)
+        M.rerank_topk(cache, qs, cand, wl.k, topk=top, ws=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0, "device status set during warm-up"
+
+    # ---- timed region: K steps, L2 flushed between steps ----
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in kev:  # materialise the events so their handles exist
+        a.record(stream)
+        b.record(stream)
+    clocks = Clocks(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()
+        M.debug_time_scoring(*kev[i])
+        ev[i][0].record(stream)
+        M.pool_keys(cache, new_keys, new_scale, pos, stream=stream)
+        M.route_heads(cache, qs, wl.h, heads=heads, ws=ws, stream=stream)
+        M.score_topk(cache, qs, heads, wl.k_prime, topk=cand, ws=ws, stream=stream)
+        M.debug_time_scoring(None, None)
+        M.rerank_topk(cache, qs, cand, wl.k, topk=top, ws=ws, stream=stream)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    kern_ms = [a.elapsed_time(b) for a, b in kev]
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    assert cache.device_status() == 0, "device status set during timing"
+
+    per_step_work = sum(work_per_query(wl, int(inp.q_pos[i]) + 1) for i in range(wl.n_q))
+    ms_per_step = total_ms / args.steps
+    value = world * per_step_work / (ms_per_step * 1e-3)
+    qps = world * wl.n_q / (ms_per_step * 1e-3)
+
+    # ---- dense DSA indexer on the same batch (context: the work MISA replaces) ----
+    dense_ms = []
+    for _ in range(3):
+        flush.zero_()
+        M.dense_score_topk(cache, qs, wl.k, ws=ws, stream=stream)
+    for _ in range(5):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        M.dense_score_topk(cache, qs, wl.k, ws=ws, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        dense_ms.append(a.elapsed_time(b))
+
+    # ---- end to end through the public API with pinned host buffers ----
+    h_keys = torch.from_numpy(last).pin_memory()
+    h_scale = new_scale.cpu().pin_memory()
+    h_q = torch.from_numpy(inp.q.view(np.int16)).pin_memory()
+    h_w = torch.from_numpy(inp.w).pin_memory()
+    h_pos = torch.from_numpy(inp.q_pos.copy()).pin_memory()
+    h_top = torch.empty(wl.n_q, wl.k, dtype=torch.int32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_keys, h_scale, h_q, h_w, h_pos))
+    d2h = h_top.numel() * h_top.element_size()
+    e2e_ms = []
+    for i in range(max(3, args.steps // 2)):
+        flush.zero_()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        new_keys.copy_(h_keys, non_blocking=True)
+        new_scale.copy_(h_scale, non_blocking=True)
+        qs.q.copy_(h_q, non_blocking=True)
+        qs.w.copy_(h_w, non_blocking=True)
+        pos.copy_(h_pos, non_blocking=True)
+        step()
+        h_top.copy_(top, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    e2e_step = float(np.mean(e2e_ms[1:] if len(e2e_ms) > 1 else e2e_ms))
+    e2e_value = world * per_step_work / (e2e_step * 1e-3)
+
+    if rank == 0:
+        hbm, _, src = peaks()
+        kb = score_kernel_bytes(wl)
+        k_ms = float(np.mean(kern_ms))
+        achieved = kb / (k_ms * 1e-3) / 1e9
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            v, q, dt, cores, n = cpu_oracle_rate(wl, inp, 2, min_seconds=10.0)
+            cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "queries_per_s": q,
+                   "sample": f"{n} queries of this batch in {dt:.1f} s: full MISA-dagger pass "
+                             f"(dequantise, pool, route, routed score + top-k', dense re-rank + top-k) in numpy fp64"}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3 keys -> f16 MMA, f32 accumulate",
+            "data": "synthetic (seeded generator), resident in HBM",
+            "config": config_block(wl, l2="flushed between steps (256 MiB write)"),
+            "queries_per_s": qps,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_step},
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "roofline": {"kernel": "routed token scoring (score_mma_kernel<1, fp8>)", "bound": "hbm",
+                         "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "traffic": None, "algorithmic_bytes_per_launch": kb, "ms_per_launch": k_ms,
+                         "peak_source": f"{src} hbm_gbs"},
+            "dense_dsa": {"ms": float(np.median(dense_ms)), "misa_dagger_step_ms": ms_per_step,
+                          "speedup_vs_dense": float(np.median(dense_ms)) / ms_per_step},
+            "clocks": clk,
+        }
+        if cpu:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

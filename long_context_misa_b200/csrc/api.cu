@@ -1,0 +1,268 @@
+// C ABI of the MISA / DSA indexer: argument validation, workspace layout and
+// dispatch to the kernels.  Declarations and semantics: include/misa.h.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+std::atomic<int> g_fail_next{0};
+std::atomic<void *> g_ev_start{nullptr}, g_ev_stop{nullptr};
+
+// Launch the scoring kernel, bracketed by the profiling events when set.
+template <class F>
+cudaError_t timed_scoring(cudaStream_t stream, F &&launch) {
+  void *a = g_ev_start.load(), *b = g_ev_stop.load();
+  if (a && b) {
+    cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(a), stream);
+    if (e != cudaSuccess) return e;
+  }
+  cudaError_t e = launch();
+  if (e == cudaSuccess && a && b) e = cudaEventRecord(static_cast<cudaEvent_t>(b), stream);
+  return e;
+}
+
+misa_status fail(misa_status st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+misa_status cuda_fail(cudaError_t e, const char *where) {
+  return fail(MISA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Consume one injected failure, if any (after validation, before any launch).
+bool injected_failure(const char *where, misa_status *st) {
+  int n = g_fail_next.load();
+  while (n > 0) {
+    if (g_fail_next.compare_exchange_weak(n, n - 1)) {
+      *st = fail(MISA_ERR_CUDA, "%s: injected failure (misa_debug_fail_next)", where);
+      return true;
+    }
+  }
+  return false;
+}
+
+misa_status check_cache(const misa_cache *c, bool need_pool) {
+  if (!c) return fail(MISA_ERR_INVALID, "cache is NULL");
+  if (!c->keys || !c->seq_len) return fail(MISA_ERR_INVALID, "cache keys/seq_len is NULL");
+  if (need_pool && !c->pool) return fail(MISA_ERR_INVALID, "cache pool is NULL");
+  if (c->dtype != MISA_KEY_BF16 && c->dtype != MISA_KEY_FP8_E4M3)
+    return fail(MISA_ERR_INVALID, "unknown key dtype %d", c->dtype);
+  if ((c->dtype == MISA_KEY_FP8_E4M3) != (c->scale != nullptr))
+    return fail(MISA_ERR_INVALID, "scale must be non-NULL exactly for fp8 keys");
+  if (c->d != MISA_D) return fail(MISA_ERR_UNSUPPORTED, "d=%d unsupported (only %d)", c->d, MISA_D);
+  if (c->n_seq < 1 || c->L_cap < 1 || c->B < 1)
+    return fail(MISA_ERR_INVALID, "n_seq=%d L_cap=%d B=%d must be >= 1", c->n_seq, c->L_cap, c->B);
+  if (c->L_cap > MISA_MAX_L) return fail(MISA_ERR_UNSUPPORTED, "L_cap=%d above %d", c->L_cap, MISA_MAX_L);
+  if (!aligned16(c->keys)) return fail(MISA_ERR_INVALID, "keys must be 16-byte aligned");
+  if (c->pool && !aligned16(c->pool)) return fail(MISA_ERR_INVALID, "pool must be 16-byte aligned");
+  return MISA_OK;
+}
+
+misa_status check_queries(const misa_queries *q) {
+  if (!q) return fail(MISA_ERR_INVALID, "queries is NULL");
+  if (q->n_q < 0 || q->n_q > 65535) return fail(MISA_ERR_INVALID, "n_q=%d outside [0, 65535]", q->n_q);
+  if (q->H < 1 || q->H > MISA_MAX_H) return fail(MISA_ERR_UNSUPPORTED, "H=%d outside [1, %d]", q->H, MISA_MAX_H);
+  if (q->n_q > 0 && (!q->q || !q->w || !q->q_seq || !q->q_pos))
+    return fail(MISA_ERR_INVALID, "queries q/w/q_seq/q_pos is NULL");
+  if (q->q && !aligned16(q->q)) return fail(MISA_ERR_INVALID, "q must be 16-byte aligned");
+  return MISA_OK;
+}
+
+misa::CacheView view(const misa_cache *c) {
+  misa::CacheView v;
+  v.keys = c->keys;
+  v.scale = c->scale;
+  v.seq_len = c->seq_len;
+  v.pool = c->pool;
+  v.status = c->status;
+  v.n_seq = c->n_seq;
+  v.L_cap = c->L_cap;
+  v.B = c->B;
+  v.fp8 = c->dtype == MISA_KEY_FP8_E4M3;
+  return v;
+}
+
+misa::QueryView view(const misa_queries *q) {
+  misa::QueryView v;
+  v.q = q->q;
+  v.w = q->w;
+  v.q_seq = q->q_seq;
+  v.q_pos = q->q_pos;
+  v.n_q = q->n_q;
+  v.H = q->H;
+  return v;
+}
+
+size_t round_up(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t ws_score(const misa_cache *c, const misa_queries *q) {
+  return round_up(sizeof(float) * (size_t)q->n_q * c->L_cap);
+}
+
+misa_status check_ws(void *ws, size_t have, size_t need) {
+  if (have < need) return fail(MISA_ERR_WORKSPACE, "workspace %zu bytes, need %zu", have, need);
+  if (need > 0 && (!ws || !aligned16(ws))) return fail(MISA_ERR_INVALID, "workspace NULL or not 16-byte aligned");
+  return MISA_OK;
+}
+
+// Scores then top-k, shared by the routed and dense entry points.
+misa_status score_then_topk(const char *who, const misa_cache *cache, const misa_queries *qs,
+                            const int32_t *heads, int h, int k, int32_t *topk, float *scores_out, void *ws,
+                            cudaStream_t stream) {
+  misa::CacheView c = view(cache);
+  misa::QueryView q = view(qs);
+  float *scores = scores_out ? scores_out : static_cast<float *>(ws);
+  cudaError_t e = timed_scoring(stream, [&] {
+    return misa::launch_score_mma(c, q, heads, h, nullptr, 0, scores, cache->L_cap, stream);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  e = misa::launch_topk(c, q, scores, cache->L_cap, 0, nullptr, k, topk, stream);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  return MISA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+misa_status misa_pool_keys(const misa_cache *cache, const void *new_keys, const float *new_scale,
+                           const int32_t *new_pos, int32_t count, misa_stream stream) {
+  misa_status st = check_cache(cache, true);
+  if (st != MISA_OK) return st;
+  if (count < 0) return fail(MISA_ERR_INVALID, "count=%d < 0", count);
+  if (count > 0) {
+    if (!new_keys || !new_pos) return fail(MISA_ERR_INVALID, "append needs new_keys and new_pos");
+    if ((cache->dtype == MISA_KEY_FP8_E4M3) != (new_scale != nullptr))
+      return fail(MISA_ERR_INVALID, "new_scale must be non-NULL exactly for fp8 keys");
+    if (!aligned16(new_keys)) return fail(MISA_ERR_INVALID, "new_keys must be 16-byte aligned");
+    if (count > cache->L_cap) return fail(MISA_ERR_INVALID, "count=%d above L_cap=%d", count, cache->L_cap);
+  }
+  if (injected_failure("misa_pool_keys", &st)) return st;
+  misa::CacheView c = view(cache);
+  cudaError_t e = count == 0 ? misa::launch_pool_rebuild(c, stream)
+                             : misa::launch_pool_append(c, new_keys, new_scale, new_pos, count, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "misa_pool_keys");
+  return MISA_OK;
+}
+
+size_t misa_workspace_bytes(int32_t op, const misa_cache *cache, const misa_queries *qs, int32_t h, int32_t k,
+                            int32_t k_prime) {
+  (void)h;
+  (void)k;
+  if (!cache || !qs || cache->B < 1 || cache->L_cap < 1 || qs->n_q < 0 || qs->H < 1) return 0;
+  switch (op) {
+    case MISA_OP_ROUTE:
+      return round_up(misa::route_ws_bytes(qs->n_q, qs->H, misa::cdiv(cache->L_cap, cache->B)));
+    case MISA_OP_SCORE_TOPK:
+    case MISA_OP_DENSE_TOPK:
+      return ws_score(cache, qs);
+    case MISA_OP_RERANK_TOPK:
+      return k_prime > 0 ? round_up(sizeof(float) * (size_t)qs->n_q * k_prime) : 0;
+    default:
+      return 0;
+  }
+}
+
+misa_status misa_route_heads(const misa_cache *cache, const misa_queries *qs, int32_t h, int32_t *heads,
+                             float *router_scores, void *ws, size_t ws_bytes, misa_stream stream) {
+  misa_status st = check_cache(cache, true);
+  if (st != MISA_OK) return st;
+  if ((st = check_queries(qs)) != MISA_OK) return st;
+  if (h < 1 || h > qs->H) return fail(MISA_ERR_INVALID, "h=%d outside [1, H=%d]", h, qs->H);
+  if (qs->n_q > 0 && !heads) return fail(MISA_ERR_INVALID, "heads is NULL");
+  if ((st = check_ws(ws, ws_bytes, misa_workspace_bytes(MISA_OP_ROUTE, cache, qs, h, 0, 0))) != MISA_OK) return st;
+  if (injected_failure("misa_route_heads", &st)) return st;
+  cudaError_t e = misa::launch_route(view(cache), view(qs), h, heads, router_scores, ws, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "misa_route_heads");
+  return MISA_OK;
+}
+
+misa_status misa_score_topk(const misa_cache *cache, const misa_queries *qs, const int32_t *heads, int32_t h,
+                            int32_t k, int32_t *topk, float *scores_out, void *ws, size_t ws_bytes,
+                            misa_stream stream) {
+  misa_status st = check_cache(cache, false);
+  if (st != MISA_OK) return st;
+  if ((st = check_queries(qs)) != MISA_OK) return st;
+  if (h < 1 || h > qs->H) return fail(MISA_ERR_INVALID, "h=%d outside [1, H=%d]", h, qs->H);
+  if (k < 1) return fail(MISA_ERR_INVALID, "k=%d < 1", k);
+  if (qs->n_q > 0 && (!heads || !topk)) return fail(MISA_ERR_INVALID, "heads/topk is NULL");
+  const size_t need = scores_out ? 0 : misa_workspace_bytes(MISA_OP_SCORE_TOPK, cache, qs, h, k, 0);
+  if ((st = check_ws(ws, ws_bytes, need)) != MISA_OK) return st;
+  if (injected_failure("misa_score_topk", &st)) return st;
+  if (qs->n_q == 0) return MISA_OK;
+  return score_then_topk("misa_score_topk", cache, qs, heads, h, k, topk, scores_out, ws, stream);
+}
+
+misa_status dsa_dense_score_topk(const misa_cache *cache, const misa_queries *qs, int32_t k, int32_t *topk,
+                                 float *scores_out, void *ws, size_t ws_bytes, misa_stream stream) {
+  misa_status st = check_cache(cache, false);
+  if (st != MISA_OK) return st;
+  if ((st = check_queries(qs)) != MISA_OK) return st;
+  if (k < 1) return fail(MISA_ERR_INVALID, "k=%d < 1", k);
+  if (qs->n_q > 0 && !topk) return fail(MISA_ERR_INVALID, "topk is NULL");
+  const size_t need = scores_out ? 0 : misa_workspace_bytes(MISA_OP_DENSE_TOPK, cache, qs, qs->H, k, 0);
+  if ((st = check_ws(ws, ws_bytes, need)) != MISA_OK) return st;
+  if (injected_failure("dsa_dense_score_topk", &st)) return st;
+  if (qs->n_q == 0) return MISA_OK;
+  return score_then_topk("dsa_dense_score_topk", cache, qs, nullptr, qs->H, k, topk, scores_out, ws, stream);
+}
+
+misa_status misa_rerank_topk(const misa_cache *cache, const misa_queries *qs, const int32_t *cand,
+                             int32_t k_prime, int32_t k, int32_t *topk, float *scores_out, void *ws,
+                             size_t ws_bytes, misa_stream stream) {
+  misa_status st = check_cache(cache, false);
+  if (st != MISA_OK) return st;
+  if ((st = check_queries(qs)) != MISA_OK) return st;
+  if (k < 1 || k_prime < k) return fail(MISA_ERR_INVALID, "need 1 <= k=%d <= k_prime=%d", k, k_prime);
+  if (k_prime > MISA_MAX_L) return fail(MISA_ERR_UNSUPPORTED, "k_prime=%d above %d", k_prime, MISA_MAX_L);
+  if (qs->n_q > 0 && (!cand || !topk)) return fail(MISA_ERR_INVALID, "cand/topk is NULL");
+  const size_t need = scores_out ? 0 : misa_workspace_bytes(MISA_OP_RERANK_TOPK, cache, qs, 0, k, k_prime);
+  if ((st = check_ws(ws, ws_bytes, need)) != MISA_OK) return st;
+  if (injected_failure("misa_rerank_topk", &st)) return st;
+  if (qs->n_q == 0) return MISA_OK;
+  misa::CacheView c = view(cache);
+  misa::QueryView q = view(qs);
+  float *scores = scores_out ? scores_out : static_cast<float *>(ws);
+  cudaError_t e = timed_scoring(stream, [&] {
+    return misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, scores, k_prime, stream);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
+  e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, k, topk, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
+  return MISA_OK;
+}
+
+const char *misa_last_error(void) { return g_err; }
+
+const char *misa_status_name(int32_t status) {
+  switch (status) {
+    case MISA_OK: return "MISA_OK";
+    case MISA_ERR_INVALID: return "MISA_ERR_INVALID";
+    case MISA_ERR_UNSUPPORTED: return "MISA_ERR_UNSUPPORTED";
+    case MISA_ERR_WORKSPACE: return "MISA_ERR_WORKSPACE";
+    case MISA_ERR_CUDA: return "MISA_ERR_CUDA";
+    default: return "MISA_STATUS_UNKNOWN";
+  }
+}
+
+int32_t misa_version(void) { return 1; }
+
+void misa_debug_fail_next(int32_t n) { g_fail_next.store(n > 0 ? n : 0); }
+
+void misa_debug_time_scoring(void *start, void *stop) {
+  g_ev_start.store(start);
+  g_ev_stop.store(stop);
+}
+
+}  // extern "C"

@@ -1,0 +1,115 @@
+// Shared device helpers of the MISA / DSA indexer library (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "../../include/misa.h"
+
+namespace misa {
+
+constexpr int D = MISA_D;  // index-key width
+
+// Device view of the caller's cache and queries (plain pointers, by value).
+struct CacheView {
+  const void *keys;
+  const float *scale;
+  int32_t *seq_len;
+  float *pool;
+  uint32_t *status;
+  int n_seq, L_cap, B, fp8;
+};
+
+struct QueryView {
+  const uint16_t *q;
+  const float *w;
+  const int32_t *q_seq;
+  const int32_t *q_pos;
+  int n_q, H;
+};
+
+__device__ __forceinline__ void flag(const CacheView &c, uint32_t bit) {
+  if (c.status) atomicOr(c.status, bit);
+}
+
+// Prefix length L_i = q_pos + 1 of query i, clamped to its sequence.
+__device__ __forceinline__ int query_prefix(const CacheView &c, const QueryView &qv, int i, int *seq) {
+  int s = qv.q_seq[i], p = qv.q_pos[i];
+  if (s < 0 || s >= c.n_seq || p < 0) {
+    flag(c, MISA_DEV_BAD_POSITION);
+    *seq = 0;
+    return 0;
+  }
+  int len = min(c.seq_len[s], c.L_cap);
+  int L = p + 1;
+  if (L > len) {
+    flag(c, MISA_DEV_BAD_POSITION);
+    L = max(len, 0);
+  }
+  *seq = s;
+  return L;
+}
+
+// Order-preserving map of fp32 onto uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b16) { return __uint_as_float(b16 << 16); }
+
+// Two packed bf16 (low half first) -> float2.
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
+  return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+
+// Two e4m3 codes (low byte first) -> two exact f16 values packed in one register.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+  __half2_raw r = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)v, __NV_E4M3);
+  return (uint32_t)r.x | ((uint32_t)r.y << 16);
+}
+
+__device__ __forceinline__ float2 f16x2_to_float2(uint32_t v) {
+  __half2 h = *reinterpret_cast<__half2 *>(&v);
+  return __half22float2(h);
+}
+
+// bf16 bits -> f16 bits (round to nearest; exact for |x| in [2^-14, 65504]
+// and for bf16 values whose 8 significant bits fit f16 subnormals).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  float2 f = bf16x2_to_float2(v);
+  __half2 h = __floats2half2_rn(f.x, f.y);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Warp-level tensor-core MMA m16n8k16, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const void *p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace misa

@@ -1,0 +1,36 @@
+// Host-side launchers shared between the translation units of libmisa.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace misa {
+
+// pool.cu
+cudaError_t launch_pool_rebuild(const CacheView &c, cudaStream_t s);
+cudaError_t launch_pool_append(const CacheView &c, const void *new_keys, const float *new_scale,
+                               const int32_t *new_pos, int count, cudaStream_t s);
+
+// route.cu
+int route_chunks(int M_cap);
+size_t route_ws_bytes(int n_q, int H, int M_cap);
+cudaError_t launch_route(const CacheView &c, const QueryView &q, int h, int32_t *heads, float *router_scores,
+                         void *ws, cudaStream_t s);
+
+// score_mma.cu: scores[i][t] (row stride ld) for t < L_i, heads given per query
+// (heads == nullptr: all H heads, dense).  `gather` != nullptr: row i scores the
+// tokens gather[i][0..n_cols) instead of the prefix (re-rank).
+cudaError_t launch_score_mma(const CacheView &c, const QueryView &q, const int32_t *heads, int h,
+                             const int32_t *gather, int n_cols, float *scores, long long ld, cudaStream_t s);
+
+// topk.cu: per row, the k largest scores; ties to the lower position.
+// Row length comes from the query prefix (gather == nullptr) or is n_cols with
+// positions whose gather entry is < 0 excluded; outputs are token indices
+// (gather[pos] or pos), ascending when gather is ascending.
+cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
+                        const int32_t *gather, int k, int32_t *out, cudaStream_t s);
+
+}  // namespace misa

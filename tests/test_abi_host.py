@@ -1,0 +1,114 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+symbol, validates arguments before any launch, sizes workspaces, and injects
+failures.  None of these touch a GPU (bad arguments are rejected before any
+CUDA call, and injected failures fire before any launch)."""
+import ctypes
+
+import pytest
+
+from long_context_misa_b200 import misa as M
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced on the host
+
+
+def cache(**kw):
+    f = dict(keys=FAKE, scale=None, seq_len=FAKE, pool=FAKE, status=None, n_seq=2, L_cap=4096, d=128, B=64,
+             dtype=M.MISA_KEY_BF16)
+    f.update(kw)
+    return M.misa_cache(**f)
+
+
+def queries(**kw):
+    f = dict(q=FAKE, w=FAKE, q_seq=FAKE, q_pos=FAKE, n_q=2, H=64)
+    f.update(kw)
+    return M.misa_queries(**f)
+
+
+L = M._lib
+by = ctypes.byref
+
+
+def test_exports_every_declared_symbol():
+    names = M.header_symbols()
+    assert len(names) == 11
+    for n in names:
+        assert hasattr(L, n), n
+    assert M.version() == 1
+
+
+def test_status_names():
+    assert M.status_name(M.MISA_ERR_WORKSPACE) == "MISA_ERR_WORKSPACE"
+    assert M.status_name(99) == "MISA_STATUS_UNKNOWN"
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(d=64), M.MISA_ERR_UNSUPPORTED),
+    (dict(B=0), M.MISA_ERR_INVALID),
+    (dict(L_cap=(1 << 18) + 1), M.MISA_ERR_UNSUPPORTED),
+    (dict(keys=None), M.MISA_ERR_INVALID),
+    (dict(keys=FAKE + 8), M.MISA_ERR_INVALID),
+    (dict(dtype=M.MISA_KEY_FP8_E4M3), M.MISA_ERR_INVALID),   # fp8 without scale
+    (dict(scale=FAKE), M.MISA_ERR_INVALID),                  # bf16 with scale
+    (dict(dtype=7), M.MISA_ERR_INVALID),
+])
+def test_cache_validation(bad, status):
+    c = cache(**bad)
+    assert L.misa_route_heads(by(c), by(queries()), 8, FAKE, None, FAKE, 1 << 30, None) == status
+    assert M.last_error() != ""
+
+
+def test_route_argument_checks():
+    c, q = cache(), queries()
+    assert L.misa_route_heads(by(c), by(q), 0, FAKE, None, FAKE, 1 << 30, None) == M.MISA_ERR_INVALID
+    assert L.misa_route_heads(by(c), by(q), 65, FAKE, None, FAKE, 1 << 30, None) == M.MISA_ERR_INVALID
+    assert L.misa_route_heads(by(c), by(queries(H=129)), 8, FAKE, None, FAKE, 1 << 30, None) == \
+        M.MISA_ERR_UNSUPPORTED
+    assert L.misa_route_heads(by(cache(pool=None)), by(q), 8, FAKE, None, FAKE, 1 << 30, None) == \
+        M.MISA_ERR_INVALID
+    assert L.misa_route_heads(by(c), by(q), 8, FAKE, None, FAKE, 16, None) == M.MISA_ERR_WORKSPACE
+    assert "workspace" in M.last_error()
+    assert L.misa_route_heads(None, by(q), 8, FAKE, None, FAKE, 1 << 30, None) == M.MISA_ERR_INVALID
+
+
+def test_score_and_rerank_argument_checks():
+    c, q = cache(), queries()
+    big = 1 << 30
+    assert L.misa_score_topk(by(c), by(q), FAKE, 8, 0, FAKE, None, FAKE, big, None) == M.MISA_ERR_INVALID
+    assert L.misa_score_topk(by(c), by(q), None, 8, 16, FAKE, None, FAKE, big, None) == M.MISA_ERR_INVALID
+    assert L.misa_score_topk(by(c), by(q), FAKE, 8, 16, FAKE, None, FAKE, 100, None) == M.MISA_ERR_WORKSPACE
+    assert L.dsa_dense_score_topk(by(c), by(q), -1, FAKE, None, FAKE, big, None) == M.MISA_ERR_INVALID
+    assert L.misa_rerank_topk(by(c), by(q), FAKE, 8, 16, FAKE, None, FAKE, big, None) == M.MISA_ERR_INVALID
+    assert L.misa_rerank_topk(by(c), by(q), None, 64, 16, FAKE, None, FAKE, big, None) == M.MISA_ERR_INVALID
+    assert L.misa_pool_keys(by(c), FAKE, None, None, 3, None) == M.MISA_ERR_INVALID      # append without pos
+    assert L.misa_pool_keys(by(c), FAKE, None, FAKE, -1, None) == M.MISA_ERR_INVALID
+    assert L.misa_pool_keys(by(cache(dtype=M.MISA_KEY_FP8_E4M3, scale=FAKE)), FAKE, None, FAKE, 1, None) == \
+        M.MISA_ERR_INVALID                                                                   # fp8 append w/o scale
+
+
+def test_workspace_sizes():
+    c, q = cache(n_seq=1, L_cap=1000, B=100), queries(n_q=3, H=16)
+    assert M._lib.misa_workspace_bytes(M.OP_ROUTE, by(c), by(q), 4, 0, 0) >= 4 * 3 * 1 * 16
+    assert M._lib.misa_workspace_bytes(M.OP_SCORE_TOPK, by(c), by(q), 4, 8, 0) >= 4 * 3 * 1000
+    assert M._lib.misa_workspace_bytes(M.OP_RERANK_TOPK, by(c), by(q), 0, 8, 77) >= 4 * 3 * 77
+    assert M._lib.misa_workspace_bytes(9, by(c), by(q), 0, 8, 77) == 0
+    for op in range(4):
+        assert M._lib.misa_workspace_bytes(op, by(c), by(q), 4, 8, 77) % 256 == 0
+
+
+def test_injected_failure_fires_after_validation_before_launch():
+    c, q = cache(), queries()
+    M.debug_fail_next(2)
+    try:
+        # invalid arguments still report INVALID and do not consume an injection
+        assert L.misa_route_heads(by(c), by(q), 0, FAKE, None, FAKE, 1 << 30, None) == M.MISA_ERR_INVALID
+        assert L.misa_route_heads(by(c), by(q), 8, FAKE, None, FAKE, 1 << 30, None) == M.MISA_ERR_CUDA
+        assert "injected" in M.last_error()
+        assert L.misa_score_topk(by(c), by(q), FAKE, 8, 16, FAKE, None, FAKE, 1 << 30, None) == M.MISA_ERR_CUDA
+    finally:
+        M.debug_fail_next(0)
+
+
+def test_python_wrapper_raises():
+    with pytest.raises(M.MisaError) as ei:
+        M._check(M.MISA_ERR_WORKSPACE)
+    assert ei.value.status == M.MISA_ERR_WORKSPACE

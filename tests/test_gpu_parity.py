@@ -1,0 +1,277 @@
+"""GPU parity: every entry point of libmisa against the CPU oracle.
+
+Inputs come from the seeded generator; expected values from the oracle only
+(the oracle's head sets and candidate lists feed the GPU calls that take
+them).  Sizes span several tiles with ragged tails; ragged sequence lengths,
+tiny prefixes, k >= L and h = H_I are covered.
+"""
+import numpy as np
+import pytest
+import torch
+
+from long_context_misa_b200 import inputs as G
+from long_context_misa_b200 import misa as M
+from oracle import misa_oracle as O
+from tests.parity import assert_close, compare_selection, to_device
+
+pytestmark = pytest.mark.gpu
+
+W = G.WORKLOADS
+CASES = {
+    "bf16_normal": W["tiny_decode"].scaled(L=1000, k=50),
+    "bf16_mixture": W["batched_decode"].scaled(n_seq=3, L=2500, B=64, k=100),
+    "fp8_mixture": W["misa_dagger_decode_128k"].scaled(n_seq=3, L=3001, B=128, k=64, k_prime=300),
+    "bf16_prefill": W["causal_prefill"].scaled(L=1500, n_q=70, k=64),
+    "fp8_prefill_h32": W["long_prefill_128k"].scaled(L=2100, n_q=40, B=100, k=33),
+}
+
+
+def make(case, seed=0, ragged=True):
+    wl = CASES[case]
+    inp = G.make_inputs(wl, seed)
+    if ragged and wl.mode == "decode":
+        inp.seq_len = (wl.L - 37 * np.arange(wl.n_seq)).astype(np.int32)
+        inp.q_pos = (inp.seq_len - 1).astype(np.int32)
+    return inp
+
+
+class Ref:
+    """Oracle views of one input set."""
+
+    def __init__(self, inp):
+        self.inp, self.wl = inp, inp.wl
+        self.K = [O.seq_keys(inp.keys, inp.scale, self.wl.key_dtype, s) for s in range(self.wl.n_seq)]
+
+    def query(self, i):
+        q, w = O.query_arrays(self.inp.q, self.inp.w, i)
+        s = int(self.inp.q_seq[i])
+        return q, w, self.K[s], int(self.inp.q_pos[i]) + 1
+
+
+def device_status(cache):
+    torch.cuda.synchronize()
+    return cache.device_status()
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_pool_rebuild(case):
+    inp = make(case)
+    ref = Ref(inp)
+    cache, _ = to_device(inp, torch)
+    M.pool_keys(cache)
+    pool = cache.pool.cpu().numpy()
+    for s in range(inp.wl.n_seq):
+        n = int(inp.seq_len[s])
+        expect = O.pool_keys(ref.K[s], n, inp.wl.B)
+        assert_close(pool[s, :expect.shape[0]], expect, f"pool seq {s}")
+    assert device_status(cache) == 0
+
+
+@pytest.mark.parametrize("case", ["bf16_mixture", "fp8_mixture"])
+@pytest.mark.parametrize("count", [1, 37, 200])
+def test_pool_append(case, count):
+    inp = make(case)
+    wl = inp.wl
+    full_len = inp.seq_len.copy()
+    start = (full_len - count).astype(np.int32)
+    inp_short = make(case)
+    inp_short.seq_len = start.copy()
+    cache, _ = to_device(inp_short, torch)
+    M.pool_keys(cache)                                    # pool of the shorter prefix
+    new = np.stack([inp.keys[s, start[s]:start[s] + count] for s in range(wl.n_seq)])
+    nk = torch.from_numpy(new.view(np.int16) if new.dtype == np.uint16 else new).cuda().contiguous()
+    ns = None
+    if inp.scale is not None:
+        ns = torch.from_numpy(np.stack([inp.scale[s, start[s]:start[s] + count] for s in range(wl.n_seq)])).cuda()
+    # overwrite the cache tail with garbage first so the append must write it
+    for s in range(wl.n_seq):
+        cache.keys[s, start[s]:start[s] + count] = 0
+    pos = torch.from_numpy(start).cuda()
+    M.pool_keys(cache, nk, ns, pos)
+    M.pool_keys(cache, nk, ns, pos)                       # idempotent
+    assert np.array_equal(cache.seq_len.cpu().numpy(), full_len)
+    keys = cache.keys.cpu().numpy()
+    ref = Ref(inp)
+    for s in range(wl.n_seq):
+        n = int(full_len[s])
+        assert np.array_equal(keys[s, :n].view(inp.keys.dtype), inp.keys[s, :n])
+        expect = O.pool_keys(ref.K[s], n, wl.B)
+        assert_close(cache.pool[s, :expect.shape[0]].cpu().numpy(), expect, f"pool after append seq {s}")
+    assert device_status(cache) == 0
+
+
+def test_pool_append_past_capacity_is_flagged():
+    inp = make("bf16_mixture")
+    cache, _ = to_device(inp, torch)
+    M.pool_keys(cache)
+    before = cache.seq_len.clone()
+    nk = torch.zeros(inp.wl.n_seq, 4, 128, dtype=torch.int16, device="cuda")
+    pos = torch.full((inp.wl.n_seq,), inp.wl.L - 2, dtype=torch.int32, device="cuda")
+    M.pool_keys(cache, nk, None, pos)
+    assert device_status(cache) & M.DEV_APPEND_RANGE
+    assert torch.equal(cache.seq_len, before)
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+@pytest.mark.parametrize("h", [1, 8, "H"])
+def test_route_heads(case, h):
+    inp = make(case)
+    ref = Ref(inp)
+    wl = inp.wl
+    h = wl.H if h == "H" else h
+    cache, qs = to_device(inp, torch)
+    M.pool_keys(cache)
+    r_gpu = torch.empty(wl.n_q, wl.H, dtype=torch.float32, device="cuda")
+    heads = M.route_heads(cache, qs, h, router_scores=r_gpu).cpu().numpy()
+    r_gpu = r_gpu.cpu().numpy()
+    ties = 0
+    for i in range(wl.n_q):
+        q, w, K, Li = ref.query(i)
+        r, hs = O.route_query(q, w, K, Li, wl.B, h)
+        assert_close(r_gpu[i], r, f"router scores q{i}")
+        assert np.all(np.diff(heads[i]) > 0)               # ascending, distinct
+        ties += compare_selection(heads[i], hs, lambda j: r[j], h, f"heads q{i}")
+    assert ties <= max(1, wl.n_q // 10), f"{ties} head boundary ties"
+    assert device_status(cache) == 0
+
+
+def _score_case(case, kind, k=None, h=None, seed=0):
+    inp = make(case, seed)
+    ref = Ref(inp)
+    wl = inp.wl
+    k = wl.k if k is None else k
+    h = wl.h if h is None else h
+    cache, qs = to_device(inp, torch)
+    scores = torch.full((wl.n_q, wl.L), float("nan"), dtype=torch.float32, device="cuda")
+    exp = []
+    if kind == "misa":
+        heads_ref = []
+        for i in range(wl.n_q):
+            q, w, K, Li = ref.query(i)
+            heads_ref.append(O.route_query(q, w, K, Li, wl.B, h)[1])
+        heads_dev = torch.from_numpy(np.stack(heads_ref).astype(np.int32)).cuda()
+        top = M.score_topk(cache, qs, heads_dev, k, scores_out=scores).cpu().numpy()
+        for i in range(wl.n_q):
+            q, w, K, Li = ref.query(i)
+            I = O.index_scores(q, w, K[:Li], heads_ref[i])
+            exp.append((I, O.top_k(I, k), Li))
+    else:
+        top = M.dense_score_topk(cache, qs, k, scores_out=scores).cpu().numpy()
+        for i in range(wl.n_q):
+            q, w, K, Li = ref.query(i)
+            d = O.dense_query(q, w, K, Li, k)
+            exp.append((d["scores"], d["topk"], Li))
+    sc = scores.cpu().numpy()
+    ties = 0
+    for i, (I, tk, Li) in enumerate(exp):
+        assert_close(sc[i, :Li], I, f"{kind} scores q{i}")
+        ties += compare_selection(top[i], tk, lambda t: I[t], k, f"{kind} top-k q{i}")
+        got = top[i][top[i] >= 0]
+        assert np.all(np.diff(got) > 0)                    # ascending, distinct
+        assert np.all(top[i][len(got):] == -1) and len(got) == min(k, Li)
+    assert device_status(cache) == 0
+    return ties
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+@pytest.mark.parametrize("kind", ["misa", "dense"])
+def test_score_topk(case, kind):
+    ties = _score_case(case, kind)
+    assert ties <= 4, ties
+
+
+@pytest.mark.parametrize("k", [1, 7, 999, 5000])
+def test_score_topk_k_edges(k):
+    _score_case("bf16_mixture", "misa", k=k)
+
+
+@pytest.mark.parametrize("case", ["bf16_mixture", "fp8_mixture"])
+def test_misa_all_heads_equals_dense(case):
+    # structural reduction (h = H_I routes every head) holds on the GPU path too
+    inp = make(case)
+    wl = inp.wl
+    cache, qs = to_device(inp, torch)
+    heads = torch.arange(wl.H, dtype=torch.int32, device="cuda").repeat(wl.n_q, 1).contiguous()
+    s1 = torch.empty(wl.n_q, wl.L, device="cuda")
+    s2 = torch.empty(wl.n_q, wl.L, device="cuda")
+    a = M.score_topk(cache, qs, heads, wl.k, scores_out=s1)
+    b = M.dense_score_topk(cache, qs, wl.k, scores_out=s2)
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_rerank(case):
+    inp = make(case)
+    ref = Ref(inp)
+    wl = inp.wl
+    kp = wl.k_prime or 4 * wl.k
+    cache, qs = to_device(inp, torch)
+    cands, fine = [], []
+    for i in range(wl.n_q):
+        q, w, K, Li = ref.query(i)
+        c = O.misa_query(q, w, K, Li, wl.B, wl.h, kp)["topk"]
+        cands.append(c)
+        fine.append(O.rerank_query(q, w, K, c, wl.k))
+    cand_dev = torch.from_numpy(np.stack(cands)).cuda()
+    sc = torch.full((wl.n_q, kp), float("nan"), device="cuda")
+    top = M.rerank_topk(cache, qs, cand_dev, wl.k, scores_out=sc).cpu().numpy()
+    sc = sc.cpu().numpy()
+    ties = 0
+    for i in range(wl.n_q):
+        valid = cands[i] >= 0
+        assert_close(sc[i][valid], fine[i]["scores"], f"rerank scores q{i}")
+        smap = dict(zip(fine[i]["cand"].tolist(), fine[i]["scores"].tolist()))
+        ties += compare_selection(top[i], fine[i]["topk"], lambda t: smap[t], wl.k, f"rerank q{i}")
+    assert ties <= 4
+    assert device_status(cache) == 0
+
+
+def test_rerank_with_all_candidates_is_dense():
+    inp = make("bf16_mixture")
+    wl = inp.wl
+    cache, qs = to_device(inp, torch)
+    L = int(inp.seq_len.max())
+    cand = np.full((wl.n_q, L), -1, dtype=np.int32)
+    for i in range(wl.n_q):
+        n = int(inp.q_pos[i]) + 1
+        cand[i, :n] = np.arange(n)
+    a = M.rerank_topk(cache, qs, torch.from_numpy(cand).cuda(), wl.k)
+    b = M.dense_score_topk(cache, qs, wl.k)
+    assert torch.equal(a, b)
+
+
+def test_tiny_prefixes_and_bad_positions():
+    wl = CASES["bf16_prefill"].scaled(L=300, n_q=8, B=64, k=70)
+    inp = G.make_inputs(wl, 3)
+    inp.q_pos = np.array([0, 1, 62, 63, 64, 65, 299, 299], dtype=np.int32)
+    ref = Ref(inp)
+    cache, qs = to_device(inp, torch)
+    M.pool_keys(cache)
+    heads = M.route_heads(cache, qs, 4)
+    top = M.dense_score_topk(cache, qs, wl.k).cpu().numpy()
+    for i in range(wl.n_q):
+        q, w, K, Li = ref.query(i)
+        d = O.dense_query(q, w, K, Li, wl.k)
+        compare_selection(top[i], d["topk"], lambda t: d["scores"][t], wl.k, f"q{i}")
+    assert device_status(cache) == 0
+    # a query past its sequence is clamped and flagged
+    qs.q_pos[0] = 10_000
+    M.dense_score_topk(cache, qs, wl.k)
+    assert device_status(cache) & M.DEV_BAD_POSITION
+
+
+def test_empty_query_batch():
+    inp = make("bf16_mixture")
+    cache, _ = to_device(inp, torch)
+    e = torch.empty(0, 64, 128, dtype=torch.int16, device="cuda")
+    qs = M.Queries(e, torch.empty(0, 64, device="cuda"), torch.empty(0, dtype=torch.int32, device="cuda"),
+                   torch.empty(0, dtype=torch.int32, device="cuda"))
+    assert M.dense_score_topk(cache, qs, 16).shape == (0, 16)
+
+
+def test_needles_selected_by_dense_gpu():
+    inp = make("bf16_mixture", ragged=False)
+    cache, qs = to_device(inp, torch)
+    top = M.dense_score_topk(cache, qs, inp.wl.k).cpu().numpy()
+    for s, p, qi in inp.needles:
+        assert p in set(top[qi].tolist())
