@@ -24,7 +24,6 @@ import argparse
 import json
 import math
 import os
-import subprocess
 import sys
 import time
 
@@ -60,48 +59,63 @@ def score_kernel_bytes(wl):
 
 
 class Clocks:
-    """nvidia-smi sampling during the timed region."""
+    """SM clock and clock-event reasons sampled through NVML (read-only) every
+    ~2 ms in a background thread while the timed region runs."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, index):
-        self.index, self.proc, self.path = index, None, None
+    def __init__(self, torch_device):
+        self.dev, self.samples, self.thread, self.err = torch_device, [], None, None
+
+    def _handle(self, N):
+        import torch
+        p = torch.cuda.get_device_properties(self.dev)
+        try:
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return N.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return N.nvmlDeviceGetHandleByIndex(self.dev.index or 0)
 
     def start(self):
-        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{self.index}.csv")
+        import threading
         try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=self.f, stderr=subprocess.DEVNULL)
-        except (FileNotFoundError, OSError):
-            self.proc = None
+            import pynvml as N
+            N.nvmlInit()
+            h = self._handle(N)
+            self.smax = float(N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM))
+        except Exception as e:  # no NVML: report it, never guess
+            self.err = f"nvml unavailable: {e}"
+            return
+        self.stop_flag = False
+
+        def run():
+            while not self.stop_flag:
+                try:
+                    self.samples.append((float(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)),
+                                         int(N.nvmlDeviceGetCurrentClocksEventReasons(h)),
+                                         N.nvmlDeviceGetPowerUsage(h) / 1000.0))
+                except Exception as e:
+                    self.err = str(e)
+                time.sleep(0.002)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+        time.sleep(0.01)
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        self.proc.wait(timeout=10)
-        self.f.close()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        if self.thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0, "reasons": [self.err or "no samples"]}
+        self.stop_flag = True
+        self.thread.join(timeout=5)
+        sm = [x[0] for x in self.samples]
+        bits = 0
+        for x in self.samples:
+            bits |= x[1]
+        reasons = sorted(n for n, b in self.REASONS.items() if bits & b)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": self.smax, "samples": len(sm),
+                "power_w_max": max((x[2] for x in self.samples), default=None), "reasons": reasons,
+                "source": "NVML polling every ~2 ms during the timed steps"}
 
 
 def cpu_oracle_rate(wl, inp, n_queries, min_seconds=0.0):
@@ -170,8 +184,8 @@ def config_block(wl, l2):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="misa", choices=["misa", "reference"])
     ap.add_argument("--workload", default="misa_dagger_decode_128k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -208,53 +222,61 @@ def main():
     new_keys = torch.from_numpy(last).to(dev).contiguous()
     new_scale = torch.from_numpy(np.stack([inp.scale[s, inp.q_pos[s]:inp.q_pos[s] + 1]
                                            for s in range(wl.n_seq)])).to(dev).contiguous()
-    ws = M.Workspace(dev)
-    heads = torch.empty(wl.n_q, wl.h, dtype=torch.int32, device=dev)
-    cand = torch.empty(wl.n_q, wl.k_prime, dtype=torch.int32, device=dev)
-    top = torch.empty(wl.n_q, wl.k, dtype=torch.int32, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    step = M.MisaDaggerDecode(cache, qs, wl.h, wl.k_prime, wl.k, new_keys, new_scale, pos)
     stream = torch.cuda.current_stream(dev)
-    LAUNCHES_PER_STEP = 7  # append 1, route 2, score+top-k' 2, rerank+top-k 2
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device=dev)
 
-    def step():
-        M.pool_keys(cache, new_keys, new_scale, pos, stream=stream)
-        M.route_heads(cache, qs, wl.h, heads=heads, ws=ws, stream=stream)
-        M.score_topk(cache, qs, heads, wl.k_prime, topk=cand, ws=ws, stream=stream)
-        M.rerank_topk(cache, qs, cand, wl.k, topk=top, ws=ws, stream=stream)
+    def flush_l2():
+        # write 256 MiB, then read another 256 MiB: the inputs leave L2 and the
+        # lines left behind are clean (no write-back lands in the next step)
+        flush.zero_()
+        flush_rd.sum()
+
+    LAUNCHES_PER_STEP = M.MisaDaggerDecode.LAUNCHES
 
     for _ in range(args.warmup):
-        flush.zero_()
-        step()
+        flush_l2()
+        step.run()
     torch.cuda.synchronize()
     assert cache.device_status() == 0, "device status set during warm-up"
 
+    # The step is replayed as one CUDA graph (the kernels of one step, no host
+    # work between them); the routed scoring kernel is bracketed by two event
+    # nodes inside the graph so its own duration is read on every step.
+    ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ka.record(stream)
+    kb.record(stream)
+    M.debug_time_scoring(ka, kb)
+    step.run()
+    torch.cuda.synchronize()
+    step.capture()
+    M.debug_time_scoring(None, None)
+    for _ in range(3):
+        flush_l2()
+        step.replay()
+    torch.cuda.synchronize()
+
     # ---- timed region: K steps, L2 flushed between steps ----
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for a, b in kev:  # materialise the events so their handles exist
-        a.record(stream)
-        b.record(stream)
-    clocks = Clocks(local)
+    step_ms, kern_ms = [], []
+    clocks = Clocks(dev)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
     for i in range(args.steps):
-        flush.zero_()
-        M.debug_time_scoring(*kev[i])
+        flush_l2()
         ev[i][0].record(stream)
-        M.pool_keys(cache, new_keys, new_scale, pos, stream=stream)
-        M.route_heads(cache, qs, wl.h, heads=heads, ws=ws, stream=stream)
-        M.score_topk(cache, qs, heads, wl.k_prime, topk=cand, ws=ws, stream=stream)
-        M.debug_time_scoring(None, None)
-        M.rerank_topk(cache, qs, cand, wl.k, topk=top, ws=ws, stream=stream)
+        step.replay()
         ev[i][1].record(stream)
+        ev[i][1].synchronize()
+        step_ms.append(ev[i][0].elapsed_time(ev[i][1]))
+        kern_ms.append(ka.elapsed_time(kb))
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    kern_ms = [a.elapsed_time(b) for a, b in kev]
     total_ms = float(sum(step_ms))
     if world > 1:
         t = torch.tensor([total_ms], device=dev)
@@ -268,12 +290,13 @@ def main():
     qps = world * wl.n_q / (ms_per_step * 1e-3)
 
     # ---- dense DSA indexer on the same batch (context: the work MISA replaces) ----
+    ws = M.Workspace(dev)
     dense_ms = []
     for _ in range(3):
-        flush.zero_()
+        flush_l2()
         M.dense_score_topk(cache, qs, wl.k, ws=ws, stream=stream)
     for _ in range(5):
-        flush.zero_()
+        flush_l2()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         M.dense_score_topk(cache, qs, wl.k, ws=ws, stream=stream)
@@ -281,7 +304,7 @@ def main():
         torch.cuda.synchronize()
         dense_ms.append(a.elapsed_time(b))
 
-    # ---- end to end through the public API with pinned host buffers ----
+    # ---- end to end through the public API: pinned host inputs in, top-k out ----
     h_keys = torch.from_numpy(last).pin_memory()
     h_scale = new_scale.cpu().pin_memory()
     h_q = torch.from_numpy(inp.q.view(np.int16)).pin_memory()
@@ -290,23 +313,33 @@ def main():
     h_top = torch.empty(wl.n_q, wl.k, dtype=torch.int32).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (h_keys, h_scale, h_q, h_w, h_pos))
     d2h = h_top.numel() * h_top.element_size()
-    e2e_ms = []
-    for i in range(max(3, args.steps // 2)):
-        flush.zero_()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
+
+    def e2e_body():
         new_keys.copy_(h_keys, non_blocking=True)
         new_scale.copy_(h_scale, non_blocking=True)
         qs.q.copy_(h_q, non_blocking=True)
         qs.w.copy_(h_w, non_blocking=True)
         pos.copy_(h_pos, non_blocking=True)
-        step()
-        h_top.copy_(top, non_blocking=True)
+        step.run()
+        h_top.copy_(step.topk, non_blocking=True)
+
+    e2e_body()
+    torch.cuda.synchronize()
+    g_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_e2e):
+        e2e_body()
+    e2e_ms = []
+    for i in range(max(5, args.steps // 2)):
+        flush_l2()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g_e2e.replay()
         b.record(stream)
         b.synchronize()
         e2e_ms.append(a.elapsed_time(b))
-    e2e_step = float(np.mean(e2e_ms[1:] if len(e2e_ms) > 1 else e2e_ms))
+    assert np.array_equal(h_top.numpy(), step.topk.cpu().numpy())
+    e2e_step = float(np.mean(e2e_ms[1:]))
     e2e_value = world * per_step_work / (e2e_step * 1e-3)
 
     if rank == 0:
@@ -323,14 +356,14 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "e4m3 keys -> f16 MMA, f32 accumulate",
+            "vs_baseline": None, "dtype": "e4m3 keys x e4m3 query split (mma.sync), f32 accumulate",
             "data": "synthetic (seeded generator), resident in HBM",
-            "config": config_block(wl, l2="flushed between steps (256 MiB write)"),
+            "config": config_block(wl, l2="flushed between steps: 256 MiB write then 256 MiB read (clean lines)"),
             "queries_per_s": qps,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_step},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
-            "roofline": {"kernel": "routed token scoring (score_mma_kernel<1, fp8>)", "bound": "hbm",
+            "roofline": {"kernel": "routed token scoring (score_stream_kernel<1, e4m3>)", "bound": "hbm",
                          "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                          "traffic": None, "algorithmic_bytes_per_launch": kb, "ms_per_launch": k_ms,
                          "peak_source": f"{src} hbm_gbs"},

@@ -17,12 +17,14 @@ std::atomic<void *> g_ev_start{nullptr}, g_ev_stop{nullptr};
 template <class F>
 cudaError_t timed_scoring(cudaStream_t stream, F &&launch) {
   void *a = g_ev_start.load(), *b = g_ev_stop.load();
+  // External records: inside a stream capture they become event-record nodes
+  // that stamp the time on every graph launch.
   if (a && b) {
-    cudaError_t e = cudaEventRecord(static_cast<cudaEvent_t>(a), stream);
+    cudaError_t e = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a), stream, cudaEventRecordExternal);
     if (e != cudaSuccess) return e;
   }
   cudaError_t e = launch();
-  if (e == cudaSuccess && a && b) e = cudaEventRecord(static_cast<cudaEvent_t>(b), stream);
+  if (e == cudaSuccess && a && b) e = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(b), stream, cudaEventRecordExternal);
   return e;
 }
 

@@ -7,7 +7,9 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
-#include "../../include/misa.h"
+#include <atomic>
+
+#include "misa.h"  // include/ (on the -I path)
 
 namespace misa {
 
@@ -111,5 +113,100 @@ __device__ __forceinline__ uint4 ldg_stream(const void *p) {
 }
 
 __host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// Per-device cached integer (device attributes, occupancy results): computed
+// once per device by `f` on first use, then read without driver calls.
+constexpr int MAX_DEVICES = 64;
+template <class Tag, class F>
+inline int cached_per_device(F &&f) {
+  static std::atomic<int> cache[MAX_DEVICES];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= MAX_DEVICES) return f();
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    v = f();
+    cache[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
+struct SmCountTag {};
+inline int device_sms() {
+  return cached_per_device<SmCountTag>([] {
+    int dev = 0, v = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    return v;
+  });
+}
+
+}  // namespace misa
+
+namespace misa {
+
+// ---------------------------------------------------------------------------
+// mbarrier / bulk-copy helpers (sm_90+ PTX), with time-bounded waits.
+// ---------------------------------------------------------------------------
+
+// Longest time any on-chip pipeline wait may take before the kernel gives up,
+// records MISA_DEV_WAIT_TIMEOUT and returns (nanoseconds of %globaltimer).
+constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete; false if WAIT_LIMIT_NS passed.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) return false;
+  return true;
+}
+
+// Bulk (non-tensor) copy global -> this CTA's shared memory, completing on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
 
 }  // namespace misa

@@ -26,6 +26,11 @@ cudaError_t launch_route(const CacheView &c, const QueryView &q, int h, int32_t 
 cudaError_t launch_score_mma(const CacheView &c, const QueryView &q, const int32_t *heads, int h,
                              const int32_t *gather, int n_cols, float *scores, long long ld, cudaStream_t s);
 
+// score_stream.cu: prefix scoring through the bulk-copy pipeline (used by
+// launch_score_mma when gather == nullptr).
+cudaError_t launch_score_stream(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
+                                long long ld, cudaStream_t s);
+
 // topk.cu: per row, the k largest scores; ties to the lower position.
 // Row length comes from the query prefix (gather == nullptr) or is n_cols with
 // positions whose gather entry is < 0 excluded; outputs are token indices

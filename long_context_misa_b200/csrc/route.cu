@@ -9,11 +9,14 @@
 // where the block cut by the query's prefix end is recomputed from its keys
 // (tokens floor(L_i/B)*B .. q_pos), so routing never sees a future token.
 //
-// route_partial_kernel: grid (chunks of 32 pooled keys, queries), 8 warps.
-//   Lane l of every warp owns pooled key m = chunk*32 + l; warp w owns heads
-//   w, w+8, ...; the query heads and the 32 pooled keys sit in shared memory
-//   as fp32 (pooled rows padded to 129 floats so the 32 lanes hit 32 banks).
-//   Each warp writes sum_m ReLU(q_j . kbar_m) over its lanes for its heads.
+// route_partial_kernel: grid (chunks of 64 pooled keys, queries), 4 warps.
+//   The affinities q_j . kbar_m are a [64 blocks x 128] x [128 x H] product
+//   on mma.sync m16n8k16: each fp32 pooled key is split into bf16 hi + lo
+//   (hi = RN(k), lo = RN(k - hi)) and both halves are multiplied by the bf16
+//   query, so the product keeps ~16 significant bits of the pooled key with
+//   exact products and fp32 accumulation.  Warp w owns blocks 16w..16w+15 of
+//   the chunk; ReLU and the sum over blocks happen on the accumulator
+//   registers, and the four warps' column sums meet in shared memory.
 // route_finish_kernel: one CTA per query sums the chunk partials in a fixed
 //   order, applies |w_j| and keeps the h best heads: head j is kept iff fewer
 //   than h heads beat it (larger r, or equal r and lower index); the kept
@@ -24,21 +27,30 @@
 namespace misa {
 namespace {
 
-constexpr int RB = 32;             // pooled keys per CTA
-constexpr int ROUTE_THREADS = 256; // 8 warps
-constexpr int ROUTE_WARPS = ROUTE_THREADS / 32;
-constexpr int PROW = D + 1;        // padded pooled-row stride (floats)
-constexpr int HG = 8;              // heads accumulated together by one warp
+constexpr int RB = 64;               // pooled keys per CTA
+constexpr int ROUTE_THREADS = 128;   // 4 warps x 16 pooled keys
+constexpr int PSTRIDE = D + 16;      // floats per staged pooled row: conflict-free 16-byte loads
+constexpr int KT = 8;                // k-tiles of 16 over d = 128
+constexpr int MAX_NT = MISA_MAX_H / 8;
 
-size_t route_smem_bytes(int H) { return sizeof(float) * ((size_t)H * D + RB * PROW + 16 * D + D); }
+size_t route_smem_bytes(int H) {
+  const int NT = (H + 7) / 8;
+  return sizeof(float) * ((size_t)RB * PSTRIDE + 16 * D + D + 4 * MAX_NT * 8) + sizeof(uint2) * KT * NT * 32;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
 
 __global__ void __launch_bounds__(ROUTE_THREADS) route_partial_kernel(CacheView c, QueryView qv, float *partial,
                                                                       int n_chunks) {
-  extern __shared__ float smem[];
-  float *q_s = smem;                 // [H][128]
-  float *p_s = q_s + qv.H * D;       // [RB][PROW]
-  float *part = p_s + RB * PROW;     // [16][128] key-sum scratch
-  float *tail = part + 16 * D;       // [128]
+  extern __shared__ __align__(16) float smem[];
+  float *p_s = smem;                          // [RB][PSTRIDE] pooled keys (fp32)
+  float *part = p_s + RB * PSTRIDE;           // [16][128] key-sum scratch
+  float *tail = part + 16 * D;                // [128]
+  float *colsum = tail + D;                   // [4 warps][H]
+  uint2 *bfrag = reinterpret_cast<uint2 *>(colsum + 4 * MAX_NT * 8);  // [kt][nt][lane]
   const int i = blockIdx.y, chunk = blockIdx.x;
   int s;
   const int Li = query_prefix(c, qv, i, &s);
@@ -48,58 +60,117 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_partial_kernel(CacheView 
   const int full = Li / c.B;         // blocks wholly inside the prefix
   const int M_cap = cdiv(c.L_cap, c.B);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int H = qv.H;
+  const int g = lane >> 2, cq = lane & 3;
+  const int H = qv.H, NT = (H + 7) / 8;
 
-  const uint32_t *qsrc = reinterpret_cast<const uint32_t *>(qv.q + (size_t)i * H * D);
-  for (int v = tid; v < H * D / 2; v += blockDim.x) {
-    float2 f = bf16x2_to_float2(__ldg(qsrc + v));
-    q_s[2 * v] = f.x;
-    q_s[2 * v + 1] = f.y;
+  // query heads as B fragments: k-tile kt, lane (g, cq) holds head n = 8nt + g,
+  // physical elements 16kt + 4cq + {0,1} (b0) and + {2,3} (b1)
+  // (fixed trip counts, loads first: one memory round trip, not one per element)
+  {
+    constexpr int PER = KT * MAX_NT * 32 / ROUTE_THREADS;
+    uint2 v[PER];
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+      const int e = tid + it * ROUTE_THREADS;
+      const int l = e & 31, nt = (e >> 5) % NT, kt = (e >> 5) / NT;
+      const int n = nt * 8 + (l >> 2);
+      v[it] = make_uint2(0u, 0u);
+      if (e < KT * NT * 32 && n < H)
+        v[it] = __ldg(reinterpret_cast<const uint2 *>(qv.q + ((size_t)i * H + n) * D + 16 * kt + 4 * (l & 3)));
+    }
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+      const int e = tid + it * ROUTE_THREADS;
+      if (e < KT * NT * 32) bfrag[e] = v[it];
+    }
   }
+  // pooled keys of whole blocks; the rest of the chunk is zero (ReLU(0) = 0)
   const int nb = min(RB, Mi - m0);
-  for (int v = tid; v < RB * D; v += blockDim.x) {
-    const int r = v / D, e = v % D, m = m0 + r;
-    p_s[r * PROW + e] = (r < nb && m < full) ? c.pool[((size_t)s * M_cap + m) * D + e] : 0.f;
+  {
+    constexpr int PER = RB * (D / 4) / ROUTE_THREADS;
+    float4 x[PER];
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+      const int v = tid + it * ROUTE_THREADS;
+      const int r = v / (D / 4), e4 = v % (D / 4), m = m0 + r;
+      x[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < nb && m < full) x[it] = __ldg(reinterpret_cast<const float4 *>(c.pool + ((size_t)s * M_cap + m) * D + 4 * e4));
+    }
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+      const int v = tid + it * ROUTE_THREADS;
+      *reinterpret_cast<float4 *>(p_s + (v / (D / 4)) * PSTRIDE + 4 * (v % (D / 4))) = x[it];
+    }
   }
   const bool has_tail = full < Mi && full >= m0 && full < m0 + RB;  // uniform
   if (has_tail) {
-    block_key_sum<false>(c, s, full * c.B, Li, part, tail);
+    block_key_sum<128>(c, s, full * c.B, Li, part, tail);
     const float inv = 1.f / (float)(Li - full * c.B);
-    if (tid < D) p_s[(full - m0) * PROW + tid] = tail[tid] * inv;
+    p_s[(full - m0) * PSTRIDE + tid] = tail[tid] * inv;
   }
   __syncthreads();
 
-  const bool valid = lane < nb;
-  const float *prow = p_s + lane * PROW;
-  for (int j0 = warp * HG; j0 < H; j0 += ROUTE_WARPS * HG) {
-    float acc[HG];
+  // warp w: pooled keys 16w + g and 16w + g + 8
+  float racc[MAX_NT][2];
 #pragma unroll
-    for (int g = 0; g < HG; ++g) acc[g] = 0.f;
-    for (int d0 = 0; d0 < D; d0 += 32) {
-      float kr[32];
+  for (int nt = 0; nt < MAX_NT; ++nt) racc[nt][0] = racc[nt][1] = 0.f;
+  const float *rowA = p_s + (16 * warp + g) * PSTRIDE;
+  const float *rowB = rowA + 8 * PSTRIDE;
+  float acc[MAX_NT][4];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) kr[e] = prow[d0 + e];
+  for (int nt = 0; nt < MAX_NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 #pragma unroll
-      for (int g = 0; g < HG; ++g) {
-        const int j = min(j0 + g, H - 1);
-        const float4 *qq = reinterpret_cast<const float4 *>(q_s + j * D + d0);
+  for (int kt = 0; kt < KT; ++kt) {
+    const float4 xa = *reinterpret_cast<const float4 *>(rowA + 16 * kt + 4 * cq);
+    const float4 xb = *reinterpret_cast<const float4 *>(rowB + 16 * kt + 4 * cq);
+    uint32_t hi[4], lo[4];
+    hi[0] = pack_bf16(xa.x, xa.y);
+    hi[1] = pack_bf16(xb.x, xb.y);
+    hi[2] = pack_bf16(xa.z, xa.w);
+    hi[3] = pack_bf16(xb.z, xb.w);
+    {
+      const float2 h0 = bf16x2_to_float2(hi[0]), h1 = bf16x2_to_float2(hi[1]);
+      const float2 h2 = bf16x2_to_float2(hi[2]), h3 = bf16x2_to_float2(hi[3]);
+      lo[0] = pack_bf16(xa.x - h0.x, xa.y - h0.y);
+      lo[1] = pack_bf16(xb.x - h1.x, xb.y - h1.y);
+      lo[2] = pack_bf16(xa.z - h2.x, xa.w - h2.y);
+      lo[3] = pack_bf16(xb.z - h3.x, xb.w - h3.y);
+    }
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 qv4 = qq[e4];
-          acc[g] = fmaf(qv4.x, kr[4 * e4 + 0], acc[g]);
-          acc[g] = fmaf(qv4.y, kr[4 * e4 + 1], acc[g]);
-          acc[g] = fmaf(qv4.z, kr[4 * e4 + 2], acc[g]);
-          acc[g] = fmaf(qv4.w, kr[4 * e4 + 3], acc[g]);
-        }
+    for (int nt = 0; nt < MAX_NT; ++nt) {
+      if (nt < NT) {
+        const uint2 b = bfrag[(kt * NT + nt) * 32 + lane];
+        mma_bf16_16816(acc[nt], hi, b.x, b.y);
+        mma_bf16_16816(acc[nt], lo, b.x, b.y);
       }
     }
+  }
 #pragma unroll
-    for (int g = 0; g < HG; ++g) {
-      float v = valid ? fmaxf(acc[g], 0.f) : 0.f;
+  for (int nt = 0; nt < MAX_NT; ++nt) {
+    racc[nt][0] = fmaxf(acc[nt][0], 0.f) + fmaxf(acc[nt][2], 0.f);  // head 8nt + 2cq
+    racc[nt][1] = fmaxf(acc[nt][1], 0.f) + fmaxf(acc[nt][3], 0.f);  // head 8nt + 2cq + 1
+  }
+  // sum over the 8 row groups of the warp (lanes with equal cq)
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0 && j0 + g < H) partial[((size_t)i * n_chunks + chunk) * H + j0 + g] = v;
-    }
+  for (int nt = 0; nt < MAX_NT; ++nt)
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) racc[nt][u] += __shfl_xor_sync(0xffffffffu, racc[nt][u], o);
+  if (g == 0) {
+#pragma unroll
+    for (int nt = 0; nt < MAX_NT; ++nt)
+      if (nt < NT) {
+        colsum[warp * (MAX_NT * 8) + 8 * nt + 2 * cq] = racc[nt][0];
+        colsum[warp * (MAX_NT * 8) + 8 * nt + 2 * cq + 1] = racc[nt][1];
+      }
+  }
+  __syncthreads();
+  if (tid < H) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) v += colsum[w * (MAX_NT * 8) + tid];
+    partial[((size_t)i * n_chunks + chunk) * H + tid] = v;
   }
 }
 
@@ -115,7 +186,8 @@ __global__ void __launch_bounds__(MISA_MAX_H) route_finish_kernel(CacheView c, Q
   float r = 0.f;
   if (j < H) {
     float acc = 0.f;
-    for (int ch = 0; ch < nc; ++ch) acc += partial[((size_t)i * n_chunks + ch) * H + j];
+#pragma unroll 16
+    for (int ch = 0; ch < nc; ++ch) acc += __ldg(partial + ((size_t)i * n_chunks + ch) * H + j);
     r = fabsf(qv.w[(size_t)i * H + j]) * acc;
     r_s[j] = r;
     if (router_scores) router_scores[(size_t)i * H + j] = r;
@@ -154,8 +226,13 @@ cudaError_t launch_route(const CacheView &c, const QueryView &q, int h, int32_t 
   const int M_cap = cdiv(c.L_cap, c.B);
   const int n_chunks = route_chunks(M_cap);
   const size_t smem = route_smem_bytes(q.H);
-  cudaError_t e = cudaFuncSetAttribute(route_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  struct Tag {};
+  const int opt_in = cached_per_device<Tag>([] {
+    return cudaFuncSetAttribute(route_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)route_smem_bytes(MISA_MAX_H)) == cudaSuccess ? 1 : -1;
+  });
+  if (opt_in < 0) return cudaErrorInvalidConfiguration;
+  cudaError_t e;
   float *partial = static_cast<float *>(ws);
   route_partial_kernel<<<dim3(n_chunks, q.n_q), ROUTE_THREADS, smem, s>>>(c, q, partial, n_chunks);
   e = cudaGetLastError();

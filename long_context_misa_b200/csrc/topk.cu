@@ -8,17 +8,20 @@
 // (the lower token index, since positions are ascending token indices).
 //
 // One cluster of CS CTAs (CS in {1,2,4,8}) owns one row; each CTA holds a
-// slice of up to 512*E scores in registers as order-preserving 32-bit keys.
-// Every element has a unique 64-bit composite key (score key, ~position).
-// Radix passes over 8-bit digits of that composite narrow down the k-th
-// largest composite: each pass builds a 256-bin histogram of the still
-// undecided elements in shared memory (warp-aggregated with match.any), the
-// CTAs of the cluster add each other's histograms through distributed shared
-// memory, and every CTA takes the same decision.  A pass stops the search as
-// soon as the undecided elements of the chosen bin are exactly the ones still
-// needed.  The selected positions are then written in ascending order
-// (ballots within a warp, a scan over warps, a prefix over cluster ranks), so
-// the output is deterministic and sorted.  Scores are read once from memory.
+// slice of T*E scores in registers as order-preserving 32-bit keys.  Every
+// element has a unique composite key (score key, 2^18-1-position).  Radix
+// passes over digits of that composite (12, 12, 8 bits of the score key, then
+// 12 and 6 bits of the position, the latter only when scores tie) narrow down
+// the k-th largest composite: each pass builds a 4096-bin histogram of the
+// still undecided elements in shared memory plus a 256-bin coarse summary;
+// after one cluster barrier every CTA adds the cluster's coarse bins through
+// distributed shared memory, picks the coarse bin, then adds only the 16 fine
+// bins inside it (272 remote words per rank instead of 4096), so every CTA
+// takes the same decision at a small exchange cost.  The search stops as soon as the undecided
+// elements of the chosen bin are exactly the ones still needed.  The selected
+// positions are written in ascending order (ballots within a warp, a scan
+// over warps, a prefix over cluster ranks): deterministic and sorted.  Scores
+// are read from memory once; pass 0 also counts the valid elements.
 #include <cooperative_groups.h>
 
 #include "internal.h"
@@ -28,35 +31,53 @@ namespace cg = cooperative_groups;
 namespace misa {
 namespace {
 
-constexpr int TK_THREADS = 512;
-constexpr int TK_WARPS = TK_THREADS / 32;
+constexpr int NB = 4096;              // bins per pass (12-bit digits)
+constexpr int POS_BITS = 18;          // positions < 2^18 = MISA_MAX_L
+constexpr uint32_t POS_MAX = (1u << POS_BITS) - 1u;
 
-struct TopkShared {
-  uint32_t hist[2][256];
-  uint32_t warp_tot[TK_WARPS];
-  uint32_t cta_valid;   // valid elements of this CTA
-  uint32_t cta_sel;     // selected elements of this CTA
-  uint32_t digit, above, in_bin;
-};
+// digit layout of pass p: value (0 = score key, 1 = position key), shift, width
+__device__ __forceinline__ void pass_digit(int p, int &which, int &shift, int &bits) {
+  switch (p) {
+    case 0: which = 0; shift = 20; bits = 12; break;
+    case 1: which = 0; shift = 8; bits = 12; break;
+    case 2: which = 0; shift = 0; bits = 8; break;
+    case 3: which = 1; shift = 6; bits = 12; break;
+    default: which = 1; shift = 0; bits = 6; break;
+  }
+}
+constexpr int N_PASSES = 5;
 
-__device__ __forceinline__ uint32_t block_sum_u32(uint32_t v, uint32_t *scratch /*[TK_WARPS]*/) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+constexpr int NC = NB / 16;           // coarse bins (256)
+constexpr int MAX_CS = 8;
+
+// Sum of word `idx` of `arr` over the first `n` cluster ranks; the remote
+// loads are issued together (fixed trip count) and the own rank reads its
+// shared memory directly.
+__device__ __forceinline__ uint32_t cluster_sum(cg::cluster_group &cl, const uint32_t *arr, int idx, int n, int self) {
+  uint32_t v[MAX_CS];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if (lane == 0) scratch[warp] = v;
-  __syncthreads();
+  for (int r = 0; r < MAX_CS; ++r)
+    v[r] = (r < n) ? (r == self ? arr[idx] : cl.map_shared_rank(arr, r)[idx]) : 0u;
   uint32_t t = 0;
 #pragma unroll
-  for (int w = 0; w < TK_WARPS; ++w) t += scratch[w];
-  __syncthreads();
+  for (int r = 0; r < MAX_CS; ++r) t += v[r];
   return t;
 }
 
-template <int E>
-__global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(CacheView c, QueryView qv, const float *scores,
-                                                             long long ld, int n_cols, const int32_t *gather, int k,
-                                                             int32_t *out) {
-  __shared__ TopkShared sh;
+template <int T>
+struct TopkShared {
+  uint32_t hist[2][NB];                // fine histograms (double-buffered across passes)
+  uint32_t coarse[2][NC];              // sums of 16 fine bins
+  uint32_t warp_tot[T / 32];
+  uint32_t cta_sel;
+  uint32_t digit, above, in_bin, cdigit, cabove;
+};
+
+template <int T, int E, bool GATHER>
+__global__ void __launch_bounds__(T, 1) topk_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
+                                                    int n_cols, const int32_t *gather, int k, int32_t *out) {
+  constexpr int W = T / 32;
+  __shared__ TopkShared<T> sh;
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
@@ -64,85 +85,116 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(CacheView c, QueryV
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int s;
   const int Li = query_prefix(c, qv, row, &s);
-  const int ncols = gather ? n_cols : Li;
-  const int base = rank * (TK_THREADS * E) + warp * (32 * E) + lane;  // position of element e: base + 32e
+  const int ncols = GATHER ? n_cols : Li;
+  const int base = rank * (T * E) + warp * (32 * E) + lane;  // position of element e: base + 32e
 
   uint32_t key[E];
+  int tokid[GATHER ? E : 1];
   uint64_t valid = 0;
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     const int p = base + 32 * e;
     bool v = p < ncols;
-    if (gather && v) {
-      const int t = gather[(size_t)row * n_cols + p];
-      v = t >= 0 && t < Li;
+    if (GATHER) {
+      const int t = v ? __ldg(gather + (size_t)row * n_cols + p) : -1;
+      tokid[GATHER ? e : 0] = t;
+      v = v && t >= 0 && t < Li;
     }
-    key[e] = v ? ordered_key(scores[(size_t)row * ld + p]) : 0u;
+    key[e] = v ? ordered_key(__ldg(scores + (size_t)row * ld + p)) : 0u;
     valid |= (uint64_t)v << e;
   }
 
-  // number of valid elements in the row
-  uint32_t nv = block_sum_u32((uint32_t)__popcll(valid), sh.warp_tot);
-  if (tid == 0) sh.cta_valid = nv;
-  cluster.sync();
-  uint32_t n_valid = 0;
-  for (int r = 0; r < CS; ++r) n_valid += cluster.map_shared_rank(&sh, r)->cta_valid;
-  const uint32_t kk = min((uint32_t)k, n_valid);
-
-  // Composite key K = (key, ~pos); find the kk-th largest by 8-bit digits.
   uint32_t P_hi = 0, M_hi = 0, P_lo = 0, M_lo = 0;
-  uint32_t need = kk;
-  bool done = (kk == n_valid);  // everything valid is selected
-  for (int pass = 0; pass < 8 && !done; ++pass) {
+  uint32_t need = 0, kk = 0;
+  bool done = false;
+  for (int pass = 0; pass < N_PASSES && !done; ++pass) {
+    int which, shift, bits;
+    pass_digit(pass, which, shift, bits);
+    const uint32_t dmask = (1u << bits) - 1u;
     uint32_t *hist = sh.hist[pass & 1];
-    for (int b = tid; b < 256; b += TK_THREADS) hist[b] = 0;
+    for (int b = tid; b < NB; b += T) hist[b] = 0;
     __syncthreads();
-    const int shift = 24 - 8 * (pass & 3);
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      const uint32_t lo = ~(uint32_t)(base + 32 * e);
+      const uint32_t lo = POS_MAX - (uint32_t)(base + 32 * e);
       const bool cand = ((valid >> e) & 1) && (key[e] & M_hi) == P_hi && (lo & M_lo) == P_lo;
-      const uint32_t dig = ((pass < 4 ? key[e] : lo) >> shift) & 255u;
-      const uint32_t tag = cand ? dig : 256u;
-      const unsigned peers = __match_any_sync(0xffffffffu, tag);
-      if (cand && lane == __ffs(peers) - 1) atomicAdd(&hist[dig], (uint32_t)__popc(peers));
+      if (cand) atomicAdd(&hist[((which ? lo : key[e]) >> shift) & dmask], 1u);
+    }
+    __syncthreads();
+    // coarse histogram: 256 bins of 16 fine bins each (local)
+    uint32_t *coarse = sh.coarse[pass & 1];
+    if (tid < NC) {
+      const uint4 *f4 = reinterpret_cast<const uint4 *>(hist + 16 * tid);
+      uint32_t t = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 x = f4[j];
+        t += x.x + x.y + x.z + x.w;
+      }
+      coarse[tid] = t;
     }
     cluster.sync();
-    // totals per bin over the cluster; threads 0..255 own one bin each
-    uint32_t tot = 0;
-    if (tid < 256)
-      for (int r = 0; r < CS; ++r) tot += cluster.map_shared_rank(hist, r)[tid];
-    // suffix sums over bins (bin 255 is the largest digit)
-    uint32_t suf = tot;  // inclusive suffix within the warp (lanes above)
-    if (tid < 256) {
+    // coarse digit from the cluster-wide coarse totals (threads 0..255, one bin each)
+    uint32_t ctot = 0;
+    if (tid < NC) ctot = cluster_sum(cluster, coarse, tid, CS, rank);
+    uint32_t suf = ctot;
+    if (tid < NC) {
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const uint32_t v = __shfl_down_sync(0xffffffffu, suf, o);
         if (lane + o < 32) suf += v;
       }
-      if (lane == 0) sh.warp_tot[warp] = suf;  // warp total
+      if (lane == 0) sh.warp_tot[warp] = suf;
     }
     __syncthreads();
-    if (tid < 256) {
-      uint32_t after = 0;  // bins in higher warps
-      for (int w = warp + 1; w < 8; ++w) after += sh.warp_tot[w];
-      const uint32_t incl = suf + after;       // sum of bins >= tid
-      const uint32_t excl = incl - tot;        // sum of bins > tid
-      if (incl >= need && excl < need) {
-        sh.digit = tid;
-        sh.above = excl;
-        sh.in_bin = tot;
+    if (pass == 0) {
+      uint32_t all = 0;
+      for (int w = 0; w < NC / 32; ++w) all += sh.warp_tot[w];
+      kk = min((uint32_t)k, all);
+      need = kk;
+      if (kk == all) {  // every valid element is selected (uniform decision)
+        done = true;
+        __syncthreads();  // warp_tot is reused below
+        break;
+      }
+    }
+    if (tid < NC) {
+      uint32_t after = 0;
+      for (int w = warp + 1; w < NC / 32; ++w) after += sh.warp_tot[w];
+      const uint32_t incl = suf + after, excl = incl - ctot;
+      if (excl < need && incl >= need) {
+        sh.cdigit = tid;
+        sh.cabove = excl;
+      }
+    }
+    __syncthreads();
+    // fine digit inside the chosen coarse bin (warp 0, lanes 0..15)
+    if (warp == 0) {
+      const uint32_t cd = sh.cdigit, need2 = need - sh.cabove;
+      uint32_t f = 0;
+      if (lane < 16) f = cluster_sum(cluster, hist, 16 * cd + lane, CS, rank);
+      uint32_t fs = f;
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xffffffffu, fs, o);
+        if (lane + o < 16) fs += v;
+      }
+      const uint32_t fex = fs - f;
+      if (lane < 16 && fex < need2 && fs >= need2) {
+        sh.digit = 16 * cd + lane;
+        sh.above = sh.cabove + fex;
+        sh.in_bin = f;
       }
     }
     __syncthreads();
     const uint32_t dsel = sh.digit;
     need -= sh.above;
-    if (pass < 4) {
+    if (which == 0) {
       P_hi |= dsel << shift;
-      M_hi |= 255u << shift;
+      M_hi |= dmask << shift;
     } else {
       P_lo |= dsel << shift;
-      M_lo |= 255u << shift;
+      M_lo |= dmask << shift;
     }
     done = (sh.in_bin == need);
     __syncthreads();
@@ -150,7 +202,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(CacheView c, QueryV
 
   // selection predicate: composite >= (P_hi, P_lo) on the decided bits
   auto selected = [&](int e) -> bool {
-    const uint32_t lo = ~(uint32_t)(base + 32 * e);
+    const uint32_t lo = POS_MAX - (uint32_t)(base + 32 * e);
     const uint32_t kh = key[e] & M_hi, kl = lo & M_lo;
     return ((valid >> e) & 1) && (kh > P_hi || (kh == P_hi && kl >= P_lo));
   };
@@ -160,37 +212,37 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(CacheView c, QueryV
   if (lane == 0) sh.warp_tot[warp] = warp_sel;
   __syncthreads();
   uint32_t off = 0, cta_sel = 0;
-  for (int w = 0; w < TK_WARPS; ++w) {
+  for (int w = 0; w < W; ++w) {
     const uint32_t v = sh.warp_tot[w];
     off += (w < warp) ? v : 0;
     cta_sel += v;
   }
   if (tid == 0) sh.cta_sel = cta_sel;
   cluster.sync();
-  for (int r = 0; r < rank; ++r) off += cluster.map_shared_rank(&sh, r)->cta_sel;
+  off += cluster_sum(cluster, &sh.cta_sel, 0, rank, rank);
   int32_t *orow = out + (size_t)row * k;
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     const uint32_t m = __ballot_sync(0xffffffffu, selected(e));
     if ((m >> lane) & 1) {
       const int p = base + 32 * e;
-      const int t = gather ? gather[(size_t)row * n_cols + p] : p;
+      const int t = GATHER ? tokid[GATHER ? e : 0] : p;
       const uint32_t o = off + __popc(m & ((1u << lane) - 1u));
       if (o < (uint32_t)k) orow[o] = t;
     }
     off += __popc(m);
   }
   if (rank == CS - 1)
-    for (int p = (int)kk + tid; p < k; p += TK_THREADS) orow[p] = -1;
+    for (int p = (int)kk + tid; p < k; p += T) orow[p] = -1;
   cluster.sync();  // no CTA leaves while others may still read its shared memory
 }
 
-template <int E>
-cudaError_t launch_e(int CS, int rows, const CacheView &c, const QueryView &q, const float *scores, long long ld,
-                     int n_cols, const int32_t *gather, int k, int32_t *out, cudaStream_t s) {
+template <int T, int E, bool GATHER>
+cudaError_t launch_te(int CS, int rows, const CacheView &c, const QueryView &q, const float *scores, long long ld,
+                      int n_cols, const int32_t *gather, int k, int32_t *out, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(CS, rows);
-  cfg.blockDim = dim3(TK_THREADS);
+  cfg.blockDim = dim3(T);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -200,7 +252,7 @@ cudaError_t launch_e(int CS, int rows, const CacheView &c, const QueryView &q, c
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, topk_kernel<E>, c, q, scores, ld, n_cols, gather, k, out);
+  return cudaLaunchKernelEx(&cfg, topk_kernel<T, E, GATHER>, c, q, scores, ld, n_cols, gather, k, out);
 }
 
 }  // namespace
@@ -208,23 +260,28 @@ cudaError_t launch_e(int CS, int rows, const CacheView &c, const QueryView &q, c
 cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
                         const int32_t *gather, int k, int32_t *out, cudaStream_t s) {
   if (q.n_q == 0) return cudaSuccess;
-  const int cols = gather ? n_cols : c.L_cap;
-  // smallest register slice E (elements per thread) with at most 8 CTAs per row,
-  // then as many CTAs as the row needs
-  int E = 4;
-  while (E < 64 && (long long)8 * TK_THREADS * E < cols) E *= 2;
-  if (E < 16 && cols > TK_THREADS * E) E = 16;  // rows longer than one CTA: 16 per thread
-  int CS = 1;
-  while ((long long)CS * TK_THREADS * E < cols) CS *= 2;
-  if (CS > 8) return cudaErrorInvalidValue;
-  switch (E) {
-    case 4: return launch_e<4>(CS, q.n_q, c, q, scores, ld, n_cols, gather, k, out, s);
-    case 8: return launch_e<8>(CS, q.n_q, c, q, scores, ld, n_cols, gather, k, out, s);
-    case 16: return launch_e<16>(CS, q.n_q, c, q, scores, ld, n_cols, gather, k, out, s);
-    case 32: return launch_e<32>(CS, q.n_q, c, q, scores, ld, n_cols, gather, k, out, s);
-    case 64: return launch_e<64>(CS, q.n_q, c, q, scores, ld, n_cols, gather, k, out, s);
-    default: return cudaErrorInvalidValue;
-  }
+  const long long cols = gather ? n_cols : c.L_cap;
+  // 1024 threads x E in {4, 8, 16} per CTA and up to 8 CTAs per row; the
+  // longest rows (above 131072) use 512 threads x 64.
+  auto go = [&](int T, int E) -> cudaError_t {
+    int CS = 1;
+    while ((long long)CS * T * E < cols) CS *= 2;
+    if (CS > 8) return cudaErrorInvalidValue;
+    if (gather) {
+      if (T == 1024 && E == 4) return launch_te<1024, 4, true>(CS, q.n_q, c, q, scores, ld, n_cols, gather, k, out, s);
+      if (T == 1024 && E == 8) return launch_te<1024, 8, true>(CS, q.n_q, c, q, scores, ld, n_cols, gather, k, out, s);
+      if (T == 1024 && E == 16) return launch_te<1024, 16, true>(CS, q.n_q, c, q, scores, ld, n_cols, gather, k, out, s);
+      return launch_te<512, 64, true>(CS, q.n_q, c, q, scores, ld, n_cols, gather, k, out, s);
+    }
+    if (T == 1024 && E == 4) return launch_te<1024, 4, false>(CS, q.n_q, c, q, scores, ld, n_cols, gather, k, out, s);
+    if (T == 1024 && E == 8) return launch_te<1024, 8, false>(CS, q.n_q, c, q, scores, ld, n_cols, gather, k, out, s);
+    if (T == 1024 && E == 16) return launch_te<1024, 16, false>(CS, q.n_q, c, q, scores, ld, n_cols, gather, k, out, s);
+    return launch_te<512, 64, false>(CS, q.n_q, c, q, scores, ld, n_cols, gather, k, out, s);
+  };
+  if (cols <= 1024 * 4) return go(1024, 4);
+  if (cols <= 1024 * 8) return go(1024, 8);
+  if (cols <= 8LL * 1024 * 16) return go(1024, 16);
+  return go(512, 64);
 }
 
 }  // namespace misa

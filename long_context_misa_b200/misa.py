@@ -271,3 +271,54 @@ def device_inputs(inp, device="cuda"):
     qs = Queries(q, torch.from_numpy(inp.w).to(device), torch.from_numpy(inp.q_seq).to(device),
                  torch.from_numpy(inp.q_pos).to(device))
     return cache, qs
+
+
+class MisaDaggerDecode:
+    """One MISA-dagger decode step for a batch of sequences, one query each.
+
+    The step appends each query's own index key to the cache (block mean
+    refreshed in the same kernel), routes every query to its top-h heads,
+    keeps the top-k' tokens of the routed scores and re-ranks them with all
+    heads down to k.  All buffers are allocated here once; ``capture()``
+    records the step as a CUDA graph so that ``replay()`` launches all of its
+    kernels with one call.
+
+    new_keys  [n_seq][1][128] (cache dtype), new_scale [n_seq][1] (e4m3 only)
+    and new_pos [n_seq] are device tensors the caller refills between steps
+    (new_pos is normally q_pos).
+    """
+
+    LAUNCHES = 7  # append 1, route 2, score + top-k' 2, re-rank + top-k 2
+
+    def __init__(self, cache: KeyCache, qs: Queries, h: int, k_prime: int, k: int, new_keys: torch.Tensor,
+                 new_scale: Optional[torch.Tensor], new_pos: torch.Tensor):
+        dev = qs.q.device
+        self.cache, self.qs, self.h, self.k_prime, self.k = cache, qs, h, k_prime, k
+        self.new_keys, self.new_scale, self.new_pos = new_keys, new_scale, new_pos
+        self.heads = torch.empty(qs.n_q, h, dtype=torch.int32, device=dev)
+        self.cand = torch.empty(qs.n_q, k_prime, dtype=torch.int32, device=dev)
+        self.topk = torch.empty(qs.n_q, k, dtype=torch.int32, device=dev)
+        need = max(workspace_bytes(OP_ROUTE, cache, qs, h), workspace_bytes(OP_SCORE_TOPK, cache, qs, h, k_prime),
+                   workspace_bytes(OP_RERANK_TOPK, cache, qs, 0, k, k_prime))
+        self.ws = Workspace(dev)
+        self.ws.get(need)
+        self.graph = None
+
+    def run(self, stream=None) -> torch.Tensor:
+        pool_keys(self.cache, self.new_keys, self.new_scale, self.new_pos, stream=stream)
+        route_heads(self.cache, self.qs, self.h, heads=self.heads, ws=self.ws, stream=stream)
+        score_topk(self.cache, self.qs, self.heads, self.k_prime, topk=self.cand, ws=self.ws, stream=stream)
+        rerank_topk(self.cache, self.qs, self.cand, self.k, topk=self.topk, ws=self.ws, stream=stream)
+        return self.topk
+
+    def capture(self) -> "MisaDaggerDecode":
+        """Record run() as a CUDA graph (call run() once before, outside any capture)."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.run()
+        self.graph = g
+        return self
+
+    def replay(self) -> torch.Tensor:
+        self.graph.replay()
+        return self.topk
