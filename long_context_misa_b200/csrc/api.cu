@@ -19,12 +19,16 @@ cudaError_t timed_scoring(cudaStream_t stream, F &&launch) {
   void *a = g_ev_start.load(), *b = g_ev_stop.load();
   // External records: inside a stream capture they become event-record nodes
   // that stamp the time on every graph launch.
+  unsigned flags = 0;
   if (a && b) {
-    cudaError_t e = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a), stream, cudaEventRecordExternal);
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+      flags = cudaEventRecordExternal;
+    cudaError_t e = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(a), stream, flags);
     if (e != cudaSuccess) return e;
   }
   cudaError_t e = launch();
-  if (e == cudaSuccess && a && b) e = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(b), stream, cudaEventRecordExternal);
+  if (e == cudaSuccess && a && b) e = cudaEventRecordWithFlags(static_cast<cudaEvent_t>(b), stream, flags);
   return e;
 }
 
