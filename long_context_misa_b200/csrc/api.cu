@@ -112,6 +112,10 @@ misa::QueryView view(const misa_queries *q) {
 
 size_t round_up(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Workspace of the score + top-k calls: [row histograms][scores (unless the
+// caller passes scores_out)].
+size_t ws_hist(const misa_queries *q) { return round_up(sizeof(uint32_t) * (size_t)q->n_q * misa::TOPK_HIST_BINS); }
+
 size_t ws_score(const misa_cache *c, const misa_queries *q) {
   return round_up(sizeof(float) * (size_t)q->n_q * c->L_cap);
 }
@@ -128,12 +132,15 @@ misa_status score_then_topk(const char *who, const misa_cache *cache, const misa
                             cudaStream_t stream) {
   misa::CacheView c = view(cache);
   misa::QueryView q = view(qs);
-  float *scores = scores_out ? scores_out : static_cast<float *>(ws);
-  cudaError_t e = timed_scoring(stream, [&] {
-    return misa::launch_score_mma(c, q, heads, h, nullptr, 0, scores, cache->L_cap, stream);
+  uint32_t *hist = static_cast<uint32_t *>(ws);
+  float *scores = scores_out ? scores_out : reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + ws_hist(qs));
+  cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  e = timed_scoring(stream, [&] {
+    return misa::launch_score_mma(c, q, heads, h, nullptr, 0, scores, cache->L_cap, hist, stream);
   });
   if (e != cudaSuccess) return cuda_fail(e, who);
-  e = misa::launch_topk(c, q, scores, cache->L_cap, 0, nullptr, k, topk, stream);
+  e = misa::launch_topk(c, q, scores, cache->L_cap, 0, nullptr, hist, k, topk, stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   return MISA_OK;
 }
@@ -172,9 +179,9 @@ size_t misa_workspace_bytes(int32_t op, const misa_cache *cache, const misa_quer
       return round_up(misa::route_ws_bytes(qs->n_q, qs->H, misa::cdiv(cache->L_cap, cache->B)));
     case MISA_OP_SCORE_TOPK:
     case MISA_OP_DENSE_TOPK:
-      return ws_score(cache, qs);
+      return ws_hist(qs) + ws_score(cache, qs);
     case MISA_OP_RERANK_TOPK:
-      return k_prime > 0 ? round_up(sizeof(float) * (size_t)qs->n_q * k_prime) : 0;
+      return k_prime > 0 ? ws_hist(qs) + round_up(sizeof(float) * (size_t)qs->n_q * k_prime) : 0;
     default:
       return 0;
   }
@@ -203,7 +210,7 @@ misa_status misa_score_topk(const misa_cache *cache, const misa_queries *qs, con
   if (h < 1 || h > qs->H) return fail(MISA_ERR_INVALID, "h=%d outside [1, H=%d]", h, qs->H);
   if (k < 1) return fail(MISA_ERR_INVALID, "k=%d < 1", k);
   if (qs->n_q > 0 && (!heads || !topk)) return fail(MISA_ERR_INVALID, "heads/topk is NULL");
-  const size_t need = scores_out ? 0 : misa_workspace_bytes(MISA_OP_SCORE_TOPK, cache, qs, h, k, 0);
+  const size_t need = ws_hist(qs) + (scores_out ? 0 : ws_score(cache, qs));
   if ((st = check_ws(ws, ws_bytes, need)) != MISA_OK) return st;
   if (injected_failure("misa_score_topk", &st)) return st;
   if (qs->n_q == 0) return MISA_OK;
@@ -217,7 +224,7 @@ misa_status dsa_dense_score_topk(const misa_cache *cache, const misa_queries *qs
   if ((st = check_queries(qs)) != MISA_OK) return st;
   if (k < 1) return fail(MISA_ERR_INVALID, "k=%d < 1", k);
   if (qs->n_q > 0 && !topk) return fail(MISA_ERR_INVALID, "topk is NULL");
-  const size_t need = scores_out ? 0 : misa_workspace_bytes(MISA_OP_DENSE_TOPK, cache, qs, qs->H, k, 0);
+  const size_t need = ws_hist(qs) + (scores_out ? 0 : ws_score(cache, qs));
   if ((st = check_ws(ws, ws_bytes, need)) != MISA_OK) return st;
   if (injected_failure("dsa_dense_score_topk", &st)) return st;
   if (qs->n_q == 0) return MISA_OK;
@@ -233,18 +240,21 @@ misa_status misa_rerank_topk(const misa_cache *cache, const misa_queries *qs, co
   if (k < 1 || k_prime < k) return fail(MISA_ERR_INVALID, "need 1 <= k=%d <= k_prime=%d", k, k_prime);
   if (k_prime > MISA_MAX_L) return fail(MISA_ERR_UNSUPPORTED, "k_prime=%d above %d", k_prime, MISA_MAX_L);
   if (qs->n_q > 0 && (!cand || !topk)) return fail(MISA_ERR_INVALID, "cand/topk is NULL");
-  const size_t need = scores_out ? 0 : misa_workspace_bytes(MISA_OP_RERANK_TOPK, cache, qs, 0, k, k_prime);
+  const size_t need = ws_hist(qs) + (scores_out ? 0 : round_up(sizeof(float) * (size_t)qs->n_q * k_prime));
   if ((st = check_ws(ws, ws_bytes, need)) != MISA_OK) return st;
   if (injected_failure("misa_rerank_topk", &st)) return st;
   if (qs->n_q == 0) return MISA_OK;
   misa::CacheView c = view(cache);
   misa::QueryView q = view(qs);
-  float *scores = scores_out ? scores_out : static_cast<float *>(ws);
-  cudaError_t e = timed_scoring(stream, [&] {
-    return misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, scores, k_prime, stream);
+  uint32_t *hist = static_cast<uint32_t *>(ws);
+  float *scores = scores_out ? scores_out : reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + ws_hist(qs));
+  cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
+  e = timed_scoring(stream, [&] {
+    return misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, scores, k_prime, hist, stream);
   });
   if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
-  e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, k, topk, stream);
+  e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, hist, k, topk, stream);
   if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
   return MISA_OK;
 }

@@ -9,6 +9,10 @@
 
 namespace misa {
 
+// Bins of the per-row score histogram the scoring kernels build for the top-k
+// selection: the top 11 bits of the order-preserving key of each score.
+constexpr int TOPK_HIST_BINS = 2048;
+
 // pool.cu
 cudaError_t launch_pool_rebuild(const CacheView &c, cudaStream_t s);
 cudaError_t launch_pool_append(const CacheView &c, const void *new_keys, const float *new_scale,
@@ -23,19 +27,23 @@ cudaError_t launch_route(const CacheView &c, const QueryView &q, int h, int32_t 
 // score_mma.cu: scores[i][t] (row stride ld) for t < L_i, heads given per query
 // (heads == nullptr: all H heads, dense).  `gather` != nullptr: row i scores the
 // tokens gather[i][0..n_cols) instead of the prefix (re-rank).
+// Every launch also adds each written score to row_hist[i][key >> 21] (the
+// caller zeroes row_hist, [n_q][TOPK_HIST_BINS] uint32, beforehand).
 cudaError_t launch_score_mma(const CacheView &c, const QueryView &q, const int32_t *heads, int h,
-                             const int32_t *gather, int n_cols, float *scores, long long ld, cudaStream_t s);
+                             const int32_t *gather, int n_cols, float *scores, long long ld, uint32_t *row_hist,
+                             cudaStream_t s);
 
 // score_stream.cu: prefix scoring through the bulk-copy pipeline (used by
 // launch_score_mma when gather == nullptr).
 cudaError_t launch_score_stream(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
-                                long long ld, cudaStream_t s);
+                                long long ld, uint32_t *row_hist, cudaStream_t s);
 
 // topk.cu: per row, the k largest scores; ties to the lower position.
 // Row length comes from the query prefix (gather == nullptr) or is n_cols with
 // positions whose gather entry is < 0 excluded; outputs are token indices
-// (gather[pos] or pos), ascending when gather is ascending.
+// (gather[pos] or pos), ascending when gather is ascending.  row_hist is the
+// histogram the scoring kernel built over exactly the valid scores.
 cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
-                        const int32_t *gather, int k, int32_t *out, cudaStream_t s);
+                        const int32_t *gather, const uint32_t *row_hist, int k, int32_t *out, cudaStream_t s);
 
 }  // namespace misa

@@ -24,11 +24,13 @@ constexpr int SC_WARPS = SC_THREADS / 32;
 template <int NT, bool FP8>
 __global__ void __launch_bounds__(SC_THREADS) score_gather_kernel(CacheView c, QueryView qv, const int32_t *heads,
                                                                   int h, const int32_t *gather, int n_cols,
-                                                                  float *scores, long long ld, int chunk) {
+                                                                  float *scores, long long ld, int chunk,
+                                                                  uint32_t *row_hist) {
   using F = FragCfg<FP8>;
   constexpr int NV = F::NV, ROW = F::ROW;
   __shared__ uint2 bfrag[F::KT * F::TERMS * NT * 32];
   __shared__ float w_s[NT * 8], scale_s[NT * 8];
+  __shared__ uint32_t shist[TOPK_HIST_BINS];  // this CTA's share of the row histogram
   const int i = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, cq = lane & 3;
@@ -38,6 +40,7 @@ __global__ void __launch_bounds__(SC_THREADS) score_gather_kernel(CacheView c, Q
   if (col0 >= n_cols) return;  // uniform over the CTA
   const int col1 = min(col0 + chunk, n_cols);
 
+  for (int b = tid; b < TOPK_HIST_BINS; b += SC_THREADS) shist[b] = 0;
   build_query_frags<NT, FP8, SC_THREADS>(c, qv, i, heads, h, bfrag, w_s, scale_s, tid, [] { __syncthreads(); });
   __syncthreads();
   float wr[NT][2];
@@ -68,12 +71,13 @@ __global__ void __launch_bounds__(SC_THREADS) score_gather_kernel(CacheView c, Q
   };
 
   int r0 = col0 + warp * 16;
-  if (r0 >= col1) return;  // no barrier follows
-  int tok[2];
+  int tok[2] = {-1, -1};
   uint4 kv[2][NV];
-  tokens(r0, tok);
-  load(tok, kv);
-  while (true) {
+  if (r0 < col1) {
+    tokens(r0, tok);
+    load(tok, kv);
+  }
+  while (r0 < col1) {
     const int rn = r0 + SC_WARPS * 16;
     int tok_n[2] = {-1, -1};
     uint4 kv_n[2][NV];
@@ -87,7 +91,11 @@ __global__ void __launch_bounds__(SC_THREADS) score_gather_kernel(CacheView c, Q
     float acc[NT][4];
     tile_mma<NT, FP8>(kv, bfrag, lane, acc);
     const float2 sums = tile_reduce<NT>(acc, wr);
-    if (cq < 2 && tok[me] >= 0) scores[(size_t)i * ld + r0 + g + 8 * me] = (me ? sums.y : sums.x) * sc;
+    if (cq < 2 && tok[me] >= 0) {
+      const float v = (me ? sums.y : sums.x) * sc;
+      scores[(size_t)i * ld + r0 + g + 8 * me] = v;
+      atomicAdd(&shist[ordered_key(v) >> 21], 1u);
+    }
     if (rn >= col1) break;
     r0 = rn;
 #pragma unroll
@@ -97,21 +105,30 @@ __global__ void __launch_bounds__(SC_THREADS) score_gather_kernel(CacheView c, Q
       for (int ch = 0; ch < NV; ++ch) kv[hr][ch] = kv_n[hr][ch];
     }
   }
+  __syncthreads();
+  uint32_t *rh = row_hist + (size_t)i * TOPK_HIST_BINS;
+  for (int b = tid; b < TOPK_HIST_BINS; b += SC_THREADS) {
+    const uint32_t v = shist[b];
+    if (v) atomicAdd(rh + b, v);
+  }
 }
 
 template <int NT, bool FP8>
 cudaError_t launch_gather(dim3 grid, const CacheView &c, const QueryView &q, const int32_t *heads, int h,
-                          const int32_t *gather, int n_cols, float *scores, long long ld, int chunk, cudaStream_t s) {
-  score_gather_kernel<NT, FP8><<<grid, SC_THREADS, 0, s>>>(c, q, heads, h, gather, n_cols, scores, ld, chunk);
+                          const int32_t *gather, int n_cols, float *scores, long long ld, int chunk,
+                          uint32_t *row_hist, cudaStream_t s) {
+  score_gather_kernel<NT, FP8><<<grid, SC_THREADS, 0, s>>>(c, q, heads, h, gather, n_cols, scores, ld, chunk,
+                                                           row_hist);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_score_mma(const CacheView &c, const QueryView &q, const int32_t *heads, int h,
-                             const int32_t *gather, int n_cols, float *scores, long long ld, cudaStream_t s) {
+                             const int32_t *gather, int n_cols, float *scores, long long ld, uint32_t *row_hist,
+                             cudaStream_t s) {
   if (q.n_q == 0) return cudaSuccess;
-  if (!gather) return launch_score_stream(c, q, heads, h, scores, ld, s);
+  if (!gather) return launch_score_stream(c, q, heads, h, scores, ld, row_hist, s);
   const int h_eff = heads ? h : q.H;
   int NT = 1;
   while (NT * 8 < h_eff) NT *= 2;
@@ -125,8 +142,8 @@ cudaError_t launch_score_mma(const CacheView &c, const QueryView &q, const int32
   const dim3 grid(splits, q.n_q);
 #define MISA_GATHER_CASE(N)                                                                          \
   case N:                                                                                            \
-    return c.fp8 ? launch_gather<N, true>(grid, c, q, heads, h, gather, n_cols, scores, ld, chunk, s) \
-                 : launch_gather<N, false>(grid, c, q, heads, h, gather, n_cols, scores, ld, chunk, s);
+    return c.fp8 ? launch_gather<N, true>(grid, c, q, heads, h, gather, n_cols, scores, ld, chunk, row_hist, s) \
+                 : launch_gather<N, false>(grid, c, q, heads, h, gather, n_cols, scores, ld, chunk, row_hist, s);
   switch (NT) {
     MISA_GATHER_CASE(1)
     MISA_GATHER_CASE(2)

@@ -63,7 +63,8 @@ __device__ __forceinline__ void cp_async_wait() {
 // groups inside the cache); otherwise they are read one by one.
 template <int NT, bool FP8>
 __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, QueryView qv, const int32_t *heads,
-                                                               int h, float *scores, long long ld, int scale_vec) {
+                                                               int h, float *scores, long long ld, int scale_vec,
+                                                               uint32_t *row_hist) {
   using Cfg = StreamCfg<NT, FP8>;
   using F = FragCfg<FP8>;
   constexpr int NS = Cfg::NS, ROW = Cfg::ROW, NV = F::NV, TT = Cfg::TT;
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint2 bfrag[NB * 32];
   __shared__ float w_s[NT * 8], scale_s[NT * 8];
+  __shared__ uint32_t shist[TOPK_HIST_BINS];  // this CTA's share of the row histogram
 
   const int i = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -120,6 +122,7 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
   };
 #pragma unroll
   for (int j = 0; j < NS - 1; ++j) issue(j);  // start streaming before the query set-up
+  for (int b = tid; b < TOPK_HIST_BINS; b += THREADS) shist[b] = 0;
 
   build_query_frags<NT, FP8, THREADS>(c, qv, i, heads, h, bfrag, w_s, scale_s, tid, [] { __syncthreads(); });
   __syncthreads();
@@ -174,15 +177,25 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
         tile_mma<NT, FP8>(kv[m], bfrag, lane, acc);
       const float2 sums = tile_reduce<NT>(acc, wr);
       const int trow = t0 + 16 * m + g + 8 * me;
-      if (cq < 2 && trow < Li) scores[(size_t)i * ld + trow] = (me ? sums.y : sums.x) * sc[m];
+      if (cq < 2 && trow < Li) {
+        const float v = (me ? sums.y : sums.x) * sc[m];
+        scores[(size_t)i * ld + trow] = v;
+        atomicAdd(&shist[ordered_key(v) >> 21], 1u);
+      }
     }
   }
   cp_async_wait<0>();
+  __syncthreads();
+  uint32_t *rh = row_hist + (size_t)i * TOPK_HIST_BINS;
+  for (int b = tid; b < TOPK_HIST_BINS; b += THREADS) {
+    const uint32_t v = shist[b];
+    if (v) atomicAdd(rh + b, v);
+  }
 }
 
 template <int NT, bool FP8>
 cudaError_t launch_nt(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
-                      long long ld, cudaStream_t s) {
+                      long long ld, uint32_t *row_hist, cudaStream_t s) {
   constexpr int SMEM = WARPS * StreamCfg<NT, FP8>::WARP_BYTES;
   const int sms = device_sms();
   // resident CTAs per SM (also sets the shared-memory opt-in), once per device
@@ -202,22 +215,23 @@ cudaError_t launch_nt(const CacheView &c, const QueryView &q, const int32_t *hea
   int splits = max(1, per_sm * sms / q.n_q);
   splits = min(splits, max(1, cdiv(cdiv(c.L_cap, StreamCfg<NT, FP8>::TT), 2 * WARPS)));  // >= 2 tiles per warp
   const int scale_vec = FP8 && (reinterpret_cast<uintptr_t>(c.scale) & 15) == 0 && c.L_cap % 4 == 0;
-  score_stream_kernel<NT, FP8><<<dim3(splits, q.n_q), THREADS, SMEM, s>>>(c, q, heads, h, scores, ld, scale_vec);
+  score_stream_kernel<NT, FP8><<<dim3(splits, q.n_q), THREADS, SMEM, s>>>(c, q, heads, h, scores, ld, scale_vec,
+                                                                                      row_hist);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_score_stream(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
-                                long long ld, cudaStream_t s) {
+                                long long ld, uint32_t *row_hist, cudaStream_t s) {
   if (q.n_q == 0) return cudaSuccess;
   const int h_eff = heads ? h : q.H;
   int NT = 1;
   while (NT * 8 < h_eff) NT *= 2;
 #define MISA_STREAM_CASE(N)                                                   \
   case N:                                                                     \
-    return c.fp8 ? launch_nt<N, true>(c, q, heads, h, scores, ld, s)          \
-                 : launch_nt<N, false>(c, q, heads, h, scores, ld, s);
+    return c.fp8 ? launch_nt<N, true>(c, q, heads, h, scores, ld, row_hist, s) \
+                 : launch_nt<N, false>(c, q, heads, h, scores, ld, row_hist, s);
   switch (NT) {
     MISA_STREAM_CASE(1)
     MISA_STREAM_CASE(2)

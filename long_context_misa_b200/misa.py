@@ -223,8 +223,7 @@ def score_topk(cache: KeyCache, qs: Queries, heads: torch.Tensor, k: int, topk: 
     h = int(heads.shape[1])
     if topk is None:
         topk = torch.empty(qs.n_q, k, dtype=torch.int32, device=dev)
-    nb = 0 if scores_out is not None else workspace_bytes(OP_SCORE_TOPK, cache, qs, h, k)
-    buf, nb = _ws(ws, nb, dev)
+    buf, nb = _ws(ws, workspace_bytes(OP_SCORE_TOPK, cache, qs, h, k), dev)
     _check(_lib.misa_score_topk(ctypes.byref(cache.struct), ctypes.byref(qs.struct), _ptr(heads), h, k,
                                 _ptr(topk), _ptr(scores_out), _ptr(buf), nb, _stream(stream)))
     return topk
@@ -236,8 +235,7 @@ def dense_score_topk(cache: KeyCache, qs: Queries, k: int, topk: Optional[torch.
     dev = qs.q.device
     if topk is None:
         topk = torch.empty(qs.n_q, k, dtype=torch.int32, device=dev)
-    nb = 0 if scores_out is not None else workspace_bytes(OP_DENSE_TOPK, cache, qs, qs.H, k)
-    buf, nb = _ws(ws, nb, dev)
+    buf, nb = _ws(ws, workspace_bytes(OP_DENSE_TOPK, cache, qs, qs.H, k), dev)
     _check(_lib.dsa_dense_score_topk(ctypes.byref(cache.struct), ctypes.byref(qs.struct), k, _ptr(topk),
                                      _ptr(scores_out), _ptr(buf), nb, _stream(stream)))
     return topk
@@ -250,8 +248,7 @@ def rerank_topk(cache: KeyCache, qs: Queries, cand: torch.Tensor, k: int, topk: 
     k_prime = int(cand.shape[1])
     if topk is None:
         topk = torch.empty(qs.n_q, k, dtype=torch.int32, device=dev)
-    nb = 0 if scores_out is not None else workspace_bytes(OP_RERANK_TOPK, cache, qs, 0, k, k_prime)
-    buf, nb = _ws(ws, nb, dev)
+    buf, nb = _ws(ws, workspace_bytes(OP_RERANK_TOPK, cache, qs, 0, k, k_prime), dev)
     _check(_lib.misa_rerank_topk(ctypes.byref(cache.struct), ctypes.byref(qs.struct), _ptr(cand), k_prime, k,
                                  _ptr(topk), _ptr(scores_out), _ptr(buf), nb, _stream(stream)))
     return topk
