@@ -210,6 +210,39 @@ MISA_API misa_status misa_rerank_topk(const misa_cache *cache, const misa_querie
                              void *ws, size_t ws_bytes, misa_stream stream);
 
 /*
+ * misa_rerank_topk without a caller workspace and without any allocation.
+ * The paper has no counterpart of this call: it changes where the scratch
+ * lives, not what is computed.  Outputs, ordering and errors are those of
+ * misa_rerank_topk.
+ *
+ * Who needs it: a caller that cannot hand the library device memory, such as
+ * a plain C host program with no device allocator of its own, or an engine
+ * that has reserved all free device memory for its key cache up front, where
+ * a cudaMalloc would fail or stall the device.  The scratch (the per-row score
+ * histograms and, when scores_out is NULL, the candidate scores) lives in a
+ * fixed array of MISA_NOALLOC_SCRATCH_BYTES inside the library's device
+ * image, one per device.  The call allocates and frees nothing; it zeroes the
+ * histogram part of the array on `stream` before use.
+ *
+ * Scratch needed: 8 KiB per query for the histograms, plus 4 * k_prime bytes
+ * per query when scores_out is NULL, each part rounded up to 256 bytes (8
+ * queries with k_prime = 8192: 320 KiB).  A larger need returns
+ * MISA_ERR_WORKSPACE and launches nothing; use misa_rerank_topk then.
+ *
+ * Limits of a shared array: calls that may overlap on one device (different
+ * streams, or host threads without ordering between them) race on it and
+ * give wrong results; calls in stream order on one stream are safe.  The
+ * first call on each device looks up the array's device address with that
+ * device current (it may load the library's device code), so make it once
+ * before any stream capture.  A failed lookup returns MISA_ERR_CUDA.
+ */
+#define MISA_NOALLOC_SCRATCH_BYTES (4u << 20) /* 4 MiB per device */
+
+MISA_API misa_status misa_rerank_topk_noalloc(const misa_cache *cache, const misa_queries *qs,
+                                              const int32_t *cand, int32_t k_prime, int32_t k,
+                                              int32_t *topk, float *scores_out, misa_stream stream);
+
+/*
  * Workspace bytes the call `op` (misa_op) needs for these shapes; 0 on
  * invalid arguments.  Host-only, launches nothing.
  */

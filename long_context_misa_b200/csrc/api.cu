@@ -145,6 +145,30 @@ misa_status score_then_topk(const char *who, const misa_cache *cache, const misa
   return MISA_OK;
 }
 
+// Scratch of misa_rerank_topk_noalloc: part of the library's device image, so
+// the caller never supplies memory and the call never allocates any.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MISA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up on the
+// first call per device (with that device current) and cached.
+misa_status noalloc_scratch(const char *who, void **out) {
+  static std::atomic<void *> addr[misa::MAX_DEVICES];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  if (dev < 0 || dev >= misa::MAX_DEVICES)
+    return fail(MISA_ERR_UNSUPPORTED, "%s: device %d outside [0, %d)", who, dev, misa::MAX_DEVICES);
+  void *p = addr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk_noalloc: cudaGetSymbolAddress");
+    if (!p) return fail(MISA_ERR_CUDA, "%s: cudaGetSymbolAddress returned NULL", who);
+    addr[dev].store(p, std::memory_order_release);
+  }
+  *out = p;
+  return MISA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -256,6 +280,41 @@ misa_status misa_rerank_topk(const misa_cache *cache, const misa_queries *qs, co
   if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
   e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, hist, k, topk, stream);
   if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
+  return MISA_OK;
+}
+
+misa_status misa_rerank_topk_noalloc(const misa_cache *cache, const misa_queries *qs, const int32_t *cand,
+                                     int32_t k_prime, int32_t k, int32_t *topk, float *scores_out,
+                                     misa_stream stream) {
+  const char *who = "misa_rerank_topk_noalloc";
+  misa_status st = check_cache(cache, false);
+  if (st != MISA_OK) return st;
+  if ((st = check_queries(qs)) != MISA_OK) return st;
+  if (k < 1 || k_prime < k) return fail(MISA_ERR_INVALID, "need 1 <= k=%d <= k_prime=%d", k, k_prime);
+  if (k_prime > MISA_MAX_L) return fail(MISA_ERR_UNSUPPORTED, "k_prime=%d above %d", k_prime, MISA_MAX_L);
+  if (qs->n_q > 0 && (!cand || !topk)) return fail(MISA_ERR_INVALID, "cand/topk is NULL");
+  const size_t need = ws_hist(qs) + (scores_out ? 0 : round_up(sizeof(float) * (size_t)qs->n_q * k_prime));
+  if (need > MISA_NOALLOC_SCRATCH_BYTES)
+    return fail(MISA_ERR_WORKSPACE,
+                "%s: n_q=%d, k_prime=%d need %zu bytes of scratch, the fixed array holds %u; pass scores_out, "
+                "split the batch, or call misa_rerank_topk with a workspace",
+                who, qs->n_q, k_prime, need, MISA_NOALLOC_SCRATCH_BYTES);
+  if (injected_failure(who, &st)) return st;
+  void *ws = nullptr;
+  if ((st = noalloc_scratch(who, &ws)) != MISA_OK) return st;
+  if (qs->n_q == 0) return MISA_OK;
+  misa::CacheView c = view(cache);
+  misa::QueryView q = view(qs);
+  uint32_t *hist = static_cast<uint32_t *>(ws);
+  float *scores = scores_out ? scores_out : reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + ws_hist(qs));
+  cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  e = timed_scoring(stream, [&] {
+    return misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, scores, k_prime, hist, stream);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, hist, k, topk, stream);
+  if (e != cudaSuccess) return cuda_fail(e, who);
   return MISA_OK;
 }
 

@@ -32,6 +32,7 @@ MISA_KEY_BF16, MISA_KEY_FP8_E4M3 = 0, 1
 OP_ROUTE, OP_SCORE_TOPK, OP_DENSE_TOPK, OP_RERANK_TOPK = range(4)
 DEV_BAD_POSITION, DEV_APPEND_RANGE, DEV_WAIT_TIMEOUT, DEV_BAD_HEAD = 1, 2, 4, 8
 D = 128
+NOALLOC_SCRATCH_BYTES = 4 << 20  # MISA_NOALLOC_SCRATCH_BYTES
 
 
 class MisaError(RuntimeError):
@@ -63,6 +64,7 @@ def _load() -> ctypes.CDLL:
         "misa_score_topk": (I32, [C, Q, P, I32, I32, P, P, P, SZ, P]),
         "dsa_dense_score_topk": (I32, [C, Q, I32, P, P, P, SZ, P]),
         "misa_rerank_topk": (I32, [C, Q, P, I32, I32, P, P, P, SZ, P]),
+        "misa_rerank_topk_noalloc": (I32, [C, Q, P, I32, I32, P, P, P]),
         "misa_workspace_bytes": (SZ, [I32, C, Q, I32, I32, I32]),
         "misa_last_error": (ctypes.c_char_p, []),
         "misa_status_name": (ctypes.c_char_p, [I32]),
@@ -251,6 +253,19 @@ def rerank_topk(cache: KeyCache, qs: Queries, cand: torch.Tensor, k: int, topk: 
     buf, nb = _ws(ws, workspace_bytes(OP_RERANK_TOPK, cache, qs, 0, k, k_prime), dev)
     _check(_lib.misa_rerank_topk(ctypes.byref(cache.struct), ctypes.byref(qs.struct), _ptr(cand), k_prime, k,
                                  _ptr(topk), _ptr(scores_out), _ptr(buf), nb, _stream(stream)))
+    return topk
+
+
+def rerank_topk_noalloc(cache: KeyCache, qs: Queries, cand: torch.Tensor, topk: torch.Tensor,
+                        scores_out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """misa_rerank_topk_noalloc: the fine stage with the library's fixed scratch.
+
+    Neither this wrapper nor the library allocates: ``topk`` ([n_q][k] int32,
+    k = topk.shape[1]) and the optional ``scores_out`` are the caller's.
+    """
+    k_prime, k = int(cand.shape[1]), int(topk.shape[1])
+    _check(_lib.misa_rerank_topk_noalloc(ctypes.byref(cache.struct), ctypes.byref(qs.struct), _ptr(cand), k_prime,
+                                         k, _ptr(topk), _ptr(scores_out), _stream(stream)))
     return topk
 
 

@@ -30,7 +30,7 @@ by = ctypes.byref
 
 def test_exports_every_declared_symbol():
     names = M.header_symbols()
-    assert len(names) == 11
+    assert len(names) == 12
     for n in names:
         assert hasattr(L, n), n
     assert M.version() == 1
@@ -112,3 +112,21 @@ def test_python_wrapper_raises():
     with pytest.raises(M.MisaError) as ei:
         M._check(M.MISA_ERR_WORKSPACE)
     assert ei.value.status == M.MISA_ERR_WORKSPACE
+
+
+def test_noalloc_rerank_rejects_before_any_cuda_call():
+    c, q = cache(), queries(n_q=8)
+    assert L.misa_rerank_topk_noalloc(by(c), by(q), FAKE, 8, 16, FAKE, None, None) == M.MISA_ERR_INVALID
+    assert L.misa_rerank_topk_noalloc(by(c), by(q), None, 64, 16, FAKE, None, None) == M.MISA_ERR_INVALID
+    # 8 queries x 131072 candidate scores do not fit the fixed scratch array
+    assert L.misa_rerank_topk_noalloc(by(c), by(q), FAKE, 131072, 16, FAKE, None, None) == M.MISA_ERR_WORKSPACE
+    assert "fixed array" in M.last_error()
+    # histograms alone of 1024 queries (8 MiB) do not fit either, even with scores_out
+    assert L.misa_rerank_topk_noalloc(by(c), by(queries(n_q=1024)), FAKE, 64, 16, FAKE, FAKE, None) == \
+        M.MISA_ERR_WORKSPACE
+    M.debug_fail_next(1)
+    try:
+        assert L.misa_rerank_topk_noalloc(by(c), by(q), FAKE, 64, 16, FAKE, None, None) == M.MISA_ERR_CUDA
+        assert "injected" in M.last_error()
+    finally:
+        M.debug_fail_next(0)
