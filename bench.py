@@ -58,6 +58,13 @@ def score_kernel_bytes(wl):
     return wl.n_seq * wl.L * row + wl.n_q * wl.h * (wl.d * 2 + 4)
 
 
+# DRAM bytes (read + write) of one routed scoring launch on the MISA-dagger
+# decode workload at L = 128K, from the ncu capture summarised in
+# profiles/score_stream_kernel_misa_dagger_decode_128k.md.  Valid only for
+# that workload and that kernel version; reported as null elsewhere.
+STREAM_TRAFFIC_BYTES = {"misa_dagger_decode_128k": 143_097_344}
+
+
 class Clocks:
     """SM clock and clock-event reasons sampled through NVML (read-only) every
     ~2 ms in a background thread while the timed region runs."""
@@ -356,7 +363,8 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "e4m3 keys x e4m3 query split (mma.sync), f32 accumulate",
+            "vs_baseline": None, "dtype": "e4m3",
+            "dtype_detail": "e4m3 keys x two-term e4m3 split of the bf16 query (mma.sync), f32 accumulate",
             "data": "synthetic (seeded generator), resident in HBM",
             "config": config_block(wl, l2="flushed between steps: 256 MiB write then 256 MiB read (clean lines)"),
             "queries_per_s": qps,
@@ -365,7 +373,7 @@ def main():
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "roofline": {"kernel": "routed token scoring (score_stream_kernel<1, e4m3>)", "bound": "hbm",
                          "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                         "traffic": None, "algorithmic_bytes_per_launch": kb, "ms_per_launch": k_ms,
+                         "traffic": STREAM_TRAFFIC_BYTES.get(wl.name), "algorithmic_bytes_per_launch": kb, "ms_per_launch": k_ms,
                          "peak_source": f"{src} hbm_gbs"},
             "dense_dsa": {"ms": float(np.median(dense_ms)), "misa_dagger_step_ms": ms_per_step,
                           "speedup_vs_dense": float(np.median(dense_ms)) / ms_per_step},
