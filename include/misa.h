@@ -20,7 +20,9 @@
  *  - Every pointer inside misa_cache / misa_queries and every buffer argument
  *    is DEVICE memory owned by the caller.  The library never allocates or
  *    frees memory; scratch space is the caller's workspace `ws`, sized by
- *    misa_workspace_bytes() and 16-byte aligned.
+ *    misa_workspace_bytes() and 16-byte aligned.  The top-k calls need a
+ *    workspace even when scores_out is given (per-row score histograms and,
+ *    for few long rows, a compact candidate list).
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
  *    default stream).  Outputs are valid in stream order.  Nothing blocks the
  *    host; the library keeps no state between calls other than cached device
@@ -197,8 +199,9 @@ MISA_API misa_status dsa_dense_score_topk(const misa_cache *cache, const misa_qu
  * Fine stage of MISA-dagger ("Hierarchical variant": the original DSA indexer
  * with all H_I heads re-scores only the k' candidates from the routed pass
  * and recovers the final top-k).
- *   cand       [n_q][k_prime] int32 token indices (any order; -1 entries and
- *              indices outside the query's prefix are ignored)
+ *   cand       [n_q][k_prime] int32 distinct token indices in any order (-1
+ *              entries and indices outside the query's prefix are ignored;
+ *              a repeated token is returned at most once)
  *   topk       [n_q][k] int32 out (ascending token indices, -1 padded)
  *   scores_out [n_q][k_prime] fp32 out or NULL: dense score of cand[i][j]
  *              (unspecified where the candidate is ignored)
@@ -224,9 +227,9 @@ MISA_API misa_status misa_rerank_topk(const misa_cache *cache, const misa_querie
  * image, one per device.  The call allocates and frees nothing; it zeroes the
  * histogram part of the array on `stream` before use.
  *
- * Scratch needed: 8 KiB per query for the histograms, plus 4 * k_prime bytes
- * per query when scores_out is NULL, each part rounded up to 256 bytes (8
- * queries with k_prime = 8192: 320 KiB).  A larger need returns
+ * Scratch needed: 8196 bytes per query for the histograms, plus 4 * k_prime
+ * bytes per query when scores_out is NULL, each part rounded up to 256 bytes
+ * (8 queries with k_prime = 8192: about 320 KiB).  A larger need returns
  * MISA_ERR_WORKSPACE and launches nothing; use misa_rerank_topk then.
  *
  * Limits of a shared array: calls that may overlap on one device (different
@@ -243,8 +246,10 @@ MISA_API misa_status misa_rerank_topk_noalloc(const misa_cache *cache, const mis
                                               int32_t *topk, float *scores_out, misa_stream stream);
 
 /*
- * Workspace bytes the call `op` (misa_op) needs for these shapes; 0 on
- * invalid arguments.  Host-only, launches nothing.
+ * Workspace bytes the call `op` (misa_op) needs for these shapes (k is the
+ * call's k: k' for the coarse MISA-dagger stage); 0 on invalid arguments.
+ * This is the need without scores_out; with scores_out it is smaller.
+ * Host-only, launches nothing.
  */
 MISA_API size_t misa_workspace_bytes(int32_t op, const misa_cache *cache, const misa_queries *qs,
                             int32_t h, int32_t k, int32_t k_prime);

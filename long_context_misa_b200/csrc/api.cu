@@ -112,9 +112,14 @@ misa::QueryView view(const misa_queries *q) {
 
 size_t round_up(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Workspace of the score + top-k calls: [row histograms][scores (unless the
-// caller passes scores_out)].
-size_t ws_hist(const misa_queries *q) { return round_up(sizeof(uint32_t) * (size_t)q->n_q * misa::TOPK_HIST_BINS); }
+// Workspace of the score + top-k calls: [row histograms + top-k list
+// counters (zeroed together)][scores, unless the caller passes scores_out]
+// [top-k list, prefix rows that use one].
+size_t hist_words(const misa_queries *q) { return (size_t)q->n_q * (misa::TOPK_HIST_BINS + 1); }
+size_t ws_hist(const misa_queries *q) { return round_up(sizeof(uint32_t) * hist_words(q)); }
+size_t ws_list(const misa_cache *c, const misa_queries *q, int k) {
+  return round_up(8 * misa::topk_list_entries(q->n_q, c->L_cap, k));
+}
 
 size_t ws_score(const misa_cache *c, const misa_queries *q) {
   return round_up(sizeof(float) * (size_t)q->n_q * c->L_cap);
@@ -132,15 +137,18 @@ misa_status score_then_topk(const char *who, const misa_cache *cache, const misa
                             cudaStream_t stream) {
   misa::CacheView c = view(cache);
   misa::QueryView q = view(qs);
-  uint32_t *hist = static_cast<uint32_t *>(ws);
-  float *scores = scores_out ? scores_out : reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + ws_hist(qs));
-  cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
+  uint8_t *w8 = static_cast<uint8_t *>(ws);
+  uint32_t *hist = reinterpret_cast<uint32_t *>(w8);
+  uint32_t *list_cnt = hist + (size_t)qs->n_q * misa::TOPK_HIST_BINS;
+  float *scores = scores_out ? scores_out : reinterpret_cast<float *>(w8 + ws_hist(qs));
+  void *list = w8 + ws_hist(qs) + (scores_out ? 0 : ws_score(cache, qs));
+  cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * hist_words(qs), stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   e = timed_scoring(stream, [&] {
     return misa::launch_score_mma(c, q, heads, h, nullptr, 0, scores, cache->L_cap, hist, stream);
   });
   if (e != cudaSuccess) return cuda_fail(e, who);
-  e = misa::launch_topk(c, q, scores, cache->L_cap, 0, nullptr, hist, k, topk, stream);
+  e = misa::launch_topk(c, q, scores, cache->L_cap, 0, nullptr, hist, list, list_cnt, k, topk, stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   return MISA_OK;
 }
@@ -196,14 +204,13 @@ misa_status misa_pool_keys(const misa_cache *cache, const void *new_keys, const 
 size_t misa_workspace_bytes(int32_t op, const misa_cache *cache, const misa_queries *qs, int32_t h, int32_t k,
                             int32_t k_prime) {
   (void)h;
-  (void)k;
   if (!cache || !qs || cache->B < 1 || cache->L_cap < 1 || qs->n_q < 0 || qs->H < 1) return 0;
   switch (op) {
     case MISA_OP_ROUTE:
       return round_up(misa::route_ws_bytes(qs->n_q, qs->H, misa::cdiv(cache->L_cap, cache->B)));
     case MISA_OP_SCORE_TOPK:
     case MISA_OP_DENSE_TOPK:
-      return ws_hist(qs) + ws_score(cache, qs);
+      return ws_hist(qs) + ws_score(cache, qs) + (k > 0 ? ws_list(cache, qs, k) : 0);
     case MISA_OP_RERANK_TOPK:
       return k_prime > 0 ? ws_hist(qs) + round_up(sizeof(float) * (size_t)qs->n_q * k_prime) : 0;
     default:
@@ -234,7 +241,7 @@ misa_status misa_score_topk(const misa_cache *cache, const misa_queries *qs, con
   if (h < 1 || h > qs->H) return fail(MISA_ERR_INVALID, "h=%d outside [1, H=%d]", h, qs->H);
   if (k < 1) return fail(MISA_ERR_INVALID, "k=%d < 1", k);
   if (qs->n_q > 0 && (!heads || !topk)) return fail(MISA_ERR_INVALID, "heads/topk is NULL");
-  const size_t need = ws_hist(qs) + (scores_out ? 0 : ws_score(cache, qs));
+  const size_t need = ws_hist(qs) + (scores_out ? 0 : ws_score(cache, qs)) + ws_list(cache, qs, k);
   if ((st = check_ws(ws, ws_bytes, need)) != MISA_OK) return st;
   if (injected_failure("misa_score_topk", &st)) return st;
   if (qs->n_q == 0) return MISA_OK;
@@ -248,7 +255,7 @@ misa_status dsa_dense_score_topk(const misa_cache *cache, const misa_queries *qs
   if ((st = check_queries(qs)) != MISA_OK) return st;
   if (k < 1) return fail(MISA_ERR_INVALID, "k=%d < 1", k);
   if (qs->n_q > 0 && !topk) return fail(MISA_ERR_INVALID, "topk is NULL");
-  const size_t need = ws_hist(qs) + (scores_out ? 0 : ws_score(cache, qs));
+  const size_t need = ws_hist(qs) + (scores_out ? 0 : ws_score(cache, qs)) + ws_list(cache, qs, k);
   if ((st = check_ws(ws, ws_bytes, need)) != MISA_OK) return st;
   if (injected_failure("dsa_dense_score_topk", &st)) return st;
   if (qs->n_q == 0) return MISA_OK;
@@ -278,7 +285,7 @@ misa_status misa_rerank_topk(const misa_cache *cache, const misa_queries *qs, co
     return misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, scores, k_prime, hist, stream);
   });
   if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
-  e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, hist, k, topk, stream);
+  e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, hist, nullptr, nullptr, k, topk, stream);
   if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
   return MISA_OK;
 }
@@ -313,7 +320,7 @@ misa_status misa_rerank_topk_noalloc(const misa_cache *cache, const misa_queries
     return misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, scores, k_prime, hist, stream);
   });
   if (e != cudaSuccess) return cuda_fail(e, who);
-  e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, hist, k, topk, stream);
+  e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, hist, nullptr, nullptr, k, topk, stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   return MISA_OK;
 }

@@ -38,12 +38,21 @@ cudaError_t launch_score_mma(const CacheView &c, const QueryView &q, const int32
 cudaError_t launch_score_stream(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
                                 long long ld, uint32_t *row_hist, cudaStream_t s);
 
-// topk.cu: per row, the k largest scores; ties to the lower position.
-// Row length comes from the query prefix (gather == nullptr) or is n_cols with
-// positions whose gather entry is < 0 excluded; outputs are token indices
-// (gather[pos] or pos), ascending when gather is ascending.  row_hist is the
-// histogram the scoring kernel built over exactly the valid scores.
+// topk.cu: per row, the k largest scores, ties to the lower token index;
+// outputs are token indices in ascending order, -1 padded.  Row length comes
+// from the query prefix (gather == nullptr), or the row holds n_cols
+// candidates whose tokens are gather[i][p] (entries < 0 or beyond the prefix
+// excluded).  row_hist is the histogram the scoring kernel built over exactly
+// the valid scores.  Prefix rows with few queries and long caches go through
+// a compact list of the elements at or above the histogram's boundary bin:
+// list_ws holds topk_list_entries() entries of 8 bytes and list_cnt n_q
+// counters, zeroed beforehand (both may be null: no list).
+constexpr int TOPK_LIST_MAX_ROWS = 64;   // rows served by the list path at most
+constexpr int TOPK_LIST_MIN_L = 16384;   // shorter caches never use it
+constexpr int TOPK_LIST_EXTRA = 8192;    // boundary-bin elements listed per row beyond k
+size_t topk_list_entries(int n_q, int L_cap, int k);
 cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
-                        const int32_t *gather, const uint32_t *row_hist, int k, int32_t *out, cudaStream_t s);
+                        const int32_t *gather, const uint32_t *row_hist, void *list_ws, uint32_t *list_cnt, int k,
+                        int32_t *out, cudaStream_t s);
 
 }  // namespace misa

@@ -1,435 +1,668 @@
-// Top-k token selection: radix select over a thread-block cluster, starting
-// from a histogram the scoring kernel built while writing the scores.
+// Top-k token selection from the scores and the per-row histogram the
+// scoring kernel built while writing them.
 //
 // "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM Inference":
 // the indexer keeps the k highest-scoring prefix tokens for the main sparse
 // attention (abstract; technical summary "Methodology: MISA", step 2), and
 // MISA-dagger keeps k' candidates from the routed pass ("Hierarchical
-// variant").  Order: larger score first, equal scores to the lower position
-// (the lower token index, since positions are ascending token indices).
+// variant").  Order: larger score first, equal scores to the lower token
+// index.  Every element's composite key (order-preserving image of the score,
+// 2^18-1-token) is unique in a row; the result is every element whose
+// composite is at least the kk-th largest (kk = min(k, valid elements)),
+// written as token indices in ascending order.
 //
-// Keys: the order-preserving 32-bit image of each score; each element's
-// composite key is (score key, 2^18-1-position), unique in a row.  The result
-// is every element whose composite is at least the kk-th largest one
-// (kk = min(k, valid elements)), written in ascending position order.
+// The scoring kernel counted the row's keys by their top 11 bits (row_hist,
+// 2048 bins).  From it every kernel here finds the same boundary bin d0:
+// elements above d0 are selected outright, elements below are not, and only
+// the elements inside d0 need the remaining 21 key bits and the token.
 //
-// The scoring kernel has already counted the row's keys by their top 11 bits
-// (row_hist, 2048 bins).  One cluster of CS CTAs (CS in {1,2,4,8}) owns a row;
-// each CTA keeps its slice of T*E keys in shared memory.
-//   1. Every CTA reads row_hist and finds the same boundary bin d0 (block
-//      scan, no exchange); it counts its keys above and in d0 and, unless the
-//      whole bin is needed, appends its keys in d0 to a shared list.  (barrier 1)
-//   2. Rank 0 gathers the lists through distributed shared memory, finishes
-//      the radix select on the remaining 21 key bits and the position in its
-//      shared memory (2048-bin passes with early exit), and turns the
-//      per-rank counts into output offsets.                       (barrier 2)
-//   3. Every CTA reads the threshold and its offset and writes its selected
-//      positions in order (warp ballots, a scan over warps).      (barrier 3)
-// A boundary bin too large to gather falls back to cluster-wide passes.
-#include <cooperative_groups.h>
-
+// select_kernel, one CTA per row:
+//   1. boundary bin from the histogram (one warp);
+//   2. one pass over the row -- or over the compact list the filter kernel
+//      wrote -- marks every element above d0 in a token bitmap in shared
+//      memory and lists the elements of d0 (key, token) in shared memory;
+//   3. radix passes over the listed d0 elements only (11 key bits; then,
+//      once at most 512 elements remain in the boundary bin, their exact
+//      ranks by counting) fix the threshold; the winners are marked;
+//   4. a popcount scan of the bitmap writes the tokens in ascending order,
+//      the outputs split evenly over the threads.
+//   A d0 too large to list (degenerate score distributions) falls back to
+//   the same radix passes over the whole row, read from global memory.
+// filter_kernel (few long rows: decode): many CTAs per row copy the elements
+//   at or above d0 into a per-row list, so that the one CTA per row above
+//   reads about k + |d0| entries instead of the whole row.
 #include "internal.h"
-
-namespace cg = cooperative_groups;
 
 namespace misa {
 namespace {
 
-constexpr int POS_BITS = 18;                 // positions < 2^18 = MISA_MAX_L
+constexpr int POS_BITS = 18;                 // token indices < 2^18 = MISA_MAX_L
 constexpr uint32_t POS_MAX = (1u << POS_BITS) - 1u;
-constexpr int MAX_CS = 8;
-constexpr int CAP = 8192;                    // boundary-bin elements rank 0 can gather
-constexpr int RB = TOPK_HIST_BINS;           // bins per pass (11-bit digits)
-constexpr uint32_t TOP_MASK = 0xFFE00000u;   // the histogram's 11 bits
-// passes after the histogram: key bits 20..10, 9..0, then position bits 17..9, 8..0
+constexpr int RB = TOPK_HIST_BINS;           // bins of the histogram and of each refinement pass
+constexpr int HIST_SHIFT = 21;               // the histogram holds key bits 31..21
+constexpr uint32_t TOP_MASK = 0xFFE00000u;
+constexpr int CAP = TOPK_LIST_EXTRA;         // d0 elements refined in shared memory
+constexpr int SEL_T = 512;                   // select_kernel threads
+constexpr int SEL_W = SEL_T / 32;
+constexpr int FILT_T = 256;                  // filter_kernel threads
+constexpr int U = 16;                        // elements per thread per sweep iteration
+constexpr int HPAD = RB + RB / 64;           // shared histogram: one pad word per 64 bins
+// refinement passes: key bits 20..10, 9..0, then the token's tie bits 17..9, 8..0
 __device__ constexpr int kShift[4] = {10, 0, 9, 0};
 __device__ constexpr int kWidth[4] = {11, 10, 9, 9};
 
-template <int T>
-struct SelShared {
-  uint32_t lhist[RB];
-  uint32_t wtot[T / 32];                     // per-warp totals
-  uint32_t wscan[T / 32];                    // scans of wtot
-  uint32_t n_cand, n_hi, n_in;               // this CTA: listed, above d0, in d0
-  uint32_t res[3];                           // digit, above, in_bin of the last search
-  uint32_t dec[4];                           // rank 0's threshold: P_hi, M_hi, P_lo, M_lo
-  uint32_t offs[MAX_CS];                     // rank 0's output offset per rank
-  uint32_t sel_cnt[MAX_CS];                  // rank 0: selected listed elements per rank
-  uint32_t cand_key[CAP];
-  uint32_t cand_lo[CAP];
-  uint8_t cand_rank[CAP];
-};
-
-template <int T, int E>
-constexpr int sel_smem_bytes() {
-  return (int)sizeof(SelShared<T>) + T * E * 4;
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
 }
 
-// Exclusive scan of the warps' values `mine` (warp w's at wscan[w]) by warp 0;
-// returns the block total.  Two barriers.
+// Bin b of a shared refinement histogram: lane l's 64 bins start at word
+// 65 l, so the lanes of a warp read distinct banks.
+__device__ __forceinline__ int hpos(int b) { return b + (b >> 6); }
+
+// One whole warp: the bin of a RB-bin histogram (larger bin = larger key)
+// holding the want-th largest element.  Lane l sums bins [64 l, 64 l + 64);
+// the range that holds it is then searched two bins per lane.  Returns to every lane
+// {bin, elements in higher bins, its count, total}; bin = ~0 when want is 0
+// or above the total.  PAD: shared histogram in the hpos layout, else a
+// plain array in global memory.
+template <bool PAD>
+__device__ __forceinline__ uint4 warp_select_bin(const uint32_t *h, uint32_t want) {
+  const int lane = threadIdx.x & 31;
+  uint32_t s = 0;
+  if (PAD) {
+#pragma unroll 16
+    for (int j = 0; j < 64; ++j) s += h[lane * 65 + j];
+  } else {
+    const uint4 *p = reinterpret_cast<const uint4 *>(h + lane * 64);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const uint4 v = __ldg(p + j);
+      s += v.x + v.y + v.z + v.w;
+    }
+  }
+  uint32_t suf = s;  // elements in lanes >= this one
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += v;
+  }
+  const uint32_t total = __shfl_sync(0xffffffffu, suf, 0);
+  if (want == 0 || want > total) return make_uint4(~0u, 0u, 0u, total);
+  const uint32_t above_l = suf - s;
+  const int owner = __ffs(__ballot_sync(0xffffffffu, above_l < want && suf >= want)) - 1;
+  // the owner's 64 bins, two per lane, searched by the whole warp
+  const uint32_t base_above = __shfl_sync(0xffffffffu, above_l, owner);
+  const int b0 = owner * 64 + 2 * lane;
+  uint32_t c0, c1;
+  if (PAD) {
+    c0 = h[hpos(b0)];
+    c1 = h[hpos(b0 + 1)];
+  } else {
+    const uint2 v = __ldg(reinterpret_cast<const uint2 *>(h + b0));
+    c0 = v.x;
+    c1 = v.y;
+  }
+  const uint32_t pair = c0 + c1;
+  uint32_t psuf = pair;  // elements in the owner's bins >= b0
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_down_sync(0xffffffffu, psuf, o);
+    if (lane + o < 32) psuf += v;
+  }
+  const uint32_t a1 = base_above + psuf - pair;  // elements above bin b0 + 1
+  const bool hit1 = a1 < want && a1 + c1 >= want;
+  const bool hit0 = a1 + c1 < want && a1 + pair >= want;
+  const int src = __ffs(__ballot_sync(0xffffffffu, hit1 || hit0)) - 1;
+  const uint32_t bin = hit1 ? b0 + 1 : b0;
+  const uint32_t above = hit1 ? a1 : a1 + c1;
+  const uint32_t cnt = hit1 ? c1 : c0;
+  return make_uint4(__shfl_sync(0xffffffffu, bin, src), __shfl_sync(0xffffffffu, above, src),
+                    __shfl_sync(0xffffffffu, cnt, src), total);
+}
+// Boundary of a row from its histogram: kk, total, and (unless every valid
+// element is selected) the bin d0 with the counts above it and in it.
+struct Boundary {
+  uint32_t total, kk, d0, above, in0, all_in;
+  // elements still to take from d0
+  __device__ uint32_t need() const { return kk - above; }
+  // a compact list of the elements at or above d0 serves this row: it holds
+  // kk (whole bin taken) or fewer than kk + CAP (d0 listed) entries
+  __device__ bool listable() const { return kk > 0 && !all_in && (need() == in0 || in0 <= (uint32_t)CAP); }
+};
+
+// One whole warp: the row's boundary (valid in every lane).
+__device__ __forceinline__ Boundary warp_boundary(const uint32_t *rh, int k) {
+  const uint4 r = warp_select_bin<false>(rh, (uint32_t)k);
+  Boundary b;
+  b.total = r.w;
+  b.kk = min((uint32_t)k, r.w);
+  b.all_in = (uint32_t)k >= r.w;
+  b.d0 = b.all_in ? 0u : r.x;
+  b.above = b.all_in ? 0u : r.y;
+  b.in0 = b.all_in ? 0u : r.z;
+  return b;
+}
+
+// Exclusive prefix of `v` over the threads in thread order; *total = block sum.
 template <int T>
-__device__ __forceinline__ uint32_t warp_totals_scan(uint32_t mine, uint32_t *wtot, uint32_t *wscan) {
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *total, uint32_t *wa, uint32_t *wb) {
   constexpr int W = T / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (lane == 0) wtot[warp] = mine;
+  uint32_t inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t u = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += u;
+  }
+  if (lane == 31) wa[warp] = inc;
   __syncthreads();
   if (warp == 0) {
-    const uint32_t v = lane < W ? wtot[lane] : 0u;
-    uint32_t inc = v;
+    const uint32_t x = lane < W ? wa[lane] : 0u;
+    uint32_t s = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t u = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += u;
+    }
+    if (lane < W) wb[lane] = s - x;
+    if (lane == W - 1) wb[W] = s;
+  }
+  __syncthreads();
+  *total = wb[W];
+  const uint32_t r = wb[warp] + inc - v;
+  __syncthreads();  // wa, wb free again on return
+  return r;
+}
+
+struct SelShared {
+  Boundary bd;
+  uint4 res;                       // a warp search result
+  uint32_t thr[2];                 // threshold composite from the counting step
+  uint32_t n_small;
+  uint32_t wa[SEL_W], wb[SEL_W + 1];
+  uint32_t toff[SEL_T];            // output offset of each thread's bitmap words
+  uint32_t hist[HPAD];
+  uint32_t small_key[SEL_T], small_tie[SEL_T];
+  uint32_t cand_key[CAP];
+  uint32_t cand_tie[CAP];
+};
+
+// Visit every element of the row in warp- and block-uniform sweeps:
+// fn(key, token, ok, base) gets U elements per thread; element u of thread t
+// is position base + u*T + t.  Prefix rows: position p is token p with score
+// srow[p], p < Li.  Gathered rows: position p is token grow[p] (ok when
+// 0 <= token < Li) with score srow[p], p < n.
+template <int T, bool GATHER, class F>
+__device__ __forceinline__ void sweep_row(const float *srow, const int32_t *grow, int n, int Li, F &&fn) {
+  for (int base = 0; base < n; base += T * U) {
+    int tk[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int p = base + u * T + threadIdx.x;
+      tk[u] = p < n ? (GATHER ? __ldg(grow + p) : p) : -1;
+    }
+    float sv[U];
+    bool ok[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int p = base + u * T + threadIdx.x;
+      ok[u] = tk[u] >= 0 && tk[u] < Li;
+      sv[u] = ok[u] ? __ldg(srow + p) : 0.f;
+    }
+    uint32_t key[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) key[u] = ordered_key(sv[u]);
+    fn(key, tk, ok, base);
+  }
+}
+
+// Visit the filter kernel's list of n entries (key, token), all valid.
+template <int T, class F>
+__device__ __forceinline__ void sweep_list(const uint2 *lrow, int n, F &&fn) {
+  for (int base = 0; base < n; base += T * U) {
+    uint32_t key[U];
+    int tk[U];
+    bool ok[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int p = base + u * T + threadIdx.x;
+      uint2 e = make_uint2(0u, 0u);
+      if (p < n) e = __ldg(lrow + p);
+      ok[u] = p < n;
+      key[u] = e.x;
+      tk[u] = (int)e.y;
+    }
+    fn(key, tk, ok, base);
+  }
+}
+
+// Software-pipelined sweeps for the select kernel: the caller issues the
+// first sweep's loads (load_row / load_list) before the row's length and
+// boundary are known, and every sweep requests the next one before visiting
+// its own elements.  Loads stay below n_load, the row's allocation.
+template <bool GATHER>
+__device__ __forceinline__ void load_row(const float *srow, const int32_t *grow, int n_load, int base, int (&tk)[U],
+                                         float (&sv)[U]) {
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int p = base + u * SEL_T + threadIdx.x;
+    const bool in = p < n_load;
+    tk[u] = in ? (GATHER ? __ldg(grow + p) : p) : -1;
+    sv[u] = in ? __ldg(srow + p) : 0.f;
+  }
+}
+
+template <bool GATHER, class F>
+__device__ __forceinline__ void sweep_row_pf(const float *srow, const int32_t *grow, int n_load, int n, int Li,
+                                             int (&tk)[U], float (&sv)[U], F &&fn) {
+  for (int base = 0; base < n; base += SEL_T * U) {
+    int ct[U];
+    uint32_t key[U];
+    bool ok[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int p = base + u * SEL_T + threadIdx.x;
+      ct[u] = tk[u];
+      ok[u] = p < n && tk[u] >= 0 && tk[u] < Li;
+      key[u] = ordered_key(sv[u]);
+    }
+    if (base + SEL_T * U < n) load_row<GATHER>(srow, grow, n_load, base + SEL_T * U, tk, sv);
+    fn(key, ct, ok, base);
+  }
+}
+
+__device__ __forceinline__ void load_list(const uint2 *lrow, int n_load, int base, uint2 (&e)[U]) {
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int p = base + u * SEL_T + threadIdx.x;
+    e[u] = p < n_load ? __ldg(lrow + p) : make_uint2(0u, 0u);
+  }
+}
+
+template <class F>
+__device__ __forceinline__ void sweep_list_pf(const uint2 *lrow, int n_load, int n, uint2 (&e)[U], F &&fn) {
+  for (int base = 0; base < n; base += SEL_T * U) {
+    int ct[U];
+    uint32_t key[U];
+    bool ok[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      ok[u] = base + u * SEL_T + (int)threadIdx.x < n;
+      key[u] = e[u].x;
+      ct[u] = (int)e[u].y;
+    }
+    if (base + SEL_T * U < n) load_list(lrow, n_load, base + SEL_T * U, e);
+    fn(key, ct, ok, base);
+  }
+}
+
+__device__ __forceinline__ void mark(uint32_t *bm, int tok) { atomicOr(bm + (tok >> 5), 1u << (tok & 31)); }
+
+__device__ __forceinline__ bool at_least(uint32_t kx, uint32_t lx, uint32_t P_hi, uint32_t M_hi, uint32_t P_lo,
+                                         uint32_t M_lo) {
+  const uint32_t kh = kx & M_hi, kl = lx & M_lo;
+  return kh > P_hi || (kh == P_hi && kl >= P_lo);
+}
+
+// Radix refinement of the threshold among the elements the visitor presents
+// (visit(fn) calls fn(key, tie, active) for each, block-uniformly).  P/M:
+// prefix and mask decided so far on the key and on the tie; need: elements
+// still to take among the in_bin that match the prefix.  With `small`, once
+// at most SEL_T elements match, their exact ranks finish the job.
+template <bool SMALL, class Visit>
+__device__ __forceinline__ void refine(SelShared &sh, uint32_t &P_hi, uint32_t &M_hi, uint32_t &P_lo,
+                                       uint32_t &M_lo, uint32_t need, uint32_t in_bin, Visit &&visit) {
+  const int tid = threadIdx.x;
+  bool done = in_bin == need;
+  for (int p = 0; p < 4 && !done; ++p) {
+    if (SMALL && p > 0 && in_bin <= (uint32_t)SEL_T) {
+      // the in_bin elements matching the prefix: rank each by counting
+      visit([&](uint32_t kx, uint32_t lx, bool act) {
+        if (act && (kx & M_hi) == P_hi && (lx & M_lo) == P_lo) {
+          const uint32_t slot = atomicAdd(&sh.n_small, 1u);
+          if (slot < (uint32_t)SEL_T) {
+            sh.small_key[slot] = kx;
+            sh.small_tie[slot] = lx;
+          }
+        }
+      });
+      __syncthreads();
+      const int ns = min((int)sh.n_small, SEL_T);
+      if (tid < ns) {
+        const uint32_t ki = sh.small_key[tid], li = sh.small_tie[tid];
+        uint32_t rank = 0;
+        for (int j = 0; j < ns; ++j) {
+          const uint32_t kj = sh.small_key[j], lj = sh.small_tie[j];
+          rank += (kj > ki || (kj == ki && lj > li)) ? 1u : 0u;
+        }
+        if (rank == need - 1) {
+          sh.thr[0] = ki;
+          sh.thr[1] = li;
+        }
+      }
+      __syncthreads();
+      P_hi = sh.thr[0];
+      M_hi = ~0u;
+      P_lo = sh.thr[1];
+      M_lo = POS_MAX;
+      return;
+    }
+    const bool lo_word = p >= 2;
+    const int sft = kShift[p];
+    const uint32_t dm = (1u << kWidth[p]) - 1u;
+    for (int b = tid; b < HPAD; b += SEL_T) sh.hist[b] = 0;
+    __syncthreads();
+    visit([&](uint32_t kx, uint32_t lx, bool act) {
+      if (act && (kx & M_hi) == P_hi && (lx & M_lo) == P_lo)
+        atomicAdd(&sh.hist[hpos(((lo_word ? lx : kx) >> sft) & dm)], 1u);
+    });
+    __syncthreads();
+    if (tid < 32) {
+      const uint4 r = warp_select_bin<true>(sh.hist, need);
+      if (tid == 0) sh.res = r;
+    }
+    __syncthreads();
+    const uint4 r = sh.res;
+    need -= r.y;
+    in_bin = r.z;
+    if (!lo_word) {
+      P_hi |= r.x << sft;
+      M_hi |= dm << sft;
+    } else {
+      P_lo |= r.x << sft;
+      M_lo |= dm << sft;
+    }
+    done = in_bin == need;
+  }
+}
+
+template <bool GATHER, bool FROM_LIST>
+__global__ void __launch_bounds__(SEL_T) select_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
+                                                       int n_cols, const int32_t *gather, const uint32_t *row_hist,
+                                                       const uint2 *list, const uint32_t *list_cnt, int list_cap,
+                                                       int k, int32_t *out) {
+  extern __shared__ __align__(16) uint8_t sel_smem[];
+  SelShared &sh = *reinterpret_cast<SelShared *>(sel_smem);
+  uint32_t *bm = reinterpret_cast<uint32_t *>(sel_smem + sizeof(SelShared));  // token bitmap
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float *srow = scores + (size_t)row * ld;
+  const int32_t *grow = GATHER ? gather + (size_t)row * n_cols : nullptr;
+  const uint2 *lrow = FROM_LIST ? list + (size_t)row * list_cap : nullptr;
+  const int n_load = GATHER ? n_cols : c.L_cap;  // the row's allocation
+  int32_t *orow = out + (size_t)row * k;
+
+  // 1. requested together: the first sweep (row or list), the list length,
+  //    the query's prefix and the row histogram; every warp then finds the
+  //    boundary bin by itself
+  int tk[U];
+  float sv[U];
+  uint2 le[U];
+  if (FROM_LIST)
+    load_list(lrow, list_cap, 0, le);
+  else
+    load_row<GATHER>(srow, grow, n_load, 0, tk, sv);
+  const int lcnt = FROM_LIST ? min((int)list_cnt[row], list_cap) : 0;
+  int s;
+  const int Li = query_prefix(c, qv, row, &s);
+  const int n = GATHER ? n_cols : Li;
+  const int words = cdiv(Li, 32);
+  const Boundary bd = warp_boundary(row_hist + (size_t)row * RB, k);
+  if (tid == 0) sh.n_small = 0;
+  for (int w = tid; w < words; w += SEL_T) bm[w] = 0;
+  __syncthreads();
+
+  if (bd.kk > 0) {
+    const uint32_t d0 = bd.d0;
+    const uint32_t need = bd.need();
+    const bool whole = bd.all_in || need == bd.in0;  // no refinement needed
+    const bool listed = !whole && bd.in0 <= (uint32_t)CAP;
+    uint32_t P_hi = d0 << HIST_SHIFT, M_hi = TOP_MASK, P_lo = 0, M_lo = 0;
+    const bool via_list = FROM_LIST && bd.listable();
+    // tokens of a warp's 32 consecutive row positions are consecutive: their
+    // bitmap word is the warp's ballot
+    const bool word_marks = !GATHER && !via_list;
+    auto mark_sweep = [&](const bool(&sel)[U], const int(&tk)[U], int base) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if (word_marks) {
+          const uint32_t m = __ballot_sync(0xffffffffu, sel[u]);
+          const int p0 = base + u * SEL_T + warp * 32;
+          if (lane == 0 && p0 < n) bm[p0 >> 5] = m;
+        } else if (sel[u]) {
+          mark(bm, tk[u]);
+        }
+      }
+    };
+    if (whole || listed) {
+      // 2. mark everything above the boundary (and d0 too when whole); list
+      //    d0 with ballots and one scan over the warps per sweep
+      uint32_t n_listed = 0;
+      auto visit = [&](const uint32_t(&key)[U], const int(&tk)[U], const bool(&ok)[U], int base) {
+        bool sel[U];
+        uint32_t lm[U], cnt = 0;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const uint32_t bin = key[u] >> HIST_SHIFT;
+          sel[u] = ok[u] && (bd.all_in || bin > d0 || (whole && bin == d0));
+          lm[u] = __ballot_sync(0xffffffffu, listed && ok[u] && bin == d0);
+          cnt += __popc(lm[u]);
+        }
+        mark_sweep(sel, tk, base);
+        if (listed) {
+          if (lane == 0) sh.wa[warp] = cnt;
+          __syncthreads();
+          const uint32_t x = lane < SEL_W ? sh.wa[lane] : 0u;
+          const uint32_t before = __reduce_add_sync(0xffffffffu, lane < warp ? x : 0u);
+          const uint32_t tot = __reduce_add_sync(0xffffffffu, x);
+          __syncthreads();
+          uint32_t slot = n_listed + before;
+          const uint32_t lt = lanemask_lt();
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            if ((lm[u] >> lane) & 1) {
+              const uint32_t o = slot + __popc(lm[u] & lt);
+              if (o < (uint32_t)CAP) {
+                sh.cand_key[o] = key[u];
+                sh.cand_tie[o] = POS_MAX - (uint32_t)tk[u];
+              }
+            }
+            slot += __popc(lm[u]);
+          }
+          n_listed += tot;
+        }
+      };
+      if (via_list)
+        sweep_list_pf(lrow, list_cap, lcnt, le, visit);
+      else if (!FROM_LIST)
+        sweep_row_pf<GATHER>(srow, grow, n_load, n, Li, tk, sv, visit);
+      else
+        sweep_row<SEL_T, GATHER>(srow, grow, n, Li, visit);
+      __syncthreads();
+      if (listed) {
+        // 3. exact threshold among the listed elements of d0, then their winners
+        const int nc = min((int)n_listed, CAP);
+        refine<true>(sh, P_hi, M_hi, P_lo, M_lo, need, bd.in0, [&](auto &&fn) {
+          for (int x = tid; x < nc; x += SEL_T) fn(sh.cand_key[x], sh.cand_tie[x], true);
+        });
+        for (int x = tid; x < nc; x += SEL_T)
+          if (at_least(sh.cand_key[x], sh.cand_tie[x], P_hi, M_hi, P_lo, M_lo))
+            mark(bm, (int)(POS_MAX - sh.cand_tie[x]));
+        __syncthreads();
+      }
+    } else {
+      // d0 too large to list: radix passes over the whole row, then one
+      // marking pass (composite at or above the threshold on the decided bits)
+      refine<false>(sh, P_hi, M_hi, P_lo, M_lo, need, bd.in0, [&](auto &&fn) {
+        sweep_row<SEL_T, GATHER>(srow, grow, n, Li,
+                                 [&](const uint32_t(&key)[U], const int(&tk)[U], const bool(&ok)[U], int) {
+#pragma unroll
+                                   for (int u = 0; u < U; ++u) fn(key[u], POS_MAX - (uint32_t)tk[u], ok[u]);
+                                 });
+      });
+      sweep_row<SEL_T, GATHER>(srow, grow, n, Li,
+                               [&](const uint32_t(&key)[U], const int(&tk)[U], const bool(&ok)[U], int base) {
+                                 bool sel[U];
+#pragma unroll
+                                 for (int u = 0; u < U; ++u)
+                                   sel[u] = ok[u] && at_least(key[u], POS_MAX - (uint32_t)tk[u], P_hi, M_hi, P_lo,
+                                                              M_lo);
+                                 mark_sweep(sel, tk, base);
+                               });
+      __syncthreads();
+    }
+  }
+
+  // 4. ascending output.  Thread t owns bitmap words [t*per, t*per + per);
+  //    the outputs are split evenly over the threads (each finds the word
+  //    holding its first output by a search over the owners' offsets).
+  const int per = cdiv(words, SEL_T);
+  {
+    const int w0 = min(tid * per, words), w1 = min(w0 + per, words);
+    uint32_t cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+    uint32_t n_sel;
+    sh.toff[tid] = block_excl_scan<SEL_T>(cnt, &n_sel, sh.wa, sh.wb);
+    __syncthreads();
+    const uint32_t j0 = n_sel * (uint32_t)tid / SEL_T, j1 = n_sel * (uint32_t)(tid + 1) / SEL_T;
+    if (j0 < j1) {
+      int lo = 0, hi = SEL_T - 1;  // last owner whose offset is <= j0
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (sh.toff[mid] <= j0) lo = mid;
+        else hi = mid - 1;
+      }
+      uint32_t r = j0 - sh.toff[lo];
+      int w = lo * per;
+      uint32_t m = bm[w];
+      while ((uint32_t)__popc(m) <= r) {
+        r -= __popc(m);
+        m = bm[++w];
+      }
+      for (; r > 0; --r) m &= m - 1;
+      for (uint32_t j = j0; j < j1; ++j) {
+        while (m == 0) m = bm[++w];
+        const int b = __ffs(m) - 1;
+        m &= m - 1;
+        if (j < (uint32_t)k) orow[j] = w * 32 + b;
+      }
+    }
+    for (int p = (int)n_sel + tid; p < k; p += SEL_T) orow[p] = -1;
+  }
+}
+
+// Few long prefix rows: every CTA takes a chunk of one row and appends the
+// elements at or above the boundary bin, (key, token), to the row's list
+// (list_cnt zeroed beforehand).  Rows the list cannot serve are skipped; the
+// select kernel reads those rows itself.
+__global__ void __launch_bounds__(FILT_T) filter_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
+                                                        const uint32_t *row_hist, uint2 *list, uint32_t *list_cnt,
+                                                        int list_cap, int k, int chunk) {
+  constexpr int FU = 16;
+  const int row = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int p0 = blockIdx.x * chunk;
+  const int pl = min(c.L_cap, p0 + chunk);  // loads stay inside the row's allocation
+  const float *srow = scores + (size_t)row * ld;
+  // the first sweep's scores are requested with the prefix and the histogram
+  float sv[FU];
+#pragma unroll
+  for (int u = 0; u < FU; ++u) {
+    const int p = p0 + u * FILT_T + threadIdx.x;
+    sv[u] = p < pl ? __ldg(srow + p) : 0.f;
+  }
+  int s;
+  const int Li = query_prefix(c, qv, row, &s);
+  if (p0 >= Li) return;  // uniform over the CTA
+  const int p1 = min(Li, pl);
+  const Boundary bd = warp_boundary(row_hist + (size_t)row * RB, k);  // every warp
+  if (!bd.listable()) return;  // uniform
+  uint2 *lrow = list + (size_t)row * list_cap;
+  for (int base = p0; base < p1; base += FILT_T * FU) {
+    if (base != p0) {
+#pragma unroll
+      for (int u = 0; u < FU; ++u) {
+        const int p = base + u * FILT_T + threadIdx.x;
+        sv[u] = p < p1 ? __ldg(srow + p) : 0.f;
+      }
+    }
+    uint32_t key[FU], n = 0;
+#pragma unroll
+    for (int u = 0; u < FU; ++u) {
+      const int p = base + u * FILT_T + threadIdx.x;
+      key[u] = ordered_key(sv[u]);
+      n += (p < p1 && (key[u] >> HIST_SHIFT) >= bd.d0) ? 1u : 0u;
+    }
+    uint32_t inc = n;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t u = __shfl_up_sync(0xffffffffu, inc, o);
       if (lane >= o) inc += u;
     }
-    if (lane < W) wscan[lane] = inc - v;
-    if (lane == 31) wtot[0] = inc;  // block total (wtot is not read again)
+    const uint32_t tot = __shfl_sync(0xffffffffu, inc, 31);
+    if (tot == 0) continue;  // warp-uniform
+    uint32_t slot = 0;
+    if (lane == 31) slot = atomicAdd(list_cnt + row, tot);
+    slot = __shfl_sync(0xffffffffu, slot, 31) + inc - n;
+#pragma unroll
+    for (int u = 0; u < FU; ++u) {
+      const int p = base + u * FILT_T + threadIdx.x;
+      if (p < p1 && (key[u] >> HIST_SHIFT) >= bd.d0) {
+        if (slot < (uint32_t)list_cap) lrow[slot] = make_uint2(key[u], (uint32_t)p);
+        ++slot;
+      }
+    }
   }
-  __syncthreads();
-  return wtot[0];
 }
 
-// Bin holding the need-th largest element of a 2048-bin histogram whose bins
-// [2*tid, 2*tid+1] are c0, c1 (bins grow with the key): res[0..2] = digit,
-// count above it, its count.  Three barriers; everyone reads res afterwards.
-template <int T>
-__device__ __forceinline__ void hist_search(uint32_t c0, uint32_t c1, uint32_t need, SelShared<T> &sh) {
-  static_assert(RB == 2 * T, "two bins per thread");
-  constexpr int W = T / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t mine = c0 + c1;
-  uint32_t suf = mine;  // inclusive suffix over the lanes of this warp
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t u = __shfl_down_sync(0xffffffffu, suf, o);
-    if (lane + o < 32) suf += u;
-  }
-  if (lane == 0) sh.wtot[warp] = suf;
-  __syncthreads();
-  if (warp == 0) {  // wscan[w] = elements in warps above w
-    const uint32_t v = lane < W ? sh.wtot[lane] : 0u;
-    uint32_t sfx = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t u = __shfl_down_sync(0xffffffffu, sfx, o);
-      if (lane + o < 32) sfx += u;
-    }
-    if (lane < W) sh.wscan[lane] = sfx - v;
-  }
-  __syncthreads();
-  const uint32_t above1 = (suf - mine) + sh.wscan[warp];  // elements in bins above 2*tid+1
-  if (above1 < need && above1 + c1 >= need) {
-    sh.res[0] = 2 * threadIdx.x + 1;
-    sh.res[1] = above1;
-    sh.res[2] = c1;
-  } else if (above1 + c1 < need && above1 + c1 + c0 >= need) {
-    sh.res[0] = 2 * threadIdx.x;
-    sh.res[1] = above1 + c1;
-    sh.res[2] = c0;
-  }
-  __syncthreads();
-}
+int sel_smem_bytes(int L_cap) { return (int)sizeof(SelShared) + 4 * cdiv(L_cap, 32); }
+constexpr int SEL_SMEM_MAX = (int)sizeof(SelShared) + 4 * (MISA_MAX_L / 32);
 
-template <int T, int E, bool GATHER>
-__global__ void __launch_bounds__(T, 1) select_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
-                                                      int n_cols, const int32_t *gather,
-                                                      const uint32_t *row_hist, int k, int32_t *out) {
-  extern __shared__ __align__(16) uint8_t sel_smem[];
-  SelShared<T> &sh = *reinterpret_cast<SelShared<T> *>(sel_smem);
-  uint32_t *skey = reinterpret_cast<uint32_t *>(sel_smem + sizeof(SelShared<T>));  // [E][T]
-#define KEY(e) skey[(e) * T + tid]
-  cg::cluster_group cluster = cg::this_cluster();
-  const int CS = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
-  const int row = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int s;
-  const int Li = query_prefix(c, qv, row, &s);
-  const int ncols = GATHER ? n_cols : Li;
-  const int base = rank * (T * E) + warp * (32 * E) + lane;  // position of element e: base + 32e
-
-  // ---- load: this thread's keys and two bins of the row histogram ----
-  const uint32_t *rh = row_hist + (size_t)row * RB;
-  const uint32_t h0 = rh[2 * tid], h1 = rh[2 * tid + 1];
-  uint32_t valid = 0;
-  {
-    int tk[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int p = base + 32 * e;
-      tk[e] = (GATHER && p < ncols) ? __ldg(gather + (size_t)row * n_cols + p) : p;
-    }
-    float sv[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int p = base + 32 * e;
-      const bool v = p < ncols && (!GATHER || (tk[e] >= 0 && tk[e] < Li));
-      sv[e] = v ? scores[(size_t)row * ld + p] : 0.f;
-      valid |= (uint32_t)v << e;
-    }
-#pragma unroll
-    for (int e = 0; e < E; ++e) KEY(e) = ((valid >> e) & 1) ? ordered_key(sv[e]) : 0u;
-  }
-  if (tid == 0) {
-    sh.n_cand = 0;
-    sh.n_hi = 0;
-    sh.n_in = 0;
-  }
-  if (tid < MAX_CS) sh.sel_cnt[tid] = 0;
-
-  // ---- 1. boundary bin from the histogram (same result in every CTA) ----
-  const uint32_t all = warp_totals_scan<T>(__reduce_add_sync(0xffffffffu, h0 + h1), sh.wtot, sh.wscan);
-  const uint32_t kk = min((uint32_t)k, all);
-  uint32_t need = kk;
-  uint32_t P_hi = 0, M_hi = 0, P_lo = 0, M_lo = 0;
-  const bool all_in = kk == all;  // uniform: every valid element is selected
-  uint32_t d0 = 0, in0 = 0;
-  if (!all_in) {
-    hist_search<T>(h0, h1, need, sh);
-    d0 = sh.res[0];
-    need -= sh.res[1];
-    in0 = sh.res[2];
-    P_hi = d0 << 21;
-    M_hi = TOP_MASK;
-  }
-  const bool listed = !all_in && in0 != need && in0 <= CAP;   // uniform
-  const bool fallback = !all_in && in0 != need && in0 > CAP;  // uniform
-  uint32_t n_hi = 0, n_in = 0;
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const uint32_t kx = KEY(e);
-    const bool v = (valid >> e) & 1;
-    n_hi += (v && (all_in || (kx >> 21) > d0)) ? 1u : 0u;
-    const bool cd = v && !all_in && (kx >> 21) == d0;
-    n_in += cd ? 1u : 0u;
-    if (listed) {
-      const unsigned m = __ballot_sync(0xffffffffu, cd);
-      if (m) {
-        uint32_t slot = 0;
-        if (lane == 0) slot = atomicAdd(&sh.n_cand, (uint32_t)__popc(m));
-        slot = __shfl_sync(0xffffffffu, slot, 0);
-        if (cd) {
-          const uint32_t o = slot + __popc(m & ((1u << lane) - 1u));
-          sh.cand_key[o] = kx;
-          sh.cand_lo[o] = POS_MAX - (uint32_t)(base + 32 * e);
-          sh.cand_rank[o] = (uint8_t)rank;
-        }
-      }
-    }
-  }
-  n_hi = __reduce_add_sync(0xffffffffu, n_hi);
-  n_in = __reduce_add_sync(0xffffffffu, n_in);
-  if (lane == 0) {
-    atomicAdd(&sh.n_hi, n_hi);
-    atomicAdd(&sh.n_in, n_in);
-  }
-  cluster.sync();  // barrier 1
-
-  // ---- 2. rank 0: exact threshold and output offsets ----
-  if (rank == 0 && !fallback) {
-    uint32_t cnt_hi[MAX_CS], cnt_in[MAX_CS], cbase[MAX_CS + 1];
-    cbase[0] = 0;
-#pragma unroll
-    for (int r = 0; r < MAX_CS; ++r) {
-      const SelShared<T> *o = cluster.map_shared_rank(&sh, r < CS ? r : 0);
-      cnt_hi[r] = r < CS ? o->n_hi : 0u;
-      cnt_in[r] = r < CS ? o->n_in : 0u;
-      cbase[r + 1] = cbase[r] + (r < CS && listed ? o->n_cand : 0u);
-    }
-    if (listed) {
-      const uint32_t C = cbase[MAX_CS];
-      // the other ranks' lists go behind this CTA's own
-#pragma unroll 4
-      for (uint32_t x = cbase[1] + tid; x < C; x += T) {
-        int r = 1;
-#pragma unroll
-        for (int q = 2; q < MAX_CS; ++q) r = (x >= cbase[q]) ? q : r;
-        const SelShared<T> *o = cluster.map_shared_rank(&sh, r);
-        const uint32_t idx = x - cbase[r];
-        sh.cand_key[x] = o->cand_key[idx];
-        sh.cand_lo[x] = o->cand_lo[idx];
-        sh.cand_rank[x] = o->cand_rank[idx];
-      }
-      __syncthreads();
-      bool done = false;
-      for (int p = 0; p < 4 && !done; ++p) {
-        const bool lo_word = p >= 2;
-        const int sft = kShift[p];
-        const uint32_t dm = (1u << kWidth[p]) - 1u;
-        for (int b = tid; b < RB; b += T) sh.lhist[b] = 0;
-        __syncthreads();
-        for (uint32_t x = tid; x < C; x += T) {
-          const uint32_t kx = sh.cand_key[x], lx = sh.cand_lo[x];
-          if ((kx & M_hi) == P_hi && (lx & M_lo) == P_lo) atomicAdd(&sh.lhist[((lo_word ? lx : kx) >> sft) & dm], 1u);
-        }
-        __syncthreads();
-        hist_search<T>(sh.lhist[2 * tid], sh.lhist[2 * tid + 1], need, sh);
-        const uint32_t dg = sh.res[0];
-        need -= sh.res[1];
-        if (!lo_word) {
-          P_hi |= dg << sft;
-          M_hi |= dm << sft;
-        } else {
-          P_lo |= dg << sft;
-          M_lo |= dm << sft;
-        }
-        done = sh.res[2] == need;
-      }
-      // selected listed elements, per source rank
-      for (uint32_t x = tid; x < C; x += T) {
-        const uint32_t kh = sh.cand_key[x] & M_hi, kl = sh.cand_lo[x] & M_lo;
-        if (kh > P_hi || (kh == P_hi && kl >= P_lo)) atomicAdd(&sh.sel_cnt[sh.cand_rank[x]], 1u);
-      }
-      __syncthreads();
-    }
-    if (tid == 0) {
-      uint32_t off = 0;
-      for (int r = 0; r < MAX_CS; ++r) {
-        sh.offs[r] = off;
-        off += cnt_hi[r] + (listed ? sh.sel_cnt[r] : cnt_in[r]);  // unlisted: the whole bin d0 is in
-      }
-      sh.dec[0] = P_hi;
-      sh.dec[1] = M_hi;
-      sh.dec[2] = P_lo;
-      sh.dec[3] = M_lo;
-    }
-  }
-  cluster.sync();  // barrier 2
-  uint32_t off = 0;
-  if (!fallback) {
-    const SelShared<T> *r0 = cluster.map_shared_rank(&sh, 0);
-    off = r0->offs[rank];
-    P_hi = r0->dec[0];
-    M_hi = r0->dec[1];
-    P_lo = r0->dec[2];
-    M_lo = r0->dec[3];
-  } else {
-    // Boundary bin beyond the gather capacity: cluster-wide passes over the
-    // slices (the histograms meet through distributed shared memory).
-    bool done = false;
-    for (int p = 0; p < 4 && !done; ++p) {
-      const bool lo_word = p >= 2;
-      const int sft = kShift[p];
-      const uint32_t dm = (1u << kWidth[p]) - 1u;
-      for (int b = tid; b < RB; b += T) sh.lhist[b] = 0;
-      __syncthreads();
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        const uint32_t lo = POS_MAX - (uint32_t)(base + 32 * e), kx = KEY(e);
-        if (((valid >> e) & 1) && (kx & M_hi) == P_hi && (lo & M_lo) == P_lo)
-          atomicAdd(&sh.lhist[((lo_word ? lo : kx) >> sft) & dm], 1u);
-      }
-      cluster.sync();
-      uint32_t c0 = 0, c1 = 0;
-      for (int r = 0; r < CS; ++r) {
-        const uint32_t *hr = cluster.map_shared_rank(sh.lhist, r);
-        c0 += hr[2 * tid];
-        c1 += hr[2 * tid + 1];
-      }
-      cluster.sync();  // every rank has read every histogram before any clears its own
-      hist_search<T>(c0, c1, need, sh);
-      const uint32_t dg = sh.res[0];
-      need -= sh.res[1];
-      if (!lo_word) {
-        P_hi |= dg << sft;
-        M_hi |= dm << sft;
-      } else {
-        P_lo |= dg << sft;
-        M_lo |= dm << sft;
-      }
-      done = sh.res[2] == need;
-    }
-  }
-
-  // ---- 3. ordered output: composite >= (P_hi, P_lo) on the decided bits ----
-  uint32_t selm = 0;
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const uint32_t lo = POS_MAX - (uint32_t)(base + 32 * e);
-    const uint32_t kh = KEY(e) & M_hi, kl = lo & M_lo;
-    selm |= (uint32_t)(((valid >> e) & 1) && (kh > P_hi || (kh == P_hi && kl >= P_lo))) << e;
-  }
-  uint32_t wsel = 0;
-#pragma unroll
-  for (int e = 0; e < E; ++e) wsel += __popc(__ballot_sync(0xffffffffu, (selm >> e) & 1));
-  const uint32_t cta_sel = warp_totals_scan<T>(wsel, sh.wtot, sh.wscan);
-  if (fallback) {  // offsets from a prefix over the ranks' selected counts
-    if (tid == 0) sh.n_hi = cta_sel;
-    cluster.sync();
-    for (int r = 0; r < rank; ++r) off += cluster.map_shared_rank(&sh, r)->n_hi;
-  }
-  off += sh.wscan[warp];
-  int32_t *orow = out + (size_t)row * k;
-#pragma unroll
-  for (int e = 0; e < E; ++e) {
-    const uint32_t m = __ballot_sync(0xffffffffu, (selm >> e) & 1);
-    if ((m >> lane) & 1) {
-      const int p = base + 32 * e;
-      const int t = GATHER ? __ldg(gather + (size_t)row * n_cols + p) : p;
-      const uint32_t o = off + __popc(m & ((1u << lane) - 1u));
-      if (o < (uint32_t)k) orow[o] = t;
-    }
-    off += __popc(m);
-  }
-  if (rank == CS - 1)
-    for (int p = (int)kk + tid; p < k; p += T) orow[p] = -1;
-  cluster.sync();  // barrier 3: no CTA leaves while others may still read its shared memory
-#undef KEY
-}
-
-template <int T, int E, bool GATHER>
-cudaError_t launch_te(int CS, int rows, const CacheView &c, const QueryView &q, const float *scores, long long ld,
-                      int n_cols, const int32_t *gather, const uint32_t *row_hist, int k, int32_t *out,
-                      cudaStream_t s) {
-  constexpr int SMEM = sel_smem_bytes<T, E>();
+template <bool GATHER, bool FROM_LIST>
+cudaError_t launch_select(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
+                          const int32_t *gather, const uint32_t *row_hist, const uint2 *list,
+                          const uint32_t *list_cnt, int list_cap, int k, int32_t *out, cudaStream_t s) {
   struct Tag {};
   const int ok = cached_per_device<Tag>([] {
-    return cudaFuncSetAttribute(select_kernel<T, E, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) ==
-                   cudaSuccess
+    return cudaFuncSetAttribute(select_kernel<GATHER, FROM_LIST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SEL_SMEM_MAX) == cudaSuccess
                ? 1
                : -1;
   });
   if (ok < 0) return cudaErrorInvalidConfiguration;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(CS, rows);
-  cfg.blockDim = dim3(T);
-  cfg.dynamicSmemBytes = SMEM;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CS;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, select_kernel<T, E, GATHER>, c, q, scores, ld, n_cols, gather, row_hist, k, out);
+  select_kernel<GATHER, FROM_LIST><<<q.n_q, SEL_T, sel_smem_bytes(c.L_cap), s>>>(
+      c, q, scores, ld, n_cols, gather, row_hist, list, list_cnt, list_cap, k, out);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
+size_t topk_list_entries(int n_q, int L_cap, int k) {
+  if (n_q < 1 || n_q > TOPK_LIST_MAX_ROWS || L_cap <= TOPK_LIST_MIN_L || k < 1) return 0;
+  return (size_t)n_q * ((size_t)k + TOPK_LIST_EXTRA);
+}
+
 cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
-                        const int32_t *gather, const uint32_t *row_hist, int k, int32_t *out, cudaStream_t s) {
+                        const int32_t *gather, const uint32_t *row_hist, void *list_ws, uint32_t *list_cnt, int k,
+                        int32_t *out, cudaStream_t s) {
   if (q.n_q == 0) return cudaSuccess;
-  const long long cols = gather ? n_cols : c.L_cap;
-  // 1024 threads x E keys per CTA (E in {4, 8, 16, 32}), up to 8 CTAs per row
-  int E = 4;
-  while (E < 32 && (long long)MAX_CS * 1024 * E < cols) E *= 2;
-  if (E < 8 && cols > 1024LL * E) E = 8;
-  int CS = 1;
-  while ((long long)CS * 1024 * E < cols) CS *= 2;
-  if (CS > MAX_CS) return cudaErrorInvalidValue;
-#define MISA_TOPK_CASE(EE)                                                                                     \
-  case EE:                                                                                                     \
-    return gather ? launch_te<1024, EE, true>(CS, q.n_q, c, q, scores, ld, n_cols, gather, row_hist, k, out, s) \
-                  : launch_te<1024, EE, false>(CS, q.n_q, c, q, scores, ld, n_cols, gather, row_hist, k, out, s);
-  switch (E) {
-    MISA_TOPK_CASE(4)
-    MISA_TOPK_CASE(8)
-    MISA_TOPK_CASE(16)
-    MISA_TOPK_CASE(32)
-    default:
-      return cudaErrorInvalidValue;
-  }
-#undef MISA_TOPK_CASE
+  if (gather)
+    return launch_select<true, false>(c, q, scores, ld, n_cols, gather, row_hist, nullptr, nullptr, 0, k, out, s);
+  if (topk_list_entries(q.n_q, c.L_cap, k) == 0 || !list_ws || !list_cnt)
+    return launch_select<false, false>(c, q, scores, ld, 0, nullptr, row_hist, nullptr, nullptr, 0, k, out, s);
+  const int list_cap = k + TOPK_LIST_EXTRA;
+  uint2 *list = static_cast<uint2 *>(list_ws);
+  // about two CTAs per SM over all rows, at least 4096 elements each
+  const int sms = device_sms();
+  const int per_row = max(1, min(cdiv(c.L_cap, 4096), 2 * sms / q.n_q));
+  const int chunk = cdiv(cdiv(c.L_cap, per_row), FILT_T) * FILT_T;
+  filter_kernel<<<dim3(cdiv(c.L_cap, chunk), q.n_q), FILT_T, 0, s>>>(c, q, scores, ld, row_hist, list, list_cnt,
+                                                                     list_cap, k, chunk);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_select<false, true>(c, q, scores, ld, 0, nullptr, row_hist, list, list_cnt, list_cap, k, out, s);
 }
 
 }  // namespace misa

@@ -23,6 +23,8 @@ CASES = {
     "fp8_mixture": W["misa_dagger_decode_128k"].scaled(n_seq=3, L=3001, B=128, k=64, k_prime=300),
     "bf16_prefill": W["causal_prefill"].scaled(L=1500, n_q=70, k=64),
     "fp8_prefill_h32": W["long_prefill_128k"].scaled(L=2100, n_q=40, B=100, k=33),
+    # few long rows: the top-k goes through the compact boundary-bin list
+    "fp8_long": W["misa_dagger_decode_128k"].scaled(n_seq=2, L=40000, B=128, k=600, k_prime=4000),
 }
 
 
@@ -275,3 +277,66 @@ def test_needles_selected_by_dense_gpu():
     top = M.dense_score_topk(cache, qs, inp.wl.k).cpu().numpy()
     for s, p, qi in inp.needles:
         assert p in set(top[qi].tolist())
+
+
+def _tied_case(L, pattern, k):
+    """bf16 cache whose keys take two values (pattern[t] = 0 or 1), so that
+    scores tie massively; expected top-k from the oracle (ties to the lower
+    token index)."""
+    wl = W["batched_decode"].scaled(n_seq=2, L=L, B=128, k=k)
+    inp = G.make_inputs(wl, 4)
+    a, b = inp.keys[0, 0].copy(), inp.keys[0, 1].copy()
+    for s_ in range(wl.n_seq):
+        inp.keys[s_] = np.where(pattern[:, None] == 1, b[None, :], a[None, :])
+    ref = Ref(inp)
+    cache, qs = to_device(inp, torch)
+    top = M.dense_score_topk(cache, qs, k).cpu().numpy()
+    for i in range(wl.n_q):
+        q, w, K, Li = ref.query(i)
+        d = O.dense_query(q, w, K, Li, k)
+        np.testing.assert_array_equal(top[i], d["topk"], err_msg=f"q{i}")
+    assert device_status(cache) == 0
+
+
+@pytest.mark.parametrize("L", [3000, 40000])
+@pytest.mark.parametrize("k", [1, 100, 2999])
+def test_topk_all_scores_equal(L, k):
+    # one boundary bin holds every element: ties decide (listed refinement for
+    # short rows, whole-row passes when the bin is too large to list)
+    _tied_case(L, np.zeros(L, dtype=np.int64), k)
+
+
+@pytest.mark.parametrize("L", [3000, 40000])
+def test_topk_two_score_levels(L):
+    # half the tokens share one score, half another: k equal to one half takes
+    # a whole bin; k a little larger cuts into the other half by index
+    pat = (np.arange(L) % 2).astype(np.int64)
+    for k in (L // 2, L // 2 + 37):
+        _tied_case(L, pat, k)
+
+
+def test_rerank_candidate_order_does_not_matter():
+    # outputs are token indices in ascending order whatever the candidate
+    # order, and the selection is the oracle's (ties to the lower token)
+    inp = make("fp8_long")
+    ref = Ref(inp)
+    wl = inp.wl
+    kp = wl.k_prime
+    rng = np.random.default_rng(9)
+    cache, qs = to_device(inp, torch)
+    cands = []
+    for i in range(wl.n_q):
+        Li = int(inp.q_pos[i]) + 1
+        cands.append(rng.choice(Li, size=kp, replace=False).astype(np.int32))
+    c_sorted = torch.from_numpy(np.sort(np.stack(cands), axis=1)).cuda()
+    c_shuf = torch.from_numpy(np.stack(cands)).cuda()
+    a = M.rerank_topk(cache, qs, c_sorted, wl.k).cpu().numpy()
+    b = M.rerank_topk(cache, qs, c_shuf, wl.k).cpu().numpy()
+    np.testing.assert_array_equal(a, b)
+    for i in range(wl.n_q):
+        q, w, K, Li = ref.query(i)
+        f = O.rerank_query(q, w, K, cands[i], wl.k)
+        smap = dict(zip(f["cand"].tolist(), f["scores"].tolist()))
+        compare_selection(b[i], f["topk"], lambda t: smap[t], wl.k, f"q{i}")
+        got = b[i][b[i] >= 0]
+        assert np.all(np.diff(got) > 0)
