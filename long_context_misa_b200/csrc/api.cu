@@ -142,13 +142,22 @@ misa_status score_then_topk(const char *who, const misa_cache *cache, const misa
   uint32_t *list_cnt = hist + (size_t)qs->n_q * misa::TOPK_HIST_BINS;
   float *scores = scores_out ? scores_out : reinterpret_cast<float *>(w8 + ws_hist(qs));
   void *list = w8 + ws_hist(qs) + (scores_out ? 0 : ws_score(cache, qs));
-  cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * hist_words(qs), stream);
-  if (e != cudaSuccess) return cuda_fail(e, who);
+  // many queries per sequence (prefill chunks): tensor-core scoring, and the
+  // selection counts each row itself; otherwise the streaming scorer builds
+  // the row histograms on the way
+  const bool umma = misa::umma_applies(c, q, heads, h);
+  cudaError_t e = cudaSuccess;
+  if (!umma) {
+    e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * hist_words(qs), stream);
+    if (e != cudaSuccess) return cuda_fail(e, who);
+  }
   e = timed_scoring(stream, [&] {
-    return misa::launch_score_mma(c, q, heads, h, nullptr, 0, scores, cache->L_cap, hist, stream);
+    return umma ? misa::launch_score_umma(c, q, heads, h, scores, cache->L_cap, stream)
+                : misa::launch_score_mma(c, q, heads, h, nullptr, 0, scores, cache->L_cap, hist, stream);
   });
   if (e != cudaSuccess) return cuda_fail(e, who);
-  e = misa::launch_topk(c, q, scores, cache->L_cap, 0, nullptr, hist, list, list_cnt, k, topk, stream);
+  e = misa::launch_topk(c, q, scores, cache->L_cap, 0, nullptr, umma ? nullptr : hist, list, list_cnt, k, topk,
+                        stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   return MISA_OK;
 }

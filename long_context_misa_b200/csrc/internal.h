@@ -38,12 +38,18 @@ cudaError_t launch_score_mma(const CacheView &c, const QueryView &q, const int32
 cudaError_t launch_score_stream(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
                                 long long ld, uint32_t *row_hist, cudaStream_t s);
 
+// score_umma.cu: prefix scoring of query batches with many queries per
+// sequence (prefill chunks) on tcgen05 tensor cores; writes no histogram.
+bool umma_applies(const CacheView &c, const QueryView &q, const int32_t *heads, int h);
+cudaError_t launch_score_umma(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
+                              long long ld, cudaStream_t s);
+
 // topk.cu: per row, the k largest scores, ties to the lower token index;
 // outputs are token indices in ascending order, -1 padded.  Row length comes
 // from the query prefix (gather == nullptr), or the row holds n_cols
 // candidates whose tokens are gather[i][p] (entries < 0 or beyond the prefix
 // excluded).  row_hist is the histogram the scoring kernel built over exactly
-// the valid scores.  Prefix rows with few queries and long caches go through
+// the valid scores, or null: the selection then counts the row itself.  Prefix rows with few queries and long caches go through
 // a compact list of the elements at or above the histogram's boundary bin:
 // list_ws holds topk_list_entries() entries of 8 bytes and list_cnt n_q
 // counters, zeroed beforehand (both may be null: no list).

@@ -1,0 +1,518 @@
+// Token scoring of prefill chunks on the fifth-generation tensor cores
+// (tcgen05.mma, accumulators in tensor memory, key tiles staged by TMA).
+//
+// "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM Inference",
+// technical summary, "Methodology: MISA" step 2 (the routed heads S_i score
+// every prefix token) and "Problem statement" (the dense indexer, S_i = all
+// H_I heads):
+//     I_{i,t} = s_t * sum_{j in S_i} w_{i,j} * ReLU(q_{i,j} . k_t),  t < L_i.
+// The key k_t is shared by all heads, so the scoring heads of a group of
+// queries stack into one matrix Q' [256 x 128] (query-major, HPQ columns per
+// query, HPQ = the number of scoring heads rounded up to a power of two, at
+// least 4) and
+// every 128-token tile of keys is one dense MMA  D[t][n] = K[t] . Q'[n]:
+// tokens on the M side, query-heads on the N side, fp32 accumulators in
+// tensor memory.  The epilogue reads a token row per thread, applies ReLU and
+// the weights, sums each query's HPQ columns, multiplies by s_t and writes
+// the causal part of the query's score row; per-head products never reach
+// global memory.
+//
+// bf16 keys: kind::f16 MMA on bf16 keys and the bf16 query heads.
+// e4m3 keys: kind::f8f6f4 MMA on the keys as stored and an exact two-term
+//   e4m3 split of each query head (scaled by a power of two folded into its
+//   weight), both terms accumulating into the same tensor-memory columns.
+//
+// One persistent CTA per SM walks a contiguous range of (query group, token
+// tile) items.  Warp 0 issues the TMA loads of key tiles into a ring of
+// shared-memory stages, warp 1 (which also owns the tensor memory) issues the
+// MMAs from one thread, warps 2..9 drain the accumulators (two warps per
+// lane quarter, half of the columns each); two accumulator
+// buffers of 256 columns let the MMAs of one tile overlap the epilogue of the
+// previous.  Every wait is bounded: a wait that runs out sets
+// MISA_DEV_WAIT_TIMEOUT and the CTA winds down.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "frag.cuh"
+#include "internal.h"
+
+namespace misa {
+namespace {
+
+constexpr int UM_M = 128;                 // tokens per tile
+constexpr int UM_N = 256;                 // query-head columns per tile
+constexpr int EPI_WARPS = 8;                // two per tensor-memory lane quarter
+constexpr int UM_THREADS = 64 + 32 * EPI_WARPS;
+constexpr int B_BYTES = 65536;            // Q' tile: 256 x 128 bf16, or two e4m3 terms
+
+template <bool FP8>
+struct UCfg {
+  static constexpr int ROW = FP8 ? 128 : 256;           // key bytes per token
+  static constexpr int A_BYTES = UM_M * ROW;            // one key tile
+  static constexpr int STAGES = FP8 ? 8 : 4;
+  static constexpr int KSTEPS = FP8 ? 4 : 8;            // MMAs per term and tile (K = 32 / 16)
+  static constexpr int TERMS = FP8 ? 2 : 1;
+};
+
+struct UmmaShared {
+  alignas(16) float wcol[UM_N];     // weight of every column (0 for padding); read as float4
+  uint64_t full[8], empty[8];       // key stages: loaded / consumed
+  uint64_t tfull[2], tempty[2];     // accumulator buffers: written / drained
+  uint32_t tmem_base;
+  int abort;
+  int n_pass;
+  int pass_seq[UM_N];               // distinct sequences of the group's queries
+  int pass_len[UM_N];               // longest prefix among them
+  int q_len[UM_N];                  // per query of the group: prefix length (0: none)
+  int q_seq[UM_N];
+  int q_lenp[UM_N];                 // prefix length if the query belongs to the current pass, else 0
+};
+
+template <bool FP8>
+constexpr int umma_smem_bytes() {
+  return 1024 /* alignment slack */ + UCfg<FP8>::STAGES * UCfg<FP8>::A_BYTES + B_BYTES + (int)sizeof(UmmaShared);
+}
+
+// ---- PTX wrappers -------------------------------------------------------
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+  // K-major, 128-byte swizzle: 8-row atoms of 128 B, 1024 B apart (SBO);
+  // LBO unused (1); descriptor version 1; layout type 2 = SWIZZLE_128B.
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+template <bool FP8>
+__device__ __forceinline__ uint32_t instr_desc() {
+  // D fp32, A/B K-major, N = 256, M = 128; A/B format bf16 (1) or e4m3 (0)
+  const uint32_t fmt = FP8 ? 0u : 1u;
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(UM_N >> 3) << 17) | ((uint32_t)(UM_M >> 4) << 24);
+}
+
+template <bool FP8>
+__device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  if (FP8)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Bounded wait shared by all roles: false once this CTA has given up (here or
+// in another role).
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort, const CacheView &c) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+      *abort = 1;
+      flag(c, MISA_DEV_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// ---- the kernel -----------------------------------------------------------
+
+// Items: (group g, tile tau) flattened as g * n_tiles + tau; this CTA takes
+// [item0, item1).  A group holds QPT = 256 / HPQ consecutive queries.
+template <bool FP8, int HPQ>
+__global__ void __maxnreg__(128)
+    score_umma_kernel(const __grid_constant__ CUtensorMap kmap, CacheView c, QueryView qv, const int32_t *heads,
+                      int h, float *scores, long long ld, int n_tiles, long long n_items) {
+  using Cfg = UCfg<FP8>;
+  constexpr int QPT = UM_N / HPQ;
+  extern __shared__ uint8_t um_raw[];
+  uint8_t *base = um_raw + ((1024u - (smem_addr(um_raw) & 1023u)) & 1023u);  // 1024-aligned (swizzle atoms)
+  uint8_t *a_smem = base;                                    // STAGES x A_BYTES (1024-aligned each)
+  uint8_t *b_smem = base + Cfg::STAGES * Cfg::A_BYTES;       // B_BYTES
+  UmmaShared &sh = *reinterpret_cast<UmmaShared *>(b_smem + B_BYTES);
+  volatile int *abort = &sh.abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = qv.H;
+  const int h_eff = heads ? h : H;
+
+  const long long per = (n_items + gridDim.x - 1) / gridDim.x;
+  const long long item0 = min(n_items, (long long)blockIdx.x * per);
+  const long long item1 = min(n_items, item0 + per);
+  if (item0 >= item1) return;  // uniform; nothing allocated yet
+
+  if (tid == 0) {
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sh.tfull[b], 1);
+      mbar_init(&sh.tempty[b], EPI_WARPS);
+    }
+    sh.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_addr(&sh.tmem_base)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem_base;
+
+  // pipeline counters (same sequence of tiles in every role)
+  uint32_t it_load = 0, it_mma = 0, j_mma = 0, j_epi = 0;
+  uint32_t last_fill_parity[8];
+#pragma unroll
+  for (int s = 0; s < 8; ++s) last_fill_parity[s] = 2;  // 2: never filled
+  bool mma_issued = false;
+
+  for (long long item = item0; item < item1 && !*abort;) {
+    const int g = (int)(item / n_tiles);
+    const int tau0 = (int)(item % n_tiles);
+    const int tau1 = (int)min((long long)n_tiles, item1 - (long long)g * n_tiles);  // exclusive
+    item = (long long)g * n_tiles + tau1;
+
+    // ---- segment set-up: the group's queries, weights and Q' tile ----
+    for (int ql = tid; ql < QPT; ql += UM_THREADS) {
+      const int qi = g * QPT + ql;
+      int s = -1, Li = 0;
+      if (qi < qv.n_q) Li = query_prefix(c, qv, qi, &s);
+      sh.q_len[ql] = Li;
+      sh.q_seq[ql] = Li > 0 ? s : -1;
+    }
+    // rows n = ql * HPQ + j of Q': query g*QPT + ql, its j-th scoring head
+    for (int n = tid; n < UM_N; n += UM_THREADS) {
+      const int ql = n / HPQ, j = n % HPQ, qi = g * QPT + ql;
+      int hd = -1;
+      if (qi < qv.n_q && j < h_eff) {
+        hd = heads ? __ldg(heads + (size_t)qi * h + j) : j;
+        if (hd < 0 || hd >= H) {
+          flag(c, MISA_DEV_BAD_HEAD);
+          hd = 0;
+        }
+      }
+      float wv = 0.f;
+      const uint4 *row = reinterpret_cast<const uint4 *>(qv.q + ((size_t)(hd >= 0 ? qi : 0) * H + max(hd, 0)) * D);
+      if (hd >= 0) wv = __ldg(qv.w + (size_t)qi * H + hd);
+      if (!FP8) {
+        // 16-byte chunk u of the row: K-block u / 8, chunk u % 8 of the 128-byte swizzled row
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint4 v[8];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) v[x] = hd >= 0 ? __ldg(row + half * 8 + x) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+          for (int x = 0; x < 8; ++x)
+            *reinterpret_cast<uint4 *>(b_smem + half * (UM_N * 128) + n * 128 + ((x ^ (n & 7)) << 4)) = v[x];
+        }
+      } else {
+        float m = 0.f;
+        if (hd >= 0) {
+#pragma unroll 4
+          for (int u = 0; u < 16; ++u) {
+            const uint4 v = __ldg(row + u);
+            const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const float2 f = bf16x2_to_float2(ww[p]);
+              m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+          }
+        }
+        const float sc = e4m3_head_scale(m);
+        wv = wv / sc;  // exact: sc is a power of two
+        // input chunk u (8 elements) -> 8 bytes of each term at byte 8u of the row
+#pragma unroll 4
+        for (int u = 0; u < 16; ++u) {
+          const uint4 v = hd >= 0 ? __ldg(row + u) : make_uint4(0u, 0u, 0u, 0u);
+          uint2 t1, t2;
+          split_e4m3(v, sc, t1, t2);
+          const int ch = u >> 1, half = u & 1;
+          const int off = n * 128 + ((ch ^ (n & 7)) << 4) + half * 8;
+          *reinterpret_cast<uint2 *>(b_smem + off) = t1;
+          *reinterpret_cast<uint2 *>(b_smem + UM_N * 128 + off) = t2;
+        }
+      }
+      sh.wcol[n] = wv;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    if (tid == 0) {  // distinct sequences of the group, with their longest prefix
+      int np = 0;
+      for (int ql = 0; ql < QPT; ++ql) {
+        const int s = sh.q_seq[ql];
+        if (s < 0) continue;
+        int p = 0;
+        while (p < np && sh.pass_seq[p] != s) ++p;
+        if (p == np) {
+          sh.pass_seq[np] = s;
+          sh.pass_len[np] = 0;
+          ++np;
+        }
+        sh.pass_len[p] = max(sh.pass_len[p], sh.q_len[ql]);
+      }
+      sh.n_pass = np;
+    }
+    __syncthreads();
+    const int n_pass = sh.n_pass;
+
+    for (int pass = 0; pass < n_pass; ++pass) {
+      const int seq = sh.pass_seq[pass];
+      for (int ql = tid; ql < QPT; ql += UM_THREADS) sh.q_lenp[ql] = sh.q_seq[ql] == seq ? sh.q_len[ql] : 0;
+      __syncthreads();
+      const int t_end = min(tau1, cdiv(sh.pass_len[pass], UM_M));  // tiles [tau0, t_end) hold prefix tokens
+      if (warp == 0) {
+        // ---- TMA producer ----
+        if (lane == 0) {
+          for (int tau = tau0; tau < t_end; ++tau, ++it_load) {
+            const int st = it_load % Cfg::STAGES;
+            if (!wait_bar(&sh.empty[st], ((it_load / Cfg::STAGES) & 1) ^ 1, abort, c)) break;
+            mbar_arrive_expect_tx(&sh.full[st], Cfg::A_BYTES);
+            const uint32_t dst = smem_addr(a_smem + st * Cfg::A_BYTES);
+            const int y = seq * c.L_cap + tau * UM_M;
+            if (FP8) {
+              tma_load_2d(dst, &kmap, 0, y, &sh.full[st]);
+            } else {
+              tma_load_2d(dst, &kmap, 0, y, &sh.full[st]);
+              tma_load_2d(dst + UM_M * 128, &kmap, 64, y, &sh.full[st]);
+            }
+            last_fill_parity[st] = (it_load / Cfg::STAGES) & 1;
+          }
+        }
+      } else if (warp == 1) {
+        // ---- MMA issuer ----
+        if (lane == 0) {
+          const uint32_t idesc = instr_desc<FP8>();
+          const uint32_t b_base = smem_addr(b_smem);
+          for (int tau = tau0; tau < t_end; ++tau, ++it_mma, ++j_mma) {
+            const int st = it_mma % Cfg::STAGES, buf = j_mma & 1;
+            if (!wait_bar(&sh.tempty[buf], ((j_mma >> 1) & 1) ^ 1, abort, c)) break;
+            tc_fence_after();
+            if (!wait_bar(&sh.full[st], (it_mma / Cfg::STAGES) & 1, abort, c)) break;
+            tc_fence_after();
+            const uint32_t a_base = smem_addr(a_smem + st * Cfg::A_BYTES);
+            const uint32_t d = tmem + buf * UM_N;
+#pragma unroll
+            for (int t = 0; t < Cfg::TERMS; ++t) {
+#pragma unroll
+              for (int kk = 0; kk < Cfg::KSTEPS; ++kk) {
+                uint32_t aoff, boff;
+                if (FP8) {
+                  aoff = kk * 32;
+                  boff = t * (UM_N * 128) + kk * 32;
+                } else {
+                  aoff = (kk >> 2) * (UM_M * 128) + (kk & 3) * 32;
+                  boff = (kk >> 2) * (UM_N * 128) + (kk & 3) * 32;
+                }
+                umma<FP8>(d, smem_desc_sw128(a_base + aoff), smem_desc_sw128(b_base + boff), idesc,
+                          (t | kk) ? 1u : 0u);
+              }
+            }
+            umma_commit(&sh.empty[st]);
+            umma_commit(&sh.tfull[buf]);
+            mma_issued = true;
+          }
+        }
+      } else {
+        // ---- epilogue: one token row per thread, half of the columns per warp ----
+        const int e = warp - 2;
+        const int quarter = warp & 3;           // tensor-memory lanes this warp may read
+        const int col0 = (e / 4) * (UM_N / 2);  // its half of the columns
+        const int r = quarter * 32 + lane;
+        const float4 *wv = reinterpret_cast<const float4 *>(sh.wcol + col0);
+        for (int tau = tau0; tau < t_end; ++tau, ++j_epi) {
+          const int buf = j_epi & 1;
+          const int t = tau * UM_M + r;
+          const float st_scale = (FP8 && t < c.L_cap) ? __ldg(c.scale + (size_t)seq * c.L_cap + t) : 1.f;
+          float *out_t = scores + (size_t)g * QPT * ld + t;  // row of query g*QPT + ql at + ql*ld
+          if (!wait_bar(&sh.tfull[buf], (j_epi >> 1) & 1, abort, c)) break;
+          tc_fence_after();
+          const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * UM_N + col0;
+          float acc = 0.f;  // running sum of a query wider than one chunk
+#pragma unroll
+          for (int ch = 0; ch < UM_N / 64; ch += 2) {
+            uint32_t v0[32], v1[32];
+            tmem_ld32(taddr + ch * 32, v0);
+            tmem_ld32(taddr + ch * 32 + 32, v1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int hc = 0; hc < 2; ++hc) {
+              const uint32_t(&v)[32] = hc ? v1 : v0;
+              const int cb = (ch + hc) * 32;  // first column of this chunk (within the half)
+              float part[32 / 4];
+#pragma unroll
+              for (int x4 = 0; x4 < 8; ++x4) {
+                const float4 w4 = wv[(cb >> 2) + x4];
+                float p = w4.x * fmaxf(__uint_as_float(v[4 * x4]), 0.f);
+                p = fmaf(w4.y, fmaxf(__uint_as_float(v[4 * x4 + 1]), 0.f), p);
+                p = fmaf(w4.z, fmaxf(__uint_as_float(v[4 * x4 + 2]), 0.f), p);
+                part[x4] = fmaf(w4.w, fmaxf(__uint_as_float(v[4 * x4 + 3]), 0.f), p);
+              }
+              // queries of this chunk: HPQ / 4 partial sums each (HPQ <= 32),
+              // or the chunk is part of one query (HPQ > 32)
+              if constexpr (HPQ <= 32) {
+                constexpr int QPC = 32 / HPQ;  // queries per chunk
+                constexpr int PPQ = 8 / QPC;                   // partial sums per query
+#pragma unroll
+                for (int qc = 0; qc < QPC; ++qc) {
+                  float sum = 0.f;
+#pragma unroll
+                  for (int x = 0; x < PPQ; ++x) sum += part[qc * PPQ + x];
+                  const int ql = (col0 + cb) / HPQ + qc;
+                  if (t < sh.q_lenp[ql]) out_t[(size_t)ql * ld] = sum * st_scale;
+                }
+              } else {
+#pragma unroll
+                for (int x = 0; x < 8; ++x) acc += part[x];
+                if (((col0 + cb + 32) % HPQ) == 0) {
+                  const int ql = (col0 + cb) / HPQ;
+                  if (t < sh.q_lenp[ql]) out_t[(size_t)ql * ld] = acc * st_scale;
+                  acc = 0.f;
+                }
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.tempty[buf]);
+        }
+      }
+      __syncthreads();  // every role is done with this pass
+      if (*abort) break;
+    }
+    __syncthreads();  // Q' and the group's tables are free again
+  }
+
+  // ---- wind-down: nothing in flight when the tensor memory is released ----
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < Cfg::STAGES; ++s)
+      if (last_fill_parity[s] < 2) wait_bar(&sh.full[s], last_fill_parity[s], abort, c);
+  }
+  if (warp == 1 && lane == 0 && mma_issued) {
+    const uint32_t jl = j_mma - 1;  // the last committed accumulator buffer
+    wait_bar(&sh.tfull[jl & 1], (jl >> 1) & 1, abort, c);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+  }
+}
+
+// ---- host side ----------------------------------------------------------
+
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (EncodeTiled) nullptr;
+    return reinterpret_cast<EncodeTiled>(p);
+  }();
+  return fn;
+}
+
+template <bool FP8, int HPQ>
+cudaError_t launch_hpq(const CUtensorMap &map, const CacheView &c, const QueryView &q, const int32_t *heads, int h,
+                       float *scores, long long ld, cudaStream_t s) {
+  constexpr int SMEM = umma_smem_bytes<FP8>();
+  struct Tag {};
+  // the attribute call's status, cached per device (+1 so that 0 means unset)
+  const int st = cached_per_device<Tag>([] {
+    return 1 + (int)cudaFuncSetAttribute(score_umma_kernel<FP8, HPQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM);
+  });
+  if (st != 1) return (cudaError_t)(st - 1);
+  constexpr int QPT = UM_N / HPQ;
+  const int n_groups = cdiv(q.n_q, QPT);
+  const int n_tiles = cdiv(c.L_cap, UM_M);
+  const long long n_items = (long long)n_groups * n_tiles;
+  const int grid = (int)std::min<long long>(device_sms(), n_items);
+  score_umma_kernel<FP8, HPQ><<<grid, UM_THREADS, SMEM, s>>>(map, c, q, heads, h, scores, ld, n_tiles, n_items);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool umma_applies(const CacheView &c, const QueryView &q, const int32_t *heads, int h) {
+  const int h_eff = heads ? h : q.H;
+  return q.n_q >= 64 && q.n_q >= 8 * c.n_seq && h_eff <= UM_N && encode_fn() != nullptr;
+}
+
+cudaError_t launch_score_umma(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
+                              long long ld, cudaStream_t s) {
+  if (q.n_q == 0) return cudaSuccess;
+  EncodeTiled enc = encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)c.n_seq * (cuuint64_t)c.L_cap};
+  const cuuint64_t strides[1] = {(cuuint64_t)(c.fp8 ? D : 2 * D)};
+  const cuuint32_t box[2] = {(cuuint32_t)(c.fp8 ? 128 : 64), (cuuint32_t)UM_M};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(&map, c.fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                         const_cast<void *>(c.keys), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  const int h_eff = heads ? h : q.H;
+  int hpq = 4;  // at least 4 columns per query (zero-weight padding)
+  while (hpq < h_eff) hpq *= 2;
+#define MISA_UMMA_CASE(N)                                                                                  \
+  case N:                                                                                                  \
+    return c.fp8 ? launch_hpq<true, N>(map, c, q, heads, h, scores, ld, s)                                 \
+                 : launch_hpq<false, N>(map, c, q, heads, h, scores, ld, s);
+  switch (hpq) {
+    MISA_UMMA_CASE(4)
+    MISA_UMMA_CASE(8)
+    MISA_UMMA_CASE(16)
+    MISA_UMMA_CASE(32)
+    MISA_UMMA_CASE(64)
+    MISA_UMMA_CASE(128)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef MISA_UMMA_CASE
+}
+
+}  // namespace misa

@@ -145,6 +145,19 @@ __device__ __forceinline__ Boundary warp_boundary(const uint32_t *rh, int k) {
   return b;
 }
 
+// The same from a histogram in shared memory (hpos layout).
+__device__ __forceinline__ Boundary warp_boundary_smem(const uint32_t *hs, int k) {
+  const uint4 r = warp_select_bin<true>(hs, (uint32_t)k);
+  Boundary b;
+  b.total = r.w;
+  b.kk = min((uint32_t)k, r.w);
+  b.all_in = (uint32_t)k >= r.w;
+  b.d0 = b.all_in ? 0u : r.x;
+  b.above = b.all_in ? 0u : r.y;
+  b.in0 = b.all_in ? 0u : r.z;
+  return b;
+}
+
 // Exclusive prefix of `v` over the threads in thread order; *total = block sum.
 template <int T>
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *total, uint32_t *wa, uint32_t *wb) {
@@ -378,7 +391,7 @@ __device__ __forceinline__ void refine(SelShared &sh, uint32_t &P_hi, uint32_t &
   }
 }
 
-template <bool GATHER, bool FROM_LIST>
+template <bool GATHER, bool FROM_LIST, bool OWN_HIST>
 __global__ void __launch_bounds__(SEL_T) select_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
                                                        int n_cols, const int32_t *gather, const uint32_t *row_hist,
                                                        const uint2 *list, const uint32_t *list_cnt, int list_cap,
@@ -409,9 +422,23 @@ __global__ void __launch_bounds__(SEL_T) select_kernel(CacheView c, QueryView qv
   const int Li = query_prefix(c, qv, row, &s);
   const int n = GATHER ? n_cols : Li;
   const int words = cdiv(Li, 32);
-  const Boundary bd = warp_boundary(row_hist + (size_t)row * RB, k);
+  Boundary bd;
+  if (!OWN_HIST) bd = warp_boundary(row_hist + (size_t)row * RB, k);
   if (tid == 0) sh.n_small = 0;
   for (int w = tid; w < words; w += SEL_T) bm[w] = 0;
+  if (OWN_HIST) {
+    // no histogram from the scoring kernel: count the row's top 11 key bits
+    for (int b = tid; b < HPAD; b += SEL_T) sh.hist[b] = 0;
+    __syncthreads();
+    sweep_row_pf<GATHER>(srow, grow, n_load, n, Li, tk, sv,
+                         [&](const uint32_t(&key)[U], const int(&)[U], const bool(&ok)[U], int) {
+#pragma unroll
+                           for (int u = 0; u < U; ++u)
+                             if (ok[u]) atomicAdd(&sh.hist[hpos(key[u] >> HIST_SHIFT)], 1u);
+                         });
+    __syncthreads();
+    bd = warp_boundary_smem(sh.hist, k);
+  }
   __syncthreads();
 
   if (bd.kk > 0) {
@@ -476,7 +503,7 @@ __global__ void __launch_bounds__(SEL_T) select_kernel(CacheView c, QueryView qv
       };
       if (via_list)
         sweep_list_pf(lrow, list_cap, lcnt, le, visit);
-      else if (!FROM_LIST)
+      else if (!FROM_LIST && !OWN_HIST)
         sweep_row_pf<GATHER>(srow, grow, n_load, n, Li, tk, sv, visit);
       else
         sweep_row<SEL_T, GATHER>(srow, grow, n, Li, visit);
@@ -620,19 +647,19 @@ __global__ void __launch_bounds__(FILT_T) filter_kernel(CacheView c, QueryView q
 int sel_smem_bytes(int L_cap) { return (int)sizeof(SelShared) + 4 * cdiv(L_cap, 32); }
 constexpr int SEL_SMEM_MAX = (int)sizeof(SelShared) + 4 * (MISA_MAX_L / 32);
 
-template <bool GATHER, bool FROM_LIST>
+template <bool GATHER, bool FROM_LIST, bool OWN_HIST = false>
 cudaError_t launch_select(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
                           const int32_t *gather, const uint32_t *row_hist, const uint2 *list,
                           const uint32_t *list_cnt, int list_cap, int k, int32_t *out, cudaStream_t s) {
   struct Tag {};
   const int ok = cached_per_device<Tag>([] {
-    return cudaFuncSetAttribute(select_kernel<GATHER, FROM_LIST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(select_kernel<GATHER, FROM_LIST, OWN_HIST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 SEL_SMEM_MAX) == cudaSuccess
                ? 1
                : -1;
   });
   if (ok < 0) return cudaErrorInvalidConfiguration;
-  select_kernel<GATHER, FROM_LIST><<<q.n_q, SEL_T, sel_smem_bytes(c.L_cap), s>>>(
+  select_kernel<GATHER, FROM_LIST, OWN_HIST><<<q.n_q, SEL_T, sel_smem_bytes(c.L_cap), s>>>(
       c, q, scores, ld, n_cols, gather, row_hist, list, list_cnt, list_cap, k, out);
   return cudaGetLastError();
 }
@@ -650,6 +677,8 @@ cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *sco
   if (q.n_q == 0) return cudaSuccess;
   if (gather)
     return launch_select<true, false>(c, q, scores, ld, n_cols, gather, row_hist, nullptr, nullptr, 0, k, out, s);
+  if (!row_hist)
+    return launch_select<false, false, true>(c, q, scores, ld, 0, nullptr, nullptr, nullptr, nullptr, 0, k, out, s);
   if (topk_list_entries(q.n_q, c.L_cap, k) == 0 || !list_ws || !list_cnt)
     return launch_select<false, false>(c, q, scores, ld, 0, nullptr, row_hist, nullptr, nullptr, 0, k, out, s);
   const int list_cap = k + TOPK_LIST_EXTRA;

@@ -25,12 +25,18 @@ CASES = {
     "fp8_prefill_h32": W["long_prefill_128k"].scaled(L=2100, n_q=40, B=100, k=33),
     # few long rows: the top-k goes through the compact boundary-bin list
     "fp8_long": W["misa_dagger_decode_128k"].scaled(n_seq=2, L=40000, B=128, k=600, k_prime=4000),
+    # prefill chunks of >= 64 queries score on the tcgen05 tensor-core path
+    "fp8_prefill_umma": W["long_prefill_128k"].scaled(L=3000, n_q=96, B=100, k=33),
+    # query groups that span two sequences (two passes over different keys)
+    "bf16_prefill_2seq": W["causal_prefill"].scaled(n_seq=2, L=1300, n_q=80, k=40),
 }
 
 
 def make(case, seed=0, ragged=True):
     wl = CASES[case]
     inp = G.make_inputs(wl, seed)
+    if case.endswith("_2seq"):  # blocks of 20 queries alternate between the sequences
+        inp.q_seq = ((np.arange(wl.n_q) // 20) % 2).astype(np.int32)
     if ragged and wl.mode == "decode":
         inp.seq_len = (wl.L - 37 * np.arange(wl.n_seq)).astype(np.int32)
         inp.q_pos = (inp.seq_len - 1).astype(np.int32)
