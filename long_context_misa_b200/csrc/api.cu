@@ -146,18 +146,14 @@ misa_status score_then_topk(const char *who, const misa_cache *cache, const misa
   // selection counts each row itself; otherwise the streaming scorer builds
   // the row histograms on the way
   const bool umma = misa::umma_applies(c, q, heads, h);
-  cudaError_t e = cudaSuccess;
-  if (!umma) {
-    e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * hist_words(qs), stream);
-    if (e != cudaSuccess) return cuda_fail(e, who);
-  }
+  cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * hist_words(qs), stream);
+  if (e != cudaSuccess) return cuda_fail(e, who);
   e = timed_scoring(stream, [&] {
     return umma ? misa::launch_score_umma(c, q, heads, h, scores, cache->L_cap, stream)
                 : misa::launch_score_mma(c, q, heads, h, nullptr, 0, scores, cache->L_cap, hist, stream);
   });
   if (e != cudaSuccess) return cuda_fail(e, who);
-  e = misa::launch_topk(c, q, scores, cache->L_cap, 0, nullptr, umma ? nullptr : hist, list, list_cnt, k, topk,
-                        stream);
+  e = misa::launch_topk(c, q, scores, cache->L_cap, 0, nullptr, hist, !umma, list, list_cnt, k, topk, stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   return MISA_OK;
 }
@@ -294,7 +290,7 @@ misa_status misa_rerank_topk(const misa_cache *cache, const misa_queries *qs, co
     return misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, scores, k_prime, hist, stream);
   });
   if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
-  e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, hist, nullptr, nullptr, k, topk, stream);
+  e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, hist, true, nullptr, nullptr, k, topk, stream);
   if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
   return MISA_OK;
 }
@@ -329,7 +325,7 @@ misa_status misa_rerank_topk_noalloc(const misa_cache *cache, const misa_queries
     return misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, scores, k_prime, hist, stream);
   });
   if (e != cudaSuccess) return cuda_fail(e, who);
-  e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, hist, nullptr, nullptr, k, topk, stream);
+  e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, hist, true, nullptr, nullptr, k, topk, stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   return MISA_OK;
 }

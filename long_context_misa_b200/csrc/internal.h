@@ -48,17 +48,18 @@ cudaError_t launch_score_umma(const CacheView &c, const QueryView &q, const int3
 // outputs are token indices in ascending order, -1 padded.  Row length comes
 // from the query prefix (gather == nullptr), or the row holds n_cols
 // candidates whose tokens are gather[i][p] (entries < 0 or beyond the prefix
-// excluded).  row_hist is the histogram the scoring kernel built over exactly
-// the valid scores, or null: the selection then counts the row itself.  Prefix rows with few queries and long caches go through
-// a compact list of the elements at or above the histogram's boundary bin:
-// list_ws holds topk_list_entries() entries of 8 bytes and list_cnt n_q
-// counters, zeroed beforehand (both may be null: no list).
-constexpr int TOPK_LIST_MAX_ROWS = 64;   // rows served by the list path at most
-constexpr int TOPK_LIST_MIN_L = 16384;   // shorter caches never use it
+// excluded).  row_hist ([n_q][TOPK_HIST_BINS], zeroed beforehand) holds the
+// scoring kernel's histogram over exactly the valid scores when hist_ready;
+// otherwise it is filled here first.  Prefix rows of caches longer than
+// TOPK_LIST_MIN_L go through a compact list of the elements at or above the
+// histogram's boundary bin: list_ws holds topk_list_entries() entries of 8
+// bytes and list_cnt n_q counters, zeroed beforehand (both may be null: no
+// list; the selection then reads the rows itself).
+constexpr int TOPK_LIST_MIN_L = 16384;   // shorter caches never use the list
 constexpr int TOPK_LIST_EXTRA = 8192;    // boundary-bin elements listed per row beyond k
 size_t topk_list_entries(int n_q, int L_cap, int k);
 cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
-                        const int32_t *gather, const uint32_t *row_hist, void *list_ws, uint32_t *list_cnt, int k,
-                        int32_t *out, cudaStream_t s);
+                        const int32_t *gather, uint32_t *row_hist, bool hist_ready, void *list_ws,
+                        uint32_t *list_cnt, int k, int32_t *out, cudaStream_t s);
 
 }  // namespace misa

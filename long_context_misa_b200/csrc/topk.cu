@@ -324,25 +324,25 @@ __device__ __forceinline__ bool at_least(uint32_t kx, uint32_t lx, uint32_t P_hi
 // prefix and mask decided so far on the key and on the tie; need: elements
 // still to take among the in_bin that match the prefix.  With `small`, once
 // at most SEL_T elements match, their exact ranks finish the job.
-template <bool SMALL, class Visit>
-__device__ __forceinline__ void refine(SelShared &sh, uint32_t &P_hi, uint32_t &M_hi, uint32_t &P_lo,
+template <bool SMALL, int T = SEL_T, class Sh, class Visit>
+__device__ __forceinline__ void refine(Sh &sh, uint32_t &P_hi, uint32_t &M_hi, uint32_t &P_lo,
                                        uint32_t &M_lo, uint32_t need, uint32_t in_bin, Visit &&visit) {
   const int tid = threadIdx.x;
   bool done = in_bin == need;
   for (int p = 0; p < 4 && !done; ++p) {
-    if (SMALL && p > 0 && in_bin <= (uint32_t)SEL_T) {
+    if (SMALL && p > 0 && in_bin <= (uint32_t)T) {
       // the in_bin elements matching the prefix: rank each by counting
       visit([&](uint32_t kx, uint32_t lx, bool act) {
         if (act && (kx & M_hi) == P_hi && (lx & M_lo) == P_lo) {
           const uint32_t slot = atomicAdd(&sh.n_small, 1u);
-          if (slot < (uint32_t)SEL_T) {
+          if (slot < (uint32_t)T) {
             sh.small_key[slot] = kx;
             sh.small_tie[slot] = lx;
           }
         }
       });
       __syncthreads();
-      const int ns = min((int)sh.n_small, SEL_T);
+      const int ns = min((int)sh.n_small, T);
       if (tid < ns) {
         const uint32_t ki = sh.small_key[tid], li = sh.small_tie[tid];
         uint32_t rank = 0;
@@ -365,7 +365,7 @@ __device__ __forceinline__ void refine(SelShared &sh, uint32_t &P_hi, uint32_t &
     const bool lo_word = p >= 2;
     const int sft = kShift[p];
     const uint32_t dm = (1u << kWidth[p]) - 1u;
-    for (int b = tid; b < HPAD; b += SEL_T) sh.hist[b] = 0;
+    for (int b = tid; b < HPAD; b += T) sh.hist[b] = 0;
     __syncthreads();
     visit([&](uint32_t kx, uint32_t lx, bool act) {
       if (act && (kx & M_hi) == P_hi && (lx & M_lo) == P_lo)
@@ -389,6 +389,68 @@ __device__ __forceinline__ void refine(SelShared &sh, uint32_t &P_hi, uint32_t &
     }
     done = in_bin == need;
   }
+}
+
+// Ascending output of the marked tokens: thread t owns bitmap words
+// [t*per, t*per + per); the outputs are split evenly over the threads (each
+// finds the word holding its first output by a search over the owners'
+// offsets), then -1 padding up to k.
+// Staged output j lives at word j + j / 32: threads writing runs of outputs
+// 16 apart then hit distinct banks.
+__device__ __forceinline__ uint32_t spad(uint32_t j) { return j + (j >> 5); }
+
+template <int T = SEL_T>
+__device__ __forceinline__ void write_ascending(const uint32_t *bm, int words, int k, int32_t *orow, uint32_t *toff,
+                                                uint32_t *wa, uint32_t *wb, int32_t *stage, int stage_cap) {
+  const int tid = threadIdx.x;
+  const int per = cdiv(words, T);
+  const int w0 = min(tid * per, words), w1 = min(w0 + per, words);
+  uint32_t cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+  uint32_t n_sel;
+  toff[tid] = block_excl_scan<T>(cnt, &n_sel, wa, wb);
+  __syncthreads();
+  const uint32_t n_out = min(n_sel, (uint32_t)k);
+  const uint32_t cap = (uint32_t)stage_cap * 32 / 33;  // entries per chunk, padding included
+  for (uint32_t base = 0; base < n_out; base += cap) {
+    // outputs [base, base + chunk) are spread evenly over the threads, staged
+    // in shared memory, then written with coalesced stores
+    const uint32_t chunk = min(cap, n_out - base);
+    const uint32_t j0 = base + chunk * (uint32_t)tid / T, j1 = base + chunk * (uint32_t)(tid + 1) / T;
+    // each output is found inside the words of its owner thread (found by a
+    // binary search over the owners' offsets), so a run of empty words
+    // between clusters of selected tokens is jumped, never walked
+    uint32_t j = j0;
+    while (j < j1) {
+      int lo = 0, hi = T - 1;  // last owner whose offset is <= j
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (toff[mid] <= j) lo = mid;
+        else hi = mid - 1;
+      }
+      uint32_t r = j - toff[lo];
+      const int wend = min(lo * per + per, words);
+      for (int w = lo * per; w < wend && j < j1; ++w) {
+        uint32_t m = bm[w];
+        const uint32_t pc = __popc(m);
+        if (pc <= r) {
+          r -= pc;
+          continue;
+        }
+        for (; r > 0; --r) m &= m - 1;
+        while (m && j < j1) {
+          const int b = __ffs(m) - 1;
+          m &= m - 1;
+          stage[spad(j - base)] = w * 32 + b;
+          ++j;
+        }
+      }
+    }
+    __syncthreads();
+    for (uint32_t j = tid; j < chunk; j += T) orow[base + j] = stage[spad(j)];
+    __syncthreads();
+  }
+  for (int p = (int)n_out + tid; p < k; p += T) orow[p] = -1;
 }
 
 template <bool GATHER, bool FROM_LIST, bool OWN_HIST>
@@ -423,7 +485,10 @@ __global__ void __launch_bounds__(SEL_T) select_kernel(CacheView c, QueryView qv
   const int n = GATHER ? n_cols : Li;
   const int words = cdiv(Li, 32);
   Boundary bd;
-  if (!OWN_HIST) bd = warp_boundary(row_hist + (size_t)row * RB, k);
+  if (!OWN_HIST && warp == 0) {  // one warp: every warp reading 8 KB would cost 16x the wavefronts
+    const Boundary b = warp_boundary(row_hist + (size_t)row * RB, k);
+    if (lane == 0) sh.bd = b;
+  }
   if (tid == 0) sh.n_small = 0;
   for (int w = tid; w < words; w += SEL_T) bm[w] = 0;
   if (OWN_HIST) {
@@ -437,9 +502,13 @@ __global__ void __launch_bounds__(SEL_T) select_kernel(CacheView c, QueryView qv
                              if (ok[u]) atomicAdd(&sh.hist[hpos(key[u] >> HIST_SHIFT)], 1u);
                          });
     __syncthreads();
-    bd = warp_boundary_smem(sh.hist, k);
+    if (warp == 0) {
+      const Boundary b = warp_boundary_smem(sh.hist, k);
+      if (lane == 0) sh.bd = b;
+    }
   }
   __syncthreads();
+  bd = sh.bd;
 
   if (bd.kk > 0) {
     const uint32_t d0 = bd.d0;
@@ -542,42 +611,8 @@ __global__ void __launch_bounds__(SEL_T) select_kernel(CacheView c, QueryView qv
     }
   }
 
-  // 4. ascending output.  Thread t owns bitmap words [t*per, t*per + per);
-  //    the outputs are split evenly over the threads (each finds the word
-  //    holding its first output by a search over the owners' offsets).
-  const int per = cdiv(words, SEL_T);
-  {
-    const int w0 = min(tid * per, words), w1 = min(w0 + per, words);
-    uint32_t cnt = 0;
-    for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
-    uint32_t n_sel;
-    sh.toff[tid] = block_excl_scan<SEL_T>(cnt, &n_sel, sh.wa, sh.wb);
-    __syncthreads();
-    const uint32_t j0 = n_sel * (uint32_t)tid / SEL_T, j1 = n_sel * (uint32_t)(tid + 1) / SEL_T;
-    if (j0 < j1) {
-      int lo = 0, hi = SEL_T - 1;  // last owner whose offset is <= j0
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (sh.toff[mid] <= j0) lo = mid;
-        else hi = mid - 1;
-      }
-      uint32_t r = j0 - sh.toff[lo];
-      int w = lo * per;
-      uint32_t m = bm[w];
-      while ((uint32_t)__popc(m) <= r) {
-        r -= __popc(m);
-        m = bm[++w];
-      }
-      for (; r > 0; --r) m &= m - 1;
-      for (uint32_t j = j0; j < j1; ++j) {
-        while (m == 0) m = bm[++w];
-        const int b = __ffs(m) - 1;
-        m &= m - 1;
-        if (j < (uint32_t)k) orow[j] = w * 32 + b;
-      }
-    }
-    for (int p = (int)n_sel + tid; p < k; p += SEL_T) orow[p] = -1;
-  }
+  // 4. ascending output, staged in the candidate list's space
+  write_ascending(bm, words, k, orow, sh.toff, sh.wa, sh.wb, reinterpret_cast<int32_t *>(sh.cand_key), 2 * CAP);
 }
 
 // Few long prefix rows: every CTA takes a chunk of one row and appends the
@@ -604,7 +639,15 @@ __global__ void __launch_bounds__(FILT_T) filter_kernel(CacheView c, QueryView q
   const int Li = query_prefix(c, qv, row, &s);
   if (p0 >= Li) return;  // uniform over the CTA
   const int p1 = min(Li, pl);
-  const Boundary bd = warp_boundary(row_hist + (size_t)row * RB, k);  // every warp
+  // one warp finds the boundary (every warp reading the 8 KB histogram would
+  // multiply the L2 traffic by the warps of all CTAs)
+  __shared__ Boundary sbd;
+  if (threadIdx.x < 32) {
+    const Boundary b = warp_boundary(row_hist + (size_t)row * RB, k);
+    if (threadIdx.x == 0) sbd = b;
+  }
+  __syncthreads();
+  const Boundary bd = sbd;
   if (!bd.listable()) return;  // uniform
   uint2 *lrow = list + (size_t)row * list_cap;
   for (int base = p0; base < p1; base += FILT_T * FU) {
@@ -644,6 +687,323 @@ __global__ void __launch_bounds__(FILT_T) filter_kernel(CacheView c, QueryView q
   }
 }
 
+// Row histograms when the scoring kernel built none (tensor-core prefill):
+// every CTA counts the top 11 key bits of a chunk of one row in shared memory
+// and adds its non-zero bins to row_hist (zeroed beforehand).
+constexpr int HIST_T = 256;
+__global__ void __launch_bounds__(HIST_T) hist_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
+                                                      uint32_t *row_hist, int chunk) {
+  constexpr int HU = 16;
+  __shared__ uint32_t hs[RB];
+  const int row = blockIdx.y;
+  const int p0 = blockIdx.x * chunk;
+  const int pl = min(c.L_cap, p0 + chunk);
+  const float *srow = scores + (size_t)row * ld;
+  float v[HU];
+#pragma unroll
+  for (int u = 0; u < HU; ++u) {
+    const int p = p0 + u * HIST_T + threadIdx.x;
+    v[u] = p < pl ? __ldg(srow + p) : 0.f;
+  }
+  int s;
+  const int Li = query_prefix(c, qv, row, &s);
+  if (p0 >= Li) return;  // uniform over the CTA
+  const int p1 = min(Li, pl);
+  for (int b = threadIdx.x; b < RB; b += HIST_T) hs[b] = 0;
+  __syncthreads();
+  for (int base = p0; base < p1; base += HIST_T * HU) {
+    if (base != p0) {
+#pragma unroll
+      for (int u = 0; u < HU; ++u) {
+        const int p = base + u * HIST_T + threadIdx.x;
+        v[u] = p < p1 ? __ldg(srow + p) : 0.f;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < HU; ++u)
+      if (base + u * HIST_T + (int)threadIdx.x < p1) atomicAdd(&hs[ordered_key(v[u]) >> HIST_SHIFT], 1u);
+  }
+  __syncthreads();
+  uint32_t *rh = row_hist + (size_t)row * RB;
+  for (int b = threadIdx.x; b < RB; b += HIST_T)
+    if (hs[b]) atomicAdd(rh + b, hs[b]);
+}
+
+// ---------------------------------------------------------------------------
+// One-round-trip selection for rows whose data fits in shared memory: the
+// re-rank rows (scores and candidate tokens) and the filter kernel's lists.
+// One thread brings the row's histogram and data into shared memory with
+// bulk copies on one mbarrier; every later phase works on shared memory only.
+// A list row the filter could not serve falls back to sweeps of the global
+// row.
+// ---------------------------------------------------------------------------
+constexpr int FAST_T = 1024;              // threads of the staged selection
+constexpr int FAST_W = FAST_T / 32;
+constexpr int FAST_DATA_MAX = 128 * 1024;  // bytes of row data staged in shared memory
+
+struct FastShared {
+  alignas(16) uint32_t rhist[RB];  // the row histogram (bulk copy)
+  Boundary bd;
+  uint64_t bar;
+  uint4 res;
+  uint32_t thr[2];
+  uint32_t n_small;
+  int ok;
+  uint32_t wa[FAST_W], wb[FAST_W + 1];
+  uint32_t toff[FAST_T];
+  uint32_t hist[HPAD];
+  uint32_t small_key[FAST_T], small_tie[FAST_T];
+  uint32_t n_d0;
+};
+constexpr int D0CAP = 6144;  // boundary-bin elements compacted in shared memory
+
+// One whole warp: boundary from the unpadded histogram in shared memory.
+__device__ __forceinline__ Boundary warp_boundary_plain_smem(const uint32_t *h, int k) {
+  const int lane = threadIdx.x & 31;
+  uint32_t s = 0;
+  // lane l sums bins [64 l, 64 l + 64) starting at a rotated offset, so the
+  // lanes of each load hit 32 distinct banks
+#pragma unroll 16
+  for (int j = 0; j < 64; ++j) s += h[lane * 64 + ((j + lane) & 63)];
+  uint32_t suf = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += v;
+  }
+  Boundary b;
+  b.total = __shfl_sync(0xffffffffu, suf, 0);
+  b.kk = min((uint32_t)k, b.total);
+  b.all_in = (uint32_t)k >= b.total;
+  b.d0 = 0;
+  b.above = 0;
+  b.in0 = 0;
+  if (b.all_in) return b;
+  const uint32_t want = b.kk;
+  const uint32_t above_l = suf - s;
+  const int owner = __ffs(__ballot_sync(0xffffffffu, above_l < want && suf >= want)) - 1;
+  const uint32_t base_above = __shfl_sync(0xffffffffu, above_l, owner);
+  const int b0 = owner * 64 + 2 * lane;
+  const uint2 cc = *reinterpret_cast<const uint2 *>(h + b0);
+  const uint32_t pair = cc.x + cc.y;
+  uint32_t psuf = pair;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_down_sync(0xffffffffu, psuf, o);
+    if (lane + o < 32) psuf += v;
+  }
+  const uint32_t a1 = base_above + psuf - pair;
+  const bool hit1 = a1 < want && a1 + cc.y >= want;
+  const bool hit0 = a1 + cc.y < want && a1 + pair >= want;
+  const int src = __ffs(__ballot_sync(0xffffffffu, hit1 || hit0)) - 1;
+  b.d0 = __shfl_sync(0xffffffffu, hit1 ? b0 + 1 : b0, src);
+  b.above = __shfl_sync(0xffffffffu, hit1 ? a1 : a1 + cc.y, src);
+  b.in0 = __shfl_sync(0xffffffffu, hit1 ? cc.y : cc.x, src);
+  return b;
+}
+
+// LIST: the filter kernel's list (key, token) of the row; else GATHER rows
+// (scores and candidate tokens, n_cols of each).
+template <bool LIST>
+__global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryView qv, const float *scores,
+                                                            long long ld, int n_cols, const int32_t *gather,
+                                                            const uint32_t *row_hist, const uint2 *list,
+                                                            const uint32_t *list_cnt, int list_cap, int k,
+                                                            int32_t *out) {
+  extern __shared__ __align__(16) uint8_t fs_smem[];
+  FastShared &sh = *reinterpret_cast<FastShared *>(fs_smem);
+  uint8_t *data = fs_smem + sizeof(FastShared);  // 16-byte aligned (sizeof is a multiple of 16)
+  const int data_bytes = LIST ? list_cap * 8 : n_cols * 8;
+  uint32_t *bm = reinterpret_cast<uint32_t *>(data + data_bytes);
+  uint32_t *d0_key = bm + cdiv(c.L_cap, 32);                              // [D0CAP]
+  uint32_t *d0_tie = d0_key + D0CAP;                                       // [D0CAP]
+  const uint2 *ent = reinterpret_cast<const uint2 *>(data);                // LIST
+  const float *sc = reinterpret_cast<const float *>(data);                 // GATHER
+  const int32_t *tk = reinterpret_cast<const int32_t *>(data + n_cols * 4);  // GATHER
+  const int row = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5;
+
+  if (tid == 0) {
+    mbar_init(&sh.bar, 1);
+    fence_mbar_init();
+    const uint32_t bytes = RB * 4 + (LIST ? list_cap * 8 : n_cols * 8);
+    mbar_arrive_expect_tx(&sh.bar, bytes);
+    bulk_g2s(sh.rhist, row_hist + (size_t)row * RB, RB * 4, &sh.bar);
+    if (LIST) {
+      bulk_g2s(data, list + (size_t)row * list_cap, list_cap * 8, &sh.bar);
+    } else {
+      bulk_g2s(data, scores + (size_t)row * ld, n_cols * 4, &sh.bar);
+      bulk_g2s(data + n_cols * 4, gather + (size_t)row * n_cols, n_cols * 4, &sh.bar);
+    }
+    sh.n_small = 0;
+    sh.n_d0 = 0;
+  }
+  const int lcnt = LIST ? min((int)list_cnt[row], list_cap) : 0;
+  int s;
+  const int Li = query_prefix(c, qv, row, &s);
+  const int words = cdiv(Li, 32);
+  for (int w = tid; w < words; w += FAST_T) bm[w] = 0;
+  __syncthreads();  // barrier initialised, bitmap clear
+  {
+    const bool got = mbar_wait(&sh.bar, 0);
+    if (!got) flag(c, MISA_DEV_WAIT_TIMEOUT);
+    if (tid == 0) sh.ok = got;
+  }
+  __syncthreads();
+  int32_t *orow = out + (size_t)row * k;
+  if (!sh.ok) {  // uniform: give up on this row (flagged above)
+    for (int p = tid; p < k; p += FAST_T) orow[p] = -1;
+    return;
+  }
+  if (warp == 0) {
+    const Boundary b = warp_boundary_plain_smem(sh.rhist, k);
+    if ((tid & 31) == 0) sh.bd = b;
+  }
+  __syncthreads();
+  const Boundary bd = sh.bd;
+  const float *srow = scores + (size_t)row * ld;
+
+  if (bd.kk > 0) {
+    const uint32_t d0 = bd.d0;
+    const uint32_t need = bd.need();
+    const bool whole = bd.all_in || need == bd.in0;
+    // staged elements: (key, token, valid); a list row the filter skipped is
+    // read from the global row instead (prefix rows: token = position)
+    const bool staged = !LIST || bd.listable();
+    auto each = [&](auto &&fn) {
+      if (staged) {
+        const int n = LIST ? lcnt : n_cols;
+        for (int i = tid; i < n; i += FAST_T) {
+          if (LIST) {
+            const uint2 e = ent[i];
+            fn(e.x, (int)e.y, true);
+          } else {
+            const int t = tk[i];
+            fn(ordered_key(sc[i]), t, t >= 0 && t < Li);
+          }
+        }
+      } else {
+        for (int i = tid; i < Li; i += FAST_T) fn(ordered_key(__ldg(srow + i)), i, true);
+      }
+    };
+    const bool compact = staged && !whole && bd.in0 <= (uint32_t)D0CAP;
+    if (compact) {
+      // 2. one pass, four elements per thread and step: mark everything above
+      //    the boundary; compact the boundary bin's elements (key, tie) with
+      //    one shared atomic per warp and step
+      const int n = LIST ? lcnt : n_cols;
+      const int lane = tid & 31;
+      const uint32_t lt = lanemask_lt();
+      for (int base = 0; base < n; base += FAST_T * 4) {
+        const int i0 = base + tid * 4;
+        uint32_t key[4];
+        int t[4];
+        bool v[4];
+        if (LIST) {
+          const uint4 *e4 = reinterpret_cast<const uint4 *>(ent + i0);
+          const uint4 a = i0 < n ? e4[0] : make_uint4(0u, 0u, 0u, 0u);
+          const uint4 b = i0 + 2 < n ? e4[1] : make_uint4(0u, 0u, 0u, 0u);
+          key[0] = a.x; t[0] = (int)a.y; key[1] = a.z; t[1] = (int)a.w;
+          key[2] = b.x; t[2] = (int)b.y; key[3] = b.z; t[3] = (int)b.w;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) v[e] = i0 + e < n;
+        } else {
+          const float4 f = i0 < n ? reinterpret_cast<const float4 *>(sc)[i0 >> 2] : make_float4(0.f, 0.f, 0.f, 0.f);
+          const int4 q = i0 < n ? reinterpret_cast<const int4 *>(tk)[i0 >> 2] : make_int4(-1, -1, -1, -1);
+          key[0] = ordered_key(f.x); key[1] = ordered_key(f.y); key[2] = ordered_key(f.z); key[3] = ordered_key(f.w);
+          t[0] = q.x; t[1] = q.y; t[2] = q.z; t[3] = q.w;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) v[e] = t[e] >= 0 && t[e] < Li;
+        }
+        uint32_t flags = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t bin = key[e] >> HIST_SHIFT;
+          if (v[e] && bin > d0) mark(bm, t[e]);
+          flags |= (uint32_t)(v[e] && bin == d0) << e;
+        }
+        const uint32_t cnt = __popc(flags);
+        uint32_t inc = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t u = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += u;
+        }
+        const uint32_t tot = __shfl_sync(0xffffffffu, inc, 31);
+        if (tot) {
+          uint32_t slot = 0;
+          if (lane == 31) slot = atomicAdd(&sh.n_d0, tot);
+          slot = __shfl_sync(0xffffffffu, slot, 31) + inc - cnt;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if ((flags >> e) & 1) {
+              if (slot < (uint32_t)D0CAP) {
+                d0_key[slot] = key[e];
+                d0_tie[slot] = POS_MAX - (uint32_t)t[e];
+              }
+              ++slot;
+            }
+        }
+        (void)lt;
+      }
+      __syncthreads();
+      // 3. threshold among the boundary bin's elements only, then their winners
+      const int nd = min((int)sh.n_d0, D0CAP);
+      uint32_t P_hi = d0 << HIST_SHIFT, M_hi = TOP_MASK, P_lo = 0, M_lo = 0;
+      refine<true, FAST_T>(sh, P_hi, M_hi, P_lo, M_lo, need, bd.in0, [&](auto &&fn) {
+        for (int x = tid; x < nd; x += FAST_T) fn(d0_key[x], d0_tie[x], true);
+      });
+      for (int x = tid; x < nd; x += FAST_T)
+        if (at_least(d0_key[x], d0_tie[x], P_hi, M_hi, P_lo, M_lo)) mark(bm, (int)(POS_MAX - d0_tie[x]));
+      __syncthreads();
+    } else {
+    // 2. everything above the boundary (and the boundary bin when whole)
+    each([&](uint32_t kx, int t, bool v) {
+      const uint32_t bin = kx >> HIST_SHIFT;
+      if (v && (bd.all_in || bin > d0 || (whole && bin == d0))) mark(bm, t);
+    });
+    __syncthreads();
+    if (!whole) {
+      // 3. threshold inside d0, then its winners
+      uint32_t P_hi = d0 << HIST_SHIFT, M_hi = TOP_MASK, P_lo = 0, M_lo = 0;
+      refine<true, FAST_T>(sh, P_hi, M_hi, P_lo, M_lo, need, bd.in0, [&](auto &&fn) {
+        each([&](uint32_t kx, int t, bool v) { fn(kx, POS_MAX - (uint32_t)t, v); });
+      });
+      each([&](uint32_t kx, int t, bool v) {
+        if (v && (kx >> HIST_SHIFT) == d0 && at_least(kx, POS_MAX - (uint32_t)t, P_hi, M_hi, P_lo, M_lo)) mark(bm, t);
+      });
+      __syncthreads();
+    }
+    }
+  }
+  // 4. ascending output, staged in the row data's space (no longer read)
+  write_ascending<FAST_T>(bm, words, k, orow, sh.toff, sh.wa, sh.wb, reinterpret_cast<int32_t *>(data),
+                  data_bytes / 4);
+}
+
+constexpr int SMEM_OPTIN_MAX = 227 * 1024;  // largest dynamic shared memory a CTA may opt into
+
+int fast_smem_bytes(bool list, int n_cols, int list_cap, int L_cap) {
+  return (int)sizeof(FastShared) + (list ? list_cap * 8 : n_cols * 8) + 4 * cdiv(L_cap, 32) + 8 * D0CAP;
+}
+
+template <bool LIST>
+cudaError_t launch_select_smem(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
+                               const int32_t *gather, const uint32_t *row_hist, const uint2 *list,
+                               const uint32_t *list_cnt, int list_cap, int k, int32_t *out, cudaStream_t s) {
+  constexpr int SMEM_MAX = SMEM_OPTIN_MAX;
+  struct Tag {};
+  const int st = cached_per_device<Tag>([] {
+    return 1 + (int)cudaFuncSetAttribute(select_smem_kernel<LIST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM_MAX);
+  });
+  if (st != 1) return (cudaError_t)(st - 1);
+  const int smem = fast_smem_bytes(LIST, n_cols, list_cap, c.L_cap);
+  select_smem_kernel<LIST><<<q.n_q, FAST_T, smem, s>>>(c, q, scores, ld, n_cols, gather, row_hist, list, list_cnt,
+                                                      list_cap, k, out);
+  return cudaGetLastError();
+}
+
 int sel_smem_bytes(int L_cap) { return (int)sizeof(SelShared) + 4 * cdiv(L_cap, 32); }
 constexpr int SEL_SMEM_MAX = (int)sizeof(SelShared) + 4 * (MISA_MAX_L / 32);
 
@@ -667,30 +1027,49 @@ cudaError_t launch_select(const CacheView &c, const QueryView &q, const float *s
 }  // namespace
 
 size_t topk_list_entries(int n_q, int L_cap, int k) {
-  if (n_q < 1 || n_q > TOPK_LIST_MAX_ROWS || L_cap <= TOPK_LIST_MIN_L || k < 1) return 0;
+  if (n_q < 1 || L_cap <= TOPK_LIST_MIN_L || k < 1) return 0;
   return (size_t)n_q * ((size_t)k + TOPK_LIST_EXTRA);
 }
 
 cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
-                        const int32_t *gather, const uint32_t *row_hist, void *list_ws, uint32_t *list_cnt, int k,
-                        int32_t *out, cudaStream_t s) {
+                        const int32_t *gather, uint32_t *row_hist, bool hist_ready, void *list_ws,
+                        uint32_t *list_cnt, int k, int32_t *out, cudaStream_t s) {
   if (q.n_q == 0) return cudaSuccess;
-  if (gather)
+  auto aligned16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (gather) {
+    // rows staged whole in shared memory when they fit and the copies stay
+    // 16-byte aligned; otherwise swept from global memory
+    if (hist_ready && n_cols % 4 == 0 && ld % 4 == 0 && 8LL * n_cols <= FAST_DATA_MAX && aligned16(scores) &&
+        aligned16(gather) && aligned16(row_hist) && fast_smem_bytes(false, n_cols, 0, c.L_cap) <= SMEM_OPTIN_MAX)
+      return launch_select_smem<false>(c, q, scores, ld, n_cols, gather, row_hist, nullptr, nullptr, 0, k, out, s);
     return launch_select<true, false>(c, q, scores, ld, n_cols, gather, row_hist, nullptr, nullptr, 0, k, out, s);
-  if (!row_hist)
+  }
+  const bool list_mode = topk_list_entries(q.n_q, c.L_cap, k) != 0 && list_ws && list_cnt && row_hist;
+  if (!hist_ready && !list_mode)
     return launch_select<false, false, true>(c, q, scores, ld, 0, nullptr, nullptr, nullptr, nullptr, 0, k, out, s);
-  if (topk_list_entries(q.n_q, c.L_cap, k) == 0 || !list_ws || !list_cnt)
+  const int sms = device_sms();
+  cudaError_t e = cudaSuccess;
+  if (!hist_ready) {
+    // wide pass over the scores: about 16K elements per CTA
+    const int per_row = cdiv(c.L_cap, 16384);
+    const int chunk = cdiv(cdiv(c.L_cap, per_row), HIST_T) * HIST_T;
+    hist_kernel<<<dim3(cdiv(c.L_cap, chunk), q.n_q), HIST_T, 0, s>>>(c, q, scores, ld, row_hist, chunk);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (!list_mode)
     return launch_select<false, false>(c, q, scores, ld, 0, nullptr, row_hist, nullptr, nullptr, 0, k, out, s);
   const int list_cap = k + TOPK_LIST_EXTRA;
   uint2 *list = static_cast<uint2 *>(list_ws);
-  // about two CTAs per SM over all rows, at least 4096 elements each
-  const int sms = device_sms();
-  const int per_row = max(1, min(cdiv(c.L_cap, 4096), 2 * sms / q.n_q));
+  // about two CTAs per SM over all rows (few rows) or at most 16K elements
+  // per CTA (many rows), at least 4096 elements each
+  const int per_row = max(1, min(cdiv(c.L_cap, 4096), max(2 * sms / q.n_q, cdiv(c.L_cap, 16384))));
   const int chunk = cdiv(cdiv(c.L_cap, per_row), FILT_T) * FILT_T;
   filter_kernel<<<dim3(cdiv(c.L_cap, chunk), q.n_q), FILT_T, 0, s>>>(c, q, scores, ld, row_hist, list, list_cnt,
                                                                      list_cap, k, chunk);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (8LL * list_cap <= FAST_DATA_MAX && list_cap % 2 == 0 && aligned16(list) && aligned16(row_hist) &&
+      fast_smem_bytes(true, 0, list_cap, c.L_cap) <= SMEM_OPTIN_MAX)
+    return launch_select_smem<true>(c, q, scores, ld, 0, nullptr, row_hist, list, list_cnt, list_cap, k, out, s);
   return launch_select<false, true>(c, q, scores, ld, 0, nullptr, row_hist, list, list_cnt, list_cap, k, out, s);
 }
 
