@@ -77,7 +77,8 @@ typedef enum {
   MISA_OP_ROUTE = 0,        /* misa_route_heads */
   MISA_OP_SCORE_TOPK = 1,   /* misa_score_topk */
   MISA_OP_DENSE_TOPK = 2,   /* dsa_dense_score_topk */
-  MISA_OP_RERANK_TOPK = 3   /* misa_rerank_topk */
+  MISA_OP_RERANK_TOPK = 3,  /* misa_rerank_topk */
+  MISA_OP_DAGGER_TOPK = 4   /* misa_dagger_topk */
 } misa_op;
 
 /* Bits OR-ed into misa_cache.status by the device. */
@@ -211,6 +212,22 @@ MISA_API misa_status misa_rerank_topk(const misa_cache *cache, const misa_querie
                              const int32_t *cand, int32_t k_prime, int32_t k,
                              int32_t *topk, float *scores_out,
                              void *ws, size_t ws_bytes, misa_stream stream);
+
+/*
+ * MISA-dagger in one call ("Hierarchical variant": the routed pass keeps the
+ * top-k' candidates, the original DSA indexer with all H_I heads re-scores
+ * only those and keeps the final top-k).  Same result as misa_score_topk
+ * with k = k_prime followed by misa_rerank_topk on its output, without the
+ * intermediate ascending ordering of the k' candidates.
+ *   heads [n_q][h] int32 in [0, H) (from misa_route_heads)
+ *   topk  [n_q][k] int32 out (ascending token indices, -1 padded)
+ * Workspace: misa_workspace_bytes(MISA_OP_DAGGER_TOPK, ..., h, k, k_prime).
+ * Errors: MISA_ERR_INVALID for h outside [1, H], 1 <= k <= k_prime violated
+ * or NULL pointers; MISA_ERR_UNSUPPORTED for k_prime above MISA_MAX_L.
+ */
+MISA_API misa_status misa_dagger_topk(const misa_cache *cache, const misa_queries *qs,
+                                      const int32_t *heads, int32_t h, int32_t k_prime, int32_t k,
+                                      int32_t *topk, void *ws, size_t ws_bytes, misa_stream stream);
 
 /*
  * misa_rerank_topk without a caller workspace and without any allocation.

@@ -125,6 +125,13 @@ size_t ws_score(const misa_cache *c, const misa_queries *q) {
   return round_up(sizeof(float) * (size_t)q->n_q * c->L_cap);
 }
 
+// Workspace of misa_dagger_topk: [histograms + list counters][routed scores]
+// [top-k' list][candidates n_q x k'][re-rank scores n_q x k'].
+size_t ws_dagger(const misa_cache *c, const misa_queries *q, int k_prime) {
+  const size_t cand = round_up(sizeof(int32_t) * (size_t)q->n_q * k_prime);
+  return ws_hist(q) + ws_score(c, q) + ws_list(c, q, k_prime) + 2 * cand;
+}
+
 misa_status check_ws(void *ws, size_t have, size_t need) {
   if (have < need) return fail(MISA_ERR_WORKSPACE, "workspace %zu bytes, need %zu", have, need);
   if (need > 0 && (!ws || !aligned16(ws))) return fail(MISA_ERR_INVALID, "workspace NULL or not 16-byte aligned");
@@ -218,6 +225,8 @@ size_t misa_workspace_bytes(int32_t op, const misa_cache *cache, const misa_quer
       return ws_hist(qs) + ws_score(cache, qs) + (k > 0 ? ws_list(cache, qs, k) : 0);
     case MISA_OP_RERANK_TOPK:
       return k_prime > 0 ? ws_hist(qs) + round_up(sizeof(float) * (size_t)qs->n_q * k_prime) : 0;
+    case MISA_OP_DAGGER_TOPK:
+      return k_prime > 0 ? ws_dagger(cache, qs, k_prime) : 0;
     default:
       return 0;
   }
@@ -326,6 +335,52 @@ misa_status misa_rerank_topk_noalloc(const misa_cache *cache, const misa_queries
   });
   if (e != cudaSuccess) return cuda_fail(e, who);
   e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, hist, true, nullptr, nullptr, k, topk, stream);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  return MISA_OK;
+}
+
+misa_status misa_dagger_topk(const misa_cache *cache, const misa_queries *qs, const int32_t *heads, int32_t h,
+                             int32_t k_prime, int32_t k, int32_t *topk, void *ws, size_t ws_bytes,
+                             misa_stream stream) {
+  const char *who = "misa_dagger_topk";
+  misa_status st = check_cache(cache, false);
+  if (st != MISA_OK) return st;
+  if ((st = check_queries(qs)) != MISA_OK) return st;
+  if (h < 1 || h > qs->H) return fail(MISA_ERR_INVALID, "h=%d outside [1, H=%d]", h, qs->H);
+  if (k < 1 || k_prime < k) return fail(MISA_ERR_INVALID, "need 1 <= k=%d <= k_prime=%d", k, k_prime);
+  if (k_prime > MISA_MAX_L) return fail(MISA_ERR_UNSUPPORTED, "k_prime=%d above %d", k_prime, MISA_MAX_L);
+  if (qs->n_q > 0 && (!heads || !topk)) return fail(MISA_ERR_INVALID, "heads/topk is NULL");
+  if ((st = check_ws(ws, ws_bytes, ws_dagger(cache, qs, k_prime))) != MISA_OK) return st;
+  if (injected_failure(who, &st)) return st;
+  if (qs->n_q == 0) return MISA_OK;
+  misa::CacheView c = view(cache);
+  misa::QueryView q = view(qs);
+  uint8_t *w8 = static_cast<uint8_t *>(ws);
+  uint32_t *hist = reinterpret_cast<uint32_t *>(w8);
+  uint32_t *list_cnt = hist + (size_t)qs->n_q * misa::TOPK_HIST_BINS;
+  float *scores = reinterpret_cast<float *>(w8 + ws_hist(qs));
+  void *list = w8 + ws_hist(qs) + ws_score(cache, qs);
+  int32_t *cand = reinterpret_cast<int32_t *>(w8 + ws_hist(qs) + ws_score(cache, qs) + ws_list(cache, qs, k_prime));
+  float *rscores = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(cand) +
+                                             round_up(sizeof(int32_t) * (size_t)qs->n_q * k_prime));
+  // routed pass: scores, then the k' candidates in any order
+  const bool umma = misa::umma_applies(c, q, heads, h);
+  cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * hist_words(qs), stream);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  e = timed_scoring(stream, [&] {
+    return umma ? misa::launch_score_umma(c, q, heads, h, scores, cache->L_cap, stream)
+                : misa::launch_score_mma(c, q, heads, h, nullptr, 0, scores, cache->L_cap, hist, stream);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  e = misa::launch_topk(c, q, scores, cache->L_cap, 0, nullptr, hist, !umma, list, list_cnt, k_prime, cand, stream,
+                        false);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  // fine pass: every head on the candidates, ascending final top-k
+  e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  e = misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, rscores, k_prime, hist, stream);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  e = misa::launch_topk(c, q, rscores, k_prime, k_prime, cand, hist, true, nullptr, nullptr, k, topk, stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   return MISA_OK;
 }

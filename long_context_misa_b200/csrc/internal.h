@@ -54,12 +54,13 @@ cudaError_t launch_score_umma(const CacheView &c, const QueryView &q, const int3
 // TOPK_LIST_MIN_L go through a compact list of the elements at or above the
 // histogram's boundary bin: list_ws holds topk_list_entries() entries of 8
 // bytes and list_cnt n_q counters, zeroed beforehand (both may be null: no
-// list; the selection then reads the rows itself).
+// list; the selection then reads the rows itself).  ordered == false allows
+// the selected tokens of a row in any order (followed by -1 padding).
 constexpr int TOPK_LIST_MIN_L = 16384;   // shorter caches never use the list
 constexpr int TOPK_LIST_EXTRA = 8192;    // boundary-bin elements listed per row beyond k
 size_t topk_list_entries(int n_q, int L_cap, int k);
 cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
                         const int32_t *gather, uint32_t *row_hist, bool hist_ready, void *list_ws,
-                        uint32_t *list_cnt, int k, int32_t *out, cudaStream_t s);
+                        uint32_t *list_cnt, int k, int32_t *out, cudaStream_t s, bool ordered = true);
 
 }  // namespace misa

@@ -754,6 +754,7 @@ struct FastShared {
   uint32_t hist[HPAD];
   uint32_t small_key[FAST_T], small_tie[FAST_T];
   uint32_t n_d0;
+  uint32_t n_out;
 };
 constexpr int D0CAP = 6144;  // boundary-bin elements compacted in shared memory
 
@@ -804,7 +805,7 @@ __device__ __forceinline__ Boundary warp_boundary_plain_smem(const uint32_t *h, 
 
 // LIST: the filter kernel's list (key, token) of the row; else GATHER rows
 // (scores and candidate tokens, n_cols of each).
-template <bool LIST>
+template <bool LIST, bool ORDERED>
 __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryView qv, const float *scores,
                                                             long long ld, int n_cols, const int32_t *gather,
                                                             const uint32_t *row_hist, const uint2 *list,
@@ -837,6 +838,7 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
     }
     sh.n_small = 0;
     sh.n_d0 = 0;
+    sh.n_out = 0;
   }
   const int lcnt = LIST ? min((int)list_cnt[row], list_cap) : 0;
   int s;
@@ -851,6 +853,20 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
   }
   __syncthreads();
   int32_t *orow = out + (size_t)row * k;
+  // a winner: marked in the token bitmap (ascending output), or appended to
+  // the output at once (any order; one shared atomic per group of lanes)
+  auto emit = [&](int tok) {
+    if (ORDERED) {
+      mark(bm, tok);
+    } else {
+      const unsigned m = __activemask();
+      const int lane = tid & 31, leader = __ffs(m) - 1;
+      uint32_t base = 0;
+      if (lane == leader) base = atomicAdd(&sh.n_out, (uint32_t)__popc(m));
+      base = __shfl_sync(m, base, leader) + __popc(m & lanemask_lt());
+      if (base < (uint32_t)k) orow[base] = tok;
+    }
+  };
   if (!sh.ok) {  // uniform: give up on this row (flagged above)
     for (int p = tid; p < k; p += FAST_T) orow[p] = -1;
     return;
@@ -919,7 +935,7 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const uint32_t bin = key[e] >> HIST_SHIFT;
-          if (v[e] && bin > d0) mark(bm, t[e]);
+          if (v[e] && bin > d0) emit(t[e]);
           flags |= (uint32_t)(v[e] && bin == d0) << e;
         }
         const uint32_t cnt = __popc(flags);
@@ -954,13 +970,13 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
         for (int x = tid; x < nd; x += FAST_T) fn(d0_key[x], d0_tie[x], true);
       });
       for (int x = tid; x < nd; x += FAST_T)
-        if (at_least(d0_key[x], d0_tie[x], P_hi, M_hi, P_lo, M_lo)) mark(bm, (int)(POS_MAX - d0_tie[x]));
+        if (at_least(d0_key[x], d0_tie[x], P_hi, M_hi, P_lo, M_lo)) emit((int)(POS_MAX - d0_tie[x]));
       __syncthreads();
     } else {
     // 2. everything above the boundary (and the boundary bin when whole)
     each([&](uint32_t kx, int t, bool v) {
       const uint32_t bin = kx >> HIST_SHIFT;
-      if (v && (bd.all_in || bin > d0 || (whole && bin == d0))) mark(bm, t);
+      if (v && (bd.all_in || bin > d0 || (whole && bin == d0))) emit(t);
     });
     __syncthreads();
     if (!whole) {
@@ -970,15 +986,20 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
         each([&](uint32_t kx, int t, bool v) { fn(kx, POS_MAX - (uint32_t)t, v); });
       });
       each([&](uint32_t kx, int t, bool v) {
-        if (v && (kx >> HIST_SHIFT) == d0 && at_least(kx, POS_MAX - (uint32_t)t, P_hi, M_hi, P_lo, M_lo)) mark(bm, t);
+        if (v && (kx >> HIST_SHIFT) == d0 && at_least(kx, POS_MAX - (uint32_t)t, P_hi, M_hi, P_lo, M_lo)) emit(t);
       });
       __syncthreads();
     }
     }
   }
-  // 4. ascending output, staged in the row data's space (no longer read)
-  write_ascending<FAST_T>(bm, words, k, orow, sh.toff, sh.wa, sh.wb, reinterpret_cast<int32_t *>(data),
-                  data_bytes / 4);
+  // 4. output
+  if (ORDERED) {
+    write_ascending<FAST_T>(bm, words, k, orow, sh.toff, sh.wa, sh.wb, reinterpret_cast<int32_t *>(data),
+                            data_bytes / 4);
+  } else {
+    __syncthreads();
+    for (int p = (int)min(sh.n_out, (uint32_t)k) + tid; p < k; p += FAST_T) orow[p] = -1;
+  }
 }
 
 constexpr int SMEM_OPTIN_MAX = 227 * 1024;  // largest dynamic shared memory a CTA may opt into
@@ -987,19 +1008,19 @@ int fast_smem_bytes(bool list, int n_cols, int list_cap, int L_cap) {
   return (int)sizeof(FastShared) + (list ? list_cap * 8 : n_cols * 8) + 4 * cdiv(L_cap, 32) + 8 * D0CAP;
 }
 
-template <bool LIST>
+template <bool LIST, bool ORDERED = true>
 cudaError_t launch_select_smem(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
                                const int32_t *gather, const uint32_t *row_hist, const uint2 *list,
                                const uint32_t *list_cnt, int list_cap, int k, int32_t *out, cudaStream_t s) {
   constexpr int SMEM_MAX = SMEM_OPTIN_MAX;
   struct Tag {};
   const int st = cached_per_device<Tag>([] {
-    return 1 + (int)cudaFuncSetAttribute(select_smem_kernel<LIST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return 1 + (int)cudaFuncSetAttribute(select_smem_kernel<LIST, ORDERED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          SMEM_MAX);
   });
   if (st != 1) return (cudaError_t)(st - 1);
   const int smem = fast_smem_bytes(LIST, n_cols, list_cap, c.L_cap);
-  select_smem_kernel<LIST><<<q.n_q, FAST_T, smem, s>>>(c, q, scores, ld, n_cols, gather, row_hist, list, list_cnt,
+  select_smem_kernel<LIST, ORDERED><<<q.n_q, FAST_T, smem, s>>>(c, q, scores, ld, n_cols, gather, row_hist, list, list_cnt,
                                                       list_cap, k, out);
   return cudaGetLastError();
 }
@@ -1033,7 +1054,7 @@ size_t topk_list_entries(int n_q, int L_cap, int k) {
 
 cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
                         const int32_t *gather, uint32_t *row_hist, bool hist_ready, void *list_ws,
-                        uint32_t *list_cnt, int k, int32_t *out, cudaStream_t s) {
+                        uint32_t *list_cnt, int k, int32_t *out, cudaStream_t s, bool ordered) {
   if (q.n_q == 0) return cudaSuccess;
   auto aligned16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   if (gather) {
@@ -1069,7 +1090,11 @@ cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *sco
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (8LL * list_cap <= FAST_DATA_MAX && list_cap % 2 == 0 && aligned16(list) && aligned16(row_hist) &&
       fast_smem_bytes(true, 0, list_cap, c.L_cap) <= SMEM_OPTIN_MAX)
-    return launch_select_smem<true>(c, q, scores, ld, 0, nullptr, row_hist, list, list_cnt, list_cap, k, out, s);
+    return ordered
+               ? launch_select_smem<true, true>(c, q, scores, ld, 0, nullptr, row_hist, list, list_cnt, list_cap, k,
+                                                out, s)
+               : launch_select_smem<true, false>(c, q, scores, ld, 0, nullptr, row_hist, list, list_cnt, list_cap, k,
+                                                 out, s);
   return launch_select<false, true>(c, q, scores, ld, 0, nullptr, row_hist, list, list_cnt, list_cap, k, out, s);
 }
 

@@ -29,7 +29,7 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "misa.h")
 
 MISA_OK, MISA_ERR_INVALID, MISA_ERR_UNSUPPORTED, MISA_ERR_WORKSPACE, MISA_ERR_CUDA = range(5)
 MISA_KEY_BF16, MISA_KEY_FP8_E4M3 = 0, 1
-OP_ROUTE, OP_SCORE_TOPK, OP_DENSE_TOPK, OP_RERANK_TOPK = range(4)
+OP_ROUTE, OP_SCORE_TOPK, OP_DENSE_TOPK, OP_RERANK_TOPK, OP_DAGGER_TOPK = range(5)
 DEV_BAD_POSITION, DEV_APPEND_RANGE, DEV_WAIT_TIMEOUT, DEV_BAD_HEAD = 1, 2, 4, 8
 D = 128
 NOALLOC_SCRATCH_BYTES = 4 << 20  # MISA_NOALLOC_SCRATCH_BYTES
@@ -65,6 +65,7 @@ def _load() -> ctypes.CDLL:
         "dsa_dense_score_topk": (I32, [C, Q, I32, P, P, P, SZ, P]),
         "misa_rerank_topk": (I32, [C, Q, P, I32, I32, P, P, P, SZ, P]),
         "misa_rerank_topk_noalloc": (I32, [C, Q, P, I32, I32, P, P, P]),
+        "misa_dagger_topk": (I32, [C, Q, P, I32, I32, I32, P, P, SZ, P]),
         "misa_workspace_bytes": (SZ, [I32, C, Q, I32, I32, I32]),
         "misa_last_error": (ctypes.c_char_p, []),
         "misa_status_name": (ctypes.c_char_p, [I32]),
@@ -256,6 +257,19 @@ def rerank_topk(cache: KeyCache, qs: Queries, cand: torch.Tensor, k: int, topk: 
     return topk
 
 
+def dagger_topk(cache: KeyCache, qs: Queries, heads: torch.Tensor, k_prime: int, k: int,
+                topk: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None, stream=None) -> torch.Tensor:
+    """MISA-dagger in one call: routed top-k' candidates re-ranked with every head to k."""
+    dev = qs.q.device
+    h = int(heads.shape[1])
+    if topk is None:
+        topk = torch.empty(qs.n_q, k, dtype=torch.int32, device=dev)
+    buf, nb = _ws(ws, workspace_bytes(OP_DAGGER_TOPK, cache, qs, h, k, k_prime), dev)
+    _check(_lib.misa_dagger_topk(ctypes.byref(cache.struct), ctypes.byref(qs.struct), _ptr(heads), h, k_prime, k,
+                                 _ptr(topk), _ptr(buf), nb, _stream(stream)))
+    return topk
+
+
 def rerank_topk_noalloc(cache: KeyCache, qs: Queries, cand: torch.Tensor, topk: torch.Tensor,
                         scores_out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """misa_rerank_topk_noalloc: the fine stage with the library's fixed scratch.
@@ -300,7 +314,7 @@ class MisaDaggerDecode:
     (new_pos is normally q_pos).
     """
 
-    LAUNCHES = 7  # append 1, route 2, score + top-k' 2, re-rank + top-k 2
+    LAUNCHES = 8  # append 1, route 2, score 1, top-k' 2 (filter, select), re-rank 1, top-k 1
 
     def __init__(self, cache: KeyCache, qs: Queries, h: int, k_prime: int, k: int, new_keys: torch.Tensor,
                  new_scale: Optional[torch.Tensor], new_pos: torch.Tensor):
@@ -308,10 +322,8 @@ class MisaDaggerDecode:
         self.cache, self.qs, self.h, self.k_prime, self.k = cache, qs, h, k_prime, k
         self.new_keys, self.new_scale, self.new_pos = new_keys, new_scale, new_pos
         self.heads = torch.empty(qs.n_q, h, dtype=torch.int32, device=dev)
-        self.cand = torch.empty(qs.n_q, k_prime, dtype=torch.int32, device=dev)
         self.topk = torch.empty(qs.n_q, k, dtype=torch.int32, device=dev)
-        need = max(workspace_bytes(OP_ROUTE, cache, qs, h), workspace_bytes(OP_SCORE_TOPK, cache, qs, h, k_prime),
-                   workspace_bytes(OP_RERANK_TOPK, cache, qs, 0, k, k_prime))
+        need = max(workspace_bytes(OP_ROUTE, cache, qs, h), workspace_bytes(OP_DAGGER_TOPK, cache, qs, h, k, k_prime))
         self.ws = Workspace(dev)
         self.ws.get(need)
         self.graph = None
@@ -319,8 +331,7 @@ class MisaDaggerDecode:
     def run(self, stream=None) -> torch.Tensor:
         pool_keys(self.cache, self.new_keys, self.new_scale, self.new_pos, stream=stream)
         route_heads(self.cache, self.qs, self.h, heads=self.heads, ws=self.ws, stream=stream)
-        score_topk(self.cache, self.qs, self.heads, self.k_prime, topk=self.cand, ws=self.ws, stream=stream)
-        rerank_topk(self.cache, self.qs, self.cand, self.k, topk=self.topk, ws=self.ws, stream=stream)
+        dagger_topk(self.cache, self.qs, self.heads, self.k_prime, self.k, topk=self.topk, ws=self.ws, stream=stream)
         return self.topk
 
     def capture(self) -> "MisaDaggerDecode":

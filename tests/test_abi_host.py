@@ -30,7 +30,7 @@ by = ctypes.byref
 
 def test_exports_every_declared_symbol():
     names = M.header_symbols()
-    assert len(names) == 12
+    assert len(names) == 13
     for n in names:
         assert hasattr(L, n), n
     assert M.version() == 1
@@ -91,7 +91,8 @@ def test_workspace_sizes():
     assert M._lib.misa_workspace_bytes(M.OP_SCORE_TOPK, by(c), by(q), 4, 8, 0) >= 4 * 3 * 1000
     assert M._lib.misa_workspace_bytes(M.OP_RERANK_TOPK, by(c), by(q), 0, 8, 77) >= 4 * 3 * 77
     assert M._lib.misa_workspace_bytes(9, by(c), by(q), 0, 8, 77) == 0
-    for op in range(4):
+    assert M._lib.misa_workspace_bytes(M.OP_DAGGER_TOPK, by(c), by(q), 4, 8, 77) >= 4 * 3 * (1000 + 2 * 77)
+    for op in range(5):
         assert M._lib.misa_workspace_bytes(op, by(c), by(q), 4, 8, 77) % 256 == 0
 
 
@@ -130,3 +131,12 @@ def test_noalloc_rerank_rejects_before_any_cuda_call():
         assert "injected" in M.last_error()
     finally:
         M.debug_fail_next(0)
+
+
+def test_dagger_argument_checks():
+    c, q = cache(), queries()
+    big = 1 << 30
+    assert L.misa_dagger_topk(by(c), by(q), FAKE, 8, 8, 16, FAKE, FAKE, big, None) == M.MISA_ERR_INVALID  # k > k'
+    assert L.misa_dagger_topk(by(c), by(q), FAKE, 0, 64, 16, FAKE, FAKE, big, None) == M.MISA_ERR_INVALID  # h
+    assert L.misa_dagger_topk(by(c), by(q), None, 8, 64, 16, FAKE, FAKE, big, None) == M.MISA_ERR_INVALID
+    assert L.misa_dagger_topk(by(c), by(q), FAKE, 8, 64, 16, FAKE, FAKE, 100, None) == M.MISA_ERR_WORKSPACE

@@ -346,3 +346,24 @@ def test_rerank_candidate_order_does_not_matter():
         compare_selection(b[i], f["topk"], lambda t: smap[t], wl.k, f"q{i}")
         got = b[i][b[i] >= 0]
         assert np.all(np.diff(got) > 0)
+
+
+@pytest.mark.parametrize("case", ["fp8_mixture", "fp8_long", "bf16_mixture", "bf16_prefill", "fp8_prefill_umma"])
+def test_dagger_topk_equals_composition(case):
+    # one call (its k' candidates stay unordered inside) returns exactly what
+    # the coarse stage followed by the fine stage returns; both stages are
+    # checked against the oracle by test_score_topk and test_rerank
+    inp = make(case)
+    wl = inp.wl
+    kp = wl.k_prime or 4 * wl.k
+    cache, qs = to_device(inp, torch)
+    M.pool_keys(cache)
+    heads = M.route_heads(cache, qs, wl.h)
+    cand = M.score_topk(cache, qs, heads, kp)
+    two = M.rerank_topk(cache, qs, cand, wl.k).cpu().numpy()
+    one = M.dagger_topk(cache, qs, heads, kp, wl.k).cpu().numpy()
+    np.testing.assert_array_equal(one, two)
+    for i in range(wl.n_q):
+        got = one[i][one[i] >= 0]
+        assert np.all(np.diff(got) > 0)
+    assert device_status(cache) == 0
