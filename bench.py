@@ -182,6 +182,57 @@ METRIC = "indexer scored head*tokens/s (MISA-dagger decode, L=128K)"
 UNIT = "head*tokens/s"
 
 
+def prefill_roofline(M, torch, dev, peak_tflops, peak_src):
+    """Tensor-core prefill scoring on the two prefill workloads (context for
+    the decode headline): the scoring kernel's useful TFLOP/s against the
+    measured bf16 peak, and the whole score + top-k call."""
+    out = {}
+    for name in ("causal_prefill", "long_prefill_128k"):
+        wl = G.WORKLOADS[name]
+        inp = G.make_inputs(wl, 0)
+        cache, qs = M.device_inputs(inp, dev)
+        M.pool_keys(cache)
+        heads = M.route_heads(cache, qs, wl.h)
+        ws = M.Workspace(dev)
+        li = inp.q_pos.astype(np.int64) + 1
+        rec = {}
+        for kind, n_heads in (("misa", wl.h), ("dense", wl.H)):
+            def run():
+                if kind == "misa":
+                    M.score_topk(cache, qs, heads, wl.k, ws=ws)
+                else:
+                    M.dense_score_topk(cache, qs, wl.k, ws=ws)
+            for _ in range(2):
+                run()
+            torch.cuda.synchronize()
+            ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ka.record()
+            kb.record()
+            torch.cuda.synchronize()
+            M.debug_time_scoring(ka, kb)
+            kt, tt = [], []
+            for _ in range(5):
+                a.record()
+                run()
+                b.record()
+                torch.cuda.synchronize()
+                kt.append(ka.elapsed_time(kb))
+                tt.append(a.elapsed_time(b))
+            M.debug_time_scoring(None, None)
+            k_ms = float(np.median(kt))
+            flops = 2.0 * wl.d * n_heads * float(li.sum())
+            tf = flops / (k_ms * 1e-3) / 1e12
+            rec[kind] = {"scoring_us": k_ms * 1e3, "score_topk_us": float(np.median(tt)) * 1e3,
+                         "achieved": tf, "peak": peak_tflops, "unit": "TFLOP/s", "frac": tf / peak_tflops,
+                         "peak_source": peak_src}
+        out[name] = {"kernel": "score_umma_kernel (tcgen05, TMA, TMEM)", "n_q": wl.n_q, "L": wl.L,
+                     "key_dtype": wl.key_dtype, **rec}
+        del cache, qs, ws
+        torch.cuda.empty_cache()
+    return out
+
+
 def config_block(wl, l2):
     return {"workload": wl.name, "n_seq": wl.n_seq, "L": wl.L, "H_I": wl.H, "h": wl.h, "B": wl.B,
             "k_prime": wl.k_prime, "k": wl.k, "d": wl.d, "key_dtype": "fp8_e4m3+fp32 scale", "q_dtype": "bf16",
@@ -196,6 +247,7 @@ def main():
     ap.add_argument("--impl", default="misa", choices=["misa", "reference"])
     ap.add_argument("--workload", default="misa_dagger_decode_128k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill tensor-core context figures")
     args = ap.parse_args()
     wl = G.WORKLOADS[args.workload]
     assert wl.k_prime is not None and wl.mode == "decode", "the bench step is the MISA-dagger decode step"
@@ -381,6 +433,10 @@ def main():
         }
         if cpu:
             line["cpu_baseline"] = cpu
+        if not args.no_prefill and world == 1:
+            pk = peaks()
+            line["prefill"] = prefill_roofline(M, torch, dev, pk[1], f"{pk[2]} bf16_tflops (e4m3 runs two MMAs "
+                                               "per K step at twice the rate: same time per useful flop)")
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
