@@ -62,7 +62,7 @@ def score_kernel_bytes(wl):
 # decode workload at L = 128K, from the ncu capture summarised in
 # profiles/score_stream_kernel_misa_dagger_decode_128k.md.  Valid only for
 # that workload and that kernel version; reported as null elsewhere.
-STREAM_TRAFFIC_BYTES = {"misa_dagger_decode_128k": 143_097_344}
+STREAM_TRAFFIC_BYTES = {"misa_dagger_decode_128k": 143_242_496}
 
 
 class Clocks:
