@@ -153,7 +153,7 @@ misa_status score_then_topk(const char *who, const misa_cache *cache, const misa
   // selection counts each row itself; otherwise the streaming scorer builds
   // the row histograms on the way
   const bool umma = misa::umma_applies(c, q, heads, h);
-  cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * hist_words(qs), stream);
+  cudaError_t e = misa::launch_zero(hist, hist_words(qs), stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   e = timed_scoring(stream, [&] {
     return umma ? misa::launch_score_umma(c, q, heads, h, scores, cache->L_cap, stream)
@@ -293,7 +293,7 @@ misa_status misa_rerank_topk(const misa_cache *cache, const misa_queries *qs, co
   misa::QueryView q = view(qs);
   uint32_t *hist = static_cast<uint32_t *>(ws);
   float *scores = scores_out ? scores_out : reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + ws_hist(qs));
-  cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
+  cudaError_t e = misa::launch_zero(hist, (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
   if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
   e = timed_scoring(stream, [&] {
     return misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, scores, k_prime, hist, stream);
@@ -328,7 +328,7 @@ misa_status misa_rerank_topk_noalloc(const misa_cache *cache, const misa_queries
   misa::QueryView q = view(qs);
   uint32_t *hist = static_cast<uint32_t *>(ws);
   float *scores = scores_out ? scores_out : reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + ws_hist(qs));
-  cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
+  cudaError_t e = misa::launch_zero(hist, (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   e = timed_scoring(stream, [&] {
     return misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, scores, k_prime, hist, stream);
@@ -365,7 +365,7 @@ misa_status misa_dagger_topk(const misa_cache *cache, const misa_queries *qs, co
                                              round_up(sizeof(int32_t) * (size_t)qs->n_q * k_prime));
   // routed pass: scores, then the k' candidates in any order
   const bool umma = misa::umma_applies(c, q, heads, h);
-  cudaError_t e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * hist_words(qs), stream);
+  cudaError_t e = misa::launch_zero(hist, hist_words(qs), stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   e = timed_scoring(stream, [&] {
     return umma ? misa::launch_score_umma(c, q, heads, h, scores, cache->L_cap, stream)
@@ -376,7 +376,7 @@ misa_status misa_dagger_topk(const misa_cache *cache, const misa_queries *qs, co
                         false);
   if (e != cudaSuccess) return cuda_fail(e, who);
   // fine pass: every head on the candidates, ascending final top-k
-  e = cudaMemsetAsync(hist, 0, sizeof(uint32_t) * (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
+  e = misa::launch_zero(hist, (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   e = misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, rscores, k_prime, hist, stream);
   if (e != cudaSuccess) return cuda_fail(e, who);

@@ -59,6 +59,8 @@ cudaError_t launch_score_umma(const CacheView &c, const QueryView &q, const int3
 constexpr int TOPK_LIST_MIN_L = 16384;   // shorter caches never use the list
 constexpr int TOPK_LIST_EXTRA = 8192;    // boundary-bin elements listed per row beyond k
 size_t topk_list_entries(int n_q, int L_cap, int k);
+// n words set to zero on stream s (a small kernel)
+cudaError_t launch_zero(uint32_t *p, size_t n, cudaStream_t s);
 cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
                         const int32_t *gather, uint32_t *row_hist, bool hist_ready, void *list_ws,
                         uint32_t *list_cnt, int k, int32_t *out, cudaStream_t s, bool ordered = true);

@@ -76,14 +76,12 @@ __global__ void __launch_bounds__(APPEND_THREADS) pool_append_kernel(CacheView c
 
 cudaError_t launch_pool_rebuild(const CacheView &c, cudaStream_t s) {
   dim3 grid(cdiv(c.L_cap, c.B), c.n_seq);
-  pool_rebuild_kernel<<<grid, REBUILD_THREADS, 0, s>>>(c);
-  return cudaGetLastError();
+  return launch_kernel(pool_rebuild_kernel, grid, dim3(REBUILD_THREADS), 0, s, c);
 }
 
 cudaError_t launch_pool_append(const CacheView &c, const void *new_keys, const float *new_scale,
                                const int32_t *new_pos, int count, cudaStream_t s) {
-  pool_append_kernel<<<c.n_seq, APPEND_THREADS, 0, s>>>(c, new_keys, new_scale, new_pos, count);
-  return cudaGetLastError();
+  return launch_kernel(pool_append_kernel, dim3(c.n_seq), dim3(APPEND_THREADS), 0, s, c, new_keys, new_scale, new_pos, count);
 }
 
 }  // namespace misa

@@ -234,11 +234,10 @@ cudaError_t launch_route(const CacheView &c, const QueryView &q, int h, int32_t 
   if (opt_in < 0) return cudaErrorInvalidConfiguration;
   cudaError_t e;
   float *partial = static_cast<float *>(ws);
-  route_partial_kernel<<<dim3(n_chunks, q.n_q), ROUTE_THREADS, smem, s>>>(c, q, partial, n_chunks);
-  e = cudaGetLastError();
+  e = launch_kernel(route_partial_kernel, dim3(n_chunks, q.n_q), dim3(ROUTE_THREADS), smem, s, c, q, partial, n_chunks);
   if (e != cudaSuccess) return e;
-  route_finish_kernel<<<q.n_q, MISA_MAX_H, 0, s>>>(c, q, partial, n_chunks, h, heads, router_scores);
-  return cudaGetLastError();
+  return launch_kernel(route_finish_kernel, dim3(q.n_q), dim3(MISA_MAX_H), 0, s, c, q, partial, n_chunks, h, heads,
+                    router_scores);
 }
 
 }  // namespace misa

@@ -154,9 +154,8 @@ cudaError_t launch_gather(dim3 grid, const CacheView &c, const QueryView &q, con
                                          SMEM);
   });
   if (st != 1) return (cudaError_t)(st - 1);
-  score_gather_kernel<NT, FP8><<<grid, SC_THREADS, SMEM, s>>>(c, q, heads, h, gather, n_cols, scores, ld, chunk,
-                                                              row_hist);
-  return cudaGetLastError();
+  return launch_kernel(score_gather_kernel<NT, FP8>, grid, dim3(SC_THREADS), SMEM, s, c, q, heads, h, gather, n_cols,
+                    scores, ld, chunk, row_hist);
 }
 
 }  // namespace

@@ -203,9 +203,8 @@ cudaError_t launch_nt(const CacheView &c, const QueryView &q, const int32_t *hea
   int splits = max(1, per_sm * sms / q.n_q);
   splits = min(splits, max(1, cdiv(cdiv(c.L_cap, StreamCfg<NT, FP8>::TT), 2 * WARPS)));  // >= 2 tiles per warp
   const int scale_vec = FP8 && (reinterpret_cast<uintptr_t>(c.scale) & 15) == 0 && c.L_cap % 4 == 0;
-  score_stream_kernel<NT, FP8><<<dim3(splits, q.n_q), THREADS, SMEM, s>>>(c, q, heads, h, scores, ld, scale_vec,
-                                                                                      row_hist);
-  return cudaGetLastError();
+  return launch_kernel(score_stream_kernel<NT, FP8>, dim3(splits, q.n_q), dim3(THREADS), SMEM, s, c, q, heads, h, scores,
+                    ld, scale_vec, row_hist);
 }
 
 }  // namespace

@@ -469,8 +469,8 @@ cudaError_t launch_hpq(const CUtensorMap &map, const CacheView &c, const QueryVi
   const int n_tiles = cdiv(c.L_cap, UM_M);
   const long long n_items = (long long)n_groups * n_tiles;
   const int grid = (int)std::min<long long>(device_sms(), n_items);
-  score_umma_kernel<FP8, HPQ><<<grid, UM_THREADS, SMEM, s>>>(map, c, q, heads, h, scores, ld, n_tiles, n_items);
-  return cudaGetLastError();
+  return launch_kernel(score_umma_kernel<FP8, HPQ>, dim3(grid), dim3(UM_THREADS), SMEM, s, map, c, q, heads, h, scores,
+                    ld, n_tiles, n_items);
 }
 
 }  // namespace

@@ -31,6 +31,8 @@
 // filter_kernel (few long rows: decode): many CTAs per row copy the elements
 //   at or above d0 into a per-row list, so that the one CTA per row above
 //   reads about k + |d0| entries instead of the whole row.
+#include <algorithm>
+
 #include "internal.h"
 
 namespace misa {
@@ -1020,9 +1022,14 @@ cudaError_t launch_select_smem(const CacheView &c, const QueryView &q, const flo
   });
   if (st != 1) return (cudaError_t)(st - 1);
   const int smem = fast_smem_bytes(LIST, n_cols, list_cap, c.L_cap);
-  select_smem_kernel<LIST, ORDERED><<<q.n_q, FAST_T, smem, s>>>(c, q, scores, ld, n_cols, gather, row_hist, list, list_cnt,
-                                                      list_cap, k, out);
-  return cudaGetLastError();
+  return launch_kernel(select_smem_kernel<LIST, ORDERED>, dim3(q.n_q), dim3(FAST_T), smem, s, c, q, scores, ld, n_cols,
+                    gather, row_hist, list, list_cnt, list_cap, k, out);
+}
+
+// Zero n words (the histograms and list counters before a scoring pass); a
+// kernel measured as fast as a memset node in the decode step's graph.
+__global__ void __launch_bounds__(256) zero_kernel(uint32_t *p, size_t n) {
+  for (size_t x = blockIdx.x * 256 + threadIdx.x; x < n; x += (size_t)gridDim.x * 256) p[x] = 0u;
 }
 
 int sel_smem_bytes(int L_cap) { return (int)sizeof(SelShared) + 4 * cdiv(L_cap, 32); }
@@ -1040,12 +1047,17 @@ cudaError_t launch_select(const CacheView &c, const QueryView &q, const float *s
                : -1;
   });
   if (ok < 0) return cudaErrorInvalidConfiguration;
-  select_kernel<GATHER, FROM_LIST, OWN_HIST><<<q.n_q, SEL_T, sel_smem_bytes(c.L_cap), s>>>(
-      c, q, scores, ld, n_cols, gather, row_hist, list, list_cnt, list_cap, k, out);
-  return cudaGetLastError();
+  return launch_kernel(select_kernel<GATHER, FROM_LIST, OWN_HIST>, dim3(q.n_q), dim3(SEL_T), sel_smem_bytes(c.L_cap), s, c,
+                    q, scores, ld, n_cols, gather, row_hist, list, list_cnt, list_cap, k, out);
 }
 
 }  // namespace
+
+cudaError_t launch_zero(uint32_t *p, size_t n, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const int blocks = (int)std::min<size_t>((n + 255) / 256, (size_t)2 * device_sms());
+  return launch_kernel(zero_kernel, dim3(blocks), dim3(256), 0, s, p, n);
+}
 
 size_t topk_list_entries(int n_q, int L_cap, int k) {
   if (n_q < 1 || L_cap <= TOPK_LIST_MIN_L || k < 1) return 0;
@@ -1074,8 +1086,9 @@ cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *sco
     // wide pass over the scores: about 16K elements per CTA
     const int per_row = cdiv(c.L_cap, 16384);
     const int chunk = cdiv(cdiv(c.L_cap, per_row), HIST_T) * HIST_T;
-    hist_kernel<<<dim3(cdiv(c.L_cap, chunk), q.n_q), HIST_T, 0, s>>>(c, q, scores, ld, row_hist, chunk);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = launch_kernel(hist_kernel, dim3(cdiv(c.L_cap, chunk), q.n_q), dim3(HIST_T), 0, s, c, q, scores, ld, row_hist,
+                   chunk);
+    if (e != cudaSuccess) return e;
   }
   if (!list_mode)
     return launch_select<false, false>(c, q, scores, ld, 0, nullptr, row_hist, nullptr, nullptr, 0, k, out, s);
@@ -1085,9 +1098,9 @@ cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *sco
   // per CTA (many rows), at least 4096 elements each
   const int per_row = max(1, min(cdiv(c.L_cap, 4096), max(2 * sms / q.n_q, cdiv(c.L_cap, 16384))));
   const int chunk = cdiv(cdiv(c.L_cap, per_row), FILT_T) * FILT_T;
-  filter_kernel<<<dim3(cdiv(c.L_cap, chunk), q.n_q), FILT_T, 0, s>>>(c, q, scores, ld, row_hist, list, list_cnt,
-                                                                     list_cap, k, chunk);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  e = launch_kernel(filter_kernel, dim3(cdiv(c.L_cap, chunk), q.n_q), dim3(FILT_T), 0, s, c, q, scores, ld, row_hist,
+                 list, list_cnt, list_cap, k, chunk);
+  if (e != cudaSuccess) return e;
   if (8LL * list_cap <= FAST_DATA_MAX && list_cap % 2 == 0 && aligned16(list) && aligned16(row_hist) &&
       fast_smem_bytes(true, 0, list_cap, c.L_cap) <= SMEM_OPTIN_MAX)
     return ordered
