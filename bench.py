@@ -182,6 +182,23 @@ METRIC = "indexer scored head*tokens/s (MISA-dagger decode, L=128K)"
 UNIT = "head*tokens/s"
 
 
+def aggregate(total_ms, steps, per_step_work, queries_per_step, world, dist=None, device="cpu"):
+    """Whole-job throughput from the ranks' timed totals.
+
+    Every rank processed its own batch (weak scaling); the job took as long as
+    the slowest rank, so the time is the max over ranks (an all-reduce when
+    dist is given) and the work is world x one rank's.  Returns (ms per step,
+    head*tokens/s, queries/s).
+    """
+    import torch
+    if dist is not None and world > 1:
+        t = torch.tensor([float(total_ms)], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms = total_ms / steps
+    return ms, world * per_step_work / (ms * 1e-3), world * queries_per_step / (ms * 1e-3)
+
+
 def prefill_roofline(M, torch, dev, peak_tflops, peak_src):
     """Tensor-core prefill scoring on the two prefill workloads (context for
     the decode headline): the scoring kernel's useful TFLOP/s against the
@@ -348,16 +365,11 @@ def main():
         g_kernel.replay()
         torch.cuda.synchronize()
         kern_ms.append(ka.elapsed_time(kb))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
     assert cache.device_status() == 0, "device status set during timing"
 
     per_step_work = sum(work_per_query(wl, int(inp.q_pos[i]) + 1) for i in range(wl.n_q))
-    ms_per_step = total_ms / args.steps
-    value = world * per_step_work / (ms_per_step * 1e-3)
-    qps = world * wl.n_q / (ms_per_step * 1e-3)
+    ms_per_step, value, qps = aggregate(total_ms, args.steps, per_step_work, wl.n_q, world,
+                                        dist if world > 1 else None, dev)
 
     # ---- dense DSA indexer on the same batch (context: the work MISA replaces) ----
     ws = M.Workspace(dev)
