@@ -1,5 +1,6 @@
 // C ABI of the MISA / DSA indexer: argument validation, workspace layout and
 // dispatch to the kernels.  Declarations and semantics: include/misa.h.
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -218,8 +219,11 @@ size_t misa_workspace_bytes(int32_t op, const misa_cache *cache, const misa_quer
   (void)h;
   if (!cache || !qs || cache->B < 1 || cache->L_cap < 1 || qs->n_q < 0 || qs->H < 1) return 0;
   switch (op) {
-    case MISA_OP_ROUTE:
-      return round_up(misa::route_ws_bytes(qs->n_q, qs->H, misa::cdiv(cache->L_cap, cache->B)));
+    case MISA_OP_ROUTE: {
+      const int M_cap = misa::cdiv(cache->L_cap, cache->B);
+      return round_up(std::max(misa::route_ws_bytes(qs->n_q, qs->H, M_cap),
+                               misa::route_umma_ws_bytes(qs->n_q, qs->H, M_cap, cache->n_seq)));
+    }
     case MISA_OP_SCORE_TOPK:
     case MISA_OP_DENSE_TOPK:
       return ws_hist(qs) + ws_score(cache, qs) + (k > 0 ? ws_list(cache, qs, k) : 0);

@@ -23,6 +23,12 @@ int route_chunks(int M_cap);
 size_t route_ws_bytes(int n_q, int H, int M_cap);
 cudaError_t launch_route(const CacheView &c, const QueryView &q, int h, int32_t *heads, float *router_scores,
                          void *ws, cudaStream_t s);
+// route_umma.cu: the same routing for many queries per sequence (prefill) on
+// tcgen05 tensor cores; launch_route dispatches to it when it applies.
+bool route_umma_applies(const CacheView &c, const QueryView &q);
+size_t route_umma_ws_bytes(int n_q, int H, int M_cap, int n_seq);
+cudaError_t launch_route_umma(const CacheView &c, const QueryView &q, int h, int32_t *heads, float *router_scores,
+                              void *ws, cudaStream_t s);
 
 // score_mma.cu: scores[i][t] (row stride ld) for t < L_i, heads given per query
 // (heads == nullptr: all H heads, dense).  `gather` != nullptr: row i scores the

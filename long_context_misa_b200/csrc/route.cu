@@ -223,6 +223,7 @@ size_t route_ws_bytes(int n_q, int H, int M_cap) {
 cudaError_t launch_route(const CacheView &c, const QueryView &q, int h, int32_t *heads, float *router_scores,
                          void *ws, cudaStream_t s) {
   if (q.n_q == 0) return cudaSuccess;
+  if (route_umma_applies(c, q)) return launch_route_umma(c, q, h, heads, router_scores, ws, s);
   const int M_cap = cdiv(c.L_cap, c.B);
   const int n_chunks = route_chunks(M_cap);
   const size_t smem = route_smem_bytes(q.H);

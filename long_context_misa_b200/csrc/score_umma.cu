@@ -36,6 +36,7 @@
 
 #include "frag.cuh"
 #include "internal.h"
+#include "umma.cuh"
 
 namespace misa {
 namespace {
@@ -72,80 +73,6 @@ struct UmmaShared {
 template <bool FP8>
 constexpr int umma_smem_bytes() {
   return 1024 /* alignment slack */ + UCfg<FP8>::STAGES * UCfg<FP8>::A_BYTES + B_BYTES + (int)sizeof(UmmaShared);
-}
-
-// ---- PTX wrappers -------------------------------------------------------
-
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
-  // K-major, 128-byte swizzle: 8-row atoms of 128 B, 1024 B apart (SBO);
-  // LBO unused (1); descriptor version 1; layout type 2 = SWIZZLE_128B.
-  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-template <bool FP8>
-__device__ __forceinline__ uint32_t instr_desc() {
-  // D fp32, A/B K-major, N = 256, M = 128; A/B format bf16 (1) or e4m3 (0)
-  const uint32_t fmt = FP8 ? 0u : 1u;
-  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((uint32_t)(UM_N >> 3) << 17) | ((uint32_t)(UM_M >> 4) << 24);
-}
-
-template <bool FP8>
-__device__ __forceinline__ void umma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  if (FP8)
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc));
-  else
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc));
-}
-
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
-      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
-        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
-        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
-        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
-      : "memory");
-}
-
-// Bounded wait shared by all roles: false once this CTA has given up (here or
-// in another role).
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort, const CacheView &c) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
-      *abort = 1;
-      flag(c, MISA_DEV_WAIT_TIMEOUT);
-      return false;
-    }
-  }
-  return true;
 }
 
 // ---- the kernel -----------------------------------------------------------
@@ -188,10 +115,10 @@ __global__ void __maxnreg__(128)
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_addr(&sh.tmem_base)));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-    tc_fence_before();
+    umma::fence_before();
   }
   __syncthreads();
-  tc_fence_after();
+  umma::fence_after();
   const uint32_t tmem = sh.tmem_base;
 
   // pipeline counters (same sequence of tiles in every role)
@@ -301,15 +228,15 @@ __global__ void __maxnreg__(128)
         if (lane == 0) {
           for (int tau = tau0; tau < t_end; ++tau, ++it_load) {
             const int st = it_load % Cfg::STAGES;
-            if (!wait_bar(&sh.empty[st], ((it_load / Cfg::STAGES) & 1) ^ 1, abort, c)) break;
+            if (!umma::wait_bar(&sh.empty[st], ((it_load / Cfg::STAGES) & 1) ^ 1, abort, c)) break;
             mbar_arrive_expect_tx(&sh.full[st], Cfg::A_BYTES);
             const uint32_t dst = smem_addr(a_smem + st * Cfg::A_BYTES);
             const int y = seq * c.L_cap + tau * UM_M;
             if (FP8) {
-              tma_load_2d(dst, &kmap, 0, y, &sh.full[st]);
+              umma::tma_load_2d(dst, &kmap, 0, y, &sh.full[st]);
             } else {
-              tma_load_2d(dst, &kmap, 0, y, &sh.full[st]);
-              tma_load_2d(dst + UM_M * 128, &kmap, 64, y, &sh.full[st]);
+              umma::tma_load_2d(dst, &kmap, 0, y, &sh.full[st]);
+              umma::tma_load_2d(dst + UM_M * 128, &kmap, 64, y, &sh.full[st]);
             }
             last_fill_parity[st] = (it_load / Cfg::STAGES) & 1;
           }
@@ -317,14 +244,14 @@ __global__ void __maxnreg__(128)
       } else if (warp == 1) {
         // ---- MMA issuer ----
         if (lane == 0) {
-          const uint32_t idesc = instr_desc<FP8>();
+          const uint32_t idesc = umma::instr_desc<FP8, UM_M, UM_N>();
           const uint32_t b_base = smem_addr(b_smem);
           for (int tau = tau0; tau < t_end; ++tau, ++it_mma, ++j_mma) {
             const int st = it_mma % Cfg::STAGES, buf = j_mma & 1;
-            if (!wait_bar(&sh.tempty[buf], ((j_mma >> 1) & 1) ^ 1, abort, c)) break;
-            tc_fence_after();
-            if (!wait_bar(&sh.full[st], (it_mma / Cfg::STAGES) & 1, abort, c)) break;
-            tc_fence_after();
+            if (!umma::wait_bar(&sh.tempty[buf], ((j_mma >> 1) & 1) ^ 1, abort, c)) break;
+            umma::fence_after();
+            if (!umma::wait_bar(&sh.full[st], (it_mma / Cfg::STAGES) & 1, abort, c)) break;
+            umma::fence_after();
             const uint32_t a_base = smem_addr(a_smem + st * Cfg::A_BYTES);
             const uint32_t d = tmem + buf * UM_N;
 #pragma unroll
@@ -339,12 +266,12 @@ __global__ void __maxnreg__(128)
                   aoff = (kk >> 2) * (UM_M * 128) + (kk & 3) * 32;
                   boff = (kk >> 2) * (UM_N * 128) + (kk & 3) * 32;
                 }
-                umma<FP8>(d, smem_desc_sw128(a_base + aoff), smem_desc_sw128(b_base + boff), idesc,
+                umma::mma<FP8>(d, umma::smem_desc_sw128(a_base + aoff), umma::smem_desc_sw128(b_base + boff), idesc,
                           (t | kk) ? 1u : 0u);
               }
             }
-            umma_commit(&sh.empty[st]);
-            umma_commit(&sh.tfull[buf]);
+            umma::commit(&sh.empty[st]);
+            umma::commit(&sh.tfull[buf]);
             mma_issued = true;
           }
         }
@@ -360,16 +287,16 @@ __global__ void __maxnreg__(128)
           const int t = tau * UM_M + r;
           const float st_scale = (FP8 && t < c.L_cap) ? __ldg(c.scale + (size_t)seq * c.L_cap + t) : 1.f;
           float *out_t = scores + (size_t)g * QPT * ld + t;  // row of query g*QPT + ql at + ql*ld
-          if (!wait_bar(&sh.tfull[buf], (j_epi >> 1) & 1, abort, c)) break;
-          tc_fence_after();
+          if (!umma::wait_bar(&sh.tfull[buf], (j_epi >> 1) & 1, abort, c)) break;
+          umma::fence_after();
           const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * UM_N + col0;
           float acc = 0.f;  // running sum of a query wider than one chunk
 #pragma unroll
           for (int ch = 0; ch < UM_N / 64; ch += 2) {
             uint32_t v0[32], v1[32];
-            tmem_ld32(taddr + ch * 32, v0);
-            tmem_ld32(taddr + ch * 32 + 32, v1);
-            tmem_ld_wait();
+            umma::ld32(taddr + ch * 32, v0);
+            umma::ld32(taddr + ch * 32 + 32, v1);
+            umma::ld_wait();
 #pragma unroll
             for (int hc = 0; hc < 2; ++hc) {
               const uint32_t(&v)[32] = hc ? v1 : v0;
@@ -407,7 +334,7 @@ __global__ void __maxnreg__(128)
               }
             }
           }
-          tc_fence_before();
+          umma::fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.tempty[buf]);
         }
@@ -421,37 +348,21 @@ __global__ void __maxnreg__(128)
   // ---- wind-down: nothing in flight when the tensor memory is released ----
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < Cfg::STAGES; ++s)
-      if (last_fill_parity[s] < 2) wait_bar(&sh.full[s], last_fill_parity[s], abort, c);
+      if (last_fill_parity[s] < 2) umma::wait_bar(&sh.full[s], last_fill_parity[s], abort, c);
   }
   if (warp == 1 && lane == 0 && mma_issued) {
     const uint32_t jl = j_mma - 1;  // the last committed accumulator buffer
-    wait_bar(&sh.tfull[jl & 1], (jl >> 1) & 1, abort, c);
+    umma::wait_bar(&sh.tfull[jl & 1], (jl >> 1) & 1, abort, c);
   }
-  tc_fence_before();
+  umma::fence_before();
   __syncthreads();
   if (warp == 1) {
-    tc_fence_after();
+    umma::fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
   }
 }
 
 // ---- host side ----------------------------------------------------------
-
-using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiled encode_fn() {
-  static EncodeTiled fn = [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return (EncodeTiled) nullptr;
-    return reinterpret_cast<EncodeTiled>(p);
-  }();
-  return fn;
-}
 
 template <bool FP8, int HPQ>
 cudaError_t launch_hpq(const CUtensorMap &map, const CacheView &c, const QueryView &q, const int32_t *heads, int h,
@@ -477,24 +388,15 @@ cudaError_t launch_hpq(const CUtensorMap &map, const CacheView &c, const QueryVi
 
 bool umma_applies(const CacheView &c, const QueryView &q, const int32_t *heads, int h) {
   const int h_eff = heads ? h : q.H;
-  return q.n_q >= 64 && q.n_q >= 8 * c.n_seq && h_eff <= UM_N && encode_fn() != nullptr;
+  return q.n_q >= 64 && q.n_q >= 8 * c.n_seq && h_eff <= UM_N && umma::encoder_available();
 }
 
 cudaError_t launch_score_umma(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
                               long long ld, cudaStream_t s) {
   if (q.n_q == 0) return cudaSuccess;
-  EncodeTiled enc = encode_fn();
-  if (!enc) return cudaErrorNotSupported;
   CUtensorMap map;
-  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)c.n_seq * (cuuint64_t)c.L_cap};
-  const cuuint64_t strides[1] = {(cuuint64_t)(c.fp8 ? D : 2 * D)};
-  const cuuint32_t box[2] = {(cuuint32_t)(c.fp8 ? 128 : 64), (cuuint32_t)UM_M};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(&map, c.fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                         const_cast<void *>(c.keys), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  if (!umma::make_map_2d(&map, c.keys, c.fp8, (unsigned long long)c.n_seq * c.L_cap, c.fp8 ? 128 : 64, UM_M))
+    return cudaErrorNotSupported;
   const int h_eff = heads ? h : q.H;
   int hpq = 4;  // at least 4 columns per query (zero-weight padding)
   while (hpq < h_eff) hpq *= 2;
@@ -515,4 +417,37 @@ cudaError_t launch_score_umma(const CacheView &c, const QueryView &q, const int3
 #undef MISA_UMMA_CASE
 }
 
+namespace umma {
+
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiled encode_fn() {
+  static EncodeTiled fn = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (EncodeTiled) nullptr;
+    return reinterpret_cast<EncodeTiled>(p);
+  }();
+  return fn;
+}
+
+bool encoder_available() { return encode_fn() != nullptr; }
+
+bool make_map_2d(CUtensorMap *map, const void *base, bool u8, unsigned long long rows, int box_x, int box_rows) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(u8 ? D : 2 * D)};
+  const cuuint32_t box[2] = {(cuuint32_t)box_x, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base),
+             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace umma
 }  // namespace misa
