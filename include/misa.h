@@ -296,6 +296,16 @@ MISA_API void misa_debug_fail_next(int32_t n);
  */
 MISA_API void misa_debug_time_scoring(void *start, void *stop);
 
+/*
+ * Failure-path check: launch one kernel that waits, with the same bounded
+ * wait every on-chip pipeline of the library uses, on an mbarrier that never
+ * completes.  After limit_ns (at most 10 s) the wait gives up, ORs
+ * MISA_DEV_WAIT_TIMEOUT into *status (device memory) and the kernel returns
+ * normally: no fault, no trap, the context stays usable.  Errors:
+ * MISA_ERR_INVALID for a NULL status or a limit above 10 s.
+ */
+MISA_API misa_status misa_debug_wait_timeout(uint32_t *status, uint64_t limit_ns, misa_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -166,6 +166,19 @@ misa_status score_then_topk(const char *who, const misa_cache *cache, const misa
   return MISA_OK;
 }
 
+// The bounded wait every pipeline of the library uses, on an mbarrier that
+// never completes: after limit_ns it records MISA_DEV_WAIT_TIMEOUT and the
+// kernel returns normally (the failure path, exercised without a fault).
+__global__ void wait_timeout_kernel(uint32_t *status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    misa::mbar_init(&bar, 1);
+    misa::fence_mbar_init();
+  }
+  __syncthreads();
+  if (!misa::mbar_wait(&bar, 0, limit_ns) && threadIdx.x == 0) atomicOr(status, MISA_DEV_WAIT_TIMEOUT);
+}
+
 // Scratch of misa_rerank_topk_noalloc: part of the library's device image, so
 // the caller never supplies memory and the call never allocates any.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[MISA_NOALLOC_SCRATCH_BYTES];
@@ -386,6 +399,15 @@ misa_status misa_dagger_topk(const misa_cache *cache, const misa_queries *qs, co
   if (e != cudaSuccess) return cuda_fail(e, who);
   e = misa::launch_topk(c, q, rscores, k_prime, k_prime, cand, hist, true, nullptr, nullptr, k, topk, stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
+  return MISA_OK;
+}
+
+misa_status misa_debug_wait_timeout(uint32_t *status, uint64_t limit_ns, misa_stream stream) {
+  if (!status) return fail(MISA_ERR_INVALID, "status is NULL");
+  if (limit_ns > 10000000000ull) return fail(MISA_ERR_INVALID, "limit_ns=%llu above 10 s", (unsigned long long)limit_ns);
+  cudaError_t e = misa::launch_kernel(wait_timeout_kernel, dim3(1), dim3(32), 0, stream, status,
+                                      (unsigned long long)limit_ns);
+  if (e != cudaSuccess) return cuda_fail(e, "misa_debug_wait_timeout");
   return MISA_OK;
 }
 

@@ -206,12 +206,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of `bar` to complete; false if WAIT_LIMIT_NS passed.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// Wait for phase `parity` of `bar` to complete; false once `limit_ns`
+// (default WAIT_LIMIT_NS) has passed.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns = WAIT_LIMIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity))
-    if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   return true;
 }
 

@@ -72,6 +72,7 @@ def _load() -> ctypes.CDLL:
         "misa_version": (I32, []),
         "misa_debug_fail_next": (None, [I32]),
         "misa_debug_time_scoring": (None, [P, P]),
+        "misa_debug_wait_timeout": (I32, [P, ctypes.c_uint64, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -108,6 +109,11 @@ def debug_time_scoring(start=None, stop=None) -> None:
     """Bracket every scoring kernel with these torch.cuda.Event objects (None, None: off)."""
     _lib.misa_debug_time_scoring(None if start is None else start.cuda_event,
                                  None if stop is None else stop.cuda_event)
+
+
+def debug_wait_timeout(status: torch.Tensor, limit_ns: int, stream=None) -> None:
+    """Run the library's bounded wait on a barrier that never completes (see misa.h)."""
+    _check(_lib.misa_debug_wait_timeout(_ptr(status), int(limit_ns), _stream(stream)))
 
 
 def _check(st: int) -> None:

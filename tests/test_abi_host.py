@@ -30,7 +30,7 @@ by = ctypes.byref
 
 def test_exports_every_declared_symbol():
     names = M.header_symbols()
-    assert len(names) == 13
+    assert len(names) == 14
     for n in names:
         assert hasattr(L, n), n
     assert M.version() == 1
@@ -140,3 +140,8 @@ def test_dagger_argument_checks():
     assert L.misa_dagger_topk(by(c), by(q), FAKE, 0, 64, 16, FAKE, FAKE, big, None) == M.MISA_ERR_INVALID  # h
     assert L.misa_dagger_topk(by(c), by(q), None, 8, 64, 16, FAKE, FAKE, big, None) == M.MISA_ERR_INVALID
     assert L.misa_dagger_topk(by(c), by(q), FAKE, 8, 64, 16, FAKE, FAKE, 100, None) == M.MISA_ERR_WORKSPACE
+
+
+def test_wait_timeout_argument_checks():
+    assert L.misa_debug_wait_timeout(None, 1000, None) == M.MISA_ERR_INVALID
+    assert L.misa_debug_wait_timeout(FAKE, 11_000_000_000, None) == M.MISA_ERR_INVALID
