@@ -46,9 +46,10 @@ def peaks():
 
 
 def work_per_query(wl, L_i):
-    """Algorithmic head.tokens of one MISA-dagger query (cost model of the method)."""
+    """Algorithmic head.tokens of one MISA (or MISA-dagger, when the workload has a
+    k') query: h*L + H_I*M (+ H_I*min(k', L)), the method's cost model."""
     M = -(-L_i // wl.B)
-    return wl.h * L_i + wl.H * M + wl.H * min(wl.k_prime, L_i)
+    return wl.h * L_i + wl.H * M + (wl.H * min(wl.k_prime, L_i) if wl.k_prime else 0)
 
 
 def score_kernel_bytes(wl):
@@ -126,8 +127,9 @@ class Clocks:
 
 
 def cpu_oracle_rate(wl, inp, n_queries, min_seconds=0.0):
-    """Time the CPU oracle's MISA-dagger pass over a sample of queries (cycling
-    through the batch until both n_queries and min_seconds are reached)."""
+    """Time the CPU oracle's MISA-dagger pass (plain MISA when the workload has no
+    k') over a sample of queries, cycling through the batch until both n_queries
+    and min_seconds are reached."""
     from oracle import misa_oracle as O
     try:
         from threadpoolctl import threadpool_info
@@ -144,7 +146,10 @@ def cpu_oracle_rate(wl, inp, n_queries, min_seconds=0.0):
         Li = int(inp.q_pos[i]) + 1
         K = O.seq_keys(inp.keys, inp.scale, wl.key_dtype, s, Li)
         q, w = O.query_arrays(inp.q, inp.w, i)
-        O.misa_dagger_query(q, w, K, Li, wl.B, wl.h, wl.k_prime, wl.k)
+        if wl.k_prime:
+            O.misa_dagger_query(q, w, K, Li, wl.B, wl.h, wl.k_prime, wl.k)
+        else:
+            O.misa_query(q, w, K, Li, wl.B, wl.h, wl.k)
         work += work_per_query(wl, Li)
     dt = time.perf_counter() - t0
     return work / dt, done / dt, dt, cores, done
@@ -172,7 +177,8 @@ def run_reference(args, wl):
         "config": config_block(wl, l2="n/a (CPU)"),
         "queries_per_s": float(np.mean(qps)),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"1 query per step (sequence 0 of {wl.name}), full MISA-dagger pass in numpy fp64"},
+                         "sample": f"1 query per step (first query of {wl.name}), full "
+                                   f"{'MISA-dagger' if wl.k_prime else 'MISA'} pass in numpy fp64"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -267,10 +273,10 @@ def main():
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill tensor-core context figures")
     args = ap.parse_args()
     wl = G.WORKLOADS[args.workload]
-    assert wl.k_prime is not None and wl.mode == "decode", "the bench step is the MISA-dagger decode step"
     if args.impl == "reference":
         run_reference(args, wl)
         return
+    assert wl.k_prime is not None and wl.mode == "decode", "the bench step is the MISA-dagger decode step"
 
     import torch
     import torch.distributed as dist
