@@ -33,6 +33,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstring>
 
 #include "frag.cuh"
 #include "internal.h"
@@ -46,15 +47,6 @@ constexpr int UM_N = 256;                 // query-head columns per tile
 constexpr int EPI_WARPS = 8;                // two per tensor-memory lane quarter
 constexpr int UM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr int B_BYTES = 65536;            // Q' tile: 256 x 128 bf16, or two e4m3 terms
-
-template <bool FP8>
-struct UCfg {
-  static constexpr int ROW = FP8 ? 128 : 256;           // key bytes per token
-  static constexpr int A_BYTES = UM_M * ROW;            // one key tile
-  static constexpr int STAGES = FP8 ? 8 : 4;
-  static constexpr int KSTEPS = FP8 ? 4 : 8;            // MMAs per term and tile (K = 32 / 16)
-  static constexpr int TERMS = FP8 ? 2 : 1;
-};
 
 struct UmmaShared {
   alignas(16) float wcol[UM_N];     // weight of every column (0 for padding); read as float4
@@ -70,10 +62,29 @@ struct UmmaShared {
   int q_lenp[UM_N];                 // prefix length if the query belongs to the current pass, else 0
 };
 
-template <bool FP8>
-constexpr int umma_smem_bytes() {
-  return 1024 /* alignment slack */ + UCfg<FP8>::STAGES * UCfg<FP8>::A_BYTES + B_BYTES + (int)sizeof(UmmaShared);
-}
+constexpr int SMEM_OPTIN = 232448;  // 227 KB of shared memory per CTA (opt-in maximum)
+
+template <bool FP8, int HPQ>
+struct UCfg {
+  static constexpr int ROW = FP8 ? 128 : 256;           // key bytes per token
+  static constexpr int A_BYTES = UM_M * ROW;            // one key tile
+  static constexpr int KSTEPS = FP8 ? 4 : 8;            // MMAs per term and tile (K = 32 / 16)
+  static constexpr int TERMS = FP8 ? 2 : 1;
+  // With 8 or 16 queries per half of the columns (HPQ = 16 or 8, the routed
+  // case) score tiles leave through TMA stores: every epilogue warp stages its
+  // 32 tokens x QH queries in two private buffers.  With fewer queries a
+  // warp writes at most 4 scores per tile and plain stores are cheaper than
+  // small TMA boxes; with 32 (HPQ = 4) the staging would not fit.
+  static constexpr int QH = (UM_N / 2) / HPQ;
+  static constexpr bool TMA_OUT = QH >= 8 && QH <= 16;
+  static constexpr int OUT_BUF = TMA_OUT ? 32 * QH * 4 : 0;  // bytes of one staging buffer
+  static constexpr int FIXED = 1024 /* alignment slack */ + B_BYTES + 2 * EPI_WARPS * OUT_BUF + (int)sizeof(UmmaShared);
+  static constexpr int STAGES_MAX = FP8 ? 8 : 4;
+  static constexpr int STAGES =
+      (SMEM_OPTIN - FIXED) / A_BYTES < STAGES_MAX ? (SMEM_OPTIN - FIXED) / A_BYTES : STAGES_MAX;
+  static constexpr int SMEM = FIXED + STAGES * A_BYTES;
+  static_assert(STAGES >= 2 && SMEM <= SMEM_OPTIN, "shared memory layout");
+};
 
 // ---- the kernel -----------------------------------------------------------
 
@@ -81,15 +92,17 @@ constexpr int umma_smem_bytes() {
 // [item0, item1).  A group holds QPT = 256 / HPQ consecutive queries.
 template <bool FP8, int HPQ>
 __global__ void __maxnreg__(128)
-    score_umma_kernel(const __grid_constant__ CUtensorMap kmap, CacheView c, QueryView qv, const int32_t *heads,
-                      int h, float *scores, long long ld, int n_tiles, long long n_items) {
-  using Cfg = UCfg<FP8>;
+    score_umma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap omap,
+                      int out_tma, CacheView c, QueryView qv, const int32_t *heads, int h, float *scores,
+                      long long ld, int n_tiles, long long n_items) {
+  using Cfg = UCfg<FP8, HPQ>;
   constexpr int QPT = UM_N / HPQ;
   extern __shared__ uint8_t um_raw[];
   uint8_t *base = um_raw + ((1024u - (smem_addr(um_raw) & 1023u)) & 1023u);  // 1024-aligned (swizzle atoms)
   uint8_t *a_smem = base;                                    // STAGES x A_BYTES (1024-aligned each)
   uint8_t *b_smem = base + Cfg::STAGES * Cfg::A_BYTES;       // B_BYTES
-  UmmaShared &sh = *reinterpret_cast<UmmaShared *>(b_smem + B_BYTES);
+  float *out_smem = reinterpret_cast<float *>(b_smem + B_BYTES);  // 2 x EPI_WARPS staging buffers
+  UmmaShared &sh = *reinterpret_cast<UmmaShared *>(b_smem + B_BYTES + 2 * EPI_WARPS * Cfg::OUT_BUF);
   volatile int *abort = &sh.abort;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = qv.H;
@@ -123,6 +136,7 @@ __global__ void __maxnreg__(128)
 
   // pipeline counters (same sequence of tiles in every role)
   uint32_t it_load = 0, it_mma = 0, j_mma = 0, j_epi = 0;
+  uint32_t ob = 0;  // epilogue: staging buffer of the next TMA store
   uint32_t last_fill_parity[8];
 #pragma unroll
   for (int s = 0; s < 8; ++s) last_fill_parity[s] = 2;  // 2: never filled
@@ -282,11 +296,41 @@ __global__ void __maxnreg__(128)
         const int col0 = (e / 4) * (UM_N / 2);  // its half of the columns
         const int r = quarter * 32 + lane;
         const float4 *wv = reinterpret_cast<const float4 *>(sh.wcol + col0);
+        // TMA stores of whole [QH queries x 32 tokens] boxes, when every
+        // query of this warp's half belongs to this pass (tokens past a
+        // query's prefix are written too; they are unspecified)
+        const int qa = col0 / HPQ;  // first query of the half
+        bool tma_ok = false;
+        if constexpr (Cfg::TMA_OUT) {
+          if (out_tma) {
+            tma_ok = true;
+            for (int x = 0; x < Cfg::QH; ++x) {
+              const int s2 = sh.q_seq[qa + x];
+              tma_ok &= (s2 == seq || s2 < 0);
+            }
+          }
+        }
+        // e4m3 token scales are loaded one tile ahead, so that their latency
+        // hides behind a tile of epilogue work instead of stalling the stores
+        const float *scale_row = FP8 ? c.scale + (size_t)seq * c.L_cap : nullptr;
+        float st_next = (FP8 && tau0 < t_end && tau0 * UM_M + r < c.L_cap) ? __ldg(scale_row + tau0 * UM_M + r) : 1.f;
         for (int tau = tau0; tau < t_end; ++tau, ++j_epi) {
           const int buf = j_epi & 1;
           const int t = tau * UM_M + r;
-          const float st_scale = (FP8 && t < c.L_cap) ? __ldg(c.scale + (size_t)seq * c.L_cap + t) : 1.f;
+          const float st_scale = st_next;
+          if (FP8 && tau + 1 < t_end) st_next = t + UM_M < c.L_cap ? __ldg(scale_row + t + UM_M) : 1.f;
           float *out_t = scores + (size_t)g * QPT * ld + t;  // row of query g*QPT + ql at + ql*ld
+          float *stg = out_smem + (e * 2 + (int)ob) * (Cfg::OUT_BUF / 4);  // [QH][32]
+          if (tma_ok) {  // the store that last read this buffer is done reading it
+            if (lane == 0) umma::bulk_wait_read<1>();
+            __syncwarp();
+          }
+          auto emit = [&](int ql, float x) {
+            if (tma_ok)
+              stg[(ql - qa) * 32 + lane] = x;
+            else if (t < sh.q_lenp[ql])
+              out_t[(size_t)ql * ld] = x;
+          };
           if (!umma::wait_bar(&sh.tfull[buf], (j_epi >> 1) & 1, abort, c)) break;
           umma::fence_after();
           const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * UM_N + col0;
@@ -320,15 +364,13 @@ __global__ void __maxnreg__(128)
                   float sum = 0.f;
 #pragma unroll
                   for (int x = 0; x < PPQ; ++x) sum += part[qc * PPQ + x];
-                  const int ql = (col0 + cb) / HPQ + qc;
-                  if (t < sh.q_lenp[ql]) out_t[(size_t)ql * ld] = sum * st_scale;
+                  emit((col0 + cb) / HPQ + qc, sum * st_scale);
                 }
               } else {
 #pragma unroll
                 for (int x = 0; x < 8; ++x) acc += part[x];
                 if (((col0 + cb + 32) % HPQ) == 0) {
-                  const int ql = (col0 + cb) / HPQ;
-                  if (t < sh.q_lenp[ql]) out_t[(size_t)ql * ld] = acc * st_scale;
+                  emit((col0 + cb) / HPQ, acc * st_scale);
                   acc = 0.f;
                 }
               }
@@ -337,6 +379,15 @@ __global__ void __maxnreg__(128)
           umma::fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.tempty[buf]);
+          if (tma_ok) {
+            umma::fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              umma::tma_store_2d(&omap, smem_addr(stg), tau * UM_M + quarter * 32, g * QPT + qa);
+              umma::bulk_commit();
+            }
+            ob ^= 1u;
+          }
         }
       }
       __syncthreads();  // every role is done with this pass
@@ -354,6 +405,7 @@ __global__ void __maxnreg__(128)
     const uint32_t jl = j_mma - 1;  // the last committed accumulator buffer
     umma::wait_bar(&sh.tfull[jl & 1], (jl >> 1) & 1, abort, c);
   }
+  if (warp >= 2 && lane == 0) umma::bulk_wait_all();  // score stores complete, staging free
   umma::fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -367,7 +419,8 @@ __global__ void __maxnreg__(128)
 template <bool FP8, int HPQ>
 cudaError_t launch_hpq(const CUtensorMap &map, const CacheView &c, const QueryView &q, const int32_t *heads, int h,
                        float *scores, long long ld, cudaStream_t s) {
-  constexpr int SMEM = umma_smem_bytes<FP8>();
+  using Cfg = UCfg<FP8, HPQ>;
+  constexpr int SMEM = Cfg::SMEM;
   struct Tag {};
   // the attribute call's status, cached per device (+1 so that 0 means unset)
   const int st = cached_per_device<Tag>([] {
@@ -380,8 +433,13 @@ cudaError_t launch_hpq(const CUtensorMap &map, const CacheView &c, const QueryVi
   const int n_tiles = cdiv(c.L_cap, UM_M);
   const long long n_items = (long long)n_groups * n_tiles;
   const int grid = (int)std::min<long long>(device_sms(), n_items);
-  return launch_kernel(score_umma_kernel<FP8, HPQ>, dim3(grid), dim3(UM_THREADS), SMEM, s, map, c, q, heads, h, scores,
-                    ld, n_tiles, n_items);
+  CUtensorMap omap;
+  memset(&omap, 0, sizeof(omap));
+  const int out_tma =
+      Cfg::TMA_OUT && umma::make_map_f32_rows(&omap, scores, (unsigned long long)c.L_cap, (unsigned long long)q.n_q,
+                                              (unsigned long long)ld, 32, Cfg::TMA_OUT ? Cfg::QH : 1);
+  return launch_kernel(score_umma_kernel<FP8, HPQ>, dim3(grid), dim3(UM_THREADS), SMEM, s, map, omap, out_tma, c, q,
+                       heads, h, scores, ld, n_tiles, n_items);
 }
 
 }  // namespace
@@ -447,6 +505,19 @@ bool make_map_2d(CUtensorMap *map, const void *base, bool u8, unsigned long long
   return enc(map, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base),
              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_f32_rows(CUtensorMap *map, const float *base, unsigned long long cols, unsigned long long rows,
+                       unsigned long long ld, int box_x, int box_rows) {
+  EncodeTiled enc = encode_fn();
+  if (!enc || (reinterpret_cast<uintptr_t>(base) & 15u) || (ld * sizeof(float)) % 16 != 0) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(ld * sizeof(float))};
+  const cuuint32_t box[2] = {(cuuint32_t)box_x, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace umma

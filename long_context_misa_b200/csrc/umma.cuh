@@ -67,6 +67,24 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
       : "memory");
 }
+// TMA tile store from shared memory (bulk-group completion): box of the map at
+// element coordinates (x, y); elements outside the tensor are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until at most N of this thread's bulk groups still read shared memory
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// wait until all of this thread's bulk groups are complete
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// generic-proxy shared-memory writes become visible to the async proxy (TMA)
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // Bounded wait shared by all roles: false once this CTA has given up (here or
 // in another role); a timeout records MISA_DEV_WAIT_TIMEOUT.
@@ -88,6 +106,11 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
 // boxes of box_x elements x box_rows rows); false if the driver entry point
 // or the encoding is unavailable.
 bool make_map_2d(CUtensorMap *map, const void *base, bool u8, unsigned long long rows, int box_x, int box_rows);
+// Host: a 2-D fp32 tensor map over rows of `cols` elements, `ld` elements
+// apart, no swizzle, boxes of box_x x box_rows; false if unavailable or if
+// the base or the row pitch is not 16-byte aligned.
+bool make_map_f32_rows(CUtensorMap *map, const float *base, unsigned long long cols, unsigned long long rows,
+                       unsigned long long ld, int box_x, int box_rows);
 bool encoder_available();
 
 }  // namespace umma

@@ -106,7 +106,13 @@ def debug_fail_next(n: int) -> None:
 
 
 def debug_time_scoring(start=None, stop=None) -> None:
-    """Bracket every scoring kernel with these torch.cuda.Event objects (None, None: off)."""
+    """Bracket every scoring kernel with these torch.cuda.Event objects (None, None: off).
+
+    An event not yet created (never recorded) is recorded once here so that
+    it has a CUDA event handle to pass."""
+    for e in (start, stop):
+        if e is not None and not e.cuda_event:
+            e.record()
     _lib.misa_debug_time_scoring(None if start is None else start.cuda_event,
                                  None if stop is None else stop.cuda_event)
 

@@ -5,10 +5,12 @@ Usage (one GPU):  python -m long_context_misa_b200.report [--workloads NAME ...]
 For every workload of ``inputs.WORKLOADS`` at full size: the MISA call
 (route + routed score + top-k; MISA-dagger through ``dagger_topk`` where the
 workload has a k') and the dense DSA indexer, timed with CUDA events around
-the calls (median of 5, L2 flushed before each), the throughput in queries/s
-and scored head*tokens/s, the fraction of the roofline the workload is bound
-by (key bytes against the measured copy bandwidth for decode, useful tensor
-flops against the measured bf16 peak for prefill), and the recall and IoU of
+the calls (median of 5, L2 flushed before each), the token-scoring kernels' own
+durations (routed with k' or k, and dense), the throughput in queries/s and
+scored head*tokens/s, the fraction of the roofline the workload is bound by
+(key bytes against the measured copy bandwidth for decode, useful tensor
+flops against the measured bf16 peak for prefill) for the whole call and for
+each scorer, and the recall and IoU of
 MISA's final selection against the dense DSA selection (for MISA-dagger also
 those of the routed pass alone cut to k).  Prints a markdown table.  The CPU
 oracle's rate on the same workloads comes from the throughput script's
@@ -49,6 +51,24 @@ def _timed(fn, flush):
         if it >= 2:
             ts.append(a.elapsed_time(b))
     return float(np.median(ts)), out
+
+
+def _scorer_ms(fn, flush):
+    """Median duration of the token-scoring kernel inside fn(), read from the
+    library's scoring event hook."""
+    ts = []
+    for it in range(7):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()  # creates the events; the library records them again around the kernel
+        b.record()
+        M.debug_time_scoring(a, b)
+        flush()
+        fn()
+        torch.cuda.synchronize()
+        M.debug_time_scoring(None, None)
+        if it >= 2:
+            ts.append(a.elapsed_time(b))
+    return float(np.median(ts))
 
 
 def overlap(sel, ref):
@@ -104,33 +124,43 @@ def main():
         torch.cuda.synchronize()
         t_misa, sel = _timed(misa, flush)
         t_dense, ref = _timed(dense, flush)
+        heads = M.route_heads(cache, qs, wl.h, ws=ws)
+        k_route = wl.k_prime or wl.k
+        s_misa = _scorer_ms(lambda: M.score_topk(cache, qs, heads, k_route, ws=ws), flush)
+        s_dense = _scorer_ms(dense, flush)
         assert cache.device_status() == 0
         work = float((wl.h * li + wl.H * M_i + (wl.H * np.minimum(wl.k_prime, li) if wl.k_prime else 0)).sum())
         row_bytes = wl.d * (1 if wl.key_dtype == "fp8" else 2) + (4 if wl.key_dtype == "fp8" else 0)
         if wl.mode == "decode":
             key_bytes = float(li.sum()) * row_bytes
-            frac = key_bytes / (t_misa * 1e-3) / 1e9 / hbm
-            bound = f"HBM {frac:.2f} (whole call)"
+            q_bytes = wl.n_q * wl.d * 2.0
+            call = key_bytes / (t_misa * 1e-3) / 1e9 / hbm
+            sm = (key_bytes + q_bytes * wl.h) / (s_misa * 1e-3) / 1e9 / hbm
+            sd = (key_bytes + q_bytes * wl.H) / (s_dense * 1e-3) / 1e9 / hbm
+            bound = f"HBM: call {call:.2f}, routed scorer {sm:.2f}, dense scorer {sd:.2f}"
         else:
             flops = 2.0 * wl.d * (wl.h * float(li.sum()) + wl.H * float(M_i.sum()))
-            frac = flops / (t_misa * 1e-3) / 1e12 / tflops
-            bound = f"tensor {frac:.2f} (whole call)"
+            call = flops / (t_misa * 1e-3) / 1e12 / tflops
+            sm = 2.0 * wl.d * wl.h * float(li.sum()) / (s_misa * 1e-3) / 1e12 / tflops
+            sd = 2.0 * wl.d * wl.H * float(li.sum()) / (s_dense * 1e-3) / 1e12 / tflops
+            bound = f"tensor: call {call:.2f}, routed scorer {sm:.2f}, dense scorer {sd:.2f}"
         ref_np = ref.cpu().numpy()
         rec = "%.3f / %.3f" % overlap(sel.cpu().numpy(), ref_np)
         if wl.k_prime:  # the routed pass alone, cut to k
             plain = M.score_topk(cache, qs, M.route_heads(cache, qs, wl.h, ws=ws), wl.k, ws=ws)
             rec += " (routed only: %.3f / %.3f)" % overlap(plain.cpu().numpy(), ref_np)
-        rows.append((name, wl.n_q, t_misa, t_dense, wl.n_q / (t_misa * 1e-3), work / (t_misa * 1e-3), bound, rec))
+        rows.append((name, wl.n_q, t_misa, t_dense, s_misa, s_dense, wl.n_q / (t_misa * 1e-3),
+                     work / (t_misa * 1e-3), bound, rec))
         del cache, qs, ws
         torch.cuda.empty_cache()
         print(f"done {name}", flush=True)
 
     print(f"\npeaks: {hbm} GB/s, {tflops} TFLOP/s ({src})\n")
-    print("| workload | queries | MISA call ms | dense DSA ms | MISA queries/s | MISA head*tokens/s | of roofline | "
-          "recall / IoU vs dense |")
-    print("|---|---|---|---|---|---|---|---|")
-    for name, nq, tm, td, qps, hts, bound, rec in rows:
-        print(f"| {name} | {nq} | {tm:.3f} | {td:.3f} | {qps:.3e} | {hts:.3e} | {bound} | {rec} |")
+    print("| workload | queries | MISA call ms | dense DSA ms | routed / dense scorer ms | MISA queries/s | "
+          "MISA head*tokens/s | of roofline | recall / IoU vs dense |")
+    print("|---|---|---|---|---|---|---|---|---|")
+    for name, nq, tm, td, sm, sd, qps, hts, bound, rec in rows:
+        print(f"| {name} | {nq} | {tm:.3f} | {td:.3f} | {sm:.3f} / {sd:.3f} | {qps:.3e} | {hts:.3e} | {bound} | {rec} |")
 
 
 if __name__ == "__main__":

@@ -29,6 +29,9 @@ CASES = {
     "fp8_prefill_umma": W["long_prefill_128k"].scaled(L=3000, n_q=96, B=100, k=33),
     # query groups that span two sequences (two passes over different keys)
     "bf16_prefill_2seq": W["causal_prefill"].scaled(n_seq=2, L=1300, n_q=80, k=40),
+    # score rows whose pitch is not a multiple of 16 bytes (plain stores, no
+    # TMA store) and a last query group cut short by n_q
+    "bf16_prefill_odd": W["causal_prefill"].scaled(L=1501, n_q=100, k=37),
 }
 
 
