@@ -31,6 +31,12 @@
 // filter_kernel (few long rows: decode): many CTAs per row copy the elements
 //   at or above d0 into a per-row list, so that the one CTA per row above
 //   reads about k + |d0| entries instead of the whole row.
+// Tensor-core prefill rows come without a histogram.  sample_thr_kernel
+//   reads a sample of each row and writes a bound below its k-th largest key
+//   (with high probability); filter_thr_kernel lists the elements at or above
+//   the bound; the staged selection counts the list itself (OWN).  A row whose
+//   list came out short or overfull is counted and selected from its whole
+//   score row instead, so the result never depends on the sample.
 #include <algorithm>
 
 #include "internal.h"
@@ -651,6 +657,7 @@ __global__ void __launch_bounds__(FILT_T) filter_kernel(CacheView c, QueryView q
   __syncthreads();
   const Boundary bd = sbd;
   if (!bd.listable()) return;  // uniform
+  const uint32_t d0 = bd.d0;
   uint2 *lrow = list + (size_t)row * list_cap;
   for (int base = p0; base < p1; base += FILT_T * FU) {
     if (base != p0) {
@@ -665,7 +672,7 @@ __global__ void __launch_bounds__(FILT_T) filter_kernel(CacheView c, QueryView q
     for (int u = 0; u < FU; ++u) {
       const int p = base + u * FILT_T + threadIdx.x;
       key[u] = ordered_key(sv[u]);
-      n += (p < p1 && (key[u] >> HIST_SHIFT) >= bd.d0) ? 1u : 0u;
+      n += (p < p1 && (key[u] >> HIST_SHIFT) >= d0) ? 1u : 0u;
     }
     uint32_t inc = n;
 #pragma unroll
@@ -681,9 +688,88 @@ __global__ void __launch_bounds__(FILT_T) filter_kernel(CacheView c, QueryView q
 #pragma unroll
     for (int u = 0; u < FU; ++u) {
       const int p = base + u * FILT_T + threadIdx.x;
-      if (p < p1 && (key[u] >> HIST_SHIFT) >= bd.d0) {
+      if (p < p1 && (key[u] >> HIST_SHIFT) >= d0) {
         if (slot < (uint32_t)list_cap) lrow[slot] = make_uint2(key[u], (uint32_t)p);
         ++slot;
+      }
+    }
+  }
+}
+
+// Tensor-core prefill rows (16-byte aligned rows): every CTA streams a chunk
+// of one row with 16-byte loads, eight per thread in flight, and appends the
+// elements whose key is at least thr[row] (the sampled bound) to the row's
+// list (list_cnt zeroed beforehand; it counts past list_cap).
+constexpr int FT_T = 256;
+constexpr int FT_V = 8;  // float4 loads per thread and sweep
+__global__ void __launch_bounds__(FT_T) filter_thr_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
+                                                          const uint32_t *thr, uint2 *list, uint32_t *list_cnt,
+                                                          int list_cap, int chunk) {
+  const int row = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int p0 = blockIdx.x * chunk;
+  const int pl = min(c.L_cap, p0 + chunk);  // 16-byte loads below pl stay inside the row (ld % 4 == 0)
+  const float *srow = scores + (size_t)row * ld;
+  float4 v[FT_V];
+#pragma unroll
+  for (int u = 0; u < FT_V; ++u) {
+    const int p = p0 + (u * FT_T + (int)threadIdx.x) * 4;
+    v[u] = p < pl ? __ldg(reinterpret_cast<const float4 *>(srow + p)) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  int s;
+  const int Li = query_prefix(c, qv, row, &s);
+  if (p0 >= Li) return;  // uniform over the CTA
+  const int p1 = min(Li, pl);
+  // key >= bound as a float compare (the key map is monotonic; at worst -0
+  // passes a +0 bound, an extra entry the selection sorts out); bound 0 takes all
+  const uint32_t bound = __ldg(thr + row);
+  const bool all = bound == 0u;
+  const float tau = __uint_as_float((bound & 0x80000000u) ? (bound & 0x7FFFFFFFu) : ~bound);
+  uint2 *lrow = list + (size_t)row * list_cap;
+  for (int base = p0; base < p1; base += FT_T * 4 * FT_V) {
+    if (base != p0) {
+#pragma unroll
+      for (int u = 0; u < FT_V; ++u) {
+        const int p = base + (u * FT_T + (int)threadIdx.x) * 4;
+        v[u] = p < p1 ? __ldg(reinterpret_cast<const float4 *>(srow + p)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    uint32_t n = 0;
+    const bool full = base + FT_T * 4 * FT_V <= p1;  // uniform: no element of this sweep past the prefix
+    if (full) {
+#pragma unroll
+      for (int u = 0; u < FT_V; ++u)
+        n += (all || v[u].x >= tau) + (all || v[u].y >= tau) + (all || v[u].z >= tau) + (all || v[u].w >= tau);
+    } else {
+#pragma unroll
+      for (int u = 0; u < FT_V; ++u) {
+        const int p = base + (u * FT_T + (int)threadIdx.x) * 4;
+        n += (p < p1 && (all || v[u].x >= tau)) + (p + 1 < p1 && (all || v[u].y >= tau)) +
+             (p + 2 < p1 && (all || v[u].z >= tau)) + (p + 3 < p1 && (all || v[u].w >= tau));
+      }
+    }
+    uint32_t inc = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += x;
+    }
+    const uint32_t tot = __shfl_sync(0xffffffffu, inc, 31);
+    if (tot == 0) continue;  // warp-uniform
+    uint32_t slot = 0;
+    if (lane == 31) slot = atomicAdd(list_cnt + row, tot);
+    slot = __shfl_sync(0xffffffffu, slot, 31) + inc - n;
+    if (n == 0) continue;
+#pragma unroll
+    for (int u = 0; u < FT_V; ++u) {
+      const int p = base + (u * FT_T + (int)threadIdx.x) * 4;
+      const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (p + e < p1 && (all || f[e] >= tau)) {
+          if (slot < (uint32_t)list_cap) lrow[slot] = make_uint2(ordered_key(f[e]), (uint32_t)(p + e));
+          ++slot;
+        }
       }
     }
   }
@@ -759,6 +845,8 @@ struct FastShared {
   uint32_t n_out;
 };
 constexpr int D0CAP = 6144;  // boundary-bin elements compacted in shared memory
+// bitmap words, rounded so that the arrays after it stay 16-byte aligned
+__host__ __device__ __forceinline__ int bm_words(int L_cap) { return (L_cap + 127) / 128 * 4; }
 
 // One whole warp: boundary from the unpadded histogram in shared memory.
 __device__ __forceinline__ Boundary warp_boundary_plain_smem(const uint32_t *h, int k) {
@@ -805,9 +893,86 @@ __device__ __forceinline__ Boundary warp_boundary_plain_smem(const uint32_t *h, 
   return b;
 }
 
+// Sampled boundary bound (tensor-core prefill, where the scoring kernel
+// builds no histogram): one CTA per row counts the top 11 key bits of a
+// sample of the row -- the whole row up to SMP_N elements, else SMP_BLOCKS
+// blocks of 32 consecutive tokens (one 128-byte line each; scattered single
+// sectors read slowly from HBM) spread evenly over the prefix -- and writes
+// thr[row] from the want-th largest sampled element.  want is the sample's
+// expected share of the top k, plus three standard deviations of a count
+// whose 32-token blocks move together, plus 8:
+// the elements at or above thr[row] then number at least k with high
+// probability.  A whole-row sample takes want = min(k, L_i), which is exact.
+// thr[row] is a key bound: the want-th largest sampled key cut to its top 22
+// bits (boundary bin, then the next 11 bits inside it); 0 takes every
+// element.
+constexpr int SMP_T = 256;
+constexpr int SMP_BL = 32;  // tokens per sample block
+constexpr int SMP_BLOCKS = 256;
+constexpr int SMP_N = SMP_BLOCKS * SMP_BL;
+__global__ void __launch_bounds__(SMP_T) sample_thr_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
+                                                           int k, uint32_t *thr) {
+  __shared__ uint32_t hs[RB];
+  __shared__ Boundary sb;
+  const int row = blockIdx.x;
+  int s;
+  const int Li = query_prefix(c, qv, row, &s);
+  for (int b = threadIdx.x; b < RB; b += SMP_T) hs[b] = 0;
+  __syncthreads();
+  const float *srow = scores + (size_t)row * ld;
+  const bool whole = Li <= SMP_N;
+  const int n = whole ? max(Li, 0) : SMP_N;
+  // all of this thread's samples are requested before any is counted
+  constexpr int PER = SMP_N / SMP_T;
+  float v[PER];
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int i = u * SMP_T + (int)threadIdx.x;
+    int p = i;
+    if (!whole) p = (int)((long long)(i / SMP_BL) * (Li - SMP_BL) / (SMP_BLOCKS - 1)) + (i % SMP_BL);
+    v[u] = i < n ? __ldg(srow + p) : 0.f;
+  }
+#pragma unroll
+  for (int u = 0; u < PER; ++u)
+    if (u * SMP_T + (int)threadIdx.x < n) atomicAdd(&hs[ordered_key(v[u]) >> HIST_SHIFT], 1u);
+  __syncthreads();
+  uint32_t want = (uint32_t)min(k, max(Li, 0));
+  if (!whole) {
+    const double r = (double)k * SMP_N / Li;
+    want = (uint32_t)min(2.0 * SMP_N, ceil(r + 3.0 * sqrt((double)SMP_BL * r) + 8.0));
+  }
+  if (threadIdx.x < 32) {
+    const Boundary b = warp_boundary_plain_smem(hs, (int)want);
+    if (threadIdx.x == 0) sb = b;
+  }
+  __syncthreads();
+  const Boundary b = sb;
+  if (b.all_in) {
+    if (threadIdx.x == 0) thr[row] = 0u;
+    return;
+  }
+  // second level: the next 11 key bits of the samples inside the boundary bin
+  for (int x = threadIdx.x; x < RB; x += SMP_T) hs[x] = 0;
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int i = u * SMP_T + (int)threadIdx.x;
+    const uint32_t key = ordered_key(v[u]);
+    if (i < n && (key >> HIST_SHIFT) == b.d0) atomicAdd(&hs[(key >> 10) & (RB - 1)], 1u);
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const Boundary b2 = warp_boundary_plain_smem(hs, (int)(want - b.above));
+    if (threadIdx.x == 0) thr[row] = (b.d0 << HIST_SHIFT) | ((b2.all_in ? 0u : b2.d0) << 10);
+  }
+}
+
 // LIST: the filter kernel's list (key, token) of the row; else GATHER rows
-// (scores and candidate tokens, n_cols of each).
-template <bool LIST, bool ORDERED>
+// (scores and candidate tokens, n_cols of each).  OWN (with LIST): there is
+// no row histogram; the list holds the elements at or above a sampled bound,
+// and the kernel counts the listed keys itself -- or, when the list missed
+// (fewer than min(k, L_i) entries, or more than it holds), the whole row.
+template <bool LIST, bool ORDERED, bool OWN = false>
 __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryView qv, const float *scores,
                                                             long long ld, int n_cols, const int32_t *gather,
                                                             const uint32_t *row_hist, const uint2 *list,
@@ -818,7 +983,7 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
   uint8_t *data = fs_smem + sizeof(FastShared);  // 16-byte aligned (sizeof is a multiple of 16)
   const int data_bytes = LIST ? list_cap * 8 : n_cols * 8;
   uint32_t *bm = reinterpret_cast<uint32_t *>(data + data_bytes);
-  uint32_t *d0_key = bm + cdiv(c.L_cap, 32);                              // [D0CAP]
+  uint32_t *d0_key = bm + bm_words(c.L_cap);                              // [D0CAP]
   uint32_t *d0_tie = d0_key + D0CAP;                                       // [D0CAP]
   const uint2 *ent = reinterpret_cast<const uint2 *>(data);                // LIST
   const float *sc = reinterpret_cast<const float *>(data);                 // GATHER
@@ -826,15 +991,23 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
   const int row = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5;
 
+  int s;
+  const int Li = query_prefix(c, qv, row, &s);
+  const float *srow = scores + (size_t)row * ld;
   if (tid == 0) {
     mbar_init(&sh.bar, 1);
     fence_mbar_init();
-    const uint32_t bytes = RB * 4 + (LIST ? list_cap * 8 : n_cols * 8);
-    mbar_arrive_expect_tx(&sh.bar, bytes);
-    bulk_g2s(sh.rhist, row_hist + (size_t)row * RB, RB * 4, &sh.bar);
     if (LIST) {
-      bulk_g2s(data, list + (size_t)row * list_cap, list_cap * 8, &sh.bar);
+      // the listed entries only, rounded up to an even count (16-byte copies;
+      // list_cap is even)
+      const uint32_t n_copy = min(list_cnt[row], (uint32_t)list_cap);
+      const uint32_t ent_bytes = ((n_copy + 1u) & ~1u) * 8u;
+      mbar_arrive_expect_tx(&sh.bar, (OWN ? 0u : (uint32_t)RB * 4u) + ent_bytes);
+      if (!OWN) bulk_g2s(sh.rhist, row_hist + (size_t)row * RB, RB * 4, &sh.bar);
+      if (ent_bytes) bulk_g2s(data, list + (size_t)row * list_cap, ent_bytes, &sh.bar);
     } else {
+      mbar_arrive_expect_tx(&sh.bar, RB * 4 + n_cols * 8);
+      bulk_g2s(sh.rhist, row_hist + (size_t)row * RB, RB * 4, &sh.bar);
       bulk_g2s(data, scores + (size_t)row * ld, n_cols * 4, &sh.bar);
       bulk_g2s(data + n_cols * 4, gather + (size_t)row * n_cols, n_cols * 4, &sh.bar);
     }
@@ -843,8 +1016,6 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
     sh.n_out = 0;
   }
   const int lcnt = LIST ? min((int)list_cnt[row], list_cap) : 0;
-  int s;
-  const int Li = query_prefix(c, qv, row, &s);
   const int words = cdiv(Li, 32);
   for (int w = tid; w < words; w += FAST_T) bm[w] = 0;
   __syncthreads();  // barrier initialised, bitmap clear
@@ -873,13 +1044,23 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
     for (int p = tid; p < k; p += FAST_T) orow[p] = -1;
     return;
   }
+  bool list_ok = false;
+  if (OWN) {
+    const uint32_t cnt = list_cnt[row];
+    list_ok = cnt <= (uint32_t)list_cap && cnt >= (uint32_t)min(k, max(Li, 0));
+    for (int b = tid; b < RB; b += FAST_T) sh.rhist[b] = 0;
+    __syncthreads();
+    const int n = list_ok ? lcnt : max(Li, 0);
+    for (int i = tid; i < n; i += FAST_T)
+      atomicAdd(&sh.rhist[(list_ok ? ent[i].x : ordered_key(__ldg(srow + i))) >> HIST_SHIFT], 1u);
+    __syncthreads();
+  }
   if (warp == 0) {
     const Boundary b = warp_boundary_plain_smem(sh.rhist, k);
     if ((tid & 31) == 0) sh.bd = b;
   }
   __syncthreads();
   const Boundary bd = sh.bd;
-  const float *srow = scores + (size_t)row * ld;
 
   if (bd.kk > 0) {
     const uint32_t d0 = bd.d0;
@@ -887,7 +1068,7 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
     const bool whole = bd.all_in || need == bd.in0;
     // staged elements: (key, token, valid); a list row the filter skipped is
     // read from the global row instead (prefix rows: token = position)
-    const bool staged = !LIST || bd.listable();
+    const bool staged = OWN ? list_ok : (!LIST || bd.listable());
     auto each = [&](auto &&fn) {
       if (staged) {
         const int n = LIST ? lcnt : n_cols;
@@ -1007,23 +1188,23 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
 constexpr int SMEM_OPTIN_MAX = 227 * 1024;  // largest dynamic shared memory a CTA may opt into
 
 int fast_smem_bytes(bool list, int n_cols, int list_cap, int L_cap) {
-  return (int)sizeof(FastShared) + (list ? list_cap * 8 : n_cols * 8) + 4 * cdiv(L_cap, 32) + 8 * D0CAP;
+  return (int)sizeof(FastShared) + (list ? list_cap * 8 : n_cols * 8) + 4 * bm_words(L_cap) + 8 * D0CAP;
 }
 
-template <bool LIST, bool ORDERED = true>
+template <bool LIST, bool ORDERED = true, bool OWN = false>
 cudaError_t launch_select_smem(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
                                const int32_t *gather, const uint32_t *row_hist, const uint2 *list,
                                const uint32_t *list_cnt, int list_cap, int k, int32_t *out, cudaStream_t s) {
   constexpr int SMEM_MAX = SMEM_OPTIN_MAX;
   struct Tag {};
   const int st = cached_per_device<Tag>([] {
-    return 1 + (int)cudaFuncSetAttribute(select_smem_kernel<LIST, ORDERED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_MAX);
+    return 1 + (int)cudaFuncSetAttribute(select_smem_kernel<LIST, ORDERED, OWN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_MAX);
   });
   if (st != 1) return (cudaError_t)(st - 1);
   const int smem = fast_smem_bytes(LIST, n_cols, list_cap, c.L_cap);
-  return launch_kernel(select_smem_kernel<LIST, ORDERED>, dim3(q.n_q), dim3(FAST_T), smem, s, c, q, scores, ld, n_cols,
-                    gather, row_hist, list, list_cnt, list_cap, k, out);
+  return launch_kernel(select_smem_kernel<LIST, ORDERED, OWN>, dim3(q.n_q), dim3(FAST_T), smem, s, c, q, scores, ld,
+                       n_cols, gather, row_hist, list, list_cnt, list_cap, k, out);
 }
 
 // Zero n words (the histograms and list counters before a scoring pass); a
@@ -1082,27 +1263,45 @@ cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *sco
     return launch_select<false, false, true>(c, q, scores, ld, 0, nullptr, nullptr, nullptr, nullptr, 0, k, out, s);
   const int sms = device_sms();
   cudaError_t e = cudaSuccess;
-  if (!hist_ready) {
-    // wide pass over the scores: about 16K elements per CTA
-    const int per_row = cdiv(c.L_cap, 16384);
-    const int chunk = cdiv(cdiv(c.L_cap, per_row), HIST_T) * HIST_T;
-    e = launch_kernel(hist_kernel, dim3(cdiv(c.L_cap, chunk), q.n_q), dim3(HIST_T), 0, s, c, q, scores, ld, row_hist,
-                   chunk);
-    if (e != cudaSuccess) return e;
-  }
-  if (!list_mode)
-    return launch_select<false, false>(c, q, scores, ld, 0, nullptr, row_hist, nullptr, nullptr, 0, k, out, s);
   const int list_cap = k + TOPK_LIST_EXTRA;
   uint2 *list = static_cast<uint2 *>(list_ws);
+  const bool smem_list = 8LL * list_cap <= FAST_DATA_MAX && list_cap % 2 == 0 && aligned16(list) &&
+                         aligned16(row_hist) && fast_smem_bytes(true, 0, list_cap, c.L_cap) <= SMEM_OPTIN_MAX;
   // about two CTAs per SM over all rows (few rows) or at most 16K elements
   // per CTA (many rows), at least 4096 elements each
   const int per_row = max(1, min(cdiv(c.L_cap, 4096), max(2 * sms / q.n_q, cdiv(c.L_cap, 16384))));
   const int chunk = cdiv(cdiv(c.L_cap, per_row), FILT_T) * FILT_T;
-  e = launch_kernel(filter_kernel, dim3(cdiv(c.L_cap, chunk), q.n_q), dim3(FILT_T), 0, s, c, q, scores, ld, row_hist,
-                 list, list_cnt, list_cap, k, chunk);
+  const dim3 fgrid(cdiv(c.L_cap, chunk), q.n_q);
+  if (!hist_ready && smem_list && ld % 4 == 0 && aligned16(scores)) {
+    // no histogram: a sampled lower bound of each row's top-k keys (in the
+    // histogram's place), the elements at or above it listed, the list
+    // counted and selected in shared memory
+    uint32_t *thr = row_hist;
+    e = launch_kernel(sample_thr_kernel, dim3(q.n_q), dim3(SMP_T), 0, s, c, q, scores, ld, k, thr);
+    if (e != cudaSuccess) return e;
+    const int tchunk = 4 * FT_T * FT_V * 2;  // two sweeps per CTA
+    e = launch_kernel(filter_thr_kernel, dim3(cdiv(c.L_cap, tchunk), q.n_q), dim3(FT_T), 0, s, c, q, scores, ld, thr,
+                      list, list_cnt, list_cap, tchunk);
+    if (e != cudaSuccess) return e;
+    return ordered ? launch_select_smem<true, true, true>(c, q, scores, ld, 0, nullptr, thr, list, list_cnt, list_cap,
+                                                          k, out, s)
+                   : launch_select_smem<true, false, true>(c, q, scores, ld, 0, nullptr, thr, list, list_cnt,
+                                                           list_cap, k, out, s);
+  }
+  if (!hist_ready) {
+    // wide pass over the scores: about 16K elements per CTA
+    const int hper_row = cdiv(c.L_cap, 16384);
+    const int hchunk = cdiv(cdiv(c.L_cap, hper_row), HIST_T) * HIST_T;
+    e = launch_kernel(hist_kernel, dim3(cdiv(c.L_cap, hchunk), q.n_q), dim3(HIST_T), 0, s, c, q, scores, ld, row_hist,
+                      hchunk);
+    if (e != cudaSuccess) return e;
+  }
+  if (!list_mode)
+    return launch_select<false, false>(c, q, scores, ld, 0, nullptr, row_hist, nullptr, nullptr, 0, k, out, s);
+  e = launch_kernel(filter_kernel, fgrid, dim3(FILT_T), 0, s, c, q, scores, ld, row_hist, list, list_cnt,
+                    list_cap, k, chunk);
   if (e != cudaSuccess) return e;
-  if (8LL * list_cap <= FAST_DATA_MAX && list_cap % 2 == 0 && aligned16(list) && aligned16(row_hist) &&
-      fast_smem_bytes(true, 0, list_cap, c.L_cap) <= SMEM_OPTIN_MAX)
+  if (smem_list)
     return ordered
                ? launch_select_smem<true, true>(c, q, scores, ld, 0, nullptr, row_hist, list, list_cnt, list_cap, k,
                                                 out, s)

@@ -36,9 +36,10 @@ CASES = {
 
 
 def make(case, seed=0, ragged=True):
-    wl = CASES[case]
+    """Inputs of a named case, or of a Workload given directly."""
+    wl = CASES[case] if isinstance(case, str) else case
     inp = G.make_inputs(wl, seed)
-    if case.endswith("_2seq"):  # blocks of 20 queries alternate between the sequences
+    if isinstance(case, str) and case.endswith("_2seq"):  # blocks of 20 queries alternate between the sequences
         inp.q_seq = ((np.arange(wl.n_q) // 20) % 2).astype(np.int32)
     if ragged and wl.mode == "decode":
         inp.seq_len = (wl.L - 37 * np.arange(wl.n_seq)).astype(np.int32)
@@ -322,6 +323,52 @@ def test_topk_two_score_levels(L):
     pat = (np.arange(L) % 2).astype(np.int64)
     for k in (L // 2, L // 2 + 37):
         _tied_case(L, pat, k)
+
+
+# Prefill chunks over caches longer than 16K keys: tensor-core scoring, then
+# a sampled lower bound of each row's boundary bin, the elements above it
+# listed and selected; every query is checked.
+LONG_PREFILL = {
+    "bf16": W["causal_prefill"].scaled(L=20000, n_q=64, k=300),
+    "fp8": W["long_prefill_128k"].scaled(L=24000, n_q=72, B=256, k=500),
+}
+
+
+@pytest.mark.parametrize("dt", sorted(LONG_PREFILL))
+@pytest.mark.parametrize("kind", ["misa", "dense"])
+def test_long_prefill_topk(dt, kind):
+    ties = _score_case(LONG_PREFILL[dt], kind)
+    assert ties <= 4, ties
+
+
+def _tied_prefill(L, pattern, k):
+    """Prefill chunk over a bf16 cache whose keys take two values: the sampled
+    bound lists far more than a row holds, so every row falls back to counting
+    its whole score row; expected top-k from the oracle (ties to the lower
+    token index)."""
+    wl = W["causal_prefill"].scaled(L=L, n_q=64, k=k)
+    inp = G.make_inputs(wl, 5)
+    a, b = inp.keys[0, 0].copy(), inp.keys[0, 1].copy()
+    inp.keys[0] = np.where(pattern[:, None] == 1, b[None, :], a[None, :])
+    ref = Ref(inp)
+    cache, qs = to_device(inp, torch)
+    top = M.dense_score_topk(cache, qs, k).cpu().numpy()
+    for i in range(wl.n_q):
+        q, w, K, Li = ref.query(i)
+        d = O.dense_query(q, w, K, Li, k)
+        np.testing.assert_array_equal(top[i], d["topk"], err_msg=f"q{i}")
+    assert device_status(cache) == 0
+
+
+@pytest.mark.parametrize("k", [1, 700])
+def test_long_prefill_topk_all_scores_equal(k):
+    _tied_prefill(20000, np.zeros(20000, dtype=np.int64), k)
+
+
+def test_long_prefill_topk_two_score_levels():
+    L = 20000
+    pat = (np.arange(L) % 2).astype(np.int64)
+    _tied_prefill(L, pat, 8000)  # inside the upper level: ties by index
 
 
 def test_rerank_candidate_order_does_not_matter():
