@@ -906,7 +906,7 @@ __device__ __forceinline__ Boundary warp_boundary_plain_smem(const uint32_t *h, 
 // thr[row] is a key bound: the want-th largest sampled key cut to its top 22
 // bits (boundary bin, then the next 11 bits inside it); 0 takes every
 // element.
-constexpr int SMP_T = 256;
+constexpr int SMP_T = 512;
 constexpr int SMP_BL = 32;  // tokens per sample block
 constexpr int SMP_BLOCKS = 256;
 constexpr int SMP_N = SMP_BLOCKS * SMP_BL;
@@ -972,19 +972,21 @@ __global__ void __launch_bounds__(SMP_T) sample_thr_kernel(CacheView c, QueryVie
 // no row histogram; the list holds the elements at or above a sampled bound,
 // and the kernel counts the listed keys itself -- or, when the list missed
 // (fewer than min(k, L_i) entries, or more than it holds), the whole row.
+// stage_cap: list entries staged in shared memory (<= list_cap, even);
+// d0cap: boundary-bin elements compacted there.
 template <bool LIST, bool ORDERED, bool OWN = false>
 __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryView qv, const float *scores,
                                                             long long ld, int n_cols, const int32_t *gather,
                                                             const uint32_t *row_hist, const uint2 *list,
-                                                            const uint32_t *list_cnt, int list_cap, int k,
-                                                            int32_t *out) {
+                                                            const uint32_t *list_cnt, int list_cap, int stage_cap,
+                                                            int d0cap, int k, int32_t *out) {
   extern __shared__ __align__(16) uint8_t fs_smem[];
   FastShared &sh = *reinterpret_cast<FastShared *>(fs_smem);
   uint8_t *data = fs_smem + sizeof(FastShared);  // 16-byte aligned (sizeof is a multiple of 16)
-  const int data_bytes = LIST ? list_cap * 8 : n_cols * 8;
+  const int data_bytes = LIST ? stage_cap * 8 : n_cols * 8;
   uint32_t *bm = reinterpret_cast<uint32_t *>(data + data_bytes);
-  uint32_t *d0_key = bm + bm_words(c.L_cap);                              // [D0CAP]
-  uint32_t *d0_tie = d0_key + D0CAP;                                       // [D0CAP]
+  uint32_t *d0_key = bm + bm_words(c.L_cap);                              // [d0cap]
+  uint32_t *d0_tie = d0_key + d0cap;                                       // [d0cap]
   const uint2 *ent = reinterpret_cast<const uint2 *>(data);                // LIST
   const float *sc = reinterpret_cast<const float *>(data);                 // GATHER
   const int32_t *tk = reinterpret_cast<const int32_t *>(data + n_cols * 4);  // GATHER
@@ -999,8 +1001,8 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
     fence_mbar_init();
     if (LIST) {
       // the listed entries only, rounded up to an even count (16-byte copies;
-      // list_cap is even)
-      const uint32_t n_copy = min(list_cnt[row], (uint32_t)list_cap);
+      // stage_cap is even)
+      const uint32_t n_copy = min(list_cnt[row], (uint32_t)stage_cap);
       const uint32_t ent_bytes = ((n_copy + 1u) & ~1u) * 8u;
       mbar_arrive_expect_tx(&sh.bar, (OWN ? 0u : (uint32_t)RB * 4u) + ent_bytes);
       if (!OWN) bulk_g2s(sh.rhist, row_hist + (size_t)row * RB, RB * 4, &sh.bar);
@@ -1015,7 +1017,7 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
     sh.n_d0 = 0;
     sh.n_out = 0;
   }
-  const int lcnt = LIST ? min((int)list_cnt[row], list_cap) : 0;
+  const int lcnt = LIST ? min((int)list_cnt[row], stage_cap) : 0;
   const int words = cdiv(Li, 32);
   for (int w = tid; w < words; w += FAST_T) bm[w] = 0;
   __syncthreads();  // barrier initialised, bitmap clear
@@ -1047,7 +1049,7 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
   bool list_ok = false;
   if (OWN) {
     const uint32_t cnt = list_cnt[row];
-    list_ok = cnt <= (uint32_t)list_cap && cnt >= (uint32_t)min(k, max(Li, 0));
+    list_ok = cnt <= (uint32_t)stage_cap && cnt >= (uint32_t)min(k, max(Li, 0));
     for (int b = tid; b < RB; b += FAST_T) sh.rhist[b] = 0;
     __syncthreads();
     const int n = list_ok ? lcnt : max(Li, 0);
@@ -1085,7 +1087,7 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
         for (int i = tid; i < Li; i += FAST_T) fn(ordered_key(__ldg(srow + i)), i, true);
       }
     };
-    const bool compact = staged && !whole && bd.in0 <= (uint32_t)D0CAP;
+    const bool compact = staged && !whole && bd.in0 <= (uint32_t)d0cap;
     if (compact) {
       // 2. one pass, four elements per thread and step: mark everything above
       //    the boundary; compact the boundary bin's elements (key, tie) with
@@ -1136,7 +1138,7 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             if ((flags >> e) & 1) {
-              if (slot < (uint32_t)D0CAP) {
+              if (slot < (uint32_t)d0cap) {
                 d0_key[slot] = key[e];
                 d0_tie[slot] = POS_MAX - (uint32_t)t[e];
               }
@@ -1147,7 +1149,7 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
       }
       __syncthreads();
       // 3. threshold among the boundary bin's elements only, then their winners
-      const int nd = min((int)sh.n_d0, D0CAP);
+      const int nd = min((int)sh.n_d0, d0cap);
       uint32_t P_hi = d0 << HIST_SHIFT, M_hi = TOP_MASK, P_lo = 0, M_lo = 0;
       refine<true, FAST_T>(sh, P_hi, M_hi, P_lo, M_lo, need, bd.in0, [&](auto &&fn) {
         for (int x = tid; x < nd; x += FAST_T) fn(d0_key[x], d0_tie[x], true);
@@ -1187,24 +1189,26 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
 
 constexpr int SMEM_OPTIN_MAX = 227 * 1024;  // largest dynamic shared memory a CTA may opt into
 
-int fast_smem_bytes(bool list, int n_cols, int list_cap, int L_cap) {
-  return (int)sizeof(FastShared) + (list ? list_cap * 8 : n_cols * 8) + 4 * bm_words(L_cap) + 8 * D0CAP;
+int fast_smem_bytes(bool list, int n_cols, int stage_cap, int L_cap, int d0cap = D0CAP) {
+  return (int)sizeof(FastShared) + (list ? stage_cap * 8 : n_cols * 8) + 4 * bm_words(L_cap) + 8 * d0cap;
 }
 
 template <bool LIST, bool ORDERED = true, bool OWN = false>
 cudaError_t launch_select_smem(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
                                const int32_t *gather, const uint32_t *row_hist, const uint2 *list,
-                               const uint32_t *list_cnt, int list_cap, int k, int32_t *out, cudaStream_t s) {
+                               const uint32_t *list_cnt, int list_cap, int k, int32_t *out, cudaStream_t s,
+                               int stage_cap = -1, int d0cap = D0CAP) {
   constexpr int SMEM_MAX = SMEM_OPTIN_MAX;
+  if (stage_cap < 0) stage_cap = list_cap;
   struct Tag {};
   const int st = cached_per_device<Tag>([] {
     return 1 + (int)cudaFuncSetAttribute(select_smem_kernel<LIST, ORDERED, OWN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_MAX);
   });
   if (st != 1) return (cudaError_t)(st - 1);
-  const int smem = fast_smem_bytes(LIST, n_cols, list_cap, c.L_cap);
+  const int smem = fast_smem_bytes(LIST, n_cols, stage_cap, c.L_cap, d0cap);
   return launch_kernel(select_smem_kernel<LIST, ORDERED, OWN>, dim3(q.n_q), dim3(FAST_T), smem, s, c, q, scores, ld,
-                       n_cols, gather, row_hist, list, list_cnt, list_cap, k, out);
+                       n_cols, gather, row_hist, list, list_cnt, list_cap, stage_cap, d0cap, k, out);
 }
 
 // Zero n words (the histograms and list counters before a scoring pass); a
@@ -1283,10 +1287,14 @@ cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *sco
     e = launch_kernel(filter_thr_kernel, dim3(cdiv(c.L_cap, tchunk), q.n_q), dim3(FT_T), 0, s, c, q, scores, ld, thr,
                       list, list_cnt, list_cap, tchunk);
     if (e != cudaSuccess) return e;
+    // lists of up to 7168 entries and 1024 boundary-bin elements: two CTAs
+    // per SM (rows beyond take the whole-row path); larger k stages it all
+    const bool two = k <= 4096 && fast_smem_bytes(true, 0, 7168, c.L_cap, 1024) <= SMEM_OPTIN_MAX / 2 - 1024;
+    const int stage_cap = two ? 7168 : list_cap, d0cap = two ? 1024 : D0CAP;
     return ordered ? launch_select_smem<true, true, true>(c, q, scores, ld, 0, nullptr, thr, list, list_cnt, list_cap,
-                                                          k, out, s)
+                                                          k, out, s, stage_cap, d0cap)
                    : launch_select_smem<true, false, true>(c, q, scores, ld, 0, nullptr, thr, list, list_cnt,
-                                                           list_cap, k, out, s);
+                                                           list_cap, k, out, s, stage_cap, d0cap);
   }
   if (!hist_ready) {
     // wide pass over the scores: about 16K elements per CTA

@@ -1,6 +1,10 @@
 """Per-workload measurement report for the five synthetic workloads.
 
 Usage (one GPU):  python -m long_context_misa_b200.report [--workloads NAME ...]
+                  [--n-q N] [--no-dense]
+
+--n-q N keeps the first N queries of each workload (smaller captures of the
+same kernels for profilers); --no-dense skips the dense DSA calls.
 
 For every workload of ``inputs.WORKLOADS`` at full size: the MISA call
 (route + routed score + top-k; MISA-dagger through ``dagger_topk`` where the
@@ -89,6 +93,8 @@ def overlap(sel, ref):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--workloads", nargs="*", default=list(G.WORKLOADS))
+    ap.add_argument("--n-q", type=int, default=0)
+    ap.add_argument("--no-dense", action="store_true")
     args = ap.parse_args()
     hbm, tflops, src = _peaks()
     dev = torch.device("cuda")
@@ -102,6 +108,8 @@ def main():
     rows = []
     for name in args.workloads:
         wl = G.WORKLOADS[name]
+        if args.n_q and wl.mode == "prefill":
+            wl = wl.scaled(n_q=min(args.n_q, wl.n_q))
         inp = G.make_inputs(wl, 0)
         cache, qs = M.device_inputs(inp, dev)
         M.pool_keys(cache)
@@ -116,6 +124,8 @@ def main():
             return M.score_topk(cache, qs, heads, wl.k, ws=ws)
 
         def dense():
+            if args.no_dense:
+                return torch.full((wl.n_q, wl.k), -1, dtype=torch.int32, device=dev)
             return M.dense_score_topk(cache, qs, wl.k, ws=ws)
 
         for _ in range(2):
@@ -127,7 +137,7 @@ def main():
         heads = M.route_heads(cache, qs, wl.h, ws=ws)
         k_route = wl.k_prime or wl.k
         s_misa = _scorer_ms(lambda: M.score_topk(cache, qs, heads, k_route, ws=ws), flush)
-        s_dense = _scorer_ms(dense, flush)
+        s_dense = float("nan") if args.no_dense else _scorer_ms(dense, flush)
         assert cache.device_status() == 0
         work = float((wl.h * li + wl.H * M_i + (wl.H * np.minimum(wl.k_prime, li) if wl.k_prime else 0)).sum())
         row_bytes = wl.d * (1 if wl.key_dtype == "fp8" else 2) + (4 if wl.key_dtype == "fp8" else 0)
