@@ -393,23 +393,35 @@ def main():
         dense_ms.append(a.elapsed_time(b))
 
     # ---- end to end through the public API: pinned host inputs in, top-k out ----
-    h_keys = torch.from_numpy(last).pin_memory()
-    h_scale = new_scale.cpu().pin_memory()
-    h_q = torch.from_numpy(inp.q.view(np.int16)).pin_memory()
-    h_w = torch.from_numpy(inp.w).pin_memory()
-    h_pos = torch.from_numpy(inp.q_pos.copy()).pin_memory()
+    # The step's inputs (new keys and scales, positions, queries, weights) sit
+    # in one pinned host buffer laid out like one device buffer that the step
+    # reads through views: one host-to-device copy per step, one copy back.
+    parts = [("keys", torch.from_numpy(last)), ("scale", new_scale.cpu()), ("pos", torch.from_numpy(inp.q_pos.copy())),
+             ("q", torch.from_numpy(inp.q.view(np.int16))), ("w", torch.from_numpy(inp.w))]
+    offs, total = {}, 0
+    for name, t in parts:
+        offs[name] = total
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    h_in = torch.empty(total, dtype=torch.uint8).pin_memory()
+    d_in = torch.empty(total, dtype=torch.uint8, device=dev)
+
+    def view(buf, name, t):
+        n = t.numel() * t.element_size()
+        return buf[offs[name]:offs[name] + n].view(t.dtype).view(t.shape)
+
+    for name, t in parts:
+        view(h_in, name, t).copy_(t)
+    d_keys, d_scale, d_pos, d_q, d_w = (view(d_in, name, t) for name, t in parts)
+    qs_e2e = M.Queries(d_q, d_w, qs.q_seq, d_pos)
+    step_e2e = M.MisaDaggerDecode(cache, qs_e2e, wl.h, wl.k_prime, wl.k, d_keys, d_scale, d_pos)
     h_top = torch.empty(wl.n_q, wl.k, dtype=torch.int32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (h_keys, h_scale, h_q, h_w, h_pos))
+    h2d = sum(t.numel() * t.element_size() for _, t in parts)
     d2h = h_top.numel() * h_top.element_size()
 
     def e2e_body():
-        new_keys.copy_(h_keys, non_blocking=True)
-        new_scale.copy_(h_scale, non_blocking=True)
-        qs.q.copy_(h_q, non_blocking=True)
-        qs.w.copy_(h_w, non_blocking=True)
-        pos.copy_(h_pos, non_blocking=True)
-        step.run()
-        h_top.copy_(step.topk, non_blocking=True)
+        d_in.copy_(h_in, non_blocking=True)
+        step_e2e.run()
+        h_top.copy_(step_e2e.topk, non_blocking=True)
 
     e2e_body()
     torch.cuda.synchronize()
@@ -426,7 +438,7 @@ def main():
         b.record(stream)
         b.synchronize()
         e2e_ms.append(a.elapsed_time(b))
-    assert np.array_equal(h_top.numpy(), step.topk.cpu().numpy())
+    assert np.array_equal(h_top.numpy(), step.topk.cpu().numpy())  # same result as the device-resident step
     e2e_step = float(np.mean(e2e_ms[1:]))
     e2e_value = world * per_step_work / (e2e_step * 1e-3)
 
