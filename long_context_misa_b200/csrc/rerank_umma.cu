@@ -1,0 +1,295 @@
+// Re-rank scoring of gathered candidates (the MISA-dagger fine stage) on the
+// fifth-generation tensor cores.
+//
+// "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM Inference",
+// technical summary, "Hierarchical variant": the original DSA indexer -- all
+// H_I heads -- re-scores only the candidate set kept by the routed pass:
+//     I_t = s_t * sum_n w_{i,n} * ReLU(q_{i,n} . k_t),   t in gather[i].
+// For one query the candidates' keys against its heads are a dense product:
+// 128 gathered key rows on the MMA M side, the query's scoring heads on N
+// (HN columns, zero-weight padding up to a power of two >= 32), d = 128 on K.
+//
+// One CTA of 4 warps takes up to T = 2 tiles of 128 candidates of one query.  It
+// requests every key row of its tiles at once with 16-byte cp.async into the
+// 128-byte-swizzled K-major layout the MMA reads (invalid candidates are
+// zero-filled and never written), builds the query's head matrix Q' (bf16,
+// or the exact two-term e4m3 split of a bf16 query with a power-of-two scale
+// folded into the weight) while the rows are in flight, then one thread
+// issues all the tiles' MMAs into tensor memory and commits them to one
+// mbarrier.  The four warps read one candidate row per thread with
+// tcgen05.ld, apply ReLU, the weights, the head sum and the e4m3 token scale,
+// write the score and count it in the row histogram (shared memory, added to
+// row_hist once per CTA).  The wait on the MMAs is bounded: one that runs out
+// sets MISA_DEV_WAIT_TIMEOUT and the CTA returns without scores.
+#include <cuda.h>
+
+#include <algorithm>
+
+#include "frag.cuh"
+#include "internal.h"
+#include "umma.cuh"
+
+namespace misa {
+namespace {
+
+constexpr int RR_M = 128;       // candidates per tile
+constexpr int RR_THREADS = 128;  // 4 warps: loaders, then one tensor-memory lane quarter each
+
+template <bool FP8, int HN>
+struct RCfg {
+  static constexpr int ROW = FP8 ? 128 : 256;       // key bytes per token
+  static constexpr int CH = ROW / 16;               // 16-byte chunks per row
+  static constexpr int A_BYTES = RR_M * ROW;        // one tile of key rows
+  static constexpr int B_BYTES = HN * 256;          // Q': bf16 (two K blocks) or two e4m3 terms
+  static constexpr int T = 2;                       // tiles per CTA (T * HN <= 256 tensor-memory columns)
+  static constexpr int TMEM_COLS = T * HN;
+  static constexpr int SMEM = 1024 + T * A_BYTES + B_BYTES;
+};
+
+struct RerankShared {
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort;
+  alignas(16) float w[128];        // weight per column (0: padding); read as float4
+  int32_t tok[2 * RR_M];           // candidate token per slot (-1: skip)
+  float scale[2 * RR_M];           // e4m3 token scale per slot
+  uint32_t hist[TOPK_HIST_BINS];   // this CTA's share of the row histogram
+};
+
+template <bool FP8, int HN>
+__global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, QueryView qv, const int32_t *heads,
+                                                                  int h, const int32_t *gather, int n_cols,
+                                                                  float *scores, long long ld,
+                                                                  uint32_t *row_hist) {
+  using Cfg = RCfg<FP8, HN>;
+  constexpr int T = Cfg::T;
+  extern __shared__ uint8_t rr_raw[];
+  uint8_t *base = rr_raw + ((1024u - (smem_addr(rr_raw) & 1023u)) & 1023u);  // 1024-aligned (swizzle atoms)
+  uint8_t *a_smem = base;                       // T x A_BYTES
+  uint8_t *b_smem = base + T * Cfg::A_BYTES;    // B_BYTES
+  __shared__ RerankShared sh;
+  volatile int *abort = &sh.abort;
+  const int i = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = qv.H;
+  const int h_eff = heads ? h : H;
+  int s;
+  const int Li = query_prefix(c, qv, i, &s);
+  const int col0 = blockIdx.x * T * RR_M;
+  const int ntile = min(T, cdiv(n_cols - col0, RR_M));
+  const uint8_t *kbase = static_cast<const uint8_t *>(c.keys) + (size_t)max(s, 0) * c.L_cap * Cfg::ROW;
+  const float *sbase = FP8 ? c.scale + (size_t)max(s, 0) * c.L_cap : nullptr;
+
+  // 1. candidate tokens of this CTA's slots (-1: none, negative, or beyond the prefix)
+  for (int e = tid; e < T * RR_M; e += RR_THREADS) {
+    const int p = col0 + e;
+    const int t = (e < ntile * RR_M && p < n_cols) ? __ldg(gather + (size_t)i * n_cols + p) : -1;
+    sh.tok[e] = (t >= 0 && t < Li) ? t : -1;
+  }
+  if (tid == 0) {
+    mbar_init(&sh.done, 1);
+    sh.abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // 2. every key row (and e4m3 scale) of every tile requested at once:
+  //    row r, 16-byte chunk u at block (u / 8), row r, chunk (u % 8) ^ (r % 8)
+  for (int x = tid; x < ntile * RR_M * Cfg::CH; x += RR_THREADS) {
+    const int j = x / (RR_M * Cfg::CH), rem = x % (RR_M * Cfg::CH);
+    const int r = rem / Cfg::CH, u = rem % Cfg::CH;
+    const int t = sh.tok[j * RR_M + r];
+    const uint32_t dst = smem_addr(a_smem + j * Cfg::A_BYTES + (u >> 3) * (RR_M * 128) + r * 128 +
+                                   (((u & 7) ^ (r & 7)) << 4));
+    cp_async16(dst, kbase + (size_t)max(t, 0) * Cfg::ROW + 16 * u, t >= 0);
+  }
+  if (FP8)
+    for (int e = tid; e < ntile * RR_M; e += RR_THREADS) {
+      const int t = sh.tok[e];
+      cp_async4(smem_addr(&sh.scale[e]), sbase + max(t, 0), t >= 0);
+    }
+  cp_async_commit();
+
+  // 3. meanwhile: Q' rows n = the n-th scoring head (zero rows past h_eff),
+  //    two threads per row (half of its 16-byte chunks each, the pair
+  //    agreeing on the e4m3 scale through a shuffle), weights, histogram,
+  //    tensor memory
+  for (int x = tid; x < 2 * HN; x += RR_THREADS) {  // whole warps: HN >= 32
+    const int n = x >> 1, half = x & 1;
+    int hd = -1;
+    if (n < h_eff) {
+      hd = heads ? __ldg(heads + (size_t)i * h + n) : n;
+      if (hd < 0 || hd >= H) {
+        if (half == 0) flag(c, MISA_DEV_BAD_HEAD);
+        hd = -1;
+      }
+    }
+    const uint4 *row = reinterpret_cast<const uint4 *>(qv.q + ((size_t)i * H + max(hd, 0)) * D) + half * 8;
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = hd >= 0 ? __ldg(row + u) : make_uint4(0u, 0u, 0u, 0u);
+    float wv = hd >= 0 ? __ldg(qv.w + (size_t)i * H + hd) : 0.f;
+    if (!FP8) {
+#pragma unroll
+      for (int u8 = 0; u8 < 8; ++u8) {
+        const int u = half * 8 + u8;
+        *reinterpret_cast<uint4 *>(b_smem + (u >> 3) * (HN * 128) + n * 128 + (((u & 7) ^ (n & 7)) << 4)) = v[u8];
+      }
+    } else {
+      float m = 0.f;
+#pragma unroll
+      for (int u8 = 0; u8 < 8; ++u8) {
+        const uint32_t ww[4] = {v[u8].x, v[u8].y, v[u8].z, v[u8].w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float2 f = bf16x2_to_float2(ww[p]);
+          m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+      }
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      const float sc = e4m3_head_scale(m);
+      wv = wv / sc;  // exact: sc is a power of two
+      // input chunk u (8 elements) -> 8 bytes of each term at byte 8u of the row
+#pragma unroll
+      for (int u8 = 0; u8 < 8; ++u8) {
+        const int u = half * 8 + u8;
+        uint2 t1, t2;
+        split_e4m3(v[u8], sc, t1, t2);
+        const int off = n * 128 + (((u >> 1) ^ (n & 7)) << 4) + (u & 1) * 8;
+        *reinterpret_cast<uint2 *>(b_smem + off) = t1;
+        *reinterpret_cast<uint2 *>(b_smem + HN * 128 + off) = t2;
+      }
+    }
+    if (half == 0) sh.w[n] = wv;
+  }
+  for (int b = tid; b < TOPK_HIST_BINS; b += RR_THREADS) sh.hist[b] = 0;
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&sh.tmem_base)),
+                 "n"(Cfg::TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  cp_async_wait<0>();
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // rows and Q' visible to the tensor cores
+  umma::fence_before();
+  __syncthreads();
+  umma::fence_after();
+  const uint32_t tmem = sh.tmem_base;
+
+  // 4. one thread issues every tile's MMAs; one commit for all of them
+  if (tid == 0) {
+    const uint32_t idesc = umma::instr_desc<FP8, RR_M, HN>();
+    const uint32_t b_base = smem_addr(b_smem);
+    for (int j = 0; j < ntile; ++j) {
+      const uint32_t a_base = smem_addr(a_smem + j * Cfg::A_BYTES);
+#pragma unroll
+      for (int term = 0; term < (FP8 ? 2 : 1); ++term) {
+#pragma unroll
+        for (int kk = 0; kk < (FP8 ? 4 : 8); ++kk) {
+          uint32_t aoff, boff;
+          if (FP8) {
+            aoff = kk * 32;
+            boff = term * (HN * 128) + kk * 32;
+          } else {
+            aoff = (kk >> 2) * (RR_M * 128) + (kk & 3) * 32;
+            boff = (kk >> 2) * (HN * 128) + (kk & 3) * 32;
+          }
+          umma::mma<FP8>(tmem + j * HN, umma::smem_desc_sw128(a_base + aoff), umma::smem_desc_sw128(b_base + boff),
+                         idesc, (term | kk) ? 1u : 0u);
+        }
+      }
+    }
+    umma::commit(&sh.done);
+  }
+
+  // 5. epilogue: candidate row r = 32 * warp + lane of every tile
+  const bool got = umma::wait_bar(&sh.done, 0, abort, c);
+  umma::fence_after();
+  if (got) {
+    const int r = warp * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    for (int j = 0; j < ntile; ++j) {
+      float acc = 0.f;
+      const float4 *w4 = reinterpret_cast<const float4 *>(sh.w);
+#pragma unroll
+      for (int cb = 0; cb < HN; cb += 32) {
+        uint32_t v[32];
+        umma::ld32(tl + j * HN + cb, v);
+        umma::ld_wait();
+#pragma unroll
+        for (int x = 0; x < 32; x += 4) {
+          const float4 w = w4[(cb + x) >> 2];
+          acc = fmaf(w.x, fmaxf(__uint_as_float(v[x]), 0.f), acc);
+          acc = fmaf(w.y, fmaxf(__uint_as_float(v[x + 1]), 0.f), acc);
+          acc = fmaf(w.z, fmaxf(__uint_as_float(v[x + 2]), 0.f), acc);
+          acc = fmaf(w.w, fmaxf(__uint_as_float(v[x + 3]), 0.f), acc);
+        }
+      }
+      const int e = j * RR_M + r;
+      const int t = sh.tok[e];
+      if (t >= 0) {
+        const float val = FP8 ? acc * sh.scale[e] : acc;
+        scores[(size_t)i * ld + col0 + e] = val;
+        atomicAdd(&sh.hist[ordered_key(val) >> 21], 1u);
+      }
+    }
+  } else if (tid == 0) {
+    mbar_wait(&sh.done, 0);  // bounded: the MMAs finish before the tensor memory is released
+  }
+  umma::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    umma::fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(Cfg::TMEM_COLS));
+  }
+  if (got) {
+    uint32_t *rh = row_hist + (size_t)i * TOPK_HIST_BINS;
+    for (int b = tid; b < TOPK_HIST_BINS; b += RR_THREADS) {
+      const uint32_t v = sh.hist[b];
+      if (v) atomicAdd(rh + b, v);
+    }
+  }
+}
+
+template <bool FP8, int HN>
+cudaError_t launch_hn(const CacheView &c, const QueryView &q, const int32_t *heads, int h, const int32_t *gather,
+                      int n_cols, float *scores, long long ld, uint32_t *row_hist, cudaStream_t s) {
+  using Cfg = RCfg<FP8, HN>;
+  struct Tag {};
+  const int st = cached_per_device<Tag>([] {
+    return 1 + (int)cudaFuncSetAttribute(rerank_umma_kernel<FP8, HN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::SMEM);
+  });
+  if (st != 1) return (cudaError_t)(st - 1);
+  const dim3 grid(cdiv(n_cols, Cfg::T * RR_M), q.n_q);
+  return launch_kernel(rerank_umma_kernel<FP8, HN>, grid, dim3(RR_THREADS), Cfg::SMEM, s, c, q, heads, h, gather,
+                       n_cols, scores, ld, row_hist);
+}
+
+}  // namespace
+
+bool rerank_umma_applies(const QueryView &q, const int32_t *heads, int h) {
+  const int h_eff = heads ? h : q.H;
+  return h_eff >= 1 && h_eff <= 128;
+}
+
+cudaError_t launch_rerank_umma(const CacheView &c, const QueryView &q, const int32_t *heads, int h,
+                               const int32_t *gather, int n_cols, float *scores, long long ld, uint32_t *row_hist,
+                               cudaStream_t s) {
+  if (q.n_q == 0 || n_cols == 0) return cudaSuccess;
+  const int h_eff = heads ? h : q.H;
+  const int hn = h_eff <= 32 ? 32 : h_eff <= 64 ? 64 : 128;
+#define MISA_RERANK_CASE(N)                                                                        \
+  case N:                                                                                          \
+    return c.fp8 ? launch_hn<true, N>(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s)     \
+                 : launch_hn<false, N>(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s);
+  switch (hn) {
+    MISA_RERANK_CASE(32)
+    MISA_RERANK_CASE(64)
+    MISA_RERANK_CASE(128)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef MISA_RERANK_CASE
+}
+
+}  // namespace misa

@@ -165,6 +165,8 @@ cudaError_t launch_score_mma(const CacheView &c, const QueryView &q, const int32
                              cudaStream_t s) {
   if (q.n_q == 0) return cudaSuccess;
   if (!gather) return launch_score_stream(c, q, heads, h, scores, ld, row_hist, s);
+  if (rerank_umma_applies(q, heads, h))
+    return launch_rerank_umma(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s);
   const int h_eff = heads ? h : q.H;
   int NT = 1;
   while (NT * 8 < h_eff) NT *= 2;
