@@ -116,7 +116,8 @@ size_t round_up(size_t x) { return (x + 255) & ~size_t(255); }
 // Workspace of the score + top-k calls: [row histograms + top-k list
 // counters (zeroed together)][scores, unless the caller passes scores_out]
 // [top-k list, prefix rows that use one].
-size_t hist_words(const misa_queries *q) { return (size_t)q->n_q * (misa::TOPK_HIST_BINS + 1); }
+// row histograms, then two counters per row (list entries, emitted tokens)
+size_t hist_words(const misa_queries *q) { return (size_t)q->n_q * (misa::TOPK_HIST_BINS + 2); }
 size_t ws_hist(const misa_queries *q) { return round_up(sizeof(uint32_t) * hist_words(q)); }
 size_t ws_list(const misa_cache *c, const misa_queries *q, int k) {
   return round_up(8 * misa::topk_list_entries(q->n_q, c->L_cap, k));

@@ -67,8 +67,8 @@ cudaError_t launch_score_umma(const CacheView &c, const QueryView &q, const int3
 // otherwise it is filled here first.  Prefix rows of caches longer than
 // TOPK_LIST_MIN_L go through a compact list of the elements at or above the
 // histogram's boundary bin: list_ws holds topk_list_entries() entries of 8
-// bytes and list_cnt n_q counters, zeroed beforehand (both may be null: no
-// list; the selection then reads the rows itself).  ordered == false allows
+// bytes and list_cnt 2 * n_q counters, zeroed beforehand (both may be null:
+// no list; the selection then reads the rows itself).  ordered == false allows
 // the selected tokens of a row in any order (followed by -1 padding).
 constexpr int TOPK_LIST_MIN_L = 16384;   // shorter caches never use the list
 constexpr int TOPK_LIST_EXTRA = 8192;    // boundary-bin elements listed per row beyond k

@@ -626,10 +626,15 @@ __global__ void __launch_bounds__(SEL_T) select_kernel(CacheView c, QueryView qv
 // Few long prefix rows: every CTA takes a chunk of one row and appends the
 // elements at or above the boundary bin, (key, token), to the row's list
 // (list_cnt zeroed beforehand).  Rows the list cannot serve are skipped; the
-// select kernel reads those rows itself.
+// select kernel reads those rows itself.  EMIT (unordered output): the
+// elements above the boundary bin are selected whatever the refinement
+// decides, so their tokens go straight to out[row][0..above) (slots from
+// emit_cnt, zeroed beforehand) and only the boundary bin is listed.
+template <bool EMIT>
 __global__ void __launch_bounds__(FILT_T) filter_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
                                                         const uint32_t *row_hist, uint2 *list, uint32_t *list_cnt,
-                                                        int list_cap, int k, int chunk) {
+                                                        int list_cap, int k, int chunk, int32_t *out,
+                                                        uint32_t *emit_cnt) {
   constexpr int FU = 16;
   const int row = blockIdx.y;
   const int lane = threadIdx.x & 31;
@@ -667,12 +672,14 @@ __global__ void __launch_bounds__(FILT_T) filter_kernel(CacheView c, QueryView q
         sv[u] = p < p1 ? __ldg(srow + p) : 0.f;
       }
     }
+    // per thread: elements to list (low 16 bits) and, EMIT, to emit (high 16)
     uint32_t key[FU], n = 0;
 #pragma unroll
     for (int u = 0; u < FU; ++u) {
       const int p = base + u * FILT_T + threadIdx.x;
       key[u] = ordered_key(sv[u]);
-      n += (p < p1 && (key[u] >> HIST_SHIFT) >= d0) ? 1u : 0u;
+      const uint32_t bin = key[u] >> HIST_SHIFT;
+      if (p < p1) n += EMIT ? (bin == d0 ? 1u : bin > d0 ? 0x10000u : 0u) : (bin >= d0 ? 1u : 0u);
     }
     uint32_t inc = n;
 #pragma unroll
@@ -682,15 +689,25 @@ __global__ void __launch_bounds__(FILT_T) filter_kernel(CacheView c, QueryView q
     }
     const uint32_t tot = __shfl_sync(0xffffffffu, inc, 31);
     if (tot == 0) continue;  // warp-uniform
-    uint32_t slot = 0;
-    if (lane == 31) slot = atomicAdd(list_cnt + row, tot);
-    slot = __shfl_sync(0xffffffffu, slot, 31) + inc - n;
+    uint32_t slot = 0, eslot = 0;
+    if (lane == 31) {
+      if (tot & 0xFFFFu) slot = atomicAdd(list_cnt + row, tot & 0xFFFFu);
+      if (EMIT && (tot >> 16)) eslot = atomicAdd(emit_cnt + row, tot >> 16);
+    }
+    slot = __shfl_sync(0xffffffffu, slot, 31) + (inc & 0xFFFFu) - (n & 0xFFFFu);
+    if (EMIT) eslot = __shfl_sync(0xffffffffu, eslot, 31) + (inc >> 16) - (n >> 16);
+    int32_t *orow = EMIT ? out + (size_t)row * k : nullptr;
 #pragma unroll
     for (int u = 0; u < FU; ++u) {
       const int p = base + u * FILT_T + threadIdx.x;
-      if (p < p1 && (key[u] >> HIST_SHIFT) >= d0) {
+      const uint32_t bin = key[u] >> HIST_SHIFT;
+      if (p < p1 && (EMIT ? bin == d0 : bin >= d0)) {
         if (slot < (uint32_t)list_cap) lrow[slot] = make_uint2(key[u], (uint32_t)p);
         ++slot;
+      }
+      if (EMIT && p < p1 && bin > d0) {
+        if (eslot < (uint32_t)k) orow[eslot] = p;
+        ++eslot;
       }
     }
   }
@@ -974,7 +991,9 @@ __global__ void __launch_bounds__(SMP_T) sample_thr_kernel(CacheView c, QueryVie
 // (fewer than min(k, L_i) entries, or more than it holds), the whole row.
 // stage_cap: list entries staged in shared memory (<= list_cap, even);
 // d0cap: boundary-bin elements compacted there.
-template <bool LIST, bool ORDERED, bool OWN = false>
+// EMITTED (LIST, unordered): the filter already wrote the row's elements
+// above the boundary bin to out[row][0..above) and listed only the bin.
+template <bool LIST, bool ORDERED, bool OWN = false, bool EMITTED = false>
 __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryView qv, const float *scores,
                                                             long long ld, int n_cols, const int32_t *gather,
                                                             const uint32_t *row_hist, const uint2 *list,
@@ -1059,7 +1078,10 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
   }
   if (warp == 0) {
     const Boundary b = warp_boundary_plain_smem(sh.rhist, k);
-    if ((tid & 31) == 0) sh.bd = b;
+    if ((tid & 31) == 0) {
+      sh.bd = b;
+      if (EMITTED && b.listable()) sh.n_out = b.above;  // the filter's tokens come first
+    }
   }
   __syncthreads();
   const Boundary bd = sh.bd;
@@ -1193,7 +1215,7 @@ int fast_smem_bytes(bool list, int n_cols, int stage_cap, int L_cap, int d0cap =
   return (int)sizeof(FastShared) + (list ? stage_cap * 8 : n_cols * 8) + 4 * bm_words(L_cap) + 8 * d0cap;
 }
 
-template <bool LIST, bool ORDERED = true, bool OWN = false>
+template <bool LIST, bool ORDERED = true, bool OWN = false, bool EMITTED = false>
 cudaError_t launch_select_smem(const CacheView &c, const QueryView &q, const float *scores, long long ld, int n_cols,
                                const int32_t *gather, const uint32_t *row_hist, const uint2 *list,
                                const uint32_t *list_cnt, int list_cap, int k, int32_t *out, cudaStream_t s,
@@ -1202,12 +1224,12 @@ cudaError_t launch_select_smem(const CacheView &c, const QueryView &q, const flo
   if (stage_cap < 0) stage_cap = list_cap;
   struct Tag {};
   const int st = cached_per_device<Tag>([] {
-    return 1 + (int)cudaFuncSetAttribute(select_smem_kernel<LIST, ORDERED, OWN>,
+    return 1 + (int)cudaFuncSetAttribute(select_smem_kernel<LIST, ORDERED, OWN, EMITTED>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_MAX);
   });
   if (st != 1) return (cudaError_t)(st - 1);
   const int smem = fast_smem_bytes(LIST, n_cols, stage_cap, c.L_cap, d0cap);
-  return launch_kernel(select_smem_kernel<LIST, ORDERED, OWN>, dim3(q.n_q), dim3(FAST_T), smem, s, c, q, scores, ld,
+  return launch_kernel(select_smem_kernel<LIST, ORDERED, OWN, EMITTED>, dim3(q.n_q), dim3(FAST_T), smem, s, c, q, scores, ld,
                        n_cols, gather, row_hist, list, list_cnt, list_cap, stage_cap, d0cap, k, out);
 }
 
@@ -1306,15 +1328,21 @@ cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *sco
   }
   if (!list_mode)
     return launch_select<false, false>(c, q, scores, ld, 0, nullptr, row_hist, nullptr, nullptr, 0, k, out, s);
-  e = launch_kernel(filter_kernel, fgrid, dim3(FILT_T), 0, s, c, q, scores, ld, row_hist, list, list_cnt,
-                    list_cap, k, chunk);
+  // unordered output with the staged selection: the filter emits the tokens
+  // above the boundary bin itself and lists only the bin
+  const bool emit = !ordered && smem_list;
+  uint32_t *emit_cnt = list_cnt + q.n_q;
+  e = emit ? launch_kernel(filter_kernel<true>, fgrid, dim3(FILT_T), 0, s, c, q, scores, ld, row_hist, list,
+                           list_cnt, list_cap, k, chunk, out, emit_cnt)
+           : launch_kernel(filter_kernel<false>, fgrid, dim3(FILT_T), 0, s, c, q, scores, ld, row_hist, list,
+                           list_cnt, list_cap, k, chunk, out, emit_cnt);
   if (e != cudaSuccess) return e;
   if (smem_list)
     return ordered
                ? launch_select_smem<true, true>(c, q, scores, ld, 0, nullptr, row_hist, list, list_cnt, list_cap, k,
                                                 out, s)
-               : launch_select_smem<true, false>(c, q, scores, ld, 0, nullptr, row_hist, list, list_cnt, list_cap, k,
-                                                 out, s);
+               : launch_select_smem<true, false, false, true>(c, q, scores, ld, 0, nullptr, row_hist, list,
+                                                              list_cnt, list_cap, k, out, s);
   return launch_select<false, true>(c, q, scores, ld, 0, nullptr, row_hist, list, list_cnt, list_cap, k, out, s);
 }
 
