@@ -18,10 +18,11 @@
 // row over the blocks wholly inside its query's prefix; a second kernel adds
 // the causal tail block in fp32 and keeps the top-h heads.
 //
-// route_umma_kernel: one CTA per SM over contiguous groups of 128 rows;
-// warp 0 issues TMA loads (the group's query rows once, then hi/lo pool
-// tiles into a 2-stage ring), warp 1 owns the tensor memory and issues the
-// MMAs, warps 2..5 drain two accumulator buffers of 128 columns.
+// route_umma_kernel: one CTA per group of 128 rows, two CTAs per SM (their
+// set-up latencies overlap); warp 0 issues TMA loads (the group's query rows,
+// then hi/lo pool tiles of 64 blocks into a 2-stage ring), warp 1 owns the
+// tensor memory and issues the MMAs, warps 2..5 drain two accumulator
+// buffers of 64 columns.
 #include <algorithm>
 
 #include "internal.h"
@@ -32,7 +33,7 @@ namespace misa {
 namespace {
 
 constexpr int RU_M = 128;              // query-head rows per group
-constexpr int RU_N = 128;              // pooled blocks per tile
+constexpr int RU_N = 64;               // pooled blocks per tile
 constexpr int RU_STAGES = 2;
 constexpr int RU_THREADS = 192;        // TMA warp, MMA warp, 4 epilogue warps
 constexpr int RU_A_BYTES = RU_M * 256; // the group's rows: bf16, two 128-byte K blocks
@@ -44,6 +45,7 @@ struct RouteShared {
   uint32_t tmem_base;
   int abort;
   int n_pass;
+  int first_seq, multi, max_full;  // one-sequence fast path of the pass set-up
   int pass_seq[RU_M];   // distinct sequences of the group's rows
   int pass_full[RU_M];  // most whole blocks among their queries
   int row_full[RU_M];   // per row: whole blocks inside its query's prefix
@@ -67,7 +69,7 @@ __global__ void __launch_bounds__(256) pool_split_kernel(const float4 *pool, siz
   }
 }
 
-__global__ void __launch_bounds__(RU_THREADS, 1)
+__global__ void __launch_bounds__(RU_THREADS, 2)
     route_umma_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap hmap,
                       const __grid_constant__ CUtensorMap lmap, CacheView c, QueryView qv, float *rsum,
                       int n_groups) {
@@ -99,7 +101,8 @@ __global__ void __launch_bounds__(RU_THREADS, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(smem_addr(&sh.tmem_base)));
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&sh.tmem_base)),
+                 "n"(2 * RU_N));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     umma::fence_before();
   }
@@ -115,6 +118,11 @@ __global__ void __launch_bounds__(RU_THREADS, 1)
 
   for (int g = g0; g < g1 && !*abort; ++g) {
     // ---- the group's rows: query, sequence, whole blocks ----
+    if (tid == 0) {
+      sh.first_seq = -1;
+      sh.multi = 0;
+      sh.max_full = 0;
+    }
     for (int r = tid; r < RU_M; r += RU_THREADS) {
       const int row = g * RU_M + r, qi = row / H;
       int s = -1, Li = 0;
@@ -130,7 +138,19 @@ __global__ void __launch_bounds__(RU_THREADS, 1)
       a_loaded = true;
     }
     __syncthreads();
-    if (tid == 0) {
+    // the rows' sequences: one (the usual case) is settled with shared atomics
+    if (tid < RU_M && sh.row_seq[tid] >= 0) atomicCAS(&sh.first_seq, -1, sh.row_seq[tid]);
+    __syncthreads();
+    if (tid < RU_M && sh.row_seq[tid] >= 0) {
+      if (sh.row_seq[tid] != sh.first_seq) sh.multi = 1;
+      atomicMax(&sh.max_full, sh.row_full[tid]);
+    }
+    __syncthreads();
+    if (tid == 0 && !sh.multi) {
+      sh.n_pass = sh.first_seq >= 0 ? 1 : 0;
+      sh.pass_seq[0] = sh.first_seq;
+      sh.pass_full[0] = sh.max_full;
+    } else if (tid == 0) {
       int np = 0;
       for (int r = 0; r < RU_M; ++r) {
         const int s = sh.row_seq[r];
@@ -189,9 +209,10 @@ __global__ void __launch_bounds__(RU_THREADS, 1)
             for (int term = 0; term < 2; ++term) {
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t koff = (kk >> 2) * (RU_M * 128) + (kk & 3) * 32;  // RU_M == RU_N
-                umma::mma<false>(d, umma::smem_desc_sw128(a_base + koff),
-                                 umma::smem_desc_sw128(b_base + term * RU_B_TERM + koff), idesc,
+                const uint32_t aoff = (kk >> 2) * (RU_M * 128) + (kk & 3) * 32;
+                const uint32_t boff = (kk >> 2) * (RU_N * 128) + (kk & 3) * 32;
+                umma::mma<false>(d, umma::smem_desc_sw128(a_base + aoff),
+                                 umma::smem_desc_sw128(b_base + term * RU_B_TERM + boff), idesc,
                                  (term | kk) ? 1u : 0u);
               }
             }
@@ -253,7 +274,7 @@ __global__ void __launch_bounds__(RU_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     umma::fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(2 * RU_N));
   }
 }
 
@@ -352,8 +373,8 @@ cudaError_t launch_route_umma(const CacheView &c, const QueryView &q, int h, int
   });
   if (st != 1) return (cudaError_t)(st - 1);
   const int n_groups = cdiv(q.n_q * q.H, RU_M);
-  e = launch_kernel(route_umma_kernel, dim3(std::min(sms, n_groups)), dim3(RU_THREADS), SMEM, s, qmap, hmap, lmap, c,
-                    q, rsum, n_groups);
+  e = launch_kernel(route_umma_kernel, dim3(n_groups), dim3(RU_THREADS), SMEM, s, qmap, hmap, lmap, c, q, rsum,
+                    n_groups);
   if (e != cudaSuccess) return e;
   return launch_kernel(route_tail_finish_kernel, dim3(q.n_q), dim3(MISA_MAX_H), 0, s, c, q, rsum, h, heads,
                        router_scores);
