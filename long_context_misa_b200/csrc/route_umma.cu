@@ -22,7 +22,10 @@
 // set-up latencies overlap); warp 0 issues TMA loads (the group's query rows,
 // then hi/lo pool tiles of 64 blocks into a 2-stage ring), warp 1 owns the
 // tensor memory and issues the MMAs, warps 2..5 drain two accumulator
-// buffers of 64 columns.
+// buffers of 64 columns.  When the group holds whole queries (H divides 128,
+// 16 <= H) the same CTA finishes them: the tail block's mean, its affinity
+// with each head (query rows still in shared memory), r and the top-h heads;
+// otherwise route_tail_finish_kernel does that from the row sums.
 #include <algorithm>
 
 #include "internal.h"
@@ -50,6 +53,11 @@ struct RouteShared {
   int pass_full[RU_M];  // most whole blocks among their queries
   int row_full[RU_M];   // per row: whole blocks inside its query's prefix
   int row_seq[RU_M];    // per row: its sequence (-1: no query)
+  // fused finish (128 / H queries per group, at most 8); its key-sum scratch
+  // and tail sums use the pool stages, idle once the group's MMAs are done
+  int q_li[8], q_t0[8];
+  float rsc[RU_M];      // r of every row
+  int keep[RU_M];
 };
 
 constexpr int ru_smem_bytes() { return 1024 + RU_A_BYTES + RU_STAGES * RU_B_STAGE + (int)sizeof(RouteShared); }
@@ -72,7 +80,7 @@ __global__ void __launch_bounds__(256) pool_split_kernel(const float4 *pool, siz
 __global__ void __launch_bounds__(RU_THREADS, 2)
     route_umma_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap hmap,
                       const __grid_constant__ CUtensorMap lmap, CacheView c, QueryView qv, float *rsum,
-                      int n_groups) {
+                      int n_groups, int fuse, int h, int32_t *heads, float *router_scores) {
   extern __shared__ uint8_t ru_raw[];
   uint8_t *base = ru_raw + ((1024u - (smem_addr(ru_raw) & 1023u)) & 1023u);  // 1024-aligned (swizzle atoms)
   uint8_t *a_smem = base;
@@ -252,9 +260,99 @@ __global__ void __launch_bounds__(RU_THREADS, 2)
       __syncthreads();  // every role is done with this pass
       if (*abort) break;
     }
-    if (warp >= 2) {
-      const int r = (warp & 3) * 32 + lane, row = g * RU_M + r;
-      if (row / H < qv.n_q) rsum[row] = acc;
+    if (!fuse) {
+      if (warp >= 2) {
+        const int r = (warp & 3) * 32 + lane, row = g * RU_M + r;
+        if (row / H < qv.n_q) rsum[row] = acc;
+      }
+    } else if (!*abort) {
+      // ---- fused finish: the group's RU_M / H whole queries ----
+      // (every pool load was consumed and every MMA committed before the
+      // last pass ended, so the stages are free)
+      const int QG = RU_M / H;
+      float *part = reinterpret_cast<float *>(b_smem);  // [16][D] key-sum scratch
+      float *tailm = part + 16 * D;                      // [QG][D] tail-block key sums
+      int prev_li = 0, prev_t0 = -1, prev_s = -1;
+      for (int qg = 0; qg < QG; ++qg) {  // uniform: every thread takes part in the key sums
+        const int qi = g * QG + qg;
+        int s = -1, Li = 0;
+        if (qi < qv.n_q) Li = query_prefix(c, qv, qi, &s);
+        const int t0 = (Li / c.B) * c.B;
+        if (tid == 0) {
+          sh.q_li[qg] = Li;
+          sh.q_t0[qg] = t0;
+        }
+        if (Li > t0 && s == prev_s && t0 == prev_t0 && prev_li > t0 && Li >= prev_li && Li - prev_li <= 8) {
+          // the previous query's tail block plus the few keys between them
+          if (tid < D) {
+            float a = tailm[(qg - 1) * D + tid];
+            for (int t = prev_li; t < Li; ++t) {
+              const size_t e = ((size_t)s * c.L_cap + t) * D + tid;
+              if (c.fp8) {
+                const uint8_t b = __ldg(static_cast<const uint8_t *>(c.keys) + e);
+                a = fmaf(__ldg(c.scale + (size_t)s * c.L_cap + t), f16x2_to_float2(e4m3x2_to_f16x2(b)).x, a);
+              } else {
+                a += bf16_bits_to_float(__ldg(static_cast<const uint16_t *>(c.keys) + e));
+              }
+            }
+            tailm[qg * D + tid] = a;
+          }
+        } else if (Li > t0) {
+          block_key_sum<128>(c, s, t0, Li, part, tailm + qg * D);
+        }
+        __syncthreads();
+        prev_li = Li;
+        prev_t0 = t0;
+        prev_s = s;
+      }
+      __syncthreads();
+      if (warp >= 2) {
+        const int r = (warp & 3) * 32 + lane, qg = r / H, hd = r % H, qi = g * QG + qg;
+        float rr = 0.f;
+        if (qi < qv.n_q) {
+          const int Li = sh.q_li[qg], t0 = sh.q_t0[qg];
+          float a = acc;
+          if (Li > t0 && umma::wait_bar(&sh.afull, a_phase, abort, c)) {  // the query rows in shared memory
+            float dot = 0.f;
+#pragma unroll 4
+            for (int u = 0; u < 16; ++u) {
+              const uint4 v = *reinterpret_cast<const uint4 *>(a_smem + (u >> 3) * (RU_M * 128) + r * 128 +
+                                                               (((u & 7) ^ (r & 7)) << 4));
+              const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int p = 0; p < 4; ++p) {
+                const float2 f = bf16x2_to_float2(ww[p]);
+                dot = fmaf(f.x, tailm[qg * D + 8 * u + 2 * p], dot);
+                dot = fmaf(f.y, tailm[qg * D + 8 * u + 2 * p + 1], dot);
+              }
+            }
+            a += fmaxf(dot * (1.f / (float)(Li - t0)), 0.f);
+          }
+          rr = fabsf(__ldg(qv.w + (size_t)qi * H + hd)) * a;
+          if (router_scores) router_scores[(size_t)qi * H + hd] = rr;
+        }
+        sh.rsc[r] = rr;
+      }
+      __syncthreads();
+      if (warp >= 2) {  // head hd is kept iff fewer than h heads beat it (larger r, or equal r and lower index)
+        const int r = (warp & 3) * 32 + lane, qg = r / H, hd = r % H;
+        const float rr = sh.rsc[r];
+        int beaten = 0;
+        for (int o = 0; o < H; ++o) {
+          const float ro = sh.rsc[qg * H + o];
+          beaten += (ro > rr) || (ro == rr && o < hd);
+        }
+        sh.keep[r] = beaten < h;
+      }
+      __syncthreads();
+      if (warp >= 2) {  // kept heads in ascending order
+        const int r = (warp & 3) * 32 + lane, qg = r / H, hd = r % H, qi = g * QG + qg;
+        if (qi < qv.n_q && sh.keep[r]) {
+          int pos = 0;
+          for (int o = 0; o < hd; ++o) pos += sh.keep[qg * H + o];
+          if (pos < h) heads[(size_t)qi * h + pos] = hd;  // a NaN score can break the strict order
+        }
+      }
     }
     a_phase ^= 1;
     __syncthreads();  // the group's rows and tables are free again
@@ -373,9 +471,10 @@ cudaError_t launch_route_umma(const CacheView &c, const QueryView &q, int h, int
   });
   if (st != 1) return (cudaError_t)(st - 1);
   const int n_groups = cdiv(q.n_q * q.H, RU_M);
+  const int fuse = q.H >= 16 && q.H <= RU_M && RU_M % q.H == 0;  // groups of whole queries: finish in the kernel
   e = launch_kernel(route_umma_kernel, dim3(n_groups), dim3(RU_THREADS), SMEM, s, qmap, hmap, lmap, c, q, rsum,
-                    n_groups);
-  if (e != cudaSuccess) return e;
+                    n_groups, fuse, h, heads, router_scores);
+  if (e != cudaSuccess || fuse) return e;
   return launch_kernel(route_tail_finish_kernel, dim3(q.n_q), dim3(MISA_MAX_H), 0, s, c, q, rsum, h, heads,
                        router_scores);
 }
