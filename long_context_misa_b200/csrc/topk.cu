@@ -719,9 +719,11 @@ __global__ void __launch_bounds__(FILT_T) filter_kernel(CacheView c, QueryView q
 // list (list_cnt zeroed beforehand; it counts past list_cap).
 constexpr int FT_T = 256;
 constexpr int FT_V = 8;  // float4 loads per thread and sweep
+constexpr int FT_PAD = 4 * FT_V + 4;  // floats per thread in the stash (16-byte rows, staggered banks)
 __global__ void __launch_bounds__(FT_T) filter_thr_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
                                                           const uint32_t *thr, uint2 *list, uint32_t *list_cnt,
                                                           int list_cap, int chunk) {
+  __shared__ __align__(16) float stash[FT_T * FT_PAD];
   const int row = blockIdx.y;
   const int lane = threadIdx.x & 31;
   const int p0 = blockIdx.x * chunk;
@@ -751,20 +753,21 @@ __global__ void __launch_bounds__(FT_T) filter_thr_kernel(CacheView c, QueryView
         v[u] = p < p1 ? __ldg(reinterpret_cast<const float4 *>(srow + p)) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-    uint32_t n = 0;
+    // bit 4u + e: element e of this thread's u-th float4 is listed; the
+    // values wait in shared memory so that the write pass visits only the
+    // set bits (about 6 % of the elements)
     const bool full = base + FT_T * 4 * FT_V <= p1;  // uniform: no element of this sweep past the prefix
-    if (full) {
+    uint32_t mask = 0;
 #pragma unroll
-      for (int u = 0; u < FT_V; ++u)
-        n += (all || v[u].x >= tau) + (all || v[u].y >= tau) + (all || v[u].z >= tau) + (all || v[u].w >= tau);
-    } else {
-#pragma unroll
-      for (int u = 0; u < FT_V; ++u) {
-        const int p = base + (u * FT_T + (int)threadIdx.x) * 4;
-        n += (p < p1 && (all || v[u].x >= tau)) + (p + 1 < p1 && (all || v[u].y >= tau)) +
-             (p + 2 < p1 && (all || v[u].z >= tau)) + (p + 3 < p1 && (all || v[u].w >= tau));
-      }
+    for (int u = 0; u < FT_V; ++u) {
+      const int p = base + (u * FT_T + (int)threadIdx.x) * 4;
+      const bool in0 = full || p < p1, in1 = full || p + 1 < p1, in2 = full || p + 2 < p1, in3 = full || p + 3 < p1;
+      mask |= ((uint32_t)(in0 && (all || v[u].x >= tau)) | (uint32_t)(in1 && (all || v[u].y >= tau)) << 1 |
+               (uint32_t)(in2 && (all || v[u].z >= tau)) << 2 | (uint32_t)(in3 && (all || v[u].w >= tau)) << 3)
+              << (4 * u);
+      *reinterpret_cast<float4 *>(&stash[threadIdx.x * FT_PAD + 4 * u]) = v[u];
     }
+    const uint32_t n = __popc(mask);
     uint32_t inc = n;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -776,18 +779,13 @@ __global__ void __launch_bounds__(FT_T) filter_thr_kernel(CacheView c, QueryView
     uint32_t slot = 0;
     if (lane == 31) slot = atomicAdd(list_cnt + row, tot);
     slot = __shfl_sync(0xffffffffu, slot, 31) + inc - n;
-    if (n == 0) continue;
-#pragma unroll
-    for (int u = 0; u < FT_V; ++u) {
-      const int p = base + (u * FT_T + (int)threadIdx.x) * 4;
-      const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if (p + e < p1 && (all || f[e] >= tau)) {
-          if (slot < (uint32_t)list_cap) lrow[slot] = make_uint2(ordered_key(f[e]), (uint32_t)(p + e));
-          ++slot;
-        }
-      }
+    while (mask) {
+      const int bit = __ffs(mask) - 1;
+      mask &= mask - 1u;
+      const float f = stash[threadIdx.x * FT_PAD + bit];
+      if (slot < (uint32_t)list_cap)
+        lrow[slot] = make_uint2(ordered_key(f), (uint32_t)(base + ((bit >> 2) * FT_T + (int)threadIdx.x) * 4 + (bit & 3)));
+      ++slot;
     }
   }
 }
