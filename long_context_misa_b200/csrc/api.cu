@@ -127,11 +127,18 @@ size_t ws_score(const misa_cache *c, const misa_queries *q) {
   return round_up(sizeof(float) * (size_t)q->n_q * c->L_cap);
 }
 
-// Workspace of misa_dagger_topk: [histograms + list counters][routed scores]
-// [top-k' list][candidates n_q x k'][re-rank scores n_q x k'].
+// Workspace of misa_dagger_topk: [histograms + list counters][re-rank
+// histograms] (one zeroing launch for both) [routed scores][top-k' list]
+// [candidates n_q x k'][re-rank scores n_q x k'].
+// (the re-rank histograms start on a 256-byte boundary: rows are read with
+// 16-byte loads and bulk copies)
+size_t rerank_hist_words(const misa_queries *q) { return (size_t)q->n_q * misa::TOPK_HIST_BINS; }
+size_t ws_dagger_hist(const misa_queries *q) {
+  return ws_hist(q) + round_up(sizeof(uint32_t) * rerank_hist_words(q));
+}
 size_t ws_dagger(const misa_cache *c, const misa_queries *q, int k_prime) {
   const size_t cand = round_up(sizeof(int32_t) * (size_t)q->n_q * k_prime);
-  return ws_hist(q) + ws_score(c, q) + ws_list(c, q, k_prime) + 2 * cand;
+  return ws_dagger_hist(q) + ws_score(c, q) + ws_list(c, q, k_prime) + 2 * cand;
 }
 
 misa_status check_ws(void *ws, size_t have, size_t need) {
@@ -376,14 +383,17 @@ misa_status misa_dagger_topk(const misa_cache *cache, const misa_queries *qs, co
   uint8_t *w8 = static_cast<uint8_t *>(ws);
   uint32_t *hist = reinterpret_cast<uint32_t *>(w8);
   uint32_t *list_cnt = hist + (size_t)qs->n_q * misa::TOPK_HIST_BINS;
-  float *scores = reinterpret_cast<float *>(w8 + ws_hist(qs));
-  void *list = w8 + ws_hist(qs) + ws_score(cache, qs);
-  int32_t *cand = reinterpret_cast<int32_t *>(w8 + ws_hist(qs) + ws_score(cache, qs) + ws_list(cache, qs, k_prime));
+  uint32_t *rhist = reinterpret_cast<uint32_t *>(w8 + ws_hist(qs));
+  float *scores = reinterpret_cast<float *>(w8 + ws_dagger_hist(qs));
+  void *list = w8 + ws_dagger_hist(qs) + ws_score(cache, qs);
+  int32_t *cand =
+      reinterpret_cast<int32_t *>(w8 + ws_dagger_hist(qs) + ws_score(cache, qs) + ws_list(cache, qs, k_prime));
   float *rscores = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(cand) +
                                              round_up(sizeof(int32_t) * (size_t)qs->n_q * k_prime));
   // routed pass: scores, then the k' candidates in any order
   const bool umma = misa::umma_applies(c, q, heads, h);
-  cudaError_t e = misa::launch_zero(hist, hist_words(qs), stream);
+  // both passes' histograms and counters, zeroed by one launch
+  cudaError_t e = misa::launch_zero(hist, ws_hist(qs) / sizeof(uint32_t) + rerank_hist_words(qs), stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   e = timed_scoring(stream, [&] {
     return umma ? misa::launch_score_umma(c, q, heads, h, scores, cache->L_cap, stream)
@@ -394,11 +404,9 @@ misa_status misa_dagger_topk(const misa_cache *cache, const misa_queries *qs, co
                         false);
   if (e != cudaSuccess) return cuda_fail(e, who);
   // fine pass: every head on the candidates, ascending final top-k
-  e = misa::launch_zero(hist, (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
+  e = misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, rscores, k_prime, rhist, stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
-  e = misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, rscores, k_prime, hist, stream);
-  if (e != cudaSuccess) return cuda_fail(e, who);
-  e = misa::launch_topk(c, q, rscores, k_prime, k_prime, cand, hist, true, nullptr, nullptr, k, topk, stream);
+  e = misa::launch_topk(c, q, rscores, k_prime, k_prime, cand, rhist, true, nullptr, nullptr, k, topk, stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   return MISA_OK;
 }

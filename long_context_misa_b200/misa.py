@@ -326,7 +326,7 @@ class MisaDaggerDecode:
     (new_pos is normally q_pos).
     """
 
-    LAUNCHES = 10  # append 1, route 2, zero 1, score 1, top-k' 2 (filter, select), zero 1, re-rank 1, top-k 1
+    LAUNCHES = 9  # append 1, route 2, zero 1, score 1, top-k' 2 (filter, select), re-rank 1, top-k 1
 
     def __init__(self, cache: KeyCache, qs: Queries, h: int, k_prime: int, k: int, new_keys: torch.Tensor,
                  new_scale: Optional[torch.Tensor], new_pos: torch.Tensor):
