@@ -44,8 +44,6 @@ namespace {
 
 constexpr int UM_M = 128;                 // tokens per tile
 constexpr int UM_N = 256;                 // query-head columns per tile
-constexpr int EPI_WARPS = 8;                // two per tensor-memory lane quarter
-constexpr int UM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr int B_BYTES = 65536;            // Q' tile: 256 x 128 bf16, or two e4m3 terms
 
 struct UmmaShared {
@@ -70,12 +68,20 @@ struct UCfg {
   static constexpr int A_BYTES = UM_M * ROW;            // one key tile
   static constexpr int KSTEPS = FP8 ? 4 : 8;            // MMAs per term and tile (K = 32 / 16)
   static constexpr int TERMS = FP8 ? 2 : 1;
-  // With 8 or 16 queries per half of the columns (HPQ = 16 or 8, the routed
-  // case) score tiles leave through TMA stores: every epilogue warp stages its
-  // 32 tokens x QH queries in two private buffers.  With fewer queries a
-  // warp writes at most 4 scores per tile and plain stores are cheaper than
-  // small TMA boxes; with 32 (HPQ = 4) the staging would not fit.
-  static constexpr int QH = (UM_N / 2) / HPQ;
+  // Epilogue warps: four per tensor-memory lane quarter (a quarter of the
+  // columns each) when a query spans at most 8 columns (the routed case:
+  // more warps hide the latency of the ReLU / weight chains), else two (half
+  // of the columns; a query never straddles two warps).
+  static constexpr int SPLIT = HPQ <= 8 ? 4 : 2;
+  static constexpr int EPI_WARPS = 4 * SPLIT;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int SPAN = UM_N / SPLIT;  // columns per epilogue warp
+  // With 8 or 16 queries per warp's columns score tiles leave through TMA
+  // stores: every epilogue warp stages its 32 tokens x QH queries in two
+  // private buffers.  With fewer queries a warp writes at most 4 scores per
+  // tile and plain stores are cheaper than small TMA boxes; with 32 the
+  // staging would not fit.
+  static constexpr int QH = SPAN / HPQ;
   static constexpr bool TMA_OUT = QH >= 8 && QH <= 16;
   static constexpr int OUT_BUF = TMA_OUT ? 32 * QH * 4 : 0;  // bytes of one staging buffer
   static constexpr int FIXED = 1024 /* alignment slack */ + B_BYTES + 2 * EPI_WARPS * OUT_BUF + (int)sizeof(UmmaShared);
@@ -91,7 +97,7 @@ struct UCfg {
 // Items: (group g, tile tau) flattened as g * n_tiles + tau; this CTA takes
 // [item0, item1).  A group holds QPT = 256 / HPQ consecutive queries.
 template <bool FP8, int HPQ>
-__global__ void __maxnreg__(128)
+__global__ void __launch_bounds__(UCfg<FP8, HPQ>::THREADS, 1)
     score_umma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap omap,
                       int out_tma, CacheView c, QueryView qv, const int32_t *heads, int h, float *scores,
                       long long ld, int n_tiles, long long n_items) {
@@ -101,6 +107,7 @@ __global__ void __maxnreg__(128)
   uint8_t *base = um_raw + ((1024u - (smem_addr(um_raw) & 1023u)) & 1023u);  // 1024-aligned (swizzle atoms)
   uint8_t *a_smem = base;                                    // STAGES x A_BYTES (1024-aligned each)
   uint8_t *b_smem = base + Cfg::STAGES * Cfg::A_BYTES;       // B_BYTES
+  constexpr int EPI_WARPS = Cfg::EPI_WARPS, UM_THREADS = Cfg::THREADS;
   float *out_smem = reinterpret_cast<float *>(b_smem + B_BYTES);  // 2 x EPI_WARPS staging buffers
   UmmaShared &sh = *reinterpret_cast<UmmaShared *>(b_smem + B_BYTES + 2 * EPI_WARPS * Cfg::OUT_BUF);
   volatile int *abort = &sh.abort;
@@ -290,16 +297,16 @@ __global__ void __maxnreg__(128)
           }
         }
       } else {
-        // ---- epilogue: one token row per thread, half of the columns per warp ----
+        // ---- epilogue: one token row per thread, SPAN columns per warp ----
         const int e = warp - 2;
-        const int quarter = warp & 3;           // tensor-memory lanes this warp may read
-        const int col0 = (e / 4) * (UM_N / 2);  // its half of the columns
+        const int quarter = warp & 3;              // tensor-memory lanes this warp may read
+        const int col0 = (e / 4) * Cfg::SPAN;      // its columns
         const int r = quarter * 32 + lane;
         const float4 *wv = reinterpret_cast<const float4 *>(sh.wcol + col0);
         // TMA stores of whole [QH queries x 32 tokens] boxes, when every
         // query of this warp's half belongs to this pass (tokens past a
         // query's prefix are written too; they are unspecified)
-        const int qa = col0 / HPQ;  // first query of the half
+        const int qa = col0 / HPQ;  // first query of the warp's columns
         bool tma_ok = false;
         if constexpr (Cfg::TMA_OUT) {
           if (out_tma) {
@@ -336,7 +343,7 @@ __global__ void __maxnreg__(128)
           const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * UM_N + col0;
           float acc = 0.f;  // running sum of a query wider than one chunk
 #pragma unroll
-          for (int ch = 0; ch < UM_N / 64; ch += 2) {
+          for (int ch = 0; ch < Cfg::SPAN / 32; ch += 2) {
             uint32_t v0[32], v1[32];
             umma::ld32(taddr + ch * 32, v0);
             umma::ld32(taddr + ch * 32 + 32, v1);
@@ -438,7 +445,7 @@ cudaError_t launch_hpq(const CUtensorMap &map, const CacheView &c, const QueryVi
   const int out_tma =
       Cfg::TMA_OUT && umma::make_map_f32_rows(&omap, scores, (unsigned long long)c.L_cap, (unsigned long long)q.n_q,
                                               (unsigned long long)ld, 32, Cfg::TMA_OUT ? Cfg::QH : 1);
-  return launch_kernel(score_umma_kernel<FP8, HPQ>, dim3(grid), dim3(UM_THREADS), SMEM, s, map, omap, out_tma, c, q,
+  return launch_kernel(score_umma_kernel<FP8, HPQ>, dim3(grid), dim3(Cfg::THREADS), SMEM, s, map, omap, out_tma, c, q,
                        heads, h, scores, ld, n_tiles, n_items);
 }
 
