@@ -40,8 +40,10 @@ cudaError_t launch_score_mma(const CacheView &c, const QueryView &q, const int32
                              cudaStream_t s);
 
 // rerank_umma.cu: the gathered (re-rank) case of launch_score_mma on tcgen05
-// tensor cores, for up to 128 scoring heads; launch_score_mma dispatches to
-// it when it applies.  Same outputs, histogram included.
+// tensor cores, for up to 128 scoring heads, and (gather == nullptr, n_cols =
+// L_cap) prefix scoring of e4m3 caches with 32 or more heads;
+// launch_score_mma dispatches to it when it applies.  Same outputs,
+// histogram included.
 bool rerank_umma_applies(const QueryView &q, const int32_t *heads, int h);
 cudaError_t launch_rerank_umma(const CacheView &c, const QueryView &q, const int32_t *heads, int h,
                                const int32_t *gather, int n_cols, float *scores, long long ld, uint32_t *row_hist,

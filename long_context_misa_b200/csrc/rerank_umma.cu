@@ -9,6 +9,10 @@
 // 128 gathered key rows on the MMA M side, the query's scoring heads on N
 // (HN columns, zero-weight padding up to a power of two >= 32), d = 128 on K.
 //
+// gather == nullptr: the candidates are the prefix itself (slot p = token p,
+// n_cols = L_cap): dense scoring of decode queries with many heads, where the
+// same dense product on mma.sync would be compute-bound.
+//
 // One CTA of 4 warps takes up to T = 2 tiles of 128 candidates of one query.  It
 // requests every key row of its tiles at once with 16-byte cp.async into the
 // 128-byte-swizzled K-major layout the MMA reads (invalid candidates are
@@ -35,13 +39,14 @@ namespace {
 constexpr int RR_M = 128;       // candidates per tile
 constexpr int RR_THREADS = 128;  // 4 warps: loaders, then one tensor-memory lane quarter each
 
-template <bool FP8, int HN>
+template <bool FP8, int HN, int TT>
 struct RCfg {
   static constexpr int ROW = FP8 ? 128 : 256;       // key bytes per token
   static constexpr int CH = ROW / 16;               // 16-byte chunks per row
   static constexpr int A_BYTES = RR_M * ROW;        // one tile of key rows
   static constexpr int B_BYTES = HN * 256;          // Q': bf16 (two K blocks) or two e4m3 terms
-  static constexpr int T = 2;                       // tiles per CTA (T * HN <= 256 tensor-memory columns)
+  static constexpr int T = TT;                      // tiles per CTA (T * HN <= 256 tensor-memory columns)
+  static_assert(T * HN <= 256 && T <= 4, "tensor-memory columns per CTA");
   static constexpr int TMEM_COLS = T * HN;
   static constexpr int SMEM = 1024 + T * A_BYTES + B_BYTES;
 };
@@ -51,17 +56,17 @@ struct RerankShared {
   uint32_t tmem_base;
   int abort;
   alignas(16) float w[128];        // weight per column (0: padding); read as float4
-  int32_t tok[2 * RR_M];           // candidate token per slot (-1: skip)
-  float scale[2 * RR_M];           // e4m3 token scale per slot
+  int32_t tok[4 * RR_M];           // candidate token per slot (-1: skip)
+  float scale[4 * RR_M];           // e4m3 token scale per slot
   uint32_t hist[TOPK_HIST_BINS];   // this CTA's share of the row histogram
 };
 
-template <bool FP8, int HN>
+template <bool FP8, int HN, int TT>
 __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, QueryView qv, const int32_t *heads,
                                                                   int h, const int32_t *gather, int n_cols,
                                                                   float *scores, long long ld,
                                                                   uint32_t *row_hist) {
-  using Cfg = RCfg<FP8, HN>;
+  using Cfg = RCfg<FP8, HN, TT>;
   constexpr int T = Cfg::T;
   extern __shared__ uint8_t rr_raw[];
   uint8_t *base = rr_raw + ((1024u - (smem_addr(rr_raw) & 1023u)) & 1023u);  // 1024-aligned (swizzle atoms)
@@ -76,6 +81,7 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
   int s;
   const int Li = query_prefix(c, qv, i, &s);
   const int col0 = blockIdx.x * T * RR_M;
+  if (!gather && col0 >= Li) return;  // uniform: a prefix row with nothing here (no barrier or allocation yet)
   const int ntile = min(T, cdiv(n_cols - col0, RR_M));
   const uint8_t *kbase = static_cast<const uint8_t *>(c.keys) + (size_t)max(s, 0) * c.L_cap * Cfg::ROW;
   const float *sbase = FP8 ? c.scale + (size_t)max(s, 0) * c.L_cap : nullptr;
@@ -83,7 +89,7 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
   // 1. candidate tokens of this CTA's slots (-1: none, negative, or beyond the prefix)
   for (int e = tid; e < T * RR_M; e += RR_THREADS) {
     const int p = col0 + e;
-    const int t = (e < ntile * RR_M && p < n_cols) ? __ldg(gather + (size_t)i * n_cols + p) : -1;
+    const int t = (e < ntile * RR_M && p < n_cols) ? (gather ? __ldg(gather + (size_t)i * n_cols + p) : p) : -1;
     sh.tok[e] = (t >= 0 && t < Li) ? t : -1;
   }
   if (tid == 0) {
@@ -250,19 +256,30 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
   }
 }
 
-template <bool FP8, int HN>
-cudaError_t launch_hn(const CacheView &c, const QueryView &q, const int32_t *heads, int h, const int32_t *gather,
+template <bool FP8, int HN, int TT>
+cudaError_t launch_tt(const CacheView &c, const QueryView &q, const int32_t *heads, int h, const int32_t *gather,
                       int n_cols, float *scores, long long ld, uint32_t *row_hist, cudaStream_t s) {
-  using Cfg = RCfg<FP8, HN>;
+  using Cfg = RCfg<FP8, HN, TT>;
   struct Tag {};
   const int st = cached_per_device<Tag>([] {
-    return 1 + (int)cudaFuncSetAttribute(rerank_umma_kernel<FP8, HN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg::SMEM);
+    return 1 + (int)cudaFuncSetAttribute(rerank_umma_kernel<FP8, HN, TT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
   });
   if (st != 1) return (cudaError_t)(st - 1);
   const dim3 grid(cdiv(n_cols, Cfg::T * RR_M), q.n_q);
-  return launch_kernel(rerank_umma_kernel<FP8, HN>, grid, dim3(RR_THREADS), Cfg::SMEM, s, c, q, heads, h, gather,
+  return launch_kernel(rerank_umma_kernel<FP8, HN, TT>, grid, dim3(RR_THREADS), Cfg::SMEM, s, c, q, heads, h, gather,
                        n_cols, scores, ld, row_hist);
+}
+
+// Gathered candidates: 2 tiles per CTA (more CTAs shorten each gather chain);
+// a prefix row: as many tiles as the tensor memory allows, up to 4 (fewer
+// query set-ups per key byte).
+template <bool FP8, int HN>
+cudaError_t launch_hn(const CacheView &c, const QueryView &q, const int32_t *heads, int h, const int32_t *gather,
+                      int n_cols, float *scores, long long ld, uint32_t *row_hist, cudaStream_t s) {
+  constexpr int TP = (256 / HN) < 4 ? (256 / HN) : 4;
+  return gather ? launch_tt<FP8, HN, 2>(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s)
+                : launch_tt<FP8, HN, TP>(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s);
 }
 
 }  // namespace

@@ -164,7 +164,17 @@ cudaError_t launch_score_mma(const CacheView &c, const QueryView &q, const int32
                              const int32_t *gather, int n_cols, float *scores, long long ld, uint32_t *row_hist,
                              cudaStream_t s) {
   if (q.n_q == 0) return cudaSuccess;
-  if (!gather) return launch_score_stream(c, q, heads, h, scores, ld, row_hist, s);
+  if (!gather) {
+    // e4m3 keys with 32 or more scoring heads (dense decode): the dense
+    // product on tcgen05 (74.8 against 139.3 us for 8 x 128K keys and 64
+    // heads); fewer heads (routed decode), and bf16 keys (whose 32 KB tiles
+    // leave one CTA per SM there: 125 against 77 us for 32 x 32K and 64
+    // heads), stream the keys on mma.sync
+    const int he = heads ? h : q.H;
+    if (c.fp8 && he >= 32 && rerank_umma_applies(q, heads, h))
+      return launch_rerank_umma(c, q, heads, h, nullptr, c.L_cap, scores, ld, row_hist, s);
+    return launch_score_stream(c, q, heads, h, scores, ld, row_hist, s);
+  }
   if (rerank_umma_applies(q, heads, h))
     return launch_rerank_umma(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s);
   const int h_eff = heads ? h : q.H;
