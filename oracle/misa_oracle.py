@@ -73,6 +73,47 @@ def decode_e4m3(codes: np.ndarray) -> np.ndarray:
     return E4M3[np.asarray(codes, dtype=np.uint8)]
 
 
+# finite codes (0x7F / 0xFF are NaN), sorted by value; +0 stands for zero
+_FINITE = np.array([c for c in range(256) if not math.isnan(E4M3[c]) and c != 0x80], dtype=np.int64)
+_FINITE = _FINITE[np.argsort(E4M3[_FINITE], kind="stable")]
+_FINITE_V = E4M3[_FINITE]
+E4M3_MAX = 448.0
+
+
+def encode_e4m3(y: np.ndarray) -> np.ndarray:
+    """Values -> e4m3 codes: the nearest finite e4m3 value, a tie going to the
+    code with an even mantissa (round to nearest even), magnitudes above 448
+    saturating to +-448; zero keeps its sign (0x00 / 0x80).  (OCP 8-bit floating point
+    definition; used for the key-write path, see quantize_key_rows.)"""
+    y = np.asarray(y, dtype=np.float64)
+    flat = np.clip(y.reshape(-1), -E4M3_MAX, E4M3_MAX)
+    hi = np.clip(np.searchsorted(_FINITE_V, flat, side="left"), 1, len(_FINITE_V) - 1)
+    lo = hi - 1
+    d_lo = flat - _FINITE_V[lo]
+    d_hi = _FINITE_V[hi] - flat
+    pick_hi = d_hi < d_lo
+    tie = d_hi == d_lo
+    even_hi = (_FINITE[hi] & 1) == 0
+    pick_hi = np.where(tie, even_hi, pick_hi)
+    codes = np.where(pick_hi, _FINITE[hi], _FINITE[lo]).astype(np.uint8)
+    # a negative value (or -0) that rounds to zero keeps its sign: 0x80
+    codes = np.where((codes == 0) & np.signbit(flat), np.uint8(0x80), codes)
+    return codes.reshape(y.shape)
+
+
+def quantize_key_rows(bits: np.ndarray):
+    """The key-write path's quantisation of bf16 index keys to e4m3 with one
+    scale per token (reading: s_t = amax_t / 448, 1 when the row is zero; each
+    element x / s_t rounded to nearest even with saturation; amax, the scale
+    and the quotient in fp32 as the keys arrive in bf16).
+    Returns (codes uint8 [..., 128], scale float32 [...])."""
+    x = decode_bf16(bits).astype(np.float32)
+    amax = np.abs(x).max(axis=-1)
+    scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    y = (x / scale[..., None]).astype(np.float32)
+    return encode_e4m3(y), scale
+
+
 def decode_bf16(bits: np.ndarray) -> np.ndarray:
     """bf16 bit patterns -> float64 (bf16 is the top half of an IEEE binary32)."""
     with np.errstate(invalid="ignore"):
