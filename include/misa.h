@@ -154,6 +154,27 @@ MISA_API misa_status misa_pool_keys(const misa_cache *cache, const void *new_key
                            const int32_t *new_pos, int32_t count, misa_stream stream);
 
 /*
+ * The key-write path of an e4m3 cache fed bf16 index keys: quantise and
+ * append in one pass.  The pages keep the index keys in the model's cache and
+ * say nothing of their number format; this call has no counterpart there.
+ * For every s with new_pos[s] >= 0, each new key row x = new_keys[s][j]
+ * (bf16 bit patterns, layout [n_seq][count][d], 16-byte aligned) becomes
+ *     scale = amax_e |x_e| / 448   (1 for a row of zeros),
+ *     code_e = e4m3(x_e / scale)   rounded to nearest even, saturated to +-448,
+ * with amax, the scale and the quotient in fp32 (IEEE division); codes and
+ * scale are written at position new_pos[s] + j, seq_len[s] becomes
+ * new_pos[s] + count, and every block holding a written position gets its
+ * mean recomputed in the same kernel (from the quantised keys, as
+ * misa_pool_keys would).  new_pos[s] < 0 leaves sequence s untouched; an
+ * append past L_cap skips the sequence and sets MISA_DEV_APPEND_RANGE.
+ * Errors: MISA_ERR_INVALID for a cache that does not hold e4m3 keys, count
+ * outside [1, 64], NULL or misaligned new_keys, NULL new_pos (and the
+ * checks of misa_pool_keys on the cache).
+ */
+MISA_API misa_status misa_append_keys_e4m3(const misa_cache *cache, const uint16_t *new_keys,
+                                           const int32_t *new_pos, int32_t count, misa_stream stream);
+
+/*
  * Block-pooled head router ("Methodology: MISA", step 1): per-head affinities
  * against the pooled keys, aggregated into a head importance, then the top-h
  * heads of each query.  Importance of head j for query i with prefix L_i:

@@ -235,6 +235,22 @@ misa_status misa_pool_keys(const misa_cache *cache, const void *new_keys, const 
   return MISA_OK;
 }
 
+misa_status misa_append_keys_e4m3(const misa_cache *cache, const uint16_t *new_keys, const int32_t *new_pos,
+                                  int32_t count, misa_stream stream) {
+  misa_status st = check_cache(cache, true);
+  if (st != MISA_OK) return st;
+  if (cache->dtype != MISA_KEY_FP8_E4M3) return fail(MISA_ERR_INVALID, "the cache does not hold e4m3 keys");
+  if (count < 1 || count > misa::pool_append_quant_max())
+    return fail(MISA_ERR_INVALID, "count=%d outside [1, %d]", count, misa::pool_append_quant_max());
+  if (count > cache->L_cap) return fail(MISA_ERR_INVALID, "count=%d above L_cap=%d", count, cache->L_cap);
+  if (!new_keys || !new_pos) return fail(MISA_ERR_INVALID, "new_keys and new_pos must be non-NULL");
+  if (!aligned16(new_keys)) return fail(MISA_ERR_INVALID, "new_keys must be 16-byte aligned");
+  if (injected_failure("misa_append_keys_e4m3", &st)) return st;
+  cudaError_t e = misa::launch_pool_append_quant(view(cache), new_keys, new_pos, count, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "misa_append_keys_e4m3");
+  return MISA_OK;
+}
+
 size_t misa_workspace_bytes(int32_t op, const misa_cache *cache, const misa_queries *qs, int32_t h, int32_t k,
                             int32_t k_prime) {
   (void)h;

@@ -17,6 +17,11 @@ constexpr int TOPK_HIST_BINS = 2048;
 cudaError_t launch_pool_rebuild(const CacheView &c, cudaStream_t s);
 cudaError_t launch_pool_append(const CacheView &c, const void *new_keys, const float *new_scale,
                                const int32_t *new_pos, int count, cudaStream_t s);
+// e4m3 caches: bf16 keys quantised (one scale per token) while appended;
+// count <= pool_append_quant_max()
+int pool_append_quant_max();
+cudaError_t launch_pool_append_quant(const CacheView &c, const uint16_t *new_keys, const int32_t *new_pos, int count,
+                                     cudaStream_t s);
 
 // route.cu
 int route_chunks(int M_cap);

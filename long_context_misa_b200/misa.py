@@ -60,6 +60,7 @@ def _load() -> ctypes.CDLL:
     C, Q = ctypes.POINTER(misa_cache), ctypes.POINTER(misa_queries)
     sig = {
         "misa_pool_keys": (I32, [C, P, P, P, I32, P]),
+        "misa_append_keys_e4m3": (I32, [C, P, P, I32, P]),
         "misa_route_heads": (I32, [C, Q, I32, P, P, P, SZ, P]),
         "misa_score_topk": (I32, [C, Q, P, I32, I32, P, P, P, SZ, P]),
         "dsa_dense_score_topk": (I32, [C, Q, I32, P, P, P, SZ, P]),
@@ -217,6 +218,14 @@ def pool_keys(cache: KeyCache, new_keys: Optional[torch.Tensor] = None, new_scal
     count = 0 if new_keys is None else int(new_keys.shape[1])
     _check(_lib.misa_pool_keys(ctypes.byref(cache.struct), _ptr(new_keys), _ptr(new_scale), _ptr(new_pos), count,
                                _stream(stream)))
+
+
+def append_keys_e4m3(cache: KeyCache, new_keys_bf16: torch.Tensor, new_pos: torch.Tensor, stream=None) -> None:
+    """Quantise bf16 keys new_keys_bf16 [n_seq][count][128] (int16 bit patterns)
+    to e4m3 with one scale per token and append them at new_pos (see misa.h)."""
+    count = int(new_keys_bf16.shape[1])
+    _check(_lib.misa_append_keys_e4m3(ctypes.byref(cache.struct), _ptr(new_keys_bf16), _ptr(new_pos), count,
+                                      _stream(stream)))
 
 
 def route_heads(cache: KeyCache, qs: Queries, h: int, heads: Optional[torch.Tensor] = None,

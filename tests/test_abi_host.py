@@ -30,7 +30,7 @@ by = ctypes.byref
 
 def test_exports_every_declared_symbol():
     names = M.header_symbols()
-    assert len(names) == 14
+    assert len(names) == 15
     for n in names:
         assert hasattr(L, n), n
     assert M.version() == 1
@@ -145,3 +145,16 @@ def test_dagger_argument_checks():
 def test_wait_timeout_argument_checks():
     assert L.misa_debug_wait_timeout(None, 1000, None) == M.MISA_ERR_INVALID
     assert L.misa_debug_wait_timeout(FAKE, 11_000_000_000, None) == M.MISA_ERR_INVALID
+
+
+def test_append_keys_e4m3_argument_checks():
+    fp8 = cache(dtype=M.MISA_KEY_FP8_E4M3, scale=FAKE)
+    ok = dict(keys=FAKE, pos=FAKE, count=1)
+    assert L.misa_append_keys_e4m3(by(cache()), FAKE, FAKE, 1, None) == M.MISA_ERR_INVALID      # bf16 cache
+    assert L.misa_append_keys_e4m3(by(fp8), FAKE, FAKE, 0, None) == M.MISA_ERR_INVALID          # count < 1
+    assert L.misa_append_keys_e4m3(by(fp8), FAKE, FAKE, 65, None) == M.MISA_ERR_INVALID         # count > 64
+    assert L.misa_append_keys_e4m3(by(fp8), None, FAKE, 1, None) == M.MISA_ERR_INVALID          # no keys
+    assert L.misa_append_keys_e4m3(by(fp8), FAKE + 8, FAKE, 1, None) == M.MISA_ERR_INVALID      # misaligned
+    assert L.misa_append_keys_e4m3(by(fp8), FAKE, None, 1, None) == M.MISA_ERR_INVALID          # no positions
+    M.debug_fail_next(1)
+    assert L.misa_append_keys_e4m3(by(fp8), ok["keys"], ok["pos"], ok["count"], None) == M.MISA_ERR_CUDA

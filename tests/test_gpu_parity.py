@@ -112,6 +112,49 @@ def test_pool_append(case, count):
     assert device_status(cache) == 0
 
 
+@pytest.mark.parametrize("count", [1, 7, 64])
+def test_append_keys_e4m3(count):
+    # bf16 keys quantised to e4m3 with one scale per token on the way into the
+    # cache: codes and scales bit-exact against the oracle's encoder, block
+    # means within tolerance of the oracle's pool of the updated cache
+    inp = make("fp8_mixture")
+    wl = inp.wl
+    rng = np.random.default_rng(11 + count)
+    x = (rng.standard_normal((wl.n_seq, count, 128)) * rng.uniform(0.01, 100.0, (wl.n_seq, count, 1))).astype(np.float32)
+    x[0, 0] = 0.0                                          # a zero row: scale 1, codes 0
+    x[1, 0, :64] = -0.0                                    # negative zeros keep their sign
+    x[1, 0, 64:] = rng.standard_normal(64).astype(np.float32) * 1e-3   # values that land in the subnormal range
+    x[2, count - 1] *= 1e6                                 # large magnitudes
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)
+    L = inp.seq_len.astype(np.int64)
+    pos = np.array([100, int(L[1]) - count, -1], dtype=np.int32)   # middle, the end, untouched
+    cache, _ = to_device(inp, torch)
+    M.pool_keys(cache)
+    M.append_keys_e4m3(cache, torch.from_numpy(bits.view(np.int16)).cuda().contiguous(),
+                       torch.from_numpy(pos).cuda())
+    codes, scale = O.quantize_key_rows(bits)
+    keys = cache.keys.cpu().numpy()
+    sc = cache.scale.cpu().numpy()
+    seq_len = cache.seq_len.cpu().numpy()
+    new_keys, new_scale = inp.keys.copy(), inp.scale.copy()
+    for s in range(wl.n_seq):
+        if pos[s] < 0:
+            assert seq_len[s] == L[s]
+            assert np.array_equal(keys[s], inp.keys[s]) and np.array_equal(sc[s], inp.scale[s])
+            continue
+        p0 = int(pos[s])
+        assert seq_len[s] == p0 + count
+        np.testing.assert_array_equal(keys[s, p0:p0 + count], codes[s], err_msg=f"codes seq {s}")
+        np.testing.assert_array_equal(sc[s, p0:p0 + count], scale[s], err_msg=f"scales seq {s}")
+        new_keys[s, p0:p0 + count], new_scale[s, p0:p0 + count] = codes[s], scale[s]
+    pool = cache.pool.cpu().numpy()
+    for s in range(wl.n_seq):
+        n = int(seq_len[s])
+        expect = O.pool_keys(O.seq_keys(new_keys, new_scale, "fp8", s, n), n, wl.B)
+        assert_close(pool[s, :expect.shape[0]], expect, f"pool after quantised append seq {s}")
+    assert device_status(cache) == 0
+
+
 def test_pool_append_past_capacity_is_flagged():
     inp = make("bf16_mixture")
     cache, _ = to_device(inp, torch)
