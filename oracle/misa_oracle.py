@@ -23,9 +23,10 @@ selection).  For fp8 keys the dequantised key is s_t * e4m3(code_t).
 Readings where the pages are silent (each also listed in the design notes):
 
 * router aggregation: r_j = |w_j| * sum_m ReLU(q_j . kbar_m)  ("aggregates
-  these scores to estimate each head's importance", [SUM] step 1);
+  these scores to estimate each head's importance", [SUM] step 1), with the
+  signed-w, unweighted and |w| * max variants available (router_scores agg);
   parity unpinned as to the choice of aggregation (no printed number separates
-  it from signed-w, unweighted or max variants);
+  them);
 * pooled key kbar_m = arithmetic mean of the keys present in block m; a
   trailing partial block is averaged over the tokens it holds (the ceiling in
   M = ceil(L / B)); a query's prefix is tokens 0..p_i inclusive;
@@ -187,15 +188,34 @@ def index_scores(q: np.ndarray, w: np.ndarray, K: np.ndarray, heads: Sequence[in
     return I
 
 
+# Router aggregations ("aggregates these scores to estimate each head's
+# importance", [SUM] "Methodology: MISA" step 1, says no more).  The default
+# is the first; the others are the plain alternatives the wording allows.
+AGG_ABS_SUM = 0     # r_j = |w_j| * sum_m ReLU(a_jm)
+AGG_SIGNED_SUM = 1  # r_j =  w_j  * sum_m ReLU(a_jm)
+AGG_SUM = 2         # r_j =         sum_m ReLU(a_jm)
+AGG_ABS_MAX = 3     # r_j = |w_j| * max_m ReLU(a_jm)
+
+
 def router_scores(q: np.ndarray, w: np.ndarray, pooled: np.ndarray,
-                  counter: Optional[Counter] = None) -> np.ndarray:
-    """Head importance r_j = |w_j| * sum_m ReLU(q_j . kbar_m) over the pooled keys.
+                  counter: Optional[Counter] = None, agg: int = AGG_ABS_SUM) -> np.ndarray:
+    """Head importance from the affinities a_jm = q_j . kbar_m with the pooled keys.
 
     [SUM] "Methodology: MISA", step 1: per-head affinities against the
-    block-level statistics, aggregated into a per-head importance.
+    block-level statistics, aggregated into a per-head importance.  agg picks
+    the aggregation (AGG_* above; the default |w_j| * sum_m ReLU(a_jm)).
     """
-    A = head_token_scores(q, pooled, range(q.shape[0]), counter)
-    return np.abs(w.astype(np.float64)) * np.maximum(A, 0.0).sum(axis=1)
+    A = np.maximum(head_token_scores(q, pooled, range(q.shape[0]), counter), 0.0)
+    w64 = w.astype(np.float64)
+    if agg == AGG_ABS_SUM:
+        return np.abs(w64) * A.sum(axis=1)
+    if agg == AGG_SIGNED_SUM:
+        return w64 * A.sum(axis=1)
+    if agg == AGG_SUM:
+        return A.sum(axis=1)
+    if agg == AGG_ABS_MAX:
+        return np.abs(w64) * (A.max(axis=1) if A.shape[1] else np.zeros(A.shape[0]))
+    raise ValueError(agg)
 
 
 def top_h(r: np.ndarray, h: int) -> np.ndarray:
@@ -224,19 +244,19 @@ def top_k(I: np.ndarray, k: int, index: Optional[np.ndarray] = None) -> np.ndarr
 # --------------------------------------------------------------------------
 
 
-def route_query(q, w, K, L_i, B, h, counter=None):
+def route_query(q, w, K, L_i, B, h, counter=None, agg=AGG_ABS_SUM):
     """Router for one query with prefix length L_i: returns (r [H], heads [h])."""
     pooled = pool_keys(K, L_i, B)
-    r = router_scores(q, w, pooled, counter)
+    r = router_scores(q, w, pooled, counter, agg)
     return r, top_h(r, h)
 
 
-def misa_query(q, w, K, L_i, B, h, k, counter=None):
+def misa_query(q, w, K, L_i, B, h, k, counter=None, agg=AGG_ABS_SUM):
     """MISA: route, score the prefix with the routed heads, keep top-k.
 
     Returns dict(r, heads, scores, topk).
     """
-    r, heads = route_query(q, w, K, L_i, B, h, counter)
+    r, heads = route_query(q, w, K, L_i, B, h, counter, agg)
     I = index_scores(q, w, K[:L_i], heads, counter)
     return dict(r=r, heads=heads, scores=I, topk=top_k(I, k))
 
