@@ -13,8 +13,9 @@ import tests.test_oracle_pins as pins
 
 MUTATIONS = {
     "score_without_relu": ("I += w[j] * np.maximum(A[r], 0.0)", "I += w[j] * A[r]"),
-    "router_signed_w": ("np.abs(w.astype(np.float64)) * np.maximum", "w.astype(np.float64) * np.maximum"),
-    "router_without_relu": ("np.maximum(A, 0.0).sum(axis=1)", "A.sum(axis=1)"),
+    "router_signed_w": ("return np.abs(w64) * A.sum(axis=1)", "return w64 * A.sum(axis=1)"),
+    "router_without_relu": ("A = np.maximum(head_token_scores(q, pooled, range(q.shape[0]), counter), 0.0)",
+                            "A = head_token_scores(q, pooled, range(q.shape[0]), counter)"),
     "pool_divides_by_B": ("out[m] = blk.sum(axis=0) / blk.shape[0]", "out[m] = blk.sum(axis=0) / B"),
     "pool_full_block_tail": ("blk = K[m * B:min((m + 1) * B, L)]", "blk = K[m * B:(m + 1) * B]"),
     "topk_ties_to_high_index": ("order = np.lexsort((idx, -I))", "order = np.lexsort((-idx, -I))"),
