@@ -192,6 +192,27 @@ MISA_API misa_status misa_route_heads(const misa_cache *cache, const misa_querie
                              void *ws, size_t ws_bytes, misa_stream stream);
 
 /*
+ * The same router with the aggregation chosen.  The pages say only that the
+ * per-block affinities a_jm = q_j . kbar_m are aggregated into a head
+ * importance; misa_route_heads takes the first reading below, the others are
+ * the plain alternatives the wording allows:
+ *   MISA_AGG_ABS_SUM     r_j = |w_j| * sum_m ReLU(a_jm)
+ *   MISA_AGG_SIGNED_SUM  r_j =  w_j  * sum_m ReLU(a_jm)
+ *   MISA_AGG_SUM         r_j =         sum_m ReLU(a_jm)
+ *   MISA_AGG_ABS_MAX     r_j = |w_j| * max_m ReLU(a_jm)
+ * (the causal tail block counts like any other block).  Same arguments,
+ * outputs and errors as misa_route_heads, plus MISA_ERR_INVALID for an
+ * unknown agg.
+ */
+#define MISA_AGG_ABS_SUM 0
+#define MISA_AGG_SIGNED_SUM 1
+#define MISA_AGG_SUM 2
+#define MISA_AGG_ABS_MAX 3
+MISA_API misa_status misa_route_heads_agg(const misa_cache *cache, const misa_queries *qs, int32_t h, int32_t agg,
+                                          int32_t *heads, float *router_scores, void *ws, size_t ws_bytes,
+                                          misa_stream stream);
+
+/*
  * Routed sparse token scoring and top-k ("Methodology: MISA", step 2: only
  * the h selected heads score every prefix token; the top-k tokens are taken
  * on these reduced scores).

@@ -273,18 +273,25 @@ size_t misa_workspace_bytes(int32_t op, const misa_cache *cache, const misa_quer
   }
 }
 
-misa_status misa_route_heads(const misa_cache *cache, const misa_queries *qs, int32_t h, int32_t *heads,
-                             float *router_scores, void *ws, size_t ws_bytes, misa_stream stream) {
+misa_status misa_route_heads_agg(const misa_cache *cache, const misa_queries *qs, int32_t h, int32_t agg,
+                                 int32_t *heads, float *router_scores, void *ws, size_t ws_bytes,
+                                 misa_stream stream) {
   misa_status st = check_cache(cache, true);
   if (st != MISA_OK) return st;
   if ((st = check_queries(qs)) != MISA_OK) return st;
   if (h < 1 || h > qs->H) return fail(MISA_ERR_INVALID, "h=%d outside [1, H=%d]", h, qs->H);
+  if (agg < MISA_AGG_ABS_SUM || agg > MISA_AGG_ABS_MAX) return fail(MISA_ERR_INVALID, "agg=%d unknown", agg);
   if (qs->n_q > 0 && !heads) return fail(MISA_ERR_INVALID, "heads is NULL");
   if ((st = check_ws(ws, ws_bytes, misa_workspace_bytes(MISA_OP_ROUTE, cache, qs, h, 0, 0))) != MISA_OK) return st;
   if (injected_failure("misa_route_heads", &st)) return st;
-  cudaError_t e = misa::launch_route(view(cache), view(qs), h, heads, router_scores, ws, stream);
+  cudaError_t e = misa::launch_route(view(cache), view(qs), h, heads, router_scores, ws, stream, agg);
   if (e != cudaSuccess) return cuda_fail(e, "misa_route_heads");
   return MISA_OK;
+}
+
+misa_status misa_route_heads(const misa_cache *cache, const misa_queries *qs, int32_t h, int32_t *heads,
+                             float *router_scores, void *ws, size_t ws_bytes, misa_stream stream) {
+  return misa_route_heads_agg(cache, qs, h, MISA_AGG_ABS_SUM, heads, router_scores, ws, ws_bytes, stream);
 }
 
 misa_status misa_score_topk(const misa_cache *cache, const misa_queries *qs, const int32_t *heads, int32_t h,

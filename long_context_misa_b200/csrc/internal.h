@@ -23,17 +23,21 @@ int pool_append_quant_max();
 cudaError_t launch_pool_append_quant(const CacheView &c, const uint16_t *new_keys, const int32_t *new_pos, int count,
                                      cudaStream_t s);
 
-// route.cu
+// route.cu.  agg: the aggregation of the block affinities into a head's
+// importance (MISA_AGG_* of misa.h): weight factor |w|, w or 1, and a sum or
+// a maximum over the blocks.
+__host__ __device__ inline bool agg_is_max(int agg) { return agg == 3; }
+__device__ inline float agg_weight(int agg, float w) { return agg == 1 ? w : agg == 2 ? 1.f : fabsf(w); }
 int route_chunks(int M_cap);
 size_t route_ws_bytes(int n_q, int H, int M_cap);
 cudaError_t launch_route(const CacheView &c, const QueryView &q, int h, int32_t *heads, float *router_scores,
-                         void *ws, cudaStream_t s);
+                         void *ws, cudaStream_t s, int agg = 0);
 // route_umma.cu: the same routing for many queries per sequence (prefill) on
 // tcgen05 tensor cores; launch_route dispatches to it when it applies.
 bool route_umma_applies(const CacheView &c, const QueryView &q);
 size_t route_umma_ws_bytes(int n_q, int H, int M_cap, int n_seq);
 cudaError_t launch_route_umma(const CacheView &c, const QueryView &q, int h, int32_t *heads, float *router_scores,
-                              void *ws, cudaStream_t s);
+                              void *ws, cudaStream_t s, int agg = 0);
 
 // score_mma.cu: scores[i][t] (row stride ld) for t < L_i, heads given per query
 // (heads == nullptr: all H heads, dense).  `gather` != nullptr: row i scores the

@@ -44,7 +44,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
 }
 
 __global__ void __launch_bounds__(ROUTE_THREADS) route_partial_kernel(CacheView c, QueryView qv, float *partial,
-                                                                      int n_chunks) {
+                                                                      int n_chunks, int agg) {
   extern __shared__ __align__(16) float smem[];
   float *p_s = smem;                          // [RB][PSTRIDE] pooled keys (fp32)
   float *part = p_s + RB * PSTRIDE;           // [16][128] key-sum scratch
@@ -147,8 +147,13 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_partial_kernel(CacheView 
   }
 #pragma unroll
   for (int nt = 0; nt < MAX_NT; ++nt) {
-    racc[nt][0] = fmaxf(acc[nt][0], 0.f) + fmaxf(acc[nt][2], 0.f);  // head 8nt + 2cq
-    racc[nt][1] = fmaxf(acc[nt][1], 0.f) + fmaxf(acc[nt][3], 0.f);  // head 8nt + 2cq + 1
+    if (agg_is_max(agg)) {
+      racc[nt][0] = fmaxf(fmaxf(acc[nt][0], 0.f), fmaxf(acc[nt][2], 0.f));
+      racc[nt][1] = fmaxf(fmaxf(acc[nt][1], 0.f), fmaxf(acc[nt][3], 0.f));
+    } else {
+      racc[nt][0] = fmaxf(acc[nt][0], 0.f) + fmaxf(acc[nt][2], 0.f);  // head 8nt + 2cq
+      racc[nt][1] = fmaxf(acc[nt][1], 0.f) + fmaxf(acc[nt][3], 0.f);  // head 8nt + 2cq + 1
+    }
   }
   // sum over the 8 row groups of the warp (lanes with equal cq)
 #pragma unroll
@@ -156,7 +161,10 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_partial_kernel(CacheView 
 #pragma unroll
     for (int u = 0; u < 2; ++u)
 #pragma unroll
-      for (int o = 4; o < 32; o <<= 1) racc[nt][u] += __shfl_xor_sync(0xffffffffu, racc[nt][u], o);
+      for (int o = 4; o < 32; o <<= 1) {
+        const float x = __shfl_xor_sync(0xffffffffu, racc[nt][u], o);
+        racc[nt][u] = agg_is_max(agg) ? fmaxf(racc[nt][u], x) : racc[nt][u] + x;
+      }
   if (g == 0) {
 #pragma unroll
     for (int nt = 0; nt < MAX_NT; ++nt)
@@ -169,14 +177,17 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_partial_kernel(CacheView 
   if (tid < H) {
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) v += colsum[w * (MAX_NT * 8) + tid];
+    for (int w = 0; w < 4; ++w) {
+      const float x = colsum[w * (MAX_NT * 8) + tid];
+      v = agg_is_max(agg) ? fmaxf(v, x) : v + x;
+    }
     partial[((size_t)i * n_chunks + chunk) * H + tid] = v;
   }
 }
 
 __global__ void __launch_bounds__(MISA_MAX_H) route_finish_kernel(CacheView c, QueryView qv, const float *partial,
                                                                   int n_chunks, int h, int32_t *heads,
-                                                                  float *router_scores) {
+                                                                  float *router_scores, int agg) {
   __shared__ float r_s[MISA_MAX_H];
   __shared__ int warp_cnt[MISA_MAX_H / 32];
   const int i = blockIdx.x, j = threadIdx.x, H = qv.H;
@@ -187,8 +198,11 @@ __global__ void __launch_bounds__(MISA_MAX_H) route_finish_kernel(CacheView c, Q
   if (j < H) {
     float acc = 0.f;
 #pragma unroll 16
-    for (int ch = 0; ch < nc; ++ch) acc += __ldg(partial + ((size_t)i * n_chunks + ch) * H + j);
-    r = fabsf(qv.w[(size_t)i * H + j]) * acc;
+    for (int ch = 0; ch < nc; ++ch) {
+      const float x = __ldg(partial + ((size_t)i * n_chunks + ch) * H + j);
+      acc = agg_is_max(agg) ? fmaxf(acc, x) : acc + x;
+    }
+    r = agg_weight(agg, qv.w[(size_t)i * H + j]) * acc;
     r_s[j] = r;
     if (router_scores) router_scores[(size_t)i * H + j] = r;
   }
@@ -221,9 +235,9 @@ size_t route_ws_bytes(int n_q, int H, int M_cap) {
 }
 
 cudaError_t launch_route(const CacheView &c, const QueryView &q, int h, int32_t *heads, float *router_scores,
-                         void *ws, cudaStream_t s) {
+                         void *ws, cudaStream_t s, int agg) {
   if (q.n_q == 0) return cudaSuccess;
-  if (route_umma_applies(c, q)) return launch_route_umma(c, q, h, heads, router_scores, ws, s);
+  if (route_umma_applies(c, q)) return launch_route_umma(c, q, h, heads, router_scores, ws, s, agg);
   const int M_cap = cdiv(c.L_cap, c.B);
   const int n_chunks = route_chunks(M_cap);
   const size_t smem = route_smem_bytes(q.H);
@@ -235,10 +249,11 @@ cudaError_t launch_route(const CacheView &c, const QueryView &q, int h, int32_t 
   if (opt_in < 0) return cudaErrorInvalidConfiguration;
   cudaError_t e;
   float *partial = static_cast<float *>(ws);
-  e = launch_kernel(route_partial_kernel, dim3(n_chunks, q.n_q), dim3(ROUTE_THREADS), smem, s, c, q, partial, n_chunks);
+  e = launch_kernel(route_partial_kernel, dim3(n_chunks, q.n_q), dim3(ROUTE_THREADS), smem, s, c, q, partial, n_chunks,
+                    agg);
   if (e != cudaSuccess) return e;
   return launch_kernel(route_finish_kernel, dim3(q.n_q), dim3(MISA_MAX_H), 0, s, c, q, partial, n_chunks, h, heads,
-                    router_scores);
+                    router_scores, agg);
 }
 
 }  // namespace misa

@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(256) pool_split_kernel(const float4 *pool, siz
 __global__ void __launch_bounds__(RU_THREADS, 2)
     route_umma_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap hmap,
                       const __grid_constant__ CUtensorMap lmap, CacheView c, QueryView qv, float *rsum,
-                      int n_groups, int fuse, int h, int32_t *heads, float *router_scores) {
+                      int n_groups, int fuse, int h, int32_t *heads, float *router_scores, int agg) {
   extern __shared__ uint8_t ru_raw[];
   uint8_t *base = ru_raw + ((1024u - (smem_addr(ru_raw) & 1023u)) & 1023u);  // 1024-aligned (swizzle atoms)
   uint8_t *a_smem = base;
@@ -248,8 +248,9 @@ __global__ void __launch_bounds__(RU_THREADS, 2)
             const int m0 = t * RU_N + ch * 32;
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
-              if (mine && m0 + x < full) acc += fmaxf(__uint_as_float(v0[x]), 0.f);
-              if (mine && m0 + 32 + x < full) acc += fmaxf(__uint_as_float(v1[x]), 0.f);
+              const float r0 = fmaxf(__uint_as_float(v0[x]), 0.f), r1 = fmaxf(__uint_as_float(v1[x]), 0.f);
+              if (mine && m0 + x < full) acc = agg_is_max(agg) ? fmaxf(acc, r0) : acc + r0;
+              if (mine && m0 + 32 + x < full) acc = agg_is_max(agg) ? fmaxf(acc, r1) : acc + r1;
             }
           }
           umma::fence_before();
@@ -326,9 +327,10 @@ __global__ void __launch_bounds__(RU_THREADS, 2)
                 dot = fmaf(f.y, tailm[qg * D + 8 * u + 2 * p + 1], dot);
               }
             }
-            a += fmaxf(dot * (1.f / (float)(Li - t0)), 0.f);
+            const float rt = fmaxf(dot * (1.f / (float)(Li - t0)), 0.f);
+            a = agg_is_max(agg) ? fmaxf(a, rt) : a + rt;
           }
-          rr = fabsf(__ldg(qv.w + (size_t)qi * H + hd)) * a;
+          rr = agg_weight(agg, __ldg(qv.w + (size_t)qi * H + hd)) * a;
           if (router_scores) router_scores[(size_t)qi * H + hd] = rr;
         }
         sh.rsc[r] = rr;
@@ -381,7 +383,8 @@ __global__ void __launch_bounds__(RU_THREADS, 2)
 // the tail affinity), then the h best heads (fewer than h heads beat a kept
 // one: larger r, or equal r and lower index), written in ascending order.
 __global__ void __launch_bounds__(MISA_MAX_H) route_tail_finish_kernel(CacheView c, QueryView qv, const float *rsum,
-                                                                       int h, int32_t *heads, float *router_scores) {
+                                                                       int h, int32_t *heads, float *router_scores,
+                                                                       int agg) {
   __shared__ float part[16 * D];
   __shared__ float tail[D];
   __shared__ float r_s[MISA_MAX_H];
@@ -411,9 +414,10 @@ __global__ void __launch_bounds__(MISA_MAX_H) route_tail_finish_kernel(CacheView
           dot = fmaf(f.y, tail[8 * u + 2 * p + 1], dot);
         }
       }
-      acc += fmaxf(dot * inv, 0.f);
+      const float rt = fmaxf(dot * inv, 0.f);
+      acc = agg_is_max(agg) ? fmaxf(acc, rt) : acc + rt;
     }
-    r = fabsf(qv.w[(size_t)i * H + j]) * acc;
+    r = agg_weight(agg, qv.w[(size_t)i * H + j]) * acc;
     r_s[j] = r;
     if (router_scores) router_scores[(size_t)i * H + j] = r;
   }
@@ -447,7 +451,7 @@ size_t route_umma_ws_bytes(int n_q, int H, int M_cap, int n_seq) {
 bool route_umma_applies(const CacheView &c, const QueryView &q) { return umma_applies(c, q, nullptr, q.H); }
 
 cudaError_t launch_route_umma(const CacheView &c, const QueryView &q, int h, int32_t *heads, float *router_scores,
-                              void *ws, cudaStream_t s) {
+                              void *ws, cudaStream_t s, int agg) {
   if (q.n_q == 0) return cudaSuccess;
   const int M_cap = cdiv(c.L_cap, c.B);
   const size_t split = (((size_t)c.n_seq * M_cap * D * 2) + 255) & ~size_t(255);
@@ -473,10 +477,10 @@ cudaError_t launch_route_umma(const CacheView &c, const QueryView &q, int h, int
   const int n_groups = cdiv(q.n_q * q.H, RU_M);
   const int fuse = q.H >= 16 && q.H <= RU_M && RU_M % q.H == 0;  // groups of whole queries: finish in the kernel
   e = launch_kernel(route_umma_kernel, dim3(n_groups), dim3(RU_THREADS), SMEM, s, qmap, hmap, lmap, c, q, rsum,
-                    n_groups, fuse, h, heads, router_scores);
+                    n_groups, fuse, h, heads, router_scores, agg);
   if (e != cudaSuccess || fuse) return e;
   return launch_kernel(route_tail_finish_kernel, dim3(q.n_q), dim3(MISA_MAX_H), 0, s, c, q, rsum, h, heads,
-                       router_scores);
+                       router_scores, agg);
 }
 
 }  // namespace misa

@@ -62,6 +62,7 @@ def _load() -> ctypes.CDLL:
         "misa_pool_keys": (I32, [C, P, P, P, I32, P]),
         "misa_append_keys_e4m3": (I32, [C, P, P, I32, P]),
         "misa_route_heads": (I32, [C, Q, I32, P, P, P, SZ, P]),
+        "misa_route_heads_agg": (I32, [C, Q, I32, I32, P, P, P, SZ, P]),
         "misa_score_topk": (I32, [C, Q, P, I32, I32, P, P, P, SZ, P]),
         "dsa_dense_score_topk": (I32, [C, Q, I32, P, P, P, SZ, P]),
         "misa_rerank_topk": (I32, [C, Q, P, I32, I32, P, P, P, SZ, P]),
@@ -228,15 +229,23 @@ def append_keys_e4m3(cache: KeyCache, new_keys_bf16: torch.Tensor, new_pos: torc
                                       _stream(stream)))
 
 
+AGG_ABS_SUM, AGG_SIGNED_SUM, AGG_SUM, AGG_ABS_MAX = 0, 1, 2, 3  # router aggregations (misa.h)
+
+
 def route_heads(cache: KeyCache, qs: Queries, h: int, heads: Optional[torch.Tensor] = None,
                 router_scores: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None,
-                stream=None) -> torch.Tensor:
+                stream=None, agg: int = AGG_ABS_SUM) -> torch.Tensor:
+    """misa_route_heads, or misa_route_heads_agg for another aggregation."""
     dev = qs.q.device
     if heads is None:
         heads = torch.empty(qs.n_q, h, dtype=torch.int32, device=dev)
     buf, nb = _ws(ws, workspace_bytes(OP_ROUTE, cache, qs, h), dev)
-    _check(_lib.misa_route_heads(ctypes.byref(cache.struct), ctypes.byref(qs.struct), h, _ptr(heads),
-                                 _ptr(router_scores), _ptr(buf), nb, _stream(stream)))
+    args = (ctypes.byref(cache.struct), ctypes.byref(qs.struct), h)
+    tail = (_ptr(heads), _ptr(router_scores), _ptr(buf), nb, _stream(stream))
+    if agg == AGG_ABS_SUM:
+        _check(_lib.misa_route_heads(*args, *tail))
+    else:
+        _check(_lib.misa_route_heads_agg(*args, agg, *tail))
     return heads
 
 

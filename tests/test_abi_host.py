@@ -30,7 +30,7 @@ by = ctypes.byref
 
 def test_exports_every_declared_symbol():
     names = M.header_symbols()
-    assert len(names) == 15
+    assert len(names) == 16
     for n in names:
         assert hasattr(L, n), n
     assert M.version() == 1
@@ -158,3 +158,9 @@ def test_append_keys_e4m3_argument_checks():
     assert L.misa_append_keys_e4m3(by(fp8), FAKE, None, 1, None) == M.MISA_ERR_INVALID          # no positions
     M.debug_fail_next(1)
     assert L.misa_append_keys_e4m3(by(fp8), ok["keys"], ok["pos"], ok["count"], None) == M.MISA_ERR_CUDA
+
+
+def test_route_agg_argument_checks():
+    for agg in (-1, 4):
+        assert L.misa_route_heads_agg(by(cache()), by(queries()), 8, agg, FAKE, None, FAKE, 1 << 30, None) == \
+            M.MISA_ERR_INVALID

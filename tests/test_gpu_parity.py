@@ -190,6 +190,40 @@ def test_route_heads(case, h):
     assert device_status(cache) == 0
 
 
+# routing cases for the aggregation variants: the decode router, the tcgen05
+# router with its finish fused (64 and 32 heads, one and two sequences per
+# group) and with the separate finishing kernel (24 heads do not divide 128)
+AGG_CASES = {
+    "bf16_mixture": None,
+    "bf16_prefill": None,
+    "fp8_prefill_umma": None,
+    "bf16_prefill_2seq": None,
+    "prefill_h24": W["causal_prefill"].scaled(L=1500, n_q=70, H=24, k=64),
+}
+
+
+@pytest.mark.parametrize("case", sorted(AGG_CASES))
+@pytest.mark.parametrize("agg", [M.AGG_SIGNED_SUM, M.AGG_SUM, M.AGG_ABS_MAX])
+def test_route_heads_aggregations(case, agg):
+    inp = make(AGG_CASES[case] or case)
+    ref = Ref(inp)
+    wl = inp.wl
+    cache, qs = to_device(inp, torch)
+    M.pool_keys(cache)
+    r_gpu = torch.empty(wl.n_q, wl.H, dtype=torch.float32, device="cuda")
+    heads = M.route_heads(cache, qs, wl.h, router_scores=r_gpu, agg=agg).cpu().numpy()
+    r_gpu = r_gpu.cpu().numpy()
+    ties = 0
+    for i in range(wl.n_q):
+        q, w, K, Li = ref.query(i)
+        r, hs = O.route_query(q, w, K, Li, wl.B, wl.h, agg=agg)
+        assert_close(r_gpu[i], r, f"router scores q{i} agg {agg}")
+        assert np.all(np.diff(heads[i]) > 0)
+        ties += compare_selection(heads[i], hs, lambda j: r[j], wl.h, f"heads q{i} agg {agg}")
+    assert ties <= max(1, wl.n_q // 10), f"{ties} head boundary ties"
+    assert device_status(cache) == 0
+
+
 def _score_case(case, kind, k=None, h=None, seed=0):
     inp = make(case, seed)
     ref = Ref(inp)
