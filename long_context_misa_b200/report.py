@@ -1,10 +1,13 @@
 """Per-workload measurement report for the five synthetic workloads.
 
 Usage (one GPU):  python -m long_context_misa_b200.report [--workloads NAME ...]
-                  [--n-q N] [--no-dense]
+                  [--n-q N] [--no-dense] [--router-sweep]
 
 --n-q N keeps the first N queries of each workload (smaller captures of the
 same kernels for profilers); --no-dense skips the dense DSA calls.
+--router-sweep instead reports, per workload, router aggregation
+(misa_route_heads_agg) and routed head count h, the recall and IoU of MISA's
+top-k against dense DSA's and the share of planted needles MISA selects.
 
 For every workload of ``inputs.WORKLOADS`` at full size: the MISA call
 (route + routed score + top-k; MISA-dagger through ``dagger_topk`` where the
@@ -90,12 +93,42 @@ def overlap(sel, ref):
     return float(np.mean(rec)), float(np.mean(iou))
 
 
+AGG_NAMES = {M.AGG_ABS_SUM: "|w| sum", M.AGG_SIGNED_SUM: "w sum", M.AGG_SUM: "sum", M.AGG_ABS_MAX: "|w| max"}
+
+
+def router_sweep(names, dev):
+    print("| workload | aggregation | h | recall / IoU vs dense | needles selected |")
+    print("|---|---|---|---|---|")
+    for name in names:
+        wl = G.WORKLOADS[name]
+        inp = G.make_inputs(wl, 0)
+        cache, qs = M.device_inputs(inp, dev)
+        M.pool_keys(cache)
+        ws = M.Workspace(dev)
+        dense = M.dense_score_topk(cache, qs, wl.k, ws=ws).cpu().numpy()
+        for agg in AGG_NAMES:
+            for h in (4, 8, 16):
+                heads = M.route_heads(cache, qs, h, ws=ws, agg=agg)
+                top = M.score_topk(cache, qs, heads, wl.k, ws=ws).cpu().numpy()
+                hit = [p in set(top[qi].tolist()) for (_, p, qi) in inp.needles]
+                rec, iou = overlap(top, dense)
+                print(f"| {name} | {AGG_NAMES[agg]} | {h} | {rec:.3f} / {iou:.3f} | {sum(hit)} / {len(hit)} |",
+                      flush=True)
+        assert cache.device_status() == 0
+        del cache, qs, ws
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--workloads", nargs="*", default=list(G.WORKLOADS))
     ap.add_argument("--n-q", type=int, default=0)
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--router-sweep", action="store_true")
     args = ap.parse_args()
+    if args.router_sweep:
+        router_sweep(args.workloads, torch.device("cuda"))
+        return
     hbm, tflops, src = _peaks()
     dev = torch.device("cuda")
     flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
