@@ -178,6 +178,7 @@ misa_status score_then_topk(const char *who, const misa_cache *cache, const misa
 // never completes: after limit_ns it records MISA_DEV_WAIT_TIMEOUT and the
 // kernel returns normally (the failure path, exercised without a fault).
 __global__ void wait_timeout_kernel(uint32_t *status, unsigned long long limit_ns) {
+  misa::grid_dep_sync();
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
     misa::mbar_init(&bar, 1);

@@ -115,18 +115,35 @@ __device__ __forceinline__ uint4 ldg_stream(const void *p) {
 
 __host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
 
-// Kernel launch through cudaLaunchKernelEx (one place to set launch
-// attributes; none are needed at present).
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with programmatic stream serialisation and calls grid_dep_sync() as its
+// first statement: the kernel's launch and block scheduling may then overlap
+// the previous kernel's last blocks and its completion, and the wait holds
+// every thread until the previous grid has completed with its writes
+// visible.  No kernel triggers its dependents early, so a successor's blocks
+// are scheduled only as this kernel's blocks exit (waiting successor blocks
+// that sat beside a running prefill kernel cost 45 us of a 0.7 ms call).
+// Because the wait comes before any global access, tensor memory allocation
+// or early return in every kernel, every earlier kernel is complete
+// (transitively) before a kernel reads anything, and no kernel requests
+// tensor memory while its predecessor still holds some.
+__device__ __forceinline__ void grid_dep_sync() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Kernel launch through cudaLaunchKernelEx, with the programmatic
+// serialisation attribute above.
 template <class... KArgs, class... Args>
 inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                                  Args &&...args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cfg.attrs = nullptr;
-  cfg.numAttrs = 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 

@@ -28,6 +28,7 @@ constexpr int REBUILD_THREADS = 128;
 constexpr int APPEND_THREADS = 512;
 
 __global__ void __launch_bounds__(REBUILD_THREADS) pool_rebuild_kernel(CacheView c) {
+  grid_dep_sync();
   __shared__ float sm_part[(REBUILD_THREADS / 8) * D];
   __shared__ float sm_out[D];
   const int s = blockIdx.y, m = blockIdx.x;
@@ -43,6 +44,7 @@ __global__ void __launch_bounds__(REBUILD_THREADS) pool_rebuild_kernel(CacheView
 __global__ void __launch_bounds__(APPEND_THREADS) pool_append_kernel(CacheView c, const void *new_keys,
                                                                      const float *new_scale,
                                                                      const int32_t *new_pos, int count) {
+  grid_dep_sync();
   __shared__ float sm_part[(APPEND_THREADS / 8) * D];
   __shared__ float sm_out[D];
   const int s = blockIdx.x;
@@ -82,6 +84,7 @@ constexpr int QAPPEND_MAX = 64;  // new tokens per sequence in one quantising ap
 
 __global__ void __launch_bounds__(APPEND_THREADS) pool_append_quant_kernel(CacheView c, const uint16_t *new_keys,
                                                                            const int32_t *new_pos, int count) {
+  grid_dep_sync();
   __shared__ float sm_part[(APPEND_THREADS / 8) * D];
   __shared__ float sm_out[D];
   __shared__ __align__(16) uint8_t codes[QAPPEND_MAX * D];

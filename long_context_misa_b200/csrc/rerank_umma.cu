@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
                                                                   int h, const int32_t *gather, int n_cols,
                                                                   float *scores, long long ld,
                                                                   uint32_t *row_hist) {
+  grid_dep_sync();
   using Cfg = RCfg<FP8, HN, TT>;
   constexpr int T = Cfg::T;
   extern __shared__ uint8_t rr_raw[];

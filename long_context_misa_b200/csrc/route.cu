@@ -45,6 +45,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
 
 __global__ void __launch_bounds__(ROUTE_THREADS) route_partial_kernel(CacheView c, QueryView qv, float *partial,
                                                                       int n_chunks, int agg) {
+  grid_dep_sync();
   extern __shared__ __align__(16) float smem[];
   float *p_s = smem;                          // [RB][PSTRIDE] pooled keys (fp32)
   float *part = p_s + RB * PSTRIDE;           // [16][128] key-sum scratch
@@ -188,6 +189,7 @@ __global__ void __launch_bounds__(ROUTE_THREADS) route_partial_kernel(CacheView 
 __global__ void __launch_bounds__(MISA_MAX_H) route_finish_kernel(CacheView c, QueryView qv, const float *partial,
                                                                   int n_chunks, int h, int32_t *heads,
                                                                   float *router_scores, int agg) {
+  grid_dep_sync();
   __shared__ float r_s[MISA_MAX_H];
   __shared__ int warp_cnt[MISA_MAX_H / 32];
   const int i = blockIdx.x, j = threadIdx.x, H = qv.H;

@@ -66,6 +66,7 @@ __device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 v) { return *reinter
 
 // pool (fp32) -> hi, lo (bf16), four elements per step
 __global__ void __launch_bounds__(256) pool_split_kernel(const float4 *pool, size_t n4, uint2 *hi, uint2 *lo) {
+  grid_dep_sync();
   for (size_t x = blockIdx.x * (size_t)256 + threadIdx.x; x < n4; x += (size_t)gridDim.x * 256) {
     const float4 v = __ldg(pool + x);
     const __nv_bfloat162 h01 = __floats2bfloat162_rn(v.x, v.y), h23 = __floats2bfloat162_rn(v.z, v.w);
@@ -81,6 +82,7 @@ __global__ void __launch_bounds__(RU_THREADS, 2)
     route_umma_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap hmap,
                       const __grid_constant__ CUtensorMap lmap, CacheView c, QueryView qv, float *rsum,
                       int n_groups, int fuse, int h, int32_t *heads, float *router_scores, int agg) {
+  grid_dep_sync();
   extern __shared__ uint8_t ru_raw[];
   uint8_t *base = ru_raw + ((1024u - (smem_addr(ru_raw) & 1023u)) & 1023u);  // 1024-aligned (swizzle atoms)
   uint8_t *a_smem = base;
@@ -385,6 +387,7 @@ __global__ void __launch_bounds__(RU_THREADS, 2)
 __global__ void __launch_bounds__(MISA_MAX_H) route_tail_finish_kernel(CacheView c, QueryView qv, const float *rsum,
                                                                        int h, int32_t *heads, float *router_scores,
                                                                        int agg) {
+  grid_dep_sync();
   __shared__ float part[16 * D];
   __shared__ float tail[D];
   __shared__ float r_s[MISA_MAX_H];

@@ -53,6 +53,7 @@ template <int NT, bool FP8>
 __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, QueryView qv, const int32_t *heads,
                                                                int h, float *scores, long long ld, int scale_vec,
                                                                uint32_t *row_hist) {
+  grid_dep_sync();
   using Cfg = StreamCfg<NT, FP8>;
   using F = FragCfg<FP8>;
   constexpr int NS = Cfg::NS, ROW = Cfg::ROW, NV = F::NV, TT = Cfg::TT;

@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(UCfg<FP8, HPQ>::THREADS, 1)
     score_umma_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap omap,
                       int out_tma, CacheView c, QueryView qv, const int32_t *heads, int h, float *scores,
                       long long ld, int n_tiles, long long n_items) {
+  grid_dep_sync();
   using Cfg = UCfg<FP8, HPQ>;
   constexpr int QPT = UM_N / HPQ;
   extern __shared__ uint8_t um_raw[];

@@ -466,6 +466,7 @@ __global__ void __launch_bounds__(SEL_T) select_kernel(CacheView c, QueryView qv
                                                        int n_cols, const int32_t *gather, const uint32_t *row_hist,
                                                        const uint2 *list, const uint32_t *list_cnt, int list_cap,
                                                        int k, int32_t *out) {
+  grid_dep_sync();
   extern __shared__ __align__(16) uint8_t sel_smem[];
   SelShared &sh = *reinterpret_cast<SelShared *>(sel_smem);
   uint32_t *bm = reinterpret_cast<uint32_t *>(sel_smem + sizeof(SelShared));  // token bitmap
@@ -635,6 +636,7 @@ __global__ void __launch_bounds__(FILT_T) filter_kernel(CacheView c, QueryView q
                                                         const uint32_t *row_hist, uint2 *list, uint32_t *list_cnt,
                                                         int list_cap, int k, int chunk, int32_t *out,
                                                         uint32_t *emit_cnt) {
+  grid_dep_sync();
   constexpr int FU = 16;
   const int row = blockIdx.y;
   const int lane = threadIdx.x & 31;
@@ -723,6 +725,7 @@ constexpr int FT_PAD = 4 * FT_V + 4;  // floats per thread in the stash (16-byte
 __global__ void __launch_bounds__(FT_T) filter_thr_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
                                                           const uint32_t *thr, uint2 *list, uint32_t *list_cnt,
                                                           int list_cap, int chunk) {
+  grid_dep_sync();
   __shared__ __align__(16) float stash[FT_T * FT_PAD];
   const int row = blockIdx.y;
   const int lane = threadIdx.x & 31;
@@ -796,6 +799,7 @@ __global__ void __launch_bounds__(FT_T) filter_thr_kernel(CacheView c, QueryView
 constexpr int HIST_T = 256;
 __global__ void __launch_bounds__(HIST_T) hist_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
                                                       uint32_t *row_hist, int chunk) {
+  grid_dep_sync();
   constexpr int HU = 16;
   __shared__ uint32_t hs[RB];
   const int row = blockIdx.y;
@@ -927,6 +931,7 @@ constexpr int SMP_BLOCKS = 256;
 constexpr int SMP_N = SMP_BLOCKS * SMP_BL;
 __global__ void __launch_bounds__(SMP_T) sample_thr_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
                                                            int k, uint32_t *thr) {
+  grid_dep_sync();
   __shared__ uint32_t hs[RB];
   __shared__ Boundary sb;
   const int row = blockIdx.x;
@@ -997,6 +1002,7 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
                                                             const uint32_t *row_hist, const uint2 *list,
                                                             const uint32_t *list_cnt, int list_cap, int stage_cap,
                                                             int d0cap, int k, int32_t *out) {
+  grid_dep_sync();
   extern __shared__ __align__(16) uint8_t fs_smem[];
   FastShared &sh = *reinterpret_cast<FastShared *>(fs_smem);
   uint8_t *data = fs_smem + sizeof(FastShared);  // 16-byte aligned (sizeof is a multiple of 16)
@@ -1234,6 +1240,7 @@ cudaError_t launch_select_smem(const CacheView &c, const QueryView &q, const flo
 // Zero n words (the histograms and list counters before a scoring pass); a
 // kernel measured as fast as a memset node in the decode step's graph.
 __global__ void __launch_bounds__(256) zero_kernel(uint32_t *p, size_t n) {
+  grid_dep_sync();
   for (size_t x = blockIdx.x * 256 + threadIdx.x; x < n; x += (size_t)gridDim.x * 256) p[x] = 0u;
 }
 
