@@ -12,7 +12,9 @@ routed per-token scores, computed with the GPU's head set, within tolerance
 over the whole prefix; the routed top-k (k' for MISA-dagger) equal up to
 boundary ties; dense DSA scores and top-k the same way; for MISA-dagger the
 step's final top-k equal to the oracle's re-rank of the GPU's candidates up
-to boundary ties.  The boundary-tie counts are printed per workload.
+to boundary ties; the routed and dense top-k of the call without scores_out
+(scores in the workspace) equal to those with it on every query.
+The boundary-tie counts are printed per workload.
 """
 import numpy as np
 import pytest
@@ -75,12 +77,18 @@ def test_full_size_sampled(name):
     heads = M.route_heads(cache, qs, wl.h, router_scores=r_gpu)
     routed = torch.empty(wl.n_q, wl.L, dtype=torch.float32, device="cuda")
     top = M.score_topk(cache, qs, heads, k_route, scores_out=routed)
+    # without scores_out (the call the throughput figures time) the scores
+    # live in the workspace: every row's selection is the same
+    top_ws = M.score_topk(cache, qs, heads, k_route)
+    assert torch.equal(top_ws, top), f"{name}: routed top-k without scores_out differs"
     heads, r_gpu, top = heads.cpu().numpy(), r_gpu.cpu().numpy(), top.cpu().numpy()
     picks = _sample(inp)
     routed_rows = routed[picks].cpu().numpy()
     del routed
     dense = torch.empty(wl.n_q, wl.L, dtype=torch.float32, device="cuda")
-    dtop = M.dense_score_topk(cache, qs, wl.k, scores_out=dense).cpu().numpy()
+    dtop_t = M.dense_score_topk(cache, qs, wl.k, scores_out=dense)
+    assert torch.equal(M.dense_score_topk(cache, qs, wl.k), dtop_t), f"{name}: dense top-k without scores_out differs"
+    dtop = dtop_t.cpu().numpy()
     dense_rows = dense[picks].cpu().numpy()
     del dense
     torch.cuda.synchronize()
