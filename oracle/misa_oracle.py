@@ -13,6 +13,9 @@ Sources (page titles; sections in quotes):
   renderings carry the same text), sections "Problem statement",
   "Methodology: MISA" (step 1 block-pooled router, step 2 sparse token
   scoring, the complexity sentence), "Hierarchical variant (MISA-dagger)".
+* [DOSA] "DoSA: Dots Sparse Attention" (the Chinese article page and its
+  cached Hugging Face paper page), abstract: exact top-k selection with the
+  indexer's scoring made conditional by a threshold certificate.
 
 The pages do not print the indexer formula.  The reading used here is the DSA
 lightning-indexer form I_t = sum_j w_j * ReLU(q_j . k_t), with one index key
@@ -297,6 +300,68 @@ def dot_product_count(kind: str, L_i: int, B: int, H: int, h: int, k_prime: int 
     if kind == "misa_dagger":
         return h * L_i + H * M + H * min(k_prime, L_i)
     raise ValueError(kind)
+
+
+# --------------------------------------------------------------------------
+# DoSA-style certified pruning of the dense indexer ([DOSA] abstract)
+# --------------------------------------------------------------------------
+# The abstract names the parts and no formula: a seed set whose exact scores
+# bound the admission threshold from below, upper bounds on the positive
+# heads' contributions from projections and a residual bound shared by the
+# heads, and a bound on what the negative heads must subtract from their
+# activations.  The reading written out here works per block of B tokens
+# (the blocks the router pools):
+#   c_b = mean key of the block, rho_b = max_t ||k_t - c_b|| (one radius for
+#   every head), a_j = q_j . c_b; then for t in the block
+#   q_j . k_t lies in [a_j - ||q_j|| rho_b, a_j + ||q_j|| rho_b]
+#   (Cauchy-Schwarz), ReLU is non-decreasing, so
+#   I_t <= U_b = sum_{w_j >= 0} w_j ReLU(a_j + ||q_j|| rho_b)
+#              + sum_{w_j < 0}  w_j ReLU(a_j - ||q_j|| rho_b).
+# A block with U_b below the seed threshold holds no top-k token.
+
+def dosa_block_bounds(q: np.ndarray, w: np.ndarray, K: np.ndarray, L_i: int, B: int) -> np.ndarray:
+    """U_b >= max over the block's tokens of the dense score, for every block of the prefix."""
+    L_i = max(int(L_i), 0)
+    qn = np.sqrt(np.sum(q * q, axis=1))
+    out = np.empty(-(-L_i // B), dtype=np.float64)
+    for b in range(out.size):
+        Kb = K[b * B:min(L_i, (b + 1) * B)]
+        c = Kb.mean(axis=0)
+        rho = float(np.sqrt(np.sum((Kb - c) ** 2, axis=1)).max())
+        U = 0.0
+        for j in range(q.shape[0]):
+            a = float(q[j] @ c)
+            if w[j] >= 0:
+                U += w[j] * max(a + qn[j] * rho, 0.0)
+            else:
+                U += w[j] * max(a - qn[j] * rho, 0.0)
+        out[b] = U
+    return out
+
+
+def dosa_query(q, w, K, L_i, k, B, seed) -> dict:
+    """Exact dense top-k with the block certificate.
+
+    tau = the k-th largest exact dense score among the seed tokens (none:
+    fewer than k seeds).  tau is at most the prefix's k-th largest score, so a
+    block with U_b < tau holds only tokens strictly below it: those blocks are
+    skipped, the rest are scored exactly, and the top-k of what was scored
+    (ties to the lower index) is the dense top-k.
+    Returns dict(topk, tau, pruned [blocks, bool], scored = tokens scored).
+    """
+    L_i = max(int(L_i), 0)
+    seed = np.unique(np.asarray(seed, dtype=np.int64))
+    seed = seed[(seed >= 0) & (seed < L_i)]
+    tau = -math.inf
+    if seed.size >= k and k > 0:
+        tau = float(np.sort(index_scores(q, w, K[seed], range(q.shape[0])))[::-1][k - 1])
+    U = dosa_block_bounds(q, w, K, L_i, B)
+    pruned = U < tau
+    keep = np.concatenate([np.arange(b * B, min(L_i, (b + 1) * B)) for b in np.flatnonzero(~pruned)]
+                          + [np.zeros(0, dtype=np.int64)]).astype(np.int64)
+    I = index_scores(q, w, K[keep], range(q.shape[0]))
+    top = top_k(I, k, index=keep)
+    return dict(topk=top, tau=tau, pruned=pruned, scored=int(keep.size))
 
 
 # --------------------------------------------------------------------------

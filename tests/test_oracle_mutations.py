@@ -9,6 +9,7 @@ import types
 import pytest
 
 from oracle import misa_oracle
+import tests.test_oracle_dosa as dosa_pins
 import tests.test_oracle_pins as pins
 
 MUTATIONS = {
@@ -32,7 +33,21 @@ MUTATIONS = {
                             "I = index_scores(q, w, K[:L_i], range(q.shape[0] - 1), counter)"),
 }
 
+# the certified pruning of the dense indexer, against its own pins
+DOSA_MUTATIONS = {
+    "dosa_residual_sign": ("U += w[j] * max(a + qn[j] * rho, 0.0)", "U += w[j] * max(a - qn[j] * rho, 0.0)"),
+    "dosa_negative_heads_upper": ("U += w[j] * max(a - qn[j] * rho, 0.0)",
+                                  "U += w[j] * max(a + qn[j] * rho, 0.0)"),
+    "dosa_negative_heads_dropped": ("U += w[j] * max(a - qn[j] * rho, 0.0)", "U += 0.0"),
+    "dosa_prunes_at_equality": ("pruned = U < tau", "pruned = U <= tau"),
+    "dosa_threshold_from_top_seed": ("[::-1][k - 1])", "[::-1][0])"),
+    "dosa_radius_from_first_token": ("rho = float(np.sqrt(np.sum((Kb - c) ** 2, axis=1)).max())",
+                                     "rho = float(np.sqrt(np.sum((Kb[0] - c) ** 2)))"),
+}
+
 PIN_TESTS = [(n, f) for n, f in inspect.getmembers(pins, inspect.isfunction) if n.startswith("test_")]
+DOSA_PIN_TESTS = [(n, f) for n, f in inspect.getmembers(dosa_pins, inspect.isfunction)
+                  if n.startswith("test_") and n != "test_certificate_on_the_workloads"]
 
 
 def _mutant(src_from, src_to):
@@ -53,6 +68,26 @@ def _params(fn):
                 yield dict(zip(names, vals))
             return
     yield {}
+
+
+def _caught(tests):
+    caught = []
+    for tname, fn in tests:
+        for kw in _params(fn):
+            try:
+                fn(**kw)
+            except Exception:
+                caught.append(tname)
+                break
+        if caught:
+            break
+    return caught
+
+
+@pytest.mark.parametrize("name", sorted(DOSA_MUTATIONS))
+def test_dosa_pins_catch_mutation(name, monkeypatch):
+    monkeypatch.setattr(dosa_pins, "O", _mutant(*DOSA_MUTATIONS[name]))
+    assert _caught(DOSA_PIN_TESTS), f"no pin caught mutation {name}"
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
