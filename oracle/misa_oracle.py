@@ -317,7 +317,10 @@ def dot_product_count(kind: str, L_i: int, B: int, H: int, h: int, k_prime: int 
 #   (Cauchy-Schwarz), ReLU is non-decreasing, so
 #   I_t <= U_b = sum_{w_j >= 0} w_j ReLU(a_j + ||q_j|| rho_b)
 #              + sum_{w_j < 0}  w_j ReLU(a_j - ||q_j|| rho_b).
-# A block with U_b below the seed threshold holds no top-k token.
+# A block with U_b below the seed threshold holds no top-k token.  Parity
+# unpinned as to the form of this bound: its validity and the exactness of
+# the pruned top-k are pinned, but the page prints nothing that fixes which
+# bound DoSA uses.
 
 def dosa_block_bounds(q: np.ndarray, w: np.ndarray, K: np.ndarray, L_i: int, B: int) -> np.ndarray:
     """U_b >= max over the block's tokens of the dense score, for every block of the prefix."""
