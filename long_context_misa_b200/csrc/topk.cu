@@ -197,13 +197,44 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *total,
   return r;
 }
 
+// warp_select_bin with every thread of a block of T = RB / 2 threads: thread
+// t holds the pair of bins 2p, 2p + 1 with p = T - 1 - t (the highest bins
+// go to the first threads), so an exclusive scan in thread order counts the
+// elements above each pair, and the thread whose pair holds the want-th
+// element publishes the result through *res.  A shared histogram in the hpos
+// layout (PAD) or plain.  Called by every thread; returns the same result
+// everywhere.
+template <int T, bool PAD>
+__device__ __forceinline__ uint4 block_select_bin(const uint32_t *h, uint32_t want, uint32_t *wa, uint32_t *wb,
+                                                  uint4 *res) {
+  static_assert(2 * T == RB, "two bins per thread");
+  const int b0 = 2 * (T - 1 - (int)threadIdx.x);
+  uint32_t c0, c1;
+  if (PAD) {
+    c0 = h[hpos(b0)];
+    c1 = h[hpos(b0 + 1)];
+  } else {
+    const uint2 v = *reinterpret_cast<const uint2 *>(h + b0);
+    c0 = v.x;
+    c1 = v.y;
+  }
+  uint32_t total;
+  const uint32_t above = block_excl_scan<T>(c0 + c1, &total, wa, wb);  // elements in the higher pairs
+  if (want == 0 || want > total) return make_uint4(~0u, 0u, 0u, total);  // uniform
+  if (above < want && above + c1 >= want) *res = make_uint4(b0 + 1, above, c1, total);
+  if (above + c1 < want && above + c1 + c0 >= want) *res = make_uint4(b0, above + c1, c0, total);
+  __syncthreads();
+  const uint4 r = *res;
+  __syncthreads();  // *res free again on return
+  return r;
+}
+
 struct SelShared {
   Boundary bd;
   uint4 res;                       // a warp search result
   uint32_t thr[2];                 // threshold composite from the counting step
   uint32_t n_small;
   uint32_t wa[SEL_W], wb[SEL_W + 1];
-  uint32_t toff[SEL_T];            // output offset of each thread's bitmap words
   uint32_t hist[HPAD];
   uint32_t small_key[SEL_T], small_tie[SEL_T];
   uint32_t cand_key[CAP];
@@ -380,12 +411,17 @@ __device__ __forceinline__ void refine(Sh &sh, uint32_t &P_hi, uint32_t &M_hi, u
         atomicAdd(&sh.hist[hpos(((lo_word ? lx : kx) >> sft) & dm)], 1u);
     });
     __syncthreads();
-    if (tid < 32) {
-      const uint4 r = warp_select_bin<true>(sh.hist, need);
-      if (tid == 0) sh.res = r;
+    uint4 r;
+    if constexpr (2 * T == RB) {
+      r = block_select_bin<T, true>(sh.hist, need, sh.wa, sh.wb, &sh.res);
+    } else {
+      if (tid < 32) {
+        const uint4 x = warp_select_bin<true>(sh.hist, need);
+        if (tid == 0) sh.res = x;
+      }
+      __syncthreads();
+      r = sh.res;
     }
-    __syncthreads();
-    const uint4 r = sh.res;
     need -= r.y;
     in_bin = r.z;
     if (!lo_word) {
@@ -400,63 +436,29 @@ __device__ __forceinline__ void refine(Sh &sh, uint32_t &P_hi, uint32_t &M_hi, u
 }
 
 // Ascending output of the marked tokens: thread t owns bitmap words
-// [t*per, t*per + per); the outputs are split evenly over the threads (each
-// finds the word holding its first output by a search over the owners'
-// offsets), then -1 padding up to k.
-// Staged output j lives at word j + j / 32: threads writing runs of outputs
-// 16 apart then hit distinct banks.
-__device__ __forceinline__ uint32_t spad(uint32_t j) { return j + (j >> 5); }
-
+// [t*per, t*per + per), counts their bits, takes the slot of its first
+// output from a block-wide exclusive scan and writes its own tokens in order
+// (the threads of a warp write neighbouring output ranges); then -1 padding
+// up to k.  A thread whose words hold many winners writes them all (at most
+// 32 per word), which costs less than spreading the outputs evenly over the
+// threads by searching the owners' offsets.
 template <int T = SEL_T>
-__device__ __forceinline__ void write_ascending(const uint32_t *bm, int words, int k, int32_t *orow, uint32_t *toff,
-                                                uint32_t *wa, uint32_t *wb, int32_t *stage, int stage_cap) {
+__device__ __forceinline__ void write_ascending(const uint32_t *bm, int words, int k, int32_t *orow, uint32_t *wa,
+                                                uint32_t *wb) {
   const int tid = threadIdx.x;
   const int per = cdiv(words, T);
   const int w0 = min(tid * per, words), w1 = min(w0 + per, words);
   uint32_t cnt = 0;
   for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
   uint32_t n_sel;
-  toff[tid] = block_excl_scan<T>(cnt, &n_sel, wa, wb);
-  __syncthreads();
+  uint32_t j = block_excl_scan<T>(cnt, &n_sel, wa, wb);
   const uint32_t n_out = min(n_sel, (uint32_t)k);
-  const uint32_t cap = (uint32_t)stage_cap * 32 / 33;  // entries per chunk, padding included
-  for (uint32_t base = 0; base < n_out; base += cap) {
-    // outputs [base, base + chunk) are spread evenly over the threads, staged
-    // in shared memory, then written with coalesced stores
-    const uint32_t chunk = min(cap, n_out - base);
-    const uint32_t j0 = base + chunk * (uint32_t)tid / T, j1 = base + chunk * (uint32_t)(tid + 1) / T;
-    // each output is found inside the words of its owner thread (found by a
-    // binary search over the owners' offsets), so a run of empty words
-    // between clusters of selected tokens is jumped, never walked
-    uint32_t j = j0;
-    while (j < j1) {
-      int lo = 0, hi = T - 1;  // last owner whose offset is <= j
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (toff[mid] <= j) lo = mid;
-        else hi = mid - 1;
-      }
-      uint32_t r = j - toff[lo];
-      const int wend = min(lo * per + per, words);
-      for (int w = lo * per; w < wend && j < j1; ++w) {
-        uint32_t m = bm[w];
-        const uint32_t pc = __popc(m);
-        if (pc <= r) {
-          r -= pc;
-          continue;
-        }
-        for (; r > 0; --r) m &= m - 1;
-        while (m && j < j1) {
-          const int b = __ffs(m) - 1;
-          m &= m - 1;
-          stage[spad(j - base)] = w * 32 + b;
-          ++j;
-        }
-      }
+  for (int w = w0; w < w1 && j < n_out; ++w) {
+    uint32_t m = bm[w];
+    while (m && j < n_out) {
+      orow[j++] = w * 32 + (__ffs(m) - 1);
+      m &= m - 1;
     }
-    __syncthreads();
-    for (uint32_t j = tid; j < chunk; j += T) orow[base + j] = stage[spad(j)];
-    __syncthreads();
   }
   for (int p = (int)n_out + tid; p < k; p += T) orow[p] = -1;
 }
@@ -621,7 +623,7 @@ __global__ void __launch_bounds__(SEL_T) select_kernel(CacheView c, QueryView qv
   }
 
   // 4. ascending output, staged in the candidate list's space
-  write_ascending(bm, words, k, orow, sh.toff, sh.wa, sh.wb, reinterpret_cast<int32_t *>(sh.cand_key), 2 * CAP);
+  write_ascending(bm, words, k, orow, sh.wa, sh.wb);
 }
 
 // Few long prefix rows: every CTA takes a chunk of one row and appends the
@@ -857,7 +859,6 @@ struct FastShared {
   uint32_t n_small;
   int ok;
   uint32_t wa[FAST_W], wb[FAST_W + 1];
-  uint32_t toff[FAST_T];
   uint32_t hist[HPAD];
   uint32_t small_key[FAST_T], small_tie[FAST_T];
   uint32_t n_d0;
@@ -1080,9 +1081,17 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
       atomicAdd(&sh.rhist[(list_ok ? ent[i].x : ordered_key(__ldg(srow + i))) >> HIST_SHIFT], 1u);
     __syncthreads();
   }
-  if (warp == 0) {
-    const Boundary b = warp_boundary_plain_smem(sh.rhist, k);
-    if ((tid & 31) == 0) {
+  {
+    // the boundary bin of the row, searched by the whole block
+    const uint4 r = block_select_bin<FAST_T, false>(sh.rhist, (uint32_t)k, sh.wa, sh.wb, &sh.res);
+    Boundary b;
+    b.total = r.w;
+    b.kk = min((uint32_t)k, r.w);
+    b.all_in = (uint32_t)k >= r.w;
+    b.d0 = b.all_in ? 0u : r.x;
+    b.above = b.all_in ? 0u : r.y;
+    b.in0 = b.all_in ? 0u : r.z;
+    if (tid == 0) {
       sh.bd = b;
       if (EMITTED && b.listable()) sh.n_out = b.above;  // the filter's tokens come first
     }
@@ -1205,8 +1214,7 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
   }
   // 4. output
   if (ORDERED) {
-    write_ascending<FAST_T>(bm, words, k, orow, sh.toff, sh.wa, sh.wb, reinterpret_cast<int32_t *>(data),
-                            data_bytes / 4);
+    write_ascending<FAST_T>(bm, words, k, orow, sh.wa, sh.wb);
   } else {
     __syncthreads();
     for (int p = (int)min(sh.n_out, (uint32_t)k) + tid; p < k; p += FAST_T) orow[p] = -1;
