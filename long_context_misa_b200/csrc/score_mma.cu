@@ -8,7 +8,7 @@
 //   - gathered candidates (re-rank): rerank_umma_kernel, tcgen05 tensor cores
 //     (every head count the library accepts, MISA_MAX_H = 128);
 //   - prefix rows of e4m3 caches with 32 or more scoring heads (dense
-//     decode): the same kernel over contiguous tokens;
+//     decode): dense_umma_kernel (rerank_umma.cu), persistent over the prefix;
 //   - other prefix rows (routed decode, bf16 dense decode): the streaming
 //     kernel on mma.sync, which builds the row histograms on the way.
 // Prefill chunks (many queries per sequence) are scored by score_umma.cu,
@@ -24,9 +24,10 @@ cudaError_t launch_score_mma(const CacheView &c, const QueryView &q, const int32
   if (!rerank_umma_applies(q, heads, h)) return cudaErrorInvalidValue;  // more heads than the library accepts
   if (gather) return launch_rerank_umma(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s);
   // e4m3 keys with 32 or more scoring heads (dense decode): the dense product
-  // on tcgen05 (74.8 against 139.3 us for 8 x 128K keys and 64 heads); fewer
-  // heads (routed decode), and bf16 keys (whose 32 KB tiles leave one CTA per
-  // SM there: 125 against 77 us for 32 x 32K and 64 heads), stream the keys
+  // on tcgen05 (45 against 139.3 us on mma.sync for 8 x 128K keys and 64
+  // heads); fewer heads (routed decode), and bf16 keys (whose 32 KB tiles
+  // leave one CTA per SM there: 125 against 77 us for 32 x 32K and 64 heads,
+  // measured with the earlier non-persistent tcgen05 form), stream the keys
   // on mma.sync
   const int he = heads ? h : q.H;
   if (c.fp8 && he >= 32) return launch_rerank_umma(c, q, heads, h, nullptr, c.L_cap, scores, ld, row_hist, s);
