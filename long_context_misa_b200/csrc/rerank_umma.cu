@@ -275,8 +275,8 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
 // walks chunks part, part + nparts, ... of its query's prefix (DT tiles of
 // 128 tokens each), with chunks j + 1 .. j + NBUF - 1's key rows and scales
 // in flight (coalesced 16-byte cp.async into a ring of NBUF shared-memory
-// buffers) while chunk j is multiplied and drained; the grid is the resident
-// CTAs the runtime reports (two per SM at 64 heads).  Measured for 8 x 128K
+// buffers) while chunk j is multiplied and drained; the grid holds the
+// resident CTAs (two per SM for e4m3 keys).  Measured for 8 x 128K
 // e4m3 keys and 64 heads: 45 us with two-tile chunks and two buffers, 63 us
 // with one-tile chunks and three buffers (three CTAs per SM: the per-chunk
 // barriers and MMA round trip weigh more).  One mbarrier
@@ -470,19 +470,20 @@ cudaError_t launch_dense(const CacheView &c, const QueryView &q, const int32_t *
   using Cfg = DCfg<FP8, HN>;
   struct Tag {};
   const int st = cached_per_device<Tag>([] {
-    return 1 + (int)cudaFuncSetAttribute(dense_umma_kernel<FP8, HN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(dense_umma_kernel<FP8, HN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg::SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(dense_umma_kernel<FP8, HN>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               (int)cudaSharedmemCarveoutMaxShared);
+    return 1 + (int)e;
   });
   if (st != 1) return (cudaError_t)(st - 1);
-  // the resident CTAs over all rows, each walking several chunks
-  struct OccTag {};
-  const int per_sm = cached_per_device<OccTag>([] {
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dense_umma_kernel<FP8, HN>, RR_THREADS, Cfg::SMEM) !=
-        cudaSuccess)
-      return 1;
-    return std::max(n, 1);
-  });
+  // the resident CTAs over all rows, each walking several chunks: two per SM
+  // when two fit in the SM's 228 KB of shared memory (e4m3 keys: at most
+  // 94 KB each at every head count), else one.  (The runtime's occupancy
+  // query answered one per SM for e4m3 at 64 heads, and a grid sized from it
+  // took 54 us instead of 45.)
+  constexpr int per_sm = 2 * (Cfg::SMEM + (int)sizeof(DenseShared) + 1024) <= 228 * 1024 ? 2 : 1;
   const int nparts = std::max(1, std::min(cdiv(c.L_cap, Cfg::CT), per_sm * device_sms() / q.n_q));
   return launch_kernel(dense_umma_kernel<FP8, HN>, dim3(nparts, q.n_q), dim3(RR_THREADS), Cfg::SMEM, s, c, q, heads,
                        h, scores, ld, row_hist, nparts);
