@@ -25,6 +25,9 @@ CASES = {
     "fp8_prefill_h32": W["long_prefill_128k"].scaled(L=2100, n_q=40, B=100, k=33),
     # few long rows: the top-k goes through the compact boundary-bin list
     "fp8_long": W["misa_dagger_decode_128k"].scaled(n_seq=2, L=40000, B=128, k=600, k_prime=4000),
+    # 96 heads: dense decode on 128 tensor-core columns, 32 of them zero-weight
+    # padding, one-tile chunks
+    "fp8_h96": W["misa_dagger_decode_128k"].scaled(n_seq=2, L=2999, H=96, k=64, k_prime=300),
     # prefill chunks of >= 64 queries score on the tcgen05 tensor-core path
     "fp8_prefill_umma": W["long_prefill_128k"].scaled(L=3000, n_q=96, B=100, k=33),
     # query groups that span two sequences (two passes over different keys)
