@@ -139,8 +139,6 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
   volatile int *abort = &sh.abort;
   const int i = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int H = qv.H;
-  const int h_eff = heads ? h : H;
   int s;
   const int Li = query_prefix(c, qv, i, &s);
   const int col0 = blockIdx.x * T * RR_M;

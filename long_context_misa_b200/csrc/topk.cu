@@ -1015,7 +1015,7 @@ __global__ void __launch_bounds__(FAST_T) select_smem_kernel(CacheView c, QueryV
   const float *sc = reinterpret_cast<const float *>(data);                 // GATHER
   const int32_t *tk = reinterpret_cast<const int32_t *>(data + n_cols * 4);  // GATHER
   const int row = blockIdx.x;
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x;
 
   int s;
   const int Li = query_prefix(c, qv, row, &s);
