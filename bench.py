@@ -59,11 +59,13 @@ def score_kernel_bytes(wl):
     return wl.n_seq * wl.L * row + wl.n_q * wl.h * (wl.d * 2 + 4)
 
 
-# DRAM bytes (read + write) of one routed scoring launch on the MISA-dagger
-# decode workload at L = 128K, from the ncu capture summarised in
-# profiles/score_stream_kernel_misa_dagger_decode_128k.md.  Valid only for
-# that workload and that kernel version; reported as null elsewhere.
-STREAM_TRAFFIC_BYTES = {"misa_dagger_decode_128k": 143_242_496}
+# DRAM bytes (read + write) of one routed scoring launch per workload, from
+# an ncu capture of the current kernel version; reported as null where there
+# is none.  The capture summarised in
+# profiles/score_stream_kernel_misa_dagger_decode_128k.md (143,242,496 bytes
+# on the MISA-dagger decode workload) predates the grid-dependency wait every
+# kernel now starts with, so until it is retaken the figure is null.
+STREAM_TRAFFIC_BYTES = {}
 
 
 class Clocks:
