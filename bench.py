@@ -61,10 +61,10 @@ def score_kernel_bytes(wl):
 
 # DRAM bytes (read + write) of one routed scoring launch per workload, from
 # an ncu capture of the current kernel version; reported as null where there
-# is none.  The capture summarised in
-# profiles/score_stream_kernel_misa_dagger_decode_128k.md (143,242,496 bytes
-# on the MISA-dagger decode workload) predates the grid-dependency wait every
-# kernel now starts with, so until it is retaken the figure is null.
+# is none.  The last capture of the routed scorer on the MISA-dagger decode
+# workload (143,242,496 bytes, summarised with the other ncu figures under
+# profiles/) predates the grid-dependency wait every kernel now starts with,
+# so until it is retaken the figure is null.
 STREAM_TRAFFIC_BYTES = {}
 
 
