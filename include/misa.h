@@ -27,6 +27,14 @@
  *    default stream).  Outputs are valid in stream order.  Nothing blocks the
  *    host; the library keeps no state between calls other than cached device
  *    attributes and the thread-local error text.
+ *  - The library's kernels are launched with programmatic stream
+ *    serialisation.  Each waits for the work before it in the stream to
+ *    complete before touching memory, and none releases its dependents early.
+ *    A caller's kernel launched without that attribute is ordered as usual.
+ *    A caller's kernel that opts into programmatic dependent launch itself,
+ *    right after a call, must wait on its grid dependency (griddepcontrol.wait
+ *    / cudaGridDependencySynchronize) before it reads the call's outputs, as
+ *    after any kernel.
  *  - Arguments are validated on the host before any launch.  A bad argument
  *    returns MISA_ERR_INVALID (MISA_ERR_UNSUPPORTED for shapes outside the
  *    supported range, MISA_ERR_WORKSPACE for a short workspace) and launches
