@@ -6,9 +6,21 @@
 #include <cstdio>
 #include <cstring>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "internal.h"
 
 namespace {
+
+// One NVTX range per library call that launches work, named after the entry
+// point, so that a profiler's timeline shows each call around its kernels.
+// Without a profiler attached the calls are no-ops.
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 thread_local char g_err[512] = "";
 std::atomic<int> g_fail_next{0};
@@ -218,6 +230,7 @@ extern "C" {
 
 misa_status misa_pool_keys(const misa_cache *cache, const void *new_keys, const float *new_scale,
                            const int32_t *new_pos, int32_t count, misa_stream stream) {
+  NvtxRange nvtx("misa_pool_keys");
   misa_status st = check_cache(cache, true);
   if (st != MISA_OK) return st;
   if (count < 0) return fail(MISA_ERR_INVALID, "count=%d < 0", count);
@@ -238,6 +251,7 @@ misa_status misa_pool_keys(const misa_cache *cache, const void *new_keys, const 
 
 misa_status misa_append_keys_e4m3(const misa_cache *cache, const uint16_t *new_keys, const int32_t *new_pos,
                                   int32_t count, misa_stream stream) {
+  NvtxRange nvtx("misa_append_keys_e4m3");
   misa_status st = check_cache(cache, true);
   if (st != MISA_OK) return st;
   if (cache->dtype != MISA_KEY_FP8_E4M3) return fail(MISA_ERR_INVALID, "the cache does not hold e4m3 keys");
@@ -277,6 +291,7 @@ size_t misa_workspace_bytes(int32_t op, const misa_cache *cache, const misa_quer
 misa_status misa_route_heads_agg(const misa_cache *cache, const misa_queries *qs, int32_t h, int32_t agg,
                                  int32_t *heads, float *router_scores, void *ws, size_t ws_bytes,
                                  misa_stream stream) {
+  NvtxRange nvtx("misa_route_heads_agg");
   misa_status st = check_cache(cache, true);
   if (st != MISA_OK) return st;
   if ((st = check_queries(qs)) != MISA_OK) return st;
@@ -298,6 +313,7 @@ misa_status misa_route_heads(const misa_cache *cache, const misa_queries *qs, in
 misa_status misa_score_topk(const misa_cache *cache, const misa_queries *qs, const int32_t *heads, int32_t h,
                             int32_t k, int32_t *topk, float *scores_out, void *ws, size_t ws_bytes,
                             misa_stream stream) {
+  NvtxRange nvtx("misa_score_topk");
   misa_status st = check_cache(cache, false);
   if (st != MISA_OK) return st;
   if ((st = check_queries(qs)) != MISA_OK) return st;
@@ -313,6 +329,7 @@ misa_status misa_score_topk(const misa_cache *cache, const misa_queries *qs, con
 
 misa_status dsa_dense_score_topk(const misa_cache *cache, const misa_queries *qs, int32_t k, int32_t *topk,
                                  float *scores_out, void *ws, size_t ws_bytes, misa_stream stream) {
+  NvtxRange nvtx("dsa_dense_score_topk");
   misa_status st = check_cache(cache, false);
   if (st != MISA_OK) return st;
   if ((st = check_queries(qs)) != MISA_OK) return st;
@@ -328,6 +345,7 @@ misa_status dsa_dense_score_topk(const misa_cache *cache, const misa_queries *qs
 misa_status misa_rerank_topk(const misa_cache *cache, const misa_queries *qs, const int32_t *cand,
                              int32_t k_prime, int32_t k, int32_t *topk, float *scores_out, void *ws,
                              size_t ws_bytes, misa_stream stream) {
+  NvtxRange nvtx("misa_rerank_topk");
   misa_status st = check_cache(cache, false);
   if (st != MISA_OK) return st;
   if ((st = check_queries(qs)) != MISA_OK) return st;
@@ -356,6 +374,7 @@ misa_status misa_rerank_topk(const misa_cache *cache, const misa_queries *qs, co
 misa_status misa_rerank_topk_noalloc(const misa_cache *cache, const misa_queries *qs, const int32_t *cand,
                                      int32_t k_prime, int32_t k, int32_t *topk, float *scores_out,
                                      misa_stream stream) {
+  NvtxRange nvtx("misa_rerank_topk_noalloc");
   const char *who = "misa_rerank_topk_noalloc";
   misa_status st = check_cache(cache, false);
   if (st != MISA_OK) return st;
@@ -391,6 +410,7 @@ misa_status misa_rerank_topk_noalloc(const misa_cache *cache, const misa_queries
 misa_status misa_dagger_topk(const misa_cache *cache, const misa_queries *qs, const int32_t *heads, int32_t h,
                              int32_t k_prime, int32_t k, int32_t *topk, void *ws, size_t ws_bytes,
                              misa_stream stream) {
+  NvtxRange nvtx("misa_dagger_topk");
   const char *who = "misa_dagger_topk";
   misa_status st = check_cache(cache, false);
   if (st != MISA_OK) return st;
@@ -436,6 +456,7 @@ misa_status misa_dagger_topk(const misa_cache *cache, const misa_queries *qs, co
 }
 
 misa_status misa_debug_wait_timeout(uint32_t *status, uint64_t limit_ns, misa_stream stream) {
+  NvtxRange nvtx("misa_debug_wait_timeout");
   if (!status) return fail(MISA_ERR_INVALID, "status is NULL");
   if (limit_ns > 10000000000ull) return fail(MISA_ERR_INVALID, "limit_ns=%llu above 10 s", (unsigned long long)limit_ns);
   cudaError_t e = misa::launch_kernel(wait_timeout_kernel, dim3(1), dim3(32), 0, stream, status,
