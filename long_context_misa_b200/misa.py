@@ -153,8 +153,12 @@ class KeyCache:
 
     def __init__(self, keys: torch.Tensor, scale: Optional[torch.Tensor], seq_len: torch.Tensor, B: int,
                  pool: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None):
-        assert keys.dim() == 3 and keys.shape[2] == D and keys.is_contiguous()
-        assert keys.dtype in (torch.uint16, torch.int16, torch.uint8)
+        if keys.dim() != 3 or keys.shape[2] != D or not keys.is_contiguous():
+            raise ValueError(f"keys must be a contiguous [n_seq][L_cap][{D}] tensor, got {tuple(keys.shape)}")
+        if keys.dtype not in (torch.uint16, torch.int16, torch.uint8):
+            raise TypeError(f"keys must hold bf16 bits (uint16/int16) or e4m3 codes (uint8), got {keys.dtype}")
+        if int(B) < 1:
+            raise ValueError(f"block size B must be >= 1, got {B}")
         self.keys, self.scale, self.seq_len, self.B = keys, scale, seq_len, int(B)
         self.n_seq, self.L_cap = int(keys.shape[0]), int(keys.shape[1])
         self.dtype = MISA_KEY_FP8_E4M3 if keys.dtype == torch.uint8 else MISA_KEY_BF16
@@ -179,7 +183,12 @@ class Queries:
     """Index queries: q bf16 bits [n_q][H][128], w fp32 [n_q][H], q_seq/q_pos int32 [n_q]."""
 
     def __init__(self, q: torch.Tensor, w: torch.Tensor, q_seq: torch.Tensor, q_pos: torch.Tensor):
-        assert q.dim() == 3 and q.shape[2] == D and q.is_contiguous() and w.is_contiguous()
+        if q.dim() != 3 or q.shape[2] != D or not q.is_contiguous():
+            raise ValueError(f"q must be a contiguous [n_q][H][{D}] tensor, got {tuple(q.shape)}")
+        if tuple(w.shape) != tuple(q.shape[:2]) or not w.is_contiguous():
+            raise ValueError(f"w must be a contiguous [n_q][H] tensor matching q, got {tuple(w.shape)}")
+        if q_seq.numel() != q.shape[0] or q_pos.numel() != q.shape[0]:
+            raise ValueError("q_seq and q_pos must hold one entry per query")
         self.q, self.w, self.q_seq, self.q_pos = q, w, q_seq, q_pos
         self.n_q, self.H = int(q.shape[0]), int(q.shape[1])
         self._s = misa_queries(_ptr(q), _ptr(w), _ptr(q_seq), _ptr(q_pos), self.n_q, self.H)

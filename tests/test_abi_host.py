@@ -5,6 +5,7 @@ CUDA call, and injected failures fire before any launch)."""
 import ctypes
 
 import pytest
+import torch
 
 from long_context_misa_b200 import misa as M
 
@@ -164,3 +165,29 @@ def test_route_agg_argument_checks():
     for agg in (-1, 4):
         assert L.misa_route_heads_agg(by(cache()), by(queries()), 8, agg, FAKE, None, FAKE, 1 << 30, None) == \
             M.MISA_ERR_INVALID
+
+
+def test_binding_rejects_malformed_tensors():
+    """The Python classes check shapes and dtypes themselves (not asserts,
+    which python -O would strip) before anything reaches the library."""
+    keys = torch.zeros(2, 64, 128, dtype=torch.uint8)
+    seq_len = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        M.KeyCache(torch.zeros(2, 64, 64, dtype=torch.uint8), None, seq_len, 16)
+    with pytest.raises(ValueError):
+        M.KeyCache(keys.transpose(0, 1), None, seq_len, 16)
+    with pytest.raises(TypeError):
+        M.KeyCache(torch.zeros(2, 64, 128, dtype=torch.float32), None, seq_len, 16)
+    with pytest.raises(ValueError):
+        M.KeyCache(keys, torch.zeros(2, 64), seq_len, 0)
+    q = torch.zeros(3, 4, 128, dtype=torch.int16)
+    w = torch.zeros(3, 4)
+    idx = torch.zeros(3, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        M.Queries(torch.zeros(3, 4, 100, dtype=torch.int16), w, idx, idx)
+    with pytest.raises(ValueError):
+        M.Queries(q, torch.zeros(3, 5), idx, idx)
+    with pytest.raises(ValueError):
+        M.Queries(q, w, torch.zeros(2, dtype=torch.int32), idx)
+    qs = M.Queries(q, w, idx, idx)
+    assert (qs.n_q, qs.H) == (3, 4)
