@@ -1,0 +1,58 @@
+"""The prefill selection's sampled bound on the workloads' own scores (CPU).
+
+The tensor-core prefill path lists, per row, the scores at or above a key
+bound drawn from a sample of the row: 256 blocks of 32 consecutive tokens
+spread evenly over the prefix; want = r + z * sqrt(32 r) + 8 sampled
+elements with r = k * 8192 / L_i (the sample's expected share of the top k);
+the bound is the want-th largest sampled key cut to its top 22 bits.  This
+restates that rule on the oracle's routed scores of rows spread over
+causal_prefill and long_prefill_128k and checks, for the margin in use
+(z = 3), that every row's list holds at least k and at most the 7168
+entries the selection stages.  The list sizes for z = 1.5 are printed too.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from long_context_misa_b200 import inputs as G
+from oracle import misa_oracle as O
+
+BL, BLOCKS = 32, 256
+N = BL * BLOCKS
+STAGE = 7168
+
+
+def _keys(I):
+    u = np.asarray(I, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    return np.where(u & 0x80000000, (~u) & 0xFFFFFFFF, u | 0x80000000)
+
+
+def _list_size(keys, Li, k, z):
+    i = np.arange(N)
+    pos = (i // BL) * (Li - BL) // (BLOCKS - 1) + (i % BL)
+    srt = np.sort(keys[pos])[::-1]
+    r = k * N / Li
+    want = int(min(2 * N, math.ceil(r + z * math.sqrt(BL * r) + 8)))
+    bound = int(srt[want - 1]) & ~((1 << 10) - 1)
+    return int((keys >= bound).sum())
+
+
+@pytest.mark.parametrize("name", ["causal_prefill", "long_prefill_128k"])
+def test_sampled_bound_lists_fit(name):
+    wl = G.WORKLOADS[name]
+    inp = G.make_inputs(wl, 0)
+    K = O.seq_keys(inp.keys, inp.scale, wl.key_dtype, 0)
+    sizes = {3.0: [], 1.5: []}
+    for i in np.linspace(0, wl.n_q - 1, 16).astype(int):
+        q, w = O.query_arrays(inp.q, inp.w, int(i))
+        Li = int(inp.q_pos[i]) + 1
+        heads = O.route_query(q, w, K, Li, wl.B, wl.h)[1]
+        keys = _keys(O.index_scores(q, w, K[:Li], heads))
+        for z in sizes:
+            sizes[z].append(_list_size(keys, Li, wl.k, z))
+    cur = np.array(sizes[3.0])
+    assert cur.min() >= wl.k and cur.max() <= STAGE, cur
+    for z, v in sizes.items():
+        v = np.array(v)
+        print(f"\n{name} z={z}: list min / median / max {v.min()} / {int(np.median(v))} / {v.max()}")
