@@ -1,4 +1,4 @@
-"""The prefill selection's sampled bound on the workloads' own scores (CPU).
+"""The selections' sampled bound and boundary bins on the workloads' own scores (CPU).
 
 The tensor-core prefill path lists, per row, the scores at or above a key
 bound drawn from a sample of the row: 256 blocks of 32 consecutive tokens
@@ -56,3 +56,24 @@ def test_sampled_bound_lists_fit(name):
     for z, v in sizes.items():
         v = np.array(v)
         print(f"\n{name} z={z}: list min / median / max {v.min()} / {int(np.median(v))} / {v.max()}")
+
+
+def test_decode_boundary_bin_fits_the_compaction():
+    """misa_dagger_decode_128k's top-k' selection compacts the elements of
+    the boundary bin (the top 11 key bits of the k'-th score) into shared
+    memory, up to 6144 of them; more sends the row down the slower sweeping
+    path.  On every row of the workload's oracle scores the bin fits.  The
+    populations at finer first bins are printed beside it."""
+    wl = G.WORKLOADS["misa_dagger_decode_128k"]
+    inp = G.make_inputs(wl, 0)
+    for i in range(wl.n_q):
+        s = int(inp.q_seq[i])
+        K = O.seq_keys(inp.keys, inp.scale, wl.key_dtype, s)
+        Li = int(inp.q_pos[i]) + 1
+        q, w = O.query_arrays(inp.q, inp.w, i)
+        heads = O.route_query(q, w, K, Li, wl.B, wl.h)[1]
+        keys = _keys(O.index_scores(q, w, K[:Li], heads))
+        vk = np.sort(keys)[::-1][wl.k_prime - 1]
+        pops = [int(((keys >> (32 - b)) == (vk >> (32 - b))).sum()) for b in (11, 12, 13, 14)]
+        assert pops[0] <= 6144, pops
+        print(f"\nq{i}: boundary-bin population at 11 / 12 / 13 / 14 bits: {pops}")
