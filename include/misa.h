@@ -294,8 +294,9 @@ MISA_API misa_status misa_dagger_topk(const misa_cache *cache, const misa_querie
  * image, one per device.  The call allocates and frees nothing; it zeroes the
  * histogram part of the array on `stream` before use.
  *
- * Scratch needed: 8196 bytes per query for the histograms, plus 4 * k_prime
- * bytes per query when scores_out is NULL, each part rounded up to 256 bytes
+ * Scratch needed: 8200 bytes per query for the histograms (2048 bins and two
+ * counters), plus 4 * k_prime bytes per query when scores_out is NULL, each
+ * part rounded up to 256 bytes
  * (8 queries with k_prime = 8192: about 320 KiB).  A larger need returns
  * MISA_ERR_WORKSPACE and launches nothing; use misa_rerank_topk then.
  *
