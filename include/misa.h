@@ -340,10 +340,13 @@ MISA_API void misa_debug_fail_next(int32_t n);
 
 /*
  * Profiling aid: while both are non-NULL, every misa_score_topk,
- * dsa_dense_score_topk and misa_rerank_topk call records the caller's
- * cudaEvent_t `start` just before and `stop` just after its token-scoring
- * kernel, on the call's stream, so the kernel's own duration can be read with
- * cudaEventElapsedTime.  misa_debug_time_scoring(NULL, NULL) switches it off.
+ * dsa_dense_score_topk, misa_rerank_topk and misa_rerank_topk_noalloc call
+ * records the caller's cudaEvent_t `start` just before and `stop` just after
+ * its token-scoring kernel, and misa_dagger_topk around its routed scoring
+ * kernel (not the re-rank), on the call's stream, so the kernel's own
+ * duration can be read with cudaEventElapsedTime.  Inside a stream capture
+ * the records become event nodes of the graph.
+ * misa_debug_time_scoring(NULL, NULL) switches it off.
  */
 MISA_API void misa_debug_time_scoring(void *start, void *stop);
 
