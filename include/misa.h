@@ -25,8 +25,12 @@
  *    for few long rows, a compact candidate list).
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
  *    default stream).  Outputs are valid in stream order.  Nothing blocks the
- *    host; the library keeps no state between calls other than cached device
- *    attributes and the thread-local error text.
+ *    host.  Between calls the library keeps only cached device attributes,
+ *    the thread-local error text, and two process-wide test hooks that are
+ *    off unless a caller sets them: misa_debug_fail_next (a count of calls
+ *    to fail) and misa_debug_time_scoring (two events recorded around the
+ *    scoring kernels).  misa_rerank_topk_noalloc's fixed scratch array also
+ *    keeps the last call's contents (see there).
  *  - The library's kernels are launched with programmatic stream
  *    serialisation.  Each waits for the work before it in the stream to
  *    complete before touching memory, and none releases its dependents early.
@@ -291,8 +295,10 @@ MISA_API misa_status misa_dagger_topk(const misa_cache *cache, const misa_querie
  * a cudaMalloc would fail or stall the device.  The scratch (the per-row score
  * histograms and, when scores_out is NULL, the candidate scores) lives in a
  * fixed array of MISA_NOALLOC_SCRATCH_BYTES inside the library's device
- * image, one per device.  The call allocates and frees nothing; it zeroes the
- * histogram part of the array on `stream` before use.
+ * image: one per CUDA context that loads the library (normally one per
+ * device, the runtime's primary context), held until that context ends.
+ * The call allocates and frees nothing; it zeroes the histogram part of the
+ * array on `stream` before use.
  *
  * Scratch needed: 8200 bytes per query for the histograms (2048 bins and two
  * counters), plus 4 * k_prime bytes per query when scores_out is NULL, each
@@ -300,14 +306,15 @@ MISA_API misa_status misa_dagger_topk(const misa_cache *cache, const misa_querie
  * (8 queries with k_prime = 8192: about 320 KiB).  A larger need returns
  * MISA_ERR_WORKSPACE and launches nothing; use misa_rerank_topk then.
  *
- * Limits of a shared array: calls that may overlap on one device (different
+ * Limits of a shared array: calls that may overlap in one context (different
  * streams, or host threads without ordering between them) race on it and
  * give wrong results; calls in stream order on one stream are safe.  The
- * first call on each device looks up the array's device address with that
- * device current (it may load the library's device code), so make it once
- * before any stream capture.  A failed lookup returns MISA_ERR_CUDA.
+ * first call in each context looks up the array's device address there (it
+ * may load the library's device code), so make it once before any stream
+ * capture; the address is then cached per context.  A failed lookup returns
+ * MISA_ERR_CUDA.
  */
-#define MISA_NOALLOC_SCRATCH_BYTES (4u << 20) /* 4 MiB per device */
+#define MISA_NOALLOC_SCRATCH_BYTES (4u << 20) /* 4 MiB per context */
 
 MISA_API misa_status misa_rerank_topk_noalloc(const misa_cache *cache, const misa_queries *qs,
                                               const int32_t *cand, int32_t k_prime, int32_t k,

@@ -5,6 +5,9 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
+
+#include <cuda.h>
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -204,21 +207,68 @@ __global__ void wait_timeout_kernel(uint32_t *status, unsigned long long limit_n
 // the caller never supplies memory and the call never allocates any.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[MISA_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_noalloc_scratch on the current device, looked up on the
-// first call per device (with that device current) and cached.
+// Device address of g_noalloc_scratch in the current context.  Every context
+// that loads the library's device code holds its own copy of the array, so
+// the address belongs to a context, not to a device: after cudaDeviceReset,
+// or when a driver-API caller makes another context current on the same
+// device, the earlier address is dead.  Addresses are therefore cached per
+// context, keyed by the driver's context ID (unique for the life of the
+// process, where a context handle can be reused), and looked up with
+// cudaGetSymbolAddress on the first call in each context.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+
+// Current context's ID; false when there is no current context or the
+// driver entry points are unavailable (the caller then looks the address up
+// without caching it).
+bool current_context_id(unsigned long long *id) {
+  static CtxGetCurrentFn get_current = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+                   q == cudaDriverEntryPointSuccess
+               ? reinterpret_cast<CtxGetCurrentFn>(p)
+               : nullptr;
+  }();
+  static CtxGetIdFn get_id = [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+                   q == cudaDriverEntryPointSuccess
+               ? reinterpret_cast<CtxGetIdFn>(p)
+               : nullptr;
+  }();
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 misa_status noalloc_scratch(const char *who, void **out) {
-  static std::atomic<void *> addr[misa::MAX_DEVICES];
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, who);
-  if (dev < 0 || dev >= misa::MAX_DEVICES)
-    return fail(MISA_ERR_UNSUPPORTED, "%s: device %d outside [0, %d)", who, dev, misa::MAX_DEVICES);
-  void *p = addr[dev].load(std::memory_order_acquire);
-  if (!p) {
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk_noalloc: cudaGetSymbolAddress");
-    if (!p) return fail(MISA_ERR_CUDA, "%s: cudaGetSymbolAddress returned NULL", who);
-    addr[dev].store(p, std::memory_order_release);
+  constexpr int SLOTS = 64;
+  static std::mutex mu;
+  static unsigned long long ids[SLOTS];  // 0: empty (driver context IDs start at 1)
+  static void *addrs[SLOTS];
+  static int next_slot = 0;
+  unsigned long long id = 0;
+  const bool keyed = current_context_id(&id) && id != 0;
+  if (keyed) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int j = 0; j < SLOTS; ++j)
+      if (ids[j] == id) {
+        *out = addrs[j];
+        return MISA_OK;
+      }
+  }
+  void *p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk_noalloc: cudaGetSymbolAddress");
+  if (!p) return fail(MISA_ERR_CUDA, "%s: cudaGetSymbolAddress returned NULL", who);
+  // the lookup may have made the primary context current: key it now
+  if (keyed || (current_context_id(&id) && id != 0)) {
+    std::lock_guard<std::mutex> lock(mu);
+    ids[next_slot] = id;
+    addrs[next_slot] = p;
+    next_slot = (next_slot + 1) % SLOTS;
   }
   *out = p;
   return MISA_OK;

@@ -39,7 +39,7 @@ size_t route_umma_ws_bytes(int n_q, int H, int M_cap, int n_seq);
 cudaError_t launch_route_umma(const CacheView &c, const QueryView &q, int h, int32_t *heads, float *router_scores,
                               void *ws, cudaStream_t s, int agg = 0);
 
-// score_mma.cu: scores[i][t] (row stride ld) for t < L_i, heads given per query
+// score_dispatch.cu: scores[i][t] (row stride ld) for t < L_i, heads given per query
 // (heads == nullptr: all H heads, dense).  `gather` != nullptr: row i scores the
 // tokens gather[i][0..n_cols) instead of the prefix (re-rank).
 // Every launch also adds each written score to row_hist[i][key >> 21] (the

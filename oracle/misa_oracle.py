@@ -23,7 +23,7 @@ per token shared by all heads ([ABS]: the heads share one selected token set),
 and with no extra global scale (a positive global factor changes no
 selection).  For fp8 keys the dequantised key is s_t * e4m3(code_t).
 
-Readings where the pages are silent (each also listed in the design notes):
+Readings taken where the pages are silent:
 
 * router aggregation: r_j = |w_j| * sum_m ReLU(q_j . kbar_m)  ("aggregates
   these scores to estimate each head's importance", [SUM] step 1), with the

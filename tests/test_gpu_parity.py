@@ -318,6 +318,50 @@ def test_rerank(case):
     assert device_status(cache) == 0
 
 
+def _large_kprime_case():
+    """Two queries re-ranking k' = 20000 candidates: rows too long to stage in
+    shared memory, so the selection sweeps them from global memory."""
+    wl = W["misa_dagger_decode_128k"].scaled(n_seq=2, L=40000, B=128, k=1500, k_prime=20000)
+    inp = make(wl, seed=3)
+    ref = Ref(inp)
+    rng = np.random.default_rng(21)
+    cands = []
+    for i in range(wl.n_q):
+        Li = int(inp.q_pos[i]) + 1
+        c = rng.choice(Li, size=wl.k_prime, replace=False).astype(np.int32)
+        c[:5] = -1                                         # ignored entries
+        cands.append(c)
+    return inp, ref, wl, np.stack(cands)
+
+
+def check_rerank_against_oracle(ref, wl, cands, top, sc=None):
+    ties = 0
+    for i in range(wl.n_q):
+        q, w, K, Li = ref.query(i)
+        f = O.rerank_query(q, w, K, cands[i], wl.k)
+        smap = dict(zip(f["cand"].tolist(), f["scores"].tolist()))
+        if sc is not None:
+            valid = cands[i] >= 0
+            assert_close(sc[i][valid], f["scores"], f"rerank scores q{i}")
+        ties += compare_selection(top[i], f["topk"], lambda t: smap[t], wl.k, f"rerank q{i}")
+        got = top[i][top[i] >= 0]
+        assert np.all(np.diff(got) > 0) and len(got) == min(wl.k, int((cands[i] >= 0).sum()))
+    return ties
+
+
+def test_rerank_k_prime_above_16k():
+    inp, ref, wl, cands = _large_kprime_case()
+    cache, qs = to_device(inp, torch)
+    sc = torch.full((wl.n_q, wl.k_prime), float("nan"), device="cuda")
+    top = M.rerank_topk(cache, qs, torch.from_numpy(cands).cuda(), wl.k, scores_out=sc).cpu().numpy()
+    ties = check_rerank_against_oracle(ref, wl, cands, top, sc.cpu().numpy())
+    top2 = M.rerank_topk(cache, qs, torch.from_numpy(cands).cuda(), wl.k).cpu().numpy()  # scores in the workspace
+    np.testing.assert_array_equal(top, top2)
+    print(f"\nrerank k'=20000: {ties} boundary ties")
+    assert ties <= 2
+    assert device_status(cache) == 0
+
+
 def test_rerank_with_all_candidates_is_dense():
     inp = make("bf16_mixture")
     wl = inp.wl
