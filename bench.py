@@ -2,12 +2,17 @@
 
 Workload (default): 8 decode sequences at L = 131072 with fp8 e4m3 index keys
 (one fp32 scale per token), H_I = 64 index heads, block B = 128, h = 8 routed
-heads, k' = 8192 candidates re-ranked by all heads to k = 2048.  One step:
+heads, k' = 8192 candidates re-ranked by all heads to k = 2048.  One step is
+one misa_dagger_decode call (the same result as these four in sequence):
 
   1. misa_pool_keys  -- append the new token's key and refresh its block mean
   2. misa_route_heads -- block-pooled router, top-8 heads per query
   3. misa_score_topk -- routed scoring of all 131072 prefix tokens, top-k'
   4. misa_rerank_topk -- dense re-score of the k' candidates, top-k
+
+which for this batch runs as three kernels: the append, routing + routed
+scoring + top-k', and the re-rank + top-k.  The line also carries one object
+per workload (cfg_<name>) with the figures of all five at full size.
 
 Metric: scored head.tokens/s = sum over queries of (h L_i + H_I M_i + H_I k')
 per step / step time (also queries/s).  Inputs are synthetic (seeded
@@ -53,18 +58,19 @@ def work_per_query(wl, L_i):
 
 
 def score_kernel_bytes(wl):
-    """Algorithmic bytes of the routed scoring kernel per launch: keys (+scales) once,
-    the routed query heads and their weights."""
+    """Algorithmic bytes of the decode step's routed scoring kernel per launch,
+    which also routes and selects: the keys (+ scales) once, every query head
+    and weight (the router reads all H_I heads), the pooled keys, and the k'
+    candidate indices written."""
     row = wl.d * (1 if wl.key_dtype == "fp8" else 2) + (4 if wl.key_dtype == "fp8" else 0)
-    return wl.n_seq * wl.L * row + wl.n_q * wl.h * (wl.d * 2 + 4)
+    M = -(-wl.L // wl.B)
+    return (wl.n_seq * wl.L * row + wl.n_q * wl.H * (wl.d * 2 + 4) + wl.n_seq * M * wl.d * 4 +
+            wl.n_q * (wl.k_prime or wl.k) * 4)
 
 
-# DRAM bytes (read + write) of one routed scoring launch per workload, from
-# an ncu capture of the current kernel version; reported as null where there
-# is none.  The last capture of the routed scorer on the MISA-dagger decode
-# workload (143,242,496 bytes, summarised with the other ncu figures under
-# profiles/) predates the grid-dependency wait every kernel now starts with,
-# so until it is retaken the figure is null.
+# DRAM bytes (read + write) of one launch of the decode step's routed scoring
+# kernel per workload, from an ncu capture of the current kernel (summarised
+# under profiles/); null where the kernel changed since the last capture.
 STREAM_TRAFFIC_BYTES = {}
 
 
@@ -207,52 +213,97 @@ def aggregate(total_ms, steps, per_step_work, queries_per_step, world, dist=None
     return ms, world * per_step_work / (ms * 1e-3), world * queries_per_step / (ms * 1e-3)
 
 
-def prefill_roofline(M, torch, dev, peak_tflops, peak_src):
-    """Tensor-core prefill scoring on the two prefill workloads (context for
-    the decode headline): the scoring kernel's useful TFLOP/s against the
-    measured bf16 peak, and the whole score + top-k call."""
+def config_figures(M, torch, dev, hbm, tflops, flush_l2, with_oracle):
+    """Every workload at full size, one flat object each (scalars only): the
+    MISA call -- route + routed score + top-k, or for a workload with k' the
+    decode step's append + route + MISA-dagger in one call -- and the dense
+    DSA call, timed with CUDA events (median of 5, L2 flushed before each), the
+    routed scoring kernel alone, queries/s, scored head*tokens/s, the fractions
+    of the roofline the workload is bound by (key bytes against the measured
+    copy bandwidth for decode, useful tensor flops against the measured bf16
+    peak for prefill), and the CPU oracle's rate on the machine's host cores."""
     out = {}
-    for name in ("causal_prefill", "long_prefill_128k"):
-        wl = G.WORKLOADS[name]
+    for name, wl in G.WORKLOADS.items():
         inp = G.make_inputs(wl, 0)
         cache, qs = M.device_inputs(inp, dev)
         M.pool_keys(cache)
-        heads = M.route_heads(cache, qs, wl.h)
         ws = M.Workspace(dev)
         li = inp.q_pos.astype(np.int64) + 1
-        rec = {}
-        for kind, n_heads in (("misa", wl.h), ("dense", wl.H)):
-            def run():
-                if kind == "misa":
-                    M.score_topk(cache, qs, heads, wl.k, ws=ws)
-                else:
-                    M.dense_score_topk(cache, qs, wl.k, ws=ws)
+        stream = torch.cuda.current_stream(dev)
+        if wl.k_prime:
+            pos = torch.from_numpy(inp.q_pos.copy()).to(dev)
+            nk = torch.from_numpy(np.stack([inp.keys[s, inp.q_pos[s]:inp.q_pos[s] + 1] for s in range(wl.n_seq)]))
+            nk = nk.to(dev).contiguous()
+            ns = None if inp.scale is None else torch.from_numpy(
+                np.stack([inp.scale[s, inp.q_pos[s]:inp.q_pos[s] + 1] for s in range(wl.n_seq)])).to(dev)
+
+            def misa():  # appends at the same positions again: idempotent
+                M.dagger_decode(cache, qs, nk, ns, pos, wl.h, wl.k_prime, wl.k, ws=ws, stream=stream)
+        else:
+            def misa():
+                heads = M.route_heads(cache, qs, wl.h, ws=ws, stream=stream)
+                M.score_topk(cache, qs, heads, wl.k, ws=ws, stream=stream)
+
+        def dense():
+            M.dense_score_topk(cache, qs, wl.k, ws=ws, stream=stream)
+
+        def timed(fn, n=5):
             for _ in range(2):
-                run()
-            torch.cuda.synchronize()
-            ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            ka.record()
-            kb.record()
-            torch.cuda.synchronize()
-            M.debug_time_scoring(ka, kb)
-            kt, tt = [], []
-            for _ in range(5):
-                a.record()
-                run()
-                b.record()
+                fn()
+            ts = []
+            for _ in range(n):
+                flush_l2()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn()
+                b.record(stream)
                 torch.cuda.synchronize()
-                kt.append(ka.elapsed_time(kb))
-                tt.append(a.elapsed_time(b))
+                ts.append(a.elapsed_time(b))
+            return float(np.median(ts))
+
+        t_call, t_dense = timed(misa), timed(dense)
+        heads = M.route_heads(cache, qs, wl.h, ws=ws)
+        ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ka.record()
+        kb.record()
+        kt = []
+        for _ in range(5):
+            flush_l2()
+            M.debug_time_scoring(ka, kb)
+            M.score_topk(cache, qs, heads, wl.k_prime or wl.k, ws=ws)
+            torch.cuda.synchronize()
             M.debug_time_scoring(None, None)
-            k_ms = float(np.median(kt))
-            flops = 2.0 * wl.d * n_heads * float(li.sum())
-            tf = flops / (k_ms * 1e-3) / 1e12
-            rec[kind] = {"scoring_us": k_ms * 1e3, "score_topk_us": float(np.median(tt)) * 1e3,
-                         "achieved": tf, "peak": peak_tflops, "unit": "TFLOP/s", "frac": tf / peak_tflops,
-                         "peak_source": peak_src}
-        out[name] = {"kernel": "score_umma_kernel (tcgen05, TMA, TMEM)", "n_q": wl.n_q, "L": wl.L,
-                     "key_dtype": wl.key_dtype, **rec}
+            kt.append(ka.elapsed_time(kb))
+        t_scorer = float(np.median(kt))
+        assert cache.device_status() == 0, f"device status set on {name}"
+        work = float(sum(work_per_query(wl, int(x)) for x in li))
+        row = wl.d * (1 if wl.key_dtype == "fp8" else 2) + (4 if wl.key_dtype == "fp8" else 0)
+        rec = {"workload": name, "n_q": wl.n_q, "L": wl.L, "H_I": wl.H, "h": wl.h, "k": wl.k,
+               "k_prime": wl.k_prime or 0, "key_dtype": wl.key_dtype,
+               "call": "append + route + MISA-dagger (misa_dagger_decode)" if wl.k_prime
+               else "route + routed score + top-k",
+               "call_ms": t_call, "dense_dsa_ms": t_dense, "scorer_ms": t_scorer,
+               "queries_per_s": wl.n_q / (t_call * 1e-3), "head_tokens_per_s": work / (t_call * 1e-3),
+               "speedup_vs_dense": t_dense / t_call}
+        if wl.mode == "decode":
+            key_bytes = float(li.sum()) * row
+            rec.update({"bound": "hbm", "peak_gbs": hbm,
+                        "call_frac": key_bytes / (t_call * 1e-3) / 1e9 / hbm,
+                        "scorer_frac": (key_bytes + wl.n_q * wl.h * (2 * wl.d + 4)) / (t_scorer * 1e-3) / 1e9 / hbm})
+        else:
+            M_i = -(-li // wl.B)
+            flops = 2.0 * wl.d * (wl.h * float(li.sum()) + wl.H * float(M_i.sum()))
+            sflops = 2.0 * wl.d * wl.h * float(li.sum())
+            rec.update({"bound": "tensor", "peak_tflops": tflops,
+                        "call_frac": flops / (t_call * 1e-3) / 1e12 / tflops,
+                        "scorer_frac": sflops / (t_scorer * 1e-3) / 1e12 / tflops,
+                        "scorer_frac_of_e4m3_peak": (sflops / (t_scorer * 1e-3) / 1e12 / (2 * tflops)
+                                                     if wl.key_dtype == "fp8" else None)})
+        if with_oracle:
+            v, q, dt, cores, n = cpu_oracle_rate(wl, inp, 1, min_seconds=4.0)
+            rec.update({"oracle_queries_per_s": q, "oracle_head_tokens_per_s": v, "oracle_cores": cores,
+                        "oracle_sample": f"{n} queries in {dt:.1f} s, numpy fp64"})
+        out["cfg_" + name] = rec
         del cache, qs, ws
         torch.cuda.empty_cache()
     return out
@@ -272,7 +323,8 @@ def main():
     ap.add_argument("--impl", default="misa", choices=["misa", "reference"])
     ap.add_argument("--workload", default="misa_dagger_decode_128k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill tensor-core context figures")
+    ap.add_argument("--no-configs", "--no-prefill", dest="no_configs", action="store_true",
+                    help="skip the per-workload figures of all five workloads")
     args = ap.parse_args()
     wl = G.WORKLOADS[args.workload]
     if args.impl == "reference":
@@ -363,9 +415,23 @@ def main():
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clk = clocks.stop()
+    clk_timed = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = float(sum(step_ms))
+    # The timed steps last a few milliseconds, too short for NVML's sampling:
+    # the clocks are also sampled over a second of the same steps replayed
+    # back to back (L2 flushed between them), which is what the record reports.
+    clocks_w = Clocks(dev)
+    clocks_w.start()
+    t_end = time.perf_counter() + 1.0
+    while time.perf_counter() < t_end:
+        for _ in range(50):
+            flush_l2()
+            step.replay()
+        torch.cuda.synchronize()
+    clk = clocks_w.stop()
+    clk["source"] = "NVML polling every ~2 ms over 1 s of the timed step replayed back to back"
+    clk["timed_region"] = {k: clk_timed.get(k) for k in ("sm_mhz", "samples", "reasons")}
     # the routed scoring kernel's own window (event nodes inside the graph,
     # overwritten by every replay): read after each of a few more steps
     for _ in range(max(10, min(args.steps, 50))):
@@ -443,6 +509,20 @@ def main():
     assert np.array_equal(h_top.numpy(), step.topk.cpu().numpy())  # same result as the device-resident step
     e2e_step = float(np.mean(e2e_ms[1:]))
     e2e_value = world * per_step_work / (e2e_step * 1e-3)
+    # the same without the graph: every step goes through the binding and the
+    # C ABI's host-side validation and dispatch
+    eager_ms = []
+    for i in range(max(5, args.steps // 2)):
+        flush_l2()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_body()
+        b.record(stream)
+        b.synchronize()
+        eager_ms.append(a.elapsed_time(b))
+    assert np.array_equal(h_top.numpy(), step.topk.cpu().numpy())
+    eager_step = float(np.mean(eager_ms[1:]))
 
     if rank == 0:
         hbm, _, src = peaks()
@@ -459,14 +539,19 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e4m3",
-            "dtype_detail": "e4m3 keys x two-term e4m3 split of the bf16 query (mma.sync), f32 accumulate",
+            "dtype_detail": "e4m3 keys x two-term e4m3 split of the bf16 query (mma.sync routed pass, tcgen05 "
+                            "re-rank), f32 accumulate",
             "data": "synthetic (seeded generator), resident in HBM",
             "config": config_block(wl, l2="flushed between steps: 256 MiB write then 256 MiB read (clean lines)"),
             "queries_per_s": qps,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_step},
+                    "ms_per_step": e2e_step, "how": "copy in, the step, copy out, replayed as one CUDA graph"},
+            "e2e_eager": {"value": world * per_step_work / (eager_step * 1e-3), "unit": UNIT,
+                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": eager_step,
+                          "how": "copy in, misa_dagger_decode through the binding, copy out; no graph"},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
-            "roofline": {"kernel": "routed token scoring (score_stream_kernel<1, e4m3>)", "bound": "hbm",
+            "roofline": {"kernel": "routing + routed token scoring + top-k' (score_stream_kernel<1, e4m3>)",
+                         "bound": "hbm",
                          "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                          "traffic": STREAM_TRAFFIC_BYTES.get(wl.name), "algorithmic_bytes_per_launch": kb, "ms_per_launch": k_ms,
                          "peak_source": f"{src} hbm_gbs"},
@@ -476,10 +561,9 @@ def main():
         }
         if cpu:
             line["cpu_baseline"] = cpu
-        if not args.no_prefill and world == 1:
-            pk = peaks()
-            line["prefill"] = prefill_roofline(M, torch, dev, pk[1], f"{pk[2]} bf16_tflops (e4m3 runs two MMAs "
-                                               "per K step at twice the rate: same time per useful flop)")
+        if not args.no_configs and world == 1:
+            hbm_p, tf_p, _ = peaks()
+            line.update(config_figures(M, torch, dev, hbm_p, tf_p, flush_l2, not args.no_cpu_baseline))
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -90,7 +90,8 @@ typedef enum {
   MISA_OP_SCORE_TOPK = 1,   /* misa_score_topk */
   MISA_OP_DENSE_TOPK = 2,   /* dsa_dense_score_topk */
   MISA_OP_RERANK_TOPK = 3,  /* misa_rerank_topk */
-  MISA_OP_DAGGER_TOPK = 4   /* misa_dagger_topk */
+  MISA_OP_DAGGER_TOPK = 4,  /* misa_dagger_topk */
+  MISA_OP_DAGGER_DECODE = 5 /* misa_dagger_decode */
 } misa_op;
 
 /* Bits OR-ed into misa_cache.status by the device. */
@@ -98,6 +99,7 @@ typedef enum {
 #define MISA_DEV_APPEND_RANGE 2u  /* append beyond L_cap: that sequence was skipped */
 #define MISA_DEV_WAIT_TIMEOUT 4u  /* an on-chip pipeline wait ran out of time: outputs invalid */
 #define MISA_DEV_BAD_HEAD 8u      /* a head index outside [0, H): head 0 was used instead */
+#define MISA_DEV_SMEM_LAYOUT 16u  /* a kernel's shared-memory layout did not fit its allocation: it wrote nothing */
 
 /*
  * Index-key cache of n_seq sequences (one shared index key per token,
@@ -282,6 +284,34 @@ MISA_API misa_status misa_rerank_topk(const misa_cache *cache, const misa_querie
 MISA_API misa_status misa_dagger_topk(const misa_cache *cache, const misa_queries *qs,
                                       const int32_t *heads, int32_t h, int32_t k_prime, int32_t k,
                                       int32_t *topk, void *ws, size_t ws_bytes, misa_stream stream);
+
+/*
+ * One MISA-dagger decode step in one call: the composition of misa_pool_keys
+ * in append mode ("Methodology: MISA", step 1: the block means stay current
+ * as keys are written), misa_route_heads (step 1: the top-h heads of every
+ * query) and misa_dagger_topk ("Hierarchical variant": the routed top-k'
+ * candidates re-ranked with all heads to the final top-k).
+ *   new_keys, new_scale, new_pos, count: the keys appended, as in
+ *              misa_pool_keys (count >= 1); the queries' prefixes may
+ *              include them
+ *   heads      [n_q][h] int32 out, each query's routed heads ascending, or
+ *              NULL
+ *   topk       [n_q][k] int32 out (ascending token indices, -1 padded)
+ * Decode batches (few queries per sequence) whose scoring grid fits on the
+ * device at once route inside the routed scoring kernel: the C CTAs that
+ * score a query each sum the router over a slice of its blocks and then add
+ * the C partial sums in a fixed order.  misa_route_heads sums the same terms
+ * in another grouping, so a head whose importance equals another's to within
+ * rounding can be chosen differently; otherwise the results are those of the
+ * three calls in sequence (which is what runs for other shapes).
+ * Workspace: misa_workspace_bytes(MISA_OP_DAGGER_DECODE, cache, qs, h, k,
+ * k_prime).  Errors: those of the three calls; count outside [1, L_cap] is
+ * MISA_ERR_INVALID.
+ */
+MISA_API misa_status misa_dagger_decode(const misa_cache *cache, const misa_queries *qs, const void *new_keys,
+                                        const float *new_scale, const int32_t *new_pos, int32_t count, int32_t h,
+                                        int32_t k_prime, int32_t k, int32_t *heads, int32_t *topk, void *ws,
+                                        size_t ws_bytes, misa_stream stream);
 
 /*
  * misa_rerank_topk without a caller workspace and without any allocation.

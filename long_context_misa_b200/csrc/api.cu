@@ -151,9 +151,62 @@ size_t rerank_hist_words(const misa_queries *q) { return (size_t)q->n_q * misa::
 size_t ws_dagger_hist(const misa_queries *q) {
   return ws_hist(q) + round_up(sizeof(uint32_t) * rerank_hist_words(q));
 }
-size_t ws_dagger(const misa_cache *c, const misa_queries *q, int k_prime) {
+size_t ws_fz_zero(const misa_queries *q);
+size_t ws_fz_bucket(const misa_queries *q);
+size_t ws_fz_win(const misa_queries *q, int k);
+// [hist + counters][re-rank hist][fused zeroed: routed pass][fused zeroed:
+// re-rank] (zeroed by one launch) [routed scores][top-k' list][bucket]
+// [winners][candidates][re-rank scores]
+size_t ws_dagger(const misa_cache *c, const misa_queries *q, int k_prime, int k) {
   const size_t cand = round_up(sizeof(int32_t) * (size_t)q->n_q * k_prime);
-  return ws_dagger_hist(q) + ws_score(c, q) + ws_list(c, q, k_prime) + 2 * cand;
+  return ws_dagger_hist(q) + 2 * ws_fz_zero(q) + ws_score(c, q) + ws_list(c, q, k_prime) + ws_fz_bucket(q) +
+         ws_fz_win(q, k) + 2 * cand;
+}
+
+// Regions of a selection done inside the scoring kernel (misa::FusedTopk):
+// words zeroed before the launch, the boundary bucket, the winners of an
+// ascending output.  Every workspace reserves them beside the regions of the
+// separate top-k kernels; which set a call uses is decided per call
+// (misa::score_fusable).
+size_t ws_fz_zero(const misa_queries *q) { return round_up(sizeof(uint32_t) * (size_t)q->n_q * misa::FUSED_ZERO_WORDS); }
+size_t ws_fz_bucket(const misa_queries *q) { return round_up(sizeof(uint2) * (size_t)q->n_q * misa::FUSED_BCAP); }
+size_t ws_fz_win(const misa_queries *q, int k) { return round_up(sizeof(int32_t) * (size_t)q->n_q * k); }
+
+// score + top-k: [hist + counters][fused zeroed][scores, unless scores_out]
+// [top-k list][bucket][winners]
+size_t ws_score_topk(const misa_cache *c, const misa_queries *q, int k, bool scores_out) {
+  return ws_hist(q) + ws_fz_zero(q) + (scores_out ? 0 : ws_score(c, q)) + ws_list(c, q, k) + ws_fz_bucket(q) +
+         ws_fz_win(q, k);
+}
+// re-rank: [hist][fused zeroed][scores, unless scores_out][bucket][winners]
+size_t ws_rerank(const misa_queries *q, int k_prime, int k, bool scores_out) {
+  return ws_hist(q) + ws_fz_zero(q) + (scores_out ? 0 : round_up(sizeof(float) * (size_t)q->n_q * k_prime)) +
+         ws_fz_bucket(q) + ws_fz_win(q, k);
+}
+
+misa::FusedTopk fused_args(uint32_t *zeroed, void *bucket, void *winners, int32_t *out, int k, bool ordered) {
+  misa::FusedTopk f;
+  f.zeroed = zeroed;
+  f.bucket = static_cast<uint2 *>(bucket);
+  f.winners = static_cast<int32_t *>(winners);
+  f.out = out;
+  f.k = k;
+  f.ordered = ordered ? 1 : 0;
+  return f;
+}
+
+// misa_dagger_decode: [misa_dagger_topk's workspace][router: the separate
+// router's workspace, or the in-kernel router's partial sums][heads]
+size_t ws_route(const misa_cache *c, const misa_queries *q) {
+  const int M_cap = misa::cdiv(c->L_cap, c->B);
+  return round_up(std::max(misa::route_ws_bytes(q->n_q, q->H, M_cap),
+                           misa::route_umma_ws_bytes(q->n_q, q->H, M_cap, c->n_seq)));
+}
+size_t ws_decode_router(const misa_cache *c, const misa_queries *q) {
+  return std::max(ws_route(c, q), round_up(sizeof(float) * (size_t)misa::route_part_slots() * q->H));
+}
+size_t ws_decode(const misa_cache *c, const misa_queries *q, int h, int k_prime, int k) {
+  return ws_dagger(c, q, k_prime, k) + ws_decode_router(c, q) + round_up(sizeof(int32_t) * (size_t)q->n_q * h);
 }
 
 misa_status check_ws(void *ws, size_t have, size_t need) {
@@ -171,19 +224,29 @@ misa_status score_then_topk(const char *who, const misa_cache *cache, const misa
   uint8_t *w8 = static_cast<uint8_t *>(ws);
   uint32_t *hist = reinterpret_cast<uint32_t *>(w8);
   uint32_t *list_cnt = hist + (size_t)qs->n_q * misa::TOPK_HIST_BINS;
-  float *scores = scores_out ? scores_out : reinterpret_cast<float *>(w8 + ws_hist(qs));
-  void *list = w8 + ws_hist(qs) + (scores_out ? 0 : ws_score(cache, qs));
+  uint32_t *fz_zero = reinterpret_cast<uint32_t *>(w8 + ws_hist(qs));
+  uint8_t *after = w8 + ws_hist(qs) + ws_fz_zero(qs);
+  float *scores = scores_out ? scores_out : reinterpret_cast<float *>(after);
+  uint8_t *list = after + (scores_out ? 0 : ws_score(cache, qs));
+  uint8_t *bucket = list + ws_list(cache, qs, k);
+  uint8_t *winners = bucket + ws_fz_bucket(qs);
   // many queries per sequence (prefill chunks): tensor-core scoring, and the
-  // selection counts each row itself; otherwise the streaming scorer builds
-  // the row histograms on the way
+  // selection counts each row itself; otherwise the streaming scorer selects
+  // in-kernel when its grid is resident at once, or builds the row
+  // histograms on the way for the top-k kernels
   const bool umma = misa::umma_applies(c, q, heads, h);
-  cudaError_t e = misa::launch_zero(hist, hist_words(qs), stream);
+  const bool fused = !umma && misa::score_fusable(c, q, heads, h, nullptr, 0);
+  cudaError_t e = fused ? misa::launch_zero(fz_zero, (size_t)qs->n_q * misa::FUSED_ZERO_WORDS, stream)
+                        : misa::launch_zero(hist, hist_words(qs), stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
+  const misa::FusedTopk fz = fused_args(fz_zero, bucket, winners, topk, k, true);
   e = timed_scoring(stream, [&] {
     return umma ? misa::launch_score_umma(c, q, heads, h, scores, cache->L_cap, stream)
-                : misa::launch_score_mma(c, q, heads, h, nullptr, 0, scores, cache->L_cap, hist, stream);
+                : misa::launch_score_mma(c, q, heads, h, nullptr, 0, scores, cache->L_cap, hist, stream,
+                                         fused ? &fz : nullptr);
   });
   if (e != cudaSuccess) return cuda_fail(e, who);
+  if (fused) return MISA_OK;
   e = misa::launch_topk(c, q, scores, cache->L_cap, 0, nullptr, hist, !umma, list, list_cnt, k, topk, stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
   return MISA_OK;
@@ -274,6 +337,77 @@ misa_status noalloc_scratch(const char *who, void **out) {
   return MISA_OK;
 }
 
+// MISA-dagger on validated arguments (misa_dagger_topk): routed scores and
+// their k' candidates, then every head on the candidates and the final k.
+// With route_part (misa_dagger_decode, fused routed pass only) the scoring
+// kernel routes the queries itself and writes their heads to heads_out.
+// dagger_zero_words(): the words from the workspace's start that a call
+// counts into when both passes select in-kernel or neither does, or
+// everything up to the end of the fused words when the passes differ;
+// zero_done: a kernel before (the decode step's append) cleared them.
+size_t dagger_zero_words(const misa_queries *qs, bool f1, bool f2) {
+  const size_t fz_end = (ws_dagger_hist(qs) + ws_fz_zero(qs)) / sizeof(uint32_t) + (size_t)qs->n_q * misa::FUSED_ZERO_WORDS;
+  return (f1 || f2) ? fz_end : ws_hist(qs) / sizeof(uint32_t) + rerank_hist_words(qs);
+}
+
+misa_status dagger_body(const char *who, const misa_cache *cache, const misa_queries *qs, const int32_t *heads,
+                        int h, int k_prime, int k, int32_t *topk, void *ws, cudaStream_t stream,
+                        float *route_part = nullptr, int32_t *heads_out = nullptr, bool zero_done = false) {
+  misa::CacheView c = view(cache);
+  misa::QueryView q = view(qs);
+  uint8_t *w8 = static_cast<uint8_t *>(ws);
+  uint32_t *hist = reinterpret_cast<uint32_t *>(w8);
+  uint32_t *list_cnt = hist + (size_t)qs->n_q * misa::TOPK_HIST_BINS;
+  uint32_t *rhist = reinterpret_cast<uint32_t *>(w8 + ws_hist(qs));
+  uint32_t *fz1 = reinterpret_cast<uint32_t *>(w8 + ws_dagger_hist(qs));
+  uint32_t *fz2 = reinterpret_cast<uint32_t *>(w8 + ws_dagger_hist(qs) + ws_fz_zero(qs));
+  uint8_t *p = w8 + ws_dagger_hist(qs) + 2 * ws_fz_zero(qs);
+  float *scores = reinterpret_cast<float *>(p);
+  p += ws_score(cache, qs);
+  void *list = p;
+  p += ws_list(cache, qs, k_prime);
+  uint8_t *bucket = p;
+  p += ws_fz_bucket(qs);
+  uint8_t *winners = p;
+  p += ws_fz_win(qs, k);
+  int32_t *cand = reinterpret_cast<int32_t *>(p);
+  float *rscores = reinterpret_cast<float *>(p + round_up(sizeof(int32_t) * (size_t)qs->n_q * k_prime));
+  // routed pass: scores, then the k' candidates in any order; selected in the
+  // scoring kernels when their grids are resident at once
+  const bool umma = !route_part && misa::umma_applies(c, q, heads, h);
+  const bool f1 = route_part || (!umma && misa::score_fusable(c, q, heads, h, nullptr, 0));
+  const bool f2 = misa::score_fusable(c, q, nullptr, q.H, cand, k_prime);
+  // both passes' counting words, zeroed by one launch: the histograms and
+  // counters of the top-k kernels, the fused selections' words, or both
+  uint32_t *z0 = (f1 && f2) ? fz1 : hist;
+  uint32_t *z1 = hist + dagger_zero_words(qs, f1, f2);
+  cudaError_t e = zero_done ? cudaSuccess : misa::launch_zero(z0, (size_t)(z1 - z0), stream);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  const misa::FusedTopk fzc = fused_args(fz1, bucket, nullptr, cand, k_prime, false);
+  e = timed_scoring(stream, [&] {
+    if (route_part)
+      return misa::launch_score_stream(c, q, nullptr, h, scores, cache->L_cap, hist, stream, &fzc, route_part,
+                                       heads_out);
+    return umma ? misa::launch_score_umma(c, q, heads, h, scores, cache->L_cap, stream)
+                : misa::launch_score_mma(c, q, heads, h, nullptr, 0, scores, cache->L_cap, hist, stream,
+                                         f1 ? &fzc : nullptr);
+  });
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  if (!f1) {
+    e = misa::launch_topk(c, q, scores, cache->L_cap, 0, nullptr, hist, !umma, list, list_cnt, k_prime, cand, stream,
+                          false);
+    if (e != cudaSuccess) return cuda_fail(e, who);
+  }
+  // fine pass: every head on the candidates, ascending final top-k
+  const misa::FusedTopk fzr = fused_args(fz2, bucket, winners, topk, k, true);
+  e = misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, rscores, k_prime, rhist, stream, f2 ? &fzr : nullptr);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  if (f2) return MISA_OK;
+  e = misa::launch_topk(c, q, rscores, k_prime, k_prime, cand, rhist, true, nullptr, nullptr, k, topk, stream);
+  if (e != cudaSuccess) return cuda_fail(e, who);
+  return MISA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -318,21 +452,19 @@ misa_status misa_append_keys_e4m3(const misa_cache *cache, const uint16_t *new_k
 
 size_t misa_workspace_bytes(int32_t op, const misa_cache *cache, const misa_queries *qs, int32_t h, int32_t k,
                             int32_t k_prime) {
-  (void)h;
   if (!cache || !qs || cache->B < 1 || cache->L_cap < 1 || qs->n_q < 0 || qs->H < 1) return 0;
   switch (op) {
-    case MISA_OP_ROUTE: {
-      const int M_cap = misa::cdiv(cache->L_cap, cache->B);
-      return round_up(std::max(misa::route_ws_bytes(qs->n_q, qs->H, M_cap),
-                               misa::route_umma_ws_bytes(qs->n_q, qs->H, M_cap, cache->n_seq)));
-    }
+    case MISA_OP_ROUTE:
+      return ws_route(cache, qs);
     case MISA_OP_SCORE_TOPK:
     case MISA_OP_DENSE_TOPK:
-      return ws_hist(qs) + ws_score(cache, qs) + (k > 0 ? ws_list(cache, qs, k) : 0);
+      return k > 0 ? ws_score_topk(cache, qs, k, false) : 0;
     case MISA_OP_RERANK_TOPK:
-      return k_prime > 0 ? ws_hist(qs) + round_up(sizeof(float) * (size_t)qs->n_q * k_prime) : 0;
+      return k_prime > 0 && k > 0 ? ws_rerank(qs, k_prime, k, false) : 0;
     case MISA_OP_DAGGER_TOPK:
-      return k_prime > 0 ? ws_dagger(cache, qs, k_prime) : 0;
+      return k_prime > 0 && k > 0 ? ws_dagger(cache, qs, k_prime, k) : 0;
+    case MISA_OP_DAGGER_DECODE:
+      return k_prime > 0 && k > 0 && h > 0 ? ws_decode(cache, qs, h, k_prime, k) : 0;
     default:
       return 0;
   }
@@ -370,8 +502,7 @@ misa_status misa_score_topk(const misa_cache *cache, const misa_queries *qs, con
   if (h < 1 || h > qs->H) return fail(MISA_ERR_INVALID, "h=%d outside [1, H=%d]", h, qs->H);
   if (k < 1) return fail(MISA_ERR_INVALID, "k=%d < 1", k);
   if (qs->n_q > 0 && (!heads || !topk)) return fail(MISA_ERR_INVALID, "heads/topk is NULL");
-  const size_t need = ws_hist(qs) + (scores_out ? 0 : ws_score(cache, qs)) + ws_list(cache, qs, k);
-  if ((st = check_ws(ws, ws_bytes, need)) != MISA_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, ws_score_topk(cache, qs, k, scores_out != nullptr))) != MISA_OK) return st;
   if (injected_failure("misa_score_topk", &st)) return st;
   if (qs->n_q == 0) return MISA_OK;
   return score_then_topk("misa_score_topk", cache, qs, heads, h, k, topk, scores_out, ws, stream);
@@ -385,8 +516,7 @@ misa_status dsa_dense_score_topk(const misa_cache *cache, const misa_queries *qs
   if ((st = check_queries(qs)) != MISA_OK) return st;
   if (k < 1) return fail(MISA_ERR_INVALID, "k=%d < 1", k);
   if (qs->n_q > 0 && !topk) return fail(MISA_ERR_INVALID, "topk is NULL");
-  const size_t need = ws_hist(qs) + (scores_out ? 0 : ws_score(cache, qs)) + ws_list(cache, qs, k);
-  if ((st = check_ws(ws, ws_bytes, need)) != MISA_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, ws_score_topk(cache, qs, k, scores_out != nullptr))) != MISA_OK) return st;
   if (injected_failure("dsa_dense_score_topk", &st)) return st;
   if (qs->n_q == 0) return MISA_OK;
   return score_then_topk("dsa_dense_score_topk", cache, qs, nullptr, qs->H, k, topk, scores_out, ws, stream);
@@ -402,20 +532,29 @@ misa_status misa_rerank_topk(const misa_cache *cache, const misa_queries *qs, co
   if (k < 1 || k_prime < k) return fail(MISA_ERR_INVALID, "need 1 <= k=%d <= k_prime=%d", k, k_prime);
   if (k_prime > MISA_MAX_L) return fail(MISA_ERR_UNSUPPORTED, "k_prime=%d above %d", k_prime, MISA_MAX_L);
   if (qs->n_q > 0 && (!cand || !topk)) return fail(MISA_ERR_INVALID, "cand/topk is NULL");
-  const size_t need = ws_hist(qs) + (scores_out ? 0 : round_up(sizeof(float) * (size_t)qs->n_q * k_prime));
-  if ((st = check_ws(ws, ws_bytes, need)) != MISA_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, ws_rerank(qs, k_prime, k, scores_out != nullptr))) != MISA_OK) return st;
   if (injected_failure("misa_rerank_topk", &st)) return st;
   if (qs->n_q == 0) return MISA_OK;
   misa::CacheView c = view(cache);
   misa::QueryView q = view(qs);
-  uint32_t *hist = static_cast<uint32_t *>(ws);
-  float *scores = scores_out ? scores_out : reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + ws_hist(qs));
-  cudaError_t e = misa::launch_zero(hist, (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
+  uint8_t *w8 = static_cast<uint8_t *>(ws);
+  uint32_t *hist = reinterpret_cast<uint32_t *>(w8);
+  uint32_t *fz_zero = reinterpret_cast<uint32_t *>(w8 + ws_hist(qs));
+  uint8_t *after = w8 + ws_hist(qs) + ws_fz_zero(qs);
+  float *scores = scores_out ? scores_out : reinterpret_cast<float *>(after);
+  uint8_t *bucket = after + (scores_out ? 0 : round_up(sizeof(float) * (size_t)qs->n_q * k_prime));
+  uint8_t *winners = bucket + ws_fz_bucket(qs);
+  const bool fused = misa::score_fusable(c, q, nullptr, q.H, cand, k_prime);
+  cudaError_t e = fused ? misa::launch_zero(fz_zero, (size_t)qs->n_q * misa::FUSED_ZERO_WORDS, stream)
+                        : misa::launch_zero(hist, (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
   if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
+  const misa::FusedTopk fz = fused_args(fz_zero, bucket, winners, topk, k, true);
   e = timed_scoring(stream, [&] {
-    return misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, scores, k_prime, hist, stream);
+    return misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, scores, k_prime, hist, stream,
+                                  fused ? &fz : nullptr);
   });
   if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
+  if (fused) return MISA_OK;
   e = misa::launch_topk(c, q, scores, k_prime, k_prime, cand, hist, true, nullptr, nullptr, k, topk, stream);
   if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
   return MISA_OK;
@@ -469,40 +608,61 @@ misa_status misa_dagger_topk(const misa_cache *cache, const misa_queries *qs, co
   if (k < 1 || k_prime < k) return fail(MISA_ERR_INVALID, "need 1 <= k=%d <= k_prime=%d", k, k_prime);
   if (k_prime > MISA_MAX_L) return fail(MISA_ERR_UNSUPPORTED, "k_prime=%d above %d", k_prime, MISA_MAX_L);
   if (qs->n_q > 0 && (!heads || !topk)) return fail(MISA_ERR_INVALID, "heads/topk is NULL");
-  if ((st = check_ws(ws, ws_bytes, ws_dagger(cache, qs, k_prime))) != MISA_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, ws_dagger(cache, qs, k_prime, k))) != MISA_OK) return st;
   if (injected_failure(who, &st)) return st;
   if (qs->n_q == 0) return MISA_OK;
+  return dagger_body(who, cache, qs, heads, h, k_prime, k, topk, ws, stream);
+}
+
+misa_status misa_dagger_decode(const misa_cache *cache, const misa_queries *qs, const void *new_keys,
+                               const float *new_scale, const int32_t *new_pos, int32_t count, int32_t h,
+                               int32_t k_prime, int32_t k, int32_t *heads, int32_t *topk, void *ws, size_t ws_bytes,
+                               misa_stream stream) {
+  NvtxRange nvtx("misa_dagger_decode");
+  const char *who = "misa_dagger_decode";
+  misa_status st = check_cache(cache, true);
+  if (st != MISA_OK) return st;
+  if ((st = check_queries(qs)) != MISA_OK) return st;
+  if (count < 1 || count > cache->L_cap)
+    return fail(MISA_ERR_INVALID, "count=%d outside [1, L_cap=%d]", count, cache->L_cap);
+  if (!new_keys || !new_pos) return fail(MISA_ERR_INVALID, "new_keys and new_pos must be non-NULL");
+  if ((cache->dtype == MISA_KEY_FP8_E4M3) != (new_scale != nullptr))
+    return fail(MISA_ERR_INVALID, "new_scale must be non-NULL exactly for fp8 keys");
+  if (!aligned16(new_keys)) return fail(MISA_ERR_INVALID, "new_keys must be 16-byte aligned");
+  if (h < 1 || h > qs->H) return fail(MISA_ERR_INVALID, "h=%d outside [1, H=%d]", h, qs->H);
+  if (k < 1 || k_prime < k) return fail(MISA_ERR_INVALID, "need 1 <= k=%d <= k_prime=%d", k, k_prime);
+  if (k_prime > MISA_MAX_L) return fail(MISA_ERR_UNSUPPORTED, "k_prime=%d above %d", k_prime, MISA_MAX_L);
+  if (qs->n_q > 0 && !topk) return fail(MISA_ERR_INVALID, "topk is NULL");
+  if ((st = check_ws(ws, ws_bytes, ws_decode(cache, qs, h, k_prime, k))) != MISA_OK) return st;
+  if (injected_failure(who, &st)) return st;
   misa::CacheView c = view(cache);
   misa::QueryView q = view(qs);
   uint8_t *w8 = static_cast<uint8_t *>(ws);
-  uint32_t *hist = reinterpret_cast<uint32_t *>(w8);
-  uint32_t *list_cnt = hist + (size_t)qs->n_q * misa::TOPK_HIST_BINS;
-  uint32_t *rhist = reinterpret_cast<uint32_t *>(w8 + ws_hist(qs));
-  float *scores = reinterpret_cast<float *>(w8 + ws_dagger_hist(qs));
-  void *list = w8 + ws_dagger_hist(qs) + ws_score(cache, qs);
-  int32_t *cand =
-      reinterpret_cast<int32_t *>(w8 + ws_dagger_hist(qs) + ws_score(cache, qs) + ws_list(cache, qs, k_prime));
-  float *rscores = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(cand) +
-                                             round_up(sizeof(int32_t) * (size_t)qs->n_q * k_prime));
-  // routed pass: scores, then the k' candidates in any order
-  const bool umma = misa::umma_applies(c, q, heads, h);
-  // both passes' histograms and counters, zeroed by one launch
-  cudaError_t e = misa::launch_zero(hist, ws_hist(qs) / sizeof(uint32_t) + rerank_hist_words(qs), stream);
+  uint8_t *rws = w8 + ws_dagger(cache, qs, k_prime, k);
+  int32_t *hbuf = heads ? heads : reinterpret_cast<int32_t *>(rws + ws_decode_router(cache, qs));
+  // decode batches whose scoring grid is resident at once: routing inside the
+  // routed scoring kernel, both selections inside their scoring kernels, and
+  // their counting words cleared by the append kernel
+  const bool fused = qs->n_q > 0 && !misa::umma_applies(c, q, nullptr, h) &&
+                     misa::score_stream_fusable(c, q, nullptr, h, true);
+  uint32_t *z0 = nullptr;
+  size_t zn = 0;
+  if (fused) {
+    // the re-rank's fusion does not depend on the candidates' values
+    const bool f2 = misa::score_fusable(c, q, nullptr, q.H, reinterpret_cast<const int32_t *>(w8), k_prime);
+    const size_t first = f2 ? ws_dagger_hist(qs) / sizeof(uint32_t) : 0;  // both fused: only their words
+    z0 = reinterpret_cast<uint32_t *>(w8) + first;
+    zn = dagger_zero_words(qs, true, f2) - first;
+  }
+  cudaError_t e = misa::launch_pool_append(c, new_keys, new_scale, new_pos, count, stream, z0, zn);
   if (e != cudaSuccess) return cuda_fail(e, who);
-  e = timed_scoring(stream, [&] {
-    return umma ? misa::launch_score_umma(c, q, heads, h, scores, cache->L_cap, stream)
-                : misa::launch_score_mma(c, q, heads, h, nullptr, 0, scores, cache->L_cap, hist, stream);
-  });
+  if (qs->n_q == 0) return MISA_OK;
+  if (fused)
+    return dagger_body(who, cache, qs, nullptr, h, k_prime, k, topk, ws, stream, reinterpret_cast<float *>(rws),
+                       heads, true);
+  e = misa::launch_route(c, q, h, hbuf, nullptr, rws, stream, MISA_AGG_ABS_SUM);
   if (e != cudaSuccess) return cuda_fail(e, who);
-  e = misa::launch_topk(c, q, scores, cache->L_cap, 0, nullptr, hist, !umma, list, list_cnt, k_prime, cand, stream,
-                        false);
-  if (e != cudaSuccess) return cuda_fail(e, who);
-  // fine pass: every head on the candidates, ascending final top-k
-  e = misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, rscores, k_prime, rhist, stream);
-  if (e != cudaSuccess) return cuda_fail(e, who);
-  e = misa::launch_topk(c, q, rscores, k_prime, k_prime, cand, rhist, true, nullptr, nullptr, k, topk, stream);
-  if (e != cudaSuccess) return cuda_fail(e, who);
-  return MISA_OK;
+  return dagger_body(who, cache, qs, hbuf, h, k_prime, k, topk, ws, stream);
 }
 
 misa_status misa_debug_wait_timeout(uint32_t *status, uint64_t limit_ns, misa_stream stream) {

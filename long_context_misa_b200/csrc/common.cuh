@@ -164,6 +164,23 @@ inline int cached_per_device(F &&f) {
   return v;
 }
 
+// Raise a kernel's dynamic shared-memory limit to the most the device allows
+// next to the kernel's own static shared memory.  Returns that limit (bytes)
+// or -1 on failure.
+template <class K>
+inline int opt_in_max_dyn_smem(K *kernel) {
+  int dev = 0, optin = 0;
+  cudaFuncAttributes fa;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+      cudaFuncGetAttributes(&fa, kernel) != cudaSuccess)
+    return -1;
+  const int mx = optin - (int)fa.sharedSizeBytes;
+  if (mx <= 0 || cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mx) != cudaSuccess)
+    return -1;
+  return mx;
+}
+
 struct SmCountTag {};
 inline int device_sms() {
   return cached_per_device<SmCountTag>([] {
@@ -249,6 +266,25 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// The tensor-core kernels lay out their shared memory from the first
+// 1024-byte boundary of the dynamic allocation (the 128-byte-swizzle atoms of
+// TMA destinations and MMA operands need it), and every launch allocates
+// 1024 bytes of slack for that.  Returns the aligned base, or nullptr when
+// `need` bytes from it do not fit in the dynamic shared memory the kernel was
+// launched with (a layout and an allocation that disagree): thread 0 then
+// flags MISA_DEV_SMEM_LAYOUT and the caller returns before any shared-memory
+// access.  The answer is the same in every thread.
+__device__ __forceinline__ uint8_t *aligned_smem_base(uint8_t *raw, uint32_t need, const CacheView &c) {
+  const uint32_t pad = (1024u - (smem_addr(raw) & 1023u)) & 1023u;
+  uint32_t dyn;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+  if (pad + need > dyn) {
+    if (threadIdx.x == 0) flag(c, MISA_DEV_SMEM_LAYOUT);
+    return nullptr;
+  }
+  return raw + pad;
 }
 
 // Bulk (non-tensor) copy global -> this CTA's shared memory, completing on `bar`.

@@ -75,19 +75,21 @@ __device__ __forceinline__ float e4m3_head_scale(float amax) {
 // Scoring-head query fragments and weights in shared memory.
 //   bfrag [KT][TERMS][NT][32] uint2, w_s [NT*8] (head weight / query scale),
 //   scale_s [NT*8] scratch.
-// heads == nullptr: all H heads; slots >= h_eff are zero.  Threads
-// [0, NTHR) must all call; `sync` is a barrier over exactly those threads, and
-// one more is needed before the fragments are read.  Loops have fixed trip
-// counts so every load is issued before it is used.
+// heads == nullptr: all H heads; slots >= h_eff are zero.  sheads != nullptr:
+// the h heads of this query in shared memory (heads is then ignored).
+// Threads [0, NTHR) must all call; `sync` is a barrier over exactly those
+// threads, and one more is needed before the fragments are read.  Loops have
+// fixed trip counts so every load is issued before it is used.
 template <int NT, bool FP8, int NTHR, class Sync>
 __device__ __forceinline__ void build_query_frags(const CacheView &c, const QueryView &qv, int i,
                                                   const int32_t *heads, int h, uint2 *bfrag, float *w_s,
-                                                  float *scale_s, int tid, Sync sync) {
+                                                  float *scale_s, int tid, Sync sync,
+                                                  const int32_t *sheads = nullptr) {
   using F = FragCfg<FP8>;
   const int H = qv.H;
-  const int h_eff = heads ? h : H;
+  const int h_eff = (heads || sheads) ? h : H;
   auto head_of = [&](int n) -> int {
-    int j = heads ? __ldg(heads + (size_t)i * h + n) : n;
+    int j = sheads ? sheads[n] : heads ? __ldg(heads + (size_t)i * h + n) : n;
     if (j < 0 || j >= H) {
       flag(c, MISA_DEV_BAD_HEAD);
       j = 0;

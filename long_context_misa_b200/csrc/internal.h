@@ -15,8 +15,10 @@ constexpr int TOPK_HIST_BINS = 2048;
 
 // pool.cu
 cudaError_t launch_pool_rebuild(const CacheView &c, cudaStream_t s);
+// zero != nullptr: the kernel also sets zero[0..zero_n) to 0
 cudaError_t launch_pool_append(const CacheView &c, const void *new_keys, const float *new_scale,
-                               const int32_t *new_pos, int count, cudaStream_t s);
+                               const int32_t *new_pos, int count, cudaStream_t s, uint32_t *zero = nullptr,
+                               size_t zero_n = 0);
 // e4m3 caches: bf16 keys quantised (one scale per token) while appended;
 // count <= pool_append_quant_max()
 int pool_append_quant_max();
@@ -39,6 +41,26 @@ size_t route_umma_ws_bytes(int n_q, int H, int M_cap, int n_seq);
 cudaError_t launch_route_umma(const CacheView &c, const QueryView &q, int h, int32_t *heads, float *router_scores,
                               void *ws, cudaStream_t s, int agg = 0);
 
+// Selection inside the scoring kernel (rowsel.cuh): the CTAs that scored a
+// row select its top k from their on-chip scores, meeting at counters in
+// global memory.  Applies to decode rows on the streaming scorer and to
+// re-rank rows, when the launch's CTAs are all resident at once.
+constexpr int FUSED_CTR = 8;                                 // counters per row
+constexpr int FUSED_ZERO_WORDS = 2 * TOPK_HIST_BINS + FUSED_CTR;  // zeroed per row before the launch
+constexpr int FUSED_BCAP = 2048;                             // boundary-bucket entries per row
+struct FusedTopk {
+  uint32_t *zeroed;   // [n_q][FUSED_ZERO_WORDS], zero before the launch
+  uint2 *bucket;      // [n_q][FUSED_BCAP]
+  int32_t *winners;   // [n_q][k] scratch of an ascending output (ordered only)
+  int32_t *out;       // [n_q][k] the selected tokens
+  int k;
+  int ordered;        // 1: ascending token order; 0: any order
+};
+// Whether launch_score_mma can select in the scoring kernel for these shapes
+// (fused != nullptr there); otherwise the caller runs launch_topk.
+bool score_fusable(const CacheView &c, const QueryView &q, const int32_t *heads, int h, const int32_t *gather,
+                   int n_cols);
+
 // score_dispatch.cu: scores[i][t] (row stride ld) for t < L_i, heads given per query
 // (heads == nullptr: all H heads, dense).  `gather` != nullptr: row i scores the
 // tokens gather[i][0..n_cols) instead of the prefix (re-rank).
@@ -46,7 +68,7 @@ cudaError_t launch_route_umma(const CacheView &c, const QueryView &q, int h, int
 // caller zeroes row_hist, [n_q][TOPK_HIST_BINS] uint32, beforehand).
 cudaError_t launch_score_mma(const CacheView &c, const QueryView &q, const int32_t *heads, int h,
                              const int32_t *gather, int n_cols, float *scores, long long ld, uint32_t *row_hist,
-                             cudaStream_t s);
+                             cudaStream_t s, const FusedTopk *fused = nullptr);
 
 // rerank_umma.cu: the gathered (re-rank) case of launch_score_mma on tcgen05
 // tensor cores, for up to 128 scoring heads, and (gather == nullptr, n_cols =
@@ -56,12 +78,22 @@ cudaError_t launch_score_mma(const CacheView &c, const QueryView &q, const int32
 bool rerank_umma_applies(const QueryView &q, const int32_t *heads, int h);
 cudaError_t launch_rerank_umma(const CacheView &c, const QueryView &q, const int32_t *heads, int h,
                                const int32_t *gather, int n_cols, float *scores, long long ld, uint32_t *row_hist,
-                               cudaStream_t s);
+                               cudaStream_t s, const FusedTopk *fused = nullptr);
+bool rerank_fusable(const CacheView &c, const QueryView &q, const int32_t *heads, int h, int n_cols);
+// the same for prefix rows of e4m3 caches with 32 or more scoring heads
+bool dense_fusable(const CacheView &c, const QueryView &q, const int32_t *heads, int h);
 
 // score_stream.cu: prefix scoring through the bulk-copy pipeline (used by
 // launch_score_mma when gather == nullptr).
+// route_part != nullptr (with fused): the h scoring heads are routed inside
+// the kernel first (heads ignored), with route_part_slots() x H floats of
+// partial sums at route_part; heads_out ([n_q][h]) receives them if not null.
 cudaError_t launch_score_stream(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
-                                long long ld, uint32_t *row_hist, cudaStream_t s);
+                                long long ld, uint32_t *row_hist, cudaStream_t s, const FusedTopk *fused = nullptr,
+                                float *route_part = nullptr, int32_t *heads_out = nullptr);
+bool score_stream_fusable(const CacheView &c, const QueryView &q, const int32_t *heads, int h, bool route = false);
+// CTA slots (queries x CTAs per query) of the in-kernel router's partial sums
+inline int route_part_slots() { return 8 * device_sms(); }
 
 // score_umma.cu: prefix scoring of query batches with many queries per
 // sequence (prefill chunks) on tcgen05 tensor cores; writes no histogram.

@@ -41,10 +41,15 @@ __global__ void __launch_bounds__(REBUILD_THREADS) pool_rebuild_kernel(CacheView
   c.pool[((size_t)s * M_cap + m) * D + threadIdx.x] = sm_out[threadIdx.x] / (float)(t1 - t0);
 }
 
+// zero / zero_n: words the next kernels count into, cleared here too (so that
+// a decode step needs no separate zeroing launch).
 __global__ void __launch_bounds__(APPEND_THREADS) pool_append_kernel(CacheView c, const void *new_keys,
                                                                      const float *new_scale,
-                                                                     const int32_t *new_pos, int count) {
+                                                                     const int32_t *new_pos, int count,
+                                                                     uint32_t *zero, size_t zero_n) {
   grid_dep_sync();
+  for (size_t x = (size_t)blockIdx.x * APPEND_THREADS + threadIdx.x; x < zero_n; x += (size_t)gridDim.x * APPEND_THREADS)
+    zero[x] = 0u;
   __shared__ float sm_part[(APPEND_THREADS / 8) * D];
   __shared__ float sm_out[D];
   const int s = blockIdx.x;
@@ -148,8 +153,9 @@ cudaError_t launch_pool_rebuild(const CacheView &c, cudaStream_t s) {
 }
 
 cudaError_t launch_pool_append(const CacheView &c, const void *new_keys, const float *new_scale,
-                               const int32_t *new_pos, int count, cudaStream_t s) {
-  return launch_kernel(pool_append_kernel, dim3(c.n_seq), dim3(APPEND_THREADS), 0, s, c, new_keys, new_scale, new_pos, count);
+                               const int32_t *new_pos, int count, cudaStream_t s, uint32_t *zero, size_t zero_n) {
+  return launch_kernel(pool_append_kernel, dim3(c.n_seq), dim3(APPEND_THREADS), 0, s, c, new_keys, new_scale, new_pos,
+                       count, zero, zero_n);
 }
 
 }  // namespace misa

@@ -32,6 +32,7 @@
 
 #include "frag.cuh"
 #include "internal.h"
+#include "rowsel.cuh"
 #include "umma.cuh"
 
 namespace misa {
@@ -123,16 +124,23 @@ __device__ __forceinline__ void build_qprime(const CacheView &c, const QueryView
   }
 }
 
+// fz.zeroed != nullptr: the row's top fz.k are selected here (rowsel.cuh),
+// with each thread's scores kept in registers, instead of the histogram going
+// to row_hist.
 template <bool FP8, int HN, int TT>
 __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, QueryView qv, const int32_t *heads,
                                                                   int h, const int32_t *gather, int n_cols,
                                                                   float *scores, long long ld,
-                                                                  uint32_t *row_hist) {
+                                                                  uint32_t *row_hist, FusedTopk fz) {
   grid_dep_sync();
   using Cfg = RCfg<FP8, HN, TT>;
   constexpr int T = Cfg::T;
   extern __shared__ uint8_t rr_raw[];
-  uint8_t *base = rr_raw + ((1024u - (smem_addr(rr_raw) & 1023u)) & 1023u);  // 1024-aligned (swizzle atoms)
+  // the tiles and Q', or (a fused selection, afterwards) its state and scratch
+  const uint32_t sel_bytes = (uint32_t)((sizeof(RsShared<RR_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap);
+  const uint32_t need = max((uint32_t)(Cfg::SMEM - 1024), fz.zeroed ? sel_bytes : 0u);
+  uint8_t *base = aligned_smem_base(rr_raw, need, c);  // 1024-aligned (swizzle atoms)
+  if (!base) return;
   uint8_t *a_smem = base;                       // T x A_BYTES
   uint8_t *b_smem = base + T * Cfg::A_BYTES;    // B_BYTES
   __shared__ RerankShared sh;
@@ -221,10 +229,15 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
   // 5. epilogue: candidate row r = 32 * warp + lane of every tile
   const bool got = umma::wait_bar(&sh.done, 0, abort, c);
   umma::fence_after();
+  float kept[T];  // fused selection: this thread's scores
+#pragma unroll
+  for (int j = 0; j < T; ++j) kept[j] = 0.f;
   if (got) {
     const int r = warp * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    for (int j = 0; j < ntile; ++j) {
+#pragma unroll
+    for (int j = 0; j < T; ++j) {
+      if (j >= ntile) break;
       float acc = 0.f;
       const float4 *w4 = reinterpret_cast<const float4 *>(sh.w);
 #pragma unroll
@@ -246,6 +259,7 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
       if (t >= 0) {
         const float val = FP8 ? acc * sh.scale[e] : acc;
         scores[(size_t)i * ld + col0 + e] = val;
+        kept[j] = val;
         atomicAdd(&sh.hist[ordered_key(val) >> 21], 1u);
       }
     }
@@ -258,6 +272,47 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
     umma::fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(Cfg::TMEM_COLS));
   }
+  if (fz.zeroed) {
+    // the tensor memory is released before any wait on the row's other CTAs
+    // (one of them may still be waiting to allocate); a CTA whose MMAs gave
+    // up never arrives, and the row's waits run out
+    if (!got) return;
+    // the key tiles are free: the selection's shared state and scratch go there
+    RsShared<RR_THREADS> &rs = *reinterpret_cast<RsShared<RR_THREADS> *>(a_smem);
+    uint8_t *scratch = a_smem + (sizeof(RsShared<RR_THREADS>) + 15) / 16 * 16;
+    const int r = warp * 32 + lane;
+    auto each = [&](auto &&fn) {
+#pragma unroll
+      for (int j = 0; j < T; ++j) {
+        const int t = sh.tok[j * RR_M + r];
+        const bool valid = j < ntile && t >= 0;
+        fn(valid ? ordered_key(kept[j]) : 0u, t, valid);
+      }
+    };
+    const float *srow = scores + (size_t)i * ld;
+    const int32_t *grow = gather + (size_t)i * n_cols;
+    auto sweep = [&](auto &&fn) {
+      constexpr int SU = 8;
+      for (int base = 0; base < n_cols; base += RR_THREADS * SU) {
+        int tk[SU];
+        float v[SU];
+#pragma unroll
+        for (int u = 0; u < SU; ++u) {
+          const int p = base + u * RR_THREADS + tid;
+          tk[u] = p < n_cols ? __ldg(grow + p) : -1;
+          v[u] = (tk[u] >= 0 && tk[u] < Li) ? __ldcg(srow + p) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < SU; ++u) {
+          const bool ok = tk[u] >= 0 && tk[u] < Li;
+          fn(ordered_key(v[u]), POS_MAX - (uint32_t)(ok ? tk[u] : 0), ok);
+        }
+      }
+    };
+    row_select<RR_THREADS>(c, rs, sh.hist, scratch, rs_row(fz, i), gridDim.x, fz.k, Li, fz.ordered != 0, each,
+                           sweep);
+    return;
+  }
   if (got) {
     uint32_t *rh = row_hist + (size_t)i * TOPK_HIST_BINS;
     for (int b = tid; b < TOPK_HIST_BINS; b += RR_THREADS) {
@@ -267,164 +322,169 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
   }
 }
 
-// ---- dense prefix scoring (gather == nullptr) ------------------------------
-// A query's whole prefix against all its scoring heads, the same dense
-// product over contiguous tokens.  Persistent: a CTA builds Q' once, then
-// walks chunks part, part + nparts, ... of its query's prefix (DT tiles of
-// 128 tokens each), with chunks j + 1 .. j + NBUF - 1's key rows and scales
-// in flight (coalesced 16-byte cp.async into a ring of NBUF shared-memory
-// buffers) while chunk j is multiplied and drained; the grid holds the
-// resident CTAs (two per SM for e4m3 keys).  Measured for 8 x 128K
-// e4m3 keys and 64 heads: 45 us with two-tile chunks and two buffers, 63 us
-// with one-tile chunks and three buffers (three CTAs per SM: the per-chunk
-// barriers and MMA round trip weigh more).  One mbarrier
-// phase per chunk; every wait is bounded, and after each wait the CTA agrees
-// through a barrier whether to go on, so that a wait that ran out ends every
-// thread's loop at the same chunk.
-template <bool FP8, int HN>
-struct DCfg {
-  static constexpr int ROW = FP8 ? 128 : 256;
-  static constexpr int CH = ROW / 16;                    // 16-byte chunks per key row
-  static constexpr int DT = HN >= 128 ? 1 : 2;           // tiles per chunk
-  static constexpr int NBUF = 2;                         // chunks staged (the current one + 1 ahead)
-  static constexpr int CT = DT * RR_M;                   // tokens per chunk
-  static constexpr int A_BYTES = RR_M * ROW;             // one tile of key rows
-  static constexpr int CHUNK_BYTES = DT * A_BYTES;
-  static constexpr int B_BYTES = HN * 256;
-  static constexpr int TMEM_COLS = DT * HN < 32 ? 32 : DT * HN;
-  static constexpr int SMEM = 1024 + NBUF * CHUNK_BYTES + B_BYTES;
-  static_assert(DT * HN <= 256, "tensor-memory columns per CTA");
+// ---- dense prefix scoring of e4m3 caches (gather == nullptr) --------------
+// A query's whole prefix against all its scoring heads: per 128-token tile
+// the dense product D[t][n] = K[t] . Q'[n] (M = 128 tokens, N = HN columns,
+// kind::f8f6f4 on the keys as stored against the two-term e4m3 split of the
+// query).  Persistent and warp-specialised: CTA `part` of a query walks the
+// tiles part, part + nparts, ... of its prefix (one CTA per SM over all
+// queries, so the CTAs read neighbouring tiles at the same time).
+//   warp 0     TMA producer: 128-byte-swizzled key tiles (16 KB) into a ring
+//              of DS_STAGES shared-memory stages;
+//   warp 1     owns the tensor memory; one thread issues each tile's MMAs into
+//              one of two accumulator buffers and commits the stage back to
+//              the producer and the buffer to the epilogue;
+//   warps 2-5  one tensor-memory lane quarter each, one token row per thread:
+//              ReLU, the weights, the head sum and the e4m3 token scale
+//              (loaded one tile ahead), the score written and counted.
+// The two accumulator buffers let tile j + 1's MMAs run while tile j is
+// drained, and the ring keeps DS_STAGES tiles of keys in flight per SM.
+// With a fused selection every score also stays in shared memory and the
+// query's CTAs select its top k afterwards (rowsel.cuh).  Every wait is
+// bounded: one that runs out sets MISA_DEV_WAIT_TIMEOUT and the CTA winds
+// down without selecting.
+constexpr int DS_STAGES = 8;
+constexpr int DS_EPI = 4;
+constexpr int DS_THREADS = 64 + 32 * DS_EPI;
+
+template <int HN>
+struct DSCfg {
+  static constexpr int A_BYTES = RR_M * 128;  // one e4m3 key tile
+  static constexpr int B_BYTES = HN * 256;    // Q': two e4m3 terms
+  static constexpr int TMEM_COLS = 2 * HN;    // two accumulator buffers
+  static constexpr int RING = DS_STAGES * A_BYTES + B_BYTES;  // from the 1024-byte-aligned base
+  static_assert(TMEM_COLS >= 32 && TMEM_COLS <= 512, "tensor-memory columns");
 };
 
-struct DenseShared {
-  uint64_t done;
+struct DsShared {
+  uint64_t full[DS_STAGES], empty[DS_STAGES];  // key stages: loaded / consumed
+  uint64_t tfull[2], tempty[2];                // accumulators: written / drained
   uint32_t tmem_base;
   int abort;
-  alignas(16) float w[128];        // weight per column (0: padding); read as float4
-  float scale[2 * 2 * RR_M];       // the chunks' e4m3 token scales, CT per buffer
-  uint32_t hist[TOPK_HIST_BINS];   // this CTA's share of the row histogram
+  alignas(16) float w[128];                    // weight per column (0: padding)
+  uint32_t hist[TOPK_HIST_BINS];               // this CTA's share of the row histogram
 };
 
-template <bool FP8, int HN>
-__global__ void __launch_bounds__(RR_THREADS) dense_umma_kernel(CacheView c, QueryView qv, const int32_t *heads, int h,
-                                                                 float *scores, long long ld, uint32_t *row_hist,
-                                                                 int nparts) {
+// Dynamic shared memory of a dense launch: alignment slack, the ring and Q',
+// then (fused) the scores of max_tiles tiles.
+template <int HN>
+__host__ __device__ int dense_smem(int max_tiles, bool fused) {
+  return 1024 + DSCfg<HN>::RING + (fused ? max_tiles * RR_M * 4 : 0);
+}
+
+template <int HN>
+__global__ void __launch_bounds__(DS_THREADS, 1)
+    dense_umma_kernel(const __grid_constant__ CUtensorMap kmap, CacheView c, QueryView qv, const int32_t *heads, int h,
+                      float *scores, long long ld, uint32_t *row_hist, int nparts, FusedTopk fz, int max_tiles) {
   grid_dep_sync();
-  using Cfg = DCfg<FP8, HN>;
-  extern __shared__ uint8_t dn_raw[];
-  uint8_t *base = dn_raw + ((1024u - (smem_addr(dn_raw) & 1023u)) & 1023u);  // 1024-aligned (swizzle atoms)
-  static_assert(Cfg::NBUF * Cfg::CT <= 2 * 2 * RR_M, "the scale ring");
-  uint8_t *a_smem = base;                             // NBUF x CHUNK_BYTES
-  uint8_t *b_smem = base + Cfg::NBUF * Cfg::CHUNK_BYTES;  // B_BYTES
-  __shared__ DenseShared sh;
+  using Cfg = DSCfg<HN>;
+  extern __shared__ uint8_t ds_raw[];
+  const bool fused = fz.zeroed != nullptr;
+  uint8_t *base = aligned_smem_base(ds_raw, dense_smem<HN>(max_tiles, fused) - 1024, c);  // 1024-aligned
+  if (!base) return;
+  uint8_t *a_smem = base;                             // DS_STAGES x A_BYTES
+  uint8_t *b_smem = base + DS_STAGES * Cfg::A_BYTES;  // B_BYTES
+  float *sc_s = reinterpret_cast<float *>(base + Cfg::RING);  // fused: [max_tiles][128]
+  __shared__ DsShared sh;
   volatile int *abort = &sh.abort;
   const int i = blockIdx.y, part = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int s;
   const int Li = query_prefix(c, qv, i, &s);
-  const int n_chunks = cdiv(max(Li, 0), Cfg::CT);
-  const int n_my = part < n_chunks ? cdiv(n_chunks - part, nparts) : 0;
-  if (n_my == 0) return;  // uniform: nothing allocated yet
-  const uint8_t *kbase = static_cast<const uint8_t *>(c.keys) + (size_t)s * c.L_cap * Cfg::ROW;
-  const float *sbase = FP8 ? c.scale + (size_t)s * c.L_cap : nullptr;
+  const int n_tiles = cdiv(max(Li, 0), RR_M);
+  const int n_my = part < n_tiles ? cdiv(n_tiles - part, nparts) : 0;
+  // a CTA without tiles leaves at once, unless the row's selection needs it
+  if (n_my == 0 && !fused) return;  // uniform; nothing initialised yet
 
-  // chunk j's key rows (zero-filled past the prefix) and scales into buffer
-  // j % NBUF: consecutive threads take consecutive 16-byte pieces of the
-  // chunk's contiguous rows.  Always one commit group per call.
-  auto issue = [&](int j) {
-    if (j < n_my) {
-      const int t0 = (part + j * nparts) * Cfg::CT;
-      uint8_t *a = a_smem + (j % Cfg::NBUF) * Cfg::CHUNK_BYTES;
-      for (int x = tid; x < Cfg::CT * Cfg::CH; x += RR_THREADS) {
-        const int rr = x / Cfg::CH, u = x % Cfg::CH;
-        const int tile = rr / RR_M, r = rr % RR_M, t = t0 + rr;
-        const uint32_t dst =
-            smem_addr(a + tile * Cfg::A_BYTES + (u >> 3) * (RR_M * 128) + r * 128 + (((u & 7) ^ (r & 7)) << 4));
-        cp_async16(dst, kbase + (size_t)min(t, Li - 1) * Cfg::ROW + 16 * u, t < Li);
-      }
-      if (FP8)
-        for (int e = tid; e < Cfg::CT; e += RR_THREADS) {
-          const int t = t0 + e;
-          cp_async4(smem_addr(&sh.scale[(j % Cfg::NBUF) * Cfg::CT + e]), sbase + min(t, Li - 1), t < Li);
-        }
-    }
-    cp_async_commit();
-  };
-
-#pragma unroll
-  for (int j = 0; j < Cfg::NBUF - 1; ++j) issue(j);
-  build_qprime<FP8, HN>(c, qv, heads, h, i, b_smem, sh.w);
-  for (int b = tid; b < TOPK_HIST_BINS; b += RR_THREADS) sh.hist[b] = 0;
   if (tid == 0) {
-    mbar_init(&sh.done, 1);
+    for (int st = 0; st < DS_STAGES; ++st) {
+      mbar_init(&sh.full[st], 1);
+      mbar_init(&sh.empty[st], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sh.tfull[b], 1);
+      mbar_init(&sh.tempty[b], DS_EPI);
+    }
     sh.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
+  for (int b = tid; b < TOPK_HIST_BINS; b += DS_THREADS) sh.hist[b] = 0;
+  if (tid < RR_THREADS) build_qprime<true, HN>(c, qv, heads, h, i, b_smem, sh.w);
+  if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&sh.tmem_base)),
                  "n"(Cfg::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // Q' visible to the tensor cores
   umma::fence_before();
   __syncthreads();
   umma::fence_after();
   const uint32_t tmem = sh.tmem_base;
-  const uint32_t idesc = umma::instr_desc<FP8, RR_M, HN>();
-  uint32_t committed = 0, waited = 0;  // thread 0: chunks whose MMAs it committed / saw complete
+  uint32_t last_fill = 0;   // producer: tiles whose load it issued
+  uint32_t committed = 0;   // MMA thread: tiles whose MMAs it committed
 
-  for (int j = 0; j < n_my; ++j) {
-    issue(j + Cfg::NBUF - 1);                                       // into chunk j - 1's buffer
-    cp_async_wait<Cfg::NBUF - 1>();                                 // chunk j: this thread's copies landed
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // ... and Q': visible to the tensor cores
-    umma::fence_before();
-    __syncthreads();
-    umma::fence_after();
-    const int t0 = (part + j * nparts) * Cfg::CT;
-    const int ntile = min(Cfg::DT, cdiv(Li - t0, RR_M));
-    // this thread's token scales of the chunk, read before the barrier after
-    // which a thread may refill this buffer with chunk j + NBUF
-    const int r = warp * 32 + lane;
-    float scl[Cfg::DT];
-#pragma unroll
-    for (int tt = 0; tt < Cfg::DT; ++tt) scl[tt] = FP8 ? sh.scale[(j % Cfg::NBUF) * Cfg::CT + tt * RR_M + r] : 1.f;
-    if (tid == 0) {
-      const uint32_t a0 = smem_addr(a_smem + (j % Cfg::NBUF) * Cfg::CHUNK_BYTES), b_base = smem_addr(b_smem);
-      for (int tt = 0; tt < ntile; ++tt) {
-#pragma unroll
-        for (int term = 0; term < (FP8 ? 2 : 1); ++term) {
-#pragma unroll
-          for (int kk = 0; kk < (FP8 ? 4 : 8); ++kk) {
-            uint32_t aoff, boff;
-            if (FP8) {
-              aoff = kk * 32;
-              boff = term * (HN * 128) + kk * 32;
-            } else {
-              aoff = (kk >> 2) * (RR_M * 128) + (kk & 3) * 32;
-              boff = (kk >> 2) * (HN * 128) + (kk & 3) * 32;
-            }
-            umma::mma<FP8>(tmem + tt * HN, umma::smem_desc_sw128(a0 + tt * Cfg::A_BYTES + aoff),
-                           umma::smem_desc_sw128(b_base + boff), idesc, (term | kk) ? 1u : 0u);
-          }
-        }
+  if (warp == 0) {
+    // ---- TMA producer ----
+    if (lane == 0) {
+      for (int j = 0; j < n_my; ++j) {
+        const int st = j % DS_STAGES;
+        if (!umma::wait_bar(&sh.empty[st], ((j / DS_STAGES) & 1) ^ 1, abort, c)) break;
+        mbar_arrive_expect_tx(&sh.full[st], Cfg::A_BYTES);
+        const int t0 = (part + j * nparts) * RR_M;
+        umma::tma_load_2d(smem_addr(a_smem + st * Cfg::A_BYTES), &kmap, 0, s * c.L_cap + t0, &sh.full[st]);
+        last_fill = j + 1;
       }
-      umma::commit(&sh.done);
-      ++committed;
     }
-    if (umma::wait_bar(&sh.done, (uint32_t)(j & 1), abort, c) && tid == 0) ++waited;
-    __syncthreads();  // one view of *abort in every thread
-    if (*abort) break;
-    umma::fence_after();
-    // epilogue: row r = 32 * warp + lane of every tile of the chunk
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    const float4 *w4 = reinterpret_cast<const float4 *>(sh.w);
+  } else if (warp == 1) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      const uint32_t idesc = umma::instr_desc<true, RR_M, HN>();
+      const uint32_t b_base = smem_addr(b_smem);
+      for (int j = 0; j < n_my; ++j) {
+        const int st = j % DS_STAGES, buf = j & 1;
+        if (!umma::wait_bar(&sh.tempty[buf], ((j >> 1) & 1) ^ 1, abort, c)) break;
+        umma::fence_after();
+        if (!umma::wait_bar(&sh.full[st], (j / DS_STAGES) & 1, abort, c)) break;
+        umma::fence_after();
+        const uint32_t a_base = smem_addr(a_smem + st * Cfg::A_BYTES);
 #pragma unroll
-    for (int tt = 0; tt < Cfg::DT; ++tt) {
-      if (tt >= ntile) break;
+        for (int term = 0; term < 2; ++term)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma::mma<true>(tmem + buf * HN, umma::smem_desc_sw128(a_base + kk * 32),
+                            umma::smem_desc_sw128(b_base + term * (HN * 128) + kk * 32), idesc, (term | kk) ? 1u : 0u);
+        umma::commit(&sh.empty[st]);
+        umma::commit(&sh.tfull[buf]);
+        committed = j + 1;
+      }
+    }
+  } else {
+    // ---- epilogue: token row r of every tile ----
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const float4 *w4 = reinterpret_cast<const float4 *>(sh.w);
+    const float *srow_scale = c.scale + (size_t)s * c.L_cap;
+    float sc_next = 0.f;
+    if (n_my > 0) {
+      const int t = part * RR_M + r;
+      sc_next = t < Li ? __ldg(srow_scale + t) : 0.f;
+    }
+    for (int j = 0; j < n_my; ++j) {
+      const int buf = j & 1;
+      const int t = (part + j * nparts) * RR_M + r;
+      const float scl = sc_next;
+      if (j + 1 < n_my) {
+        const int tn = t + nparts * RR_M;
+        sc_next = tn < Li ? __ldg(srow_scale + tn) : 0.f;
+      }
+      if (!umma::wait_bar(&sh.tfull[buf], (j >> 1) & 1, abort, c)) break;
+      umma::fence_after();
       float acc = 0.f;
 #pragma unroll
       for (int cb = 0; cb < HN; cb += 32) {
         uint32_t v[32];
-        umma::ld32(tl + tt * HN + cb, v);
+        umma::ld32(tl + buf * HN + cb, v);
         umma::ld_wait();
 #pragma unroll
         for (int x = 0; x < 32; x += 4) {
@@ -435,80 +495,168 @@ __global__ void __launch_bounds__(RR_THREADS) dense_umma_kernel(CacheView c, Que
           acc = fmaf(w.w, fmaxf(__uint_as_float(v[x + 3]), 0.f), acc);
         }
       }
-      const int e = tt * RR_M + r, t = t0 + e;
+      umma::fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.tempty[buf]);
       if (t < Li) {
-        const float val = acc * scl[tt];
+        const float val = acc * scl;
         scores[(size_t)i * ld + t] = val;
+        if (fused) sc_s[j * RR_M + r] = val;
         atomicAdd(&sh.hist[ordered_key(val) >> 21], 1u);
       }
     }
   }
 
-  // wind-down: no copy and no MMA in flight when the memory is released
-  cp_async_wait<0>();
-  if (tid == 0 && committed > waited) mbar_wait(&sh.done, (committed - 1) & 1);  // bounded
+  // ---- wind-down: no load and no MMA in flight when the memory is released ----
+  __syncthreads();
+  if (warp == 0 && lane == 0 && *abort) {
+    // a role gave up: the last fill of each stage may still be landing (a
+    // completed one passes at once)
+    for (uint32_t j = (last_fill > DS_STAGES ? last_fill - DS_STAGES : 0); j < last_fill; ++j)
+      mbar_wait(&sh.full[j % DS_STAGES], (j / DS_STAGES) & 1);  // bounded
+  }
+  if (warp == 1 && lane == 0 && committed > 0) {
+    const uint32_t jl = committed - 1;  // the last committed accumulator buffer
+    mbar_wait(&sh.tfull[jl & 1], (jl >> 1) & 1);  // bounded
+  }
   umma::fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     umma::fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(Cfg::TMEM_COLS));
   }
-  if (!*abort) {
-    uint32_t *rh = row_hist + (size_t)i * TOPK_HIST_BINS;
-    for (int b = tid; b < TOPK_HIST_BINS; b += RR_THREADS) {
-      const uint32_t v = sh.hist[b];
-      if (v) atomicAdd(rh + b, v);
-    }
+  if (*abort) return;  // uniform (read after the barrier)
+  if (fused) {
+    // the ring is free: the selection's shared state and scratch go there
+    RsShared<DS_THREADS> &rs = *reinterpret_cast<RsShared<DS_THREADS> *>(a_smem);
+    uint8_t *scratch = a_smem + (sizeof(RsShared<DS_THREADS>) + 15) / 16 * 16;
+    const int total = max_tiles * RR_M;
+    auto each = [&](auto &&fn) {
+      for (int x = tid; x < (total + DS_THREADS - 1) / DS_THREADS * DS_THREADS; x += DS_THREADS) {
+        const int j = x / RR_M, rr = x % RR_M;
+        const int tok = (part + j * nparts) * RR_M + rr;
+        const bool valid = x < total && j < n_my && tok < Li;
+        fn(valid ? ordered_key(sc_s[x]) : 0u, tok, valid);
+      }
+    };
+    const float *srow = scores + (size_t)i * ld;
+    auto sweep = [&](auto &&fn) {
+      constexpr int SU = 8;
+      for (int b0 = 0; b0 < Li; b0 += DS_THREADS * SU) {
+        float v[SU];
+#pragma unroll
+        for (int u = 0; u < SU; ++u) {
+          const int p = b0 + u * DS_THREADS + tid;
+          v[u] = p < Li ? __ldcg(srow + p) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < SU; ++u) {
+          const int p = b0 + u * DS_THREADS + tid;
+          fn(ordered_key(v[u]), POS_MAX - (uint32_t)p, p < Li);
+        }
+      }
+    };
+    row_select<DS_THREADS>(c, rs, sh.hist, scratch, rs_row(fz, i), nparts, fz.k, Li, fz.ordered != 0, each, sweep);
+    return;
+  }
+  uint32_t *rh = row_hist + (size_t)i * TOPK_HIST_BINS;
+  for (int b = tid; b < TOPK_HIST_BINS; b += DS_THREADS) {
+    const uint32_t v = sh.hist[b];
+    if (v) atomicAdd(rh + b, v);
   }
 }
 
-template <bool FP8, int HN>
-cudaError_t launch_dense(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
-                         long long ld, uint32_t *row_hist, cudaStream_t s) {
-  using Cfg = DCfg<FP8, HN>;
+// Launch shape of a dense e4m3 call: one CTA per SM over all queries.
+struct DensePlan {
+  int nparts = 0, max_tiles = 0, smem = 0;
+  bool ok = false;
+};
+
+template <int HN>
+DensePlan plan_dense(const CacheView &c, const QueryView &q, bool fused) {
+  DensePlan p;
   struct Tag {};
-  const int st = cached_per_device<Tag>([] {
-    cudaError_t e = cudaFuncSetAttribute(dense_umma_kernel<FP8, HN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg::SMEM);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(dense_umma_kernel<FP8, HN>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                               (int)cudaSharedmemCarveoutMaxShared);
-    return 1 + (int)e;
-  });
-  if (st != 1) return (cudaError_t)(st - 1);
-  // the resident CTAs over all rows, each walking several chunks: two per SM
-  // when two fit in the SM's 228 KB of shared memory (e4m3 keys: at most
-  // 94 KB each at every head count), else one.  (The runtime's occupancy
-  // query answered one per SM for e4m3 at 64 heads, and a grid sized from it
-  // took 54 us instead of 45.)
-  constexpr int per_sm = 2 * (Cfg::SMEM + (int)sizeof(DenseShared) + 1024) <= 228 * 1024 ? 2 : 1;
-  const int nparts = std::max(1, std::min(cdiv(c.L_cap, Cfg::CT), per_sm * device_sms() / q.n_q));
-  return launch_kernel(dense_umma_kernel<FP8, HN>, dim3(nparts, q.n_q), dim3(RR_THREADS), Cfg::SMEM, s, c, q, heads,
-                       h, scores, ld, row_hist, nparts);
+  const int max_dyn = cached_per_device<Tag>([] { return opt_in_max_dyn_smem(dense_umma_kernel<HN>); });
+  const int sms = device_sms();
+  const int n_tiles = cdiv(c.L_cap, RR_M);
+  p.nparts = std::max(1, std::min(n_tiles, sms / std::max(q.n_q, 1)));
+  p.max_tiles = cdiv(n_tiles, p.nparts);
+  p.smem = dense_smem<HN>(p.max_tiles, fused);
+  p.ok = p.smem <= max_dyn && (!fused || (long long)p.nparts * q.n_q <= sms) && c.fp8 && umma::encoder_available() &&
+         (reinterpret_cast<uintptr_t>(c.keys) & 15u) == 0;
+  return p;
+}
+
+template <int HN>
+cudaError_t launch_dense(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
+                         long long ld, uint32_t *row_hist, cudaStream_t s, const FusedTopk *fz) {
+  const DensePlan p = plan_dense<HN>(c, q, fz != nullptr);
+  if (!p.ok) return cudaErrorInvalidConfiguration;
+  CUtensorMap map;
+  if (!umma::make_map_2d(&map, c.keys, true, (unsigned long long)c.n_seq * c.L_cap, 128, RR_M))
+    return cudaErrorNotSupported;
+  FusedTopk none = {};
+  return launch_kernel(dense_umma_kernel<HN>, dim3(p.nparts, q.n_q), dim3(DS_THREADS), p.smem, s, map, c, q, heads,
+                       h, scores, ld, row_hist, p.nparts, fz ? *fz : none, p.max_tiles);
+}
+
+// Dynamic shared memory of a re-rank launch: the key tiles and Q', at least
+// the fused selection's state and scratch (which reuse the tiles' space).
+template <bool FP8, int HN, int TT>
+int rerank_smem(const CacheView &c, bool fused) {
+  using Cfg = RCfg<FP8, HN, TT>;
+  const int sel = 1024 + (int)((sizeof(RsShared<RR_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap);
+  return fused ? std::max(Cfg::SMEM, sel) : Cfg::SMEM;
+}
+
+// the kernel's dynamic shared-memory limit, raised once per device (-1: failed)
+template <bool FP8, int HN, int TT>
+int rerank_max_dyn() {
+  struct Tag {};
+  return cached_per_device<Tag>([] { return opt_in_max_dyn_smem(rerank_umma_kernel<FP8, HN, TT>); });
+}
+
+// A fused selection needs every CTA of the grid resident at once.
+template <bool FP8, int HN, int TT>
+bool rerank_fits(const CacheView &c, const QueryView &q, int n_cols) {
+  using Cfg = RCfg<FP8, HN, TT>;
+  const int smem = rerank_smem<FP8, HN, TT>(c, true);
+  if (smem > rerank_max_dyn<FP8, HN, TT>()) return false;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rerank_umma_kernel<FP8, HN, TT>, RR_THREADS, smem) !=
+      cudaSuccess)
+    return false;
+  const long long grid = (long long)cdiv(n_cols, Cfg::T * RR_M) * q.n_q;
+  return grid <= (long long)per_sm * device_sms();
 }
 
 template <bool FP8, int HN, int TT>
 cudaError_t launch_tt(const CacheView &c, const QueryView &q, const int32_t *heads, int h, const int32_t *gather,
-                      int n_cols, float *scores, long long ld, uint32_t *row_hist, cudaStream_t s) {
+                      int n_cols, float *scores, long long ld, uint32_t *row_hist, cudaStream_t s,
+                      const FusedTopk *fz) {
   using Cfg = RCfg<FP8, HN, TT>;
-  struct Tag {};
-  const int st = cached_per_device<Tag>([] {
-    return 1 + (int)cudaFuncSetAttribute(rerank_umma_kernel<FP8, HN, TT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-  });
-  if (st != 1) return (cudaError_t)(st - 1);
+  if (rerank_smem<FP8, HN, TT>(c, fz != nullptr) > rerank_max_dyn<FP8, HN, TT>()) return cudaErrorInvalidConfiguration;
+  if (fz && !rerank_fits<FP8, HN, TT>(c, q, n_cols)) return cudaErrorInvalidConfiguration;
   const dim3 grid(cdiv(n_cols, Cfg::T * RR_M), q.n_q);
-  return launch_kernel(rerank_umma_kernel<FP8, HN, TT>, grid, dim3(RR_THREADS), Cfg::SMEM, s, c, q, heads, h, gather,
-                       n_cols, scores, ld, row_hist);
+  FusedTopk none = {};
+  return launch_kernel(rerank_umma_kernel<FP8, HN, TT>, grid, dim3(RR_THREADS), rerank_smem<FP8, HN, TT>(c, fz != nullptr),
+                       s, c, q, heads, h, gather, n_cols, scores, ld, row_hist, fz ? *fz : none);
 }
 
 // Gathered candidates: 2 tiles per CTA (more CTAs shorten each gather chain);
 // a prefix row: the persistent dense kernel.
 template <bool FP8, int HN>
 cudaError_t launch_hn(const CacheView &c, const QueryView &q, const int32_t *heads, int h, const int32_t *gather,
-                      int n_cols, float *scores, long long ld, uint32_t *row_hist, cudaStream_t s) {
-  return gather ? launch_tt<FP8, HN, 2>(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s)
-                : launch_dense<FP8, HN>(c, q, heads, h, scores, ld, row_hist, s);
+                      int n_cols, float *scores, long long ld, uint32_t *row_hist, cudaStream_t s,
+                      const FusedTopk *fz) {
+  if (gather) return launch_tt<FP8, HN, 2>(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s, fz);
+  if (!FP8) return cudaErrorInvalidValue;  // dense decode of bf16 keys streams on mma.sync
+  return launch_dense<HN>(c, q, heads, h, scores, ld, row_hist, s, fz);
+}
+
+int rerank_hn(const QueryView &q, const int32_t *heads, int h) {
+  const int h_eff = heads ? h : q.H;
+  return h_eff <= 32 ? 32 : h_eff <= 64 ? 64 : 128;
 }
 
 }  // namespace
@@ -520,15 +668,13 @@ bool rerank_umma_applies(const QueryView &q, const int32_t *heads, int h) {
 
 cudaError_t launch_rerank_umma(const CacheView &c, const QueryView &q, const int32_t *heads, int h,
                                const int32_t *gather, int n_cols, float *scores, long long ld, uint32_t *row_hist,
-                               cudaStream_t s) {
+                               cudaStream_t s, const FusedTopk *fused) {
   if (q.n_q == 0 || n_cols == 0) return cudaSuccess;
-  const int h_eff = heads ? h : q.H;
-  const int hn = h_eff <= 32 ? 32 : h_eff <= 64 ? 64 : 128;
-#define MISA_RERANK_CASE(N)                                                                        \
-  case N:                                                                                          \
-    return c.fp8 ? launch_hn<true, N>(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s)     \
-                 : launch_hn<false, N>(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s);
-  switch (hn) {
+#define MISA_RERANK_CASE(N)                                                                           \
+  case N:                                                                                             \
+    return c.fp8 ? launch_hn<true, N>(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s, fused) \
+                 : launch_hn<false, N>(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s, fused);
+  switch (rerank_hn(q, heads, h)) {
     MISA_RERANK_CASE(32)
     MISA_RERANK_CASE(64)
     MISA_RERANK_CASE(128)
@@ -536,6 +682,34 @@ cudaError_t launch_rerank_umma(const CacheView &c, const QueryView &q, const int
       return cudaErrorInvalidValue;
   }
 #undef MISA_RERANK_CASE
+}
+
+bool dense_fusable(const CacheView &c, const QueryView &q, const int32_t *heads, int h) {
+  if (q.n_q == 0 || !c.fp8) return false;
+  switch (rerank_hn(q, heads, h)) {
+    case 32:
+      return plan_dense<32>(c, q, true).ok;
+    case 64:
+      return plan_dense<64>(c, q, true).ok;
+    case 128:
+      return plan_dense<128>(c, q, true).ok;
+    default:
+      return false;
+  }
+}
+
+bool rerank_fusable(const CacheView &c, const QueryView &q, const int32_t *heads, int h, int n_cols) {
+  if (q.n_q == 0 || n_cols == 0) return false;
+  switch (rerank_hn(q, heads, h)) {
+    case 32:
+      return c.fp8 ? rerank_fits<true, 32, 2>(c, q, n_cols) : rerank_fits<false, 32, 2>(c, q, n_cols);
+    case 64:
+      return c.fp8 ? rerank_fits<true, 64, 2>(c, q, n_cols) : rerank_fits<false, 64, 2>(c, q, n_cols);
+    case 128:
+      return c.fp8 ? rerank_fits<true, 128, 2>(c, q, n_cols) : rerank_fits<false, 128, 2>(c, q, n_cols);
+    default:
+      return false;
+  }
 }
 
 }  // namespace misa

@@ -84,7 +84,8 @@ __global__ void __launch_bounds__(RU_THREADS, 2)
                       int n_groups, int fuse, int h, int32_t *heads, float *router_scores, int agg) {
   grid_dep_sync();
   extern __shared__ uint8_t ru_raw[];
-  uint8_t *base = ru_raw + ((1024u - (smem_addr(ru_raw) & 1023u)) & 1023u);  // 1024-aligned (swizzle atoms)
+  uint8_t *base = aligned_smem_base(ru_raw, ru_smem_bytes() - 1024, c);  // 1024-aligned (swizzle atoms)
+  if (!base) return;
   uint8_t *a_smem = base;
   uint8_t *b_smem = base + RU_A_BYTES;
   RouteShared &sh = *reinterpret_cast<RouteShared *>(b_smem + RU_STAGES * RU_B_STAGE);

@@ -25,8 +25,12 @@
 // the w-weighting and the reduction over heads run on the accumulators; the
 // per-head products never leave the SM.  s_t > 0 multiplies the reduced score.
 // Up to 16 scoring heads keep their query fragments in registers.
+#include <algorithm>
+
 #include "frag.cuh"
 #include "internal.h"
+#include "route_slice.cuh"
+#include "rowsel.cuh"
 
 namespace misa {
 namespace {
@@ -49,10 +53,19 @@ struct StreamCfg {
 
 // scale_vec: the per-token scales may be copied 4 at a time (16-byte aligned
 // groups inside the cache); otherwise they are read one by one.
+// fz.zeroed != nullptr: the row's top fz.k are selected here (rowsel.cuh)
+// instead of the histogram going to row_hist; every scored element also stays
+// in shared memory, [warp][max_tiles][TT] after the ring.
+// route_part != nullptr (with fz): the query's h scoring heads are routed
+// here first (route_slice.cuh; heads is ignored): this CTA's partial router
+// sums go to route_part[i][blockIdx.x][H], the row's CTAs meet, and every one
+// ranks the heads from all the partials; CTA 0 of the row writes them to
+// heads_out[i][h] when it is not null.
 template <int NT, bool FP8>
 __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, QueryView qv, const int32_t *heads,
                                                                int h, float *scores, long long ld, int scale_vec,
-                                                               uint32_t *row_hist) {
+                                                               uint32_t *row_hist, FusedTopk fz, int max_tiles,
+                                                               int region, float *route_part, int32_t *heads_out) {
   grid_dep_sync();
   using Cfg = StreamCfg<NT, FP8>;
   using F = FragCfg<FP8>;
@@ -76,6 +89,8 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
   const int wg = blockIdx.x * WARPS + warp;  // this warp takes tiles wg, wg + nwarps, ...
   const int my_tiles = wg < ntile_all ? cdiv(ntile_all - wg, nwarps) : 0;
   const uint32_t ring = smem_addr(smem) + warp * Cfg::WARP_BYTES;
+  const bool fused = fz.zeroed != nullptr;
+  float *sc_s = reinterpret_cast<float *>(smem + region);  // fused: this CTA's scores
   const uint8_t *gkeys = static_cast<const uint8_t *>(c.keys) + (size_t)s * c.L_cap * ROW;
   const float *gscale = FP8 ? c.scale + (size_t)s * c.L_cap : nullptr;
 
@@ -111,9 +126,38 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
   };
 #pragma unroll
   for (int j = 0; j < NS - 1; ++j) issue(j);  // start streaming before the query set-up
+
+  // routing in front of the scan: the keys stream in meanwhile
+  __shared__ float r_tail[D];                   // the causal tail block's mean
+  __shared__ float r_wsum[WARPS * MISA_MAX_H];  // per-warp partial sums
+  __shared__ float r_out[MISA_MAX_H];           // this CTA's partials, then the importances
+  __shared__ int r_keep[MISA_MAX_H];
+  __shared__ int32_t r_heads[NT * 8];
+  __shared__ struct { int ok; } r_bar;
+  const bool route = route_part != nullptr;
+  if (route) {
+    const int Mi = cdiv(Li, c.B), full = Li / c.B, C = gridDim.x;
+    const int m0 = (int)((long long)blockIdx.x * Mi / C), m1 = (int)((long long)(blockIdx.x + 1) * Mi / C);
+    if (full < Mi && full >= m0 && full < m1) {  // uniform: this CTA holds the block cut by the prefix end
+      block_key_sum<128>(c, s, full * c.B, Li, reinterpret_cast<float *>(shist), r_tail);
+      if (tid < D) r_tail[tid] *= 1.f / (float)(Li - full * c.B);
+      __syncthreads();
+    }
+    route_slice<WARPS>(c, qv, i, s, m0, m1, full, r_tail, r_wsum, r_out);
+    float *prow = route_part + (size_t)i * C * qv.H;
+    for (int j = tid; j < qv.H; j += THREADS) prow[(size_t)blockIdx.x * qv.H + j] = r_out[j];
+    if (!row_barrier(r_bar, fz.zeroed + (size_t)i * RS_ZERO_WORDS + 2 * RB + RS_ROUTE, (uint32_t)C, c)) {
+      cp_async_wait<0>();  // no copy in flight when the CTA leaves
+      return;
+    }
+    route_rank(qv, i, prow, C, h, r_out, r_keep, r_heads);
+    if (blockIdx.x == 0 && heads_out)
+      for (int n = tid; n < h; n += THREADS) heads_out[(size_t)i * h + n] = r_heads[n];
+  }
   for (int b = tid; b < TOPK_HIST_BINS; b += THREADS) shist[b] = 0;
 
-  build_query_frags<NT, FP8, THREADS>(c, qv, i, heads, h, bfrag, w_s, scale_s, tid, [] { __syncthreads(); });
+  build_query_frags<NT, FP8, THREADS>(c, qv, i, heads, h, bfrag, w_s, scale_s, tid, [] { __syncthreads(); },
+                                      route ? r_heads : nullptr);
   __syncthreads();
   float wr[NT][2];
 #pragma unroll
@@ -169,12 +213,48 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
       if (cq < 2 && trow < Li) {
         const float v = (me ? sums.y : sums.x) * sc[m];
         scores[(size_t)i * ld + trow] = v;
+        if (fused) sc_s[(warp * max_tiles + j) * TT + 16 * m + g + 8 * me] = v;
         atomicAdd(&shist[ordered_key(v) >> 21], 1u);
       }
     }
   }
   cp_async_wait<0>();
   __syncthreads();
+  if (fused) {
+    // the ring is free: the selection's shared state and scratch go there
+    RsShared<THREADS> &rs = *reinterpret_cast<RsShared<THREADS> *>(smem);
+    uint8_t *scratch = smem + (sizeof(RsShared<THREADS>) + 15) / 16 * 16;
+    const int per_w = max_tiles * TT, total = WARPS * per_w;
+    auto each = [&](auto &&fn) {
+      for (int x = tid; x < (total + THREADS - 1) / THREADS * THREADS; x += THREADS) {
+        const int w = x / per_w, j = (x % per_w) / TT, r = x % TT;
+        const int wgx = blockIdx.x * WARPS + w;
+        const int tiles_w = wgx < ntile_all ? cdiv(ntile_all - wgx, nwarps) : 0;
+        const int tok = (wgx + j * nwarps) * TT + r;
+        const bool valid = x < total && j < tiles_w && tok < Li;
+        fn(valid ? ordered_key(sc_s[x]) : 0u, tok, valid);
+      }
+    };
+    const float *srow = scores + (size_t)i * ld;
+    auto sweep = [&](auto &&fn) {
+      constexpr int SU = 8;
+      for (int base = 0; base < Li; base += THREADS * SU) {
+        float v[SU];
+#pragma unroll
+        for (int u = 0; u < SU; ++u) {
+          const int p = base + u * THREADS + tid;
+          v[u] = p < Li ? __ldcg(srow + p) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < SU; ++u) {
+          const int p = base + u * THREADS + tid;
+          fn(ordered_key(v[u]), POS_MAX - (uint32_t)p, p < Li);
+        }
+      }
+    };
+    row_select<THREADS>(c, rs, shist, scratch, rs_row(fz, i), gridDim.x, fz.k, Li, fz.ordered != 0, each, sweep);
+    return;
+  }
   uint32_t *rh = row_hist + (size_t)i * TOPK_HIST_BINS;
   for (int b = tid; b < TOPK_HIST_BINS; b += THREADS) {
     const uint32_t v = shist[b];
@@ -182,45 +262,100 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
   }
 }
 
+// Launch shape of one scoring call: splits CTAs per query (one wave of the
+// resident CTAs), dynamic shared memory, and -- for a fused selection -- the
+// tiles a warp scores at most and where its scores start.
+struct StreamPlan {
+  int splits = 0, smem = 0, max_tiles = 0, region = 0;
+  bool ok = false;
+};
+
+template <int NT, bool FP8>
+StreamPlan plan_nt(const CacheView &c, const QueryView &q, bool fused) {
+  using Cfg = StreamCfg<NT, FP8>;
+  constexpr int RING = WARPS * Cfg::WARP_BYTES;
+  StreamPlan p;
+  const int sms = device_sms();
+  // the largest dynamic shared memory any launch may ask for (also the opt-in)
+  struct Tag {};
+  const int max_dyn = cached_per_device<Tag>([] { return opt_in_max_dyn_smem(score_stream_kernel<NT, FP8>); });
+  if (max_dyn < RING) return p;
+  auto per_sm_for = [&](int smem) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, score_stream_kernel<NT, FP8>, THREADS, smem) != cudaSuccess)
+      return 0;
+    return n;
+  };
+  const int ntile = cdiv(c.L_cap, Cfg::TT);
+  auto splits_for = [&](int per_sm) {
+    // one wave: a CTA beyond the resident slots would double the kernel time
+    int sp = std::max(1, per_sm * sms / std::max(q.n_q, 1));
+    return std::min(sp, std::max(1, cdiv(ntile, 2 * WARPS)));  // >= 2 tiles per warp
+  };
+  if (!fused) {
+    struct TagR {};
+    const int per_sm = cached_per_device<TagR>([&] { return std::max(per_sm_for(RING), 1); });
+    p.splits = splits_for(per_sm);
+    p.smem = RING;
+    p.ok = true;
+    return p;
+  }
+  // fused: the ring (reused for the selection afterwards) and the scores
+  const int region = (std::max(RING, (int)((sizeof(RsShared<THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap)) +
+                      127) / 128 * 128;
+  int per_sm = per_sm_for(RING);
+  for (int it = 0; it < 3 && per_sm > 0; ++it) {
+    const int sp = splits_for(per_sm);
+    const int mt = cdiv(ntile, sp * WARPS);
+    const int smem = region + WARPS * mt * Cfg::TT * 4;
+    const int fit = smem <= max_dyn ? per_sm_for(smem) : 0;
+    if (fit >= per_sm) {  // the grid is resident at once
+      if ((long long)sp * q.n_q > (long long)fit * sms) return p;
+      p.splits = sp;
+      p.smem = smem;
+      p.max_tiles = mt;
+      p.region = region;
+      p.ok = true;
+      return p;
+    }
+    per_sm = fit;  // fewer CTAs per SM: fewer splits, more tiles each
+  }
+  return p;
+}
+
 template <int NT, bool FP8>
 cudaError_t launch_nt(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
-                      long long ld, uint32_t *row_hist, cudaStream_t s) {
-  constexpr int SMEM = WARPS * StreamCfg<NT, FP8>::WARP_BYTES;
-  const int sms = device_sms();
-  // resident CTAs per SM (also sets the shared-memory opt-in), once per device
-  struct Tag {};
-  const int per_sm = cached_per_device<Tag>([] {
-    if (cudaFuncSetAttribute(score_stream_kernel<NT, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
-        cudaSuccess)
-      return -1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, score_stream_kernel<NT, FP8>, THREADS, SMEM) !=
-        cudaSuccess)
-      return -1;
-    return max(n, 1);
-  });
-  if (per_sm < 0) return cudaErrorInvalidConfiguration;
-  // one wave: a CTA beyond the resident slots would double the kernel time
-  int splits = max(1, per_sm * sms / q.n_q);
-  splits = min(splits, max(1, cdiv(cdiv(c.L_cap, StreamCfg<NT, FP8>::TT), 2 * WARPS)));  // >= 2 tiles per warp
+                      long long ld, uint32_t *row_hist, cudaStream_t s, const FusedTopk *fz, float *route_part,
+                      int32_t *heads_out) {
+  const StreamPlan p = plan_nt<NT, FP8>(c, q, fz != nullptr);
+  if (!p.ok) return cudaErrorInvalidConfiguration;
+  if (route_part && (!fz || (long long)p.splits * q.n_q > route_part_slots())) return cudaErrorInvalidValue;
   const int scale_vec = FP8 && (reinterpret_cast<uintptr_t>(c.scale) & 15) == 0 && c.L_cap % 4 == 0;
-  return launch_kernel(score_stream_kernel<NT, FP8>, dim3(splits, q.n_q), dim3(THREADS), SMEM, s, c, q, heads, h, scores,
-                    ld, scale_vec, row_hist);
+  FusedTopk none = {};
+  return launch_kernel(score_stream_kernel<NT, FP8>, dim3(p.splits, q.n_q), dim3(THREADS), p.smem, s, c, q, heads, h,
+                       scores, ld, scale_vec, row_hist, fz ? *fz : none, p.max_tiles, p.region, route_part,
+                       heads_out);
 }
+
+int stream_nt_h(int h_eff) {
+  int NT = 1;
+  while (NT * 8 < h_eff) NT *= 2;
+  return NT;
+}
+
+int stream_nt(const QueryView &q, const int32_t *heads, int h) { return stream_nt_h(heads ? h : q.H); }
 
 }  // namespace
 
 cudaError_t launch_score_stream(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
-                                long long ld, uint32_t *row_hist, cudaStream_t s) {
+                                long long ld, uint32_t *row_hist, cudaStream_t s, const FusedTopk *fused,
+                                float *route_part, int32_t *heads_out) {
   if (q.n_q == 0) return cudaSuccess;
-  const int h_eff = heads ? h : q.H;
-  int NT = 1;
-  while (NT * 8 < h_eff) NT *= 2;
-#define MISA_STREAM_CASE(N)                                                   \
-  case N:                                                                     \
-    return c.fp8 ? launch_nt<N, true>(c, q, heads, h, scores, ld, row_hist, s) \
-                 : launch_nt<N, false>(c, q, heads, h, scores, ld, row_hist, s);
-  switch (NT) {
+#define MISA_STREAM_CASE(N)                                                                                      \
+  case N:                                                                                                        \
+    return c.fp8 ? launch_nt<N, true>(c, q, heads, h, scores, ld, row_hist, s, fused, route_part, heads_out)     \
+                 : launch_nt<N, false>(c, q, heads, h, scores, ld, row_hist, s, fused, route_part, heads_out);
+  switch (route_part ? stream_nt_h(h) : stream_nt(q, heads, h)) {
     MISA_STREAM_CASE(1)
     MISA_STREAM_CASE(2)
     MISA_STREAM_CASE(4)
@@ -228,6 +363,25 @@ cudaError_t launch_score_stream(const CacheView &c, const QueryView &q, const in
     MISA_STREAM_CASE(16)
     default:
       return cudaErrorInvalidValue;
+  }
+#undef MISA_STREAM_CASE
+}
+
+bool score_stream_fusable(const CacheView &c, const QueryView &q, const int32_t *heads, int h, bool route) {
+  if (q.n_q == 0) return false;
+#define MISA_STREAM_CASE(N)                                                                     \
+  case N: {                                                                                     \
+    const StreamPlan p = c.fp8 ? plan_nt<N, true>(c, q, true) : plan_nt<N, false>(c, q, true); \
+    return p.ok && (!route || (long long)p.splits * q.n_q <= route_part_slots());              \
+  }
+  switch (route ? stream_nt_h(h) : stream_nt(q, heads, h)) {
+    MISA_STREAM_CASE(1)
+    MISA_STREAM_CASE(2)
+    MISA_STREAM_CASE(4)
+    MISA_STREAM_CASE(8)
+    MISA_STREAM_CASE(16)
+    default:
+      return false;
   }
 #undef MISA_STREAM_CASE
 }

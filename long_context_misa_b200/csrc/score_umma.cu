@@ -105,7 +105,8 @@ __global__ void __launch_bounds__(UCfg<FP8, HPQ>::THREADS, 1)
   using Cfg = UCfg<FP8, HPQ>;
   constexpr int QPT = UM_N / HPQ;
   extern __shared__ uint8_t um_raw[];
-  uint8_t *base = um_raw + ((1024u - (smem_addr(um_raw) & 1023u)) & 1023u);  // 1024-aligned (swizzle atoms)
+  uint8_t *base = aligned_smem_base(um_raw, Cfg::SMEM - 1024, c);  // 1024-aligned (swizzle atoms)
+  if (!base) return;
   uint8_t *a_smem = base;                                    // STAGES x A_BYTES (1024-aligned each)
   uint8_t *b_smem = base + Cfg::STAGES * Cfg::A_BYTES;       // B_BYTES
   constexpr int EPI_WARPS = Cfg::EPI_WARPS, UM_THREADS = Cfg::THREADS;

@@ -29,8 +29,8 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "misa.h")
 
 MISA_OK, MISA_ERR_INVALID, MISA_ERR_UNSUPPORTED, MISA_ERR_WORKSPACE, MISA_ERR_CUDA = range(5)
 MISA_KEY_BF16, MISA_KEY_FP8_E4M3 = 0, 1
-OP_ROUTE, OP_SCORE_TOPK, OP_DENSE_TOPK, OP_RERANK_TOPK, OP_DAGGER_TOPK = range(5)
-DEV_BAD_POSITION, DEV_APPEND_RANGE, DEV_WAIT_TIMEOUT, DEV_BAD_HEAD = 1, 2, 4, 8
+OP_ROUTE, OP_SCORE_TOPK, OP_DENSE_TOPK, OP_RERANK_TOPK, OP_DAGGER_TOPK, OP_DAGGER_DECODE = range(6)
+DEV_BAD_POSITION, DEV_APPEND_RANGE, DEV_WAIT_TIMEOUT, DEV_BAD_HEAD, DEV_SMEM_LAYOUT = 1, 2, 4, 8, 16
 D = 128
 NOALLOC_SCRATCH_BYTES = 4 << 20  # MISA_NOALLOC_SCRATCH_BYTES
 
@@ -68,6 +68,7 @@ def _load() -> ctypes.CDLL:
         "misa_rerank_topk": (I32, [C, Q, P, I32, I32, P, P, P, SZ, P]),
         "misa_rerank_topk_noalloc": (I32, [C, Q, P, I32, I32, P, P, P]),
         "misa_dagger_topk": (I32, [C, Q, P, I32, I32, I32, P, P, SZ, P]),
+        "misa_dagger_decode": (I32, [C, Q, P, P, P, I32, I32, I32, I32, P, P, P, SZ, P]),
         "misa_workspace_bytes": (SZ, [I32, C, Q, I32, I32, I32]),
         "misa_last_error": (ctypes.c_char_p, []),
         "misa_status_name": (ctypes.c_char_p, [I32]),
@@ -309,6 +310,23 @@ def dagger_topk(cache: KeyCache, qs: Queries, heads: torch.Tensor, k_prime: int,
     return topk
 
 
+def dagger_decode(cache: KeyCache, qs: Queries, new_keys: torch.Tensor, new_scale: Optional[torch.Tensor],
+                  new_pos: torch.Tensor, h: int, k_prime: int, k: int, heads: Optional[torch.Tensor] = None,
+                  topk: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None, stream=None) -> torch.Tensor:
+    """One MISA-dagger decode step: append new_keys [n_seq][count][128] at
+    new_pos, route every query to h heads (written to ``heads`` when given),
+    routed top-k' candidates re-ranked with all heads to k (see misa.h)."""
+    dev = qs.q.device
+    if topk is None:
+        topk = torch.empty(qs.n_q, k, dtype=torch.int32, device=dev)
+    count = int(new_keys.shape[1])
+    buf, nb = _ws(ws, workspace_bytes(OP_DAGGER_DECODE, cache, qs, h, k, k_prime), dev)
+    _check(_lib.misa_dagger_decode(ctypes.byref(cache.struct), ctypes.byref(qs.struct), _ptr(new_keys),
+                                   _ptr(new_scale), _ptr(new_pos), count, h, k_prime, k, _ptr(heads), _ptr(topk),
+                                   _ptr(buf), nb, _stream(stream)))
+    return topk
+
+
 def rerank_topk_noalloc(cache: KeyCache, qs: Queries, cand: torch.Tensor, topk: torch.Tensor,
                         scores_out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """misa_rerank_topk_noalloc: the fine stage with the library's fixed scratch.
@@ -353,7 +371,11 @@ class MisaDaggerDecode:
     (new_pos is normally q_pos).
     """
 
-    LAUNCHES = 9  # append 1, route 2, zero 1, score 1, top-k' 2 (filter, select), re-rank 1, top-k 1
+    # kernels of one step when the batch runs fused (decode shapes whose
+    # scoring grids fit on the device at once): the append (which also clears
+    # the selections' counters), routing + routed scoring + top-k', and the
+    # all-head re-rank + top-k
+    LAUNCHES = 3
 
     def __init__(self, cache: KeyCache, qs: Queries, h: int, k_prime: int, k: int, new_keys: torch.Tensor,
                  new_scale: Optional[torch.Tensor], new_pos: torch.Tensor):
@@ -362,15 +384,14 @@ class MisaDaggerDecode:
         self.new_keys, self.new_scale, self.new_pos = new_keys, new_scale, new_pos
         self.heads = torch.empty(qs.n_q, h, dtype=torch.int32, device=dev)
         self.topk = torch.empty(qs.n_q, k, dtype=torch.int32, device=dev)
-        need = max(workspace_bytes(OP_ROUTE, cache, qs, h), workspace_bytes(OP_DAGGER_TOPK, cache, qs, h, k, k_prime))
+        need = workspace_bytes(OP_DAGGER_DECODE, cache, qs, h, k, k_prime)
         self.ws = Workspace(dev)
         self.ws.get(need)
         self.graph = None
 
     def run(self, stream=None) -> torch.Tensor:
-        pool_keys(self.cache, self.new_keys, self.new_scale, self.new_pos, stream=stream)
-        route_heads(self.cache, self.qs, self.h, heads=self.heads, ws=self.ws, stream=stream)
-        dagger_topk(self.cache, self.qs, self.heads, self.k_prime, self.k, topk=self.topk, ws=self.ws, stream=stream)
+        dagger_decode(self.cache, self.qs, self.new_keys, self.new_scale, self.new_pos, self.h, self.k_prime, self.k,
+                      heads=self.heads, topk=self.topk, ws=self.ws, stream=stream)
         return self.topk
 
     def capture(self) -> "MisaDaggerDecode":

@@ -31,7 +31,7 @@ by = ctypes.byref
 
 def test_exports_every_declared_symbol():
     names = M.header_symbols()
-    assert len(names) == 16
+    assert len(names) == 17
     for n in names:
         assert hasattr(L, n), n
     assert M.version() == 1
@@ -93,7 +93,11 @@ def test_workspace_sizes():
     assert M._lib.misa_workspace_bytes(M.OP_RERANK_TOPK, by(c), by(q), 0, 8, 77) >= 4 * 3 * 77
     assert M._lib.misa_workspace_bytes(9, by(c), by(q), 0, 8, 77) == 0
     assert M._lib.misa_workspace_bytes(M.OP_DAGGER_TOPK, by(c), by(q), 4, 8, 77) >= 4 * 3 * (1000 + 2 * 77)
-    for op in range(5):
+    # the decode step: MISA-dagger's workspace plus the router's and the heads
+    assert M._lib.misa_workspace_bytes(M.OP_DAGGER_DECODE, by(c), by(q), 4, 8, 77) >= \
+        M._lib.misa_workspace_bytes(M.OP_DAGGER_TOPK, by(c), by(q), 4, 8, 77) + 4 * 3 * 4
+    assert M._lib.misa_workspace_bytes(M.OP_DAGGER_DECODE, by(c), by(q), 0, 8, 77) == 0  # h = 0
+    for op in range(6):
         assert M._lib.misa_workspace_bytes(op, by(c), by(q), 4, 8, 77) % 256 == 0
 
 
@@ -141,6 +145,41 @@ def test_dagger_argument_checks():
     assert L.misa_dagger_topk(by(c), by(q), FAKE, 0, 64, 16, FAKE, FAKE, big, None) == M.MISA_ERR_INVALID  # h
     assert L.misa_dagger_topk(by(c), by(q), None, 8, 64, 16, FAKE, FAKE, big, None) == M.MISA_ERR_INVALID
     assert L.misa_dagger_topk(by(c), by(q), FAKE, 8, 64, 16, FAKE, FAKE, 100, None) == M.MISA_ERR_WORKSPACE
+
+
+def test_dagger_decode_argument_checks():
+    c, q = cache(), queries()
+    big = 1 << 30
+    D = L.misa_dagger_decode
+    ok = (FAKE, None, FAKE, 1, 8, 64, 16, FAKE, FAKE, FAKE, big, None)
+
+    def call(**kw):
+        names = ["new_keys", "new_scale", "new_pos", "count", "h", "k_prime", "k", "heads", "topk", "ws", "ws_bytes",
+                 "stream"]
+        args = dict(zip(names, ok))
+        args.update(kw)
+        return D(by(c), by(q), *[args[n] for n in names])
+
+    assert call(count=0) == M.MISA_ERR_INVALID
+    assert call(count=5000) == M.MISA_ERR_INVALID            # above L_cap
+    assert call(new_keys=None) == M.MISA_ERR_INVALID
+    assert call(new_pos=None) == M.MISA_ERR_INVALID
+    assert call(new_keys=FAKE + 8) == M.MISA_ERR_INVALID      # misaligned
+    assert call(new_scale=FAKE) == M.MISA_ERR_INVALID         # scale for bf16 keys
+    assert call(h=0) == M.MISA_ERR_INVALID
+    assert call(h=65) == M.MISA_ERR_INVALID
+    assert call(k=65) == M.MISA_ERR_INVALID                   # k > k'
+    assert call(k_prime=(1 << 18) + 1, k=16) == M.MISA_ERR_UNSUPPORTED
+    assert call(topk=None) == M.MISA_ERR_INVALID
+    assert call(ws_bytes=100) == M.MISA_ERR_WORKSPACE
+    c8 = cache(dtype=M.MISA_KEY_FP8_E4M3, scale=FAKE)
+    assert D(by(c8), by(q), FAKE, None, FAKE, 1, 8, 64, 16, None, FAKE, FAKE, big, None) == M.MISA_ERR_INVALID
+    M.debug_fail_next(1)
+    try:
+        assert call() == M.MISA_ERR_CUDA
+        assert "injected" in M.last_error()
+    finally:
+        M.debug_fail_next(0)
 
 
 def test_wait_timeout_argument_checks():

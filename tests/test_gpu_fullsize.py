@@ -1,10 +1,12 @@
-"""GPU parity at the five workloads' full sizes, on sampled queries.
+"""GPU parity at the five workloads' full sizes.
 
 Every workload runs whole on the GPU (all queries, full L); the oracle then
-recomputes a few sampled queries one by one: the first and the last query of
-the batch and the first needle's target query.  The MISA-dagger decode runs
-as the captured decode step (append + route + routed top-k' + re-rank), the
-launch configuration the throughput measurement replays.
+recomputes queries one by one: every query of the decode workloads, and 32
+queries spread evenly over each prefill chunk (so over its query groups of
+the tensor-core path) plus every needle's target query.  The MISA-dagger
+decode runs as the captured decode step (append + route + routed top-k' +
+re-rank in one call), the launch configuration the throughput measurement
+replays.
 
 Checks per sampled query (tolerances as in the smaller parity tests):
 router scores within tolerance and head set equal up to boundary ties; the
@@ -30,7 +32,9 @@ pytestmark = pytest.mark.gpu
 
 def _sample(inp):
     wl = inp.wl
-    picks = [0, wl.n_q - 1] + [qi for (_, _, qi) in inp.needles[:1]]
+    if wl.mode == "decode":
+        return list(range(wl.n_q))
+    picks = np.linspace(0, wl.n_q - 1, 32).astype(int).tolist() + [qi for (_, _, qi) in inp.needles]
     return sorted(set(picks))
 
 
@@ -60,6 +64,7 @@ def test_full_size_sampled(name):
                                   torch.from_numpy(sc).cuda(), torch.from_numpy(inp.q_pos.copy()).cuda())
         step.run()
         torch.cuda.synchronize()
+        step_heads = step.heads.cpu().numpy()
         # restore the short cache and replay the captured step: same result
         first = step.topk.clone()
         cache.seq_len.copy_(torch.from_numpy(inp.seq_len - 1))
@@ -108,6 +113,9 @@ def test_full_size_sampled(name):
         assert_close(r_gpu[i], r, f"{tag} router scores")
         assert np.all(np.diff(heads[i]) > 0)
         ties["heads"] += compare_selection(heads[i], hs, lambda t: r[t], wl.h, f"{tag} heads")
+        if wl.k_prime:  # the decode step routes inside its scoring kernel
+            assert np.all(np.diff(step_heads[i]) > 0)
+            ties["heads"] += compare_selection(step_heads[i], hs, lambda t: r[t], wl.h, f"{tag} step heads")
 
         I = O.index_scores(q, w, K[:Li], heads[i])
         assert_close(routed_rows[j, :Li], I, f"{tag} routed scores")
@@ -120,7 +128,9 @@ def test_full_size_sampled(name):
         _ascending_valid(dtop[i], Li, wl.k)
         ties["dense"] += compare_selection(dtop[i], d["topk"], lambda t: d["scores"][t], wl.k, f"{tag} dense top-k")
 
-        if wl.k_prime:
+        if wl.k_prime and np.array_equal(step_heads[i], heads[i]):
+            # the step's final top-k against the oracle's re-rank of the
+            # candidates of the same heads (the separate call's)
             fine = O.rerank_query(q, w, K, top[i], wl.k)
             by_tok = dict(zip(fine["cand"].tolist(), fine["scores"].tolist()))
             _ascending_valid(final[i], Li, wl.k)
@@ -128,7 +138,9 @@ def test_full_size_sampled(name):
             ties["final"] += compare_selection(final[i], fine["topk"], lambda t: by_tok[t], wl.k,
                                                f"{tag} MISA-dagger top-k")
 
-    print(f"\n{name}: sampled queries {picks}, boundary ties {ties}")
+    print(f"\n{name}: {len(picks)} queries checked against the oracle, boundary ties {ties}")
     n = len(picks)
     assert ties["heads"] <= n
     assert max(ties["routed"], ties["dense"], ties["final"]) <= 4 * n
+    if wl.k_prime:  # near-tied head importances are rare: the step routed like the router
+        assert sum(np.array_equal(step_heads[i], heads[i]) for i in picks) >= n - 1

@@ -522,6 +522,61 @@ def test_rerank_candidate_order_does_not_matter():
         assert np.all(np.diff(got) > 0)
 
 
+def _decode_step_inputs(inp):
+    """The cache one token short of every sequence's length, and that token's
+    key (and scale) to append at its position."""
+    wl = inp.wl
+    pos = (inp.seq_len - 1).astype(np.int32)
+    last = np.stack([inp.keys[s, pos[s]:pos[s] + 1] for s in range(wl.n_seq)])
+    nk = torch.from_numpy(last.view(np.int16) if last.dtype == np.uint16 else last).cuda().contiguous()
+    ns = None
+    if inp.scale is not None:
+        ns = torch.from_numpy(np.stack([inp.scale[s, pos[s]:pos[s] + 1] for s in range(wl.n_seq)])).cuda()
+    return nk, ns, torch.from_numpy(pos).cuda()
+
+
+@pytest.mark.parametrize("case", ["fp8_mixture", "fp8_long", "bf16_mixture", "fp8_h96", "bf16_normal",
+                                  "bf16_prefill", "fp8_prefill_umma"])
+def test_dagger_decode_step(case):
+    # append + route + MISA-dagger in one call: the appended cache and pool
+    # are the oracle's, the heads are the oracle's up to boundary ties, and
+    # the final top-k is what misa_dagger_topk returns with those heads (that
+    # call is checked against the oracle by the composition and re-rank
+    # tests).  Decode cases route inside the scoring kernel; prefill chunks
+    # run the three calls in sequence.
+    inp = make(case)
+    ref = Ref(inp)
+    wl = inp.wl
+    kp = wl.k_prime or 4 * wl.k
+    cache, qs = to_device(inp, torch)
+    cache.seq_len.copy_(torch.from_numpy(inp.seq_len - 1))
+    M.pool_keys(cache)
+    nk, ns, pos = _decode_step_inputs(inp)
+    heads = torch.full((wl.n_q, wl.h), -7, dtype=torch.int32, device="cuda")
+    top = M.dagger_decode(cache, qs, nk, ns, pos, wl.h, kp, wl.k, heads=heads).cpu().numpy()
+    assert np.array_equal(cache.seq_len.cpu().numpy(), inp.seq_len)
+    pool = cache.pool.cpu().numpy()
+    for s_ in range(wl.n_seq):
+        expect = O.pool_keys(ref.K[s_], int(inp.seq_len[s_]), wl.B)
+        assert_close(pool[s_, :expect.shape[0]], expect, f"pool seq {s_}")
+    hd = heads.cpu().numpy()
+    ties = 0
+    for i in range(wl.n_q):
+        q, w, K, Li = ref.query(i)
+        r, hs = O.route_query(q, w, K, Li, wl.B, wl.h)
+        assert np.all(np.diff(hd[i]) > 0), hd[i]
+        ties += compare_selection(hd[i], hs, lambda j: r[j], wl.h, f"heads q{i}")
+        got = top[i][top[i] >= 0]
+        assert np.all(np.diff(got) > 0) and len(got) == min(wl.k, Li)
+    assert ties <= max(1, wl.n_q // 10), f"{ties} head boundary ties"
+    again = M.dagger_topk(cache, qs, heads, kp, wl.k).cpu().numpy()
+    np.testing.assert_array_equal(top, again)
+    # without the heads output, and a second step at the same positions
+    top2 = M.dagger_decode(cache, qs, nk, ns, pos, wl.h, kp, wl.k).cpu().numpy()
+    np.testing.assert_array_equal(top, top2)
+    assert device_status(cache) == 0
+
+
 @pytest.mark.parametrize("case", ["fp8_mixture", "fp8_long", "bf16_mixture", "bf16_prefill", "fp8_prefill_umma"])
 def test_dagger_topk_equals_composition(case):
     # one call (its k' candidates stay unordered inside) returns exactly what
