@@ -26,10 +26,10 @@
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
  *    default stream).  Outputs are valid in stream order.  Nothing blocks the
  *    host.  Between calls the library keeps only cached device attributes,
- *    the thread-local error text, and two process-wide test hooks that are
+ *    the thread-local error text, and three process-wide test hooks that are
  *    off unless a caller sets them: misa_debug_fail_next (a count of calls
- *    to fail) and misa_debug_time_scoring (two events recorded around the
- *    scoring kernels).  misa_rerank_topk_noalloc's fixed scratch array also
+ *    to fail), misa_debug_time_scoring (two events recorded around the
+ *    scoring kernels) and misa_debug_select_in_kernel (a kernel choice).  misa_rerank_topk_noalloc's fixed scratch array also
  *    keeps the last call's contents (see there).
  *  - The library's kernels are launched with programmatic stream
  *    serialisation.  Each waits for the work before it in the stream to
@@ -374,6 +374,17 @@ MISA_API int32_t misa_version(void);
  * failing launch would.  n <= 0 switches injection off.
  */
 MISA_API void misa_debug_fail_next(int32_t n);
+
+/*
+ * Kernel-choice switch for tests and measurements: with on != 0, every call
+ * whose shapes allow it selects its top k inside the scoring kernel (the
+ * CTAs that scored a row meet at counters in the workspace and select from
+ * their on-chip scores), instead of the separate top-k kernels.  The results
+ * are the same either way.  Off by default, because on B200 the separate
+ * kernels are as fast or faster for these calls; misa_dagger_decode's routed
+ * pass selects in-kernel whatever the switch says.  Process-wide.
+ */
+MISA_API void misa_debug_select_in_kernel(int32_t on);
 
 /*
  * Profiling aid: while both are non-NULL, every misa_score_topk,

@@ -27,6 +27,16 @@ struct NvtxRange {
 
 thread_local char g_err[512] = "";
 std::atomic<int> g_fail_next{0};
+// Selection inside the scoring kernels for the calls other than the decode
+// step's routed pass (misa_debug_select_in_kernel).  Off by default: there
+// the separate top-k kernels are as fast or faster on B200 -- the fused
+// selection's cross-CTA phases (two row barriers, two histogram searches in
+// L2, the last CTA's bucket) take about 21 us, as long as the filter and
+// select kernels they replace, and a fused re-rank of 8 x 8192 candidates
+// needs four-tile CTAs to be resident at once (38.6 us against 15.5 + 12.5).
+// The decode step's routed pass selects in-kernel always: its in-kernel
+// router needs the same resident CTAs and hides behind the key prefetch.
+std::atomic<int> g_select_in_kernel{0};
 std::atomic<void *> g_ev_start{nullptr}, g_ev_stop{nullptr};
 
 // Launch the scoring kernel, bracketed by the profiling events when set.
@@ -235,7 +245,7 @@ misa_status score_then_topk(const char *who, const misa_cache *cache, const misa
   // in-kernel when its grid is resident at once, or builds the row
   // histograms on the way for the top-k kernels
   const bool umma = misa::umma_applies(c, q, heads, h);
-  const bool fused = !umma && misa::score_fusable(c, q, heads, h, nullptr, 0);
+  const bool fused = g_select_in_kernel.load() && !umma && misa::score_fusable(c, q, heads, h, nullptr, 0);
   cudaError_t e = fused ? misa::launch_zero(fz_zero, (size_t)qs->n_q * misa::FUSED_ZERO_WORDS, stream)
                         : misa::launch_zero(hist, hist_words(qs), stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
@@ -375,8 +385,8 @@ misa_status dagger_body(const char *who, const misa_cache *cache, const misa_que
   // routed pass: scores, then the k' candidates in any order; selected in the
   // scoring kernels when their grids are resident at once
   const bool umma = !route_part && misa::umma_applies(c, q, heads, h);
-  const bool f1 = route_part || (!umma && misa::score_fusable(c, q, heads, h, nullptr, 0));
-  const bool f2 = misa::score_fusable(c, q, nullptr, q.H, cand, k_prime);
+  const bool f1 = route_part || (g_select_in_kernel.load() && !umma && misa::score_fusable(c, q, heads, h, nullptr, 0));
+  const bool f2 = g_select_in_kernel.load() && misa::score_fusable(c, q, nullptr, q.H, cand, k_prime);
   // both passes' counting words, zeroed by one launch: the histograms and
   // counters of the top-k kernels, the fused selections' words, or both
   uint32_t *z0 = (f1 && f2) ? fz1 : hist;
@@ -544,7 +554,7 @@ misa_status misa_rerank_topk(const misa_cache *cache, const misa_queries *qs, co
   float *scores = scores_out ? scores_out : reinterpret_cast<float *>(after);
   uint8_t *bucket = after + (scores_out ? 0 : round_up(sizeof(float) * (size_t)qs->n_q * k_prime));
   uint8_t *winners = bucket + ws_fz_bucket(qs);
-  const bool fused = misa::score_fusable(c, q, nullptr, q.H, cand, k_prime);
+  const bool fused = g_select_in_kernel.load() && misa::score_fusable(c, q, nullptr, q.H, cand, k_prime);
   cudaError_t e = fused ? misa::launch_zero(fz_zero, (size_t)qs->n_q * misa::FUSED_ZERO_WORDS, stream)
                         : misa::launch_zero(hist, (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
   if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
@@ -649,7 +659,8 @@ misa_status misa_dagger_decode(const misa_cache *cache, const misa_queries *qs, 
   size_t zn = 0;
   if (fused) {
     // the re-rank's fusion does not depend on the candidates' values
-    const bool f2 = misa::score_fusable(c, q, nullptr, q.H, reinterpret_cast<const int32_t *>(w8), k_prime);
+    const bool f2 =
+        g_select_in_kernel.load() && misa::score_fusable(c, q, nullptr, q.H, reinterpret_cast<const int32_t *>(w8), k_prime);
     const size_t first = f2 ? ws_dagger_hist(qs) / sizeof(uint32_t) : 0;  // both fused: only their words
     z0 = reinterpret_cast<uint32_t *>(w8) + first;
     zn = dagger_zero_words(qs, true, f2) - first;
@@ -691,6 +702,8 @@ const char *misa_status_name(int32_t status) {
 int32_t misa_version(void) { return 1; }
 
 void misa_debug_fail_next(int32_t n) { g_fail_next.store(n > 0 ? n : 0); }
+
+void misa_debug_select_in_kernel(int32_t on) { g_select_in_kernel.store(on ? 1 : 0); }
 
 void misa_debug_time_scoring(void *start, void *stop) {
   g_ev_start.store(start);

@@ -178,6 +178,12 @@ inline int opt_in_max_dyn_smem(K *kernel) {
   const int mx = optin - (int)fa.sharedSizeBytes;
   if (mx <= 0 || cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mx) != cudaSuccess)
     return -1;
+  // all of the SM's configurable memory as shared memory: the occupancy
+  // query (and the co-residency a fused selection relies on) then counts
+  // the CTAs that really fit
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+    return -1;
   return mx;
 }
 

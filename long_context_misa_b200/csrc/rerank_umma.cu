@@ -137,7 +137,8 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
   constexpr int T = Cfg::T;
   extern __shared__ uint8_t rr_raw[];
   // the tiles and Q', or (a fused selection, afterwards) its state and scratch
-  const uint32_t sel_bytes = (uint32_t)((sizeof(RsShared<RR_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap);
+  const uint32_t sel_bytes =
+      (uint32_t)((sizeof(RsShared<RR_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap, T * RR_M);
   const uint32_t need = max((uint32_t)(Cfg::SMEM - 1024), fz.zeroed ? sel_bytes : 0u);
   uint8_t *base = aligned_smem_base(rr_raw, need, c);  // 1024-aligned (swizzle atoms)
   if (!base) return;
@@ -238,7 +239,7 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
 #pragma unroll
     for (int j = 0; j < T; ++j) {
       if (j >= ntile) break;
-      float acc = 0.f;
+      float a4[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
       const float4 *w4 = reinterpret_cast<const float4 *>(sh.w);
 #pragma unroll
       for (int cb = 0; cb < HN; cb += 32) {
@@ -248,12 +249,13 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
 #pragma unroll
         for (int x = 0; x < 32; x += 4) {
           const float4 w = w4[(cb + x) >> 2];
-          acc = fmaf(w.x, fmaxf(__uint_as_float(v[x]), 0.f), acc);
-          acc = fmaf(w.y, fmaxf(__uint_as_float(v[x + 1]), 0.f), acc);
-          acc = fmaf(w.z, fmaxf(__uint_as_float(v[x + 2]), 0.f), acc);
-          acc = fmaf(w.w, fmaxf(__uint_as_float(v[x + 3]), 0.f), acc);
+          a4[0] = fmaf(w.x, fmaxf(__uint_as_float(v[x]), 0.f), a4[0]);
+          a4[1] = fmaf(w.y, fmaxf(__uint_as_float(v[x + 1]), 0.f), a4[1]);
+          a4[2] = fmaf(w.z, fmaxf(__uint_as_float(v[x + 2]), 0.f), a4[2]);
+          a4[3] = fmaf(w.w, fmaxf(__uint_as_float(v[x + 3]), 0.f), a4[3]);
         }
       }
+      const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
       const int e = j * RR_M + r;
       const int t = sh.tok[e];
       if (t >= 0) {
@@ -309,8 +311,8 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
         }
       }
     };
-    row_select<RR_THREADS>(c, rs, sh.hist, scratch, rs_row(fz, i), gridDim.x, fz.k, Li, fz.ordered != 0, each,
-                           sweep);
+    row_select<RR_THREADS>(c, rs, sh.hist, scratch, rs_row(fz, i), gridDim.x, fz.k, Li, fz.ordered != 0, T * RR_M,
+                           each, sweep);
     return;
   }
   if (got) {
@@ -334,17 +336,21 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
 //   warp 1     owns the tensor memory; one thread issues each tile's MMAs into
 //              one of two accumulator buffers and commits the stage back to
 //              the producer and the buffer to the epilogue;
-//   warps 2-5  one tensor-memory lane quarter each, one token row per thread:
-//              ReLU, the weights, the head sum and the e4m3 token scale
-//              (loaded one tile ahead), the score written and counted.
+//   warps 2-9  two sets of four warps, set b draining accumulator buffer b
+//              (the even or the odd tiles); in a set one tensor-memory lane
+//              quarter per warp, one token row per thread: ReLU, the weights,
+//              the head sum (four independent partial sums) and the e4m3
+//              token scale (loaded one tile ahead), the score written and
+//              counted.
 // The two accumulator buffers let tile j + 1's MMAs run while tile j is
-// drained, and the ring keeps DS_STAGES tiles of keys in flight per SM.
+// drained, two sets drain two tiles at once, and the ring keeps DS_STAGES
+// tiles of keys in flight per SM.
 // With a fused selection every score also stays in shared memory and the
 // query's CTAs select its top k afterwards (rowsel.cuh).  Every wait is
 // bounded: one that runs out sets MISA_DEV_WAIT_TIMEOUT and the CTA winds
 // down without selecting.
 constexpr int DS_STAGES = 8;
-constexpr int DS_EPI = 4;
+constexpr int DS_EPI = 8;  // two sets of four: set b drains accumulator buffer b (tiles j with j % 2 == b)
 constexpr int DS_THREADS = 64 + 32 * DS_EPI;
 
 template <int HN>
@@ -403,7 +409,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh.tfull[b], 1);
-      mbar_init(&sh.tempty[b], DS_EPI);
+      mbar_init(&sh.tempty[b], DS_EPI / 2);
     }
     sh.abort = 0;
     fence_mbar_init();
@@ -459,42 +465,43 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
       }
     }
   } else {
-    // ---- epilogue: token row r of every tile ----
+    // ---- epilogue: set `buf` drains the tiles j = buf, buf + 2, ...; token row r ----
+    const int buf = ((warp - 2) >> 2) & 1;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + buf * HN;
     const float4 *w4 = reinterpret_cast<const float4 *>(sh.w);
     const float *srow_scale = c.scale + (size_t)s * c.L_cap;
     float sc_next = 0.f;
-    if (n_my > 0) {
-      const int t = part * RR_M + r;
+    if (buf < n_my) {
+      const int t = (part + buf * nparts) * RR_M + r;
       sc_next = t < Li ? __ldg(srow_scale + t) : 0.f;
     }
-    for (int j = 0; j < n_my; ++j) {
-      const int buf = j & 1;
+    for (int j = buf; j < n_my; j += 2) {
       const int t = (part + j * nparts) * RR_M + r;
       const float scl = sc_next;
-      if (j + 1 < n_my) {
-        const int tn = t + nparts * RR_M;
+      if (j + 2 < n_my) {
+        const int tn = t + 2 * nparts * RR_M;
         sc_next = tn < Li ? __ldg(srow_scale + tn) : 0.f;
       }
       if (!umma::wait_bar(&sh.tfull[buf], (j >> 1) & 1, abort, c)) break;
       umma::fence_after();
-      float acc = 0.f;
+      float a4[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
 #pragma unroll
       for (int cb = 0; cb < HN; cb += 32) {
         uint32_t v[32];
-        umma::ld32(tl + buf * HN + cb, v);
+        umma::ld32(tl + cb, v);
         umma::ld_wait();
 #pragma unroll
         for (int x = 0; x < 32; x += 4) {
           const float4 w = w4[(cb + x) >> 2];
-          acc = fmaf(w.x, fmaxf(__uint_as_float(v[x]), 0.f), acc);
-          acc = fmaf(w.y, fmaxf(__uint_as_float(v[x + 1]), 0.f), acc);
-          acc = fmaf(w.z, fmaxf(__uint_as_float(v[x + 2]), 0.f), acc);
-          acc = fmaf(w.w, fmaxf(__uint_as_float(v[x + 3]), 0.f), acc);
+          a4[0] = fmaf(w.x, fmaxf(__uint_as_float(v[x]), 0.f), a4[0]);
+          a4[1] = fmaf(w.y, fmaxf(__uint_as_float(v[x + 1]), 0.f), a4[1]);
+          a4[2] = fmaf(w.z, fmaxf(__uint_as_float(v[x + 2]), 0.f), a4[2]);
+          a4[3] = fmaf(w.w, fmaxf(__uint_as_float(v[x + 3]), 0.f), a4[3]);
         }
       }
+      const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
       umma::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.tempty[buf]);
@@ -556,7 +563,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
         }
       }
     };
-    row_select<DS_THREADS>(c, rs, sh.hist, scratch, rs_row(fz, i), nparts, fz.k, Li, fz.ordered != 0, each, sweep);
+    row_select<DS_THREADS>(c, rs, sh.hist, scratch, rs_row(fz, i), nparts, fz.k, Li, fz.ordered != 0, total, each,
+                           sweep);
     return;
   }
   uint32_t *rh = row_hist + (size_t)i * TOPK_HIST_BINS;
@@ -582,8 +590,10 @@ DensePlan plan_dense(const CacheView &c, const QueryView &q, bool fused) {
   p.nparts = std::max(1, std::min(n_tiles, sms / std::max(q.n_q, 1)));
   p.max_tiles = cdiv(n_tiles, p.nparts);
   p.smem = dense_smem<HN>(p.max_tiles, fused);
-  p.ok = p.smem <= max_dyn && (!fused || (long long)p.nparts * q.n_q <= sms) && c.fp8 && umma::encoder_available() &&
-         (reinterpret_cast<uintptr_t>(c.keys) & 15u) == 0;
+  // a fused selection's state and scratch reuse the ring
+  const int sel = (int)((sizeof(RsShared<DS_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap, p.max_tiles * RR_M);
+  p.ok = p.smem <= max_dyn && (!fused || ((long long)p.nparts * q.n_q <= sms && sel <= DSCfg<HN>::RING)) && c.fp8 &&
+         umma::encoder_available() && (reinterpret_cast<uintptr_t>(c.keys) & 15u) == 0;
   return p;
 }
 
@@ -605,7 +615,7 @@ cudaError_t launch_dense(const CacheView &c, const QueryView &q, const int32_t *
 template <bool FP8, int HN, int TT>
 int rerank_smem(const CacheView &c, bool fused) {
   using Cfg = RCfg<FP8, HN, TT>;
-  const int sel = 1024 + (int)((sizeof(RsShared<RR_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap);
+  const int sel = 1024 + (int)((sizeof(RsShared<RR_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap, TT * RR_M);
   return fused ? std::max(Cfg::SMEM, sel) : Cfg::SMEM;
 }
 
@@ -645,10 +655,30 @@ cudaError_t launch_tt(const CacheView &c, const QueryView &q, const int32_t *hea
 
 // Gathered candidates: 2 tiles per CTA (more CTAs shorten each gather chain);
 // a prefix row: the persistent dense kernel.
+// Tiles per CTA of a fused re-rank: two when that grid is resident at once,
+// else four (half the CTAs; at most 64 heads), else 0 (no fused selection).
+// The occupancy query answers one CTA per SM for this kernel, so the
+// four-tile form is what a batch of 8 x 8192 candidates takes.
+template <bool FP8, int HN>
+int rerank_fused_tiles(const CacheView &c, const QueryView &q, int n_cols) {
+  if (rerank_fits<FP8, HN, 2>(c, q, n_cols)) return 2;
+  if constexpr (HN <= 64) {
+    if (rerank_fits<FP8, HN, 4>(c, q, n_cols)) return 4;
+  }
+  return 0;
+}
+
 template <bool FP8, int HN>
 cudaError_t launch_hn(const CacheView &c, const QueryView &q, const int32_t *heads, int h, const int32_t *gather,
                       int n_cols, float *scores, long long ld, uint32_t *row_hist, cudaStream_t s,
                       const FusedTopk *fz) {
+  if (gather && fz) {
+    const int tt = rerank_fused_tiles<FP8, HN>(c, q, n_cols);
+    if constexpr (HN <= 64) {
+      if (tt == 4) return launch_tt<FP8, HN, 4>(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s, fz);
+    }
+    if (tt != 2) return cudaErrorInvalidConfiguration;
+  }
   if (gather) return launch_tt<FP8, HN, 2>(c, q, heads, h, gather, n_cols, scores, ld, row_hist, s, fz);
   if (!FP8) return cudaErrorInvalidValue;  // dense decode of bf16 keys streams on mma.sync
   return launch_dense<HN>(c, q, heads, h, scores, ld, row_hist, s, fz);
@@ -702,11 +732,11 @@ bool rerank_fusable(const CacheView &c, const QueryView &q, const int32_t *heads
   if (q.n_q == 0 || n_cols == 0) return false;
   switch (rerank_hn(q, heads, h)) {
     case 32:
-      return c.fp8 ? rerank_fits<true, 32, 2>(c, q, n_cols) : rerank_fits<false, 32, 2>(c, q, n_cols);
+      return (c.fp8 ? rerank_fused_tiles<true, 32>(c, q, n_cols) : rerank_fused_tiles<false, 32>(c, q, n_cols)) > 0;
     case 64:
-      return c.fp8 ? rerank_fits<true, 64, 2>(c, q, n_cols) : rerank_fits<false, 64, 2>(c, q, n_cols);
+      return (c.fp8 ? rerank_fused_tiles<true, 64>(c, q, n_cols) : rerank_fused_tiles<false, 64>(c, q, n_cols)) > 0;
     case 128:
-      return c.fp8 ? rerank_fits<true, 128, 2>(c, q, n_cols) : rerank_fits<false, 128, 2>(c, q, n_cols);
+      return (c.fp8 ? rerank_fused_tiles<true, 128>(c, q, n_cols) : rerank_fused_tiles<false, 128>(c, q, n_cols)) > 0;
     default:
       return false;
   }

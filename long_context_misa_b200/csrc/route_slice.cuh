@@ -54,94 +54,127 @@ __device__ void route_slice(const CacheView &c, const QueryView &qv, int i, int 
   const int H = qv.H, MT = cdiv(H, 16);
   const int M_cap = cdiv(c.L_cap, c.B);
   const uint16_t *qrow = qv.q + (size_t)i * H * D;
-  // one m-tile of 16 heads at a time (few live registers); the pooled keys
-  // are read again for every m-tile, from L2
-  for (int mt = 0; mt < MT; ++mt) {
-    const int ha = 16 * mt + g, hb = ha + 8;
-    float racc0 = 0.f, racc1 = 0.f;  // heads ha, hb
-    for (int nt = warp; m0 + 8 * nt < m1; nt += NW) {
-      const int m = m0 + 8 * nt + g;  // this lane's block (B column g)
-      const float *prow =
-          m >= m1 ? nullptr : m < full ? c.pool + ((size_t)s * M_cap + m) * D : m == full ? tail : nullptr;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  // warp w keeps one m-tile of 16 heads (w % MT) and takes every
+  // (NW / MT)-th n-tile of 8 blocks: all loads of an n-tile are issued
+  // together, and each warp's sums need no more than two accumulators
+  const int wpm = NW / MT;  // warps per m-tile (MT divides NW: MT in {1, 2, 4, 8})
+  const int mt = warp % MT;
+  const int ha = 16 * mt + g, hb = ha + 8;
+  float racc0 = 0.f, racc1 = 0.f;  // heads ha, hb
+  for (int nt = warp / MT; m0 + 8 * nt < m1; nt += wpm) {
+    const int m = m0 + 8 * nt + g;  // this lane's block (B column g)
+    const float *prow = m >= m1 ? nullptr : m < full ? c.pool + ((size_t)s * M_cap + m) * D : m == full ? tail : nullptr;
+    float4 x[4][2];
+    uint4 qa[4], qb[4];
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0;
-        if (prow) {
-          x0 = *reinterpret_cast<const float4 *>(prow + 32 * ch + 8 * cq);
-          x1 = *reinterpret_cast<const float4 *>(prow + 32 * ch + 8 * cq + 4);
-        }
-        const uint4 qa = ha < H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)ha * D + 32 * ch + 8 * cq))
-                                : make_uint4(0u, 0u, 0u, 0u);
-        const uint4 qb = hb < H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)hb * D + 32 * ch + 8 * cq))
-                                : make_uint4(0u, 0u, 0u, 0u);
-        uint32_t bh0, bl0, bh1, bl1;
-        const uint32_t a0[4] = {qa.x, qb.x, qa.y, qb.y};  // k-tile 2ch
-        const uint32_t a1[4] = {qa.z, qb.z, qa.w, qb.w};  // k-tile 2ch + 1
-        rsl_split(x0.x, x0.y, bh0, bl0);
-        rsl_split(x0.z, x0.w, bh1, bl1);
-        mma_bf16_16816(acc, a0, bh0, bh1);
-        mma_bf16_16816(acc, a0, bl0, bl1);
-        rsl_split(x1.x, x1.y, bh0, bl0);
-        rsl_split(x1.z, x1.w, bh1, bl1);
-        mma_bf16_16816(acc, a1, bh0, bh1);
-        mma_bf16_16816(acc, a1, bl0, bl1);
-      }
-      // ReLU of every (head, block) product, summed over this tile's blocks;
-      // absent blocks multiplied zero keys and add nothing
-      racc0 += fmaxf(acc[0], 0.f) + fmaxf(acc[1], 0.f);
-      racc1 += fmaxf(acc[2], 0.f) + fmaxf(acc[3], 0.f);
+    for (int ch = 0; ch < 4; ++ch) {
+      x[ch][0] = prow ? *reinterpret_cast<const float4 *>(prow + 32 * ch + 8 * cq) : make_float4(0.f, 0.f, 0.f, 0.f);
+      x[ch][1] = prow ? *reinterpret_cast<const float4 *>(prow + 32 * ch + 8 * cq + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+      qa[ch] = ha < H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)ha * D + 32 * ch + 8 * cq))
+                      : make_uint4(0u, 0u, 0u, 0u);
+      qb[ch] = hb < H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)hb * D + 32 * ch + 8 * cq))
+                      : make_uint4(0u, 0u, 0u, 0u);
     }
-    // the four lanes of a row group hold the same heads' sums over different blocks
-    racc0 += __shfl_xor_sync(0xffffffffu, racc0, 1);
-    racc0 += __shfl_xor_sync(0xffffffffu, racc0, 2);
-    racc1 += __shfl_xor_sync(0xffffffffu, racc1, 1);
-    racc1 += __shfl_xor_sync(0xffffffffu, racc1, 2);
-    if (cq == 0) {
-      wsum[warp * MISA_MAX_H + ha] = racc0;
-      wsum[warp * MISA_MAX_H + hb] = racc1;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+      uint32_t bh0, bl0, bh1, bl1;
+      const uint32_t a0[4] = {qa[ch].x, qb[ch].x, qa[ch].y, qb[ch].y};  // k-tile 2ch
+      const uint32_t a1[4] = {qa[ch].z, qb[ch].z, qa[ch].w, qb[ch].w};  // k-tile 2ch + 1
+      rsl_split(x[ch][0].x, x[ch][0].y, bh0, bl0);
+      rsl_split(x[ch][0].z, x[ch][0].w, bh1, bl1);
+      mma_bf16_16816(acc, a0, bh0, bh1);
+      mma_bf16_16816(acc, a0, bl0, bl1);
+      rsl_split(x[ch][1].x, x[ch][1].y, bh0, bl0);
+      rsl_split(x[ch][1].z, x[ch][1].w, bh1, bl1);
+      mma_bf16_16816(acc, a1, bh0, bh1);
+      mma_bf16_16816(acc, a1, bl0, bl1);
     }
+    // ReLU of every (head, block) product, summed over this tile's blocks;
+    // absent blocks multiplied zero keys and add nothing
+    racc0 += fmaxf(acc[0], 0.f) + fmaxf(acc[1], 0.f);
+    racc1 += fmaxf(acc[2], 0.f) + fmaxf(acc[3], 0.f);
+  }
+  // the four lanes of a row group hold the same heads' sums over different blocks
+  racc0 += __shfl_xor_sync(0xffffffffu, racc0, 1);
+  racc0 += __shfl_xor_sync(0xffffffffu, racc0, 2);
+  racc1 += __shfl_xor_sync(0xffffffffu, racc1, 1);
+  racc1 += __shfl_xor_sync(0xffffffffu, racc1, 2);
+  if (cq == 0) {
+    wsum[warp * MISA_MAX_H + ha] = racc0;
+    wsum[warp * MISA_MAX_H + hb] = racc1;
   }
   __syncthreads();
+  // head j's sum: the warps holding its m-tile, in warp order
   for (int j = tid; j < H; j += 32 * NW) {
     float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) v += wsum[w * MISA_MAX_H + j];
+    for (int w = (j >> 4) % MT; w < NW; w += MT) v += wsum[w * MISA_MAX_H + j];
     out[j] = v;
   }
   __syncthreads();
 }
 
 // After the row barrier: the query's importances from the C partial sums
-// (part[cc * H + j], written by the C CTAs, added in the order cc = 0..C-1),
-// r_j = |w_j| * sum, and its h best heads in ascending order into sheads
-// (head j is kept iff fewer than h heads beat it: larger r, or equal r and a
-// lower index).  r_s, keep_s: shared [MISA_MAX_H].  Every thread calls.
+// (part[cc * H + j], written by the C CTAs), r_j = |w_j| * sum, and its h
+// best heads in ascending order into sheads (head j is kept iff fewer than h
+// heads beat it: larger r, or equal r and a lower index).  Four threads per
+// head: each adds a quarter of the partials in order, the quarters are
+// combined in a fixed order, so every CTA of the query gets the same sums.
+// r_s, keep_s: shared [MISA_MAX_H]; stage: shared scratch of stage_cap floats
+// for the partials; every thread calls (blockDim.x a multiple of 32, at
+// least H).
 __device__ void route_rank(const QueryView &qv, int i, const float *part, int C, int h, float *r_s, int *keep_s,
-                           int32_t *sheads) {
-  const int tid = threadIdx.x, H = qv.H;
-  for (int j = tid; j < H; j += blockDim.x) {
+                           int32_t *sheads, float *stage, int stage_cap) {
+  const int tid = threadIdx.x, H = qv.H, lane = tid & 31;
+  const bool staged = C * H <= stage_cap;
+  if (staged) {  // every partial requested at once
+    for (int x = tid; x < C * H; x += blockDim.x) stage[x] = __ldcg(part + x);
+    __syncthreads();
+  }
+  const int qq = tid & 3;  // quarter
+  const int c0 = C * qq / 4, c1 = C * (qq + 1) / 4;
+  const int per = blockDim.x >> 2;  // heads per sweep
+  for (int jb = 0; jb < H; jb += per) {
+    const int j = jb + (tid >> 2);
     float acc = 0.f;
-    for (int cc = 0; cc < C; ++cc) acc += __ldcg(part + (size_t)cc * H + j);
-    r_s[j] = fabsf(__ldg(qv.w + (size_t)i * H + j)) * acc;
+    if (j < H)
+      for (int cc = c0; cc < c1; ++cc) acc += staged ? stage[cc * H + j] : __ldcg(part + (size_t)cc * H + j);
+    // quarters of a head sit in four consecutive lanes: (q0 + q1) + (q2 + q3)
+    const float o1 = __shfl_xor_sync(0xffffffffu, acc, 1);
+    const float pair = (qq & 1) ? o1 + acc : acc + o1;
+    const float o2 = __shfl_xor_sync(0xffffffffu, pair, 2);
+    const float tot = (qq & 2) ? o2 + pair : pair + o2;
+    if (j < H && qq == 0) r_s[j] = fabsf(__ldg(qv.w + (size_t)i * H + j)) * tot;
   }
   __syncthreads();
-  for (int j = tid; j < H; j += blockDim.x) {
-    const float r = r_s[j];
+  // rank: each of the four threads counts the heads of a quarter that beat j
+  for (int jb = 0; jb < H; jb += per) {
+    const int j = jb + (tid >> 2);
     int beaten = 0;
-    for (int o = 0; o < H; ++o) {
-      const float ro = r_s[o];
-      beaten += (ro > r) || (ro == r && o < j);
+    if (j < H) {
+      const float r = r_s[j];
+      for (int o = qq; o < H; o += 4) {
+        const float ro = r_s[o];
+        beaten += (ro > r) || (ro == r && o < j);
+      }
     }
-    keep_s[j] = beaten < h;
+    beaten += __shfl_xor_sync(0xffffffffu, beaten, 1);
+    beaten += __shfl_xor_sync(0xffffffffu, beaten, 2);
+    if (j < H && qq == 0) keep_s[j] = beaten < h;
   }
   __syncthreads();
-  for (int j = tid; j < H; j += blockDim.x) {
-    if (!keep_s[j]) continue;
-    int pos = 0;
-    for (int o = 0; o < j; ++o) pos += keep_s[o];
-    if (pos < h) sheads[pos] = j;  // a NaN importance can break the strict order
+  // kept heads in ascending order: a head's position counts the kept heads below it
+  if (tid < 32 * cdiv(H, 32)) {
+    const bool kept = tid < H && keep_s[tid];
+    const uint32_t m = __ballot_sync(0xffffffffu, kept);
+    uint32_t lt = 0;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt));
+    int pos = __popc(m & lt);
+    for (int w = 0; w < (tid >> 5); ++w)
+      for (int x = 32 * w; x < 32 * w + 32 && x < H; ++x) pos += keep_s[x];
+    if (kept && pos < h) sheads[pos] = tid;  // a NaN importance can break the strict order
   }
+  (void)lane;
   __syncthreads();
 }
 

@@ -46,10 +46,15 @@ static_assert(RS_ZERO_WORDS == 2 * RB + FUSED_CTR, "layout of the zeroed words")
 // bucket entries written, and the barrier of a router fused in front
 enum { RS_BAR0 = 0, RS_BAR1 = 1, RS_DONE = 2, RS_EMIT = 3, RS_BUCKET = 4, RS_ROUTE = 5 };
 
-// Shared scratch of the last CTA, beyond RsShared: the staged bucket, then
-// the token bitmap of an ascending output.
-__host__ __device__ constexpr int rs_scratch_bytes(int L_cap) {
-  return (8 * RS_BCAP > 4 * ((L_cap + 31) / 32 + 4)) ? 8 * RS_BCAP : 4 * ((L_cap + 31) / 32 + 4);
+constexpr int RS_BSTAGE = 512;  // bucket entries a CTA stages before reserving their slots
+
+// Shared scratch beyond RsShared, used in turn for: a CTA's winners and
+// bucket entries before they are written out (elems: the most elements a
+// CTA holds); the last CTA's staged bucket; the token bitmap of an
+// ascending output.
+__host__ __device__ constexpr int rs_max3(int a, int b, int c) { return a > b ? (a > c ? a : c) : (b > c ? b : c); }
+__host__ __device__ constexpr int rs_scratch_bytes(int L_cap, int elems) {
+  return rs_max3(8 * RS_BCAP, 4 * ((L_cap + 31) / 32 + 4), 4 * ((elems + 3) / 4 * 4) + 8 * RS_BSTAGE);
 }
 
 template <int T>
@@ -59,6 +64,7 @@ struct RsShared {
   uint32_t thr[2];
   uint32_t n_small;
   int ok;
+  uint32_t n_win, n_bk, base_win, base_bk;  // this CTA's staged winners and bucket entries, their slots
   uint32_t wa[T / 32], wb[T / 32 + 1];
   uint32_t hist[HPAD];
   uint32_t small_key[T], small_tie[T];
@@ -122,15 +128,16 @@ __device__ __forceinline__ uint32_t warp_append(uint32_t *cnt, bool take) {
 // The fused selection of one row (k outputs), called by every thread of each
 // of the row's C CTAs after scoring.  shist: the CTA's 11-bit counts of its
 // elements (RB words in shared memory, overwritten).  scratch: shared memory
-// of rs_scratch_bytes(L_cap) bytes (free after scoring).
+// of rs_scratch_bytes(L_cap, elems) bytes (free after scoring), elems the
+// most elements `each` presents in this CTA.
 //   each(fn):  fn(key, token, valid) for every element of this CTA, called
-//              by all 32 lanes of every warp together (warp-uniform trips).
+//              by all 32 lanes of a warp together (warp-uniform trips).
 //   sweep(fn): fn(key, tie, valid) for every element of the whole row, read
 //              from global memory through L2 (the overflow path), called by
 //              every thread in block-uniform sweeps.
 template <int T, class Each, class Sweep>
 __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist, uint8_t *scratch, const RsRow &rw,
-                           int C, int k, int Li, bool ordered, Each &&each, Sweep &&sweep) {
+                           int C, int k, int Li, bool ordered, int elems, Each &&each, Sweep &&sweep) {
   const int tid = threadIdx.x;
   uint32_t *hist1 = rw.zeroed, *hist2 = rw.zeroed + RB, *ctr = rw.zeroed + 2 * RB;
   // 1. the row histogram
@@ -180,8 +187,19 @@ __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist,
   }
   const bool bucket = lvl2 && need1 != in1;  // the 22-bit bucket is split
   int32_t *dst = ordered ? rw.winners : rw.out;
-  // 3. this CTA's sure winners, and the bucket's elements
+  // 3. this CTA's sure winners, and the bucket's elements: staged in shared
+  //    memory, then one global atomic per CTA reserves their slots (the
+  //    winners of a row's CTAs all count on one word: per-warp atomics there
+  //    serialise)
   if (bd.kk > 0) {
+    const int cap_w = (elems + 3) / 4 * 4;
+    uint32_t *st_w = reinterpret_cast<uint32_t *>(scratch);
+    uint2 *st_b = reinterpret_cast<uint2 *>(scratch + 4 * cap_w);
+    if (tid == 0) {
+      sh.n_win = 0;
+      sh.n_bk = 0;
+    }
+    __syncthreads();
     each([&](uint32_t key, int tok, bool valid) {
       const uint32_t k22 = key >> 10;
       bool sel;
@@ -191,12 +209,30 @@ __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist,
         sel = (key >> HIST_SHIFT) >= bd.d0;
       else
         sel = k22 > p22 || (!bucket && k22 == p22);
-      const uint32_t slot = warp_append(ctr + RS_EMIT, valid && sel);
-      if (valid && sel && slot < (uint32_t)k) dst[slot] = tok;
+      const uint32_t s1 = warp_append(&sh.n_win, valid && sel);
+      if (valid && sel && s1 < (uint32_t)cap_w) st_w[s1] = (uint32_t)tok;
       const bool in_b = valid && bucket && k22 == p22;
-      const uint32_t bslot = warp_append(ctr + RS_BUCKET, in_b);
-      if (in_b && bslot < (uint32_t)RS_BCAP) rw.bucket[bslot] = make_uint2(key, (uint32_t)tok);
+      const uint32_t s2 = warp_append(&sh.n_bk, in_b);
+      if (in_b && s2 < (uint32_t)RS_BSTAGE) st_b[s2] = make_uint2(key, (uint32_t)tok);
     });
+    __syncthreads();
+    const uint32_t nw = min(sh.n_win, (uint32_t)cap_w), nbk = sh.n_bk;
+    if (tid == 0) {
+      sh.base_win = nw ? atomicAdd(ctr + RS_EMIT, nw) : 0u;
+      // more bucket entries than staged: count the row past the list's
+      // capacity, so that the last CTA ranks it from the scores instead
+      sh.base_bk = nbk ? atomicAdd(ctr + RS_BUCKET, nbk <= (uint32_t)RS_BSTAGE ? nbk : (uint32_t)RS_BCAP + 1u) : 0u;
+    }
+    __syncthreads();
+    for (uint32_t x = tid; x < nw; x += T) {
+      const uint32_t slot = sh.base_win + x;
+      if (slot < (uint32_t)k) dst[slot] = (int32_t)st_w[x];
+    }
+    if (nbk <= (uint32_t)RS_BSTAGE)
+      for (uint32_t x = tid; x < nbk; x += T) {
+        const uint32_t slot = sh.base_bk + x;
+        if (slot < (uint32_t)RS_BCAP) rw.bucket[slot] = st_b[x];
+      }
   }
   // 4. the last CTA of the row finishes it
   __syncthreads();
@@ -220,14 +256,29 @@ __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist,
       }
       if (tid == 0) sh.n_small = 0;
       __syncthreads();
-      refine<true, T>(sh, P_hi, M_hi, P_lo, M_lo, need1, nb, [&](auto &&fn) {
-        for (uint32_t x = tid; x < nb; x += T) fn(bk[x], bt[x], true);
-      });
       const uint32_t nb_r = (nb + T - 1) / T * T;  // warp-uniform trips
-      for (uint32_t x = tid; x < nb_r; x += T) {
-        const bool v = x < nb && at_least(bk[x], bt[x], P_hi, M_hi, P_lo, M_lo);
+      if (nb <= (uint32_t)T) {
+        // few elements (the continuous case): each one's rank by counting
+        // the bucket's elements above it (composites are unique)
+        const uint32_t x = tid;
+        bool v = false;
+        if (x < nb) {
+          const uint32_t kx = bk[x], lx = bt[x];
+          uint32_t rank = 0;
+          for (uint32_t y = 0; y < nb; ++y) rank += (bk[y] > kx || (bk[y] == kx && bt[y] > lx)) ? 1u : 0u;
+          v = rank < need1;
+        }
         const uint32_t slot = warp_append(ctr + RS_EMIT, v);
         if (v && slot < (uint32_t)k) dst[slot] = (int32_t)(POS_MAX - bt[x]);
+      } else {
+        refine<true, T>(sh, P_hi, M_hi, P_lo, M_lo, need1, nb, [&](auto &&fn) {
+          for (uint32_t x = tid; x < nb; x += T) fn(bk[x], bt[x], true);
+        });
+        for (uint32_t x = tid; x < nb_r; x += T) {
+          const bool v = x < nb && at_least(bk[x], bt[x], P_hi, M_hi, P_lo, M_lo);
+          const uint32_t slot = warp_append(ctr + RS_EMIT, v);
+          if (v && slot < (uint32_t)k) dst[slot] = (int32_t)(POS_MAX - bt[x]);
+        }
       }
     } else {
       // more tied elements than the bucket lists: rank from the row's scores

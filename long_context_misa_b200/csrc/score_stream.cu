@@ -37,6 +37,12 @@ namespace {
 
 constexpr int WARPS = 8;
 constexpr int THREADS = 32 * WARPS;
+constexpr int ROUTE_PREFETCH = 10;  // tiles per warp asked of L2 while an in-kernel router runs
+
+// Ask L2 to fetch [p, p + bytes) (16-byte aligned start, bytes a multiple of 16).
+__device__ __forceinline__ void l2_prefetch(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
 template <int NT, bool FP8>
 struct StreamCfg {
@@ -136,6 +142,17 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
   __shared__ struct { int ok; } r_bar;
   const bool route = route_part != nullptr;
   if (route) {
+    // keep the memory busy while the router runs: ask L2 for this warp's
+    // next tiles (the ring holds only the first)
+    if (lane < ROUTE_PREFETCH) {
+      const int j = NS - 1 + lane;
+      if (j < my_tiles) {
+        const int t0 = (wg + j * nwarps) * TT;
+        const int nrow = min(TT, Li - t0);
+        l2_prefetch(gkeys + (size_t)t0 * ROW, (uint32_t)nrow * ROW);
+        if (FP8 && scale_vec) l2_prefetch(gscale + t0, (uint32_t)((nrow + 3) / 4 * 16));
+      }
+    }
     const int Mi = cdiv(Li, c.B), full = Li / c.B, C = gridDim.x;
     const int m0 = (int)((long long)blockIdx.x * Mi / C), m1 = (int)((long long)(blockIdx.x + 1) * Mi / C);
     if (full < Mi && full >= m0 && full < m1) {  // uniform: this CTA holds the block cut by the prefix end
@@ -150,7 +167,8 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
       cp_async_wait<0>();  // no copy in flight when the CTA leaves
       return;
     }
-    route_rank(qv, i, prow, C, h, r_out, r_keep, r_heads);
+    // the partials are staged in the scores' region (not yet in use), when it holds them
+    route_rank(qv, i, prow, C, h, r_out, r_keep, r_heads, sc_s, fused ? WARPS * max_tiles * TT : 0);
     if (blockIdx.x == 0 && heads_out)
       for (int n = tid; n < h; n += THREADS) heads_out[(size_t)i * h + n] = r_heads[n];
   }
@@ -224,15 +242,16 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
     // the ring is free: the selection's shared state and scratch go there
     RsShared<THREADS> &rs = *reinterpret_cast<RsShared<THREADS> *>(smem);
     uint8_t *scratch = smem + (sizeof(RsShared<THREADS>) + 15) / 16 * 16;
-    const int per_w = max_tiles * TT, total = WARPS * per_w;
+    // every warp visits the elements of its own tiles (token t0 + r of its
+    // j-th tile at [warp][j][r]); trip counts are uniform within the warp
+    const float *sc_w = sc_s + warp * max_tiles * TT;
+    const int n_el = my_tiles * TT;
     auto each = [&](auto &&fn) {
-      for (int x = tid; x < (total + THREADS - 1) / THREADS * THREADS; x += THREADS) {
-        const int w = x / per_w, j = (x % per_w) / TT, r = x % TT;
-        const int wgx = blockIdx.x * WARPS + w;
-        const int tiles_w = wgx < ntile_all ? cdiv(ntile_all - wgx, nwarps) : 0;
-        const int tok = (wgx + j * nwarps) * TT + r;
-        const bool valid = x < total && j < tiles_w && tok < Li;
-        fn(valid ? ordered_key(sc_s[x]) : 0u, tok, valid);
+      for (int x = lane; x < (n_el + 31) / 32 * 32; x += 32) {
+        const int j = x / TT, r = x % TT;
+        const int tok = (wg + j * nwarps) * TT + r;
+        const bool valid = x < n_el && tok < Li;
+        fn(valid ? ordered_key(sc_w[x]) : 0u, tok, valid);
       }
     };
     const float *srow = scores + (size_t)i * ld;
@@ -252,7 +271,8 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
         }
       }
     };
-    row_select<THREADS>(c, rs, shist, scratch, rs_row(fz, i), gridDim.x, fz.k, Li, fz.ordered != 0, each, sweep);
+    row_select<THREADS>(c, rs, shist, scratch, rs_row(fz, i), gridDim.x, fz.k, Li, fz.ordered != 0,
+                        WARPS * max_tiles * TT, each, sweep);
     return;
   }
   uint32_t *rh = row_hist + (size_t)i * TOPK_HIST_BINS;
@@ -301,12 +321,12 @@ StreamPlan plan_nt(const CacheView &c, const QueryView &q, bool fused) {
     return p;
   }
   // fused: the ring (reused for the selection afterwards) and the scores
-  const int region = (std::max(RING, (int)((sizeof(RsShared<THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap)) +
-                      127) / 128 * 128;
   int per_sm = per_sm_for(RING);
   for (int it = 0; it < 3 && per_sm > 0; ++it) {
     const int sp = splits_for(per_sm);
     const int mt = cdiv(ntile, sp * WARPS);
+    const int sel = (int)((sizeof(RsShared<THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap, WARPS * mt * Cfg::TT);
+    const int region = (std::max(RING, sel) + 127) / 128 * 128;
     const int smem = region + WARPS * mt * Cfg::TT * 4;
     const int fit = smem <= max_dyn ? per_sm_for(smem) : 0;
     if (fit >= per_sm) {  // the grid is resident at once

@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(UCfg<FP8, HPQ>::THREADS, 1)
         const float sc = e4m3_head_scale(m);
         wv = wv / sc;  // exact: sc is a power of two
         // input chunk u (8 elements) -> 8 bytes of each term at byte 8u of the row
-#pragma unroll 4
+#pragma unroll 2
         for (int u = 0; u < 16; ++u) {
           const uint4 v = hd >= 0 ? __ldg(row + u) : make_uint4(0u, 0u, 0u, 0u);
           uint2 t1, t2;
@@ -321,14 +321,16 @@ __global__ void __launch_bounds__(UCfg<FP8, HPQ>::THREADS, 1)
         }
         // e4m3 token scales are loaded one tile ahead, so that their latency
         // hides behind a tile of epilogue work instead of stalling the stores
-        const float *scale_row = FP8 ? c.scale + (size_t)seq * c.L_cap : nullptr;
-        float st_next = (FP8 && tau0 < t_end && tau0 * UM_M + r < c.L_cap) ? __ldg(scale_row + tau0 * UM_M + r) : 1.f;
+        // (addresses are recomputed where used rather than held across the
+        // tile: the routed form has 96 registers a thread)
+        const size_t srow0 = (size_t)seq * c.L_cap;
+        float st_next = (FP8 && tau0 < t_end && tau0 * UM_M + r < c.L_cap) ? __ldg(c.scale + srow0 + tau0 * UM_M + r)
+                                                                          : 1.f;
         for (int tau = tau0; tau < t_end; ++tau, ++j_epi) {
           const int buf = j_epi & 1;
           const int t = tau * UM_M + r;
           const float st_scale = st_next;
-          if (FP8 && tau + 1 < t_end) st_next = t + UM_M < c.L_cap ? __ldg(scale_row + t + UM_M) : 1.f;
-          float *out_t = scores + (size_t)g * QPT * ld + t;  // row of query g*QPT + ql at + ql*ld
+          if (FP8 && tau + 1 < t_end) st_next = t + UM_M < c.L_cap ? __ldg(c.scale + srow0 + t + UM_M) : 1.f;
           float *stg = out_smem + (e * 2 + (int)ob) * (Cfg::OUT_BUF / 4);  // [QH][32]
           if (tma_ok) {  // the store that last read this buffer is done reading it
             if (lane == 0) umma::bulk_wait_read<1>();
@@ -338,21 +340,24 @@ __global__ void __launch_bounds__(UCfg<FP8, HPQ>::THREADS, 1)
             if (tma_ok)
               stg[(ql - qa) * 32 + lane] = x;
             else if (t < sh.q_lenp[ql])
-              out_t[(size_t)ql * ld] = x;
+              scores[((size_t)g * QPT + ql) * ld + t] = x;
           };
           if (!umma::wait_bar(&sh.tfull[buf], (j_epi >> 1) & 1, abort, c)) break;
           umma::fence_after();
           const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + buf * UM_N + col0;
           float acc = 0.f;  // running sum of a query wider than one chunk
+          // CH chunks of 32 columns per tensor-memory round trip: two, or one
+          // where the CTA's 18 warps leave 96 registers a thread (routed)
+          constexpr int CH = Cfg::SPLIT == 4 ? 1 : 2;
+#pragma unroll 1
+          for (int ch = 0; ch < Cfg::SPAN / 32; ch += CH) {
+            uint32_t vv[CH][32];
 #pragma unroll
-          for (int ch = 0; ch < Cfg::SPAN / 32; ch += 2) {
-            uint32_t v0[32], v1[32];
-            umma::ld32(taddr + ch * 32, v0);
-            umma::ld32(taddr + ch * 32 + 32, v1);
+            for (int hc = 0; hc < CH; ++hc) umma::ld32(taddr + (ch + hc) * 32, vv[hc]);
             umma::ld_wait();
 #pragma unroll
-            for (int hc = 0; hc < 2; ++hc) {
-              const uint32_t(&v)[32] = hc ? v1 : v0;
+            for (int hc = 0; hc < CH; ++hc) {
+              const uint32_t(&v)[32] = vv[hc];
               const int cb = (ch + hc) * 32;  // first column of this chunk (within the half)
               float part[32 / 4];
 #pragma unroll

@@ -592,77 +592,102 @@ __device__ __forceinline__ Boundary warp_boundary_plain_smem(const uint32_t *h, 
 }
 
 // Sampled boundary bound (tensor-core prefill, where the scoring kernel
-// builds no histogram): one CTA per row counts the top 11 key bits of a
+// builds no histogram): for every row, count the top 11 key bits of a
 // sample of the row -- the whole row up to SMP_N elements, else SMP_BLOCKS
 // blocks of 32 consecutive tokens (one 128-byte line each; scattered single
-// sectors read slowly from HBM) spread evenly over the prefix -- and writes
+// sectors read slowly from HBM) spread evenly over the prefix -- and write
 // thr[row] from the want-th largest sampled element.  want is the sample's
-// expected share of the top k, plus three standard deviations of a count
-// whose 32-token blocks move together, plus 8:
-// the elements at or above thr[row] then number at least k with high
-// probability.  A whole-row sample takes want = min(k, L_i), which is exact.
-// thr[row] is a key bound: the want-th largest sampled key cut to its top 22
-// bits (boundary bin, then the next 11 bits inside it); 0 takes every
-// element.
+// expected share of the top k, plus SMP_Z standard deviations of a count
+// whose 32-token blocks move together, plus 8: the elements at or above
+// thr[row] then number at least k with high probability (a row where they do
+// not is still selected exactly, from its whole score row).  A whole-row
+// sample takes want = min(k, L_i), which is exact.  thr[row] is a key bound:
+// the want-th largest sampled key cut to its top 22 bits (boundary bin, then
+// the next 11 bits inside it); 0 takes every element.
+// Persistent: CTA b takes rows b, b + gridDim.x, ...; the next row's samples
+// are requested before the current row is counted, so their latency hides
+// behind the counting.
 constexpr int SMP_T = 512;
 constexpr int SMP_BL = 32;  // tokens per sample block
 constexpr int SMP_BLOCKS = 256;
 constexpr int SMP_N = SMP_BLOCKS * SMP_BL;
-__global__ void __launch_bounds__(SMP_T) sample_thr_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
-                                                           int k, uint32_t *thr) {
-  grid_dep_sync();
-  __shared__ uint32_t hs[RB];
-  __shared__ Boundary sb;
-  const int row = blockIdx.x;
+constexpr int SMP_PER = SMP_N / SMP_T;  // samples per thread
+constexpr double SMP_Z = 1.5;           // margin, in standard deviations of the sampled count
+
+// Request row `row`'s samples (all of this thread's before any is used).
+__device__ __forceinline__ void sample_load(const CacheView &c, const QueryView &qv, const float *scores,
+                                            long long ld, int row, float (&v)[SMP_PER], int &Li, int &n) {
   int s;
-  const int Li = query_prefix(c, qv, row, &s);
-  for (int b = threadIdx.x; b < RB; b += SMP_T) hs[b] = 0;
-  __syncthreads();
-  const float *srow = scores + (size_t)row * ld;
+  Li = query_prefix(c, qv, row, &s);
   const bool whole = Li <= SMP_N;
-  const int n = whole ? max(Li, 0) : SMP_N;
-  // all of this thread's samples are requested before any is counted
-  constexpr int PER = SMP_N / SMP_T;
-  float v[PER];
+  n = whole ? max(Li, 0) : SMP_N;
+  const float *srow = scores + (size_t)row * ld;
 #pragma unroll
-  for (int u = 0; u < PER; ++u) {
+  for (int u = 0; u < SMP_PER; ++u) {
     const int i = u * SMP_T + (int)threadIdx.x;
     int p = i;
     if (!whole) p = (int)((long long)(i / SMP_BL) * (Li - SMP_BL) / (SMP_BLOCKS - 1)) + (i % SMP_BL);
     v[u] = i < n ? __ldg(srow + p) : 0.f;
   }
+}
+
+__global__ void __launch_bounds__(SMP_T) sample_thr_kernel(CacheView c, QueryView qv, const float *scores, long long ld,
+                                                           int k, uint32_t *thr) {
+  grid_dep_sync();
+  __shared__ uint32_t hs[RB];
+  __shared__ Boundary sb;
+  int row = blockIdx.x;
+  if (row >= qv.n_q) return;  // uniform
+  float v[SMP_PER];
+  int Li, n;
+  sample_load(c, qv, scores, ld, row, v, Li, n);
+  while (true) {
+    const int next = row + (int)gridDim.x;
+    float vn[SMP_PER];
+    int Ln = 0, nn = 0;
+    if (next < qv.n_q) sample_load(c, qv, scores, ld, next, vn, Ln, nn);
+    for (int b = threadIdx.x; b < RB; b += SMP_T) hs[b] = 0;
+    __syncthreads();
 #pragma unroll
-  for (int u = 0; u < PER; ++u)
-    if (u * SMP_T + (int)threadIdx.x < n) atomicAdd(&hs[ordered_key(v[u]) >> HIST_SHIFT], 1u);
-  __syncthreads();
-  uint32_t want = (uint32_t)min(k, max(Li, 0));
-  if (!whole) {
-    const double r = (double)k * SMP_N / Li;
-    want = (uint32_t)min(2.0 * SMP_N, ceil(r + 3.0 * sqrt((double)SMP_BL * r) + 8.0));
-  }
-  if (threadIdx.x < 32) {
-    const Boundary b = warp_boundary_plain_smem(hs, (int)want);
-    if (threadIdx.x == 0) sb = b;
-  }
-  __syncthreads();
-  const Boundary b = sb;
-  if (b.all_in) {
-    if (threadIdx.x == 0) thr[row] = 0u;
-    return;
-  }
-  // second level: the next 11 key bits of the samples inside the boundary bin
-  for (int x = threadIdx.x; x < RB; x += SMP_T) hs[x] = 0;
-  __syncthreads();
+    for (int u = 0; u < SMP_PER; ++u)
+      if (u * SMP_T + (int)threadIdx.x < n) atomicAdd(&hs[ordered_key(v[u]) >> HIST_SHIFT], 1u);
+    __syncthreads();
+    uint32_t want = (uint32_t)min(k, max(Li, 0));
+    if (Li > SMP_N) {
+      const double r = (double)k * SMP_N / Li;
+      want = (uint32_t)min(2.0 * SMP_N, ceil(r + SMP_Z * sqrt((double)SMP_BL * r) + 8.0));
+    }
+    if (threadIdx.x < 32) {
+      const Boundary b = warp_boundary_plain_smem(hs, (int)want);
+      if (threadIdx.x == 0) sb = b;
+    }
+    __syncthreads();
+    const Boundary b = sb;
+    if (b.all_in) {
+      if (threadIdx.x == 0) thr[row] = 0u;
+    } else {
+      // second level: the next 11 key bits of the samples inside the boundary bin
+      for (int x = threadIdx.x; x < RB; x += SMP_T) hs[x] = 0;
+      __syncthreads();
 #pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    const int i = u * SMP_T + (int)threadIdx.x;
-    const uint32_t key = ordered_key(v[u]);
-    if (i < n && (key >> HIST_SHIFT) == b.d0) atomicAdd(&hs[(key >> 10) & (RB - 1)], 1u);
-  }
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    const Boundary b2 = warp_boundary_plain_smem(hs, (int)(want - b.above));
-    if (threadIdx.x == 0) thr[row] = (b.d0 << HIST_SHIFT) | ((b2.all_in ? 0u : b2.d0) << 10);
+      for (int u = 0; u < SMP_PER; ++u) {
+        const int i = u * SMP_T + (int)threadIdx.x;
+        const uint32_t key = ordered_key(v[u]);
+        if (i < n && (key >> HIST_SHIFT) == b.d0) atomicAdd(&hs[(key >> 10) & (RB - 1)], 1u);
+      }
+      __syncthreads();
+      if (threadIdx.x < 32) {
+        const Boundary b2 = warp_boundary_plain_smem(hs, (int)(want - b.above));
+        if (threadIdx.x == 0) thr[row] = (b.d0 << HIST_SHIFT) | ((b2.all_in ? 0u : b2.d0) << 10);
+      }
+    }
+    __syncthreads();  // hs and sb free for the next row
+    if (next >= qv.n_q) break;
+    row = next;
+    Li = Ln;
+    n = nn;
+#pragma unroll
+    for (int u = 0; u < SMP_PER; ++u) v[u] = vn[u];
   }
 }
 
@@ -994,7 +1019,8 @@ cudaError_t launch_topk(const CacheView &c, const QueryView &q, const float *sco
     // histogram's place), the elements at or above it listed, the list
     // counted and selected in shared memory
     uint32_t *thr = row_hist;
-    e = launch_kernel(sample_thr_kernel, dim3(q.n_q), dim3(SMP_T), 0, s, c, q, scores, ld, k, thr);
+    // persistent: the resident CTAs (two per SM at 512 threads) walk the rows
+    e = launch_kernel(sample_thr_kernel, dim3(std::min(q.n_q, 2 * sms)), dim3(SMP_T), 0, s, c, q, scores, ld, k, thr);
     if (e != cudaSuccess) return e;
     const int tchunk = 4 * FT_T * FT_V * 2;  // two sweeps per CTA
     e = launch_kernel(filter_thr_kernel, dim3(cdiv(c.L_cap, tchunk), q.n_q), dim3(FT_T), 0, s, c, q, scores, ld, thr,

@@ -75,6 +75,7 @@ def _load() -> ctypes.CDLL:
         "misa_version": (I32, []),
         "misa_debug_fail_next": (None, [I32]),
         "misa_debug_time_scoring": (None, [P, P]),
+        "misa_debug_select_in_kernel": (None, [I32]),
         "misa_debug_wait_timeout": (I32, [P, ctypes.c_uint64, P]),
     }
     for name, (res, args) in sig.items():
@@ -106,6 +107,11 @@ def version() -> int:
 
 def debug_fail_next(n: int) -> None:
     _lib.misa_debug_fail_next(n)
+
+
+def debug_select_in_kernel(on: bool) -> None:
+    """Select the top k inside the scoring kernels wherever shapes allow (see misa.h)."""
+    _lib.misa_debug_select_in_kernel(1 if on else 0)
 
 
 def debug_time_scoring(start=None, stop=None) -> None:
@@ -372,10 +378,10 @@ class MisaDaggerDecode:
     """
 
     # kernels of one step when the batch runs fused (decode shapes whose
-    # scoring grids fit on the device at once): the append (which also clears
-    # the selections' counters), routing + routed scoring + top-k', and the
-    # all-head re-rank + top-k
-    LAUNCHES = 3
+    # scoring grid fits on the device at once): the append (which also clears
+    # the counting words), routing + routed scoring + top-k', the all-head
+    # re-rank, and the final top-k
+    LAUNCHES = 4
 
     def __init__(self, cache: KeyCache, qs: Queries, h: int, k_prime: int, k: int, new_keys: torch.Tensor,
                  new_scale: Optional[torch.Tensor], new_pos: torch.Tensor):
