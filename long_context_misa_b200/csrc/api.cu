@@ -408,7 +408,13 @@ misa_status dagger_body(const char *who, const misa_cache *cache, const misa_que
                           false);
     if (e != cudaSuccess) return cuda_fail(e, who);
   }
-  // fine pass: every head on the candidates, ascending final top-k
+  // fine pass: every head on the candidates, ascending final top-k; one
+  // cluster kernel when a cluster holds a query's candidates
+  if (!f2 && misa::rerank_cluster_applies(c, q, k_prime, k)) {
+    e = misa::launch_rerank_cluster(c, q, cand, k_prime, k, topk, nullptr, 0, stream);
+    if (e != cudaSuccess) return cuda_fail(e, who);
+    return MISA_OK;
+  }
   const misa::FusedTopk fzr = fused_args(fz2, bucket, winners, topk, k, true);
   e = misa::launch_score_mma(c, q, nullptr, q.H, cand, k_prime, rscores, k_prime, rhist, stream, f2 ? &fzr : nullptr);
   if (e != cudaSuccess) return cuda_fail(e, who);
@@ -555,6 +561,13 @@ misa_status misa_rerank_topk(const misa_cache *cache, const misa_queries *qs, co
   uint8_t *bucket = after + (scores_out ? 0 : round_up(sizeof(float) * (size_t)qs->n_q * k_prime));
   uint8_t *winners = bucket + ws_fz_bucket(qs);
   const bool fused = g_select_in_kernel.load() && misa::score_fusable(c, q, nullptr, q.H, cand, k_prime);
+  if (!fused && misa::rerank_cluster_applies(c, q, k_prime, k)) {
+    cudaError_t e = timed_scoring(stream, [&] {
+      return misa::launch_rerank_cluster(c, q, cand, k_prime, k, topk, scores_out, k_prime, stream);
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");
+    return MISA_OK;
+  }
   cudaError_t e = fused ? misa::launch_zero(fz_zero, (size_t)qs->n_q * misa::FUSED_ZERO_WORDS, stream)
                         : misa::launch_zero(hist, (size_t)qs->n_q * misa::TOPK_HIST_BINS, stream);
   if (e != cudaSuccess) return cuda_fail(e, "misa_rerank_topk");

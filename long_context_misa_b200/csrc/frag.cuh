@@ -19,6 +19,8 @@
 //   the same fp32 accumulator; 2^-e_n is folded into the head weight.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace misa {
@@ -80,13 +82,41 @@ __device__ __forceinline__ float e4m3_head_scale(float amax) {
 // Threads [0, NTHR) must all call; `sync` is a barrier over exactly those
 // threads, and one more is needed before the fragments are read.  Loops have
 // fixed trip counts so every load is issued before it is used.
-template <int NT, bool FP8, int NTHR, class Sync>
+// QSmem: the query already sits in shared memory (qrow(j): head j's row,
+// w_in: its H weights); QGlobal: it is read from qv.
+struct QGlobal {};
+template <class QRow>
+struct QSmem {
+  QRow qrow;
+  const float *w_in;
+};
+
+template <int NT, bool FP8, int NTHR, class Sync, class QSrc = QGlobal>
 __device__ __forceinline__ void build_query_frags(const CacheView &c, const QueryView &qv, int i,
                                                   const int32_t *heads, int h, uint2 *bfrag, float *w_s,
                                                   float *scale_s, int tid, Sync sync,
-                                                  const int32_t *sheads = nullptr) {
+                                                  const int32_t *sheads = nullptr, QSrc qsrc = QSrc()) {
   using F = FragCfg<FP8>;
+  constexpr bool GQ = std::is_same<QSrc, QGlobal>::value;
   const int H = qv.H;
+  auto row_of = [&](int j) -> const uint16_t * {
+    if constexpr (GQ)
+      return qv.q + ((size_t)i * H + j) * D;
+    else
+      return qsrc.qrow(j);
+  };
+  auto ld16 = [&](const void *p) -> uint4 {
+    if constexpr (GQ)
+      return __ldg(reinterpret_cast<const uint4 *>(p));
+    else
+      return *reinterpret_cast<const uint4 *>(p);
+  };
+  auto ld8 = [&](const void *p) -> uint2 {
+    if constexpr (GQ)
+      return __ldg(reinterpret_cast<const uint2 *>(p));
+    else
+      return *reinterpret_cast<const uint2 *>(p);
+  };
   const int h_eff = (heads || sheads) ? h : H;
   auto head_of = [&](int n) -> int {
     int j = sheads ? sheads[n] : heads ? __ldg(heads + (size_t)i * h + n) : n;
@@ -101,10 +131,10 @@ __device__ __forceinline__ void build_query_frags(const CacheView &c, const Quer
   if (FP8) {
     float sc = 1.f;
     if (n_me < NT * 8 && n_me < h_eff) {
-      const uint4 *row = reinterpret_cast<const uint4 *>(qv.q + ((size_t)i * H + head_of(n_me)) * D);
+      const uint4 *row = reinterpret_cast<const uint4 *>(row_of(head_of(n_me)));
       uint4 v[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) v[u] = __ldg(row + u);
+      for (int u = 0; u < 16; ++u) v[u] = ld16(row + u);
       float m = 0.f;
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
@@ -138,13 +168,13 @@ __device__ __forceinline__ void build_query_frags(const CacheView &c, const Quer
     const int kt = (e >> 5) / NT, c4 = e & 3;
     raw[it] = make_uint4(0u, 0u, 0u, 0u);
     if (hd[it] >= 0) {
-      const uint16_t *qrow = qv.q + ((size_t)i * H + hd[it]) * D;
+      const uint16_t *qrow = row_of(hd[it]);
       if (FP8) {
         // k-tile kt = 2ch + u: a0/b0 <- elements 64ch + 16c + 8u + 0..3, a2/b1 <- + 4..7
-        raw[it] = __ldg(reinterpret_cast<const uint4 *>(qrow + 64 * (kt >> 1) + 16 * c4 + 8 * (kt & 1)));
+        raw[it] = ld16(qrow + 64 * (kt >> 1) + 16 * c4 + 8 * (kt & 1));
       } else {
         // k-tile kt = 2ch + u: a0/b0 <- elements 32ch + 8c + 4u + 0..1, a2/b1 <- + 2..3
-        const uint2 v = __ldg(reinterpret_cast<const uint2 *>(qrow + 32 * (kt >> 1) + 8 * c4 + 4 * (kt & 1)));
+        const uint2 v = ld8(qrow + 32 * (kt >> 1) + 8 * c4 + 4 * (kt & 1));
         raw[it].x = v.x;
         raw[it].y = v.y;
       }
@@ -164,7 +194,10 @@ __device__ __forceinline__ void build_query_frags(const CacheView &c, const Quer
   if (n_me < NT * 8) {
     float wv = 0.f;
     if (n_me < h_eff) {
-      wv = __ldg(qv.w + (size_t)i * H + head_of(n_me));
+      if constexpr (GQ)
+        wv = __ldg(qv.w + (size_t)i * H + head_of(n_me));
+      else
+        wv = qsrc.w_in[head_of(n_me)];
       if (FP8) wv /= scale_s[n_me];  // exact: power of two
     }
     w_s[n_me] = wv;

@@ -80,6 +80,15 @@ cudaError_t launch_rerank_umma(const CacheView &c, const QueryView &q, const int
                                const int32_t *gather, int n_cols, float *scores, long long ld, uint32_t *row_hist,
                                cudaStream_t s, const FusedTopk *fused = nullptr);
 bool rerank_fusable(const CacheView &c, const QueryView &q, const int32_t *heads, int h, int n_cols);
+// The whole fine stage (all heads on the n_cols candidates of each query,
+// then its top k in ascending token order, -1 padded) in one launch: one
+// thread-block cluster per query (rerank_cluster.cu).  Applies when a
+// cluster holds the candidates (k' <= 8192 for e4m3 keys and up to 64 heads)
+// and the device can run one; scores (optional, row pitch ld) receives every
+// valid candidate's score.
+bool rerank_cluster_applies(const CacheView &c, const QueryView &q, int n_cols, int k);
+cudaError_t launch_rerank_cluster(const CacheView &c, const QueryView &q, const int32_t *gather, int n_cols, int k,
+                                  int32_t *out, float *scores, long long ld, cudaStream_t s);
 // the same for prefix rows of e4m3 caches with 32 or more scoring heads
 bool dense_fusable(const CacheView &c, const QueryView &q, const int32_t *heads, int h);
 

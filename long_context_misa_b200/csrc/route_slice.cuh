@@ -45,42 +45,45 @@ __device__ __forceinline__ void rsl_split(float x, float y, uint32_t &hi, uint32
 // out[j] = sum_m ReLU(q_j . kbar_m) for j < H, in shared memory.  Blocks
 // below `full` come from the pool; block `full` (the one cut by the prefix
 // end) from tail[128] (shared, its mean over the present tokens).  wsum:
-// shared [NW][MISA_MAX_H].  Every thread of the CTA (NW warps) calls.
-template <int NW>
-__device__ void route_slice(const CacheView &c, const QueryView &qv, int i, int s, int m0, int m1, int full,
-                            const float *tail, float *wsum, float *out) {
+// shared [NW][MISA_MAX_H].  qrow(j): head j's query row (128 bf16) in shared
+// memory, readable once `ready` has run.  Every thread of the CTA (NW warps)
+// calls; `ready` is called once by every thread, after this warp's first
+// pool loads are in flight and before the first query read (it may hold a
+// barrier).
+template <int NW, class QRow, class Ready>
+__device__ void route_slice(const CacheView &c, int s, int H, int m0, int m1, int full, const float *tail,
+                            float *wsum, float *out, QRow &&qrow, Ready &&ready) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, cq = lane & 3;
-  const int H = qv.H, MT = cdiv(H, 16);
+  const int MT = cdiv(H, 16);
   const int M_cap = cdiv(c.L_cap, c.B);
-  const uint16_t *qrow = qv.q + (size_t)i * H * D;
   // warp w keeps one m-tile of 16 heads (w % MT) and takes every
-  // (NW / MT)-th n-tile of 8 blocks: all loads of an n-tile are issued
-  // together, and each warp's sums need no more than two accumulators
+  // (NW / MT)-th n-tile of 8 blocks, two n-tiles per round: the loads of a
+  // round are all issued before its first product
   const int wpm = NW / MT;  // warps per m-tile (MT divides NW: MT in {1, 2, 4, 8})
   const int mt = warp % MT;
   const int ha = 16 * mt + g, hb = ha + 8;
   float racc0 = 0.f, racc1 = 0.f;  // heads ha, hb
-  for (int nt = warp / MT; m0 + 8 * nt < m1; nt += wpm) {
+  bool first = true;
+  auto load = [&](int nt, float4 (&x)[4][2]) {
     const int m = m0 + 8 * nt + g;  // this lane's block (B column g)
     const float *prow = m >= m1 ? nullptr : m < full ? c.pool + ((size_t)s * M_cap + m) * D : m == full ? tail : nullptr;
-    float4 x[4][2];
-    uint4 qa[4], qb[4];
 #pragma unroll
     for (int ch = 0; ch < 4; ++ch) {
       x[ch][0] = prow ? *reinterpret_cast<const float4 *>(prow + 32 * ch + 8 * cq) : make_float4(0.f, 0.f, 0.f, 0.f);
       x[ch][1] = prow ? *reinterpret_cast<const float4 *>(prow + 32 * ch + 8 * cq + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
-      qa[ch] = ha < H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)ha * D + 32 * ch + 8 * cq))
-                      : make_uint4(0u, 0u, 0u, 0u);
-      qb[ch] = hb < H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)hb * D + 32 * ch + 8 * cq))
-                      : make_uint4(0u, 0u, 0u, 0u);
     }
+  };
+  auto product = [&](const float4 (&x)[4][2]) {
+    const uint16_t *qa_row = qrow(ha < H ? ha : 0), *qb_row = qrow(hb < H ? hb : 0);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ch = 0; ch < 4; ++ch) {
+      const uint4 qa = ha < H ? *reinterpret_cast<const uint4 *>(qa_row + 32 * ch + 8 * cq) : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 qb = hb < H ? *reinterpret_cast<const uint4 *>(qb_row + 32 * ch + 8 * cq) : make_uint4(0u, 0u, 0u, 0u);
       uint32_t bh0, bl0, bh1, bl1;
-      const uint32_t a0[4] = {qa[ch].x, qb[ch].x, qa[ch].y, qb[ch].y};  // k-tile 2ch
-      const uint32_t a1[4] = {qa[ch].z, qb[ch].z, qa[ch].w, qb[ch].w};  // k-tile 2ch + 1
+      const uint32_t a0[4] = {qa.x, qb.x, qa.y, qb.y};  // k-tile 2ch
+      const uint32_t a1[4] = {qa.z, qb.z, qa.w, qb.w};  // k-tile 2ch + 1
       rsl_split(x[ch][0].x, x[ch][0].y, bh0, bl0);
       rsl_split(x[ch][0].z, x[ch][0].w, bh1, bl1);
       mma_bf16_16816(acc, a0, bh0, bh1);
@@ -94,6 +97,21 @@ __device__ void route_slice(const CacheView &c, const QueryView &qv, int i, int 
     // absent blocks multiplied zero keys and add nothing
     racc0 += fmaxf(acc[0], 0.f) + fmaxf(acc[1], 0.f);
     racc1 += fmaxf(acc[2], 0.f) + fmaxf(acc[3], 0.f);
+  };
+  const int rounds = cdiv(max(m1 - m0, 0), 8 * 2 * wpm);  // the same in every warp
+  for (int r = 0; r < rounds || first; ++r) {
+    const int nt0 = warp / MT + 2 * wpm * r, nt1 = nt0 + wpm;
+    float4 x0[4][2], x1[4][2];
+    load(nt0, x0);
+    load(nt1, x1);
+    if (first) {
+      ready();
+      first = false;
+    }
+    if (r < rounds) {
+      product(x0);
+      product(x1);
+    }
   }
   // the four lanes of a row group hold the same heads' sums over different blocks
   racc0 += __shfl_xor_sync(0xffffffffu, racc0, 1);
@@ -115,7 +133,8 @@ __device__ void route_slice(const CacheView &c, const QueryView &qv, int i, int 
 }
 
 // After the row barrier: the query's importances from the C partial sums
-// (part[cc * H + j], written by the C CTAs), r_j = |w_j| * sum, and its h
+// (part[cc * H + j], written by the C CTAs), r_j = |w_j| * sum (w_s: the
+// query's H head weights in shared memory), and its h
 // best heads in ascending order into sheads (head j is kept iff fewer than h
 // heads beat it: larger r, or equal r and a lower index).  Four threads per
 // head: each adds a quarter of the partials in order, the quarters are
@@ -123,12 +142,25 @@ __device__ void route_slice(const CacheView &c, const QueryView &qv, int i, int 
 // r_s, keep_s: shared [MISA_MAX_H]; stage: shared scratch of stage_cap floats
 // for the partials; every thread calls (blockDim.x a multiple of 32, at
 // least H).
-__device__ void route_rank(const QueryView &qv, int i, const float *part, int C, int h, float *r_s, int *keep_s,
+__device__ void route_rank(int H, const float *w_s, const float *part, int C, int h, float *r_s, int *keep_s,
                            int32_t *sheads, float *stage, int stage_cap) {
-  const int tid = threadIdx.x, H = qv.H, lane = tid & 31;
+  const int tid = threadIdx.x, lane = tid & 31;
   const bool staged = C * H <= stage_cap;
-  if (staged) {  // every partial requested at once
-    for (int x = tid; x < C * H; x += blockDim.x) stage[x] = __ldcg(part + x);
+  if (staged) {  // every partial requested at once, eight loads in flight per thread
+    constexpr int UL = 8;
+    for (int x0 = tid; x0 < C * H; x0 += UL * (int)blockDim.x) {
+      float v[UL];
+#pragma unroll
+      for (int u = 0; u < UL; ++u) {
+        const int x = x0 + u * (int)blockDim.x;
+        v[u] = x < C * H ? __ldcg(part + x) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < UL; ++u) {
+        const int x = x0 + u * (int)blockDim.x;
+        if (x < C * H) stage[x] = v[u];
+      }
+    }
     __syncthreads();
   }
   const int qq = tid & 3;  // quarter
@@ -138,13 +170,14 @@ __device__ void route_rank(const QueryView &qv, int i, const float *part, int C,
     const int j = jb + (tid >> 2);
     float acc = 0.f;
     if (j < H)
+#pragma unroll 8
       for (int cc = c0; cc < c1; ++cc) acc += staged ? stage[cc * H + j] : __ldcg(part + (size_t)cc * H + j);
     // quarters of a head sit in four consecutive lanes: (q0 + q1) + (q2 + q3)
     const float o1 = __shfl_xor_sync(0xffffffffu, acc, 1);
     const float pair = (qq & 1) ? o1 + acc : acc + o1;
     const float o2 = __shfl_xor_sync(0xffffffffu, pair, 2);
     const float tot = (qq & 2) ? o2 + pair : pair + o2;
-    if (j < H && qq == 0) r_s[j] = fabsf(__ldg(qv.w + (size_t)i * H + j)) * tot;
+    if (j < H && qq == 0) r_s[j] = fabsf(w_s[j]) * tot;
   }
   __syncthreads();
   // rank: each of the four threads counts the heads of a quarter that beat j

@@ -37,12 +37,6 @@ namespace {
 
 constexpr int WARPS = 8;
 constexpr int THREADS = 32 * WARPS;
-constexpr int ROUTE_PREFETCH = 10;  // tiles per warp asked of L2 while an in-kernel router runs
-
-// Ask L2 to fetch [p, p + bytes) (16-byte aligned start, bytes a multiple of 16).
-__device__ __forceinline__ void l2_prefetch(const void *p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
 
 template <int NT, bool FP8>
 struct StreamCfg {
@@ -130,29 +124,36 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
     }
     cp_async_commit();
   };
-#pragma unroll
-  for (int j = 0; j < NS - 1; ++j) issue(j);  // start streaming before the query set-up
-
-  // routing in front of the scan: the keys stream in meanwhile
+  // routing in front of the scan
   __shared__ float r_tail[D];                   // the causal tail block's mean
   __shared__ float r_wsum[WARPS * MISA_MAX_H];  // per-warp partial sums
   __shared__ float r_out[MISA_MAX_H];           // this CTA's partials, then the importances
+  __shared__ float r_w[MISA_MAX_H];             // the query's head weights
   __shared__ int r_keep[MISA_MAX_H];
   __shared__ int32_t r_heads[NT * 8];
   __shared__ struct { int ok; } r_bar;
   const bool route = route_part != nullptr;
-  if (route) {
-    // keep the memory busy while the router runs: ask L2 for this warp's
-    // next tiles (the ring holds only the first)
-    if (lane < ROUTE_PREFETCH) {
-      const int j = NS - 1 + lane;
-      if (j < my_tiles) {
-        const int t0 = (wg + j * nwarps) * TT;
-        const int nrow = min(TT, Li - t0);
-        l2_prefetch(gkeys + (size_t)t0 * ROW, (uint32_t)nrow * ROW);
-        if (FP8 && scale_vec) l2_prefetch(gscale + t0, (uint32_t)((nrow + 3) / 4 * 16));
-      }
+  // with routing, the query's H rows wait in the ring's last stage (unused
+  // until the scan starts), RPW rows per warp; the host checks H <= WARPS * RPW
+  constexpr int RPW = Cfg::STAGE / (2 * D);
+  const uint32_t q_stage = smem_addr(smem) + (NS - 1) * Cfg::STAGE;
+  auto qrow_s = [&](int j) -> const uint16_t * {
+    return reinterpret_cast<const uint16_t *>(smem + (j / RPW) * Cfg::WARP_BYTES + (NS - 1) * Cfg::STAGE +
+                                              (j % RPW) * 2 * D);
+  };
+  if (!route) {
+#pragma unroll
+    for (int j = 0; j < NS - 1; ++j) issue(j);  // start streaming before the query set-up
+  } else {
+    // the router's loads go first: the query rows and weights here, this
+    // CTA's pool blocks inside route_slice; the ring's first tiles follow
+    for (int x = tid; x < qv.H * 16; x += THREADS) {
+      const int j = x >> 4, u = x & 15;
+      cp_async16(q_stage + (j / RPW) * Cfg::WARP_BYTES + (j % RPW) * 2 * D + 16 * u,
+                 qv.q + ((size_t)i * qv.H + j) * D + 8 * u);
     }
+    cp_async_commit();
+    for (int j = tid; j < qv.H; j += THREADS) r_w[j] = __ldg(qv.w + (size_t)i * qv.H + j);
     const int Mi = cdiv(Li, c.B), full = Li / c.B, C = gridDim.x;
     const int m0 = (int)((long long)blockIdx.x * Mi / C), m1 = (int)((long long)(blockIdx.x + 1) * Mi / C);
     if (full < Mi && full >= m0 && full < m1) {  // uniform: this CTA holds the block cut by the prefix end
@@ -160,7 +161,12 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
       if (tid < D) r_tail[tid] *= 1.f / (float)(Li - full * c.B);
       __syncthreads();
     }
-    route_slice<WARPS>(c, qv, i, s, m0, m1, full, r_tail, r_wsum, r_out);
+    route_slice<WARPS>(c, s, qv.H, m0, m1, full, r_tail, r_wsum, r_out, qrow_s, [&] {
+#pragma unroll
+      for (int j = 0; j < NS - 1; ++j) issue(j);
+      cp_async_wait<NS - 1>();  // the query rows (the group before the ring's)
+      __syncthreads();
+    });
     float *prow = route_part + (size_t)i * C * qv.H;
     for (int j = tid; j < qv.H; j += THREADS) prow[(size_t)blockIdx.x * qv.H + j] = r_out[j];
     if (!row_barrier(r_bar, fz.zeroed + (size_t)i * RS_ZERO_WORDS + 2 * RB + RS_ROUTE, (uint32_t)C, c)) {
@@ -168,14 +174,17 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
       return;
     }
     // the partials are staged in the scores' region (not yet in use), when it holds them
-    route_rank(qv, i, prow, C, h, r_out, r_keep, r_heads, sc_s, fused ? WARPS * max_tiles * TT : 0);
+    route_rank(qv.H, r_w, prow, C, h, r_out, r_keep, r_heads, sc_s, fused ? WARPS * max_tiles * TT : 0);
     if (blockIdx.x == 0 && heads_out)
       for (int n = tid; n < h; n += THREADS) heads_out[(size_t)i * h + n] = r_heads[n];
   }
   for (int b = tid; b < TOPK_HIST_BINS; b += THREADS) shist[b] = 0;
 
-  build_query_frags<NT, FP8, THREADS>(c, qv, i, heads, h, bfrag, w_s, scale_s, tid, [] { __syncthreads(); },
-                                      route ? r_heads : nullptr);
+  if (route)
+    build_query_frags<NT, FP8, THREADS>(c, qv, i, heads, h, bfrag, w_s, scale_s, tid, [] { __syncthreads(); },
+                                        r_heads, QSmem<decltype(qrow_s)>{qrow_s, r_w});
+  else
+    build_query_frags<NT, FP8, THREADS>(c, qv, i, heads, h, bfrag, w_s, scale_s, tid, [] { __syncthreads(); });
   __syncthreads();
   float wr[NT][2];
 #pragma unroll
@@ -343,13 +352,21 @@ StreamPlan plan_nt(const CacheView &c, const QueryView &q, bool fused) {
   return p;
 }
 
+// With routing in the kernel the query's rows are staged in the ring's last
+// stage: RPW rows of 2 * D bytes per warp.
+template <int NT, bool FP8>
+constexpr int route_q_rows() {
+  return WARPS * (StreamCfg<NT, FP8>::STAGE / (2 * D));
+}
+
 template <int NT, bool FP8>
 cudaError_t launch_nt(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
                       long long ld, uint32_t *row_hist, cudaStream_t s, const FusedTopk *fz, float *route_part,
                       int32_t *heads_out) {
   const StreamPlan p = plan_nt<NT, FP8>(c, q, fz != nullptr);
   if (!p.ok) return cudaErrorInvalidConfiguration;
-  if (route_part && (!fz || (long long)p.splits * q.n_q > route_part_slots())) return cudaErrorInvalidValue;
+  if (route_part && (!fz || (long long)p.splits * q.n_q > route_part_slots() || q.H > route_q_rows<NT, FP8>()))
+    return cudaErrorInvalidValue;
   const int scale_vec = FP8 && (reinterpret_cast<uintptr_t>(c.scale) & 15) == 0 && c.L_cap % 4 == 0;
   FusedTopk none = {};
   return launch_kernel(score_stream_kernel<NT, FP8>, dim3(p.splits, q.n_q), dim3(THREADS), p.smem, s, c, q, heads, h,
@@ -392,7 +409,8 @@ bool score_stream_fusable(const CacheView &c, const QueryView &q, const int32_t 
 #define MISA_STREAM_CASE(N)                                                                     \
   case N: {                                                                                     \
     const StreamPlan p = c.fp8 ? plan_nt<N, true>(c, q, true) : plan_nt<N, false>(c, q, true); \
-    return p.ok && (!route || (long long)p.splits * q.n_q <= route_part_slots());              \
+    const int rows = c.fp8 ? route_q_rows<N, true>() : route_q_rows<N, false>();                \
+    return p.ok && (!route || ((long long)p.splits * q.n_q <= route_part_slots() && q.H <= rows)); \
   }
   switch (route ? stream_nt_h(h) : stream_nt(q, heads, h)) {
     MISA_STREAM_CASE(1)

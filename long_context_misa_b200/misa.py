@@ -378,10 +378,11 @@ class MisaDaggerDecode:
     """
 
     # kernels of one step when the batch runs fused (decode shapes whose
-    # scoring grid fits on the device at once): the append (which also clears
-    # the counting words), routing + routed scoring + top-k', the all-head
-    # re-rank, and the final top-k
-    LAUNCHES = 4
+    # scoring grid fits on the device at once and whose k' candidates fit one
+    # thread-block cluster per query): the append (which also clears the
+    # counting words), routing + routed scoring + top-k', and the all-head
+    # re-rank with the final top-k
+    LAUNCHES = 3
 
     def __init__(self, cache: KeyCache, qs: Queries, h: int, k_prime: int, k: int, new_keys: torch.Tensor,
                  new_scale: Optional[torch.Tensor], new_pos: torch.Tensor):
