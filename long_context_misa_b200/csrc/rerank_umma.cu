@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
   extern __shared__ uint8_t rr_raw[];
   // the tiles and Q', or (a fused selection, afterwards) its state and scratch
   const uint32_t sel_bytes =
-      (uint32_t)((sizeof(RsShared<RR_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap, T * RR_M);
+      (uint32_t)((sizeof(RsShared<RR_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap, T * RR_M, RR_THREADS);
   const uint32_t need = max((uint32_t)(Cfg::SMEM - 1024), fz.zeroed ? sel_bytes : 0u);
   uint8_t *base = aligned_smem_base(rr_raw, need, c);  // 1024-aligned (swizzle atoms)
   if (!base) return;
@@ -531,7 +531,7 @@ DensePlan plan_dense(const CacheView &c, const QueryView &q, bool fused) {
   p.max_tiles = cdiv(n_tiles, p.nparts);
   p.smem = dense_smem<HN>(p.max_tiles, fused);
   // a fused selection's state and scratch reuse the ring
-  const int sel = (int)((sizeof(RsShared<DS_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap, p.max_tiles * RR_M);
+  const int sel = (int)((sizeof(RsShared<DS_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap, p.max_tiles * RR_M, DS_THREADS);
   p.ok = p.smem <= max_dyn && (!fused || ((long long)p.nparts * q.n_q <= sms && sel <= DSCfg<HN>::RING)) && c.fp8 &&
          umma::encoder_available() && (reinterpret_cast<uintptr_t>(c.keys) & 15u) == 0;
   return p;
@@ -555,7 +555,7 @@ cudaError_t launch_dense(const CacheView &c, const QueryView &q, const int32_t *
 template <bool FP8, int HN, int TT>
 int rerank_smem(const CacheView &c, bool fused) {
   using Cfg = RCfg<FP8, HN, TT>;
-  const int sel = 1024 + (int)((sizeof(RsShared<RR_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap, TT * RR_M);
+  const int sel = 1024 + (int)((sizeof(RsShared<RR_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap, TT * RR_M, RR_THREADS);
   return fused ? std::max(Cfg::SMEM, sel) : Cfg::SMEM;
 }
 

@@ -50,11 +50,14 @@ constexpr int RS_BSTAGE = 512;  // bucket entries a CTA stages before reserving 
 
 // Shared scratch beyond RsShared, used in turn for: a CTA's winners and
 // bucket entries before they are written out (elems: the most elements a
-// CTA holds); the last CTA's staged bucket; the token bitmap of an
-// ascending output.
+// CTA of T threads holds; every warp stages its winners in a private part
+// of cdiv(elems, T) * 32 words, which holds the elements a warp visits when
+// `each` deals them per warp or in block-wide sweeps); the last CTA's staged
+// bucket; the token bitmap of an ascending output.
 __host__ __device__ constexpr int rs_max3(int a, int b, int c) { return a > b ? (a > c ? a : c) : (b > c ? b : c); }
-__host__ __device__ constexpr int rs_scratch_bytes(int L_cap, int elems) {
-  return rs_max3(8 * RS_BCAP, 4 * ((L_cap + 31) / 32 + 4), 4 * ((elems + 3) / 4 * 4) + 8 * RS_BSTAGE);
+__host__ __device__ constexpr int rs_warp_cap(int elems, int T) { return (elems + T - 1) / T * 32; }
+__host__ __device__ constexpr int rs_scratch_bytes(int L_cap, int elems, int T) {
+  return rs_max3(8 * RS_BCAP, 4 * ((L_cap + 31) / 32 + 4), 4 * (T / 32) * rs_warp_cap(elems, T) + 8 * RS_BSTAGE);
 }
 
 template <int T>
@@ -66,6 +69,7 @@ struct RsShared {
   int ok;
   uint32_t n_win, n_bk, base_win, base_bk;  // this CTA's staged winners and bucket entries, their slots
   uint32_t wa[T / 32], wb[T / 32 + 1];
+  uint32_t wcnt[T / 32];  // winners staged by each warp
   uint32_t hist[HPAD];
   uint32_t small_key[T], small_tie[T];
 };
@@ -128,7 +132,7 @@ __device__ __forceinline__ uint32_t warp_append(uint32_t *cnt, bool take) {
 // The fused selection of one row (k outputs), called by every thread of each
 // of the row's C CTAs after scoring.  shist: the CTA's 11-bit counts of its
 // elements (RB words in shared memory, overwritten).  scratch: shared memory
-// of rs_scratch_bytes(L_cap, elems) bytes (free after scoring), elems the
+// of rs_scratch_bytes(L_cap, elems, T) bytes (free after scoring), elems the
 // most elements `each` presents in this CTA.
 //   each(fn):  fn(key, token, valid) for every element of this CTA, called
 //              by all 32 lanes of a warp together (warp-uniform trips).
@@ -147,7 +151,7 @@ __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist,
   }
   if (!row_barrier(sh, ctr + RS_BAR0, (uint32_t)C, c)) return;
   if (tid < 32) {
-    const uint4 r = warp_select_bin<false, true>(hist1, (uint32_t)k);
+    const uint4 r = warp_select_bin_staged(hist1, (uint32_t)k, sh.hist);
     Boundary b;
     b.total = r.w;
     b.kk = min((uint32_t)k, r.w);
@@ -176,7 +180,7 @@ __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist,
     }
     if (!row_barrier(sh, ctr + RS_BAR1, (uint32_t)C, c)) return;
     if (tid < 32) {
-      const uint4 r = warp_select_bin<false, true>(hist2, need0);
+      const uint4 r = warp_select_bin_staged(hist2, need0, sh.hist);
       if (tid == 0) sh.res = r;
     }
     __syncthreads();
@@ -188,18 +192,19 @@ __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist,
   const bool bucket = lvl2 && need1 != in1;  // the 22-bit bucket is split
   int32_t *dst = ordered ? rw.winners : rw.out;
   // 3. this CTA's sure winners, and the bucket's elements: staged in shared
-  //    memory, then one global atomic per CTA reserves their slots (the
-  //    winners of a row's CTAs all count on one word: per-warp atomics there
-  //    serialise)
+  //    memory (winners in each warp's own part, no atomics; bucket entries,
+  //    rare, through a shared counter), then one global atomic per CTA
+  //    reserves their slots (the winners of a row's CTAs all count on one
+  //    word: per-warp atomics there serialise)
   if (bd.kk > 0) {
-    const int cap_w = (elems + 3) / 4 * 4;
+    const int lane = tid & 31, warp = tid >> 5;
+    const uint32_t pw = (uint32_t)rs_warp_cap(elems, T);
     uint32_t *st_w = reinterpret_cast<uint32_t *>(scratch);
-    uint2 *st_b = reinterpret_cast<uint2 *>(scratch + 4 * cap_w);
-    if (tid == 0) {
-      sh.n_win = 0;
-      sh.n_bk = 0;
-    }
+    uint2 *st_b = reinterpret_cast<uint2 *>(scratch + 4 * (T / 32) * pw);
+    uint32_t *my_w = st_w + warp * pw;
+    if (tid == 0) sh.n_bk = 0;
     __syncthreads();
+    uint32_t n_mine = 0;  // warp-uniform
     each([&](uint32_t key, int tok, bool valid) {
       const uint32_t k22 = key >> 10;
       bool sel;
@@ -209,24 +214,33 @@ __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist,
         sel = (key >> HIST_SHIFT) >= bd.d0;
       else
         sel = k22 > p22 || (!bucket && k22 == p22);
-      const uint32_t s1 = warp_append(&sh.n_win, valid && sel);
-      if (valid && sel && s1 < (uint32_t)cap_w) st_w[s1] = (uint32_t)tok;
+      const bool win = valid && sel;
+      const uint32_t m = __ballot_sync(0xffffffffu, win);
+      const uint32_t slot = n_mine + __popc(m & lanemask_lt());
+      if (win && slot < pw) my_w[slot] = (uint32_t)tok;
+      n_mine += __popc(m);
       const bool in_b = valid && bucket && k22 == p22;
       const uint32_t s2 = warp_append(&sh.n_bk, in_b);
       if (in_b && s2 < (uint32_t)RS_BSTAGE) st_b[s2] = make_uint2(key, (uint32_t)tok);
     });
+    n_mine = min(n_mine, pw);  // (never clipped: a warp visits at most pw elements)
+    if (lane == 0) sh.wcnt[warp] = n_mine;
     __syncthreads();
-    const uint32_t nw = min(sh.n_win, (uint32_t)cap_w), nbk = sh.n_bk;
+    const uint32_t nbk = sh.n_bk;
     if (tid == 0) {
+      uint32_t nw = 0;
+      for (int w = 0; w < T / 32; ++w) nw += sh.wcnt[w];
       sh.base_win = nw ? atomicAdd(ctr + RS_EMIT, nw) : 0u;
       // more bucket entries than staged: count the row past the list's
       // capacity, so that the last CTA ranks it from the scores instead
       sh.base_bk = nbk ? atomicAdd(ctr + RS_BUCKET, nbk <= (uint32_t)RS_BSTAGE ? nbk : (uint32_t)RS_BCAP + 1u) : 0u;
     }
     __syncthreads();
-    for (uint32_t x = tid; x < nw; x += T) {
-      const uint32_t slot = sh.base_win + x;
-      if (slot < (uint32_t)k) dst[slot] = (int32_t)st_w[x];
+    uint32_t off = sh.base_win;
+    for (int w = 0; w < warp; ++w) off += sh.wcnt[w];
+    for (uint32_t x = lane; x < n_mine; x += 32) {
+      const uint32_t slot = off + x;
+      if (slot < (uint32_t)k) dst[slot] = (int32_t)my_w[x];
     }
     if (nbk <= (uint32_t)RS_BSTAGE)
       for (uint32_t x = tid; x < nbk; x += T) {

@@ -37,6 +37,7 @@ namespace {
 
 constexpr int WARPS = 8;
 constexpr int THREADS = 32 * WARPS;
+static_assert(MISA_MAX_H <= THREADS, "one thread per head in the router");
 
 template <int NT, bool FP8>
 struct StreamCfg {
@@ -153,7 +154,8 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
                  qv.q + ((size_t)i * qv.H + j) * D + 8 * u);
     }
     cp_async_commit();
-    for (int j = tid; j < qv.H; j += THREADS) r_w[j] = __ldg(qv.w + (size_t)i * qv.H + j);
+    // the weights land in registers meanwhile (H <= MISA_MAX_H <= THREADS)
+    const float w_mine = tid < qv.H ? __ldg(qv.w + (size_t)i * qv.H + tid) : 0.f;
     const int Mi = cdiv(Li, c.B), full = Li / c.B, C = gridDim.x;
     const int m0 = (int)((long long)blockIdx.x * Mi / C), m1 = (int)((long long)(blockIdx.x + 1) * Mi / C);
     if (full < Mi && full >= m0 && full < m1) {  // uniform: this CTA holds the block cut by the prefix end
@@ -164,6 +166,7 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
     route_slice<WARPS>(c, s, qv.H, m0, m1, full, r_tail, r_wsum, r_out, qrow_s, [&] {
 #pragma unroll
       for (int j = 0; j < NS - 1; ++j) issue(j);
+      if (tid < qv.H) r_w[tid] = w_mine;
       cp_async_wait<NS - 1>();  // the query rows (the group before the ring's)
       __syncthreads();
     });
@@ -334,7 +337,7 @@ StreamPlan plan_nt(const CacheView &c, const QueryView &q, bool fused) {
   for (int it = 0; it < 3 && per_sm > 0; ++it) {
     const int sp = splits_for(per_sm);
     const int mt = cdiv(ntile, sp * WARPS);
-    const int sel = (int)((sizeof(RsShared<THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap, WARPS * mt * Cfg::TT);
+    const int sel = (int)((sizeof(RsShared<THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap, WARPS * mt * Cfg::TT, THREADS);
     const int region = (std::max(RING, sel) + 127) / 128 * 128;
     const int smem = region + WARPS * mt * Cfg::TT * 4;
     const int fit = smem <= max_dyn ? per_sm_for(smem) : 0;

@@ -40,26 +40,87 @@ __device__ __forceinline__ int hpos(int b) { return b + (b >> 6); }
 
 // One whole warp: the bin of a RB-bin histogram (larger bin = larger key)
 // holding the want-th largest element.  Lane l sums bins [64 l, 64 l + 64);
-// the range that holds it is then searched two bins per lane.  Returns to every lane
+// the range that holds it is then searched (shared: two bins per lane; global:
+// by its owner, from registers).  Returns to every lane
 // {bin, elements in higher bins, its count, total}; bin = ~0 when want is 0
 // or above the total.  PAD: shared histogram in the hpos layout, else a
 // plain array in global memory, read through the read-only path, or with CG
 // through L2 only (a histogram other CTAs of the same kernel wrote).
-template <bool PAD, bool CG = false>
-__device__ __forceinline__ uint4 warp_select_bin(const uint32_t *h, uint32_t want) {
+// A histogram in global memory: every lane keeps its 64 bins in registers
+// and the owner walks them itself, so the search costs one round of loads.
+template <bool CG>
+__device__ __forceinline__ uint4 warp_select_bin_global(const uint32_t *h, uint32_t want) {
   const int lane = threadIdx.x & 31;
-  uint32_t s = 0;
-  if (PAD) {
-#pragma unroll 16
-    for (int j = 0; j < 64; ++j) s += h[lane * 65 + j];
-  } else {
-    const uint4 *p = reinterpret_cast<const uint4 *>(h + lane * 64);
+  const uint4 *p = reinterpret_cast<const uint4 *>(h + lane * 64);
+  uint4 v[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const uint4 v = CG ? __ldcg(p + j) : __ldg(p + j);
-      s += v.x + v.y + v.z + v.w;
+  for (int j = 0; j < 16; ++j) v[j] = CG ? __ldcg(p + j) : __ldg(p + j);
+  uint32_t s = 0;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) s += v[j].x + v[j].y + v[j].z + v[j].w;
+  uint32_t suf = s;  // elements in lanes >= this one
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t u = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += u;
+  }
+  const uint32_t total = __shfl_sync(0xffffffffu, suf, 0);
+  if (want == 0 || want > total) return make_uint4(~0u, 0u, 0u, total);
+  const uint32_t above_l = suf - s;
+  const int owner = __ffs(__ballot_sync(0xffffffffu, above_l < want && suf >= want)) - 1;
+  // the owner's bins from the highest down: the first that reaches `want`
+  uint32_t bin = 0, above = 0, cnt = 0, a = above_l;
+  bool found = false;
+#pragma unroll
+  for (int j = 15; j >= 0; --j) {
+    const uint32_t c4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+    for (int e = 3; e >= 0; --e) {
+      const bool hit = !found && a + c4[e] >= want;
+      if (hit) {
+        bin = (uint32_t)(lane * 64 + 4 * j + e);
+        above = a;
+        cnt = c4[e];
+      }
+      found = found || hit;
+      a += found ? 0u : c4[e];
     }
   }
+  return make_uint4(__shfl_sync(0xffffffffu, bin, owner), __shfl_sync(0xffffffffu, above, owner),
+                    __shfl_sync(0xffffffffu, cnt, owner), total);
+}
+
+template <bool PAD, bool CG = false>
+__device__ __forceinline__ uint4 warp_select_bin(const uint32_t *h, uint32_t want);
+
+// A histogram other CTAs wrote to global memory (read through L2), copied
+// by one warp into shared memory (hpos layout, HPAD words of `stage`) in
+// one round of loads and searched there; light on registers.
+__device__ __forceinline__ uint4 warp_select_bin_staged(const uint32_t *h, uint32_t want, uint32_t *stage) {
+  const int lane = threadIdx.x & 31;
+  const uint4 *p = reinterpret_cast<const uint4 *>(h + lane * 64);
+  uint4 v[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = __ldcg(p + j);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    uint32_t *d = stage + lane * 65 + 4 * j;  // hpos(64 lane + 4 j)
+    d[0] = v[j].x;
+    d[1] = v[j].y;
+    d[2] = v[j].z;
+    d[3] = v[j].w;
+  }
+  __syncwarp();
+  return warp_select_bin<true>(stage, want);
+}
+
+template <bool PAD, bool CG>
+__device__ __forceinline__ uint4 warp_select_bin(const uint32_t *h, uint32_t want) {
+  if constexpr (!PAD) return warp_select_bin_global<CG>(h, want);
+  const int lane = threadIdx.x & 31;
+  uint32_t s = 0;
+#pragma unroll 16
+  for (int j = 0; j < 64; ++j) s += h[lane * 65 + j];
   uint32_t suf = s;  // elements in lanes >= this one
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -73,15 +134,7 @@ __device__ __forceinline__ uint4 warp_select_bin(const uint32_t *h, uint32_t wan
   // the owner's 64 bins, two per lane, searched by the whole warp
   const uint32_t base_above = __shfl_sync(0xffffffffu, above_l, owner);
   const int b0 = owner * 64 + 2 * lane;
-  uint32_t c0, c1;
-  if (PAD) {
-    c0 = h[hpos(b0)];
-    c1 = h[hpos(b0 + 1)];
-  } else {
-    const uint2 v = CG ? __ldcg(reinterpret_cast<const uint2 *>(h + b0)) : __ldg(reinterpret_cast<const uint2 *>(h + b0));
-    c0 = v.x;
-    c1 = v.y;
-  }
+  const uint32_t c0 = h[hpos(b0)], c1 = h[hpos(b0 + 1)];
   const uint32_t pair = c0 + c1;
   uint32_t psuf = pair;  // elements in the owner's bins >= b0
 #pragma unroll
