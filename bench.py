@@ -70,8 +70,9 @@ def score_kernel_bytes(wl):
 
 # DRAM bytes (read + write) of one launch of the decode step's routed scoring
 # kernel per workload, from an ncu capture of the current kernel (summarised
-# under profiles/); null where the kernel changed since the last capture.
-STREAM_TRAFFIC_BYTES = {}
+# in profiles/score_stream_kernel_misa_dagger_decode_128k.md: 142,993,408
+# read + 4,683,264 written); null where the kernel changed since the capture.
+STREAM_TRAFFIC_BYTES = {"misa_dagger_decode_128k": 142993408 + 4683264}
 
 
 class Clocks:

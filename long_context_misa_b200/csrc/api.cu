@@ -202,6 +202,7 @@ misa::FusedTopk fused_args(uint32_t *zeroed, void *bucket, void *winners, int32_
   f.out = out;
   f.k = k;
   f.ordered = ordered ? 1 : 0;
+  f.defer = 0;
   return f;
 }
 
@@ -393,7 +394,11 @@ misa_status dagger_body(const char *who, const misa_cache *cache, const misa_que
   uint32_t *z1 = hist + dagger_zero_words(qs, f1, f2);
   cudaError_t e = zero_done ? cudaSuccess : misa::launch_zero(z0, (size_t)(z1 - z0), stream);
   if (e != cudaSuccess) return cuda_fail(e, who);
-  const misa::FusedTopk fzc = fused_args(fz1, bucket, nullptr, cand, k_prime, false);
+  // the fine pass in one cluster kernel: a top-k' selected in the routed
+  // scoring kernel leaves its boundary bucket for that kernel to finish
+  const bool cluster = !f2 && misa::rerank_cluster_applies(c, q, k_prime, k);
+  misa::FusedTopk fzc = fused_args(fz1, bucket, nullptr, cand, k_prime, false);
+  fzc.defer = f1 && cluster ? 1 : 0;
   e = timed_scoring(stream, [&] {
     if (route_part)
       return misa::launch_score_stream(c, q, nullptr, h, scores, cache->L_cap, hist, stream, &fzc, route_part,
@@ -410,8 +415,9 @@ misa_status dagger_body(const char *who, const misa_cache *cache, const misa_que
   }
   // fine pass: every head on the candidates, ascending final top-k; one
   // cluster kernel when a cluster holds a query's candidates
-  if (!f2 && misa::rerank_cluster_applies(c, q, k_prime, k)) {
-    e = misa::launch_rerank_cluster(c, q, cand, k_prime, k, topk, nullptr, 0, stream);
+  if (cluster) {
+    e = misa::launch_rerank_cluster(c, q, cand, k_prime, k, topk, nullptr, 0, stream, fzc.defer ? fz1 : nullptr,
+                                    fzc.defer ? reinterpret_cast<const uint2 *>(bucket) : nullptr);
     if (e != cudaSuccess) return cuda_fail(e, who);
     return MISA_OK;
   }

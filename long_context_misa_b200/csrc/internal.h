@@ -55,7 +55,16 @@ struct FusedTopk {
   int32_t *out;       // [n_q][k] the selected tokens
   int k;
   int ordered;        // 1: ascending token order; 0: any order
+  // 1 (unordered outputs only): the next kernel finishes the row.  The
+  // selecting kernel writes the sure winners to out[0, n) (n = the row's
+  // winner counter) and lists a split boundary bucket that fits FUSED_BCAP
+  // with the number still to take from it (counters FUSED_CTR_EMIT,
+  // FUSED_CTR_BUCKET, FUSED_CTR_NEED of the row's zeroed words); rows whose
+  // bucket is larger are finished as usual.  Nothing pads out[n, k).
+  int defer;
 };
+// counters among a row's zeroed words (after its two histograms)
+constexpr int FUSED_CTR_EMIT = 3, FUSED_CTR_BUCKET = 4, FUSED_CTR_NEED = 6;
 // Whether launch_score_mma can select in the scoring kernel for these shapes
 // (fused != nullptr there); otherwise the caller runs launch_topk.
 bool score_fusable(const CacheView &c, const QueryView &q, const int32_t *heads, int h, const int32_t *gather,
@@ -87,8 +96,11 @@ bool rerank_fusable(const CacheView &c, const QueryView &q, const int32_t *heads
 // and the device can run one; scores (optional, row pitch ld) receives every
 // valid candidate's score.
 bool rerank_cluster_applies(const CacheView &c, const QueryView &q, int n_cols, int k);
+// pend != nullptr: the candidates come from a top-k' selected with
+// FusedTopk::defer (pend = its zeroed words, pend_bucket = its bucket lists).
 cudaError_t launch_rerank_cluster(const CacheView &c, const QueryView &q, const int32_t *gather, int n_cols, int k,
-                                  int32_t *out, float *scores, long long ld, cudaStream_t s);
+                                  int32_t *out, float *scores, long long ld, cudaStream_t s,
+                                  const uint32_t *pend = nullptr, const uint2 *pend_bucket = nullptr);
 // the same for prefix rows of e4m3 caches with 32 or more scoring heads
 bool dense_fusable(const CacheView &c, const QueryView &q, const int32_t *heads, int h);
 

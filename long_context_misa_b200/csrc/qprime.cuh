@@ -15,12 +15,11 @@ namespace {
 // past h_eff), two threads per row (half of its 16-byte chunks each, the pair
 // agreeing on the e4m3 scale through a shuffle), in the 128-byte-swizzled
 // K-major layout the MMA reads; bf16 as is, or the exact two-term e4m3 split
-// with the power-of-two scale folded into the weight w_s[n].  Threads
-// [0, 128) call.
+// with the power-of-two scale folded into the weight w_s[n].  128 threads
+// call, numbered `tid` = 0 .. 127 (whole warps).
 template <bool FP8, int HN>
 __device__ __forceinline__ void build_qprime(const CacheView &c, const QueryView &qv, const int32_t *heads, int h,
-                                             int i, uint8_t *b_smem, float *w_s) {
-  const int tid = threadIdx.x;
+                                             int i, uint8_t *b_smem, float *w_s, int tid = threadIdx.x) {
   const int H = qv.H;
   const int h_eff = heads ? h : H;
   for (int x = tid; x < 2 * HN; x += 128) {  // whole warps: HN >= 32

@@ -70,6 +70,7 @@ struct RcCfg {
 
 template <int SLOTS>
 struct RcShared {
+  uint2 bk[FUSED_BCAP];            // a handed-over row's boundary bucket (key, token)
   uint64_t done;
   uint32_t tmem_base;
   int abort;
@@ -121,7 +122,7 @@ __device__ __forceinline__ void rc_level(int lvl, bool &lo_word, int &sft, uint3
 template <bool FP8, int HN, int TPC>
 __global__ void __cluster_dims__(RC_CL, 1, 1) __launch_bounds__(RC_THREADS, 1)
     rerank_cluster_kernel(CacheView c, QueryView qv, const int32_t *gather, int n_cols, int k, int32_t *out,
-                          float *scores, long long ld) {
+                          float *scores, long long ld, const uint32_t *pend, const uint2 *pend_bucket) {
   grid_dep_sync();
   using Cfg = RcCfg<FP8, HN, TPC>;
   constexpr int SLOTS = Cfg::SLOTS;
@@ -143,16 +144,43 @@ __global__ void __cluster_dims__(RC_CL, 1, 1) __launch_bounds__(RC_THREADS, 1)
   const uint8_t *kbase = static_cast<const uint8_t *>(c.keys) + (size_t)max(s, 0) * c.L_cap * Cfg::ROW;
   const float *sbase = FP8 ? c.scale + (size_t)max(s, 0) * c.L_cap : nullptr;
 
-  // 1. this CTA's candidates (-1: none, negative, or beyond the prefix)
+  // 1. this CTA's candidates (-1: none, negative, or beyond the prefix).
+  //    With a handed-over row (pend != nullptr) only slots below its winner
+  //    count hold candidates; the `need` best entries of its boundary bucket
+  //    (larger key first, equal keys to the lower token) fill the next ones.
+  int n_sure = n_cols, pneed = 0, nb = 0;
+  const uint32_t *pctr = nullptr;
+  if (pend) {
+    pctr = pend + (size_t)i * FUSED_ZERO_WORDS + 2 * RB;
+    n_sure = (int)min(__ldcg(pctr + FUSED_CTR_EMIT), (uint32_t)n_cols);
+    nb = (int)min(__ldcg(pctr + FUSED_CTR_BUCKET), (uint32_t)FUSED_BCAP);
+    pneed = (int)min(__ldcg(pctr + FUSED_CTR_NEED), (uint32_t)(n_cols - n_sure));
+  }
   for (int e = tid; e < SLOTS; e += RC_THREADS) {
     const int p = col0 + e;
-    const int t = p < n_cols ? __ldg(gather + (size_t)i * n_cols + p) : -1;
+    const int t = p < n_sure ? __ldg(gather + (size_t)i * n_cols + p) : -1;
     sh.tok[e] = (t >= 0 && t < Li) ? t : -1;
   }
   if (tid == 0) {
     mbar_init(&sh.done, 1);
     sh.abort = 0;
     fence_mbar_init();
+  }
+  if (pneed > 0 && n_sure + pneed > col0 && n_sure < col0 + SLOTS) {  // uniform: this CTA holds some of them
+    const uint2 *brow = pend_bucket + (size_t)i * FUSED_BCAP;
+    for (int x = tid; x < nb; x += RC_THREADS) sh.bk[x] = __ldcg(brow + x);
+    __syncthreads();
+    for (int x = tid; x < nb; x += RC_THREADS) {
+      const uint2 ex = sh.bk[x];
+      int rank = 0;
+      for (int y = 0; y < nb; ++y) {
+        const uint2 ey = sh.bk[y];
+        rank += (ey.x > ex.x || (ey.x == ex.x && ey.y < ex.y)) ? 1 : 0;
+      }
+      const int e = n_sure + rank - col0;
+      const int t = (int)ex.y;
+      if (rank < pneed && e >= 0 && e < SLOTS) sh.tok[e] = (t >= 0 && t < Li) ? t : -1;
+    }
   }
   __syncthreads();
 
@@ -460,7 +488,8 @@ int rc_tpc(int n_cols) {
 
 template <bool FP8, int HN>
 cudaError_t rc_launch_hn(const CacheView &c, const QueryView &q, const int32_t *gather, int n_cols, int k,
-                         int32_t *out, float *scores, long long ld, cudaStream_t s, bool dry) {
+                         int32_t *out, float *scores, long long ld, const uint32_t *pend, const uint2 *pend_bucket,
+                         cudaStream_t s, bool dry) {
   const int tpc = rc_tpc<FP8, HN>(n_cols);
 #define MISA_RC_CASE(T)                                                                                     \
   if (tpc == T) {                                                                                           \
@@ -468,7 +497,8 @@ cudaError_t rc_launch_hn(const CacheView &c, const QueryView &q, const int32_t *
       if (!rc_fits<FP8, HN, T>()) return cudaErrorNotSupported;                                            \
       if (dry) return cudaSuccess;                                                                          \
       return launch_kernel(rerank_cluster_kernel<FP8, HN, T>, dim3(RC_CL, q.n_q), dim3(RC_THREADS),        \
-                           RcCfg<FP8, HN, T>::SMEM, s, c, q, gather, n_cols, k, out, scores, ld);          \
+                           RcCfg<FP8, HN, T>::SMEM, s, c, q, gather, n_cols, k, out, scores, ld, pend,     \
+                           pend_bucket);                                                                   \
     }                                                                                                       \
   }
   MISA_RC_CASE(1)
@@ -480,28 +510,30 @@ cudaError_t rc_launch_hn(const CacheView &c, const QueryView &q, const int32_t *
 }
 
 cudaError_t rc_dispatch(const CacheView &c, const QueryView &q, const int32_t *gather, int n_cols, int k, int32_t *out,
-                        float *scores, long long ld, cudaStream_t s, bool dry) {
+                        float *scores, long long ld, const uint32_t *pend, const uint2 *pend_bucket, cudaStream_t s,
+                        bool dry) {
   if (q.n_q < 1 || n_cols < 1 || k < 1 || k > n_cols || q.H > 128) return cudaErrorNotSupported;
   const int hn = q.H <= 32 ? 32 : q.H <= 64 ? 64 : 128;
   if (c.fp8) {
-    if (hn == 32) return rc_launch_hn<true, 32>(c, q, gather, n_cols, k, out, scores, ld, s, dry);
-    if (hn == 64) return rc_launch_hn<true, 64>(c, q, gather, n_cols, k, out, scores, ld, s, dry);
-    return rc_launch_hn<true, 128>(c, q, gather, n_cols, k, out, scores, ld, s, dry);
+    if (hn == 32) return rc_launch_hn<true, 32>(c, q, gather, n_cols, k, out, scores, ld, pend, pend_bucket, s, dry);
+    if (hn == 64) return rc_launch_hn<true, 64>(c, q, gather, n_cols, k, out, scores, ld, pend, pend_bucket, s, dry);
+    return rc_launch_hn<true, 128>(c, q, gather, n_cols, k, out, scores, ld, pend, pend_bucket, s, dry);
   }
-  if (hn == 32) return rc_launch_hn<false, 32>(c, q, gather, n_cols, k, out, scores, ld, s, dry);
-  if (hn == 64) return rc_launch_hn<false, 64>(c, q, gather, n_cols, k, out, scores, ld, s, dry);
-  return rc_launch_hn<false, 128>(c, q, gather, n_cols, k, out, scores, ld, s, dry);
+  if (hn == 32) return rc_launch_hn<false, 32>(c, q, gather, n_cols, k, out, scores, ld, pend, pend_bucket, s, dry);
+  if (hn == 64) return rc_launch_hn<false, 64>(c, q, gather, n_cols, k, out, scores, ld, pend, pend_bucket, s, dry);
+  return rc_launch_hn<false, 128>(c, q, gather, n_cols, k, out, scores, ld, pend, pend_bucket, s, dry);
 }
 
 }  // namespace
 
 bool rerank_cluster_applies(const CacheView &c, const QueryView &q, int n_cols, int k) {
-  return rc_dispatch(c, q, nullptr, n_cols, k, nullptr, nullptr, 0, nullptr, true) == cudaSuccess;
+  return rc_dispatch(c, q, nullptr, n_cols, k, nullptr, nullptr, 0, nullptr, nullptr, nullptr, true) == cudaSuccess;
 }
 
 cudaError_t launch_rerank_cluster(const CacheView &c, const QueryView &q, const int32_t *gather, int n_cols, int k,
-                                  int32_t *out, float *scores, long long ld, cudaStream_t s) {
-  return rc_dispatch(c, q, gather, n_cols, k, out, scores, ld, s, false);
+                                  int32_t *out, float *scores, long long ld, cudaStream_t s, const uint32_t *pend,
+                                  const uint2 *pend_bucket) {
+  return rc_dispatch(c, q, gather, n_cols, k, out, scores, ld, pend, pend_bucket, s, false);
 }
 
 }  // namespace misa

@@ -271,17 +271,21 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
 // query).  Persistent and warp-specialised: CTA `part` of a query walks the
 // tiles part, part + nparts, ... of its prefix (one CTA per SM over all
 // queries, so the CTAs read neighbouring tiles at the same time).
-//   warp 0     TMA producer: 128-byte-swizzled key tiles (16 KB) into a ring
-//              of DS_STAGES shared-memory stages;
-//   warp 1     owns the tensor memory; one thread issues each tile's MMAs into
+//   warps 0-3  producers: each key tile (16 KB, 128 consecutive tokens) is
+//              copied with 16-byte cp.async into a ring of DS_STAGES stages
+//              in the 128-byte-swizzled K-major layout (every warp
+//              instruction one contiguous 512-byte span); a producer thread
+//              keeps DS_LAG tiles in flight and marks a tile full once its
+//              own copies of it have landed;
+//   warp 4     owns the tensor memory; one thread issues each tile's MMAs into
 //              one of two accumulator buffers and commits the stage back to
-//              the producer and the buffer to the epilogue;
-//   warps 2-9  two sets of four warps, set b draining accumulator buffer b
+//              the producers and the buffer to the epilogue;
+//   warps 5-12 two sets of four warps, set b draining accumulator buffer b
 //              (the even or the odd tiles); in a set one tensor-memory lane
 //              quarter per warp, one token row per thread: ReLU, the weights,
 //              the head sum (four independent partial sums) and the e4m3
-//              token scale (loaded one tile ahead), the score written and
-//              counted.
+//              token scale (requested DS_SD of the set's tiles ahead), the
+//              score written and counted.
 // The two accumulator buffers let tile j + 1's MMAs run while tile j is
 // drained, two sets drain two tiles at once, and the ring keeps DS_STAGES
 // tiles of keys in flight per SM.
@@ -290,8 +294,16 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
 // bounded: one that runs out sets MISA_DEV_WAIT_TIMEOUT and the CTA winds
 // down without selecting.
 constexpr int DS_STAGES = 8;
-constexpr int DS_EPI = 8;  // two sets of four: set b drains accumulator buffer b (tiles j with j % 2 == b)
-constexpr int DS_THREADS = 64 + 32 * DS_EPI;
+constexpr int DS_PROD = 4;                  // producer warps
+constexpr int DS_LAG = DS_STAGES - 2;       // tiles a producer thread has in flight before marking one full
+constexpr int DS_MMA_WARP = DS_PROD;
+constexpr int DS_EPI0 = DS_PROD + 1;        // first epilogue warp
+constexpr int DS_EPI = 8;  // sets of four warps, one per tensor-memory lane quarter
+constexpr int DS_SETS = DS_EPI / 4;  // 1: one set drains every tile; 2: set b drains buffer b (tiles j % 2 == b)
+static_assert(DS_SETS == 1 || DS_SETS == 2, "epilogue sets");
+constexpr int DS_THREADS = 32 * (DS_EPI0 + DS_EPI);
+constexpr int DS_SD = 6;  // set iterations a drain's token scales are requested ahead
+constexpr int DS_SQ = 8;  // their slots per epilogue thread (> DS_SD: a slot is read before it is refilled)
 
 template <int HN>
 struct DSCfg {
@@ -309,6 +321,7 @@ struct DsShared {
   int abort;
   alignas(16) float w[128];                    // weight per column (0: padding)
   uint32_t hist[TOPK_HIST_BINS];               // this CTA's share of the row histogram
+  float escl[DS_SQ][32 * DS_EPI];              // epilogue threads' token scales in flight
 };
 
 // Dynamic shared memory of a dense launch: alignment slack, the ring and Q',
@@ -320,8 +333,8 @@ __host__ __device__ int dense_smem(int max_tiles, bool fused) {
 
 template <int HN>
 __global__ void __launch_bounds__(DS_THREADS, 1)
-    dense_umma_kernel(const __grid_constant__ CUtensorMap kmap, CacheView c, QueryView qv, const int32_t *heads, int h,
-                      float *scores, long long ld, uint32_t *row_hist, int nparts, FusedTopk fz, int max_tiles) {
+    dense_umma_kernel(CacheView c, QueryView qv, const int32_t *heads, int h, float *scores, long long ld,
+                      uint32_t *row_hist, int nparts, FusedTopk fz, int max_tiles) {
   grid_dep_sync();
   using Cfg = DSCfg<HN>;
   extern __shared__ uint8_t ds_raw[];
@@ -344,19 +357,20 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
 
   if (tid == 0) {
     for (int st = 0; st < DS_STAGES; ++st) {
-      mbar_init(&sh.full[st], 1);
-      mbar_init(&sh.empty[st], 1);
+      mbar_init(&sh.full[st], 32 * DS_PROD);  // every producer thread
+      mbar_init(&sh.empty[st], 1);            // the MMAs' commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh.tfull[b], 1);
-      mbar_init(&sh.tempty[b], DS_EPI / 2);
+      mbar_init(&sh.tempty[b], 4);  // the four warps of the set that drains it
     }
     sh.abort = 0;
     fence_mbar_init();
   }
   for (int b = tid; b < TOPK_HIST_BINS; b += DS_THREADS) sh.hist[b] = 0;
-  if (tid < RR_THREADS) build_qprime<true, HN>(c, qv, heads, h, i, b_smem, sh.w);
-  if (warp == 1) {
+  if (warp >= DS_EPI0 && warp < DS_EPI0 + 4)  // the first four epilogue warps
+    build_qprime<true, HN>(c, qv, heads, h, i, b_smem, sh.w, tid - 32 * DS_EPI0);
+  if (warp == DS_MMA_WARP) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&sh.tmem_base)),
                  "n"(Cfg::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -366,22 +380,36 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
   __syncthreads();
   umma::fence_after();
   const uint32_t tmem = sh.tmem_base;
-  uint32_t last_fill = 0;   // producer: tiles whose load it issued
   uint32_t committed = 0;   // MMA thread: tiles whose MMAs it committed
 
-  if (warp == 0) {
-    // ---- TMA producer ----
-    if (lane == 0) {
-      for (int j = 0; j < n_my; ++j) {
-        const int st = j % DS_STAGES;
-        if (!umma::wait_bar(&sh.empty[st], ((j / DS_STAGES) & 1) ^ 1, abort, c)) break;
-        mbar_arrive_expect_tx(&sh.full[st], Cfg::A_BYTES);
-        const int t0 = (part + j * nparts) * RR_M;
-        umma::tma_load_2d(smem_addr(a_smem + st * Cfg::A_BYTES), &kmap, 0, s * c.L_cap + t0, &sh.full[st]);
-        last_fill = j + 1;
+  if (warp < DS_PROD) {
+    // ---- producers: thread pt copies chunk pt % 8 of rows pt / 8 + 16 m ----
+    const int pt = tid;
+    const uint8_t *kbase = static_cast<const uint8_t *>(c.keys) + (size_t)s * c.L_cap * 128;
+    int marked = 0;  // tiles this thread has marked full
+    int j = 0;
+    for (; j < n_my; ++j) {
+      const int st = j % DS_STAGES;
+      if (!umma::wait_bar(&sh.empty[st], ((j / DS_STAGES) & 1) ^ 1, abort, c)) break;
+      const int t0 = (part + j * nparts) * RR_M;
+      const uint32_t dst = smem_addr(a_smem + st * Cfg::A_BYTES);
+#pragma unroll
+      for (int m = 0; m < RR_M * 8 / (32 * DS_PROD); ++m) {
+        const int x = pt + 32 * DS_PROD * m, r = x >> 3, u = x & 7;
+        const bool ok = t0 + r < Li;
+        cp_async16(dst + r * 128 + ((u ^ (r & 7)) << 4), ok ? kbase + (size_t)(t0 + r) * 128 + 16 * u : kbase, ok);
+      }
+      cp_async_commit();
+      if (j >= DS_LAG) {  // the tile issued DS_LAG tiles ago has landed (this thread's part)
+        cp_async_wait<DS_LAG>();
+        mbar_arrive(&sh.full[(j - DS_LAG) % DS_STAGES]);
+        marked = j - DS_LAG + 1;
       }
     }
-  } else if (warp == 1) {
+    cp_async_wait<0>();  // no copy in flight past here
+    if (j == n_my)
+      for (int jj = marked; jj < n_my; ++jj) mbar_arrive(&sh.full[jj % DS_STAGES]);
+  } else if (warp == DS_MMA_WARP) {
     // ---- MMA issuer ----
     if (lane == 0) {
       const uint32_t idesc = umma::instr_desc<true, RR_M, HN>();
@@ -391,6 +419,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
         if (!umma::wait_bar(&sh.tempty[buf], ((j >> 1) & 1) ^ 1, abort, c)) break;
         umma::fence_after();
         if (!umma::wait_bar(&sh.full[st], (j / DS_STAGES) & 1, abort, c)) break;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the copied rows, to the tensor cores
         umma::fence_after();
         const uint32_t a_base = smem_addr(a_smem + st * Cfg::A_BYTES);
 #pragma unroll
@@ -405,25 +434,30 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
       }
     }
   } else {
-    // ---- epilogue: set `buf` drains the tiles j = buf, buf + 2, ...; token row r ----
-    const int buf = ((warp - 2) >> 2) & 1;
+    // ---- epilogue: set `set` drains the tiles j = set, set + DS_SETS, ...
+    //      (accumulator buffer j % 2); token row r ----
+    const int set = (warp - DS_EPI0) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16) + buf * HN;
+    const uint32_t tl0 = tmem + ((uint32_t)(quarter * 32) << 16);
     const float4 *w4 = reinterpret_cast<const float4 *>(sh.w);
     const float *srow_scale = c.scale + (size_t)s * c.L_cap;
-    float sc_next = 0.f;
-    if (buf < n_my) {
-      const int t = (part + buf * nparts) * RR_M + r;
-      sc_next = t < Li ? __ldg(srow_scale + t) : 0.f;
-    }
-    for (int j = buf; j < n_my; j += 2) {
-      const int t = (part + j * nparts) * RR_M + r;
-      const float scl = sc_next;
-      if (j + 2 < n_my) {
-        const int tn = t + 2 * nparts * RR_M;
-        sc_next = tn < Li ? __ldg(srow_scale + tn) : 0.f;
-      }
+    // the token scales of this thread's rows travel DS_SD tiles of its set
+    // ahead, by cp.async into its own slots (a load consumed two tiles later
+    // left every drain waiting on memory latency)
+    const int et = tid - 32 * DS_EPI0;
+    auto fetch = [&](int n) {  // the scale of row r of the set's n-th tile; one group per call
+      const int jn = set + DS_SETS * n, t = (part + jn * nparts) * RR_M + r;
+      const bool ok = jn < n_my && t < Li;
+      cp_async4(smem_addr(&sh.escl[n % DS_SQ][et]), ok ? srow_scale + t : srow_scale, ok);
+      cp_async_commit();
+    };
+#pragma unroll
+    for (int n = 0; n < DS_SD; ++n) fetch(n);
+    for (int j = set, n = 0; j < n_my; j += DS_SETS, ++n) {
+      const int t = (part + j * nparts) * RR_M + r, buf = j & 1;
+      const uint32_t tl = tl0 + buf * HN;
+      fetch(n + DS_SD);
       if (!umma::wait_bar(&sh.tfull[buf], (j >> 1) & 1, abort, c)) break;
       umma::fence_after();
       float a4[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
@@ -445,6 +479,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
       umma::fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.tempty[buf]);
+      cp_async_wait<DS_SD>();  // this tile's scale (older groups) has landed
+      const float scl = sh.escl[n % DS_SQ][et];
       if (t < Li) {
         const float val = acc * scl;
         scores[(size_t)i * ld + t] = val;
@@ -452,23 +488,19 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
         atomicAdd(&sh.hist[ordered_key(val) >> 21], 1u);
       }
     }
+    cp_async_wait<0>();
   }
 
-  // ---- wind-down: no load and no MMA in flight when the memory is released ----
+  // ---- wind-down: no copy (every role waited for its own) and no MMA in
+  //      flight when the memory is released ----
   __syncthreads();
-  if (warp == 0 && lane == 0 && *abort) {
-    // a role gave up: the last fill of each stage may still be landing (a
-    // completed one passes at once)
-    for (uint32_t j = (last_fill > DS_STAGES ? last_fill - DS_STAGES : 0); j < last_fill; ++j)
-      mbar_wait(&sh.full[j % DS_STAGES], (j / DS_STAGES) & 1);  // bounded
-  }
-  if (warp == 1 && lane == 0 && committed > 0) {
+  if (warp == DS_MMA_WARP && lane == 0 && committed > 0) {
     const uint32_t jl = committed - 1;  // the last committed accumulator buffer
     mbar_wait(&sh.tfull[jl & 1], (jl >> 1) & 1);  // bounded
   }
   umma::fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == DS_MMA_WARP) {
     umma::fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(Cfg::TMEM_COLS));
   }
@@ -533,7 +565,7 @@ DensePlan plan_dense(const CacheView &c, const QueryView &q, bool fused) {
   // a fused selection's state and scratch reuse the ring
   const int sel = (int)((sizeof(RsShared<DS_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap, p.max_tiles * RR_M, DS_THREADS);
   p.ok = p.smem <= max_dyn && (!fused || ((long long)p.nparts * q.n_q <= sms && sel <= DSCfg<HN>::RING)) && c.fp8 &&
-         umma::encoder_available() && (reinterpret_cast<uintptr_t>(c.keys) & 15u) == 0;
+         (reinterpret_cast<uintptr_t>(c.keys) & 15u) == 0;
   return p;
 }
 
@@ -542,12 +574,9 @@ cudaError_t launch_dense(const CacheView &c, const QueryView &q, const int32_t *
                          long long ld, uint32_t *row_hist, cudaStream_t s, const FusedTopk *fz) {
   const DensePlan p = plan_dense<HN>(c, q, fz != nullptr);
   if (!p.ok) return cudaErrorInvalidConfiguration;
-  CUtensorMap map;
-  if (!umma::make_map_2d(&map, c.keys, true, (unsigned long long)c.n_seq * c.L_cap, 128, RR_M))
-    return cudaErrorNotSupported;
   FusedTopk none = {};
-  return launch_kernel(dense_umma_kernel<HN>, dim3(p.nparts, q.n_q), dim3(DS_THREADS), p.smem, s, map, c, q, heads,
-                       h, scores, ld, row_hist, p.nparts, fz ? *fz : none, p.max_tiles);
+  return launch_kernel(dense_umma_kernel<HN>, dim3(p.nparts, q.n_q), dim3(DS_THREADS), p.smem, s, c, q, heads, h,
+                       scores, ld, row_hist, p.nparts, fz ? *fz : none, p.max_tiles);
 }
 
 // Dynamic shared memory of a re-rank launch: the key tiles and Q', at least

@@ -44,7 +44,10 @@ constexpr int RS_ZERO_WORDS = FUSED_ZERO_WORDS;
 static_assert(RS_ZERO_WORDS == 2 * RB + FUSED_CTR, "layout of the zeroed words");
 // counters: the two histogram barriers, the last-CTA count, winners and
 // bucket entries written, and the barrier of a router fused in front
-enum { RS_BAR0 = 0, RS_BAR1 = 1, RS_DONE = 2, RS_EMIT = 3, RS_BUCKET = 4, RS_ROUTE = 5 };
+enum { RS_BAR0 = 0, RS_BAR1 = 1, RS_DONE = 2, RS_EMIT = 3, RS_BUCKET = 4, RS_ROUTE = 5, RS_NEED = 6 };
+static_assert(RS_EMIT == FUSED_CTR_EMIT && RS_BUCKET == FUSED_CTR_BUCKET && RS_NEED == FUSED_CTR_NEED &&
+                  RS_NEED < FUSED_CTR,
+              "counter slots");
 
 constexpr int RS_BSTAGE = 512;  // bucket entries a CTA stages before reserving their slots
 
@@ -80,6 +83,7 @@ struct RsRow {
   uint2 *bucket;      // [RS_BCAP] (key, token)
   int32_t *winners;   // [k] winners of an ascending output; unused otherwise
   int32_t *out;       // [k] the row's output
+  bool defer;         // FusedTopk::defer
 };
 
 __device__ __forceinline__ RsRow rs_row(const FusedTopk &f, int i) {
@@ -88,6 +92,7 @@ __device__ __forceinline__ RsRow rs_row(const FusedTopk &f, int i) {
   r.bucket = f.bucket + (size_t)i * RS_BCAP;
   r.winners = f.winners ? f.winners + (size_t)i * f.k : nullptr;
   r.out = f.out + (size_t)i * f.k;
+  r.defer = f.defer != 0 && f.ordered == 0;
   return r;
 }
 
@@ -190,6 +195,10 @@ __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist,
     in1 = r.z;
   }
   const bool bucket = lvl2 && need1 != in1;  // the 22-bit bucket is split
+  // the next kernel finishes the row (rw.defer) unless the split bucket
+  // overflows its list: no last CTA then, and the bucket's entries go
+  // straight to the list (in1 of them in all, within its capacity)
+  const bool handoff = rw.defer && (!bucket || in1 <= (uint32_t)RS_BCAP);
   int32_t *dst = ordered ? rw.winners : rw.out;
   // 3. this CTA's sure winners, and the bucket's elements: staged in shared
   //    memory (winners in each warp's own part, no atomics; bucket entries,
@@ -220,8 +229,13 @@ __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist,
       if (win && slot < pw) my_w[slot] = (uint32_t)tok;
       n_mine += __popc(m);
       const bool in_b = valid && bucket && k22 == p22;
-      const uint32_t s2 = warp_append(&sh.n_bk, in_b);
-      if (in_b && s2 < (uint32_t)RS_BSTAGE) st_b[s2] = make_uint2(key, (uint32_t)tok);
+      if (handoff) {
+        const uint32_t s2 = warp_append(ctr + RS_BUCKET, in_b);
+        if (in_b && s2 < (uint32_t)RS_BCAP) rw.bucket[s2] = make_uint2(key, (uint32_t)tok);
+      } else {
+        const uint32_t s2 = warp_append(&sh.n_bk, in_b);
+        if (in_b && s2 < (uint32_t)RS_BSTAGE) st_b[s2] = make_uint2(key, (uint32_t)tok);
+      }
     });
     n_mine = min(n_mine, pw);  // (never clipped: a warp visits at most pw elements)
     if (lane == 0) sh.wcnt[warp] = n_mine;
@@ -247,6 +261,10 @@ __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist,
         const uint32_t slot = sh.base_bk + x;
         if (slot < (uint32_t)RS_BCAP) rw.bucket[slot] = st_b[x];
       }
+  }
+  if (handoff) {
+    if (bucket && blockIdx.x == 0 && tid == 0) ctr[RS_NEED] = need1;
+    return;
   }
   // 4. the last CTA of the row finishes it
   __syncthreads();

@@ -577,6 +577,36 @@ def test_dagger_decode_step(case):
     assert device_status(cache) == 0
 
 
+@pytest.mark.parametrize("period,k_prime,k", [(37, 1000, 300), (5, 3000, 700)])
+def test_dagger_decode_step_tied_scores(period, k_prime, k):
+    # every sequence repeats `period` distinct keys, so scores come in tied
+    # groups: the routed top-k' boundary falls inside a group that the
+    # scoring kernel hands to the re-rank kernel (a few hundred to a few
+    # thousand tokens), and the final top-k ties too.  Checked against the
+    # oracle with the heads the step chose.
+    wl = W["misa_dagger_decode_128k"].scaled(n_seq=3, L=20000, B=128, k=k, k_prime=k_prime)
+    inp = G.make_inputs(wl, 5)
+    t = np.arange(wl.L)
+    inp.keys[:] = inp.keys[:, t % period]
+    inp.scale[:] = inp.scale[:, t % period]
+    ref = Ref(inp)
+    cache, qs = to_device(inp, torch)
+    cache.seq_len.copy_(torch.from_numpy(inp.seq_len - 1))
+    M.pool_keys(cache)
+    nk, ns, pos = _decode_step_inputs(inp)
+    heads = torch.empty(wl.n_q, wl.h, dtype=torch.int32, device="cuda")
+    top = M.dagger_decode(cache, qs, nk, ns, pos, wl.h, k_prime, k, heads=heads).cpu().numpy()
+    hd = heads.cpu().numpy()
+    for i in range(wl.n_q):
+        q, w, K, Li = ref.query(i)
+        cand = O.top_k(O.index_scores(q, w, K[:Li], hd[i]), k_prime)
+        expect = O.rerank_query(q, w, K, cand, k)["topk"]
+        np.testing.assert_array_equal(top[i], expect, err_msg=f"query {i}")
+    again = M.dagger_topk(cache, qs, heads, k_prime, k).cpu().numpy()
+    np.testing.assert_array_equal(top, again)
+    assert device_status(cache) == 0
+
+
 @pytest.mark.parametrize("case", ["fp8_mixture", "fp8_long", "bf16_mixture", "bf16_prefill", "fp8_prefill_umma"])
 def test_dagger_topk_equals_composition(case):
     # one call (its k' candidates stay unordered inside) returns exactly what
