@@ -680,9 +680,15 @@ misa_status misa_dagger_decode(const misa_cache *cache, const misa_queries *qs, 
     // the re-rank's fusion does not depend on the candidates' values
     const bool f2 =
         g_select_in_kernel.load() && misa::score_fusable(c, q, nullptr, q.H, reinterpret_cast<const int32_t *>(w8), k_prime);
-    const size_t first = f2 ? ws_dagger_hist(qs) / sizeof(uint32_t) : 0;  // both fused: only their words
+    const bool cluster = !f2 && misa::rerank_cluster_applies(c, q, k_prime, k);
+    // words the step counts into: the routed pass's selection words, then
+    // the re-rank's (in-kernel selection), or its histograms just before them
+    // (separate top-k kernels); the cluster re-rank counts in shared memory
+    const size_t fz1 = ws_dagger_hist(qs) / sizeof(uint32_t), fzw = (size_t)qs->n_q * misa::FUSED_ZERO_WORDS;
+    const size_t first = cluster || f2 ? fz1 : ws_hist(qs) / sizeof(uint32_t);
+    const size_t last = f2 ? fz1 + round_up(sizeof(uint32_t) * fzw) / sizeof(uint32_t) + fzw : fz1 + fzw;
     z0 = reinterpret_cast<uint32_t *>(w8) + first;
-    zn = dagger_zero_words(qs, true, f2) - first;
+    zn = last - first;
   }
   cudaError_t e = misa::launch_pool_append(c, new_keys, new_scale, new_pos, count, stream, z0, zn);
   if (e != cudaSuccess) return cuda_fail(e, who);
