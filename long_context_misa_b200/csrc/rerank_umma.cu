@@ -269,39 +269,39 @@ __global__ void __launch_bounds__(RR_THREADS) rerank_umma_kernel(CacheView c, Qu
 // the dense product D[t][n] = K[t] . Q'[n] (M = 128 tokens, N = HN columns,
 // kind::f8f6f4 on the keys as stored against the two-term e4m3 split of the
 // query).  Persistent and warp-specialised: CTA `part` of a query walks the
-// tiles part, part + nparts, ... of its prefix (one CTA per SM over all
+// tiles part, part + nparts, ... of its prefix (two CTAs per SM over all
 // queries, so the CTAs read neighbouring tiles at the same time).
-//   warps 0-3  producers: each key tile (16 KB, 128 consecutive tokens) is
+//   warps 0-1  producers: each key tile (16 KB, 128 consecutive tokens) is
 //              copied with 16-byte cp.async into a ring of DS_STAGES stages
 //              in the 128-byte-swizzled K-major layout (every warp
 //              instruction one contiguous 512-byte span); a producer thread
 //              keeps DS_LAG tiles in flight and marks a tile full once its
 //              own copies of it have landed;
-//   warp 4     owns the tensor memory; one thread issues each tile's MMAs into
+//   warp 2     owns the tensor memory; one thread issues each tile's MMAs into
 //              one of two accumulator buffers and commits the stage back to
 //              the producers and the buffer to the epilogue;
-//   warps 5-12 two sets of four warps, set b draining accumulator buffer b
-//              (the even or the odd tiles); in a set one tensor-memory lane
-//              quarter per warp, one token row per thread: ReLU, the weights,
-//              the head sum (four independent partial sums) and the e4m3
-//              token scale (requested DS_SD of the set's tiles ahead), the
-//              score written and counted.
+//   warps 3-6  the epilogue, one tensor-memory lane quarter per warp, one
+//              token row per thread, draining the tiles in turn: ReLU, the
+//              weights, the head sum (four independent partial sums) and the
+//              e4m3 token scale (requested DS_SD tiles ahead), the score
+//              written and counted.
 // The two accumulator buffers let tile j + 1's MMAs run while tile j is
-// drained, two sets drain two tiles at once, and the ring keeps DS_STAGES
-// tiles of keys in flight per SM.
+// drained.  Two such CTAs per SM stream the prefix faster than one CTA with
+// twice the ring, more producers or a second epilogue set (measured).
 // With a fused selection every score also stays in shared memory and the
 // query's CTAs select its top k afterwards (rowsel.cuh).  Every wait is
 // bounded: one that runs out sets MISA_DEV_WAIT_TIMEOUT and the CTA winds
 // down without selecting.
-constexpr int DS_STAGES = 8;
-constexpr int DS_PROD = 4;                  // producer warps
+constexpr int DS_STAGES = 4;
+constexpr int DS_PROD = 2;                  // producer warps
 constexpr int DS_LAG = DS_STAGES - 2;       // tiles a producer thread has in flight before marking one full
 constexpr int DS_MMA_WARP = DS_PROD;
 constexpr int DS_EPI0 = DS_PROD + 1;        // first epilogue warp
-constexpr int DS_EPI = 8;  // sets of four warps, one per tensor-memory lane quarter
+constexpr int DS_EPI = 4;  // sets of four warps, one per tensor-memory lane quarter
 constexpr int DS_SETS = DS_EPI / 4;  // 1: one set drains every tile; 2: set b drains buffer b (tiles j % 2 == b)
 static_assert(DS_SETS == 1 || DS_SETS == 2, "epilogue sets");
 constexpr int DS_THREADS = 32 * (DS_EPI0 + DS_EPI);
+constexpr int DS_CTAS = 2;  // CTAs per SM (two pipelines stream more than one with twice the ring)
 constexpr int DS_SD = 6;  // set iterations a drain's token scales are requested ahead
 constexpr int DS_SQ = 8;  // their slots per epilogue thread (> DS_SD: a slot is read before it is refilled)
 
@@ -332,7 +332,7 @@ __host__ __device__ int dense_smem(int max_tiles, bool fused) {
 }
 
 template <int HN>
-__global__ void __launch_bounds__(DS_THREADS, 1)
+__global__ void __launch_bounds__(DS_THREADS, DS_CTAS)
     dense_umma_kernel(CacheView c, QueryView qv, const int32_t *heads, int h, float *scores, long long ld,
                       uint32_t *row_hist, int nparts, FusedTopk fz, int max_tiles) {
   grid_dep_sync();
@@ -559,12 +559,24 @@ DensePlan plan_dense(const CacheView &c, const QueryView &q, bool fused) {
   const int max_dyn = cached_per_device<Tag>([] { return opt_in_max_dyn_smem(dense_umma_kernel<HN>); });
   const int sms = device_sms();
   const int n_tiles = cdiv(c.L_cap, RR_M);
-  p.nparts = std::max(1, std::min(n_tiles, sms / std::max(q.n_q, 1)));
+  // DS_CTAS per SM (more CTAs than fit only queue); a fused selection needs
+  // its whole grid resident, so it takes what the occupancy query confirms
+  int per_sm = DS_CTAS;
+  if (fused) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, dense_umma_kernel<HN>, DS_THREADS,
+                                                      dense_smem<HN>(cdiv(n_tiles, sms), true)) != cudaSuccess) {
+      cudaGetLastError();
+      n = 1;
+    }
+    per_sm = std::max(1, std::min(n, DS_CTAS));
+  }
+  p.nparts = std::max(1, std::min(n_tiles, per_sm * sms / std::max(q.n_q, 1)));
   p.max_tiles = cdiv(n_tiles, p.nparts);
   p.smem = dense_smem<HN>(p.max_tiles, fused);
   // a fused selection's state and scratch reuse the ring
   const int sel = (int)((sizeof(RsShared<DS_THREADS>) + 15) / 16 * 16) + rs_scratch_bytes(c.L_cap, p.max_tiles * RR_M, DS_THREADS);
-  p.ok = p.smem <= max_dyn && (!fused || ((long long)p.nparts * q.n_q <= sms && sel <= DSCfg<HN>::RING)) && c.fp8 &&
+  p.ok = p.smem <= max_dyn && (!fused || ((long long)p.nparts * q.n_q <= (long long)per_sm * sms && sel <= DSCfg<HN>::RING)) && c.fp8 &&
          (reinterpret_cast<uintptr_t>(c.keys) & 15u) == 0;
   return p;
 }
