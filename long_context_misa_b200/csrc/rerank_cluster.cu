@@ -148,6 +148,14 @@ __global__ void __cluster_dims__(RC_CL, 1, 1) __launch_bounds__(RC_THREADS, 1)
   //    With a handed-over row (pend != nullptr) only slots below its winner
   //    count hold candidates; the `need` best entries of its boundary bucket
   //    (larger key first, equal keys to the lower token) fill the next ones.
+  // (the slots' tokens are requested together with the counters, then masked)
+  constexpr int EPT = (SLOTS + RC_THREADS - 1) / RC_THREADS;
+  int tk[EPT];
+#pragma unroll
+  for (int u = 0; u < EPT; ++u) {
+    const int e = tid + u * RC_THREADS, p = col0 + e;
+    tk[u] = (e < SLOTS && p < n_cols) ? __ldg(gather + (size_t)i * n_cols + p) : -1;
+  }
   int n_sure = n_cols, pneed = 0, nb = 0;
   const uint32_t *pctr = nullptr;
   if (pend) {
@@ -156,10 +164,10 @@ __global__ void __cluster_dims__(RC_CL, 1, 1) __launch_bounds__(RC_THREADS, 1)
     nb = (int)min(__ldcg(pctr + FUSED_CTR_BUCKET), (uint32_t)FUSED_BCAP);
     pneed = (int)min(__ldcg(pctr + FUSED_CTR_NEED), (uint32_t)(n_cols - n_sure));
   }
-  for (int e = tid; e < SLOTS; e += RC_THREADS) {
-    const int p = col0 + e;
-    const int t = p < n_sure ? __ldg(gather + (size_t)i * n_cols + p) : -1;
-    sh.tok[e] = (t >= 0 && t < Li) ? t : -1;
+#pragma unroll
+  for (int u = 0; u < EPT; ++u) {
+    const int e = tid + u * RC_THREADS, t = tk[u];
+    if (e < SLOTS) sh.tok[e] = (col0 + e < n_sure && t >= 0 && t < Li) ? t : -1;
   }
   if (tid == 0) {
     mbar_init(&sh.done, 1);
