@@ -49,6 +49,7 @@ constexpr int RC_M = 128;         // candidates per tile
 constexpr int RC_THREADS = 256;   // 8 warps: two per tensor-memory lane quarter
 constexpr int RC_SMALL = 256;     // boundary candidates ranked by counting
 constexpr int RC_BIN_SLICE = RB / RC_CL;  // histogram bins summed by each CTA
+static_assert(FUSED_BCAP >= RC_THREADS, "one bucket entry per thread inside the list");
 
 template <bool FP8, int HN, int TPC>
 struct RcCfg {
@@ -158,7 +159,9 @@ __global__ void __cluster_dims__(RC_CL, 1, 1) __launch_bounds__(RC_THREADS, 1)
   }
   int n_sure = n_cols, pneed = 0, nb = 0;
   const uint32_t *pctr = nullptr;
+  uint2 bk0 = make_uint2(0u, 0u);  // the bucket's first entries, requested with the counters
   if (pend) {
+    bk0 = __ldcg(pend_bucket + (size_t)i * FUSED_BCAP + tid);
     pctr = pend + (size_t)i * FUSED_ZERO_WORDS + 2 * RB;
     n_sure = (int)min(__ldcg(pctr + FUSED_CTR_EMIT), (uint32_t)n_cols);
     nb = (int)min(__ldcg(pctr + FUSED_CTR_BUCKET), (uint32_t)FUSED_BCAP);
@@ -176,7 +179,8 @@ __global__ void __cluster_dims__(RC_CL, 1, 1) __launch_bounds__(RC_THREADS, 1)
   }
   if (pneed > 0 && n_sure + pneed > col0 && n_sure < col0 + SLOTS) {  // uniform: this CTA holds some of them
     const uint2 *brow = pend_bucket + (size_t)i * FUSED_BCAP;
-    for (int x = tid; x < nb; x += RC_THREADS) sh.bk[x] = __ldcg(brow + x);
+    if (tid < nb) sh.bk[tid] = bk0;
+    for (int x = tid + RC_THREADS; x < nb; x += RC_THREADS) sh.bk[x] = __ldcg(brow + x);
     __syncthreads();
     for (int x = tid; x < nb; x += RC_THREADS) {
       const uint2 ex = sh.bk[x];

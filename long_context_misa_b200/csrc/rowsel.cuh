@@ -196,8 +196,8 @@ __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist,
   }
   const bool bucket = lvl2 && need1 != in1;  // the 22-bit bucket is split
   // the next kernel finishes the row (rw.defer) unless the split bucket
-  // overflows its list: no last CTA then, and the bucket's entries go
-  // straight to the list (in1 of them in all, within its capacity)
+  // overflows its list: no last CTA then, and the bucket's entries (in1 of
+  // them in all, within the list's capacity) go to the list like the winners
   const bool handoff = rw.defer && (!bucket || in1 <= (uint32_t)RS_BCAP);
   int32_t *dst = ordered ? rw.winners : rw.out;
   // 3. this CTA's sure winners, and the bucket's elements: staged in shared
@@ -229,12 +229,14 @@ __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist,
       if (win && slot < pw) my_w[slot] = (uint32_t)tok;
       n_mine += __popc(m);
       const bool in_b = valid && bucket && k22 == p22;
-      if (handoff) {
-        const uint32_t s2 = warp_append(ctr + RS_BUCKET, in_b);
-        if (in_b && s2 < (uint32_t)RS_BCAP) rw.bucket[s2] = make_uint2(key, (uint32_t)tok);
-      } else {
-        const uint32_t s2 = warp_append(&sh.n_bk, in_b);
-        if (in_b && s2 < (uint32_t)RS_BSTAGE) st_b[s2] = make_uint2(key, (uint32_t)tok);
+      const uint32_t s2 = warp_append(&sh.n_bk, in_b);
+      if (in_b) {
+        if (s2 < (uint32_t)RS_BSTAGE) {
+          st_b[s2] = make_uint2(key, (uint32_t)tok);
+        } else if (handoff) {  // past the staging: straight to the list (it holds all in1)
+          const uint32_t g = atomicAdd(ctr + RS_BUCKET, 1u);
+          if (g < (uint32_t)RS_BCAP) rw.bucket[g] = make_uint2(key, (uint32_t)tok);
+        }
       }
     });
     n_mine = min(n_mine, pw);  // (never clipped: a warp visits at most pw elements)
@@ -246,8 +248,12 @@ __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist,
       for (int w = 0; w < T / 32; ++w) nw += sh.wcnt[w];
       sh.base_win = nw ? atomicAdd(ctr + RS_EMIT, nw) : 0u;
       // more bucket entries than staged: count the row past the list's
-      // capacity, so that the last CTA ranks it from the scores instead
-      sh.base_bk = nbk ? atomicAdd(ctr + RS_BUCKET, nbk <= (uint32_t)RS_BSTAGE ? nbk : (uint32_t)RS_BCAP + 1u) : 0u;
+      // capacity, so that the last CTA ranks it from the scores instead (a
+      // handed-over row's list holds them all: the rest went straight there)
+      if (handoff)
+        sh.base_bk = nbk ? atomicAdd(ctr + RS_BUCKET, min(nbk, (uint32_t)RS_BSTAGE)) : 0u;
+      else
+        sh.base_bk = nbk ? atomicAdd(ctr + RS_BUCKET, nbk <= (uint32_t)RS_BSTAGE ? nbk : (uint32_t)RS_BCAP + 1u) : 0u;
     }
     __syncthreads();
     uint32_t off = sh.base_win;
@@ -256,8 +262,8 @@ __device__ void row_select(const CacheView &c, RsShared<T> &sh, uint32_t *shist,
       const uint32_t slot = off + x;
       if (slot < (uint32_t)k) dst[slot] = (int32_t)my_w[x];
     }
-    if (nbk <= (uint32_t)RS_BSTAGE)
-      for (uint32_t x = tid; x < nbk; x += T) {
+    if (handoff || nbk <= (uint32_t)RS_BSTAGE)
+      for (uint32_t x = tid; x < min(nbk, (uint32_t)RS_BSTAGE); x += T) {
         const uint32_t slot = sh.base_bk + x;
         if (slot < (uint32_t)RS_BCAP) rw.bucket[slot] = st_b[x];
       }
