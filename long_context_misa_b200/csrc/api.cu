@@ -363,7 +363,8 @@ size_t dagger_zero_words(const misa_queries *qs, bool f1, bool f2) {
 
 misa_status dagger_body(const char *who, const misa_cache *cache, const misa_queries *qs, const int32_t *heads,
                         int h, int k_prime, int k, int32_t *topk, void *ws, cudaStream_t stream,
-                        float *route_part = nullptr, int32_t *heads_out = nullptr, bool zero_done = false) {
+                        float *route_part = nullptr, int32_t *heads_out = nullptr, bool zero_done = false,
+                        const misa::PendingAppend *pending = nullptr) {
   misa::CacheView c = view(cache);
   misa::QueryView q = view(qs);
   uint8_t *w8 = static_cast<uint8_t *>(ws);
@@ -402,7 +403,7 @@ misa_status dagger_body(const char *who, const misa_cache *cache, const misa_que
   e = timed_scoring(stream, [&] {
     if (route_part)
       return misa::launch_score_stream(c, q, nullptr, h, scores, cache->L_cap, hist, stream, &fzc, route_part,
-                                       heads_out);
+                                       heads_out, pending);
     return umma ? misa::launch_score_umma(c, q, heads, h, scores, cache->L_cap, stream)
                 : misa::launch_score_mma(c, q, heads, h, nullptr, 0, scores, cache->L_cap, hist, stream,
                                          f1 ? &fzc : nullptr);
@@ -690,12 +691,20 @@ misa_status misa_dagger_decode(const misa_cache *cache, const misa_queries *qs, 
     z0 = reinterpret_cast<uint32_t *>(w8) + first;
     zn = last - first;
   }
-  cudaError_t e = misa::launch_pool_append(c, new_keys, new_scale, new_pos, count, stream, z0, zn);
+  // fused: the routed pass routes while the append runs (it reads nothing
+  // the append writes before waiting for it)
+  cudaError_t e = misa::launch_pool_append(c, new_keys, new_scale, new_pos, count, stream, z0, zn, fused);
   if (e != cudaSuccess) return cuda_fail(e, who);
   if (qs->n_q == 0) return MISA_OK;
-  if (fused)
+  if (fused) {
+    misa::PendingAppend pa;
+    pa.keys = new_keys;
+    pa.scale = new_scale;
+    pa.pos = new_pos;
+    pa.count = count;
     return dagger_body(who, cache, qs, nullptr, h, k_prime, k, topk, ws, stream, reinterpret_cast<float *>(rws),
-                       heads, true);
+                       heads, true, &pa);
+  }
   e = misa::launch_route(c, q, h, hbuf, nullptr, rws, stream, MISA_AGG_ABS_SUM);
   if (e != cudaSuccess) return cuda_fail(e, who);
   return dagger_body(who, cache, qs, hbuf, h, k_prime, k, topk, ws, stream);

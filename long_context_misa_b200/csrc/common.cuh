@@ -56,6 +56,29 @@ __device__ __forceinline__ int query_prefix(const CacheView &c, const QueryView 
   return L;
 }
 
+// query_prefix as it reads once an append kernel (launch_pool_append with
+// new_pos, count) has set the sequences' lengths: for a caller that may run
+// while that append still does.
+__device__ __forceinline__ int query_prefix_appended(const CacheView &c, const QueryView &qv, int i, int *seq,
+                                                     const int32_t *new_pos, int count) {
+  int s = qv.q_seq[i], p = qv.q_pos[i];
+  if (s < 0 || s >= c.n_seq || p < 0) {
+    flag(c, MISA_DEV_BAD_POSITION);
+    *seq = 0;
+    return 0;
+  }
+  const int ap = new_pos[s];
+  const bool appended = ap >= 0 && (long long)ap + count <= c.L_cap;  // else the append leaves the sequence alone
+  int len = min(appended ? ap + count : c.seq_len[s], c.L_cap);
+  int L = p + 1;
+  if (L > len) {
+    flag(c, MISA_DEV_BAD_POSITION);
+    L = max(len, 0);
+  }
+  *seq = s;
+  return L;
+}
+
 // Order-preserving map of fp32 onto uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t ordered_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -120,14 +143,26 @@ __host__ __device__ constexpr int cdiv(int a, int b) { return (a + b - 1) / b; }
 // first statement: the kernel's launch and block scheduling may then overlap
 // the previous kernel's last blocks and its completion, and the wait holds
 // every thread until the previous grid has completed with its writes
-// visible.  No kernel triggers its dependents early, so a successor's blocks
-// are scheduled only as this kernel's blocks exit (waiting successor blocks
-// that sat beside a running prefill kernel cost 45 us of a 0.7 ms call).
+// visible.  Kernels do not trigger their dependents early, so a successor's
+// blocks are scheduled only as this kernel's blocks exit (waiting successor
+// blocks that sat beside a running prefill kernel cost 45 us of a 0.7 ms
+// call).  One pair is the exception: the decode step's append kernel
+// triggers at once, and the routed scoring kernel after it routes before its
+// wait, reading only inputs the append does not write (score_stream.cu).
 // Because the wait comes before any global access, tensor memory allocation
 // or early return in every kernel, every earlier kernel is complete
 // (transitively) before a kernel reads anything, and no kernel requests
 // tensor memory while its predecessor still holds some.
 __device__ __forceinline__ void grid_dep_sync() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// The first statement of a kernel that may be launched early on purpose:
+// the wait, unless `early`; the kernel then calls grid_dep_sync() itself
+// before it reads anything its predecessor writes.
+__device__ __forceinline__ void grid_dep_sync_unless(bool early) {
+  if (!early) grid_dep_sync();
+}
+// Let the dependent grid be scheduled now (it still waits for this grid's
+// completion at its own grid_dep_sync()).
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // Kernel launch through cudaLaunchKernelEx, with the programmatic
 // serialisation attribute above.

@@ -15,10 +15,20 @@ constexpr int TOPK_HIST_BINS = 2048;
 
 // pool.cu
 cudaError_t launch_pool_rebuild(const CacheView &c, cudaStream_t s);
-// zero != nullptr: the kernel also sets zero[0..zero_n) to 0
+// zero != nullptr: the kernel also sets zero[0..zero_n) to 0.  early: the
+// next kernel may start before this one completes (it must read nothing this
+// one writes before its grid_dep_sync(); the decode step's routed pass)
 cudaError_t launch_pool_append(const CacheView &c, const void *new_keys, const float *new_scale,
                                const int32_t *new_pos, int count, cudaStream_t s, uint32_t *zero = nullptr,
-                               size_t zero_n = 0);
+                               size_t zero_n = 0, bool early = false);
+// The keys an append kernel still running ahead of a routed scoring launch
+// writes (launch_pool_append's arguments, with its n_seq CTAs).
+struct PendingAppend {
+  const void *keys = nullptr;
+  const float *scale = nullptr;
+  const int32_t *pos = nullptr;  // nullptr: no append pending
+  int count = 0;
+};
 // e4m3 caches: bf16 keys quantised (one scale per token) while appended;
 // count <= pool_append_quant_max()
 int pool_append_quant_max();
@@ -109,9 +119,13 @@ bool dense_fusable(const CacheView &c, const QueryView &q, const int32_t *heads,
 // route_part != nullptr (with fused): the h scoring heads are routed inside
 // the kernel first (heads ignored), with route_part_slots() x H floats of
 // partial sums at route_part; heads_out ([n_q][h]) receives them if not null.
+// pending (with route_part): launched right after launch_pool_append(...,
+// early = true) with these arguments; the kernel routes while the append
+// runs and leaves one CTA slot per appended sequence to its blocks.
 cudaError_t launch_score_stream(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
                                 long long ld, uint32_t *row_hist, cudaStream_t s, const FusedTopk *fused = nullptr,
-                                float *route_part = nullptr, int32_t *heads_out = nullptr);
+                                float *route_part = nullptr, int32_t *heads_out = nullptr,
+                                const PendingAppend *pending = nullptr);
 bool score_stream_fusable(const CacheView &c, const QueryView &q, const int32_t *heads, int h, bool route = false);
 // CTA slots (queries x CTAs per query) of the in-kernel router's partial sums
 inline int route_part_slots() { return 8 * device_sms(); }

@@ -46,8 +46,9 @@ __global__ void __launch_bounds__(REBUILD_THREADS) pool_rebuild_kernel(CacheView
 __global__ void __launch_bounds__(APPEND_THREADS) pool_append_kernel(CacheView c, const void *new_keys,
                                                                      const float *new_scale,
                                                                      const int32_t *new_pos, int count,
-                                                                     uint32_t *zero, size_t zero_n) {
+                                                                     uint32_t *zero, size_t zero_n, int early) {
   grid_dep_sync();
+  if (early) grid_dep_launch();  // the routed pass routes meanwhile
   for (size_t x = (size_t)blockIdx.x * APPEND_THREADS + threadIdx.x; x < zero_n; x += (size_t)gridDim.x * APPEND_THREADS)
     zero[x] = 0u;
   __shared__ float sm_part[(APPEND_THREADS / 8) * D];
@@ -153,9 +154,10 @@ cudaError_t launch_pool_rebuild(const CacheView &c, cudaStream_t s) {
 }
 
 cudaError_t launch_pool_append(const CacheView &c, const void *new_keys, const float *new_scale,
-                               const int32_t *new_pos, int count, cudaStream_t s, uint32_t *zero, size_t zero_n) {
+                               const int32_t *new_pos, int count, cudaStream_t s, uint32_t *zero, size_t zero_n,
+                               bool early) {
   return launch_kernel(pool_append_kernel, dim3(c.n_seq), dim3(APPEND_THREADS), 0, s, c, new_keys, new_scale, new_pos,
-                       count, zero, zero_n);
+                       count, zero, zero_n, early ? 1 : 0);
 }
 
 }  // namespace misa

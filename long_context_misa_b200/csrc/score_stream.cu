@@ -66,8 +66,12 @@ template <int NT, bool FP8>
 __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, QueryView qv, const int32_t *heads,
                                                                int h, float *scores, long long ld, int scale_vec,
                                                                uint32_t *row_hist, FusedTopk fz, int max_tiles,
-                                                               int region, float *route_part, int32_t *heads_out) {
-  grid_dep_sync();
+                                                               int region, float *route_part, int32_t *heads_out,
+                                                               PendingAppend pa) {
+  // an append kernel still running ahead (pa.pos): the router runs before
+  // the wait on it (below); otherwise the wait comes first
+  grid_dep_sync_unless(route_part != nullptr && pa.pos != nullptr);
+  const bool early = route_part != nullptr && pa.pos != nullptr;
   using Cfg = StreamCfg<NT, FP8>;
   using F = FragCfg<FP8>;
   constexpr int NS = Cfg::NS, ROW = Cfg::ROW, NV = F::NV, TT = Cfg::TT;
@@ -84,7 +88,7 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, cq = lane & 3;
   int s;
-  const int Li = query_prefix(c, qv, i, &s);
+  const int Li = early ? query_prefix_appended(c, qv, i, &s, pa.pos, pa.count) : query_prefix(c, qv, i, &s);
   const int ntile_all = cdiv(Li, TT);
   const int nwarps = gridDim.x * WARPS;
   const int wg = blockIdx.x * WARPS + warp;  // this warp takes tiles wg, wg + nwarps, ...
@@ -158,18 +162,47 @@ __global__ void __launch_bounds__(THREADS) score_stream_kernel(CacheView c, Quer
     const float w_mine = tid < qv.H ? __ldg(qv.w + (size_t)i * qv.H + tid) : 0.f;
     const int Mi = cdiv(Li, c.B), full = Li / c.B, C = gridDim.x;
     const int m0 = (int)((long long)blockIdx.x * Mi / C), m1 = (int)((long long)(blockIdx.x + 1) * Mi / C);
+    // Early: nothing the append writes is read before the wait.  Its tokens
+    // in the cut block come from its input rows (the same bytes), and a CTA
+    // whose pool blocks it rewrites waits first; the ring and every counter
+    // wait too.  All of it uniform over the CTA.
+    KeySource ks;
+    bool waited = !early;
+    if (early) {
+      const int ap = pa.pos[s];
+      if (ap >= 0 && (long long)ap + pa.count <= c.L_cap) {  // the append takes this sequence
+        ks.ovr_keys = static_cast<const uint8_t *>(pa.keys) + (size_t)s * pa.count * ROW;
+        ks.ovr_scale = FP8 ? pa.scale + (size_t)s * pa.count : nullptr;
+        ks.ovr_t0 = ap;
+        ks.ovr_n = pa.count;
+        if (ap / c.B < min(m1, full) && (ap + pa.count - 1) / c.B >= m0) {
+          grid_dep_sync();
+          waited = true;
+        }
+      }
+    }
     if (full < Mi && full >= m0 && full < m1) {  // uniform: this CTA holds the block cut by the prefix end
-      block_key_sum<128>(c, s, full * c.B, Li, reinterpret_cast<float *>(shist), r_tail);
+      block_key_sum<128>(c, s, full * c.B, Li, reinterpret_cast<float *>(shist), r_tail, ks);
       if (tid < D) r_tail[tid] *= 1.f / (float)(Li - full * c.B);
       __syncthreads();
     }
     route_slice<WARPS>(c, s, qv.H, m0, m1, full, r_tail, r_wsum, r_out, qrow_s, [&] {
+      if (waited) {
 #pragma unroll
-      for (int j = 0; j < NS - 1; ++j) issue(j);
+        for (int j = 0; j < NS - 1; ++j) issue(j);
+      }
       if (tid < qv.H) r_w[tid] = w_mine;
-      cp_async_wait<NS - 1>();  // the query rows (the group before the ring's)
+      if (waited)
+        cp_async_wait<NS - 1>();  // the query rows (the group before the ring's)
+      else
+        cp_async_wait<0>();  // the query rows (the only group yet)
       __syncthreads();
     });
+    if (!waited) {
+      grid_dep_sync();  // the append is complete: its keys, block means and cleared words are visible
+#pragma unroll
+      for (int j = 0; j < NS - 1; ++j) issue(j);
+    }
     float *prow = route_part + (size_t)i * C * qv.H;
     for (int j = tid; j < qv.H; j += THREADS) prow[(size_t)blockIdx.x * qv.H + j] = r_out[j];
     if (!row_barrier(r_bar, fz.zeroed + (size_t)i * RS_ZERO_WORDS + 2 * RB + RS_ROUTE, (uint32_t)C, c)) {
@@ -302,8 +335,10 @@ struct StreamPlan {
   bool ok = false;
 };
 
+// reserve: CTA slots left to the blocks of a kernel running alongside (an
+// append kernel that triggered this launch early: one slot per block).
 template <int NT, bool FP8>
-StreamPlan plan_nt(const CacheView &c, const QueryView &q, bool fused) {
+StreamPlan plan_nt(const CacheView &c, const QueryView &q, bool fused, int reserve = 0) {
   using Cfg = StreamCfg<NT, FP8>;
   constexpr int RING = WARPS * Cfg::WARP_BYTES;
   StreamPlan p;
@@ -321,7 +356,7 @@ StreamPlan plan_nt(const CacheView &c, const QueryView &q, bool fused) {
   const int ntile = cdiv(c.L_cap, Cfg::TT);
   auto splits_for = [&](int per_sm) {
     // one wave: a CTA beyond the resident slots would double the kernel time
-    int sp = std::max(1, per_sm * sms / std::max(q.n_q, 1));
+    int sp = std::max(1, (per_sm * sms - reserve) / std::max(q.n_q, 1));
     return std::min(sp, std::max(1, cdiv(ntile, 2 * WARPS)));  // >= 2 tiles per warp
   };
   if (!fused) {
@@ -365,8 +400,9 @@ constexpr int route_q_rows() {
 template <int NT, bool FP8>
 cudaError_t launch_nt(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
                       long long ld, uint32_t *row_hist, cudaStream_t s, const FusedTopk *fz, float *route_part,
-                      int32_t *heads_out) {
-  const StreamPlan p = plan_nt<NT, FP8>(c, q, fz != nullptr);
+                      int32_t *heads_out, const PendingAppend *pending) {
+  const PendingAppend pa = route_part && pending ? *pending : PendingAppend();
+  const StreamPlan p = plan_nt<NT, FP8>(c, q, fz != nullptr, pa.pos ? c.n_seq : 0);
   if (!p.ok) return cudaErrorInvalidConfiguration;
   if (route_part && (!fz || (long long)p.splits * q.n_q > route_part_slots() || q.H > route_q_rows<NT, FP8>()))
     return cudaErrorInvalidValue;
@@ -374,7 +410,7 @@ cudaError_t launch_nt(const CacheView &c, const QueryView &q, const int32_t *hea
   FusedTopk none = {};
   return launch_kernel(score_stream_kernel<NT, FP8>, dim3(p.splits, q.n_q), dim3(THREADS), p.smem, s, c, q, heads, h,
                        scores, ld, scale_vec, row_hist, fz ? *fz : none, p.max_tiles, p.region, route_part,
-                       heads_out);
+                       heads_out, pa);
 }
 
 int stream_nt_h(int h_eff) {
@@ -389,12 +425,14 @@ int stream_nt(const QueryView &q, const int32_t *heads, int h) { return stream_n
 
 cudaError_t launch_score_stream(const CacheView &c, const QueryView &q, const int32_t *heads, int h, float *scores,
                                 long long ld, uint32_t *row_hist, cudaStream_t s, const FusedTopk *fused,
-                                float *route_part, int32_t *heads_out) {
+                                float *route_part, int32_t *heads_out, const PendingAppend *pending) {
   if (q.n_q == 0) return cudaSuccess;
 #define MISA_STREAM_CASE(N)                                                                                      \
   case N:                                                                                                        \
-    return c.fp8 ? launch_nt<N, true>(c, q, heads, h, scores, ld, row_hist, s, fused, route_part, heads_out)     \
-                 : launch_nt<N, false>(c, q, heads, h, scores, ld, row_hist, s, fused, route_part, heads_out);
+    return c.fp8 ? launch_nt<N, true>(c, q, heads, h, scores, ld, row_hist, s, fused, route_part, heads_out,     \
+                                      pending)                                                                   \
+                 : launch_nt<N, false>(c, q, heads, h, scores, ld, row_hist, s, fused, route_part, heads_out,    \
+                                       pending);
   switch (route_part ? stream_nt_h(h) : stream_nt(q, heads, h)) {
     MISA_STREAM_CASE(1)
     MISA_STREAM_CASE(2)

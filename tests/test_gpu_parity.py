@@ -607,6 +607,83 @@ def test_dagger_decode_step_tied_scores(period, k_prime, k):
     assert device_status(cache) == 0
 
 
+# Final sequence lengths, tokens appended per sequence, the sequences not
+# appended to (new_pos -1) and the query rows' sequences, per layout.
+APPEND_LAYOUTS = {
+    "block_end": ([1024, 2432, 8960, 640], 1, (), (0, 1, 2, 3)),      # the append completes a block
+    "block_start": ([1025, 2433, 8961, 129], 1, (), (0, 1, 2, 3)),    # the append opens a block
+    "span": ([1025, 2434, 8962, 130], 3, (), (0, 1, 2, 3)),           # three keys over a block boundary
+    "skip": ([3000, 5000, 7000, 8999], 1, (1,), (0, 1, 2, 3)),        # one sequence not appended to
+    "permuted": ([4096, 3001, 6000, 8192], 1, (), (2, 0, 3, 1)),      # rows on other rows' sequences
+}
+
+
+@pytest.mark.parametrize("dtype", ["fp8", "bf16"])
+@pytest.mark.parametrize("layout", sorted(APPEND_LAYOUTS))
+def test_dagger_decode_step_append_layouts(layout, dtype):
+    # The routed pass routes while the append kernel may still run: the
+    # appended keys of a query's last (cut) block come from the append's
+    # input, and a CTA whose block means the append rewrites waits for it.
+    # The cache rows the append fills hold zeros before the step, and each
+    # appended key copies the query's best dense token, so a read of the
+    # rows before the append lands changes the selection.  Checked against
+    # the oracle with the heads the step chose; the pool and lengths after
+    # the step against the oracle's.
+    lens, count, skipped, rows = APPEND_LAYOUTS[layout]
+    base = W["misa_dagger_decode_128k"] if dtype == "fp8" else W["batched_decode"]
+    wl = base.scaled(n_seq=4, L=9000, B=128, k=256, k_prime=2048)
+    inp = G.make_inputs(wl, 21)
+    lens = np.array(lens, dtype=np.int32)
+    inp.seq_len[:] = lens
+    inp.q_seq[:] = np.array(rows, dtype=np.int32)
+    inp.q_pos[:] = lens[inp.q_seq] - 1
+    pos = np.where(np.isin(np.arange(wl.n_seq), skipped), -1, lens - count).astype(np.int32)
+    ref0 = Ref(inp)
+    for i in range(wl.n_q):  # the appended keys copy the query's best dense token before them
+        s_ = int(inp.q_seq[i])
+        if pos[s_] < 0:
+            continue
+        q, w, K, _ = ref0.query(i)
+        best = int(np.argmax(O.index_scores(q, w, K[:pos[s_]], range(wl.H))))
+        inp.keys[s_, pos[s_]:pos[s_] + count] = inp.keys[s_, best]
+        if inp.scale is not None:
+            inp.scale[s_, pos[s_]:pos[s_] + count] = inp.scale[s_, best]
+    ref = Ref(inp)
+    nk = np.stack([inp.keys[s_, max(p, 0):max(p, 0) + count] for s_, p in enumerate(pos)])
+    nk = torch.from_numpy(nk.view(np.int16) if nk.dtype == np.uint16 else nk).cuda().contiguous()
+    ns = None
+    if inp.scale is not None:
+        ns = torch.from_numpy(np.stack([inp.scale[s_, max(p, 0):max(p, 0) + count] for s_, p in enumerate(pos)])).cuda()
+    cache, qs = to_device(inp, torch)
+    short = np.where(pos >= 0, pos, lens).astype(np.int32)
+    cache.seq_len.copy_(torch.from_numpy(short))
+    for s_, p in enumerate(pos):  # the rows the append fills hold zeros until it does
+        if p >= 0:
+            cache.keys.view(torch.uint8)[s_, p:p + count] = 0
+            if cache.scale is not None:
+                cache.scale[s_, p:p + count] = 0
+    M.pool_keys(cache)
+    heads = torch.empty(wl.n_q, wl.h, dtype=torch.int32, device="cuda")
+    top = M.dagger_decode(cache, qs, nk, ns, torch.from_numpy(pos).cuda(), wl.h, wl.k_prime, wl.k,
+                          heads=heads).cpu().numpy()
+    assert np.array_equal(cache.seq_len.cpu().numpy(), lens)
+    pool = cache.pool.cpu().numpy()
+    for s_ in range(wl.n_seq):
+        expect = O.pool_keys(ref.K[s_], int(lens[s_]), wl.B)
+        assert_close(pool[s_, :expect.shape[0]], expect, f"pool seq {s_}")
+    hd = heads.cpu().numpy()
+    ties = 0
+    for i in range(wl.n_q):
+        q, w, K, Li = ref.query(i)
+        r, hs = O.route_query(q, w, K, Li, wl.B, wl.h)
+        ties += compare_selection(hd[i], hs, lambda j: r[j], wl.h, f"heads q{i}")
+        cand = O.top_k(O.index_scores(q, w, K[:Li], hd[i]), wl.k_prime)
+        expect = O.rerank_query(q, w, K, cand, wl.k)["topk"]
+        np.testing.assert_array_equal(top[i], expect, err_msg=f"query {i}")
+    assert ties <= 1, f"{ties} head boundary ties"
+    assert device_status(cache) == 0
+
+
 @pytest.mark.parametrize("case", ["fp8_mixture", "fp8_long", "bf16_mixture", "bf16_prefill", "fp8_prefill_umma"])
 def test_dagger_topk_equals_composition(case):
     # one call (its k' candidates stay unordered inside) returns exactly what
