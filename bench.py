@@ -72,7 +72,7 @@ def score_kernel_bytes(wl):
 # kernel per workload, from an ncu capture of the current kernel (summarised
 # in profiles/score_stream_kernel_misa_dagger_decode_128k.md: 142,993,408
 # read + 4,683,264 written); null where the kernel changed since the capture.
-STREAM_TRAFFIC_BYTES = {"misa_dagger_decode_128k": 142969088 + 4147712}
+STREAM_TRAFFIC_BYTES = {"misa_dagger_decode_128k": 142973696 + 4446464}
 
 
 class Clocks:
