@@ -32,8 +32,11 @@
  *    scoring kernels) and misa_debug_select_in_kernel (a kernel choice).  misa_rerank_topk_noalloc's fixed scratch array also
  *    keeps the last call's contents (see there).
  *  - The library's kernels are launched with programmatic stream
- *    serialisation.  Each waits for the work before it in the stream to
- *    complete before touching memory, and none releases its dependents early.
+ *    serialisation.  No kernel touches memory before the caller's work ahead
+ *    of the call has completed.  Inside misa_dagger_decode the append kernel
+ *    lets the routed pass start at once (it reads only what the append does
+ *    not write until it waits for it); no call's last kernel releases its
+ *    dependents early.
  *    A caller's kernel launched without that attribute is ordered as usual.
  *    A caller's kernel that opts into programmatic dependent launch itself,
  *    right after a call, must wait on its grid dependency (griddepcontrol.wait
