@@ -608,13 +608,17 @@ def test_dagger_decode_step_tied_scores(period, k_prime, k):
 
 
 # Final sequence lengths, tokens appended per sequence, the sequences not
-# appended to (new_pos -1) and the query rows' sequences, per layout.
+# appended to (new_pos -1), the query rows' sequences and (None: each row's
+# last token) their positions, per layout.
 APPEND_LAYOUTS = {
-    "block_end": ([1024, 2432, 8960, 640], 1, (), (0, 1, 2, 3)),      # the append completes a block
-    "block_start": ([1025, 2433, 8961, 129], 1, (), (0, 1, 2, 3)),    # the append opens a block
-    "span": ([1025, 2434, 8962, 130], 3, (), (0, 1, 2, 3)),           # three keys over a block boundary
-    "skip": ([3000, 5000, 7000, 8999], 1, (1,), (0, 1, 2, 3)),        # one sequence not appended to
-    "permuted": ([4096, 3001, 6000, 8192], 1, (), (2, 0, 3, 1)),      # rows on other rows' sequences
+    "block_end": ([1024, 2432, 8960, 640], 1, (), (0, 1, 2, 3), None),      # the append completes a block
+    "block_start": ([1025, 2433, 8961, 129], 1, (), (0, 1, 2, 3), None),    # the append opens a block
+    "span": ([1025, 2434, 8962, 130], 3, (), (0, 1, 2, 3), None),           # three keys over a block boundary
+    "skip": ([3000, 5000, 7000, 8999], 1, (1,), (0, 1, 2, 3), None),        # one sequence not appended to
+    "permuted": ([4096, 3001, 6000, 8192], 1, (), (2, 0, 3, 1), None),      # rows on other rows' sequences
+    # two rows per sequence: one at the appended token, one whose prefix ends
+    # before it (in the same block, and at the end of the full block before)
+    "shared": ([5000, 7681], 1, (), (0, 0, 1, 1), (4999, 4995, 7680, 7679)),
 }
 
 
@@ -629,14 +633,16 @@ def test_dagger_decode_step_append_layouts(layout, dtype):
     # rows before the append lands changes the selection.  Checked against
     # the oracle with the heads the step chose; the pool and lengths after
     # the step against the oracle's.
-    lens, count, skipped, rows = APPEND_LAYOUTS[layout]
+    lens, count, skipped, rows, qpos = APPEND_LAYOUTS[layout]
     base = W["misa_dagger_decode_128k"] if dtype == "fp8" else W["batched_decode"]
-    wl = base.scaled(n_seq=4, L=9000, B=128, k=256, k_prime=2048)
+    # a batch with rows != sequences is drawn as a prefill chunk, then laid out here
+    wl = base.scaled(n_seq=len(lens), n_q=len(rows), L=9000, B=128, k=256, k_prime=2048,
+                     mode=base.mode if len(rows) == len(lens) else "prefill")
     inp = G.make_inputs(wl, 21)
     lens = np.array(lens, dtype=np.int32)
     inp.seq_len[:] = lens
     inp.q_seq[:] = np.array(rows, dtype=np.int32)
-    inp.q_pos[:] = lens[inp.q_seq] - 1
+    inp.q_pos[:] = lens[inp.q_seq] - 1 if qpos is None else np.array(qpos, dtype=np.int32)
     pos = np.where(np.isin(np.arange(wl.n_seq), skipped), -1, lens - count).astype(np.int32)
     ref0 = Ref(inp)
     for i in range(wl.n_q):  # the appended keys copy the query's best dense token before them
