@@ -222,7 +222,7 @@ def config_figures(M, torch, dev, hbm, tflops, flush_l2, with_oracle):
     routed scoring kernel alone, queries/s, scored head*tokens/s, the fractions
     of the roofline the workload is bound by (key bytes against the measured
     copy bandwidth for decode, useful tensor flops against the measured bf16
-    peak for prefill), and the CPU oracle's rate on the machine's host cores."""
+    peak for prefill), and the CPU oracle's rate on the host's cores."""
     out = {}
     for name, wl in G.WORKLOADS.items():
         inp = G.make_inputs(wl, 0)

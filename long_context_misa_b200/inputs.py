@@ -82,7 +82,7 @@ class Workload:
         return w
 
 
-# The five synthetic workloads (one-line descriptions follow the benchmark's config list).
+# The five synthetic workloads, each with a one-line description.
 WORKLOADS = {
     # 1 query, H=64, L=4096, B=64, h=8, k=256, N(0,1) bf16, one needle.
     "tiny_decode": Workload("tiny_decode", 1, 4096, 64, 64, 8, 256, None,
